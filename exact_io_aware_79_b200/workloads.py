@@ -1,0 +1,173 @@
+"""Seeded synthetic workloads for the attention forward and the paged decode.
+
+This module only draws inputs. It holds none of the attention arithmetic, so
+both the CUDA path and the fp64 oracle can be fed from it without sharing any
+of the method's code.
+
+Workload recipe (the pages publish no dataset for this path, so every tensor
+is synthetic):
+  * Q, K, V are drawn i.i.d. N(0, 1) in fp32 from ``torch.Generator`` seeded
+    per workload, multiplied by ``sigma`` and then rounded to fp16/bf16.
+    Layout is [B, N, H, d], contiguous.
+  * ALiBi slopes for head h of H heads are 2^(-8 (h + 1) / H).
+  * The paged decode draws per-sequence cache lengths uniformly from
+    [len_lo, len_hi] (inclusive), builds a K/V page pool of
+    B * ceil(len_hi / page_size) pages of ``page_size`` tokens each and a
+    block table that is a seeded random permutation of that pool, reshaped
+    to [B, max_blocks].
+
+Small workloads are drawn on the CPU. The full-size paged decode (34 GB of
+K/V) is drawn directly on the device with a seeded CUDA generator; every
+consumer (kernel and oracle) then reads the same tensor.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class FwdWorkload:
+    name: str
+    B: int
+    H: int
+    Nq: int
+    Nk: int
+    d: int
+    dtype: torch.dtype
+    causal: bool = False
+    window_left: int = -1
+    window_right: int = -1
+    alibi: bool = False
+    softcap: float = 0.0
+    sigma: float = 1.0
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    B: int
+    H: int
+    d: int
+    dtype: torch.dtype
+    page_size: int
+    len_lo: int
+    len_hi: int
+    window_left: int = -1
+    alibi: bool = False
+    softcap: float = 0.0
+    sigma: float = 1.0
+    seed: int = 4
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def max_blocks(self) -> int:
+        return -(-self.len_hi // self.page_size)
+
+    @property
+    def num_pages(self) -> int:
+        return self.B * self.max_blocks
+
+
+# The five workloads of the benchmark suite (tiny parity case, causal training
+# shape, long sliding window and its Nq < Nk variant, ALiBi + softcap, paged
+# decode).
+TINY = FwdWorkload("tiny_fp16_b1h2n128d64", 1, 2, 128, 128, 64, torch.float16, seed=0)
+CAUSAL_2K = FwdWorkload("causal_bf16_b8h16n2048d128", 8, 16, 2048, 2048, 128, torch.bfloat16,
+                        causal=True, seed=1)
+WINDOW_16K = FwdWorkload("window_bf16_b1h16n16384d128_wl4096", 1, 16, 16384, 16384, 128,
+                         torch.bfloat16, causal=True, window_left=4096, window_right=0, seed=2)
+WINDOW_Q4K_K16K = FwdWorkload("window_bf16_b1h16nq4096nk16384d128_wl4096", 1, 16, 4096, 16384, 128,
+                              torch.bfloat16, causal=True, window_left=4096, window_right=0, seed=2)
+CAUSAL_Q4K_K16K = FwdWorkload("causal_bf16_b1h16nq4096nk16384d128", 1, 16, 4096, 16384, 128,
+                              torch.bfloat16, causal=True, seed=2)
+ALIBI_SOFTCAP = FwdWorkload("alibi_softcap50_bf16_b4h32n4096d128", 4, 32, 4096, 4096, 128,
+                            torch.bfloat16, causal=True, alibi=True, softcap=50.0, sigma=2.0, seed=3)
+DECODE = DecodeWorkload("paged_decode_bf16_b64h32d128_page256", 64, 32, 128, torch.bfloat16,
+                        page_size=256, len_lo=1024, len_hi=32768, seed=4)
+
+FWD_WORKLOADS = [TINY, CAUSAL_2K, WINDOW_16K, WINDOW_Q4K_K16K, CAUSAL_Q4K_K16K, ALIBI_SOFTCAP]
+
+
+def alibi_slopes(H: int) -> torch.Tensor:
+    """Per-head ALiBi slopes 2^(-8 (h + 1) / H), fp32, shape [H]."""
+    h = torch.arange(H, dtype=torch.float64)
+    return torch.pow(2.0, -8.0 * (h + 1.0) / H).to(torch.float32)
+
+
+def _normal(shape, gen: torch.Generator, sigma: float, dtype: torch.dtype, device) -> torch.Tensor:
+    x = torch.randn(*shape, generator=gen, dtype=torch.float32, device=device)
+    if sigma != 1.0:
+        x.mul_(sigma)
+    return x.to(dtype)
+
+
+def _normal_pages(shape, gen: torch.Generator, sigma: float, dtype: torch.dtype, device,
+                  pages_per_draw: int = 256) -> torch.Tensor:
+    """Like _normal for a page pool, drawn ``pages_per_draw`` pages at a time
+    so the fp32 staging buffer stays small."""
+    out = torch.empty(shape, dtype=dtype, device=device)
+    for p0 in range(0, shape[0], pages_per_draw):
+        p1 = min(shape[0], p0 + pages_per_draw)
+        out[p0:p1] = _normal((p1 - p0,) + tuple(shape[1:]), gen, sigma, dtype, device)
+    return out
+
+
+def make_fwd_inputs(w: FwdWorkload, device="cpu", seed: Optional[int] = None):
+    """Returns dict(q, k, v, slopes) for a forward workload.
+
+    q is [B, Nq, H, d]; k, v are [B, Nk, H, d]; all ``w.dtype``; slopes is
+    fp32 [H] or None. Values are drawn on the CPU so they do not depend on
+    the device.
+    """
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(w.seed if seed is None else seed)
+    q = _normal((w.B, w.Nq, w.H, w.d), gen, w.sigma, w.dtype, "cpu")
+    k = _normal((w.B, w.Nk, w.H, w.d), gen, w.sigma, w.dtype, "cpu")
+    v = _normal((w.B, w.Nk, w.H, w.d), gen, w.sigma, w.dtype, "cpu")
+    slopes = alibi_slopes(w.H) if w.alibi else None
+    out = dict(q=q.to(device), k=k.to(device), v=v.to(device),
+               slopes=None if slopes is None else slopes.to(device))
+    return out
+
+
+def make_decode_inputs(w: DecodeWorkload, device="cpu", seed: Optional[int] = None,
+                       seqlens: Optional[torch.Tensor] = None):
+    """Returns dict(q, k_cache, v_cache, block_table, cache_seqlens, slopes).
+
+    q is [B, 1, H, d]; k_cache, v_cache are [num_pages, page_size, H, d];
+    block_table is int32 [B, max_blocks]; cache_seqlens is int32 [B].
+    Integer tensors and q are drawn on the CPU; the K/V pool is drawn on
+    ``device`` with a generator of that device (so the 34 GB pool of the
+    full-size workload never passes through host memory).
+    """
+    s = w.seed if seed is None else seed
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(s)
+    if seqlens is None:
+        seqlens = torch.randint(w.len_lo, w.len_hi + 1, (w.B,), generator=gen, dtype=torch.int64)
+    seqlens = seqlens.to(torch.int32)
+    perm = torch.randperm(w.num_pages, generator=gen, dtype=torch.int64)
+    block_table = perm.view(w.B, w.max_blocks).to(torch.int32)
+    q = _normal((w.B, 1, w.H, w.d), gen, w.sigma, w.dtype, "cpu")
+    dev = torch.device(device)
+    kv_gen = torch.Generator(device=dev)
+    kv_gen.manual_seed(s + 1000)
+    shape = (w.num_pages, w.page_size, w.H, w.d)
+    k_cache = _normal_pages(shape, kv_gen, w.sigma, w.dtype, dev)
+    v_cache = _normal_pages(shape, kv_gen, w.sigma, w.dtype, dev)
+    slopes = alibi_slopes(w.H) if w.alibi else None
+    return dict(q=q.to(dev), k_cache=k_cache, v_cache=v_cache,
+                block_table=block_table.to(dev), cache_seqlens=seqlens.to(dev),
+                slopes=None if slopes is None else slopes.to(dev))

@@ -1,0 +1,219 @@
+"""fp64 CPU oracle for exact attention (test infrastructure).
+
+Only the tests, the package smoke check and the benchmark's CPU-baseline leg
+may import this package. It loads ``liboracle.so`` (built from
+``attn_oracle.c``; see that file's header for the definition it follows and
+the readings of the pages it takes) and shares no code with the CUDA path.
+
+Inputs may be torch CPU tensors (fp16, bf16 or fp64) or numpy arrays
+(float16 / float64, or uint16 bit patterns with an explicit ``dtype``).
+Everything is returned as float64 numpy arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+F16, BF16, F64 = 0, 1, 2
+
+_lib = None
+
+
+def load_library(path: Optional[str] = None):
+    """(Re)binds the oracle to a compiled library; the default is the one
+    built from attn_oracle.c. Tests use this to load deliberately broken
+    copies of the oracle and check that the pins catch them."""
+    global _lib
+    _lib = None
+    return lib(path)
+
+
+def lib(path: Optional[str] = None):
+    global _lib
+    if _lib is None:
+        path = path or _build.build()
+        L = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int)
+        vp = ctypes.c_void_p
+        i, d = ctypes.c_int, ctypes.c_double
+        L.oracle_attn_fwd.argtypes = [vp, vp, vp, i, dp, dp, dp, i, i, i, i, i, d, i, i, i, dp, d,
+                                      ip, i, i]
+        L.oracle_attn_fwd.restype = i
+        L.oracle_attn_decode_paged.argtypes = [vp, vp, vp, i, ip, ip, dp, dp, i, i, i, i, i, i, d, i,
+                                               dp, d, ip, i, i, i]
+        L.oracle_attn_decode_paged.restype = i
+        L.oracle_combine_splits.argtypes = [dp, dp, i, ctypes.c_long, i, dp, dp]
+        L.oracle_combine_splits.restype = i
+        L.oracle_widen.argtypes = [vp, i, dp, ctypes.c_long]
+        L.oracle_widen.restype = i
+        L.oracle_max_threads.restype = i
+        _lib = L
+    return _lib
+
+
+def max_threads() -> int:
+    return int(lib().oracle_max_threads())
+
+
+def _as_storage(x, dtype_code: Optional[int] = None):
+    """Returns (contiguous numpy array, storage code) for a tensor or array."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().contiguous()
+            if x.dtype == torch.bfloat16:
+                return x.view(torch.int16).numpy().view(np.uint16), BF16
+            if x.dtype == torch.float16:
+                return x.view(torch.int16).numpy().view(np.uint16), F16
+            return np.ascontiguousarray(x.to(torch.float64).numpy()), F64
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.ascontiguousarray(x)
+    if dtype_code is not None:
+        return x, dtype_code
+    if x.dtype == np.float16:
+        return x.view(np.uint16), F16
+    return np.ascontiguousarray(x, dtype=np.float64), F64
+
+
+def _dptr(a: Optional[np.ndarray]):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _iptr(a: Optional[np.ndarray]):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+
+
+def _f64_vec(x) -> Optional[np.ndarray]:
+    if x is None:
+        return None
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().to(torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _i32_vec(x) -> Optional[np.ndarray]:
+    if x is None:
+        return None
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(x, dtype=np.int32)
+
+
+def widen(x, dtype_code: Optional[int] = None) -> np.ndarray:
+    """The oracle's exact widening of fp16/bf16 storage to fp64."""
+    a, code = _as_storage(x, dtype_code)
+    out = np.empty(a.shape, dtype=np.float64)
+    rc = lib().oracle_widen(a.ctypes.data, code, _dptr(out), a.size)
+    if rc:
+        raise ValueError("oracle_widen failed: %d" % rc)
+    return out
+
+
+def attn_fwd(q, k, v, scale: float, causal: bool = False, window_left: int = -1,
+             window_right: int = -1, alibi_slopes=None, softcap: float = 0.0,
+             rows: Optional[Sequence[int]] = None, return_probs: bool = False,
+             num_threads: int = 0, dtype_code: Optional[int] = None):
+    """Plain-definition attention. q [B,Nq,H,d], k/v [B,Nk,H,d].
+
+    Returns (o [B,R,H,d], lse [B,H,R]) or (o, lse, p [B,H,R,Nk]) where R is
+    len(rows) (all Nq rows when rows is None).
+    """
+    qa, code = _as_storage(q, dtype_code)
+    ka, kc = _as_storage(k, dtype_code)
+    va, vc = _as_storage(v, dtype_code)
+    if not (code == kc == vc):
+        raise ValueError("q, k, v must share one storage type")
+    B, Nq, H, d = qa.shape
+    Nk = ka.shape[1]
+    if ka.shape != (B, Nk, H, d) or va.shape != ka.shape:
+        raise ValueError("shape mismatch")
+    r = _i32_vec(rows)
+    R = Nq if r is None else len(r)
+    o = np.empty((B, R, H, d), dtype=np.float64)
+    lse = np.empty((B, H, R), dtype=np.float64)
+    p = np.empty((B, H, R, Nk), dtype=np.float64) if return_probs else None
+    slopes = _f64_vec(alibi_slopes)
+    rc = lib().oracle_attn_fwd(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, code, _dptr(o),
+                               _dptr(lse), _dptr(p), B, H, Nq, Nk, d, float(scale), int(causal),
+                               int(window_left), int(window_right), _dptr(slopes), float(softcap),
+                               _iptr(r), R, int(num_threads))
+    if rc:
+        raise ValueError("oracle_attn_fwd failed: %d" % rc)
+    return (o, lse, p) if return_probs else (o, lse)
+
+
+def attn_decode_paged(q, k_cache, v_cache, block_table, cache_seqlens, scale: float,
+                      window_left: int = -1, alibi_slopes=None, softcap: float = 0.0,
+                      batch: Optional[Sequence[int]] = None, num_splits: int = 1,
+                      num_threads: int = 0, dtype_code: Optional[int] = None):
+    """Paged decode. q [B,1,H,d]; caches [num_pages,page_size,H,d].
+
+    num_splits <= 1: returns (o [R,1,H,d], lse [R,H,1]).
+    num_splits > 1: returns the split partials (o [S,R,H,d], lse [S,R,H]).
+    R is len(batch) (all B sequences when batch is None).
+    """
+    qa, code = _as_storage(q, dtype_code)
+    ka, kc = _as_storage(k_cache, dtype_code)
+    va, vc = _as_storage(v_cache, dtype_code)
+    if not (code == kc == vc):
+        raise ValueError("q and caches must share one storage type")
+    B, one, H, d = qa.shape
+    num_pages, page_size = ka.shape[0], ka.shape[1]
+    if one != 1 or ka.shape != (num_pages, page_size, H, d) or va.shape != ka.shape:
+        raise ValueError("shape mismatch")
+    bt = _i32_vec(block_table)
+    sl = _i32_vec(cache_seqlens)
+    max_blocks = bt.shape[1]
+    bsel = _i32_vec(batch)
+    R = B if bsel is None else len(bsel)
+    S = max(1, int(num_splits))
+    if S > 1:
+        o = np.empty((S, R, H, d), dtype=np.float64)
+        lse = np.empty((S, R, H), dtype=np.float64)
+    else:
+        o = np.empty((R, 1, H, d), dtype=np.float64)
+        lse = np.empty((R, H, 1), dtype=np.float64)
+    slopes = _f64_vec(alibi_slopes)
+    rc = lib().oracle_attn_decode_paged(qa.ctypes.data, ka.ctypes.data, va.ctypes.data, code,
+                                        _iptr(bt), _iptr(sl), _dptr(o), _dptr(lse), B, H, d,
+                                        num_pages, page_size, max_blocks, float(scale),
+                                        int(window_left), _dptr(slopes), float(softcap),
+                                        _iptr(bsel), R, S, int(num_threads))
+    if rc:
+        raise ValueError("oracle_attn_decode_paged failed: %d" % rc)
+    return o, lse
+
+
+def combine_splits(o_part: np.ndarray, lse_part: np.ndarray):
+    """Merge of split partials: o_part [S, ..., d], lse_part [S, ...]."""
+    S = o_part.shape[0]
+    d = o_part.shape[-1]
+    rest = lse_part.shape[1:]
+    n = int(np.prod(rest)) if rest else 1
+    op = np.ascontiguousarray(o_part, dtype=np.float64).reshape(S, n, d)
+    lp = np.ascontiguousarray(lse_part, dtype=np.float64).reshape(S, n)
+    o = np.empty((n, d), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    rc = lib().oracle_combine_splits(_dptr(op), _dptr(lp), S, n, d, _dptr(o), _dptr(lse))
+    if rc:
+        raise ValueError("oracle_combine_splits failed: %d" % rc)
+    return o.reshape(rest + (d,)), lse.reshape(rest)

@@ -1,0 +1,433 @@
+"""Pins for the fp64 oracle, against facts fixed by the mathematics and the pages.
+
+None of these tests re-types the oracle's formula and compares: each one
+checks an invariant, a closed form, a special case that reduces to something
+simpler, or a brute-force enumeration on a tiny input, chosen so that a
+plausible slip in the oracle (a dropped scale, a wrong sign, a top-left
+instead of bottom-right mask, an off-by-one window, a transposed operand, a
+wrong page index, a wrong merge weight) fails at least one of them.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+TOL = 1e-12
+
+
+def rnd(shape, seed, sigma=1.0):
+    g = np.random.default_rng(seed)
+    return g.standard_normal(shape) * sigma
+
+
+# ---------------------------------------------------------------- storage widening
+
+def test_widen_fp16_every_bit_pattern():
+    bits = np.arange(65536, dtype=np.uint16)
+    got = oracle.widen(bits, oracle.F16)
+    want = bits.view(np.float16).astype(np.float64)
+    same = (got == want) | (np.isnan(got) & np.isnan(want))
+    assert same.all()
+
+
+def test_widen_bf16_every_bit_pattern():
+    bits = np.arange(65536, dtype=np.uint16)
+    got = oracle.widen(bits, oracle.BF16)
+    want = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    same = (got == want) | (np.isnan(got) & np.isnan(want))
+    assert same.all()
+
+
+# ---------------------------------------------------------------- invariants named by the spec
+
+MASKS = [
+    dict(causal=False),
+    dict(causal=True),
+    dict(causal=True, window_left=3, window_right=0),
+    dict(causal=False, window_left=2, window_right=1),
+]
+
+
+@pytest.mark.parametrize("Nq,Nk", [(7, 7), (5, 11), (11, 5)])
+@pytest.mark.parametrize("mask", MASKS)
+def test_probability_rows_sum_to_one(Nq, Nk, mask):
+    B, H, d = 2, 3, 8
+    q, k, v = rnd((B, Nq, H, d), 1), rnd((B, Nk, H, d), 2), rnd((B, Nk, H, d), 3)
+    o, lse, p = oracle.attn_fwd(q, k, v, 0.4, alibi_slopes=[0.5, 0.1, 0.0], softcap=3.0,
+                                return_probs=True, **mask)
+    sums = p.sum(axis=-1)
+    nonempty = np.isfinite(lse)
+    assert np.allclose(sums[nonempty], 1.0, atol=TOL, rtol=0)
+    assert np.all(sums[~nonempty] == 0.0)
+    assert (p >= 0).all()
+    # the same fact seen through O: with V = 1 every non-empty row of O is 1
+    o1, _ = oracle.attn_fwd(q, k, np.ones_like(v), 0.4, alibi_slopes=[0.5, 0.1, 0.0], softcap=3.0,
+                            **mask)
+    ne = np.transpose(nonempty, (0, 2, 1))  # [B, Nq, H]
+    assert np.allclose(o1[ne], 1.0, atol=TOL, rtol=0)
+    assert np.all(o1[~ne] == 0.0)
+
+
+def test_single_key_returns_v():
+    B, H, Nq, d = 2, 3, 9, 16
+    q, k, v = rnd((B, Nq, H, d), 4), rnd((B, 1, H, d), 5), rnd((B, 1, H, d), 6)
+    o, lse = oracle.attn_fwd(q, k, v, 0.25)
+    assert np.allclose(o, np.broadcast_to(v, o.shape), atol=TOL, rtol=0)
+    # with one key the LSE is that key's scaled score
+    s = 0.25 * np.einsum("bihc,bhc->bhi", q, k[:, 0])
+    assert np.allclose(lse, s, atol=TOL, rtol=0)
+
+
+@pytest.mark.parametrize("Nk", [1, 6, 33])
+def test_zero_query_gives_column_mean_and_ln_n(Nk):
+    B, H, Nq, d = 2, 2, 5, 8
+    q = np.zeros((B, Nq, H, d))
+    k, v = rnd((B, Nk, H, d), 7), rnd((B, Nk, H, d), 8)
+    o, lse = oracle.attn_fwd(q, k, v, 1.0)
+    mean = v.mean(axis=1)  # [B, H, d]
+    assert np.allclose(o, mean[:, None], atol=TOL, rtol=0)
+    assert np.allclose(lse, math.log(Nk), atol=TOL, rtol=0)
+
+
+def test_joint_permutation_of_keys_and_values():
+    B, H, Nq, Nk, d = 2, 3, 6, 13, 8
+    q, k, v = rnd((B, Nq, H, d), 9), rnd((B, Nk, H, d), 10), rnd((B, Nk, H, d), 11)
+    perm = np.random.default_rng(12).permutation(Nk)
+    o1, l1 = oracle.attn_fwd(q, k, v, 0.3, softcap=2.0)
+    o2, l2 = oracle.attn_fwd(q, k[:, perm], v[:, perm], 0.3, softcap=2.0)
+    assert np.allclose(o1, o2, atol=TOL, rtol=0)
+    assert np.allclose(l1, l2, atol=TOL, rtol=0)
+    # but the permutation must move V with K: permuting V alone changes O
+    o3, _ = oracle.attn_fwd(q, k, v[:, perm], 0.3, softcap=2.0)
+    assert np.abs(o3 - o1).max() > 1e-3
+
+
+def brute_force(q, k, v, scale, causal=False, wl=-1, wr=-1, slopes=None, softcap=0.0):
+    """Enumerates every (b, i, h) and every key with Python floats."""
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    o = np.zeros((B, Nq, H, d))
+    lse = np.zeros((B, H, Nq))
+    for b in range(B):
+        for h in range(H):
+            for i in range(Nq):
+                pos = i + Nk - Nq          # bottom-right: last query row meets last key
+                terms = []
+                for j in range(Nk):
+                    if causal and j > pos:
+                        continue
+                    if wl >= 0 and j < pos - wl:
+                        continue
+                    if wr >= 0 and j > pos + wr:
+                        continue
+                    x = scale * sum(float(q[b, i, h, c]) * float(k[b, j, h, c]) for c in range(d))
+                    if softcap > 0:
+                        x = softcap * math.tanh(x / softcap)
+                    if slopes is not None:
+                        x -= slopes[h] * abs(pos - j)
+                    terms.append((j, x))
+                if not terms:
+                    lse[b, h, i] = -math.inf
+                    continue
+                mx = max(x for _, x in terms)
+                z = sum(math.exp(x - mx) for _, x in terms)
+                for j, x in terms:
+                    o[b, i, h] += math.exp(x - mx) / z * v[b, j, h]
+                lse[b, h, i] = mx + math.log(z)
+    return o, lse
+
+
+@pytest.mark.parametrize("Nq,Nk", [(4, 9), (9, 9), (9, 4), (1, 7)])
+@pytest.mark.parametrize("opts", [
+    dict(causal=True),
+    dict(causal=True, wl=2, wr=0),
+    dict(causal=False, wl=1, wr=2),
+    dict(causal=True, slopes=[0.7, 0.05]),
+    dict(causal=False, softcap=1.5),
+    dict(causal=True, wl=3, wr=0, slopes=[0.3, 1.1], softcap=2.5),
+])
+def test_matches_brute_force_with_bottom_right_alignment(Nq, Nk, opts):
+    B, H, d = 2, 2, 5
+    q, k, v = rnd((B, Nq, H, d), 13, 1.5), rnd((B, Nk, H, d), 14, 1.5), rnd((B, Nk, H, d), 15)
+    want_o, want_l = brute_force(q, k, v, 0.6, **opts)
+    o, lse = oracle.attn_fwd(q, k, v, 0.6, causal=opts.get("causal", False),
+                             window_left=opts.get("wl", -1), window_right=opts.get("wr", -1),
+                             alibi_slopes=opts.get("slopes"), softcap=opts.get("softcap", 0.0))
+    assert np.allclose(o, want_o, atol=1e-11, rtol=0)
+    fin = np.isfinite(want_l)
+    assert np.array_equal(fin, np.isfinite(lse))
+    assert np.allclose(lse[fin], want_l[fin], atol=1e-11, rtol=0)
+
+
+def test_unbounded_window_is_full_attention():
+    B, H, Nq, Nk, d = 1, 2, 10, 14, 8
+    q, k, v = rnd((B, Nq, H, d), 16), rnd((B, Nk, H, d), 17), rnd((B, Nk, H, d), 18)
+    for causal in (False, True):
+        o1, l1 = oracle.attn_fwd(q, k, v, 0.3, causal=causal)
+        o2, l2 = oracle.attn_fwd(q, k, v, 0.3, causal=causal, window_left=10**9, window_right=10**9)
+        assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_huge_softcap_and_zero_slopes_are_plain_attention():
+    B, H, Nq, Nk, d = 2, 3, 8, 8, 8
+    q, k, v = rnd((B, Nq, H, d), 19), rnd((B, Nk, H, d), 20), rnd((B, Nk, H, d), 21)
+    o0, l0 = oracle.attn_fwd(q, k, v, 0.3, causal=True)
+    o1, l1 = oracle.attn_fwd(q, k, v, 0.3, causal=True, softcap=1e30)
+    o2, l2 = oracle.attn_fwd(q, k, v, 0.3, causal=True, alibi_slopes=[0.0, 0.0, 0.0])
+    for o, l in ((o1, l1), (o2, l2)):
+        assert np.allclose(o, o0, atol=TOL, rtol=0) and np.allclose(l, l0, atol=TOL, rtol=0)
+
+
+# ---------------------------------------------------------------- closed forms
+
+def visible_count(Nq, Nk, i, causal, wl, wr):
+    """Number of keys row i sees, from interval arithmetic (no enumeration)."""
+    pos = i + Nk - Nq
+    lo = 0 if wl < 0 else max(0, pos - wl)
+    hi = Nk - 1
+    if causal:
+        hi = min(hi, pos)
+    if wr >= 0:
+        hi = min(hi, pos + wr)
+    return max(0, hi - lo + 1), lo, hi
+
+
+@pytest.mark.parametrize("Nq,Nk", [(16, 16), (6, 20), (20, 6)])
+@pytest.mark.parametrize("causal,wl,wr", [(True, -1, -1), (True, 4, 0), (False, 3, 2), (False, 0, 0),
+                                          (False, -1, 5)])
+def test_zero_query_counts_visible_keys(Nq, Nk, causal, wl, wr):
+    """With Q = 0 every visible score is 0, so LSE_i = ln(count_i) and O_i is
+    the mean of the visible V rows; this fixes the mask of every row."""
+    B, H, d = 1, 2, 4
+    q = np.zeros((B, Nq, H, d))
+    k, v = rnd((B, Nk, H, d), 22), rnd((B, Nk, H, d), 23)
+    o, lse = oracle.attn_fwd(q, k, v, 1.0, causal=causal, window_left=wl, window_right=wr)
+    for i in range(Nq):
+        n, lo, hi = visible_count(Nq, Nk, i, causal, wl, wr)
+        if n == 0:
+            assert np.all(lse[:, :, i] == -np.inf) and np.all(o[:, i] == 0)
+        else:
+            assert np.allclose(lse[:, :, i], math.log(n), atol=TOL, rtol=0)
+            assert np.allclose(o[:, i], v[:, lo:hi + 1].mean(axis=1), atol=TOL, rtol=0)
+
+
+@pytest.mark.parametrize("Nq,Nk", [(8, 8), (3, 8), (8, 3)])
+def test_one_hot_probe_pins_each_key(Nq, Nk):
+    """K row t is lam * e0 and all others are 0; Q = e0. Then row i puts
+    (almost) all weight on key t when t is visible, and else spreads it evenly
+    over its visible keys (all other scores are 0)."""
+    B, H, d, lam = 1, 1, 4, 200.0
+    for causal, wl, wr in [(True, -1, -1), (True, 2, 0), (False, 1, 1)]:
+        for t in range(Nk):
+            q = np.zeros((B, Nq, H, d))
+            q[..., 0] = 1.0
+            k = np.zeros((B, Nk, H, d))
+            k[0, t, 0, 0] = lam
+            v = rnd((B, Nk, H, d), 24 + t)
+            o, lse = oracle.attn_fwd(q, k, v, 1.0, causal=causal, window_left=wl, window_right=wr)
+            for i in range(Nq):
+                n, lo, hi = visible_count(Nq, Nk, i, causal, wl, wr)
+                if n == 0:
+                    assert lse[0, 0, i] == -np.inf
+                elif lo <= t <= hi:
+                    assert np.allclose(o[0, i, 0], v[0, t, 0], atol=1e-60 + 1e-80, rtol=1e-12)
+                    assert abs(lse[0, 0, i] - lam) < 1e-12 * lam
+                else:
+                    assert np.allclose(o[0, i, 0], v[0, lo:hi + 1, 0].mean(axis=0), atol=TOL)
+
+
+@pytest.mark.parametrize("slope", [0.0, 0.03, 0.5, 2.0])
+def test_alibi_is_a_geometric_series(slope):
+    """Q = 0, causal, Nq = Nk: row i has scores -slope*(i - j), j <= i, so with
+    r = exp(-slope) the LSE is ln((1 - r^(i+1)) / (1 - r)) (or ln(i+1) for
+    r = 1) and the weight on key j is r^(i-j) / sum."""
+    B, H, N, d = 1, 1, 12, 4
+    q = np.zeros((B, N, H, d))
+    k = rnd((B, N, H, d), 40)
+    v = np.zeros((B, N, H, d))
+    v[0, :, 0, 0] = np.arange(N)          # O_i[0] is then the mean key index under P
+    o, lse = oracle.attn_fwd(q, k, v, 1.0, causal=True, alibi_slopes=[slope])
+    r = math.exp(-slope)
+    for i in range(N):
+        z = (i + 1.0) if slope == 0 else (1 - r ** (i + 1)) / (1 - r)
+        assert abs(lse[0, 0, i] - math.log(z)) < 1e-12
+        mean_j = sum(j * r ** (i - j) for j in range(i + 1)) / z
+        assert abs(o[0, i, 0, 0] - mean_j) < 1e-12
+
+
+@pytest.mark.parametrize("cap", [0.5, 2.0, 50.0])
+def test_softcap_two_key_closed_form(cap):
+    """Two keys with raw scaled scores a and b: softcap maps them to
+    c*tanh(a/c), c*tanh(b/c); the weight of key 0 is the logistic of their
+    difference. scale = 0.5 is applied before the cap."""
+    q = np.zeros((1, 1, 1, 2))
+    q[0, 0, 0] = [1.0, 0.0]
+    k = np.zeros((1, 2, 1, 2))
+    k[0, 0, 0, 0], k[0, 1, 0, 0] = 6.0, -2.0          # raw dots 6, -2 -> scaled 3, -1
+    v = np.zeros((1, 2, 1, 2))
+    v[0, 0, 0, 0] = 1.0                               # O[0] = weight of key 0
+    o, lse = oracle.attn_fwd(q, k, v, 0.5, softcap=cap)
+    a, b = cap * math.tanh(3.0 / cap), cap * math.tanh(-1.0 / cap)
+    w0 = 1.0 / (1.0 + math.exp(b - a))
+    assert abs(o[0, 0, 0, 0] - w0) < 1e-14
+    assert abs(lse[0, 0, 0] - (a + math.log1p(math.exp(b - a)))) < 1e-14
+
+
+def test_fully_masked_rows_are_empty():
+    B, H, Nq, Nk, d = 1, 2, 9, 4, 8
+    q, k, v = rnd((B, Nq, H, d), 25), rnd((B, Nk, H, d), 26), rnd((B, Nk, H, d), 27)
+    o, lse = oracle.attn_fwd(q, k, v, 0.3, causal=True)
+    # bottom-right alignment: rows 0..Nq-Nk-1 sit before the first key
+    assert np.all(lse[:, :, :Nq - Nk] == -np.inf)
+    assert np.all(o[:, :Nq - Nk] == 0.0)
+    assert np.all(np.isfinite(lse[:, :, Nq - Nk:]))
+
+
+def test_row_subset_matches_full():
+    B, H, Nq, Nk, d = 2, 2, 17, 23, 8
+    q, k, v = rnd((B, Nq, H, d), 28), rnd((B, Nk, H, d), 29), rnd((B, Nk, H, d), 30)
+    o, lse = oracle.attn_fwd(q, k, v, 0.3, causal=True, window_left=5)
+    rows = [0, 3, 16, 8]
+    os_, ls = oracle.attn_fwd(q, k, v, 0.3, causal=True, window_left=5, rows=rows)
+    assert np.array_equal(os_, o[:, rows]) and np.array_equal(ls, lse[:, :, rows])
+
+
+def test_float64_library_softmax_on_tiny_shapes():
+    """torch's float64 softmax (a library routine) over an explicitly masked
+    score matrix agrees with the oracle."""
+    B, H, Nq, Nk, d = 2, 2, 6, 10, 8
+    q, k, v = rnd((B, Nq, H, d), 31), rnd((B, Nk, H, d), 32), rnd((B, Nk, H, d), 33)
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    s = torch.einsum("bihc,bjhc->bhij", tq, tk) * 0.35
+    i = torch.arange(Nq)[:, None] + (Nk - Nq)
+    j = torch.arange(Nk)[None, :]
+    s = s.masked_fill(j > i, float("-inf"))
+    p = torch.softmax(s, dim=-1)
+    want = torch.einsum("bhij,bjhc->bihc", p, tv).numpy()
+    o, lse = oracle.attn_fwd(q, k, v, 0.35, causal=True)
+    assert np.allclose(o, want, atol=TOL, rtol=0)
+    assert np.allclose(lse, torch.logsumexp(s, dim=-1).numpy(), atol=TOL, rtol=0)
+
+
+def test_half_precision_storage_is_widened_exactly():
+    B, H, Nq, Nk, d = 1, 2, 5, 7, 8
+    for dt in (torch.float16, torch.bfloat16):
+        q = torch.randn(B, Nq, H, d).to(dt)
+        k = torch.randn(B, Nk, H, d).to(dt)
+        v = torch.randn(B, Nk, H, d).to(dt)
+        o1, l1 = oracle.attn_fwd(q, k, v, 0.3, causal=True)
+        o2, l2 = oracle.attn_fwd(q.double(), k.double(), v.double(), 0.3, causal=True)
+        assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+# ---------------------------------------------------------------- paged decode
+
+def contiguous_from_pages(w_k, w_v, table, lens, page):
+    """Builds per-sequence contiguous K/V [B, Lmax, H, d] by walking pages."""
+    B = table.shape[0]
+    Lmax = int(max(lens))
+    H, d = w_k.shape[2], w_k.shape[3]
+    k = np.zeros((B, Lmax, H, d))
+    v = np.zeros((B, Lmax, H, d))
+    for b in range(B):
+        for t in range(int(lens[b])):
+            pg = table[b, t // page]
+            k[b, t] = w_k[pg, t % page]
+            v[b, t] = w_v[pg, t % page]
+    return k, v
+
+
+def decode_case(seed, B=3, H=2, d=8, page=4, max_blocks=5, lens=(7, 20, 1)):
+    g = np.random.default_rng(seed)
+    num_pages = B * max_blocks
+    kc = g.standard_normal((num_pages, page, H, d))
+    vc = g.standard_normal((num_pages, page, H, d))
+    table = g.permutation(num_pages).reshape(B, max_blocks).astype(np.int32)
+    q = g.standard_normal((B, 1, H, d))
+    return q, kc, vc, table, np.array(lens, dtype=np.int32)
+
+
+def test_identity_block_table_equals_contiguous_cache():
+    B, H, d, page, mb = 2, 2, 8, 4, 5
+    g = np.random.default_rng(50)
+    k = g.standard_normal((B, mb * page, H, d))
+    v = g.standard_normal((B, mb * page, H, d))
+    q = g.standard_normal((B, 1, H, d))
+    lens = np.array([13, 20], dtype=np.int32)
+    table = np.arange(B * mb, dtype=np.int32).reshape(B, mb)      # identity
+    kc = k.reshape(B * mb, page, H, d)
+    vc = v.reshape(B * mb, page, H, d)
+    o, lse = oracle.attn_decode_paged(q, kc, vc, table, lens, 0.3)
+    for b in range(B):
+        L = int(lens[b])
+        want_o, want_l = oracle.attn_fwd(q[b:b + 1], k[b:b + 1, :L], v[b:b + 1, :L], 0.3, causal=True)
+        assert np.allclose(o[b], want_o[0], atol=TOL, rtol=0)
+        assert np.allclose(lse[b], want_l[0], atol=TOL, rtol=0)
+
+
+@pytest.mark.parametrize("opts", [dict(), dict(window_left=5), dict(alibi_slopes=[0.2, 0.6], softcap=2.0)])
+def test_permuted_block_table_is_a_reindexing(opts):
+    q, kc, vc, table, lens = decode_case(51)
+    o, lse = oracle.attn_decode_paged(q, kc, vc, table, lens, 0.3, **opts)
+    k, v = contiguous_from_pages(kc, vc, table, lens, 4)
+    for b in range(len(lens)):
+        L = int(lens[b])
+        wo, wl = brute_force(q[b:b + 1], k[b:b + 1, :L], v[b:b + 1, :L], 0.3, causal=True,
+                             wl=opts.get("window_left", -1), slopes=opts.get("alibi_slopes"),
+                             softcap=opts.get("softcap", 0.0))
+        assert np.allclose(o[b], wo[0], atol=1e-11, rtol=0)
+        assert np.allclose(lse[b], wl[0], atol=1e-11, rtol=0)
+
+
+def test_decode_query_sees_all_cached_keys():
+    """The decode example of the causal-alignment change: one query against
+    N+1 keys attends to every key, i.e. equals non-causal attention."""
+    q, kc, vc, table, lens = decode_case(52, lens=(9, 17, 4))
+    o, lse = oracle.attn_decode_paged(q, kc, vc, table, lens, 0.3)
+    k, v = contiguous_from_pages(kc, vc, table, lens, 4)
+    for b in range(3):
+        L = int(lens[b])
+        wo, wl = oracle.attn_fwd(q[b:b + 1], k[b:b + 1, :L], v[b:b + 1, :L], 0.3, causal=False)
+        assert np.allclose(o[b], wo[0], atol=TOL, rtol=0) and np.allclose(lse[b], wl[0], atol=TOL)
+
+
+def test_empty_sequence_is_empty():
+    q, kc, vc, table, lens = decode_case(53, lens=(0, 5, 0))
+    o, lse = oracle.attn_decode_paged(q, kc, vc, table, lens, 0.3)
+    assert np.all(o[0] == 0) and np.all(lse[0] == -np.inf) and np.all(lse[2] == -np.inf)
+    assert np.all(np.isfinite(lse[1]))
+
+
+@pytest.mark.parametrize("S", [2, 3, 4, 5, 8, 16])
+@pytest.mark.parametrize("opts", [dict(), dict(window_left=6), dict(alibi_slopes=[0.2, 0.6], softcap=2.0)])
+def test_any_split_count_matches_one_split(S, opts):
+    q, kc, vc, table, lens = decode_case(54, lens=(7, 20, 1))
+    o1, l1 = oracle.attn_decode_paged(q, kc, vc, table, lens, 0.3, **opts)
+    op, lp = oracle.attn_decode_paged(q, kc, vc, table, lens, 0.3, num_splits=S, **opts)
+    o, lse = oracle.combine_splits(op, lp)
+    assert np.allclose(o, o1[:, 0], atol=TOL, rtol=0)
+    assert np.allclose(lse, l1[:, :, 0], atol=TOL, rtol=0)
+    # the partials cover disjoint key ranges: their exp(lse) add up to exp(lse)
+    total = np.exp(lp).sum(axis=0)
+    assert np.allclose(total, np.exp(l1[:, :, 0]), rtol=1e-12, atol=0)
+
+
+def test_combine_of_all_empty_splits_is_empty():
+    op = np.zeros((3, 2, 4))
+    lp = np.full((3, 2), -np.inf)
+    lp[1, 1] = 0.5
+    op[1, 1] = [1, 2, 3, 4]
+    o, lse = oracle.combine_splits(op, lp)
+    assert lse[0] == -np.inf and np.all(o[0] == 0)
+    assert abs(lse[1] - 0.5) < TOL and np.allclose(o[1], [1, 2, 3, 4], atol=TOL)
+
+
+def test_decode_rejects_bad_block_table():
+    q, kc, vc, table, lens = decode_case(55)
+    bad = table.copy()
+    bad[1, 0] = kc.shape[0]            # page index past the pool
+    with pytest.raises(ValueError):
+        oracle.attn_decode_paged(q, kc, vc, bad, lens, 0.3)
