@@ -1,1 +1,181 @@
-"""Exact IO-aware attention for B200 (sm_100a): C-ABI library and its Python binding."""
+"""Exact IO-aware attention for B200 (sm_100a).
+
+Python binding of the C ABI in include/fa.h (libfa_b200.so, built in-tree by
+``python -m exact_io_aware_79_b200.build``). The binding only marshals
+arguments: shapes are read off the torch tensors, pointers and the current
+CUDA stream are passed through, and a non-OK status raises FaError. All
+computation happens in the library's CUDA kernels; there is no fallback, and
+every call raises if the library cannot be loaded.
+
+Entry points with the C names:
+    fa_fwd(q, k, v, out, lse, scale, causal, window_left, window_right,
+           alibi_slopes, softcap)
+    fa_fwd_kvcache(q, k_cache, v_cache, block_table, cache_seqlens, out, lse,
+                   scale, window_left, alibi_slopes, softcap, num_splits,
+                   workspace)
+    fa_kvcache_num_splits(...), fa_kvcache_workspace_size(...),
+    fa_status_string(code)
+and allocating conveniences ``attention`` and ``decode``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa_b200.so")
+
+FA_FP16, FA_BF16 = 0, 1
+FA_MAX_SPLITS = 64
+STATUS = {
+    0: "FA_OK", 1: "FA_ERR_NULL", 2: "FA_ERR_SHAPE", 3: "FA_ERR_DTYPE", 4: "FA_ERR_HEADDIM",
+    5: "FA_ERR_ARG", 6: "FA_ERR_WORKSPACE", 7: "FA_ERR_CUDA", 8: "FA_ERR_DEVICE",
+}
+
+
+class FaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__("%s failed: %s" % (where, _lib_handle().fa_status_string(code).decode()))
+
+
+_LIB = None
+
+
+def _lib_handle():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libfa_b200.so not found at %s; build it with "
+                              "`python -m exact_io_aware_79_b200.build`" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, f, vp]
+        L.fa_fwd.restype = i
+        L.fa_fwd_kvcache.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp, f, i, vp, sz,
+                                     vp]
+        L.fa_fwd_kvcache.restype = i
+        L.fa_kvcache_num_splits.argtypes = [i, i, i, i, i, i]
+        L.fa_kvcache_num_splits.restype = i
+        L.fa_kvcache_workspace_size.argtypes = [i, i, i, i, i, i]
+        L.fa_kvcache_workspace_size.restype = sz
+        L.fa_status_string.argtypes = [i]
+        L.fa_status_string.restype = ctypes.c_char_p
+        _LIB = L
+    return _LIB
+
+
+def library() -> ctypes.CDLL:
+    """The loaded libfa_b200.so (raises ImportError if it is missing)."""
+    return _lib_handle()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return FA_FP16
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    return -1
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise FaError(code, where)
+
+
+def fa_status_string(code: int) -> str:
+    return _lib_handle().fa_status_string(code).decode()
+
+
+def fa_fwd(q, k, v, out, lse, scale: float, causal: bool = False, window_left: int = -1,
+           window_right: int = -1, alibi_slopes=None, softcap: float = 0.0, stream=None) -> None:
+    """q [B,Nq,H,d], k/v [B,Nk,H,d], out like q, lse fp32 [B,H,Nq]; all on the device."""
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    for t in (q, k, v, out, lse):
+        if not t.is_contiguous():
+            raise ValueError("fa_fwd needs contiguous tensors")
+    if tuple(k.shape) != (B, Nk, H, d) or tuple(v.shape) != (B, Nk, H, d) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("fa_fwd: shape mismatch")
+    if tuple(lse.shape) != (B, H, Nq) or lse.dtype != torch.float32:
+        raise ValueError("fa_fwd: lse must be fp32 [B, H, Nq]")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype):
+        raise ValueError("fa_fwd: q, k, v, out must share one dtype")
+    code = _lib_handle().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Nq, Nk, d,
+                                _dtype_code(q), float(scale), int(bool(causal)), int(window_left),
+                                int(window_right), _ptr(alibi_slopes), float(softcap), _stream(stream))
+    _check(code, "fa_fwd")
+
+
+def fa_kvcache_num_splits(B: int, H: int, d: int, max_blocks: int, page_size: int, num_splits: int = 0) -> int:
+    return int(_lib_handle().fa_kvcache_num_splits(B, H, d, max_blocks, page_size, num_splits))
+
+
+def fa_kvcache_workspace_size(B: int, H: int, d: int, max_blocks: int, page_size: int,
+                              num_splits: int = 0) -> int:
+    return int(_lib_handle().fa_kvcache_workspace_size(B, H, d, max_blocks, page_size, num_splits))
+
+
+def fa_fwd_kvcache(q, k_cache, v_cache, block_table, cache_seqlens, out, lse, scale: float,
+                   window_left: int = -1, alibi_slopes=None, softcap: float = 0.0, num_splits: int = 0,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """q [B,1,H,d]; caches [num_pages,page_size,H,d]; block_table int32 [B,max_blocks];
+    cache_seqlens int32 [B]; out like q; lse fp32 [B,H,1]; workspace a byte tensor."""
+    B, one, H, d = q.shape
+    num_pages, page_size = k_cache.shape[0], k_cache.shape[1]
+    max_blocks = block_table.shape[1]
+    for t in (q, k_cache, v_cache, block_table, cache_seqlens, out, lse):
+        if not t.is_contiguous():
+            raise ValueError("fa_fwd_kvcache needs contiguous tensors")
+    if one != 1 or tuple(k_cache.shape) != (num_pages, page_size, H, d) or \
+            tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("fa_fwd_kvcache: shape mismatch")
+    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32 or block_table.shape[0] != B:
+        raise ValueError("fa_fwd_kvcache: block_table / cache_seqlens must be int32 [B, ...]")
+    if tuple(lse.shape) != (B, H, 1) or lse.dtype != torch.float32:
+        raise ValueError("fa_fwd_kvcache: lse must be fp32 [B, H, 1]")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = _lib_handle().fa_fwd_kvcache(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(cache_seqlens), _ptr(out), _ptr(lse),
+        B, H, d, num_pages, page_size, max_blocks, _dtype_code(q), float(scale), int(window_left),
+        _ptr(alibi_slopes), float(softcap), int(num_splits), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(code, "fa_fwd_kvcache")
+
+
+def attention(q, k, v, scale: Optional[float] = None, causal: bool = False, window_left: int = -1,
+              window_right: int = -1, alibi_slopes=None, softcap: float = 0.0):
+    """Allocating form of fa_fwd; returns (out, lse)."""
+    B, Nq, H, d = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    fa_fwd(q, k, v, out, lse, d ** -0.5 if scale is None else scale, causal, window_left, window_right,
+           alibi_slopes, softcap)
+    return out, lse
+
+
+def decode(q, k_cache, v_cache, block_table, cache_seqlens, scale: Optional[float] = None,
+           window_left: int = -1, alibi_slopes=None, softcap: float = 0.0, num_splits: int = 0):
+    """Allocating form of fa_fwd_kvcache; returns (out, lse)."""
+    B, _, H, d = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, 1), dtype=torch.float32, device=q.device)
+    nbytes = fa_kvcache_workspace_size(B, H, d, block_table.shape[1], k_cache.shape[1], num_splits)
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device) if nbytes else None
+    fa_fwd_kvcache(q, k_cache, v_cache, block_table, cache_seqlens, out, lse,
+                   d ** -0.5 if scale is None else scale, window_left, alibi_slopes, softcap, num_splits, ws)
+    return out, lse

@@ -1,0 +1,239 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument validation,
+// device check, TMA tensor-map encoding, split-count resolution and launches.
+#include "fa.h"
+#include "fa_internal.h"
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace {
+
+constexpr int kNumSms = 148;           // B200; only steers the automatic split count
+constexpr long long kMaxSeq = 1 << 28; // Nq, Nk limit of fa_fwd
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 0 = unknown, 1 = sm_100, 2 = other
+std::atomic<int> g_device_kind[kMaxDevices];
+
+fa_status check_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    cudaGetLastError();
+    return FA_ERR_DEVICE;
+  }
+  if (dev < kMaxDevices) {
+    const int k = g_device_kind[dev].load(std::memory_order_relaxed);
+    if (k == 1) return FA_OK;
+    if (k == 2) return FA_ERR_DEVICE;
+  }
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_DEVICE;
+  }
+  const bool ok = major == 10 && minor == 0;
+  if (dev < kMaxDevices) g_device_kind[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
+  return ok ? FA_OK : FA_ERR_DEVICE;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// [B, N, H, d] 16-bit tensor as a 4-D map (d, H, N, B), box (64, 1, 128, 1),
+// 128-byte swizzle; rows past N read as zero.
+bool make_map(CUtensorMap* map, const void* base, bool bf16, int B, int N, int H, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t n = static_cast<cuuint64_t>(N > 0 ? N : 1);
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), n, static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
+                           n * static_cast<cuuint64_t>(H) * d * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool finite(float x) { return std::isfinite(x); }
+
+// Automatic split count: enough splits that a split of the longest possible
+// sequence holds at most ~2048 keys, and, for small batches, enough CTAs to
+// cover the GPU several times (but never splits shorter than 256 keys).
+int auto_splits(int B, int H, long long max_len) {
+  const long long units = static_cast<long long>(B) * H;
+  long long s = (max_len + 2047) / 2048;
+  const long long fill = (4LL * kNumSms + units - 1) / units;
+  const long long min_chunk = (max_len + 255) / 256;
+  s = std::max(s, std::min(fill, min_chunk));
+  s = std::max(1LL, std::min(s, static_cast<long long>(FA_MAX_SPLITS)));
+  return static_cast<int>(s);
+}
+
+bool kvcache_sizes_ok(int B, int H, int d, int max_blocks, int page_size) {
+  if (B < 0 || H < 1 || max_blocks < 1 || page_size < 1) return false;
+  if (d != 64 && d != 128) return false;
+  if (static_cast<long long>(max_blocks) * page_size >= (1LL << 31)) return false;
+  if (static_cast<long long>(B) * H * FA_MAX_SPLITS >= (1LL << 31)) return false;
+  if (B > 65535) return false;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_NULL: return "FA_ERR_NULL: a required pointer is NULL";
+    case FA_ERR_SHAPE: return "FA_ERR_SHAPE: a size is out of range";
+    case FA_ERR_DTYPE: return "FA_ERR_DTYPE: dtype must be FA_FP16 or FA_BF16";
+    case FA_ERR_HEADDIM: return "FA_ERR_HEADDIM: head dimension must be 64 or 128";
+    case FA_ERR_ARG: return "FA_ERR_ARG: invalid scalar argument or unaligned pointer";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: split-KV workspace missing, misaligned or too small";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call or kernel launch failed";
+    case FA_ERR_DEVICE: return "FA_ERR_DEVICE: no CUDA device or the device is not sm_100";
+  }
+  return "unknown fa_status";
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int Nq, int Nk,
+                 int d, fa_dtype dtype, float scale, int causal, int window_left, int window_right,
+                 const float* alibi_slopes, float softcap, cudaStream_t stream) {
+  if (B < 0 || H < 0 || Nq < 0 || Nk < 0) return FA_ERR_SHAPE;
+  if (Nq > kMaxSeq || Nk > kMaxSeq || static_cast<long long>(B) * H >= (1LL << 31)) return FA_ERR_SHAPE;
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  if (!finite(scale) || !finite(softcap) || softcap < 0.0f) return FA_ERR_ARG;
+  if (window_left < -1 || window_right < -1 || (causal != 0 && causal != 1)) return FA_ERR_ARG;
+  if (static_cast<long long>(B) * H * Nq == 0) return FA_OK;
+  if (!q || !out || !lse) return FA_ERR_NULL;
+  if (Nk > 0 && (!k || !v)) return FA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k) || !aligned16(v) || !aligned16(lse)) return FA_ERR_ARG;
+  const int pairs = (Nq + 255) / 256;
+  if (static_cast<long long>(pairs) * B * H >= (1LL << 31)) return FA_ERR_SHAPE;
+  fa_status st = check_device();
+  if (st != FA_OK) return st;
+
+  const bool bf16 = dtype == FA_BF16;
+  CUtensorMap tq, tk, tv;
+  // With Nk == 0 no K/V tile is ever loaded; q stands in as a valid base.
+  const void* kb = Nk > 0 ? k : q;
+  const void* vb = Nk > 0 ? v : q;
+  if (!make_map(&tq, q, bf16, B, Nq, H, d) || !make_map(&tk, kb, bf16, B, Nk, H, d) ||
+      !make_map(&tv, vb, bf16, B, Nk, H, d))
+    return FA_ERR_CUDA;
+
+  fa::FwdParams p{};
+  p.out = out;
+  p.lse = lse;
+  p.slopes = alibi_slopes;
+  p.B = B;
+  p.H = H;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.num_pairs = pairs;
+  p.causal = causal;
+  p.window_left = window_left;
+  p.window_right = window_right;
+  p.use_softcap = softcap > 0.0f;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.cap_scale = softcap > 0.0f ? scale / softcap : 0.0f;
+  p.cap_log2 = softcap * fa::kLog2e;
+  return fa::launch_fwd(bf16, d, tq, tk, tv, p, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_kvcache_num_splits(int B, int H, int d, int max_blocks, int page_size, int num_splits) {
+  if (!kvcache_sizes_ok(B, H, d, max_blocks, page_size)) return -1;
+  if (num_splits < 0 || num_splits > FA_MAX_SPLITS) return -1;
+  if (num_splits > 0) return num_splits;
+  if (B == 0) return 1;
+  return auto_splits(B, H, static_cast<long long>(max_blocks) * page_size);
+}
+
+size_t fa_kvcache_workspace_size(int B, int H, int d, int max_blocks, int page_size, int num_splits) {
+  const int s = fa_kvcache_num_splits(B, H, d, max_blocks, page_size, num_splits);
+  if (s <= 1) return 0;
+  const size_t rows = static_cast<size_t>(s) * B * H;
+  size_t o_bytes = rows * d * sizeof(float);
+  o_bytes = (o_bytes + 255) & ~size_t(255);
+  return o_bytes + rows * sizeof(float);
+}
+
+fa_status fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                         const int* cache_seqlens, void* out, float* lse, int B, int H, int d, int num_pages,
+                         int page_size, int max_blocks, fa_dtype dtype, float scale, int window_left,
+                         const float* alibi_slopes, float softcap, int num_splits, void* workspace,
+                         size_t workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || H < 1 || num_pages < 1 || max_blocks < 1) return FA_ERR_SHAPE;
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  if (page_size < 1 || num_splits < 0 || num_splits > FA_MAX_SPLITS) return FA_ERR_ARG;
+  if (!finite(scale) || !finite(softcap) || softcap < 0.0f || window_left < -1) return FA_ERR_ARG;
+  if (!kvcache_sizes_ok(B, H, d, max_blocks, page_size)) return FA_ERR_SHAPE;
+  if (B == 0) return FA_OK;
+  if (!q || !k_cache || !v_cache || !block_table || !cache_seqlens || !out || !lse) return FA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return FA_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_ARG;
+  const int S = fa_kvcache_num_splits(B, H, d, max_blocks, page_size, num_splits);
+  const size_t need = fa_kvcache_workspace_size(B, H, d, max_blocks, page_size, num_splits);
+  if (S > 1 && (!workspace || !aligned16(workspace) || workspace_bytes < need)) return FA_ERR_WORKSPACE;
+  fa_status st = check_device();
+  if (st != FA_OK) return st;
+
+  fa::DecodeParams p{};
+  p.q = q;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.block_table = block_table;
+  p.cache_seqlens = cache_seqlens;
+  p.out = out;
+  p.lse = lse;
+  if (S > 1) {
+    const size_t rows = static_cast<size_t>(S) * B * H;
+    size_t o_bytes = (rows * d * sizeof(float) + 255) & ~size_t(255);
+    p.o_part = static_cast<float*>(workspace);
+    p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + o_bytes);
+  }
+  p.slopes = alibi_slopes;
+  p.B = B;
+  p.H = H;
+  p.num_pages = num_pages;
+  p.page_size = page_size;
+  p.max_blocks = max_blocks;
+  p.num_splits = S;
+  p.window_left = window_left;
+  p.use_softcap = softcap > 0.0f;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.cap_scale = softcap > 0.0f ? scale / softcap : 0.0f;
+  p.cap_log2 = softcap * fa::kLog2e;
+  return fa::launch_decode(dtype == FA_BF16, d, p, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // extern "C"

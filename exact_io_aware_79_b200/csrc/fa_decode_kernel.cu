@@ -1,0 +1,281 @@
+// fa_decode_kernel.cu -- split-KV ("flash-decoding") attention of one query
+// token over a paged KV cache, plus the merge of the split partials.
+//
+// Method ("Flash-Attention v2.0 到 v2.7 更新", section v2.2: instead of one
+// block walking the whole KV, the KV cache is cut along the sequence, each
+// block takes one piece and an extra kernel merges the pieces; section v2.5:
+// the cache is non-contiguous and addressed through a block table;
+// "FlashAttention深度解析", section on inference: with a short query the goal
+// is to load the KV cache as efficiently as possible).
+//
+// The split kernel is bound by HBM bandwidth (about 1 flop per byte), so it
+// is written for the memory system rather than the tensor cores: every lane
+// issues 16-byte loads, the d/8 lanes that share one token read its 2*d-byte
+// row in one coalesced transaction, and each lane keeps U tokens' K and V
+// loads in flight before it touches any of them. One CTA (4 warps) handles
+// one (sequence, head, split); its tokens are interleaved across warps in
+// groups of U*32/(d/8) tokens. Per token: page = block_table[b][t / page],
+// row = t % page; the dot product is reduced across the token's lanes with
+// shuffles; the online softmax keeps (m, l, acc) per lane group and the four
+// warps' states are merged through shared memory at the end.
+#include "fa_internal.h"
+#include "sm100_ptx.cuh"
+
+#include <type_traits>
+
+namespace fa {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kUnroll = 4;
+
+__device__ __forceinline__ uint4 load_stream(const void* ptr) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(ptr));
+  return v;
+}
+
+template <typename T>
+__device__ __forceinline__ void widen8(const uint4& v, float (&f)[8]) {
+  const float2 a = unpack2<T>(v.x), b = unpack2<T>(v.y), c = unpack2<T>(v.z), d = unpack2<T>(v.w);
+  f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+  f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+
+// Key range [t0, t1) of split s: the visible keys [lo, hi) cut into
+// num_splits near-equal chunks whose length is a whole number of pages.
+__device__ __forceinline__ void split_range(int lo, int hi, int num_splits, int s, int page, int& t0, int& t1) {
+  t0 = t1 = hi;
+  if (hi <= lo) return;
+  const long long n = hi - lo;
+  long long chunk = (n + num_splits - 1) / num_splits;
+  chunk = (chunk + page - 1) / page * page;
+  const long long a = lo + static_cast<long long>(s) * chunk;
+  t0 = static_cast<int>(min(a, static_cast<long long>(hi)));
+  t1 = static_cast<int>(min(a + chunk, static_cast<long long>(hi)));
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(const DecodeParams p) {
+  constexpr int LPT = D / 8;    // lanes per token
+  constexpr int TPW = 32 / LPT; // tokens per warp per load step
+  constexpr int kStep = kWarps * TPW * kUnroll;
+  __shared__ float sm_m[kWarps], sm_l[kWarps];
+  __shared__ float sm_acc[kWarps][D];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane / LPT;   // token slot within the warp
+  const int cl = lane % LPT;  // 8-element chunk of the head dimension
+  const int h = blockIdx.x % p.H;
+  const int s = blockIdx.x / p.H;
+  const int b = blockIdx.y;
+
+  const int L_raw = p.cache_seqlens[b];
+  const long long max_len = static_cast<long long>(p.max_blocks) * p.page_size;
+  bool bad = L_raw < 0 || L_raw > max_len;
+  const int L = bad ? 0 : L_raw;
+  const int pos = L - 1;  // the query's key position (bottom-right alignment)
+  const int lo = p.window_left >= 0 ? max(0, pos - p.window_left) : 0;
+  int t0, t1;
+  split_range(lo, L, p.num_splits, s, p.page_size, t0, t1);
+
+  // query chunk, pre-scaled so the dot product is already in its final units
+  float qf[8];
+  widen8<T>(*reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.q) +
+                                            (static_cast<size_t>(b) * p.H + h) * D + cl * 8),
+            qf);
+  const float qscale = p.use_softcap ? p.cap_scale : p.scale_log2;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) qf[e] *= qscale;
+  const bool alibi = p.slopes != nullptr;
+  const float slope_l2 = alibi ? p.slopes[h] * kLog2e : 0.0f;
+
+  const size_t tok_stride = static_cast<size_t>(p.H) * D;  // elements
+  const size_t page_stride = static_cast<size_t>(p.page_size) * tok_stride;
+  const T* kbase = reinterpret_cast<const T*>(p.k_cache) + static_cast<size_t>(h) * D + cl * 8;
+  const T* vbase = reinterpret_cast<const T*>(p.v_cache) + static_cast<size_t>(h) * D + cl * 8;
+  const int* bt = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+
+  float m = -INFINITY, lsum = 0.0f;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+
+  for (int base = t0 + warp * TPW * kUnroll; base < t1; base += kStep) {
+    uint4 kr[kUnroll], vr[kUnroll];
+    bool valid[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int tok = base + u * TPW + g;
+      valid[u] = tok < t1;
+      kr[u] = vr[u] = make_uint4(0, 0, 0, 0);
+      if (valid[u]) {
+        const int pg = bt[tok / p.page_size];
+        if (pg < 0 || pg >= p.num_pages) {
+          bad = true;
+          valid[u] = false;
+        } else {
+          const size_t off = static_cast<size_t>(pg) * page_stride + static_cast<size_t>(tok % p.page_size) * tok_stride;
+          kr[u] = load_stream(kbase + off);
+          vr[u] = load_stream(vbase + off);
+        }
+      }
+    }
+    float sc[kUnroll];
+    float mt = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      float kf[8];
+      widen8<T>(kr[u], kf);
+      float dot = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dot = fmaf(qf[e], kf[e], dot);
+#pragma unroll
+      for (int o = LPT / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      float t = p.use_softcap ? p.cap_log2 * tanh_via_exp2(dot) : dot;
+      const int tok = base + u * TPW + g;
+      if (alibi) t -= slope_l2 * static_cast<float>(pos - tok);
+      sc[u] = valid[u] ? t : -INFINITY;
+      mt = fmaxf(mt, sc[u]);
+    }
+    const float m_new = fmaxf(m, mt);
+    if (m_new == -INFINITY) continue;  // nothing visible yet in this lane group
+    const float alpha = ex2(m - m_new);
+    lsum *= alpha;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] *= alpha;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const float pu = ex2(sc[u] - m_new);
+      lsum += pu;
+      float vf[8];
+      widen8<T>(vr[u], vf);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaf(pu, vf[e], acc[e]);
+    }
+    m = m_new;
+  }
+
+  // merge the TPW lane groups of this warp
+#pragma unroll
+  for (int o = LPT; o < 32; o <<= 1) {
+    const float m_o = __shfl_xor_sync(0xffffffffu, m, o);
+    const float l_o = __shfl_xor_sync(0xffffffffu, lsum, o);
+    const float mm = fmaxf(m, m_o);
+    const float a = (m == -INFINITY) ? 0.0f : ex2(m - mm);
+    const float a_o = (m_o == -INFINITY) ? 0.0f : ex2(m_o - mm);
+    lsum = lsum * a + l_o * a_o;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float x_o = __shfl_xor_sync(0xffffffffu, acc[e], o);
+      acc[e] = acc[e] * a + x_o * a_o;
+    }
+    m = mm;
+  }
+  if (lane < LPT) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sm_acc[warp][cl * 8 + e] = acc[e];
+  }
+  if (lane == 0) {
+    sm_m[warp] = m;
+    sm_l[warp] = lsum;
+  }
+  const bool any_bad = __syncthreads_or(bad) != 0;
+
+  // merge the warps; thread c owns output element c
+  const int c = threadIdx.x;
+  if (c >= D) return;
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w]);
+  float ltot = 0.0f, oc = 0.0f;
+  if (M != -INFINITY) {
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float a = (sm_m[w] == -INFINITY) ? 0.0f : ex2(sm_m[w] - M);
+      ltot += sm_l[w] * a;
+      oc += sm_acc[w][c] * a;
+    }
+  }
+  const float nan = __int_as_float(0x7fc00000);
+  float o_val, lse_val;
+  if (any_bad) {
+    o_val = nan;
+    lse_val = nan;
+  } else if (ltot > 0.0f) {
+    o_val = oc / ltot;
+    lse_val = (M + lg2(ltot)) * kLn2;
+  } else {
+    o_val = 0.0f;
+    lse_val = -INFINITY;
+  }
+  const size_t row = static_cast<size_t>(b) * p.H + h;
+  if (p.num_splits == 1) {
+    T* out = reinterpret_cast<T*>(p.out) + row * D;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) out[c] = __float2bfloat16_rn(o_val);
+    else out[c] = __float2half_rn(o_val);
+    if (c == 0) p.lse[row] = lse_val;
+  } else {
+    const size_t prow = static_cast<size_t>(s) * p.B * p.H + row;
+    p.o_part[prow * D + c] = o_val;
+    if (c == 0) p.lse_part[prow] = lse_val;
+  }
+}
+
+// Merge of the split partials of one (sequence, head): lse = ln sum_s exp(lse_s),
+// O = sum_s exp(lse_s - lse) O_s; empty splits (lse_s = -inf) weigh nothing,
+// a NaN partial (invalid block-table entry) makes the row NaN.
+template <typename T, int D>
+__global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeParams p) {
+  const int row = blockIdx.x;  // b * H + h
+  const int c = threadIdx.x;
+  const int BH = p.B * p.H;
+  const int S = p.num_splits;
+  float M = -INFINITY;
+  bool nan_in = false;
+  for (int s = 0; s < S; ++s) {
+    const float x = p.lse_part[static_cast<size_t>(s) * BH + row];
+    nan_in |= (x != x);
+    M = fmaxf(M, x);
+  }
+  const float nan = __int_as_float(0x7fc00000);
+  float o_val = 0.0f, lse_val = -INFINITY;
+  if (nan_in) {
+    o_val = lse_val = nan;
+  } else if (M != -INFINITY) {
+    float wsum = 0.0f, oc = 0.0f;
+    for (int s = 0; s < S; ++s) {
+      const size_t prow = static_cast<size_t>(s) * BH + row;
+      const float w = ex2((p.lse_part[prow] - M) * kLog2e);
+      wsum += w;
+      oc += w * p.o_part[prow * D + c];
+    }
+    o_val = oc / wsum;
+    lse_val = M + lg2(wsum) * kLn2;
+  }
+  T* out = reinterpret_cast<T*>(p.out) + static_cast<size_t>(row) * D;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) out[c] = __float2bfloat16_rn(o_val);
+  else out[c] = __float2half_rn(o_val);
+  if (c == 0) p.lse[row] = lse_val;
+}
+
+template <typename T, int D>
+cudaError_t launch(const DecodeParams& p, cudaStream_t stream) {
+  dim3 grid(p.H * p.num_splits, p.B);
+  decode_split_kernel<T, D><<<grid, kWarps * 32, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || p.num_splits == 1) return e;
+  decode_combine_kernel<T, D><<<p.B * p.H, D, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(bool bf16, int d, const DecodeParams& p, cudaStream_t stream) {
+  if (bf16) return d == 128 ? launch<__nv_bfloat16, 128>(p, stream) : launch<__nv_bfloat16, 64>(p, stream);
+  return d == 128 ? launch<__half, 128>(p, stream) : launch<__half, 64>(p, stream);
+}
+
+}  // namespace fa

@@ -1,0 +1,487 @@
+// fa_fwd_kernel.cu -- tiled exact-attention forward for sm_100a.
+//
+// Method (pages: "IO感知技术革命", sections on block tiling, online softmax and
+// asynchronous copy; "FlashAttention深度解析", section "重新定义注意力计算";
+// masking and score modifiers from "Flash-Attention v2.0 到 v2.7 更新",
+// sections v2.1, v2.3, v2.4, v2.6): Q is split into 128-row tiles that stay
+// on chip; K and V stream through in 128-key tiles; each K/V tile updates a
+// running row max m and row sum l and rescales the partial output, so the
+// N x N scores never leave the SM.
+//
+// B200 mapping. One CTA owns two adjacent Q tiles (A and B) of one (batch,
+// head) and runs ten warps:
+//   warps 0-3  softmax for tile A, one query row per thread (row = TMEM lane)
+//   warps 4-7  softmax for tile B
+//   warp  8    TMA producer: Q tiles once, then K_j, V_j into a ring of
+//              shared-memory slots (128-byte swizzle), mbarrier expect-tx
+//   warp  9    TMEM owner and MMA issuer (one elected thread)
+// Tensor memory (512 columns x 128 lanes x 32 bit):
+//   cols   0..127  S_A (fp32 scores), later P_A (16-bit, first 64 columns)
+//   cols 128..255  O_A (fp32, d columns)
+//   cols 256..383  S_B / P_B
+//   cols 384..511  O_B
+// Per K/V tile j the MMA thread issues, in order,
+//   O_A += P_A(j) V_j,  S_A(j+1) = Q_A K_{j+1}^T,  O_B += P_B(j) V_j,
+//   S_B(j+1) = Q_B K_{j+1}^T,
+// so while one softmax group works on its tile the tensor core runs the
+// other group's two products (ping-pong). tcgen05 operations of one thread
+// complete in issue order, so the arrival that publishes S_X(j+1) also proves
+// that O_X += P_X(j) V_j has finished; the softmax group may then rescale O_X
+// in place before it publishes P_X(j+1).
+//
+// Rescaling is lazy: a row keeps its old max unless the new tile raises it by
+// more than 8 (log2 units), so P stays <= 2^8 and O is rescaled only when it
+// must be. The result is the same softmax (m cancels in O / l).
+#include "fa_internal.h"
+#include "sm100_ptx.cuh"
+
+#include <cfloat>
+#include <climits>
+#include <type_traits>
+
+namespace fa {
+namespace {
+
+constexpr int BM = 128;  // query rows per Q tile
+constexpr int BN = 128;  // keys per K/V tile
+constexpr int kThreads = 320;
+constexpr int kMaxSlots = 8;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct Cfg {
+  static constexpr int kChunkBytes = BM * 128;         // 128 rows x 64 elements x 2 bytes
+  static constexpr int kTileBytes = BM * D * 2;        // one Q, K or V tile
+  static constexpr int kSlots = (D == 128) ? 5 : 8;    // K/V ring depth
+  static constexpr int kSmemBytes = 1024 + (2 + kSlots) * kTileBytes + 1024;
+};
+
+struct Barriers {
+  uint64_t q_full;
+  uint64_t slot_full[kMaxSlots];
+  uint64_t slot_empty[kMaxSlots];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_final[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Visible key interval [lo, hi] of query row q (empty when lo > hi).
+struct RowRange {
+  int lo, hi;
+};
+
+__device__ __forceinline__ RowRange row_range(const FwdParams& p, int q) {
+  const long long pos = static_cast<long long>(q) + p.Nk - p.Nq;
+  long long lo = 0, hi = static_cast<long long>(p.Nk) - 1;
+  if (p.window_left >= 0) lo = max(lo, pos - p.window_left);
+  if (p.causal) hi = min(hi, pos);
+  if (p.window_right >= 0) hi = min(hi, pos + p.window_right);
+  RowRange r;
+  r.lo = static_cast<int>(min(lo, static_cast<long long>(p.Nk)));
+  r.hi = static_cast<int>(max(hi, -1ll));
+  return r;
+}
+
+// Waits without checking the abort flag (used only to drain work in flight).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  int dummy = 0;
+  mbar_wait(bar, parity, &dummy);
+}
+
+template <typename T, int D>
+__device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV, uint8_t* sQ,
+                         uint8_t* sKV, Barriers* bars, int b, int h, int q0, const bool (&has)[2], int u0, int u1) {
+  using C = Cfg<D>;
+  volatile int* abort = &bars->abort;
+  const uint64_t pol_q = l2_policy_evict_first();
+  const uint64_t pol_kv = l2_policy_evict_last();
+  const uint32_t qbytes = (has[0] ? C::kTileBytes : 0) + (has[1] ? C::kTileBytes : 0);
+  mbar_arrive_expect_tx(&bars->q_full, qbytes);
+#pragma unroll
+  for (int X = 0; X < 2; ++X) {
+    if (!has[X]) continue;
+#pragma unroll
+    for (int ch = 0; ch < D / 64; ++ch)
+      tma_load_4d(tmQ, &bars->q_full, sQ + X * C::kTileBytes + ch * C::kChunkBytes, ch * 64, h, q0 + X * BM, b,
+                  pol_q);
+  }
+  uint32_t it = 0;
+  bool ok = true;
+  for (int j = u0; j <= u1 && ok; ++j) {
+#pragma unroll
+    for (int kv = 0; kv < 2; ++kv) {
+      const uint32_t slot = it % C::kSlots, n = it / C::kSlots;
+      if (n > 0 && !mbar_wait(&bars->slot_empty[slot], (n - 1) & 1, abort)) {
+        ok = false;
+        break;
+      }
+      mbar_arrive_expect_tx(&bars->slot_full[slot], C::kTileBytes);
+      const CUtensorMap* map = kv ? tmV : tmK;
+#pragma unroll
+      for (int ch = 0; ch < D / 64; ++ch)
+        tma_load_4d(map, &bars->slot_full[slot], sKV + slot * C::kTileBytes + ch * C::kChunkBytes, ch * 64, h,
+                    j * BN, b, pol_kv);
+      ++it;
+    }
+  }
+  // Every load issued must land before the CTA may exit. On the normal path
+  // they all have (the MMA thread consumed them); after an abort, wait.
+  drain_wait(&bars->q_full, 0);
+  const uint32_t first = it > static_cast<uint32_t>(C::kSlots) ? it - C::kSlots : 0;
+  for (uint32_t i = first; i < it; ++i) drain_wait(&bars->slot_full[i % C::kSlots], (i / C::kSlots) & 1);
+}
+
+template <typename T, int D>
+__device__ void mma_issuer(uint8_t* sQ, uint8_t* sKV, Barriers* bars, uint32_t tmem, const bool (&has)[2],
+                           const int (&f)[2], const int (&l)[2], int u0, int u1) {
+  using C = Cfg<D>;
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  constexpr uint32_t idesc_qk = instr_desc_f16(kBf16, BM, BN, false);
+  constexpr uint32_t idesc_pv = instr_desc_f16(kBf16, BM, D, true);
+  volatile int* abort = &bars->abort;
+  const uint32_t sQaddr = smem_addr(sQ);
+  const uint32_t sKVaddr = smem_addr(sKV);
+
+  auto in = [&](int X, int j) { return has[X] && j >= f[X] && j <= l[X]; };
+  uint32_t it = 0;
+  auto acquire = [&](uint32_t& addr, uint32_t& slot) -> bool {
+    slot = it % C::kSlots;
+    const bool ok = mbar_wait(&bars->slot_full[slot], (it / C::kSlots) & 1, abort);
+    addr = sKVaddr + slot * C::kTileBytes;
+    ++it;
+    return ok;
+  };
+  // S_X = Q_X K^T: M = 128 query rows, N = 128 keys, K = d in steps of 16.
+  // Both operands are K-major, 128-byte swizzled, 64 elements per 16 KB chunk.
+  auto qk = [&](int X, uint32_t kaddr) {
+    const uint32_t qaddr = sQaddr + X * C::kTileBytes;
+    const uint32_t d_t = tmem + X * 256;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t off = (kk / 4) * C::kChunkBytes + (kk % 4) * 32;
+      mma_ss(d_t, smem_desc_sw128(qaddr + off, 16, 1024), smem_desc_sw128(kaddr + off, 16, 1024), idesc_qk,
+             kk > 0 ? 1u : 0u);
+    }
+  };
+  // O_X (+)= P_X V: A = P from TMEM (16-bit, two keys per column), B = V tile
+  // stored keys x d with d contiguous (MN-major): 16 keys = 2048 bytes,
+  // the second 64-wide d chunk lies 16 KB further (leading byte offset).
+  auto pv = [&](int X, uint32_t vaddr, bool accumulate) {
+    const uint32_t a_t = tmem + X * 256;
+    const uint32_t d_t = tmem + X * 256 + 128;
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk)
+      mma_ts(d_t, a_t + kk * 8, smem_desc_sw128(vaddr + kk * 2048, C::kChunkBytes, 1024), idesc_pv,
+             (accumulate || kk > 0) ? 1u : 0u);
+  };
+
+  uint32_t pcount[2] = {0, 0};
+  bool ok = mbar_wait(&bars->q_full, 0, abort);
+  uint32_t aK = 0, slotK = 0, aV = 0, slotV = 0;
+  if (ok) ok = acquire(aK, slotK);
+  if (ok) {
+    tc_fence_after();
+    if (in(0, u0)) {
+      qk(0, aK);
+      tc_commit(&bars->s_full[0]);
+    }
+    if (in(1, u0)) {
+      qk(1, aK);
+      tc_commit(&bars->s_full[1]);
+    }
+    tc_commit(&bars->slot_empty[slotK]);
+  }
+  for (int j = u0; j <= u1 && ok; ++j) {
+    if (!(ok = acquire(aV, slotV))) break;
+    if (in(0, j)) {
+      if (!(ok = mbar_wait(&bars->p_full[0], pcount[0]++ & 1, abort))) break;
+      tc_fence_after();
+      pv(0, aV, j > f[0]);
+      if (j == l[0]) tc_commit(&bars->o_final[0]);
+    }
+    const bool next = j < u1;
+    if (next) {
+      if (!(ok = acquire(aK, slotK))) break;
+      if (in(0, j + 1)) {
+        qk(0, aK);
+        tc_commit(&bars->s_full[0]);
+      }
+    }
+    if (in(1, j)) {
+      if (!(ok = mbar_wait(&bars->p_full[1], pcount[1]++ & 1, abort))) break;
+      tc_fence_after();
+      pv(1, aV, j > f[1]);
+      if (j == l[1]) tc_commit(&bars->o_final[1]);
+    }
+    tc_commit(&bars->slot_empty[slotV]);
+    if (next) {
+      if (in(1, j + 1)) {
+        qk(1, aK);
+        tc_commit(&bars->s_full[1]);
+      }
+      tc_commit(&bars->slot_empty[slotK]);
+    }
+  }
+  // All MMAs of this thread must be complete before TMEM is released.
+  tc_commit(&bars->mma_done);
+  drain_wait(&bars->mma_done, 0);
+}
+
+template <typename T, int D>
+__device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem, int X, int b, int h, int q0,
+                              bool has, int f, int l) {
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int r = (warp & 3) * 32 + lane;  // row of the tile == TMEM lane
+  const int q = q0 + X * BM + r;
+  const bool row_ok = q < p.Nq;
+  const RowRange rr = row_range(p, row_ok ? q : p.Nq - 1);
+  const int pos = q + p.Nk - p.Nq;
+  const uint32_t lane_sel = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const uint32_t tS = tmem + lane_sel + X * 256;
+  const uint32_t tO = tS + 128;
+  const bool alibi = p.slopes != nullptr;
+  const float slope_l2 = alibi ? p.slopes[h] * kLog2e : 0.0f;
+
+  float m = -INFINITY;  // running max (log2 units)
+  float lsum = 0.0f;    // running sum of exp2(t - m)
+  bool ok = true;
+  const int n = has ? l - f + 1 : 0;
+  for (int it = 0; it < n; ++it) {
+    const int j = f + it;
+    ok = mbar_wait(&bars->s_full[X], it & 1, abort);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
+    tc_fence_after();
+    uint32_t s[4][32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s[c]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) reg_fence(s[c]);
+
+    // scores -> log2 domain with softcap, ALiBi and mask; tile max
+    const int key0 = j * BN;
+    const bool full_tile = key0 >= rr.lo && key0 + BN - 1 <= rr.hi;
+    float mt = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int key = key0 + 32 * c + e;
+        const float x = __uint_as_float(s[c][e]);
+        float t = p.use_softcap ? p.cap_log2 * tanh_via_exp2(x * p.cap_scale) : x * p.scale_log2;
+        if (alibi) t -= slope_l2 * fabsf(static_cast<float>(pos - key));
+        if (!full_tile && (key < rr.lo || key > rr.hi)) t = -INFINITY;
+        s[c][e] = __float_as_uint(t);
+        mt = fmaxf(mt, t);
+      }
+    }
+    // lazy max update
+    const float m_new = fmaxf(m, mt);
+    float alpha = 1.0f;
+    bool rescale = false;
+    if (m == -INFINITY) {
+      m = m_new;  // nothing accumulated yet for this row (O row is 0, l is 0)
+    } else if (m_new > m + kRescaleThreshold) {
+      alpha = ex2(m - m_new);
+      m = m_new;
+      rescale = true;
+    }
+    lsum *= alpha;
+    const float m_eff = (m == -INFINITY) ? 0.0f : m;
+    // P = exp2(t - m) into the first 64 columns of S (frees the score registers)
+    float rs = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float p0 = ex2(__uint_as_float(s[c][2 * e]) - m_eff);
+        const float p1 = ex2(__uint_as_float(s[c][2 * e + 1]) - m_eff);
+        rs += p0 + p1;
+        pk[e] = pack2<T>(p0, p1);
+      }
+      tmem_st16(tS + 16 * c, pk);
+    }
+    // O_X is idle here (its last product finished before S_X was published)
+    if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * cc, o);
+        tmem_wait_ld();
+        reg_fence(o);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+        tmem_st32(tO + 32 * cc, o);
+      }
+    }
+    lsum += rs;
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars->p_full[X]);
+  }
+  if (ok && n > 0) {
+    ok = mbar_wait(&bars->o_final[X], 0, abort);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+  }
+
+  // epilogue: O / l -> dtype, LSE = (m + log2 l) ln 2
+  T* orow = reinterpret_cast<T*>(p.out) + ((static_cast<size_t>(b) * p.Nq + (row_ok ? q : 0)) * p.H + h) * D;
+  const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+  const float nan = __int_as_float(0x7fc00000);
+  if (ok && n > 0) {
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t o[32];
+      tmem_ld32(tO + 32 * cc, o);
+      tmem_wait_ld();
+      reg_fence(o);
+      if (row_ok) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack2<T>(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cc);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+      }
+    }
+  } else if (row_ok) {
+    const float fill = ok ? 0.0f : nan;
+    const uint32_t w = pack2<T>(fill, fill);
+    uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+    for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(w, w, w, w);
+  }
+  if (row_ok) {
+    float lse_v;
+    if (!ok) lse_v = nan;
+    else if (lsum > 0.0f) lse_v = (m + lg2(lsum)) * kLn2;
+    else lse_v = -INFINITY;
+    p.lse[(static_cast<size_t>(b) * p.H + h) * p.Nq + q] = lse_v;
+  }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + 2 * C::kTileBytes;
+  Barriers* bars = reinterpret_cast<Barriers*>(sKV + C::kSlots * C::kTileBytes);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // 1-D grid, the pairs of one (b, h) adjacent so they share K/V in L2;
+  // within a head the longest causal work is dispatched first.
+  const int bh = static_cast<int>(blockIdx.x) / p.num_pairs;
+  const int pair = p.num_pairs - 1 - static_cast<int>(blockIdx.x) % p.num_pairs;
+  const int b = bh / p.H, h = bh % p.H;
+  const int q0 = pair * 2 * BM;
+
+  // K/V tile range of each Q tile (rows' visible intervals are monotone in q)
+  bool has[2];
+  int f[2], l[2];
+#pragma unroll
+  for (int X = 0; X < 2; ++X) {
+    const int r0 = q0 + X * BM;
+    has[X] = false;
+    f[X] = 0;
+    l[X] = -1;
+    if (r0 < p.Nq) {
+      const int r1 = min(r0 + BM - 1, p.Nq - 1);
+      const RowRange a = row_range(p, r0), z = row_range(p, r1);
+      if (a.lo <= z.hi) {
+        has[X] = true;
+        f[X] = a.lo / BN;
+        l[X] = z.hi / BN;
+      }
+    }
+  }
+  const bool any = has[0] || has[1];
+  const int u0 = has[0] ? f[0] : f[1];
+  const int u1 = has[1] ? l[1] : l[0];
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int i = 0; i < C::kSlots; ++i) {
+      mbar_init(&bars->slot_full[i], 1);
+      mbar_init(&bars->slot_empty[i], 1);
+    }
+    for (int X = 0; X < 2; ++X) {
+      mbar_init(&bars->s_full[X], 1);
+      mbar_init(&bars->p_full[X], 4);
+      mbar_init(&bars->o_final[X], 1);
+    }
+    mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp < 8) {
+    const int X = warp >> 2;
+    softmax_group<T, D>(p, bars, tmem, X, b, h, q0, has[X], f[X], l[X]);
+  } else if (warp == 8) {
+    if (lane == 0 && any) producer<T, D>(&tmQ, &tmK, &tmV, sQ, sKV, bars, b, h, q0, has, u0, u1);
+  } else {
+    if (lane == 0 && any) mma_issuer<T, D>(sQ, sKV, bars, tmem, has, f, l, u0, u1);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const FwdParams& p,
+                   cudaStream_t stream) {
+  using C = Cfg<D>;
+  static_assert(sizeof(Barriers) <= 1024, "barrier block exceeds its reserve");
+  static_assert(C::kSmemBytes <= 232448, "shared memory budget exceeded");
+  auto kernel = fwd_kernel<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.num_pairs * p.B * p.H);
+  kernel<<<grid, kThreads, C::kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(bool bf16, int d, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                       const FwdParams& p, cudaStream_t stream) {
+  if (bf16) return d == 128 ? launch<__nv_bfloat16, 128>(tmQ, tmK, tmV, p, stream)
+                            : launch<__nv_bfloat16, 64>(tmQ, tmK, tmV, p, stream);
+  return d == 128 ? launch<__half, 128>(tmQ, tmK, tmV, p, stream) : launch<__half, 64>(tmQ, tmK, tmV, p, stream);
+}
+
+}  // namespace fa

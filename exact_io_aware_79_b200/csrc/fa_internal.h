@@ -1,0 +1,55 @@
+// fa_internal.h -- parameter blocks and launchers shared between the C-ABI
+// layer (fa_api.cu) and the kernel translation units. Not part of the ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime_api.h>
+
+namespace fa {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Forward: one CTA owns two adjacent 128-row query tiles of one (b, h).
+struct FwdParams {
+  void* out;            // [B, Nq, H, d]
+  float* lse;           // [B, H, Nq]
+  const float* slopes;  // [H] or nullptr
+  int B, H, Nq, Nk;
+  int num_pairs;        // ceil(Nq / 256)
+  int causal;
+  int window_left, window_right;  // -1 = unbounded
+  int use_softcap;
+  float scale_log2;  // scale * log2(e)                  (no softcap)
+  float cap_scale;   // scale / softcap                   (softcap)
+  float cap_log2;    // softcap * log2(e)                 (softcap)
+};
+
+// Paged decode, split kernel + merge kernel.
+struct DecodeParams {
+  const void* q;        // [B, 1, H, d]
+  const void* k_cache;  // [num_pages, page_size, H, d]
+  const void* v_cache;
+  const int* block_table;    // [B, max_blocks]
+  const int* cache_seqlens;  // [B]
+  void* out;                 // [B, 1, H, d]   (num_splits == 1)
+  float* lse;                // [B, H, 1]      (num_splits == 1)
+  float* o_part;             // [S, B, H, d]   (num_splits > 1)
+  float* lse_part;           // [S, B, H]      (num_splits > 1)
+  const float* slopes;       // [H] or nullptr
+  int B, H, num_pages, page_size, max_blocks, num_splits;
+  int window_left;
+  int use_softcap;
+  float scale_log2, cap_scale, cap_log2;
+};
+
+// Launches the forward kernel for (dtype, d); the tensor maps describe Q, K, V
+// as 4-D tensors (d, H, N, B) with a (64, 1, 128, 1) box and 128-byte swizzle.
+cudaError_t launch_fwd(bool bf16, int d, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                       const FwdParams& p, cudaStream_t stream);
+
+cudaError_t launch_decode(bool bf16, int d, const DecodeParams& p, cudaStream_t stream);
+
+}  // namespace fa

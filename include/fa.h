@@ -1,0 +1,166 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library.
+ *
+ * Two operations, both exact scaled-dot-product attention
+ *     O = softmax(S) V,   S = scale * Q K^T  (+ score modifiers, + mask),
+ * computed tile by tile with an online softmax so that neither the score
+ * matrix S nor the probability matrix P ever reaches device memory, plus the
+ * per-row natural log-sum-exp LSE_i = ln sum_j exp(S_ij).
+ *
+ * Sources (web pages about FlashAttention; their formulas were lost in
+ * extraction, so the readings below state the plain form that the rest of the
+ * text supports):
+ *   - standard attention and its N x N intermediates: "FlashAttention及变种改进",
+ *     section 二.1 "标准自注意力的计算瓶颈";
+ *   - tiling into on-chip blocks, online (row-block) softmax, async copy
+ *     overlapped with compute: "IO感知技术革命：FlashAttention如何重塑大模型训练的
+ *     经济学", sections "分块计算的投资回报模型", "在线Softmax的现金流优化",
+ *     "异步执行的供应链思维"; softmax fused with both matmuls:
+ *     "FlashAttention深度解析", section "重新定义注意力计算";
+ *   - bottom-right causal alignment, split-KV decode with a merge kernel,
+ *     sliding window, ALiBi, paged KV cache through a block table, tanh
+ *     softcapping: "Flash-Attention v2.0 到 v2.7 更新", opening paragraph and
+ *     sections v2.1, v2.2, v2.3, v2.4, v2.5, v2.6.
+ *
+ * Conventions shared by both calls
+ *   - Every tensor pointer is a DEVICE pointer to contiguous memory, 16-byte
+ *     aligned, owned by the caller. The library allocates nothing, keeps no
+ *     pointer after a call returns and holds no global state besides a
+ *     per-device cache of device properties.
+ *   - Element types: Q, K, V and O are fp16 or bf16 (fa_dtype); LSE is fp32;
+ *     block tables and lengths are int32; ALiBi slopes are fp32. Arithmetic
+ *     is fp32 (the two products run on tensor cores with fp32 accumulation).
+ *   - Score modifiers, applied in this order to s = scale * (q . k):
+ *       softcap > 0:   s = softcap * tanh(s / softcap)
+ *       alibi_slopes:  s += -alibi_slopes[h] * |pos_i - j|
+ *       mask:          s = -inf for every key j that query i may not see.
+ *     Query row i (0-based) of Nq sits at key position pos_i = i + Nk - Nq
+ *     (bottom-right alignment: the last query meets the last key). Key j is
+ *     visible iff
+ *       (!causal || j <= pos_i) and
+ *       (window_left  < 0 || j >= pos_i - window_left) and
+ *       (window_right < 0 || j <= pos_i + window_right).
+ *   - A query row that sees no key gets O = 0 and LSE = -inf.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream): they
+ *     validate their arguments, enqueue kernels and return; they never
+ *     synchronise. Invalid arguments are reported before anything is
+ *     enqueued; FA_ERR_CUDA reports a failed launch or CUDA call.
+ *   - Requires a compute-capability 10.0 device (B200); elsewhere the calls
+ *     return FA_ERR_DEVICE.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_NULL = 1,      /* a required pointer is NULL */
+    FA_ERR_SHAPE = 2,     /* a size is negative or beyond a stated limit */
+    FA_ERR_DTYPE = 3,     /* dtype is not FA_FP16 / FA_BF16 */
+    FA_ERR_HEADDIM = 4,   /* d is not 64 or 128 */
+    FA_ERR_ARG = 5,       /* scale/softcap not finite or negative cap, window < -1,
+                             page_size < 1, num_splits outside [0, FA_MAX_SPLITS],
+                             or a pointer not 16-byte aligned */
+    FA_ERR_WORKSPACE = 6, /* split-KV workspace missing, misaligned or too small */
+    FA_ERR_CUDA = 7,      /* a CUDA runtime/driver call or a launch failed */
+    FA_ERR_DEVICE = 8     /* no device, or the current device is not sm_100 */
+} fa_status;
+
+typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
+
+#define FA_MAX_SPLITS 64
+
+/*
+ * fa_fwd -- tiled attention forward (prefill / training shape).
+ *
+ *   q    [B, Nq, H, d]   fp16/bf16, read
+ *   k, v [B, Nk, H, d]   fp16/bf16, read
+ *   out  [B, Nq, H, d]   same dtype, written
+ *   lse  [B, H, Nq]      fp32, written (natural log)
+ *   scale                multiplies q . k (typically 1/sqrt(d)); finite
+ *   causal               0/1, bottom-right aligned as above
+ *   window_left/right    -1 = unbounded, else >= 0 (inclusive bounds)
+ *   alibi_slopes         [H] fp32 device array, or NULL for no ALiBi
+ *   softcap              0 = off, else > 0 and finite
+ *
+ * Limits: B, H, Nq, Nk >= 0; B*H < 2^31; Nq <= 2^24. B*H*Nq == 0 is a no-op;
+ * Nk == 0 makes every row empty. d is 64 or 128. out must not alias q, k or v.
+ */
+fa_status fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
+                 int B, int H, int Nq, int Nk, int d, fa_dtype dtype, float scale,
+                 int causal, int window_left, int window_right,
+                 const float *alibi_slopes, float softcap, cudaStream_t stream);
+
+/*
+ * fa_fwd_kvcache -- split-KV ("flash-decoding") attention of one new query
+ * token per sequence over a paged KV cache.
+ *
+ *   q             [B, 1, H, d]                      fp16/bf16, read
+ *   k_cache,
+ *   v_cache       [num_pages, page_size, H, d]      fp16/bf16, read
+ *   block_table   [B, max_blocks] int32: token t of sequence b is row
+ *                 t % page_size of page block_table[b][t / page_size]
+ *   cache_seqlens [B] int32: L_b, the number of cached tokens of sequence b
+ *                 (the new token's own k/v must already be in the cache)
+ *   out           [B, 1, H, d]                      same dtype, written
+ *   lse           [B, H, 1]                         fp32, written
+ *   window_left   -1 = unbounded, else keys j >= L_b - 1 - window_left
+ *   alibi_slopes  [H] fp32 or NULL;  softcap as in fa_fwd
+ *   num_splits    0 = automatic (fa_kvcache_num_splits), else 1..FA_MAX_SPLITS
+ *   workspace     device scratch of at least fa_kvcache_workspace_size(...)
+ *                 bytes, 16-byte aligned; may be NULL when that size is 0.
+ *                 Its contents on entry do not matter; it is clobbered.
+ *
+ * The query sits at position L_b - 1, so causally it sees all L_b keys (the
+ * decode example of bottom-right alignment). Each sequence's visible keys are
+ * cut into num_splits contiguous ranges of equal whole-page length; a
+ * split kernel computes a partial (O_s, LSE_s) per range and, when more than
+ * one split is used, a merge kernel forms LSE = ln sum_s exp(LSE_s) and
+ * O = sum_s exp(LSE_s - LSE) O_s.
+ *
+ * Device-side values cannot be checked before launch. An L_b outside
+ * [0, max_blocks * page_size] or a referenced block-table entry outside
+ * [0, num_pages) is never dereferenced; that sequence's O and LSE rows are
+ * set to NaN instead. L_b == 0 gives O = 0, LSE = -inf.
+ *
+ * Limits: B >= 0 (0 is a no-op), H >= 1, B*H*FA_MAX_SPLITS < 2^31,
+ * num_pages >= 1, page_size >= 1, max_blocks >= 1,
+ * max_blocks * page_size < 2^31.
+ */
+fa_status fa_fwd_kvcache(const void *q, const void *k_cache, const void *v_cache,
+                         const int *block_table, const int *cache_seqlens,
+                         void *out, float *lse,
+                         int B, int H, int d, int num_pages, int page_size, int max_blocks,
+                         fa_dtype dtype, float scale, int window_left,
+                         const float *alibi_slopes, float softcap, int num_splits,
+                         void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Number of splits fa_fwd_kvcache uses for these sizes: num_splits itself
+ * when it is 1..FA_MAX_SPLITS, else the automatic choice, which depends only
+ * on B, H and the longest possible sequence max_blocks * page_size (host-side
+ * sizes, so no device read is needed). Returns -1 for invalid sizes.
+ */
+int fa_kvcache_num_splits(int B, int H, int d, int max_blocks, int page_size, int num_splits);
+
+/*
+ * Bytes of workspace fa_fwd_kvcache needs for these sizes (0 when a single
+ * split is used). Returns 0 for invalid sizes as well; fa_fwd_kvcache then
+ * reports the invalid argument.
+ */
+size_t fa_kvcache_workspace_size(int B, int H, int d, int max_blocks, int page_size, int num_splits);
+
+/* Static, human-readable name of a status code. */
+const char *fa_status_string(fa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

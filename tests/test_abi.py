@@ -1,0 +1,146 @@
+"""C-ABI checks that need no GPU: symbols, status strings, argument validation,
+split-count and workspace arithmetic.
+
+Validation happens before any CUDA call, so on a machine without a device the
+invalid calls return their own status and valid ones return FA_ERR_DEVICE.
+Fake device addresses are passed for pointers; nothing dereferences them.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_79_b200 import build as fbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+OK, NULL, SHAPE, DTYPE, HEADDIM, ARG, WORKSPACE, CUDA, DEVICE = range(9)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fbuild.build()
+    import exact_io_aware_79_b200 as fa
+    return fa.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    assert {"fa_fwd", "fa_fwd_kvcache", "fa_kvcache_num_splits", "fa_kvcache_workspace_size",
+            "fa_status_string"} <= set(names)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(9):
+        s = lib.fa_status_string(code).decode()
+        assert s.startswith(["FA_OK", "FA_ERR_NULL", "FA_ERR_SHAPE", "FA_ERR_DTYPE", "FA_ERR_HEADDIM",
+                             "FA_ERR_ARG", "FA_ERR_WORKSPACE", "FA_ERR_CUDA", "FA_ERR_DEVICE"][code])
+    assert "unknown" in lib.fa_status_string(99).decode()
+
+
+P = 0x10000  # fake 16-byte-aligned device address
+
+
+def fwd(lib, q=P, k=P, v=P, out=P, lse=P, B=1, H=2, Nq=128, Nk=128, d=128, dtype=1, scale=0.1, causal=0,
+        wl=-1, wr=-1, slopes=None, cap=0.0):
+    return lib.fa_fwd(q, k, v, out, lse, B, H, Nq, Nk, d, dtype, scale, causal, wl, wr, slopes, cap, None)
+
+
+def test_fwd_validation(lib):
+    assert fwd(lib, d=96) == HEADDIM
+    assert fwd(lib, d=256) == HEADDIM
+    assert fwd(lib, dtype=2) == DTYPE
+    assert fwd(lib, B=-1) == SHAPE
+    assert fwd(lib, Nq=-3) == SHAPE
+    assert fwd(lib, Nk=1 << 29) == SHAPE
+    assert fwd(lib, wl=-2) == ARG
+    assert fwd(lib, wr=-5) == ARG
+    assert fwd(lib, cap=-1.0) == ARG
+    assert fwd(lib, cap=float("inf")) == ARG
+    assert fwd(lib, scale=float("nan")) == ARG
+    assert fwd(lib, causal=2) == ARG
+    assert fwd(lib, q=None) == NULL
+    assert fwd(lib, lse=None) == NULL
+    assert fwd(lib, k=None) == NULL
+    assert fwd(lib, out=P + 8) == ARG          # misaligned
+    # empty problems are no-ops, even with NULL pointers
+    assert fwd(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == OK
+    assert fwd(lib, Nq=0) == OK
+    # Nk == 0 needs no K/V pointers
+    r = fwd(lib, Nk=0, k=None, v=None)
+    assert r in (OK, DEVICE)
+
+
+def test_fwd_reaches_the_device_check_without_gpu(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert fwd(lib) == DEVICE
+
+
+def kv(lib, q=P, kc=P, vc=P, bt=P, sl=P, out=P, lse=P, B=4, H=2, d=128, num_pages=64, page=256, mb=16,
+       dtype=1, scale=0.1, wl=-1, slopes=None, cap=0.0, splits=1, ws=None, ws_bytes=0):
+    return lib.fa_fwd_kvcache(q, kc, vc, bt, sl, out, lse, B, H, d, num_pages, page, mb, dtype, scale, wl,
+                              slopes, cap, splits, ws, ws_bytes, None)
+
+
+def test_kvcache_validation(lib):
+    assert kv(lib, d=80) == HEADDIM
+    assert kv(lib, dtype=7) == DTYPE
+    assert kv(lib, H=0) == SHAPE
+    assert kv(lib, num_pages=0) == SHAPE
+    assert kv(lib, page=0) == ARG
+    assert kv(lib, splits=65) == ARG
+    assert kv(lib, splits=-1) == ARG
+    assert kv(lib, wl=-2) == ARG
+    assert kv(lib, cap=-0.5) == ARG
+    assert kv(lib, B=70000) == SHAPE
+    assert kv(lib, mb=1 << 24, page=256) == SHAPE
+    assert kv(lib, bt=None) == NULL
+    assert kv(lib, sl=None) == NULL
+    assert kv(lib, kc=P + 2) == ARG
+    assert kv(lib, sl=P + 2) == ARG
+    assert kv(lib, B=0, q=None) == OK
+    need = lib.fa_kvcache_workspace_size(4, 2, 128, 16, 256, 4)
+    assert need > 0
+    assert kv(lib, splits=4, ws=None, ws_bytes=0) == WORKSPACE
+    assert kv(lib, splits=4, ws=P, ws_bytes=need - 1) == WORKSPACE
+    assert kv(lib, splits=4, ws=P + 4, ws_bytes=need) == WORKSPACE
+    assert kv(lib, splits=4, ws=P, ws_bytes=need) in (OK, DEVICE)
+    assert kv(lib, splits=1, ws=None) in (OK, DEVICE)
+
+
+def test_split_count_resolution(lib):
+    ns = lib.fa_kvcache_num_splits
+    assert ns(64, 32, 128, 128, 256, 0) == 16      # 32K max length -> 2048-key splits
+    assert ns(64, 32, 128, 128, 256, 5) == 5       # explicit
+    assert ns(1, 8, 128, 16, 256, 0) == 16         # small batch: fill the GPU, >= 256 keys a split
+    assert ns(1, 1, 128, 1, 256, 0) == 1           # one page: nothing to split
+    assert ns(1024, 32, 128, 4, 256, 0) == 1       # short sequences, many heads
+    assert ns(4, 2, 128, 16, 256, 65) == -1
+    assert ns(4, 2, 96, 16, 256, 0) == -1
+    for args in [(64, 32, 128, 128, 256), (3, 5, 64, 7, 16), (1, 1, 128, 2000, 16)]:
+        assert 1 <= ns(*args, 0) <= 64
+
+
+def test_workspace_size(lib):
+    ws = lib.fa_kvcache_workspace_size
+    assert ws(64, 32, 128, 128, 256, 1) == 0
+    rows = 16 * 64 * 32
+    o_bytes = (rows * 128 * 4 + 255) // 256 * 256
+    assert ws(64, 32, 128, 128, 256, 16) == o_bytes + rows * 4
+    assert ws(64, 32, 128, 128, 256, 0) == ws(64, 32, 128, 128, 256, 16)
+    assert ws(4, 2, 96, 16, 256, 4) == 0          # invalid head dim
