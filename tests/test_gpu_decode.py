@@ -1,6 +1,6 @@
 """GPU parity of fa_fwd_kvcache (through the C ABI) against the fp64 oracle.
 
-Same tolerances as the forward. Block-table indexing is checked bit-exactly
+Same tolerances as the forward (O bound times the input scale sigma). Block-table indexing is checked bit-exactly
 with one-hot probes whose expected output is an integer code of the probed
 token's logical index.
 """
@@ -37,13 +37,13 @@ def run_gpu(q, kc, vc, table, lens, scale, wl=-1, slopes=None, cap=0.0, splits=0
     return out.float().cpu().numpy(), lse.cpu().numpy()
 
 
-def compare(out, lse, o_ref, l_ref, dtype, what):
+def compare(out, lse, o_ref, l_ref, dtype, what, sigma=1.0):
     fin = np.isfinite(l_ref)
     assert np.array_equal(np.isfinite(lse), fin), what
     assert np.all(lse[~fin] == -np.inf), what
     o_err = float(np.abs(out - o_ref).max())
     l_err = float(np.abs(lse[fin] - l_ref[fin]).max()) if fin.any() else 0.0
-    assert o_err <= O_TOL[dtype], "%s: O error %.3g" % (what, o_err)
+    assert o_err <= O_TOL[dtype] * sigma, "%s: O error %.3g" % (what, o_err)
     assert l_err <= LSE_TOL, "%s: LSE error %.3g" % (what, l_err)
 
 
@@ -68,7 +68,7 @@ def test_decode_matches_oracle(case, splits):
     scale = 1.0 / math.sqrt(d)
     out, lse = run_gpu(q, kc, vc, table, lens_t, scale, wl, slopes, cap, splits)
     o_ref, l_ref = oracle.attn_decode_paged(q, kc, vc, table, lens_t, scale, wl, slopes, cap)
-    compare(out, lse, o_ref, l_ref, dtype, "%s splits=%d" % (case, splits))
+    compare(out, lse, o_ref, l_ref, dtype, "%s splits=%d" % (case, splits), sigma)
 
 
 def test_identity_table_equals_contiguous_forward():

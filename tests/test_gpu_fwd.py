@@ -2,7 +2,10 @@
 
 Tolerances (the spec's): max |O_gpu - O_oracle| <= 1.6e-2 for bf16 and 4e-3
 for fp16; max |LSE_gpu - LSE_oracle| <= 1e-3 where finite; rows the oracle
-finds empty must be exactly O = 0, LSE = -inf. Mask membership is checked
+finds empty must be exactly O = 0, LSE = -inf. O is linear in V, and the O
+bounds are stated for unit-scale inputs; a case whose inputs are drawn with
+scale sigma gets sigma times the O bound (with sigma = 2 some |O| exceed 8,
+where half a bf16 ulp of the output alone is 0.031). Mask membership is checked
 bit-exactly on every row by the boundary probes.
 """
 import math
@@ -30,13 +33,13 @@ def gpu_fwd(q, k, v, scale, causal=False, wl=-1, wr=-1, slopes=None, softcap=0.0
     return out.float().cpu().numpy(), lse.cpu().numpy()
 
 
-def compare(out, lse, o_ref, l_ref, dtype, what=""):
+def compare(out, lse, o_ref, l_ref, dtype, what="", sigma=1.0):
     fin = np.isfinite(l_ref)
     assert np.array_equal(np.isfinite(lse), fin), what + ": empty-row pattern differs"
     assert np.all(lse[~fin] == -np.inf), what
     o_err = float(np.abs(out - o_ref).max()) if out.size else 0.0
     l_err = float(np.abs(lse[fin] - l_ref[fin]).max()) if fin.any() else 0.0
-    assert o_err <= O_TOL[dtype], "%s: O max-abs error %.3g" % (what, o_err)
+    assert o_err <= O_TOL[dtype] * sigma, "%s: O max-abs error %.3g" % (what, o_err)
     assert l_err <= LSE_TOL, "%s: LSE max-abs error %.3g" % (what, l_err)
     return o_err, l_err
 
@@ -76,7 +79,7 @@ def test_small_cases_match_oracle(case):
     scale = 1.0 / math.sqrt(d)
     out, lse = gpu_fwd(q, k, v, scale, causal, wl, wr, slopes, cap)
     o_ref, l_ref = oracle.attn_fwd(q, k, v, scale, causal, wl, wr, slopes, cap)
-    compare(out, lse, o_ref, l_ref, dtype, str(case))
+    compare(out, lse, o_ref, l_ref, dtype, str(case), sigma)
 
 
 def test_no_keys_gives_empty_rows():
@@ -113,7 +116,7 @@ def test_full_size_workloads_on_sampled_rows(w):
                                    x["slopes"], w.softcap, rows=rows)
     o = out[:, rows].float().cpu().numpy()
     l = lse[:, :, rows].cpu().numpy()
-    compare(o, l, o_ref, l_ref, w.dtype, w.name)
+    compare(o, l, o_ref, l_ref, w.dtype, w.name, w.sigma)
     assert torch.isfinite(out).all().item()
 
 
