@@ -30,6 +30,7 @@ LIB_PATH = os.path.join(_PKG, "libfa_b200.so")
 
 FA_FP16, FA_BF16 = 0, 1
 FA_MAX_SPLITS = 64
+FA_NOALLOC_SCRATCH_BYTES = 32 << 20
 STATUS = {
     0: "FA_OK", 1: "FA_ERR_NULL", 2: "FA_ERR_SHAPE", 3: "FA_ERR_DTYPE", 4: "FA_ERR_HEADDIM",
     5: "FA_ERR_ARG", 6: "FA_ERR_WORKSPACE", 7: "FA_ERR_CUDA", 8: "FA_ERR_DEVICE",
@@ -58,6 +59,9 @@ def _lib_handle():
         L.fa_fwd_kvcache.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp, f, i, vp, sz,
                                      vp]
         L.fa_fwd_kvcache.restype = i
+        L.fa_fwd_kvcache_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp, f, i,
+                                             vp]
+        L.fa_fwd_kvcache_noalloc.restype = i
         L.fa_kvcache_num_splits.argtypes = [i, i, i, i, i, i]
         L.fa_kvcache_num_splits.restype = i
         L.fa_kvcache_workspace_size.argtypes = [i, i, i, i, i, i]
@@ -155,6 +159,33 @@ def fa_fwd_kvcache(q, k_cache, v_cache, block_table, cache_seqlens, out, lse, sc
         B, H, d, num_pages, page_size, max_blocks, _dtype_code(q), float(scale), int(window_left),
         _ptr(alibi_slopes), float(softcap), int(num_splits), _ptr(workspace), ws_bytes, _stream(stream))
     _check(code, "fa_fwd_kvcache")
+
+
+def fa_fwd_kvcache_noalloc(q, k_cache, v_cache, block_table, cache_seqlens, out, lse, scale: float,
+                           window_left: int = -1, alibi_slopes=None, softcap: float = 0.0, num_splits: int = 0,
+                           stream=None) -> None:
+    """fa_fwd_kvcache without a workspace argument, for callers that cannot
+    allocate device memory: the split partials live in the library's own
+    fixed device array (FA_NOALLOC_SCRATCH_BYTES per GPU). Calls on one
+    device share that array, so order them on one stream."""
+    B, one, H, d = q.shape
+    num_pages, page_size = k_cache.shape[0], k_cache.shape[1]
+    max_blocks = block_table.shape[1]
+    for t in (q, k_cache, v_cache, block_table, cache_seqlens, out, lse):
+        if not t.is_contiguous():
+            raise ValueError("fa_fwd_kvcache_noalloc needs contiguous tensors")
+    if one != 1 or tuple(k_cache.shape) != (num_pages, page_size, H, d) or \
+            tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("fa_fwd_kvcache_noalloc: shape mismatch")
+    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32 or block_table.shape[0] != B:
+        raise ValueError("fa_fwd_kvcache_noalloc: block_table / cache_seqlens must be int32 [B, ...]")
+    if tuple(lse.shape) != (B, H, 1) or lse.dtype != torch.float32:
+        raise ValueError("fa_fwd_kvcache_noalloc: lse must be fp32 [B, H, 1]")
+    code = _lib_handle().fa_fwd_kvcache_noalloc(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(cache_seqlens), _ptr(out), _ptr(lse),
+        B, H, d, num_pages, page_size, max_blocks, _dtype_code(q), float(scale), int(window_left),
+        _ptr(alibi_slopes), float(softcap), int(num_splits), _stream(stream))
+    _check(code, "fa_fwd_kvcache_noalloc")
 
 
 def attention(q, k, v, scale: Optional[float] = None, causal: bool = False, window_left: int = -1,

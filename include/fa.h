@@ -26,7 +26,8 @@
  *   - Every tensor pointer is a DEVICE pointer to contiguous memory, 16-byte
  *     aligned, owned by the caller. The library allocates nothing, keeps no
  *     pointer after a call returns and holds no global state besides a
- *     per-device cache of device properties.
+ *     per-device cache of device properties and the fixed device array of
+ *     fa_fwd_kvcache_noalloc.
  *   - Element types: Q, K, V and O are fp16 or bf16 (fa_dtype); LSE is fp32;
  *     block tables and lengths are int32; ALiBi slopes are fp32. Arithmetic
  *     is fp32 (the two products run on tensor cores with fp32 accumulation).
@@ -155,6 +156,43 @@ int fa_kvcache_num_splits(int B, int H, int d, int max_blocks, int page_size, in
  * reports the invalid argument.
  */
 size_t fa_kvcache_workspace_size(int B, int H, int d, int max_blocks, int page_size, int num_splits);
+
+/* Size of the device array fa_fwd_kvcache_noalloc keeps its split partials in. */
+#define FA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * fa_fwd_kvcache_noalloc -- fa_fwd_kvcache for callers that cannot allocate
+ * device memory. The pages have no counterpart to this call; it exists for
+ * this library's users: a plain C host program or plugin without a device
+ * allocator of its own, a component inside another runtime whose memory pool
+ * already holds the free device memory (so its own cudaMalloc would fail),
+ * or a latency-bound decode loop that must not call cudaMalloc, which can
+ * synchronise the device.
+ *
+ * Arguments, layouts, results and errors are those of fa_fwd_kvcache minus
+ * the workspace: the split partials go to a file-scope device array of
+ * FA_NOALLOC_SCRATCH_BYTES (32 MiB) inside the library, which every GPU that
+ * loads the library holds until the process exits. The call allocates
+ * nothing and calls no cudaMalloc or cudaFree.
+ *   - Sizes whose partials need more than FA_NOALLOC_SCRATCH_BYTES
+ *     (fa_kvcache_workspace_size(...) > FA_NOALLOC_SCRATCH_BYTES) are
+ *     rejected with FA_ERR_WORKSPACE before anything is enqueued; pass a
+ *     smaller explicit num_splits or use fa_fwd_kvcache.
+ *   - The first call on a device that needs the array (more than one split)
+ *     looks up the array's device address for that device, with that device
+ *     current; make that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     partials. Each call overwrites every partial it reads, so nothing needs
+ *     clearing, but calls whose kernels overlap on the GPU (different streams
+ *     without ordering) race on the array: order them on one stream.
+ */
+fa_status fa_fwd_kvcache_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                 const int *block_table, const int *cache_seqlens,
+                                 void *out, float *lse,
+                                 int B, int H, int d, int num_pages, int page_size, int max_blocks,
+                                 fa_dtype dtype, float scale, int window_left,
+                                 const float *alibi_slopes, float softcap, int num_splits,
+                                 cudaStream_t stream);
 
 /* Static, human-readable name of a status code. */
 const char *fa_status_string(fa_status status);
