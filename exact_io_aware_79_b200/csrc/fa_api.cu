@@ -161,8 +161,12 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
   p.window_left = window_left;
   p.window_right = window_right;
   p.use_softcap = softcap > 0.0f;
-  p.scale_log2 = scale * fa::kLog2e;
-  p.cap_scale = softcap > 0.0f ? scale / softcap : 0.0f;
+  // softmax(scale * q.k) with scale < 0 equals softmax(|scale| * (-q).k): the
+  // kernel negates the QK^T product on the tensor core and works with |scale|.
+  p.negate_scores = scale < 0.0f;
+  const float mag = std::fabs(scale);
+  p.scale_log2 = mag * fa::kLog2e;
+  p.cap_scale = softcap > 0.0f ? mag / softcap : 0.0f;
   p.cap_log2 = softcap * fa::kLog2e;
   return fa::launch_fwd(bf16, d, tq, tk, tv, p, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

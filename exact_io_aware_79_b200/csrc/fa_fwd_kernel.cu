@@ -137,10 +137,11 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const C
 
 template <typename T, int D>
 __device__ void mma_issuer(uint8_t* sQ, uint8_t* sKV, Barriers* bars, uint32_t tmem, const bool (&has)[2],
-                           const int (&f)[2], const int (&l)[2], int u0, int u1) {
+                           const int (&f)[2], const int (&l)[2], int u0, int u1, bool negate) {
   using C = Cfg<D>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-  constexpr uint32_t idesc_qk = instr_desc_f16(kBf16, BM, BN, false);
+  // a negative softmax scale is applied as -Q K^T (A-negate bit) times |scale|
+  const uint32_t idesc_qk = instr_desc_f16(kBf16, BM, BN, false) | (negate ? (1u << 13) : 0u);
   constexpr uint32_t idesc_pv = instr_desc_f16(kBf16, BM, D, true);
   volatile int* abort = &bars->abort;
   const uint32_t sQaddr = smem_addr(sQ);
@@ -231,9 +232,22 @@ __device__ void mma_issuer(uint8_t* sQ, uint8_t* sKV, Barriers* bars, uint32_t t
   drain_wait(&bars->mma_done, 0);
 }
 
-template <typename T, int D>
+// Score transform of one element in log2 units (softcap and ALiBi paths).
+template <bool kCap, bool kAlibi>
+__device__ __forceinline__ float mod_score(const FwdParams& p, float x, float slope_l2, int dist) {
+  float t = kCap ? p.cap_log2 * tanh_via_exp2(x * p.cap_scale) : x * p.scale_log2;
+  if (kAlibi) t -= slope_l2 * fabsf(static_cast<float>(dist));
+  return t;
+}
+
+// One softmax warpgroup (tile X): one query row per thread, row == TMEM lane.
+// kCap / kAlibi select the score modifiers at compile time; whether a K tile
+// needs the element mask is decided per tile for the whole group, so the
+// common interior tiles run without per-element compares.
+template <typename T, int D, bool kCap, bool kAlibi>
 __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem, int X, int b, int h, int q0,
                               bool has, int f, int l) {
+  constexpr bool kPlain = !kCap && !kAlibi;
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -241,12 +255,17 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
   const int q = q0 + X * BM + r;
   const bool row_ok = q < p.Nq;
   const RowRange rr = row_range(p, row_ok ? q : p.Nq - 1);
+  // tile-level bounds: a K tile needs no mask when every row of the group
+  // sees all of it (rows' intervals are monotone in q)
+  const int qa = q0 + X * BM;
+  const int qz = min(qa + BM - 1, p.Nq - 1);
+  const RowRange first_row = row_range(p, qa), last_row = row_range(p, qz);
   const int pos = q + p.Nk - p.Nq;
   const uint32_t lane_sel = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const uint32_t tS = tmem + lane_sel + X * 256;
   const uint32_t tO = tS + 128;
-  const bool alibi = p.slopes != nullptr;
-  const float slope_l2 = alibi ? p.slopes[h] * kLog2e : 0.0f;
+  const float slope_l2 = kAlibi ? p.slopes[h] * kLog2e : 0.0f;
+  const float sl2 = p.scale_log2;  // >= 0 (a negative scale is folded into the MMA)
 
   float m = -INFINITY;  // running max (log2 units)
   float lsum = 0.0f;    // running sum of exp2(t - m)
@@ -259,29 +278,51 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
     if (!ok) break;
     tc_fence_after();
     uint32_t s[4][32];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s[c]);
-    tmem_wait_ld();
-#pragma unroll
-    for (int c = 0; c < 4; ++c) reg_fence(s[c]);
-
-    // scores -> log2 domain with softcap, ALiBi and mask; tile max
     const int key0 = j * BN;
-    const bool full_tile = key0 >= rr.lo && key0 + BN - 1 <= rr.hi;
-    float mt = -INFINITY;
+    const bool masked = key0 < last_row.lo || key0 + BN - 1 > first_row.hi;  // uniform over the group
+    // pass 1: transform (modifier paths) and tile max. S arrives in two
+    // halves so the second TMEM load overlaps the first half's work; four
+    // independent 3-input max chains keep the pipes busy.
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    auto half_max = [&](int c0) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+      for (int c = c0; c < c0 + 2; ++c) {
+        if (!kPlain || masked) {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int key = key0 + 32 * c + e;
-        const float x = __uint_as_float(s[c][e]);
-        float t = p.use_softcap ? p.cap_log2 * tanh_via_exp2(x * p.cap_scale) : x * p.scale_log2;
-        if (alibi) t -= slope_l2 * fabsf(static_cast<float>(pos - key));
-        if (!full_tile && (key < rr.lo || key > rr.hi)) t = -INFINITY;
-        s[c][e] = __float_as_uint(t);
-        mt = fmaxf(mt, t);
+          for (int e = 0; e < 32; ++e) {
+            float x = __uint_as_float(s[c][e]);
+            const int key = key0 + 32 * c + e;
+            if (!kPlain) x = mod_score<kCap, kAlibi>(p, x, slope_l2, pos - key);
+            if (masked) x = (key >= rr.lo && key <= rr.hi) ? x : -INFINITY;
+            s[c][e] = __float_as_uint(x);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          const int a = (e / 8) & 3;
+          mx[a] = fmax3(mx[a], __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
+          mx[a] = fmax3(mx[a], __uint_as_float(s[c][e + 2]), __uint_as_float(s[c][e + 3]));
+          mx[a] = fmax3(mx[a], __uint_as_float(s[c][e + 4]), __uint_as_float(s[c][e + 5]));
+          mx[a] = fmax3(mx[a], __uint_as_float(s[c][e + 6]), __uint_as_float(s[c][e + 7]));
+        }
       }
-    }
+    };
+    tmem_ld32(tS, s[0]);
+    tmem_ld32(tS + 32, s[1]);
+    tmem_wait_ld();
+    reg_fence(s[0]);
+    reg_fence(s[1]);
+    tmem_ld32(tS + 64, s[2]);
+    tmem_ld32(tS + 96, s[3]);
+    half_max(0);
+    tmem_wait_ld();
+    reg_fence(s[2]);
+    reg_fence(s[3]);
+    half_max(2);
+    float mt = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
+    // plain path: the max was taken over raw scores; scale after (sl2 >= 0)
+    if (kPlain) mt = (mt == -INFINITY) ? -INFINITY : mt * sl2;
+
     // lazy max update
     const float m_new = fmaxf(m, mt);
     float alpha = 1.0f;
@@ -295,20 +336,34 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
     }
     lsum *= alpha;
     const float m_eff = (m == -INFINITY) ? 0.0f : m;
-    // P = exp2(t - m) into the first 64 columns of S (frees the score registers)
-    float rs = 0.0f;
+    // pass 2: P = exp2(t - m) into the first 64 columns of S (frees the score registers)
+    float rsum[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};  // independent partial sums
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        const float p0 = ex2(__uint_as_float(s[c][2 * e]) - m_eff);
-        const float p1 = ex2(__uint_as_float(s[c][2 * e + 1]) - m_eff);
-        rs += p0 + p1;
+        const float x0 = __uint_as_float(s[c][2 * e]);
+        const float x1 = __uint_as_float(s[c][2 * e + 1]);
+        float p0, p1;
+        if (kPlain) {
+          // masked entries hold -inf; -inf * 0 would be NaN, so select them out
+          p0 = ex2(fmaf(x0, sl2, -m_eff));
+          p1 = ex2(fmaf(x1, sl2, -m_eff));
+          if (masked) {
+            p0 = (x0 == -INFINITY) ? 0.0f : p0;
+            p1 = (x1 == -INFINITY) ? 0.0f : p1;
+          }
+        } else {
+          p0 = ex2(x0 - m_eff);
+          p1 = ex2(x1 - m_eff);
+        }
+        rsum[e & 7] += p0 + p1;
         pk[e] = pack2<T>(p0, p1);
       }
       tmem_st16(tS + 16 * c, pk);
     }
+    const float rs = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) + ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
     // O_X is idle here (its last product finished before S_X was published)
     if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
@@ -371,7 +426,7 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kCap, bool kAlibi>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -445,11 +500,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     const int X = warp >> 2;
-    softmax_group<T, D>(p, bars, tmem, X, b, h, q0, has[X], f[X], l[X]);
+    softmax_group<T, D, kCap, kAlibi>(p, bars, tmem, X, b, h, q0, has[X], f[X], l[X]);
   } else if (warp == 8) {
     if (lane == 0 && any) producer<T, D>(&tmQ, &tmK, &tmV, sQ, sKV, bars, b, h, q0, has, u0, u1);
   } else {
-    if (lane == 0 && any) mma_issuer<T, D>(sQ, sKV, bars, tmem, has, f, l, u0, u1);
+    if (lane == 0 && any) mma_issuer<T, D>(sQ, sKV, bars, tmem, has, f, l, u0, u1, p.negate_scores != 0);
   }
 
   tc_fence_before();
@@ -461,13 +516,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kCap, bool kAlibi>
 cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const FwdParams& p,
                    cudaStream_t stream) {
   using C = Cfg<D>;
   static_assert(sizeof(Barriers) <= 1024, "barrier block exceeds its reserve");
   static_assert(C::kSmemBytes <= 232448, "shared memory budget exceeded");
-  auto kernel = fwd_kernel<T, D>;
+  auto kernel = fwd_kernel<T, D, kCap, kAlibi>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.num_pairs * p.B * p.H);
@@ -475,13 +530,24 @@ cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtenso
   return cudaGetLastError();
 }
 
+template <typename T, int D>
+cudaError_t launch_mods(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const FwdParams& p,
+                        cudaStream_t stream) {
+  const bool alibi = p.slopes != nullptr;
+  if (p.use_softcap) return alibi ? launch<T, D, true, true>(tmQ, tmK, tmV, p, stream)
+                                  : launch<T, D, true, false>(tmQ, tmK, tmV, p, stream);
+  return alibi ? launch<T, D, false, true>(tmQ, tmK, tmV, p, stream)
+               : launch<T, D, false, false>(tmQ, tmK, tmV, p, stream);
+}
+
 }  // namespace
 
 cudaError_t launch_fwd(bool bf16, int d, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                        const FwdParams& p, cudaStream_t stream) {
-  if (bf16) return d == 128 ? launch<__nv_bfloat16, 128>(tmQ, tmK, tmV, p, stream)
-                            : launch<__nv_bfloat16, 64>(tmQ, tmK, tmV, p, stream);
-  return d == 128 ? launch<__half, 128>(tmQ, tmK, tmV, p, stream) : launch<__half, 64>(tmQ, tmK, tmV, p, stream);
+  if (bf16) return d == 128 ? launch_mods<__nv_bfloat16, 128>(tmQ, tmK, tmV, p, stream)
+                            : launch_mods<__nv_bfloat16, 64>(tmQ, tmK, tmV, p, stream);
+  return d == 128 ? launch_mods<__half, 128>(tmQ, tmK, tmV, p, stream)
+                  : launch_mods<__half, 64>(tmQ, tmK, tmV, p, stream);
 }
 
 }  // namespace fa

@@ -22,7 +22,8 @@ struct FwdParams {
   int causal;
   int window_left, window_right;  // -1 = unbounded
   int use_softcap;
-  float scale_log2;  // scale * log2(e)                  (no softcap)
+  int negate_scores;  // 1 when scale < 0: S = -Q K^T and the scales below use |scale|
+  float scale_log2;  // |scale| * log2(e)                (no softcap)
   float cap_scale;   // scale / softcap                   (softcap)
   float cap_log2;    // softcap * log2(e)                 (softcap)
 };

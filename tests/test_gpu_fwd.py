@@ -120,10 +120,17 @@ def test_full_size_workloads_on_sampled_rows(w):
     assert torch.isfinite(out).all().item()
 
 
+PROBE_SCALE = float(np.float32(1.0 / 1.4426950408889634))
+
+
 def boundary_probe(B, H, Nq, Nk, d, causal, wl, wr, upper, dtype=torch.bfloat16):
     """Scores 128*j (upper) or -128*j (lower) for key j: each row's softmax
     collapses onto its largest (smallest) visible key, and V encodes the key
-    index as (j // 64, j % 64), so O must equal that key's code exactly."""
+    index as (j // 64, j % 64), so O must equal that key's code exactly.
+    The scale is fp32(1 / log2 e), whose product with log2 e rounds to
+    exactly 1 in fp32, so the scores in log2 units are the exact integers
+    128*j: the top key's weight is exactly 1 and every other weight is
+    2^-128 or less, which flushes to 0."""
     assert Nk <= 16384
     sign = 1.0 if upper else -1.0
     q = torch.zeros(B, Nq, H, d)
@@ -137,7 +144,7 @@ def boundary_probe(B, H, Nq, Nk, d, causal, wl, wr, upper, dtype=torch.bfloat16)
     v[..., 0] = (j // 64)[None, :, None]
     v[..., 1] = (j % 64)[None, :, None]
     q, k, v = q.to(dtype), k.to(dtype), v.to(dtype)
-    out, lse = gpu_fwd(q, k, v, 1.0, causal, wl, wr)
+    out, lse = gpu_fwd(q, k, v, PROBE_SCALE, causal, wl, wr)
     # expected visible interval of every row, by interval arithmetic
     i = np.arange(Nq)
     pos = i + Nk - Nq
@@ -175,3 +182,17 @@ PROBES = [
 @pytest.mark.parametrize("upper", [True, False], ids=["upper", "lower"])
 def test_mask_boundaries_are_exact_on_every_row(case, upper):
     boundary_probe(*case, upper=upper)
+
+
+@pytest.mark.parametrize("scale", [-0.09, 0.0])
+@pytest.mark.parametrize("mods", [dict(), dict(alibi=True, softcap=5.0)], ids=["plain", "alibi_softcap"])
+def test_negative_and_zero_scale(scale, mods):
+    """A negative scale runs as -Q K^T on the tensor core with |scale|; a zero
+    scale makes every visible score 0 (softcap and ALiBi still apply)."""
+    B, H, Nq, Nk, d = 1, 2, 300, 500, 128
+    q, k, v = make(B, H, Nq, Nk, d, torch.bfloat16, seed=77)
+    slopes = W.alibi_slopes(H) if mods.get("alibi") else None
+    cap = mods.get("softcap", 0.0)
+    out, lse = gpu_fwd(q, k, v, scale, True, 200, -1, slopes, cap)
+    o_ref, l_ref = oracle.attn_fwd(q, k, v, scale, True, 200, -1, slopes, cap)
+    compare(out, lse, o_ref, l_ref, torch.bfloat16, "scale %g %s" % (scale, mods))
