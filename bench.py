@@ -511,33 +511,35 @@ def sweep(args):
                           "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
                           "flops": fwd_flops(w), "peak_source": peak_src, "l2": "flushed"}), flush=True)
         del x, out, lse
-    if args.workloads and W.DECODE.name not in names:
-        return
-    dw = W.DECODE
-    xd = W.make_decode_inputs(dw, device=dev)
-    KVB = decode_kv_bytes(dw, xd["cache_seqlens"].cpu())
-    d_out = torch.empty_like(xd["q"])
-    d_lse = torch.empty((dw.B, dw.H, 1), dtype=torch.float32, device=dev)
-    for s in [0, 1, 2, 4, 8, 16, 32]:
-        nb = fa.fa_kvcache_workspace_size(dw.B, dw.H, dw.d, dw.max_blocks, dw.page_size, s)
-        ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
-        run = lambda: fa.fa_fwd_kvcache(xd["q"], xd["k_cache"], xd["v_cache"], xd["block_table"],
-                                        xd["cache_seqlens"], d_out, d_lse, dw.scale, -1, None, 0.0, s, ws)
-        for _ in range(args.warmup):
-            run()
-        times = []
-        for _ in range(args.steps):
-            a, b = ev(), ev()
-            a.record()
-            run()
-            b.record()
-            times.append((a, b))
-        torch.cuda.synchronize()
-        ms = statistics.median([a.elapsed_time(b) for a, b in times])
-        gbs = KVB / (ms * 1e-3) / 1e9
-        print(json.dumps({"workload": dw.name, "num_splits": s or "auto(%d)" % fa.fa_kvcache_num_splits(
-            dw.B, dw.H, dw.d, dw.max_blocks, dw.page_size, 0), "ms": round(ms, 4), "GB/s": round(gbs, 1),
-            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "kv_bytes": KVB, "peak_source": peak_src}), flush=True)
+    for dw in W.DECODE_WORKLOADS:
+        if (args.workloads and dw.name not in names) or (not args.workloads and dw is not W.DECODE):
+            continue
+        xd = W.make_decode_inputs(dw, device=dev)
+        KVB = decode_kv_bytes(dw, xd["cache_seqlens"].cpu())
+        d_out = torch.empty_like(xd["q"])
+        d_lse = torch.empty((dw.B, dw.H, 1), dtype=torch.float32, device=dev)
+        for s in [int(x) for x in args.splits.split(",")]:
+            nb = fa.fa_kvcache_workspace_size(dw.B, dw.H, dw.d, dw.max_blocks, dw.page_size, s)
+            ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+            run = lambda: fa.fa_fwd_kvcache(xd["q"], xd["k_cache"], xd["v_cache"], xd["block_table"],
+                                            xd["cache_seqlens"], d_out, d_lse, dw.scale, -1, None, 0.0, s, ws)
+            for _ in range(args.warmup):
+                run()
+            times = []
+            for _ in range(args.steps):
+                a, b = ev(), ev()
+                a.record()
+                run()
+                b.record()
+                times.append((a, b))
+            torch.cuda.synchronize()
+            ms = statistics.median([a.elapsed_time(b) for a, b in times])
+            gbs = KVB / (ms * 1e-3) / 1e9
+            print(json.dumps({"workload": dw.name, "num_splits": s or "auto(%d)" % fa.fa_kvcache_num_splits(
+                dw.B, dw.H, dw.d, dw.max_blocks, dw.page_size, 0), "ms": round(ms, 4), "GB/s": round(gbs, 1),
+                "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "kv_bytes": KVB, "peak_source": peak_src}),
+                flush=True)
+        del xd
 
 
 def main():
@@ -551,6 +553,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--workloads", default="", help="comma-separated workload names for --sweep")
+    ap.add_argument("--splits", default="0,1,2,4,8,16,32", help="decode split counts for --sweep (0 = auto)")
     args = ap.parse_args()
     if args.warmup < 3 and not args.sweep:
         args.warmup = 3

@@ -78,6 +78,25 @@ bool make_map(CUtensorMap* map, const void* base, bool bf16, int B, int N, int H
   return r == CUDA_SUCCESS;
 }
 
+// Paged cache [num_pages, page_size, H, d] as a 4-D map (d, H, page_size,
+// num_pages) with a (d, 1, 64, 1) box and no swizzle: one box is a 64-token
+// slice of one page for one head.
+bool make_cache_map(CUtensorMap* map, const void* base, bool bf16, int num_pages, int page_size, int H, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(page_size), static_cast<cuuint64_t>(num_pages)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
+                           static_cast<cuuint64_t>(page_size) * H * d * 2};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(d), 1, 64, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool finite(float x) { return std::isfinite(x); }
 
 // Automatic split count: enough splits that a split of the longest possible
@@ -237,7 +256,15 @@ fa_status fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache
   p.scale_log2 = scale * fa::kLog2e;
   p.cap_scale = softcap > 0.0f ? scale / softcap : 0.0f;
   p.cap_log2 = softcap * fa::kLog2e;
-  return fa::launch_decode(dtype == FA_BF16, d, p, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  const bool bf16 = dtype == FA_BF16;
+  if (page_size % 64 == 0) {
+    CUtensorMap tk, tv;
+    if (!make_cache_map(&tk, k_cache, bf16, num_pages, page_size, H, d) ||
+        !make_cache_map(&tv, v_cache, bf16, num_pages, page_size, H, d))
+      return FA_ERR_CUDA;
+    return fa::launch_decode(bf16, d, p, &tk, &tv, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  }
+  return fa::launch_decode(bf16, d, p, nullptr, nullptr, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -17,7 +17,9 @@
 // groups of U*32/(d/8) tokens. Per token: page = block_table[b][t / page],
 // row = t % page; the dot product is reduced across the token's lanes with
 // shuffles; the online softmax keeps (m, l, acc) per lane group and the four
-// warps' states are merged through shared memory at the end.
+// warps' states are merged through shared memory at the end. Page sizes that
+// are a multiple of 64 take a TMA-staged variant of the split kernel (below);
+// other page sizes use the direct 16-byte-load variant.
 #include "fa_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -261,10 +263,250 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeParams p)
   if (c == 0) p.lse[row] = lse_val;
 }
 
+// Split kernel for page sizes that are a multiple of 64: a producer lane
+// streams each 64-token slice of a page (K and V, one TMA box each, no
+// multicast) into a ring of shared-memory stages; four consumer warps read
+// the rows with 16-byte shared loads. Every global byte of K and V moves in
+// whole 2*d-byte rows and the producer keeps up to kStages*32 KB in flight
+// per CTA, two CTAs per SM.
+constexpr int kRows = 64;  // tokens per stage
+
+template <int D>
+struct TmaCfg {
+  static constexpr int kStages = (D == 128) ? 3 : 6;
+  static constexpr int kTile = kRows * D * 2;  // bytes of one K (or V) stage
+  static constexpr int kSmem = 2 * kStages * kTile + 4096;
+};
+
+template <int D>
+struct TmaShared {
+  uint64_t full[TmaCfg<D>::kStages];
+  uint64_t empty[TmaCfg<D>::kStages];
+  int bad[TmaCfg<D>::kStages];
+  int abort;
+  float m[kWarps], l[kWarps];
+  float acc[kWarps][D];
+};
+
 template <typename T, int D>
-cudaError_t launch(const DecodeParams& p, cudaStream_t stream) {
+__global__ void __launch_bounds__((kWarps + 1) * 32)
+    decode_split_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                            const DecodeParams p) {
+  using C = TmaCfg<D>;
+  constexpr int NST = C::kStages;
+  constexpr int LPT = D / 8;                  // lanes per token
+  constexpr int TPW = 32 / LPT;               // tokens per warp per step
+  constexpr int kSteps = kRows / kWarps / TPW; // steps per stage per warp (16 tokens a warp)
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + NST * C::kTile;
+  TmaShared<D>* sh = reinterpret_cast<TmaShared<D>*>(smem + 2 * NST * C::kTile);
+  volatile int* abort = &sh->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x % p.H;
+  const int s = blockIdx.x / p.H;
+  const int b = blockIdx.y;
+  const int L_raw = p.cache_seqlens[b];
+  const long long max_len = static_cast<long long>(p.max_blocks) * p.page_size;
+  bool bad = L_raw < 0 || L_raw > max_len;
+  const int L = bad ? 0 : L_raw;
+  const int pos = L - 1;
+  const int lo = p.window_left >= 0 ? max(0, pos - p.window_left) : 0;
+  int t0, t1;
+  split_range(lo, L, p.num_splits, s, p.page_size, t0, t1);
+  const int a0 = (t0 / kRows) * kRows;
+  const int n_st = t1 > t0 ? (t1 - a0 + kRows - 1) / kRows : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(&sh->full[i], 1);
+      mbar_init(&sh->empty[i], kWarps);
+      sh->bad[i] = 0;
+    }
+    sh->abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kWarps) {
+    // ---------------- producer
+    if (lane == 0 && n_st > 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      const int* bt = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+      int issued = 0;
+      for (int i = 0; i < n_st; ++i) {
+        const int slot = i % NST, n = i / NST;
+        if (n > 0 && !mbar_wait(&sh->empty[slot], (n - 1) & 1, abort)) break;
+        const int a = a0 + i * kRows;
+        const int pg = bt[a / p.page_size];
+        if (pg < 0 || pg >= p.num_pages) {
+          sh->bad[slot] = 1;  // never dereferenced; consumers turn it into NaN rows
+          mbar_arrive(&sh->full[slot]);
+        } else {
+          sh->bad[slot] = 0;
+          mbar_arrive_expect_tx(&sh->full[slot], 2 * C::kTile);
+          tma_load_4d(&tmK, &sh->full[slot], sK + slot * C::kTile, 0, h, a % p.page_size, pg, pol);
+          tma_load_4d(&tmV, &sh->full[slot], sV + slot * C::kTile, 0, h, a % p.page_size, pg, pol);
+        }
+        issued = i + 1;
+      }
+      // loads in flight must land before the CTA exits
+      const int first = issued > NST ? issued - NST : 0;
+      int dummy = 0;
+      for (int i = first; i < issued; ++i) mbar_wait(&sh->full[i % NST], (i / NST) & 1, &dummy);
+    }
+  } else {
+    // ---------------- consumers
+    const int g = lane / LPT;
+    const int cl = lane % LPT;
+    float qf[8];
+    widen8<T>(*reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.q) +
+                                              (static_cast<size_t>(b) * p.H + h) * D + cl * 8),
+              qf);
+    const float qscale = p.use_softcap ? p.cap_scale : p.scale_log2;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) qf[e] *= qscale;
+    const bool alibi = p.slopes != nullptr;
+    const float slope_l2 = alibi ? p.slopes[h] * kLog2e : 0.0f;
+    float m = -INFINITY, lsum = 0.0f;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+
+    for (int i = 0; i < n_st; ++i) {
+      const int slot = i % NST;
+      bool ok = mbar_wait(&sh->full[slot], (i / NST) & 1, abort);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        bad = true;
+        break;
+      }
+      if (sh->bad[slot]) {
+        bad = true;
+      } else {
+        const T* kt = reinterpret_cast<const T*>(sK + slot * C::kTile);
+        const T* vt = reinterpret_cast<const T*>(sV + slot * C::kTile);
+        const int a = a0 + i * kRows;
+        float sc[kSteps];
+        float mt = -INFINITY;
+#pragma unroll
+        for (int st = 0; st < kSteps; ++st) {
+          const int r = warp * (kRows / kWarps) + st * TPW + g;
+          float kf[8];
+          widen8<T>(*reinterpret_cast<const uint4*>(kt + r * D + cl * 8), kf);
+          float dot = 0.0f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dot = fmaf(qf[e], kf[e], dot);
+#pragma unroll
+          for (int o = LPT / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+          const int tok = a + r;
+          float t = p.use_softcap ? p.cap_log2 * tanh_via_exp2(dot) : dot;
+          if (alibi) t -= slope_l2 * static_cast<float>(pos - tok);
+          sc[st] = (tok >= t0 && tok < t1) ? t : -INFINITY;
+          mt = fmaxf(mt, sc[st]);
+        }
+        const float m_new = fmaxf(m, mt);
+        if (m_new != -INFINITY) {
+          const float alpha = ex2(m - m_new);
+          lsum *= alpha;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] *= alpha;
+#pragma unroll
+          for (int st = 0; st < kSteps; ++st) {
+            const int r = warp * (kRows / kWarps) + st * TPW + g;
+            const float pu = ex2(sc[st] - m_new);
+            lsum += pu;
+            float vf[8];
+            widen8<T>(*reinterpret_cast<const uint4*>(vt + r * D + cl * 8), vf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = fmaf(pu, vf[e], acc[e]);
+          }
+          m = m_new;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->empty[slot]);
+    }
+    // merge the lane groups of this warp, then publish the warp's state
+#pragma unroll
+    for (int o = LPT; o < 32; o <<= 1) {
+      const float m_o = __shfl_xor_sync(0xffffffffu, m, o);
+      const float l_o = __shfl_xor_sync(0xffffffffu, lsum, o);
+      const float mm = fmaxf(m, m_o);
+      const float x = (m == -INFINITY) ? 0.0f : ex2(m - mm);
+      const float x_o = (m_o == -INFINITY) ? 0.0f : ex2(m_o - mm);
+      lsum = lsum * x + l_o * x_o;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float a_o = __shfl_xor_sync(0xffffffffu, acc[e], o);
+        acc[e] = acc[e] * x + a_o * x_o;
+      }
+      m = mm;
+    }
+    if (lane < LPT) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sh->acc[warp][cl * 8 + e] = acc[e];
+    }
+    if (lane == 0) {
+      sh->m[warp] = m;
+      sh->l[warp] = lsum;
+    }
+  }
+  const bool any_bad = __syncthreads_or(bad) != 0;
+
+  const int c = threadIdx.x;
+  if (c >= D) return;
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sh->m[w]);
+  float ltot = 0.0f, oc = 0.0f;
+  if (M != -INFINITY) {
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float x = (sh->m[w] == -INFINITY) ? 0.0f : ex2(sh->m[w] - M);
+      ltot += sh->l[w] * x;
+      oc += sh->acc[w][c] * x;
+    }
+  }
+  const float nan = __int_as_float(0x7fc00000);
+  float o_val, lse_val;
+  if (any_bad) {
+    o_val = nan;
+    lse_val = nan;
+  } else if (ltot > 0.0f) {
+    o_val = oc / ltot;
+    lse_val = (M + lg2(ltot)) * kLn2;
+  } else {
+    o_val = 0.0f;
+    lse_val = -INFINITY;
+  }
+  const size_t row = static_cast<size_t>(b) * p.H + h;
+  if (p.num_splits == 1) {
+    T* out = reinterpret_cast<T*>(p.out) + row * D;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) out[c] = __float2bfloat16_rn(o_val);
+    else out[c] = __float2half_rn(o_val);
+    if (c == 0) p.lse[row] = lse_val;
+  } else {
+    const size_t prow = static_cast<size_t>(s) * p.B * p.H + row;
+    p.o_part[prow * D + c] = o_val;
+    if (c == 0) p.lse_part[prow] = lse_val;
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch(const DecodeParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV, cudaStream_t stream) {
   dim3 grid(p.H * p.num_splits, p.B);
-  decode_split_kernel<T, D><<<grid, kWarps * 32, 0, stream>>>(p);
+  if (tmK != nullptr) {
+    using C = TmaCfg<D>;
+    static_assert(sizeof(TmaShared<D>) <= 4096, "decode shared block exceeds its reserve");
+    auto kernel = decode_split_tma_kernel<T, D>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    kernel<<<grid, (kWarps + 1) * 32, C::kSmem, stream>>>(*tmK, *tmV, p);
+  } else {
+    decode_split_kernel<T, D><<<grid, kWarps * 32, 0, stream>>>(p);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || p.num_splits == 1) return e;
   decode_combine_kernel<T, D><<<p.B * p.H, D, 0, stream>>>(p);
@@ -273,9 +515,11 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t stream) {
 
 }  // namespace
 
-cudaError_t launch_decode(bool bf16, int d, const DecodeParams& p, cudaStream_t stream) {
-  if (bf16) return d == 128 ? launch<__nv_bfloat16, 128>(p, stream) : launch<__nv_bfloat16, 64>(p, stream);
-  return d == 128 ? launch<__half, 128>(p, stream) : launch<__half, 64>(p, stream);
+cudaError_t launch_decode(bool bf16, int d, const DecodeParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                          cudaStream_t stream) {
+  if (bf16) return d == 128 ? launch<__nv_bfloat16, 128>(p, tmK, tmV, stream)
+                            : launch<__nv_bfloat16, 64>(p, tmK, tmV, stream);
+  return d == 128 ? launch<__half, 128>(p, tmK, tmV, stream) : launch<__half, 64>(p, tmK, tmV, stream);
 }
 
 }  // namespace fa

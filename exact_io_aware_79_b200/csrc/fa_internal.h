@@ -51,6 +51,10 @@ struct DecodeParams {
 cudaError_t launch_fwd(bool bf16, int d, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                        const FwdParams& p, cudaStream_t stream);
 
-cudaError_t launch_decode(bool bf16, int d, const DecodeParams& p, cudaStream_t stream);
+// tmK/tmV: 4-D maps (d, H, page_size, num_pages) of the caches with a
+// (d, 1, 64, 1) box for the TMA-staged split kernel (page_size % 64 == 0), or
+// nullptr for the direct-load split kernel.
+cudaError_t launch_decode(bool bf16, int d, const DecodeParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                          cudaStream_t stream);
 
 }  // namespace fa

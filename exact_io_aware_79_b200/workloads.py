@@ -97,7 +97,13 @@ ALIBI_SOFTCAP = FwdWorkload("alibi_softcap50_bf16_b4h32n4096d128", 4, 32, 4096, 
 DECODE = DecodeWorkload("paged_decode_bf16_b64h32d128_page256", 64, 32, 128, torch.bfloat16,
                         page_size=256, len_lo=1024, len_hi=32768, seed=4)
 
+# The decode workload with 4 sequences instead of 64 (same lengths law, pool of
+# 512 pages = 2.1 GB of K/V): small enough for detailed profiler captures.
+DECODE_SMALL = DecodeWorkload("paged_decode_bf16_b4h32d128_page256", 4, 32, 128, torch.bfloat16,
+                              page_size=256, len_lo=1024, len_hi=32768, seed=4)
+
 FWD_WORKLOADS = [TINY, CAUSAL_2K, WINDOW_16K, WINDOW_Q4K_K16K, CAUSAL_Q4K_K16K, ALIBI_SOFTCAP]
+DECODE_WORKLOADS = [DECODE, DECODE_SMALL]
 
 
 def alibi_slopes(H: int) -> torch.Tensor:

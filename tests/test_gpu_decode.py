@@ -55,6 +55,8 @@ CASES = [
     (2, 2, 128, 256, 8, (2048, 777), torch.bfloat16, 300, False, 0.0, 1.0),
     (3, 2, 64, 32, 10, (320, 33, 17), torch.bfloat16, 40, True, 0.0, 1.0),
     (2, 2, 128, 256, 16, (4096, 3000), torch.float16, -1, False, 5.0, 1.5),
+    (2, 3, 64, 64, 12, (700, 65), torch.bfloat16, -1, False, 0.0, 1.0),
+    (3, 2, 128, 128, 6, (500, 129, 768), torch.float16, 100, True, 0.0, 1.0),
 ]
 
 
