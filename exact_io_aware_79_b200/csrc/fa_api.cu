@@ -153,8 +153,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
   if (!q || !out || !lse) return FA_ERR_NULL;
   if (Nk > 0 && (!k || !v)) return FA_ERR_NULL;
   if (!aligned16(q) || !aligned16(out) || !aligned16(k) || !aligned16(v) || !aligned16(lse)) return FA_ERR_ARG;
-  const int pairs = (Nq + 255) / 256;
-  if (static_cast<long long>(pairs) * B * H >= (1LL << 31)) return FA_ERR_SHAPE;
+  const int tiles = (Nq + 127) / 128;
+  if (static_cast<long long>(tiles) * B * H >= (1LL << 31)) return FA_ERR_SHAPE;
   fa_status st = check_device();
   if (st != FA_OK) return st;
 
@@ -175,7 +175,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
   p.H = H;
   p.Nq = Nq;
   p.Nk = Nk;
-  p.num_pairs = pairs;
+  p.num_tiles = tiles;
   p.causal = causal;
   p.window_left = window_left;
   p.window_right = window_right;

@@ -8,30 +8,31 @@
 // running row max m and row sum l and rescales the partial output, so the
 // N x N scores never leave the SM.
 //
-// B200 mapping. One CTA owns two adjacent Q tiles (A and B) of one (batch,
-// head) and runs ten warps:
-//   warps 0-3  softmax for tile A, one query row per thread (row = TMEM lane)
-//   warps 4-7  softmax for tile B
-//   warp  8    TMA producer: Q tiles once, then K_j, V_j into a ring of
+// B200 mapping. One CTA owns one 128-row Q tile of one (batch, head) and
+// runs six warps:
+//   warps 0-3  softmax, one query row per thread (row = TMEM lane)
+//   warp  4    TMA producer: the Q tile once, then K_j, V_j into a ring of
 //              shared-memory slots (128-byte swizzle), mbarrier expect-tx
-//   warp  9    TMEM owner and MMA issuer (one elected thread)
+//   warp  5    TMEM owner and MMA issuer (one elected thread)
 // Tensor memory (512 columns x 128 lanes x 32 bit):
-//   cols   0..127  S_A (fp32 scores), later P_A (16-bit, first 64 columns)
-//   cols 128..255  O_A (fp32, d columns)
-//   cols 256..383  S_B / P_B
-//   cols 384..511  O_B
-// Per K/V tile j the MMA thread issues, in order,
-//   O_A += P_A(j) V_j,  S_A(j+1) = Q_A K_{j+1}^T,  O_B += P_B(j) V_j,
-//   S_B(j+1) = Q_B K_{j+1}^T,
-// so while one softmax group works on its tile the tensor core runs the
-// other group's two products (ping-pong). tcgen05 operations of one thread
-// complete in issue order, so the arrival that publishes S_X(j+1) also proves
-// that O_X += P_X(j) V_j has finished; the softmax group may then rescale O_X
-// in place before it publishes P_X(j+1).
+//   cols   0..127  S buffer 0 (fp32 scores; P, 16-bit, overwrites its first
+//                  64 columns and feeds the PV product straight from TMEM)
+//   cols 128..255  S buffer 1
+//   cols 256..383  O (fp32, d columns)
+// The scores are double-buffered: for K/V tile j the MMA thread issues
+//   S(j+1) = Q K_{j+1}^T into the other buffer, then (once P(j) is ready)
+//   O += P(j) V_j,
+// so the tensor core computes the next tile's scores while the softmax
+// warps work on this one, and the step time is max(softmax, tensor core)
+// rather than their sum. The softmax warps are alone on the SM's four
+// sub-partitions, so each has a whole MUFU (exp2) unit. tcgen05 operations
+// of one thread complete in issue order, so the product that reads P(j)
+// finishes before S(j+2) overwrites the same columns.
 //
-// Rescaling is lazy: a row keeps its old max unless the new tile raises it by
+// Rescaling is lazy: a row keeps its old max unless a new tile raises it by
 // more than 8 (log2 units), so P stays <= 2^8 and O is rescaled only when it
-// must be. The result is the same softmax (m cancels in O / l).
+// must be (after waiting for the previous PV product). The result is the
+// same softmax (m cancels in O / l).
 #include "fa_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -44,26 +45,30 @@ namespace {
 
 constexpr int BM = 128;  // query rows per Q tile
 constexpr int BN = 128;  // keys per K/V tile
-constexpr int kThreads = 320;
-constexpr int kMaxSlots = 8;
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kMaxSlots = 12;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 256;
 
 template <int D>
 struct Cfg {
-  static constexpr int kChunkBytes = BM * 128;         // 128 rows x 64 elements x 2 bytes
-  static constexpr int kTileBytes = BM * D * 2;        // one Q, K or V tile
-  static constexpr int kSlots = (D == 128) ? 5 : 8;    // K/V ring depth
-  static constexpr int kSmemBytes = 1024 + (2 + kSlots) * kTileBytes + 1024;
+  static constexpr int kChunkBytes = BM * 128;       // 128 rows x 64 elements x 2 bytes
+  static constexpr int kTileBytes = BM * D * 2;      // one Q, K or V tile
+  static constexpr int kSlots = (D == 128) ? 6 : 12; // K/V ring depth
+  static constexpr int kSmemBytes = 1024 + (1 + kSlots) * kTileBytes + 1024;
 };
 
 struct Barriers {
   uint64_t q_full;
   uint64_t slot_full[kMaxSlots];
   uint64_t slot_empty[kMaxSlots];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_final[2];
+  uint64_t s_full[2];  // per S buffer
+  uint64_t p_full[2];  // per S buffer
+  uint64_t pv_done;
+  uint64_t o_final;
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
@@ -94,24 +99,20 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 
 template <typename T, int D>
 __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV, uint8_t* sQ,
-                         uint8_t* sKV, Barriers* bars, int b, int h, int q0, const bool (&has)[2], int u0, int u1) {
+                         uint8_t* sKV, Barriers* bars, int b, int h, int q0, int f, int l) {
   using C = Cfg<D>;
   volatile int* abort = &bars->abort;
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
-  const uint32_t qbytes = (has[0] ? C::kTileBytes : 0) + (has[1] ? C::kTileBytes : 0);
-  mbar_arrive_expect_tx(&bars->q_full, qbytes);
+  mbar_arrive_expect_tx(&bars->q_full, C::kTileBytes);
 #pragma unroll
-  for (int X = 0; X < 2; ++X) {
-    if (!has[X]) continue;
-#pragma unroll
-    for (int ch = 0; ch < D / 64; ++ch)
-      tma_load_4d(tmQ, &bars->q_full, sQ + X * C::kTileBytes + ch * C::kChunkBytes, ch * 64, h, q0 + X * BM, b,
-                  pol_q);
-  }
+  for (int ch = 0; ch < D / 64; ++ch)
+    tma_load_4d(tmQ, &bars->q_full, sQ + ch * C::kChunkBytes, ch * 64, h, q0, b, pol_q);
+  // load order K(f), V(f), K(f+1), V(f+1), ... (the MMA thread acquires
+  // V(j) then K(j+1) in each step, which is the same sequence)
   uint32_t it = 0;
   bool ok = true;
-  for (int j = u0; j <= u1 && ok; ++j) {
+  for (int j = f; j <= l && ok; ++j) {
 #pragma unroll
     for (int kv = 0; kv < 2; ++kv) {
       const uint32_t slot = it % C::kSlots, n = it / C::kSlots;
@@ -136,8 +137,7 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const C
 }
 
 template <typename T, int D>
-__device__ void mma_issuer(uint8_t* sQ, uint8_t* sKV, Barriers* bars, uint32_t tmem, const bool (&has)[2],
-                           const int (&f)[2], const int (&l)[2], int u0, int u1, bool negate) {
+__device__ void mma_issuer(uint8_t* sQ, uint8_t* sKV, Barriers* bars, uint32_t tmem, int f, int l, bool negate) {
   using C = Cfg<D>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   // a negative softmax scale is applied as -Q K^T (A-negate bit) times |scale|
@@ -147,7 +147,6 @@ __device__ void mma_issuer(uint8_t* sQ, uint8_t* sKV, Barriers* bars, uint32_t t
   const uint32_t sQaddr = smem_addr(sQ);
   const uint32_t sKVaddr = smem_addr(sKV);
 
-  auto in = [&](int X, int j) { return has[X] && j >= f[X] && j <= l[X]; };
   uint32_t it = 0;
   auto acquire = [&](uint32_t& addr, uint32_t& slot) -> bool {
     slot = it % C::kSlots;
@@ -156,76 +155,52 @@ __device__ void mma_issuer(uint8_t* sQ, uint8_t* sKV, Barriers* bars, uint32_t t
     ++it;
     return ok;
   };
-  // S_X = Q_X K^T: M = 128 query rows, N = 128 keys, K = d in steps of 16.
-  // Both operands are K-major, 128-byte swizzled, 64 elements per 16 KB chunk.
-  auto qk = [&](int X, uint32_t kaddr) {
-    const uint32_t qaddr = sQaddr + X * C::kTileBytes;
-    const uint32_t d_t = tmem + X * 256;
+  // S(j) = Q K_j^T into S buffer (j - f) & 1: M = 128 query rows, N = 128
+  // keys, K = d in steps of 16. Both operands are K-major, 128-byte
+  // swizzled, 64 elements per 16 KB chunk.
+  auto qk = [&](int j, uint32_t kaddr) {
+    const uint32_t d_t = tmem + ((j - f) & 1) * 128;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t off = (kk / 4) * C::kChunkBytes + (kk % 4) * 32;
-      mma_ss(d_t, smem_desc_sw128(qaddr + off, 16, 1024), smem_desc_sw128(kaddr + off, 16, 1024), idesc_qk,
+      mma_ss(d_t, smem_desc_sw128(sQaddr + off, 16, 1024), smem_desc_sw128(kaddr + off, 16, 1024), idesc_qk,
              kk > 0 ? 1u : 0u);
     }
+    tc_commit(&bars->s_full[(j - f) & 1]);
   };
-  // O_X (+)= P_X V: A = P from TMEM (16-bit, two keys per column), B = V tile
-  // stored keys x d with d contiguous (MN-major): 16 keys = 2048 bytes,
+  // O (+)= P(j) V_j: A = P from TMEM (16-bit, two keys per column), B = V
+  // tile stored keys x d with d contiguous (MN-major): 16 keys = 2048 bytes,
   // the second 64-wide d chunk lies 16 KB further (leading byte offset).
-  auto pv = [&](int X, uint32_t vaddr, bool accumulate) {
-    const uint32_t a_t = tmem + X * 256;
-    const uint32_t d_t = tmem + X * 256 + 128;
+  auto pv = [&](int j, uint32_t vaddr) {
+    const uint32_t a_t = tmem + ((j - f) & 1) * 128;
 #pragma unroll
     for (int kk = 0; kk < BN / 16; ++kk)
-      mma_ts(d_t, a_t + kk * 8, smem_desc_sw128(vaddr + kk * 2048, C::kChunkBytes, 1024), idesc_pv,
-             (accumulate || kk > 0) ? 1u : 0u);
+      mma_ts(tmem + kTmemO, a_t + kk * 8, smem_desc_sw128(vaddr + kk * 2048, C::kChunkBytes, 1024), idesc_pv,
+             (j > f || kk > 0) ? 1u : 0u);
+    tc_commit(&bars->pv_done);
+    if (j == l) tc_commit(&bars->o_final);
   };
 
-  uint32_t pcount[2] = {0, 0};
   bool ok = mbar_wait(&bars->q_full, 0, abort);
   uint32_t aK = 0, slotK = 0, aV = 0, slotV = 0;
-  if (ok) ok = acquire(aK, slotK);
-  if (ok) {
-    tc_fence_after();
-    if (in(0, u0)) {
-      qk(0, aK);
-      tc_commit(&bars->s_full[0]);
-    }
-    if (in(1, u0)) {
-      qk(1, aK);
-      tc_commit(&bars->s_full[1]);
-    }
+  if (ok && (ok = acquire(aK, slotK))) {
+    qk(f, aK);
     tc_commit(&bars->slot_empty[slotK]);
   }
-  for (int j = u0; j <= u1 && ok; ++j) {
+  for (int j = f; j <= l && ok; ++j) {
+    const bool next = j < l;
     if (!(ok = acquire(aV, slotV))) break;
-    if (in(0, j)) {
-      if (!(ok = mbar_wait(&bars->p_full[0], pcount[0]++ & 1, abort))) break;
-      tc_fence_after();
-      pv(0, aV, j > f[0]);
-      if (j == l[0]) tc_commit(&bars->o_final[0]);
-    }
-    const bool next = j < u1;
     if (next) {
+      // the next tile's scores go into the other S buffer; its previous
+      // contents (P(j-1)) were consumed by the PV product issued last step
       if (!(ok = acquire(aK, slotK))) break;
-      if (in(0, j + 1)) {
-        qk(0, aK);
-        tc_commit(&bars->s_full[0]);
-      }
-    }
-    if (in(1, j)) {
-      if (!(ok = mbar_wait(&bars->p_full[1], pcount[1]++ & 1, abort))) break;
-      tc_fence_after();
-      pv(1, aV, j > f[1]);
-      if (j == l[1]) tc_commit(&bars->o_final[1]);
-    }
-    tc_commit(&bars->slot_empty[slotV]);
-    if (next) {
-      if (in(1, j + 1)) {
-        qk(1, aK);
-        tc_commit(&bars->s_full[1]);
-      }
+      qk(j + 1, aK);
       tc_commit(&bars->slot_empty[slotK]);
     }
+    if (!(ok = mbar_wait(&bars->p_full[(j - f) & 1], ((j - f) >> 1) & 1, abort))) break;
+    tc_fence_after();
+    pv(j, aV);
+    tc_commit(&bars->slot_empty[slotV]);
   }
   // All MMAs of this thread must be complete before TMEM is released.
   tc_commit(&bars->mma_done);
@@ -240,30 +215,28 @@ __device__ __forceinline__ float mod_score(const FwdParams& p, float x, float sl
   return t;
 }
 
-// One softmax warpgroup (tile X): one query row per thread, row == TMEM lane.
+// The softmax warpgroup: one query row per thread, row == TMEM lane.
 // kCap / kAlibi select the score modifiers at compile time; whether a K tile
 // needs the element mask is decided per tile for the whole group, so the
 // common interior tiles run without per-element compares.
 template <typename T, int D, bool kCap, bool kAlibi>
-__device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem, int X, int b, int h, int q0,
-                              bool has, int f, int l) {
+__device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem, int b, int h, int q0, bool has,
+                              int f, int l) {
   constexpr bool kPlain = !kCap && !kAlibi;
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int r = (warp & 3) * 32 + lane;  // row of the tile == TMEM lane
-  const int q = q0 + X * BM + r;
+  const int r = warp * 32 + lane;  // row of the tile == TMEM lane
+  const int q = q0 + r;
   const bool row_ok = q < p.Nq;
   const RowRange rr = row_range(p, row_ok ? q : p.Nq - 1);
-  // tile-level bounds: a K tile needs no mask when every row of the group
+  // tile-level bounds: a K tile needs no mask when every row of the tile
   // sees all of it (rows' intervals are monotone in q)
-  const int qa = q0 + X * BM;
-  const int qz = min(qa + BM - 1, p.Nq - 1);
-  const RowRange first_row = row_range(p, qa), last_row = row_range(p, qz);
+  const int qz = min(q0 + BM - 1, p.Nq - 1);
+  const RowRange first_row = row_range(p, q0), last_row = row_range(p, qz);
   const int pos = q + p.Nk - p.Nq;
-  const uint32_t lane_sel = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const uint32_t tS = tmem + lane_sel + X * 256;
-  const uint32_t tO = tS + 128;
+  const uint32_t lane_sel = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t tO = tmem + lane_sel + kTmemO;
   const float slope_l2 = kAlibi ? p.slopes[h] * kLog2e : 0.0f;
   const float sl2 = p.scale_log2;  // >= 0 (a negative scale is folded into the MMA)
 
@@ -273,13 +246,14 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
   const int n = has ? l - f + 1 : 0;
   for (int it = 0; it < n; ++it) {
     const int j = f + it;
-    ok = mbar_wait(&bars->s_full[X], it & 1, abort);
+    const uint32_t tS = tmem + lane_sel + (it & 1) * 128;
+    ok = mbar_wait(&bars->s_full[it & 1], (it >> 1) & 1, abort);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
     tc_fence_after();
     uint32_t s[4][32];
     const int key0 = j * BN;
-    const bool masked = key0 < last_row.lo || key0 + BN - 1 > first_row.hi;  // uniform over the group
+    const bool masked = key0 < last_row.lo || key0 + BN - 1 > first_row.hi;  // uniform over the tile
     // pass 1: transform (modifier paths) and tile max. S arrives in two
     // halves so the second TMEM load overlaps the first half's work; four
     // independent 3-input max chains keep the pipes busy.
@@ -336,8 +310,12 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
     }
     lsum *= alpha;
     const float m_eff = (m == -INFINITY) ? 0.0f : m;
-    // pass 2: P = exp2(t - m) into the first 64 columns of S (frees the score registers)
-    float rsum[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};  // independent partial sums
+    // pass 2: P = exp2(t - m) into the first 64 columns of this S buffer.
+    // Pairs of elements go through packed fp32x2 instructions: one FMA
+    // (scale and subtract the max) and one add (row sum) per pair.
+    const uint64_t m2 = f2_pack(-m_eff, -m_eff);
+    const uint64_t mul2 = kPlain ? f2_pack(sl2, sl2) : f2_pack(1.0f, 1.0f);
+    uint64_t rsum2[4] = {0, 0, 0, 0};  // independent packed partial sums (0 bits = +0.0f)
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       uint32_t pk[16];
@@ -345,27 +323,32 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
       for (int e = 0; e < 16; ++e) {
         const float x0 = __uint_as_float(s[c][2 * e]);
         const float x1 = __uint_as_float(s[c][2 * e + 1]);
-        float p0, p1;
-        if (kPlain) {
+        float a0, a1;
+        f2_unpack(f2_fma(f2_pack(x0, x1), mul2, m2), a0, a1);
+        float p0 = ex2(a0), p1 = ex2(a1);
+        if (kPlain && masked) {
           // masked entries hold -inf; -inf * 0 would be NaN, so select them out
-          p0 = ex2(fmaf(x0, sl2, -m_eff));
-          p1 = ex2(fmaf(x1, sl2, -m_eff));
-          if (masked) {
-            p0 = (x0 == -INFINITY) ? 0.0f : p0;
-            p1 = (x1 == -INFINITY) ? 0.0f : p1;
-          }
-        } else {
-          p0 = ex2(x0 - m_eff);
-          p1 = ex2(x1 - m_eff);
+          p0 = (x0 == -INFINITY) ? 0.0f : p0;
+          p1 = (x1 == -INFINITY) ? 0.0f : p1;
         }
-        rsum[e & 7] += p0 + p1;
+        rsum2[e & 3] = f2_add(rsum2[e & 3], f2_pack(p0, p1));
         pk[e] = pack2<T>(p0, p1);
       }
       tmem_st16(tS + 16 * c, pk);
     }
-    const float rs = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) + ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
-    // O_X is idle here (its last product finished before S_X was published)
+    float r0, r1, r2, r3;
+    f2_unpack(f2_add(rsum2[0], rsum2[1]), r0, r1);
+    f2_unpack(f2_add(rsum2[2], rsum2[3]), r2, r3);
+    const float rs = (r0 + r1) + (r2 + r3);
     if (__any_sync(0xffffffffu, rescale)) {
+      // O must be idle: wait for the product of the previous tile (the only
+      // one that can still be running).
+      if (it > 0) {
+        ok = mbar_wait(&bars->pv_done, (it - 1) & 1, abort);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+      }
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -381,10 +364,10 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&bars->p_full[X]);
+    if (lane == 0) mbar_arrive(&bars->p_full[it & 1]);
   }
   if (ok && n > 0) {
-    ok = mbar_wait(&bars->o_final[X], 0, abort);
+    ok = mbar_wait(&bars->o_final, 0, abort);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
   }
@@ -434,40 +417,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sKV = smem + 2 * C::kTileBytes;
+  uint8_t* sKV = smem + C::kTileBytes;
   Barriers* bars = reinterpret_cast<Barriers*>(sKV + C::kSlots * C::kTileBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // 1-D grid, the pairs of one (b, h) adjacent so they share K/V in L2;
+  // 1-D grid, the Q tiles of one (b, h) adjacent so they share K/V in L2;
   // within a head the longest causal work is dispatched first.
-  const int bh = static_cast<int>(blockIdx.x) / p.num_pairs;
-  const int pair = p.num_pairs - 1 - static_cast<int>(blockIdx.x) % p.num_pairs;
+  const int bh = static_cast<int>(blockIdx.x) / p.num_tiles;
+  const int tile = p.num_tiles - 1 - static_cast<int>(blockIdx.x) % p.num_tiles;
   const int b = bh / p.H, h = bh % p.H;
-  const int q0 = pair * 2 * BM;
+  const int q0 = tile * BM;
 
-  // K/V tile range of each Q tile (rows' visible intervals are monotone in q)
-  bool has[2];
-  int f[2], l[2];
-#pragma unroll
-  for (int X = 0; X < 2; ++X) {
-    const int r0 = q0 + X * BM;
-    has[X] = false;
-    f[X] = 0;
-    l[X] = -1;
-    if (r0 < p.Nq) {
-      const int r1 = min(r0 + BM - 1, p.Nq - 1);
-      const RowRange a = row_range(p, r0), z = row_range(p, r1);
-      if (a.lo <= z.hi) {
-        has[X] = true;
-        f[X] = a.lo / BN;
-        l[X] = z.hi / BN;
-      }
-    }
-  }
-  const bool any = has[0] || has[1];
-  const int u0 = has[0] ? f[0] : f[1];
-  const int u1 = has[1] ? l[1] : l[0];
+  // K/V tile range of the Q tile (rows' visible intervals are monotone in q)
+  const int qz = min(q0 + BM - 1, p.Nq - 1);
+  const RowRange ra = row_range(p, q0), rz = row_range(p, qz);
+  const bool has = ra.lo <= rz.hi;
+  const int f = has ? ra.lo / BN : 0;
+  const int l = has ? rz.hi / BN : -1;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -475,20 +442,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->slot_full[i], 1);
       mbar_init(&bars->slot_empty[i], 1);
     }
-    for (int X = 0; X < 2; ++X) {
-      mbar_init(&bars->s_full[X], 1);
-      mbar_init(&bars->p_full[X], 4);
-      mbar_init(&bars->o_final[X], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 4);
     }
+    mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->o_final, 1);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -498,18 +466,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp < 8) {
-    const int X = warp >> 2;
-    softmax_group<T, D, kCap, kAlibi>(p, bars, tmem, X, b, h, q0, has[X], f[X], l[X]);
-  } else if (warp == 8) {
-    if (lane == 0 && any) producer<T, D>(&tmQ, &tmK, &tmV, sQ, sKV, bars, b, h, q0, has, u0, u1);
+  if (warp < 4) {
+    softmax_group<T, D, kCap, kAlibi>(p, bars, tmem, b, h, q0, has, f, l);
+  } else if (warp == kProducerWarp) {
+    if (lane == 0 && has) producer<T, D>(&tmQ, &tmK, &tmV, sQ, sKV, bars, b, h, q0, f, l);
   } else {
-    if (lane == 0 && any) mma_issuer<T, D>(sQ, sKV, bars, tmem, has, f, l, u0, u1, p.negate_scores != 0);
+    if (lane == 0 && has) mma_issuer<T, D>(sQ, sKV, bars, tmem, f, l, p.negate_scores != 0);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -522,10 +489,11 @@ cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtenso
   using C = Cfg<D>;
   static_assert(sizeof(Barriers) <= 1024, "barrier block exceeds its reserve");
   static_assert(C::kSmemBytes <= 232448, "shared memory budget exceeded");
+  static_assert(C::kSlots <= kMaxSlots, "too many K/V slots");
   auto kernel = fwd_kernel<T, D, kCap, kAlibi>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.num_pairs * p.B * p.H);
+  dim3 grid(p.num_tiles * p.B * p.H);
   kernel<<<grid, kThreads, C::kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
@@ -551,3 +519,4 @@ cudaError_t launch_fwd(bool bf16, int d, const CUtensorMap& tmQ, const CUtensorM
 }
 
 }  // namespace fa
+

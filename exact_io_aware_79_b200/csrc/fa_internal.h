@@ -12,13 +12,13 @@ namespace fa {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// Forward: one CTA owns two adjacent 128-row query tiles of one (b, h).
+// Forward: one CTA owns one 128-row query tile of one (b, h).
 struct FwdParams {
   void* out;            // [B, Nq, H, d]
   float* lse;           // [B, H, Nq]
   const float* slopes;  // [H] or nullptr
   int B, H, Nq, Nk;
-  int num_pairs;        // ceil(Nq / 256)
+  int num_tiles;        // ceil(Nq / 128)
   int causal;
   int window_left, window_right;  // -1 = unbounded
   int use_softcap;

@@ -126,7 +126,9 @@ PROBE_SCALE = float(np.float32(1.0 / 1.4426950408889634))
 def boundary_probe(B, H, Nq, Nk, d, causal, wl, wr, upper, dtype=torch.bfloat16):
     """Scores 128*j (upper) or -128*j (lower) for key j: each row's softmax
     collapses onto its largest (smallest) visible key, and V encodes the key
-    index as (j // 64, j % 64), so O must equal that key's code exactly.
+    index as (j // 64 + 1, j % 64 + 1), so O must equal that key's code
+    exactly (the codes start at 1 so an empty row's O = 0 cannot pass for a
+    key, and weights far below 2^-126 cannot disturb them).
     The scale is fp32(1 / log2 e), whose product with log2 e rounds to
     exactly 1 in fp32, so the scores in log2 units are the exact integers
     128*j: the top key's weight is exactly 1 and every other weight is
@@ -141,8 +143,8 @@ def boundary_probe(B, H, Nq, Nk, d, causal, wl, wr, upper, dtype=torch.bfloat16)
     k[..., 0] = (j // 64)[None, :, None]
     k[..., 1] = (j % 64)[None, :, None]
     v = torch.zeros(B, Nk, H, d)
-    v[..., 0] = (j // 64)[None, :, None]
-    v[..., 1] = (j % 64)[None, :, None]
+    v[..., 0] = (j // 64 + 1)[None, :, None]
+    v[..., 1] = (j % 64 + 1)[None, :, None]
     q, k, v = q.to(dtype), k.to(dtype), v.to(dtype)
     out, lse = gpu_fwd(q, k, v, PROBE_SCALE, causal, wl, wr)
     # expected visible interval of every row, by interval arithmetic
@@ -156,8 +158,8 @@ def boundary_probe(B, H, Nq, Nk, d, causal, wl, wr, upper, dtype=torch.bfloat16)
         hi = np.minimum(hi, pos + wr)
     empty = lo > hi
     target = hi if upper else lo
-    want0 = np.where(empty, 0, target // 64)
-    want1 = np.where(empty, 0, target % 64)
+    want0 = np.where(empty, 0, target // 64 + 1)
+    want1 = np.where(empty, 0, target % 64 + 1)
     got0 = out[:, :, :, 0]
     got1 = out[:, :, :, 1]
     assert np.array_equal(got0, np.broadcast_to(want0[None, :, None], got0.shape))
