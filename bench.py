@@ -43,6 +43,16 @@ from exact_io_aware_79_b200 import workloads as W  # noqa: E402
 METRIC = "attn fwd TFLOP/s (% of BF16 peak); paged-decode KV GB/s (% of HBM BW)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# ncu captures of the kernels as they stand; each entry names its capture.
+# Decode: a capture of the 4-sequence case read 1.003 x its K/V bytes and
+# wrote 2.8 MB of partials (profiles/decode_split_tma_paged_decode_b4h32d128_page256.md);
+# reads scale with the K/V bytes, each byte being read once.
+DECODE_READ_PER_KV_BYTE = 967926912.0 / 965165056.0
+# Forward, causal B8 H16 N2048 d128: mean of two captured launches
+# (profiles/fwd_kernel_window_b1h16n16384d128_wl4096.md, second table).
+FWD_CAUSAL_2K_TRAFFIC = (201403648 + 45780480 + 201389824 + 42561536) / 2.0
+
 
 # ---------------------------------------------------------------- algorithmic work
 
@@ -401,11 +411,15 @@ def gpu_arm(args):
         },
         "roofline": {"kernel": "decode (split + merge)", "bound": "hbm", "achieved": round(dec_gbs / world, 1),
                      "peak": peak_h, "unit": "GB/s", "frac": round(dec_gbs / world / peak_h, 4),
-                     "traffic": None, "peak_source": peak_src},
+                     "traffic": round(DECODE_READ_PER_KV_BYTE * KVB),
+                     "traffic_source": "ncu capture of the 4-sequence case, scaled by K/V bytes",
+                     "peak_source": peak_src},
         "roofline_fwd": {"kernel": "fwd_kernel", "bound": "tensor", "achieved": round(fwd_tflops / world, 2),
                          "peak": peak_t, "unit": "TFLOP/s", "frac": round(fwd_tflops / world / peak_t, 4),
                          "frac_of_burst": round(fwd_tflops / world / peaks["bf16_tflops"], 4),
-                         "traffic": None, "peak_source": peak_src + " sustained"},
+                         "traffic": round(FWD_CAUSAL_2K_TRAFFIC) if fw is W.CAUSAL_2K else None,
+                         "traffic_source": "ncu capture of this workload",
+                         "peak_source": peak_src + " sustained"},
         "decode": {"value": round(dec_gbs, 1), "unit": "GB/s", "ms_per_launch": round(dec_ms, 4)},
         "fwd_ms_per_launch": round(fwd_ms, 4),
         "e2e": {"value": round(world * F / (e_fwd_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
