@@ -9,25 +9,32 @@
 // N x N scores never leave the SM.
 //
 // B200 mapping. One CTA owns one 128-row Q tile of one (batch, head) and
-// runs six warps:
-//   warps 0-3  softmax, one query row per thread (row = TMEM lane)
-//   warp  4    TMA producer: the Q tile once, then K_j, V_j into a ring of
-//              shared-memory slots (128-byte swizzle), mbarrier expect-tx
-//   warp  5    TMEM owner and MMA issuer (one elected thread)
+// runs eleven warps:
+//   warps 0-7  softmax: warps w and w + 4 share TMEM lanes 32 (w % 4) ..
+//              + 31 (one query row per lane) and split each row's 128 keys
+//              into halves, combining the half-row maxima and sums through
+//              shared memory
+//   warp  8    TMA producer: the Q tile once, then K and V tiles into two
+//              rings of shared-memory slots (128-byte swizzle), expect-tx
+//   warp  9    QK issuer (one elected thread) and TMEM owner
+//   warp 10    PV issuer (one elected thread)
 // Tensor memory (512 columns x 128 lanes x 32 bit):
-//   cols   0..127  S buffer 0 (fp32 scores; P, 16-bit, overwrites its first
-//                  64 columns and feeds the PV product straight from TMEM)
+//   cols   0..127  S buffer 0 (fp32 scores)
 //   cols 128..255  S buffer 1
 //   cols 256..383  O (fp32, d columns)
-// The scores are double-buffered: for K/V tile j the MMA thread issues
-//   S(j+1) = Q K_{j+1}^T into the other buffer, then (once P(j) is ready)
-//   O += P(j) V_j,
-// so the tensor core computes the next tile's scores while the softmax
-// warps work on this one, and the step time is max(softmax, tensor core)
-// rather than their sum. The softmax warps are alone on the SM's four
-// sub-partitions, so each has a whole MUFU (exp2) unit. tcgen05 operations
-// of one thread complete in issue order, so the product that reads P(j)
-// finishes before S(j+2) overwrites the same columns.
+//   cols 384..447  P buffer 0 (16-bit probabilities, two per column; the PV
+//                  product reads them straight from TMEM)
+//   cols 448..511  P buffer 1
+// Tile u of the CTA's key range uses S and P buffer u & 1. The QK thread
+// computes S(u) as soon as K(u) has landed and the PV product of tile u - 2
+// (the last reader of both buffers) is done; the PV thread computes
+// O += P(u) V(u) as soon as the softmax has published P(u). The two
+// products are independent, so they sit in different threads: each thread
+// waits on its own barriers while the other keeps the tensor pipe fed (the
+// pipe queues only a couple of MMAs), and each commits once per tile. The
+// next tile's scores are computed while the softmax warps work on the
+// current one, so the step time is max(softmax, tensor core) rather than
+// their sum.
 //
 // Rescaling is lazy: a row keeps its old max unless a new tile raises it by
 // more than 8 (log2 units), so P stays <= 2^8 and O is rescaled only when it
@@ -45,33 +52,49 @@ namespace {
 
 constexpr int BM = 128;  // query rows per Q tile
 constexpr int BN = 128;  // keys per K/V tile
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kMaxSlots = 12;
+constexpr int kThreads = 352;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kQkWarp = 9;   // issues S = Q K^T; owns TMEM
+constexpr int kPvWarp = 10;  // issues O += P V
+constexpr int kMaxSlots = 6;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kTmemCols = 512;
+// Rings of completion barriers, indexed by tile number modulo kRing. No
+// waiter is ever kRing tiles behind the phase it waits for: each ring
+// advances only through steps that need the waiter to have passed first
+// (P of a later tile, or a K/V load issued after the wait).
+constexpr int kRing = 8;
 constexpr uint32_t kTmemO = 256;
+constexpr uint32_t kTmemP = 384;  // two 64-column P buffers
 
 template <int D>
 struct Cfg {
   static constexpr int kChunkBytes = BM * 128;       // 128 rows x 64 elements x 2 bytes
   static constexpr int kTileBytes = BM * D * 2;      // one Q, K or V tile
-  static constexpr int kSlots = (D == 128) ? 6 : 12; // K/V ring depth
-  static constexpr int kSmemBytes = 1024 + (1 + kSlots) * kTileBytes + 1024;
+  static constexpr int kSlotsK = (D == 128) ? 3 : 6;  // K ring depth
+  static constexpr int kSlotsV = (D == 128) ? 2 : 6;  // V ring depth
+  static constexpr int kSlots = kSlotsK + kSlotsV;
+  static constexpr int kSmemBytes = 1024 + (1 + kSlots) * kTileBytes + 4096;
 };
 
 struct Barriers {
   uint64_t q_full;
-  uint64_t slot_full[kMaxSlots];
-  uint64_t slot_empty[kMaxSlots];
-  uint64_t s_full[2];  // per S buffer
-  uint64_t p_full[2];  // per S buffer
-  uint64_t pv_done;
-  uint64_t o_final;
-  uint64_t mma_done;
+  uint64_t k_full[kMaxSlots];
+  uint64_t v_full[kMaxSlots];
+  // s_ready[u % kRing]: S(f+u) is computed (commit of the QK thread), so its
+  // K slot is free too. pv_done[u % kRing]: O += P(f+u) V(f+u) is complete
+  // (commit of the PV thread): its V slot and P buffer are free and O is idle.
+  uint64_t s_ready[kRing];
+  uint64_t pv_done[kRing];
+  uint64_t p_full[2];  // per P buffer
+  uint64_t qk_idle;    // all MMAs of the QK thread complete
+  uint64_t pv_idle;    // all MMAs of the PV thread complete
   uint32_t tmem_base;
   int abort;
+  // per row and exchange parity: the two half-row partial maxima / sums
+  // (NaN marks a half that gave up on a timed-out wait)
+  float xchg[2][2][BM];
 };
 
 // Visible key interval [lo, hi] of query row q (empty when lo > hi).
@@ -99,7 +122,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 
 template <typename T, int D>
 __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV, uint8_t* sQ,
-                         uint8_t* sKV, Barriers* bars, int b, int h, int q0, int f, int l) {
+                         uint8_t* sK, uint8_t* sV, Barriers* bars, int b, int h, int q0, int f, int l) {
   using C = Cfg<D>;
   volatile int* abort = &bars->abort;
   const uint64_t pol_q = l2_policy_evict_first();
@@ -108,103 +131,110 @@ __device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const C
 #pragma unroll
   for (int ch = 0; ch < D / 64; ++ch)
     tma_load_4d(tmQ, &bars->q_full, sQ + ch * C::kChunkBytes, ch * 64, h, q0, b, pol_q);
-  // load order K(f), V(f), K(f+1), V(f+1), ... (the MMA thread acquires
-  // V(j) then K(j+1) in each step, which is the same sequence)
-  uint32_t it = 0;
-  bool ok = true;
-  for (int j = f; j <= l && ok; ++j) {
+  // Tile u of the CTA's range goes to slot u % depth of its ring; the slot's
+  // previous tile (u - depth) is free once the product that read it is done.
+  int nk = 0, nv = 0;  // loads issued
+  auto load = [&](const CUtensorMap* map, uint8_t* ring, uint64_t* full, uint64_t* freed, int depth, int u) -> bool {
+    const int slot = u % depth;
+    if (u >= depth && !mbar_wait(&freed[(u - depth) % kRing], ((u - depth) / kRing) & 1, abort)) return false;
+    mbar_arrive_expect_tx(&full[slot], C::kTileBytes);
 #pragma unroll
-    for (int kv = 0; kv < 2; ++kv) {
-      const uint32_t slot = it % C::kSlots, n = it / C::kSlots;
-      if (n > 0 && !mbar_wait(&bars->slot_empty[slot], (n - 1) & 1, abort)) {
-        ok = false;
-        break;
-      }
-      mbar_arrive_expect_tx(&bars->slot_full[slot], C::kTileBytes);
-      const CUtensorMap* map = kv ? tmV : tmK;
-#pragma unroll
-      for (int ch = 0; ch < D / 64; ++ch)
-        tma_load_4d(map, &bars->slot_full[slot], sKV + slot * C::kTileBytes + ch * C::kChunkBytes, ch * 64, h,
-                    j * BN, b, pol_kv);
-      ++it;
-    }
+    for (int ch = 0; ch < D / 64; ++ch)
+      tma_load_4d(map, &full[slot], ring + slot * C::kTileBytes + ch * C::kChunkBytes, ch * 64, h, (f + u) * BN, b,
+                  pol_kv);
+    return true;
+  };
+  auto load_k = [&](int u) {
+    const bool ok = load(tmK, sK, bars->k_full, bars->s_ready, C::kSlotsK, u);
+    nk += ok;
+    return ok;
+  };
+  auto load_v = [&](int u) {
+    const bool ok = load(tmV, sV, bars->v_full, bars->pv_done, C::kSlotsV, u);
+    nv += ok;
+    return ok;
+  };
+  // in order of need: K(f), K(f+1), V(f), then K(f+u+2), V(f+u+1)
+  const int n = l - f + 1;
+  bool ok = load_k(0);
+  if (ok && n > 1) ok = load_k(1);
+  if (ok) ok = load_v(0);
+  for (int u = 0; u + 1 < n && ok; ++u) {
+    if (u + 2 < n) ok = load_k(u + 2);
+    if (ok) ok = load_v(u + 1);
   }
   // Every load issued must land before the CTA may exit. On the normal path
-  // they all have (the MMA thread consumed them); after an abort, wait.
+  // they all have (the MMA threads consumed them); after an abort, wait.
   drain_wait(&bars->q_full, 0);
-  const uint32_t first = it > static_cast<uint32_t>(C::kSlots) ? it - C::kSlots : 0;
-  for (uint32_t i = first; i < it; ++i) drain_wait(&bars->slot_full[i % C::kSlots], (i / C::kSlots) & 1);
+  for (int u = max(0, nk - C::kSlotsK); u < nk; ++u) drain_wait(&bars->k_full[u % C::kSlotsK], (u / C::kSlotsK) & 1);
+  for (int u = max(0, nv - C::kSlotsV); u < nv; ++u) drain_wait(&bars->v_full[u % C::kSlotsV], (u / C::kSlotsV) & 1);
 }
 
+// S(f+u) = Q K_{f+u}^T into S buffer u & 1: M = 128 query rows, N = 128
+// keys, K = d in steps of 16; both operands K-major, 128-byte swizzled, 64
+// elements per 16 KB chunk. Before overwriting the buffer the thread waits
+// for the PV product of tile u - 2: that product waited for P(u - 2), so the
+// softmax is done with S(u - 2), and once it completes P buffer u & 1 is
+// free as well; the commit that publishes S(u) therefore also tells the
+// softmax that it may write P(u).
 template <typename T, int D>
-__device__ void mma_issuer(uint8_t* sQ, uint8_t* sKV, Barriers* bars, uint32_t tmem, int f, int l, bool negate) {
+__device__ void qk_issuer(uint8_t* sQ, uint8_t* sK, Barriers* bars, uint32_t tmem, int n, bool negate) {
   using C = Cfg<D>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   // a negative softmax scale is applied as -Q K^T (A-negate bit) times |scale|
-  const uint32_t idesc_qk = instr_desc_f16(kBf16, BM, BN, false) | (negate ? (1u << 13) : 0u);
-  constexpr uint32_t idesc_pv = instr_desc_f16(kBf16, BM, D, true);
+  const uint32_t idesc = instr_desc_f16(kBf16, BM, BN, false) | (negate ? (1u << 13) : 0u);
   volatile int* abort = &bars->abort;
-  const uint32_t sQaddr = smem_addr(sQ);
-  const uint32_t sKVaddr = smem_addr(sKV);
-
-  uint32_t it = 0;
-  auto acquire = [&](uint32_t& addr, uint32_t& slot) -> bool {
-    slot = it % C::kSlots;
-    const bool ok = mbar_wait(&bars->slot_full[slot], (it / C::kSlots) & 1, abort);
-    addr = sKVaddr + slot * C::kTileBytes;
-    ++it;
-    return ok;
-  };
-  // S(j) = Q K_j^T into S buffer (j - f) & 1: M = 128 query rows, N = 128
-  // keys, K = d in steps of 16. Both operands are K-major, 128-byte
-  // swizzled, 64 elements per 16 KB chunk.
-  auto qk = [&](int j, uint32_t kaddr) {
-    const uint32_t d_t = tmem + ((j - f) & 1) * 128;
+  // Descriptors are built once per operand tile; stepping K by 16 adds a
+  // byte offset to the start-address field (16-byte units, no carry: shared
+  // addresses are below 2^18).
+  const uint64_t qdesc = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+  const uint32_t sKaddr = smem_addr(sK);
+  bool ok = mbar_wait(&bars->q_full, 0, abort);
+  for (int u = 0; u < n && ok; ++u) {
+    if (u >= 2 && !(ok = mbar_wait(&bars->pv_done[(u - 2) % kRing], ((u - 2) / kRing) & 1, abort))) break;
+    const int slot = u % C::kSlotsK;
+    if (!(ok = mbar_wait(&bars->k_full[slot], (u / C::kSlotsK) & 1, abort))) break;
+    tc_fence_after();
+    const uint32_t d_t = tmem + (u & 1) * 128;
+    const uint64_t kdesc = smem_desc_sw128(sKaddr + slot * C::kTileBytes, 16, 1024);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t off = (kk / 4) * C::kChunkBytes + (kk % 4) * 32;
-      mma_ss(d_t, smem_desc_sw128(sQaddr + off, 16, 1024), smem_desc_sw128(kaddr + off, 16, 1024), idesc_qk,
-             kk > 0 ? 1u : 0u);
+      const uint32_t off = ((kk / 4) * C::kChunkBytes + (kk % 4) * 32) >> 4;
+      mma_ss(d_t, qdesc + off, kdesc + off, idesc, kk > 0 ? 1u : 0u);
     }
-    tc_commit(&bars->s_full[(j - f) & 1]);
-  };
-  // O (+)= P(j) V_j: A = P from TMEM (16-bit, two keys per column), B = V
-  // tile stored keys x d with d contiguous (MN-major): 16 keys = 2048 bytes,
-  // the second 64-wide d chunk lies 16 KB further (leading byte offset).
-  auto pv = [&](int j, uint32_t vaddr) {
-    const uint32_t a_t = tmem + ((j - f) & 1) * 128;
-#pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk)
-      mma_ts(tmem + kTmemO, a_t + kk * 8, smem_desc_sw128(vaddr + kk * 2048, C::kChunkBytes, 1024), idesc_pv,
-             (j > f || kk > 0) ? 1u : 0u);
-    tc_commit(&bars->pv_done);
-    if (j == l) tc_commit(&bars->o_final);
-  };
-
-  bool ok = mbar_wait(&bars->q_full, 0, abort);
-  uint32_t aK = 0, slotK = 0, aV = 0, slotV = 0;
-  if (ok && (ok = acquire(aK, slotK))) {
-    qk(f, aK);
-    tc_commit(&bars->slot_empty[slotK]);
-  }
-  for (int j = f; j <= l && ok; ++j) {
-    const bool next = j < l;
-    if (!(ok = acquire(aV, slotV))) break;
-    if (next) {
-      // the next tile's scores go into the other S buffer; its previous
-      // contents (P(j-1)) were consumed by the PV product issued last step
-      if (!(ok = acquire(aK, slotK))) break;
-      qk(j + 1, aK);
-      tc_commit(&bars->slot_empty[slotK]);
-    }
-    if (!(ok = mbar_wait(&bars->p_full[(j - f) & 1], ((j - f) >> 1) & 1, abort))) break;
-    tc_fence_after();
-    pv(j, aV);
-    tc_commit(&bars->slot_empty[slotV]);
+    tc_commit(&bars->s_ready[u % kRing]);
   }
   // All MMAs of this thread must be complete before TMEM is released.
-  tc_commit(&bars->mma_done);
-  drain_wait(&bars->mma_done, 0);
+  tc_commit(&bars->qk_idle);
+  drain_wait(&bars->qk_idle, 0);
+}
+
+// O (+)= P(f+u) V_{f+u}: A = P from TMEM (16-bit, two keys per column, P
+// buffer u & 1), B = V tile stored keys x d with d contiguous (MN-major):
+// 16 keys = 2048 bytes, the second 64-wide d chunk lies 16 KB further
+// (leading byte offset).
+template <typename T, int D>
+__device__ void pv_issuer(uint8_t* sV, Barriers* bars, uint32_t tmem, int n) {
+  using C = Cfg<D>;
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  constexpr uint32_t idesc = instr_desc_f16(kBf16, BM, D, true);
+  volatile int* abort = &bars->abort;
+  const uint32_t sVaddr = smem_addr(sV);
+  bool ok = true;
+  for (int u = 0; u < n && ok; ++u) {
+    if (!(ok = mbar_wait(&bars->p_full[u & 1], (u >> 1) & 1, abort))) break;
+    const int slot = u % C::kSlotsV;
+    if (!(ok = mbar_wait(&bars->v_full[slot], (u / C::kSlotsV) & 1, abort))) break;
+    tc_fence_after();
+    const uint32_t a_t = tmem + kTmemP + (u & 1) * 64;
+    const uint64_t vdesc = smem_desc_sw128(sVaddr + slot * C::kTileBytes, C::kChunkBytes, 1024);
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk)
+      mma_ts(tmem + kTmemO, a_t + kk * 8, vdesc + ((kk * 2048) >> 4), idesc, (u > 0 || kk > 0) ? 1u : 0u);
+    tc_commit(&bars->pv_done[u % kRing]);
+  }
+  tc_commit(&bars->pv_idle);
+  drain_wait(&bars->pv_idle, 0);
 }
 
 // Score transform of one element in log2 units (softcap and ALiBi paths).
@@ -215,18 +245,46 @@ __device__ __forceinline__ float mod_score(const FwdParams& p, float x, float sl
   return t;
 }
 
-// The softmax warpgroup: one query row per thread, row == TMEM lane.
+// Softmax: eight warps, two per sub-partition. Warp w (w < 4) and warp
+// w + 4 own the same 32 query rows (TMEM lanes 32(w % 4) ..), one row per
+// thread; warp w takes keys 0-63 of each 128-key tile and warp w + 4 keys
+// 64-127. The two halves of a row exchange partial maxima through shared
+// memory under a 64-thread named barrier, so both take the same lazy
+// rescaling decision; each half writes its part of P (16-bit, into columns
+// [32 * half, 32 * half + 32) of the tile's P buffer), rescales and stores
+// its 64 columns of O, and the row sums are combined once at the end.
 // kCap / kAlibi select the score modifiers at compile time; whether a K tile
 // needs the element mask is decided per tile for the whole group, so the
 // common interior tiles run without per-element compares.
+__device__ __forceinline__ void pair_sync(int quarter) {
+  // named barrier 1 + quarter, shared by the two warps of one lane quarter
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+}
+
+// Exchange of one value between the two halves of a row. Both halves call
+// it the same number of times (the k-th exchange uses slot k & 1, so a slot
+// is rewritten only after the partner has passed the next barrier and hence
+// read it). A half that failed passes NaN; the caller sees the partner's
+// value, NaN if the partner failed.
+__device__ __forceinline__ float pair_exchange(float (&xchg)[2][2][BM], int k, int half, int r, int quarter,
+                                               float v) {
+  xchg[k & 1][half][r] = v;
+  pair_sync(quarter);
+  return xchg[k & 1][half ^ 1][r];
+}
+
 template <typename T, int D, bool kCap, bool kAlibi>
 __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem, int b, int h, int q0, bool has,
                               int f, int l) {
   constexpr bool kPlain = !kCap && !kAlibi;
+  constexpr int kHalf = BN / 2;       // keys per thread per tile
+  constexpr int kOCols = D / 2;       // O columns per thread
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int r = warp * 32 + lane;  // row of the tile == TMEM lane
+  const int quarter = warp & 3;
+  const int half = warp >> 2;
+  const int r = quarter * 32 + lane;  // row of the tile == TMEM lane
   const int q = q0 + r;
   const bool row_ok = q < p.Nq;
   const RowRange rr = row_range(p, row_ok ? q : p.Nq - 1);
@@ -235,69 +293,75 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
   const int qz = min(q0 + BM - 1, p.Nq - 1);
   const RowRange first_row = row_range(p, q0), last_row = row_range(p, qz);
   const int pos = q + p.Nk - p.Nq;
-  const uint32_t lane_sel = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t tO = tmem + lane_sel + kTmemO;
+  const uint32_t lane_sel = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t tO = tmem + lane_sel + kTmemO + half * kOCols;
   const float slope_l2 = kAlibi ? p.slopes[h] * kLog2e : 0.0f;
   const float sl2 = p.scale_log2;  // >= 0 (a negative scale is folded into the MMA)
+  const uint64_t mul2 = kPlain ? f2_pack(sl2, sl2) : f2_pack(1.0f, 1.0f);
 
-  float m = -INFINITY;  // running max (log2 units)
-  float lsum = 0.0f;    // running sum of exp2(t - m)
+  float m = -INFINITY;  // running max of the whole row (log2 units)
+  float lsum = 0.0f;    // this half's running sum of exp2(t - m)
   bool ok = true;
+  bool broke = false;   // left the loop at a shared exchange (both halves do)
   const int n = has ? l - f + 1 : 0;
+  // Each iteration performs exactly one pair exchange, and every early exit
+  // happens right after one, on a decision both halves share, so the named
+  // barriers can never be left waiting for a partner that has gone.
   for (int it = 0; it < n; ++it) {
     const int j = f + it;
     const uint32_t tS = tmem + lane_sel + (it & 1) * 128;
-    ok = mbar_wait(&bars->s_full[it & 1], (it >> 1) & 1, abort);
+    ok = ok && mbar_wait(&bars->s_ready[it % kRing], (it / kRing) & 1, abort);
     ok = __all_sync(0xffffffffu, ok);
-    if (!ok) break;
-    tc_fence_after();
-    uint32_t s[4][32];
-    const int key0 = j * BN;
-    const bool masked = key0 < last_row.lo || key0 + BN - 1 > first_row.hi;  // uniform over the tile
-    // pass 1: transform (modifier paths) and tile max. S arrives in two
-    // halves so the second TMEM load overlaps the first half's work; four
-    // independent 3-input max chains keep the pipes busy.
-    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-    auto half_max = [&](int c0) {
+    uint32_t s[2][32];
+    const int key0 = j * BN + half * kHalf;
+    const bool masked = j * BN < last_row.lo || j * BN + BN - 1 > first_row.hi;  // uniform over the tile
+    if (ok) {
+      tc_fence_after();
+      tmem_ld32(tS + half * kHalf, s[0]);
+      tmem_ld32(tS + half * kHalf + 32, s[1]);
+      tmem_wait_ld();
+    } else {
 #pragma unroll
-      for (int c = c0; c < c0 + 2; ++c) {
-        if (!kPlain || masked) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float x = __uint_as_float(s[c][e]);
-            const int key = key0 + 32 * c + e;
-            if (!kPlain) x = mod_score<kCap, kAlibi>(p, x, slope_l2, pos - key);
-            if (masked) x = (key >= rr.lo && key <= rr.hi) ? x : -INFINITY;
-            s[c][e] = __float_as_uint(x);
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          const int a = (e / 8) & 3;
-          mx[a] = fmax3(mx[a], __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
-          mx[a] = fmax3(mx[a], __uint_as_float(s[c][e + 2]), __uint_as_float(s[c][e + 3]));
-          mx[a] = fmax3(mx[a], __uint_as_float(s[c][e + 4]), __uint_as_float(s[c][e + 5]));
-          mx[a] = fmax3(mx[a], __uint_as_float(s[c][e + 6]), __uint_as_float(s[c][e + 7]));
-        }
-      }
-    };
-    tmem_ld32(tS, s[0]);
-    tmem_ld32(tS + 32, s[1]);
-    tmem_wait_ld();
+      for (int e = 0; e < 32; ++e) s[0][e] = s[1][e] = 0u;
+    }
     reg_fence(s[0]);
     reg_fence(s[1]);
-    tmem_ld32(tS + 64, s[2]);
-    tmem_ld32(tS + 96, s[3]);
-    half_max(0);
-    tmem_wait_ld();
-    reg_fence(s[2]);
-    reg_fence(s[3]);
-    half_max(2);
+    // pass 1: transform (modifier paths), mask and this half's max
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      if (!kPlain || masked) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float x = __uint_as_float(s[c][e]);
+          const int key = key0 + 32 * c + e;
+          if (!kPlain) x = mod_score<kCap, kAlibi>(p, x, slope_l2, pos - key);
+          if (masked) x = (key >= rr.lo && key <= rr.hi) ? x : -INFINITY;
+          s[c][e] = __float_as_uint(x);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 32; e += 8) {
+        const int a = (e / 8) & 3;
+        mx[a] = fmax3(mx[a], __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
+        mx[a] = fmax3(mx[a], __uint_as_float(s[c][e + 2]), __uint_as_float(s[c][e + 3]));
+        mx[a] = fmax3(mx[a], __uint_as_float(s[c][e + 4]), __uint_as_float(s[c][e + 5]));
+        mx[a] = fmax3(mx[a], __uint_as_float(s[c][e + 6]), __uint_as_float(s[c][e + 7]));
+      }
+    }
     float mt = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
+    // combine with the other half of the row
+    const float mo = pair_exchange(bars->xchg, it, half, r, quarter, ok ? mt : __int_as_float(0x7fc00000));
+    ok = __all_sync(0xffffffffu, ok && mo == mo);
+    if (!ok) {  // both halves of every row of this warp pair see the same NaN
+      broke = true;
+      break;
+    }
+    mt = fmaxf(mt, mo);
     // plain path: the max was taken over raw scores; scale after (sl2 >= 0)
     if (kPlain) mt = (mt == -INFINITY) ? -INFINITY : mt * sl2;
 
-    // lazy max update
+    // lazy max update (identical in both halves of the row)
     const float m_new = fmaxf(m, mt);
     float alpha = 1.0f;
     bool rescale = false;
@@ -310,32 +374,47 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
     }
     lsum *= alpha;
     const float m_eff = (m == -INFINITY) ? 0.0f : m;
-    // pass 2: P = exp2(t - m) into the first 64 columns of this S buffer.
-    // Pairs of elements go through packed fp32x2 instructions: one FMA
-    // (scale and subtract the max) and one add (row sum) per pair.
+    // pass 2: P = exp2(t - m) into columns [32 * half, 32 * half + 32) of the
+    // P buffer; pairs of elements go through packed fp32x2 FMA (scale,
+    // subtract max) and add
     const uint64_t m2 = f2_pack(-m_eff, -m_eff);
-    const uint64_t mul2 = kPlain ? f2_pack(sl2, sl2) : f2_pack(1.0f, 1.0f);
     uint64_t rsum2[4] = {0, 0, 0, 0};  // independent packed partial sums (0 bits = +0.0f)
+    uint32_t pk[32];
+    auto pass2 = [&](auto emu_tag) {
+      constexpr bool kEmu = decltype(emu_tag)::value;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t pk[16];
+      for (int c = 0; c < 2; ++c) {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float x0 = __uint_as_float(s[c][2 * e]);
-        const float x1 = __uint_as_float(s[c][2 * e + 1]);
-        float a0, a1;
-        f2_unpack(f2_fma(f2_pack(x0, x1), mul2, m2), a0, a1);
-        float p0 = ex2(a0), p1 = ex2(a1);
-        if (kPlain && masked) {
-          // masked entries hold -inf; -inf * 0 would be NaN, so select them out
-          p0 = (x0 == -INFINITY) ? 0.0f : p0;
-          p1 = (x1 == -INFINITY) ? 0.0f : p1;
+        for (int e = 0; e < 16; ++e) {
+          const float x0 = __uint_as_float(s[c][2 * e]);
+          const float x1 = __uint_as_float(s[c][2 * e + 1]);
+          const uint64_t a2 = f2_fma(f2_pack(x0, x1), mul2, m2);
+          float p0, p1;
+          if (kEmu && (e & 7) >= 5) {
+            // three pairs in eight take exp2 on the FMA pipe, so the MUFU is
+            // not the only unit doing exponentials
+            f2_unpack(ex2_poly_x2(a2), p0, p1);
+          } else {
+            float a0, a1;
+            f2_unpack(a2, a0, a1);
+            p0 = ex2(a0);
+            p1 = ex2(a1);
+          }
+          if (kPlain && !kEmu) {
+            // masked entries hold -inf; -inf * 0 would be NaN, so select them out
+            p0 = (x0 == -INFINITY) ? 0.0f : p0;
+            p1 = (x1 == -INFINITY) ? 0.0f : p1;
+          }
+          rsum2[e & 3] = f2_add(rsum2[e & 3], f2_pack(p0, p1));
+          pk[16 * c + e] = pack2<T>(p0, p1);
         }
-        rsum2[e & 3] = f2_add(rsum2[e & 3], f2_pack(p0, p1));
-        pk[e] = pack2<T>(p0, p1);
       }
-      tmem_st16(tS + 16 * c, pk);
-    }
+    };
+    if (masked)
+      pass2(std::false_type{});
+    else
+      pass2(std::true_type{});
+    tmem_st32(tmem + lane_sel + kTmemP + (it & 1) * 64 + half * 32, pk);
     float r0, r1, r2, r3;
     f2_unpack(f2_add(rsum2[0], rsum2[1]), r0, r1);
     f2_unpack(f2_add(rsum2[2], rsum2[3]), r2, r3);
@@ -344,13 +423,13 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
       // O must be idle: wait for the product of the previous tile (the only
       // one that can still be running).
       if (it > 0) {
-        ok = mbar_wait(&bars->pv_done, (it - 1) & 1, abort);
+        // on a timeout, carry on to the next exchange, which ends both halves
+        ok = mbar_wait(&bars->pv_done[(it - 1) % kRing], ((it - 1) / kRing) & 1, abort);
         ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
         tc_fence_after();
       }
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = 0; cc < kOCols / 32; ++cc) {
         uint32_t o[32];
         tmem_ld32(tO + 32 * cc, o);
         tmem_wait_ld();
@@ -366,19 +445,31 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars->p_full[it & 1]);
   }
+  // the loop ran the same number of exchanges in both halves: it ended at a
+  // shared break, or after all n iterations (possibly with a failed wait in
+  // one half, which the final exchange reports to the other)
+  const int n_done = broke ? -1 : n;
   if (ok && n > 0) {
-    ok = mbar_wait(&bars->o_final, 0, abort);
+    ok = mbar_wait(&bars->pv_done[(n - 1) % kRing], ((n - 1) / kRing) & 1, abort);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
   }
+  // both halves of a row must agree on success; combine the row sums
+  float ltot = lsum;
+  if (n_done >= 0) {
+    const float other = pair_exchange(bars->xchg, n_done, half, r, quarter, ok ? lsum : __int_as_float(0x7fc00000));
+    ok = ok && other == other;
+    ltot = lsum + (other == other ? other : 0.0f);
+  }
 
-  // epilogue: O / l -> dtype, LSE = (m + log2 l) ln 2
-  T* orow = reinterpret_cast<T*>(p.out) + ((static_cast<size_t>(b) * p.Nq + (row_ok ? q : 0)) * p.H + h) * D;
-  const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+  // epilogue: O / l -> dtype for this half's columns, LSE = (m + log2 l) ln 2
+  T* orow = reinterpret_cast<T*>(p.out) + ((static_cast<size_t>(b) * p.Nq + (row_ok ? q : 0)) * p.H + h) * D +
+            half * kOCols;
+  const float inv = ltot > 0.0f ? 1.0f / ltot : 0.0f;
   const float nan = __int_as_float(0x7fc00000);
   if (ok && n > 0) {
 #pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
+    for (int cc = 0; cc < kOCols / 32; ++cc) {
       uint32_t o[32];
       tmem_ld32(tO + 32 * cc, o);
       tmem_wait_ld();
@@ -398,12 +489,12 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
     const uint32_t w = pack2<T>(fill, fill);
     uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-    for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(w, w, w, w);
+    for (int v = 0; v < kOCols / 8; ++v) dst[v] = make_uint4(w, w, w, w);
   }
-  if (row_ok) {
+  if (row_ok && half == 0) {
     float lse_v;
     if (!ok) lse_v = nan;
-    else if (lsum > 0.0f) lse_v = (m + lg2(lsum)) * kLn2;
+    else if (ltot > 0.0f) lse_v = (m + lg2(ltot)) * kLn2;
     else lse_v = -INFINITY;
     p.lse[(static_cast<size_t>(b) * p.H + h) * p.Nq + q] = lse_v;
   }
@@ -417,8 +508,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sKV = smem + C::kTileBytes;
-  Barriers* bars = reinterpret_cast<Barriers*>(sKV + C::kSlots * C::kTileBytes);
+  uint8_t* sK = smem + C::kTileBytes;
+  uint8_t* sV = sK + C::kSlotsK * C::kTileBytes;
+  Barriers* bars = reinterpret_cast<Barriers*>(sV + C::kSlotsV * C::kTileBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -438,21 +530,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int i = 0; i < C::kSlots; ++i) {
-      mbar_init(&bars->slot_full[i], 1);
-      mbar_init(&bars->slot_empty[i], 1);
-    }
+    for (int i = 0; i < C::kSlotsK; ++i) mbar_init(&bars->k_full[i], 1);
+    for (int i = 0; i < C::kSlotsV; ++i) mbar_init(&bars->v_full[i], 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 4);
+      mbar_init(&bars->p_full[i], kSoftmaxWarps);
     }
-    mbar_init(&bars->pv_done, 1);
-    mbar_init(&bars->o_final, 1);
-    mbar_init(&bars->mma_done, 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&bars->s_ready[i], 1);
+      mbar_init(&bars->pv_done[i], 1);
+    }
+    mbar_init(&bars->qk_idle, 1);
+    mbar_init(&bars->pv_idle, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kQkWarp) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -466,17 +558,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp < 4) {
+  if (warp < kSoftmaxWarps) {
     softmax_group<T, D, kCap, kAlibi>(p, bars, tmem, b, h, q0, has, f, l);
   } else if (warp == kProducerWarp) {
-    if (lane == 0 && has) producer<T, D>(&tmQ, &tmK, &tmV, sQ, sKV, bars, b, h, q0, f, l);
+    if (lane == 0 && has) producer<T, D>(&tmQ, &tmK, &tmV, sQ, sK, sV, bars, b, h, q0, f, l);
+  } else if (warp == kQkWarp) {
+    if (lane == 0 && has) qk_issuer<T, D>(sQ, sK, bars, tmem, l - f + 1, p.negate_scores != 0);
   } else {
-    if (lane == 0 && has) mma_issuer<T, D>(sQ, sKV, bars, tmem, f, l, p.negate_scores != 0);
+    if (lane == 0 && has) pv_issuer<T, D>(sV, bars, tmem, l - f + 1);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kQkWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -487,9 +581,9 @@ template <typename T, int D, bool kCap, bool kAlibi>
 cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const FwdParams& p,
                    cudaStream_t stream) {
   using C = Cfg<D>;
-  static_assert(sizeof(Barriers) <= 1024, "barrier block exceeds its reserve");
+  static_assert(sizeof(Barriers) <= 4096, "barrier block exceeds its reserve");
   static_assert(C::kSmemBytes <= 232448, "shared memory budget exceeded");
-  static_assert(C::kSlots <= kMaxSlots, "too many K/V slots");
+  static_assert(C::kSlotsK <= kMaxSlots && C::kSlotsV <= kMaxSlots, "too many K/V slots");
   auto kernel = fwd_kernel<T, D, kCap, kAlibi>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
