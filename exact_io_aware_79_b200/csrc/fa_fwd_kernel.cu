@@ -8,14 +8,16 @@
 // running row max m and row sum l and rescales the partial output, so the
 // N x N scores never leave the SM.
 //
-// B200 mapping. One CTA owns one 128-row Q tile of one (batch, head) and
-// runs eleven warps:
+// B200 mapping. The grid is persistent (at most one CTA per SM); a CTA runs
+// jobs, each one 128-row Q tile of one (batch, head), back to back with
+// eleven warps:
 //   warps 0-7  softmax: warps w and w + 4 share TMEM lanes 32 (w % 4) ..
 //              + 31 (one query row per lane) and split each row's 128 keys
 //              into halves, combining the half-row maxima and sums through
 //              shared memory
-//   warp  8    TMA producer: the Q tile once, then K and V tiles into two
-//              rings of shared-memory slots (128-byte swizzle), expect-tx
+//   warp  8    TMA producer: each job's Q tile (two buffers, so the next
+//              job's Q lands early), then K and V tiles into two rings of
+//              shared-memory slots (128-byte swizzle), expect-tx
 //   warp  9    QK issuer (one elected thread) and TMEM owner
 //   warp 10    PV issuer (one elected thread)
 // Tensor memory (512 columns x 128 lanes x 32 bit):
@@ -25,10 +27,12 @@
 //   cols 384..447  P buffer 0 (16-bit probabilities, two per column; the PV
 //                  product reads them straight from TMEM)
 //   cols 448..511  P buffer 1
-// Tile u of the CTA's key range uses S and P buffer u & 1. The QK thread
-// computes S(u) as soon as K(u) has landed and the PV product of tile u - 2
-// (the last reader of both buffers) is done; the PV thread computes
-// O += P(u) V(u) as soon as the softmax has published P(u). The two
+// K/V tiles are numbered across the CTA's jobs; tile g uses S and P buffer
+// g & 1. The QK thread computes S(g) as soon as K(g) has landed and the PV
+// product of tile g - 2 (the last reader of both buffers) is done; the PV
+// thread computes O += P(g) V(g) as soon as the softmax has published P(g).
+// Across a job boundary the next job's first scores are computed while the
+// softmax warps write out the previous job's O. The two
 // products are independent, so they sit in different threads: each thread
 // waits on its own barriers while the other keeps the tensor pipe fed (the
 // pipe queues only a couple of MMAs), and each commits once per tile. The
@@ -47,6 +51,7 @@
 #include <climits>
 #include <type_traits>
 
+
 namespace fa {
 namespace {
 
@@ -57,6 +62,7 @@ constexpr int kSoftmaxWarps = 8;
 constexpr int kProducerWarp = 8;
 constexpr int kQkWarp = 9;   // issues S = Q K^T; owns TMEM
 constexpr int kPvWarp = 10;  // issues O += P V
+static_assert(kThreads == 32 * (kPvWarp + 1), "one warp per role after the softmax warps");
 constexpr int kMaxSlots = 6;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kTmemCols = 512;
@@ -72,22 +78,27 @@ template <int D>
 struct Cfg {
   static constexpr int kChunkBytes = BM * 128;       // 128 rows x 64 elements x 2 bytes
   static constexpr int kTileBytes = BM * D * 2;      // one Q, K or V tile
-  static constexpr int kSlotsK = (D == 128) ? 3 : 6;  // K ring depth
-  static constexpr int kSlotsV = (D == 128) ? 2 : 6;  // V ring depth
+  // two Q buffers, so the next job's Q lands while this one's runs
+  static constexpr int kQBufs = 2;                    // active job a uses buffer a % kQBufs
+  static constexpr int kSlotsK = (D == 128) ? 2 : 5;  // K ring depth
+  static constexpr int kSlotsV = (D == 128) ? 2 : 5;  // V ring depth
   static constexpr int kSlots = kSlotsK + kSlotsV;
-  static constexpr int kSmemBytes = 1024 + (1 + kSlots) * kTileBytes + 4096;
+  static constexpr int kSmemBytes = 1024 + (kQBufs + kSlots) * kTileBytes + 4096;
 };
 
 struct Barriers {
-  uint64_t q_full;
+  uint64_t q_full[2];   // per Q buffer (active job a uses buffer a & 1)
+  uint64_t q_empty[2];  // the QK thread is done with the buffer's job
   uint64_t k_full[kMaxSlots];
   uint64_t v_full[kMaxSlots];
-  // s_ready[u % kRing]: S(f+u) is computed (commit of the QK thread), so its
-  // K slot is free too. pv_done[u % kRing]: O += P(f+u) V(f+u) is complete
-  // (commit of the PV thread): its V slot and P buffer are free and O is idle.
+  // Tiles are numbered across the CTA's jobs (g). s_ready[g % kRing]: S(g)
+  // is computed (commit of the QK thread), so its K slot is free too.
+  // pv_done[g % kRing]: O += P(g) V(g) is complete (commit of the PV
+  // thread): its V slot and P buffer are free and O is idle.
   uint64_t s_ready[kRing];
   uint64_t pv_done[kRing];
   uint64_t p_full[2];  // per P buffer
+  uint64_t o_free;     // the softmax warps have read O of an active job
   uint64_t qk_idle;    // all MMAs of the QK thread complete
   uint64_t pv_idle;    // all MMAs of the PV thread complete
   uint32_t tmem_base;
@@ -120,119 +131,190 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   mbar_wait(bar, parity, &dummy);
 }
 
+// A CTA is persistent: it runs jobs (one 128-row Q tile of one (batch,
+// head) each) one after another, and every role walks the same job
+// sequence. Work items pair Q tile t of a head with tile T - 1 - t (T tiles
+// per head), so under a causal mask every item has the same number of K/V
+// tiles; CTA c takes items c, c + gridDim.x, ... and runs the longer tile of
+// each item first. Consecutive items belong to the same head, so the CTAs
+// running at one time share K/V in L2.
+struct Job {
+  int b, h, q0, f, l;  // K/V tiles f..l
+  bool has;            // at least one visible key
+};
+
+__device__ __forceinline__ Job make_job(const FwdParams& p, int bh, int tile) {
+  Job j;
+  j.b = bh / p.H;
+  j.h = bh % p.H;
+  j.q0 = tile * BM;
+  // K/V tile range of the Q tile (rows' visible intervals are monotone in q)
+  const int qz = min(j.q0 + BM - 1, p.Nq - 1);
+  const RowRange ra = row_range(p, j.q0), rz = row_range(p, qz);
+  j.has = ra.lo <= rz.hi;
+  j.f = j.has ? ra.lo / BN : 0;
+  j.l = j.has ? rz.hi / BN : -1;
+  return j;
+}
+
+// Calls fn(job) for every job of this CTA, in order.
+template <typename Fn>
+__device__ __forceinline__ void for_each_job(const FwdParams& p, Fn&& fn) {
+  const int per_head = (p.num_tiles + 1) / 2;
+  const int items = p.B * p.H * per_head;
+  for (int w = static_cast<int>(blockIdx.x); w < items; w += static_cast<int>(gridDim.x)) {
+    const int bh = w / per_head, pi = w % per_head;
+    const int t_long = p.num_tiles - 1 - pi;
+    fn(make_job(p, bh, t_long));
+    if (pi != t_long) fn(make_job(p, bh, pi));
+  }
+}
+
 template <typename T, int D>
-__device__ void producer(const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV, uint8_t* sQ,
-                         uint8_t* sK, uint8_t* sV, Barriers* bars, int b, int h, int q0, int f, int l) {
+__device__ void producer(const FwdParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                         uint8_t* sQ, uint8_t* sK, uint8_t* sV, Barriers* bars) {
   using C = Cfg<D>;
   volatile int* abort = &bars->abort;
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
-  mbar_arrive_expect_tx(&bars->q_full, C::kTileBytes);
-#pragma unroll
-  for (int ch = 0; ch < D / 64; ++ch)
-    tma_load_4d(tmQ, &bars->q_full, sQ + ch * C::kChunkBytes, ch * 64, h, q0, b, pol_q);
-  // Tile u of the CTA's range goes to slot u % depth of its ring; the slot's
-  // previous tile (u - depth) is free once the product that read it is done.
-  int nk = 0, nv = 0;  // loads issued
-  auto load = [&](const CUtensorMap* map, uint8_t* ring, uint64_t* full, uint64_t* freed, int depth, int u) -> bool {
-    const int slot = u % depth;
-    if (u >= depth && !mbar_wait(&freed[(u - depth) % kRing], ((u - depth) / kRing) & 1, abort)) return false;
+  // Tile g goes to slot g % depth of its ring; the slot's previous tile
+  // (g - depth) is free once the product that read it is done.
+  int g = 0, a = 0;    // tiles and active jobs so far
+  int nk = 0, nv = 0;  // K and V loads issued
+  bool ok = true;
+  auto load = [&](const CUtensorMap* map, uint8_t* ring, uint64_t* full, uint64_t* freed, int depth, int gi,
+                  const Job& jb, int key_tile) -> bool {
+    const int slot = gi % depth;
+    if (gi >= depth && !mbar_wait(&freed[(gi - depth) % kRing], ((gi - depth) / kRing) & 1, abort)) return false;
     mbar_arrive_expect_tx(&full[slot], C::kTileBytes);
 #pragma unroll
     for (int ch = 0; ch < D / 64; ++ch)
-      tma_load_4d(map, &full[slot], ring + slot * C::kTileBytes + ch * C::kChunkBytes, ch * 64, h, (f + u) * BN, b,
-                  pol_kv);
+      tma_load_4d(map, &full[slot], ring + slot * C::kTileBytes + ch * C::kChunkBytes, ch * 64, jb.h,
+                  key_tile * BN, jb.b, pol_kv);
     return true;
   };
-  auto load_k = [&](int u) {
-    const bool ok = load(tmK, sK, bars->k_full, bars->s_ready, C::kSlotsK, u);
-    nk += ok;
-    return ok;
-  };
-  auto load_v = [&](int u) {
-    const bool ok = load(tmV, sV, bars->v_full, bars->pv_done, C::kSlotsV, u);
-    nv += ok;
-    return ok;
-  };
-  // in order of need: K(f), K(f+1), V(f), then K(f+u+2), V(f+u+1)
-  const int n = l - f + 1;
-  bool ok = load_k(0);
-  if (ok && n > 1) ok = load_k(1);
-  if (ok) ok = load_v(0);
-  for (int u = 0; u + 1 < n && ok; ++u) {
-    if (u + 2 < n) ok = load_k(u + 2);
-    if (ok) ok = load_v(u + 1);
-  }
+  for_each_job(p, [&](const Job& jb) {
+    if (!jb.has || !ok) return;
+    const int n = jb.l - jb.f + 1;
+    // Q of active job a goes to buffer a & 1 once job a - 2 is through QK
+    constexpr int QB = C::kQBufs;
+    if (a >= QB && !(ok = mbar_wait(&bars->q_empty[a % QB], ((a - QB) / QB) & 1, abort))) return;
+    mbar_arrive_expect_tx(&bars->q_full[a % QB], C::kTileBytes);
+#pragma unroll
+    for (int ch = 0; ch < D / 64; ++ch)
+      tma_load_4d(tmQ, &bars->q_full[a % QB], sQ + (a % QB) * C::kTileBytes + ch * C::kChunkBytes, ch * 64, jb.h,
+                  jb.q0, jb.b, pol_q);
+    auto load_k = [&](int u) {
+      const bool r = load(tmK, sK, bars->k_full, bars->s_ready, C::kSlotsK, g + u, jb, jb.f + u);
+      nk += r;
+      return r;
+    };
+    auto load_v = [&](int u) {
+      const bool r = load(tmV, sV, bars->v_full, bars->pv_done, C::kSlotsV, g + u, jb, jb.f + u);
+      nv += r;
+      return r;
+    };
+    // in order of need: K(0), K(1), V(0), then K(u + 2), V(u + 1)
+    ok = load_k(0);
+    if (ok && n > 1) ok = load_k(1);
+    if (ok) ok = load_v(0);
+    for (int u = 0; u + 1 < n && ok; ++u) {
+      if (u + 2 < n) ok = load_k(u + 2);
+      if (ok) ok = load_v(u + 1);
+    }
+    g += n;
+    ++a;
+  });
   // Every load issued must land before the CTA may exit. On the normal path
   // they all have (the MMA threads consumed them); after an abort, wait.
-  drain_wait(&bars->q_full, 0);
+  for (int i = max(0, a - C::kQBufs); i < a; ++i) drain_wait(&bars->q_full[i % C::kQBufs], (i / C::kQBufs) & 1);
   for (int u = max(0, nk - C::kSlotsK); u < nk; ++u) drain_wait(&bars->k_full[u % C::kSlotsK], (u / C::kSlotsK) & 1);
   for (int u = max(0, nv - C::kSlotsV); u < nv; ++u) drain_wait(&bars->v_full[u % C::kSlotsV], (u / C::kSlotsV) & 1);
 }
 
-// S(f+u) = Q K_{f+u}^T into S buffer u & 1: M = 128 query rows, N = 128
-// keys, K = d in steps of 16; both operands K-major, 128-byte swizzled, 64
+// S(g) = Q K_g^T into S buffer g & 1: M = 128 query rows, N = 128 keys,
+// K = d in steps of 16; both operands K-major, 128-byte swizzled, 64
 // elements per 16 KB chunk. Before overwriting the buffer the thread waits
-// for the PV product of tile u - 2: that product waited for P(u - 2), so the
-// softmax is done with S(u - 2), and once it completes P buffer u & 1 is
-// free as well; the commit that publishes S(u) therefore also tells the
-// softmax that it may write P(u).
+// for the PV product of tile g - 2: that product waited for P(g - 2), so the
+// softmax is done with S(g - 2), and once it completes P buffer g & 1 is
+// free as well; the commit that publishes S(g) therefore also tells the
+// softmax that it may write P(g).
 template <typename T, int D>
-__device__ void qk_issuer(uint8_t* sQ, uint8_t* sK, Barriers* bars, uint32_t tmem, int n, bool negate) {
+__device__ void qk_issuer(const FwdParams& p, uint8_t* sQ, uint8_t* sK, Barriers* bars, uint32_t tmem) {
   using C = Cfg<D>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   // a negative softmax scale is applied as -Q K^T (A-negate bit) times |scale|
-  const uint32_t idesc = instr_desc_f16(kBf16, BM, BN, false) | (negate ? (1u << 13) : 0u);
+  const uint32_t idesc = instr_desc_f16(kBf16, BM, BN, false) | (p.negate_scores ? (1u << 13) : 0u);
   volatile int* abort = &bars->abort;
-  // Descriptors are built once per operand tile; stepping K by 16 adds a
-  // byte offset to the start-address field (16-byte units, no carry: shared
-  // addresses are below 2^18).
-  const uint64_t qdesc = smem_desc_sw128(smem_addr(sQ), 16, 1024);
-  const uint32_t sKaddr = smem_addr(sK);
-  bool ok = mbar_wait(&bars->q_full, 0, abort);
-  for (int u = 0; u < n && ok; ++u) {
-    if (u >= 2 && !(ok = mbar_wait(&bars->pv_done[(u - 2) % kRing], ((u - 2) / kRing) & 1, abort))) break;
-    const int slot = u % C::kSlotsK;
-    if (!(ok = mbar_wait(&bars->k_full[slot], (u / C::kSlotsK) & 1, abort))) break;
-    tc_fence_after();
-    const uint32_t d_t = tmem + (u & 1) * 128;
-    const uint64_t kdesc = smem_desc_sw128(sKaddr + slot * C::kTileBytes, 16, 1024);
+  const uint32_t sQaddr = smem_addr(sQ), sKaddr = smem_addr(sK);
+  int g = 0, a = 0;
+  bool ok = true;
+  for_each_job(p, [&](const Job& jb) {
+    if (!jb.has || !ok) return;
+    const int n = jb.l - jb.f + 1;
+    if (!(ok = mbar_wait(&bars->q_full[a % C::kQBufs], (a / C::kQBufs) & 1, abort))) return;
+    // Descriptors are built once per operand tile; stepping K by 16 adds a
+    // byte offset to the start-address field (16-byte units, no carry:
+    // shared addresses are below 2^18).
+    const uint64_t qdesc = smem_desc_sw128(sQaddr + (a % C::kQBufs) * C::kTileBytes, 16, 1024);
+    for (int u = 0; u < n; ++u) {
+      const int gi = g + u;
+      if (gi >= 2 && !(ok = mbar_wait(&bars->pv_done[(gi - 2) % kRing], ((gi - 2) / kRing) & 1, abort))) return;
+      const int slot = gi % C::kSlotsK;
+      if (!(ok = mbar_wait(&bars->k_full[slot], (gi / C::kSlotsK) & 1, abort))) return;
+      tc_fence_after();
+      const uint32_t d_t = tmem + (gi & 1) * 128;
+      const uint64_t kdesc = smem_desc_sw128(sKaddr + slot * C::kTileBytes, 16, 1024);
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t off = ((kk / 4) * C::kChunkBytes + (kk % 4) * 32) >> 4;
-      mma_ss(d_t, qdesc + off, kdesc + off, idesc, kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk / 4) * C::kChunkBytes + (kk % 4) * 32) >> 4;
+        mma_ss(d_t, qdesc + off, kdesc + off, idesc, kk > 0 ? 1u : 0u);
+      }
+      tc_commit(&bars->s_ready[gi % kRing]);
     }
-    tc_commit(&bars->s_ready[u % kRing]);
-  }
+    tc_commit(&bars->q_empty[a % C::kQBufs]);
+    g += n;
+    ++a;
+  });
   // All MMAs of this thread must be complete before TMEM is released.
   tc_commit(&bars->qk_idle);
   drain_wait(&bars->qk_idle, 0);
 }
 
-// O (+)= P(f+u) V_{f+u}: A = P from TMEM (16-bit, two keys per column, P
-// buffer u & 1), B = V tile stored keys x d with d contiguous (MN-major):
-// 16 keys = 2048 bytes, the second 64-wide d chunk lies 16 KB further
-// (leading byte offset).
+// O (+)= P(g) V_g: A = P from TMEM (16-bit, two keys per column, P buffer
+// g & 1), B = V tile stored keys x d with d contiguous (MN-major): 16 keys =
+// 2048 bytes, the second 64-wide d chunk lies 16 KB further (leading byte
+// offset). The first product of a job overwrites O, so it waits until the
+// softmax warps have read O of the previous active job.
 template <typename T, int D>
-__device__ void pv_issuer(uint8_t* sV, Barriers* bars, uint32_t tmem, int n) {
+__device__ void pv_issuer(const FwdParams& p, uint8_t* sV, Barriers* bars, uint32_t tmem) {
   using C = Cfg<D>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t idesc = instr_desc_f16(kBf16, BM, D, true);
   volatile int* abort = &bars->abort;
   const uint32_t sVaddr = smem_addr(sV);
+  int g = 0, a = 0;
   bool ok = true;
-  for (int u = 0; u < n && ok; ++u) {
-    if (!(ok = mbar_wait(&bars->p_full[u & 1], (u >> 1) & 1, abort))) break;
-    const int slot = u % C::kSlotsV;
-    if (!(ok = mbar_wait(&bars->v_full[slot], (u / C::kSlotsV) & 1, abort))) break;
-    tc_fence_after();
-    const uint32_t a_t = tmem + kTmemP + (u & 1) * 64;
-    const uint64_t vdesc = smem_desc_sw128(sVaddr + slot * C::kTileBytes, C::kChunkBytes, 1024);
+  for_each_job(p, [&](const Job& jb) {
+    if (!jb.has || !ok) return;
+    const int n = jb.l - jb.f + 1;
+    if (a >= 1 && !(ok = mbar_wait(&bars->o_free, (a - 1) & 1, abort))) return;
+    for (int u = 0; u < n; ++u) {
+      const int gi = g + u;
+      if (!(ok = mbar_wait(&bars->p_full[gi & 1], (gi >> 1) & 1, abort))) return;
+      const int slot = gi % C::kSlotsV;
+      if (!(ok = mbar_wait(&bars->v_full[slot], (gi / C::kSlotsV) & 1, abort))) return;
+      tc_fence_after();
+      const uint32_t a_t = tmem + kTmemP + (gi & 1) * 64;
+      const uint64_t vdesc = smem_desc_sw128(sVaddr + slot * C::kTileBytes, C::kChunkBytes, 1024);
 #pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk)
-      mma_ts(tmem + kTmemO, a_t + kk * 8, vdesc + ((kk * 2048) >> 4), idesc, (u > 0 || kk > 0) ? 1u : 0u);
-    tc_commit(&bars->pv_done[u % kRing]);
-  }
+      for (int kk = 0; kk < BN / 16; ++kk)
+        mma_ts(tmem + kTmemO, a_t + kk * 8, vdesc + ((kk * 2048) >> 4), idesc, (u > 0 || kk > 0) ? 1u : 0u);
+      tc_commit(&bars->pv_done[gi % kRing]);
+    }
+    g += n;
+    ++a;
+  });
   tc_commit(&bars->pv_idle);
   drain_wait(&bars->pv_idle, 0);
 }
@@ -274,8 +356,8 @@ __device__ __forceinline__ float pair_exchange(float (&xchg)[2][2][BM], int k, i
 }
 
 template <typename T, int D, bool kCap, bool kAlibi>
-__device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem, int b, int h, int q0, bool has,
-                              int f, int l) {
+__device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, const Job& jb, int g, int& xk,
+                            bool& alive) {
   constexpr bool kPlain = !kCap && !kAlibi;
   constexpr int kHalf = BN / 2;       // keys per thread per tile
   constexpr int kOCols = D / 2;       // O columns per thread
@@ -285,6 +367,7 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
   const int quarter = warp & 3;
   const int half = warp >> 2;
   const int r = quarter * 32 + lane;  // row of the tile == TMEM lane
+  const int b = jb.b, h = jb.h, q0 = jb.q0, f = jb.f, l = jb.l;
   const int q = q0 + r;
   const bool row_ok = q < p.Nq;
   const RowRange rr = row_range(p, row_ok ? q : p.Nq - 1);
@@ -301,16 +384,18 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
 
   float m = -INFINITY;  // running max of the whole row (log2 units)
   float lsum = 0.0f;    // this half's running sum of exp2(t - m)
-  bool ok = true;
+  bool ok = alive;      // after a failure in an earlier job, only fill
   bool broke = false;   // left the loop at a shared exchange (both halves do)
-  const int n = has ? l - f + 1 : 0;
+  const int n = jb.has ? l - f + 1 : 0;
+  const int n_run = ok ? n : 0;
   // Each iteration performs exactly one pair exchange, and every early exit
   // happens right after one, on a decision both halves share, so the named
   // barriers can never be left waiting for a partner that has gone.
-  for (int it = 0; it < n; ++it) {
+  for (int it = 0; it < n_run; ++it) {
     const int j = f + it;
-    const uint32_t tS = tmem + lane_sel + (it & 1) * 128;
-    ok = ok && mbar_wait(&bars->s_ready[it % kRing], (it / kRing) & 1, abort);
+    const int gi = g + it;  // tile number across the CTA's jobs
+    const uint32_t tS = tmem + lane_sel + (gi & 1) * 128;
+    ok = ok && mbar_wait(&bars->s_ready[gi % kRing], (gi / kRing) & 1, abort);
     ok = __all_sync(0xffffffffu, ok);
     uint32_t s[2][32];
     const int key0 = j * BN + half * kHalf;
@@ -351,7 +436,7 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
     }
     float mt = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
     // combine with the other half of the row
-    const float mo = pair_exchange(bars->xchg, it, half, r, quarter, ok ? mt : __int_as_float(0x7fc00000));
+    const float mo = pair_exchange(bars->xchg, xk++, half, r, quarter, ok ? mt : __int_as_float(0x7fc00000));
     ok = __all_sync(0xffffffffu, ok && mo == mo);
     if (!ok) {  // both halves of every row of this warp pair see the same NaN
       broke = true;
@@ -381,7 +466,7 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
     uint64_t rsum2[4] = {0, 0, 0, 0};  // independent packed partial sums (0 bits = +0.0f)
     uint32_t pk[32];
     auto pass2 = [&](auto emu_tag) {
-      constexpr bool kEmu = decltype(emu_tag)::value;
+      constexpr bool kMaskedTile = decltype(emu_tag)::value;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
 #pragma unroll
@@ -390,7 +475,7 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
           const float x1 = __uint_as_float(s[c][2 * e + 1]);
           const uint64_t a2 = f2_fma(f2_pack(x0, x1), mul2, m2);
           float p0, p1;
-          if (kEmu && (e & 7) >= 5) {
+          if ((e & 7) >= 5) {
             // three pairs in eight take exp2 on the FMA pipe, so the MUFU is
             // not the only unit doing exponentials
             f2_unpack(ex2_poly_x2(a2), p0, p1);
@@ -400,8 +485,9 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
             p0 = ex2(a0);
             p1 = ex2(a1);
           }
-          if (kPlain && !kEmu) {
-            // masked entries hold -inf; -inf * 0 would be NaN, so select them out
+          if (kMaskedTile) {
+            // masked entries hold -inf: the polynomial path would give a
+            // tiny nonzero value and -inf * 0 a NaN, so select them out
             p0 = (x0 == -INFINITY) ? 0.0f : p0;
             p1 = (x1 == -INFINITY) ? 0.0f : p1;
           }
@@ -411,10 +497,10 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
       }
     };
     if (masked)
-      pass2(std::false_type{});
-    else
       pass2(std::true_type{});
-    tmem_st32(tmem + lane_sel + kTmemP + (it & 1) * 64 + half * 32, pk);
+    else
+      pass2(std::false_type{});
+    tmem_st32(tmem + lane_sel + kTmemP + (gi & 1) * 64 + half * 32, pk);
     float r0, r1, r2, r3;
     f2_unpack(f2_add(rsum2[0], rsum2[1]), r0, r1);
     f2_unpack(f2_add(rsum2[2], rsum2[3]), r2, r3);
@@ -424,7 +510,7 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
       // one that can still be running).
       if (it > 0) {
         // on a timeout, carry on to the next exchange, which ends both halves
-        ok = mbar_wait(&bars->pv_done[(it - 1) % kRing], ((it - 1) / kRing) & 1, abort);
+        ok = mbar_wait(&bars->pv_done[(gi - 1) % kRing], ((gi - 1) / kRing) & 1, abort);
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
       }
@@ -443,21 +529,21 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&bars->p_full[it & 1]);
+    if (lane == 0) mbar_arrive(&bars->p_full[gi & 1]);
   }
   // the loop ran the same number of exchanges in both halves: it ended at a
   // shared break, or after all n iterations (possibly with a failed wait in
   // one half, which the final exchange reports to the other)
-  const int n_done = broke ? -1 : n;
+  const int n_done = broke ? -1 : n_run;
   if (ok && n > 0) {
-    ok = mbar_wait(&bars->pv_done[(n - 1) % kRing], ((n - 1) / kRing) & 1, abort);
+    ok = mbar_wait(&bars->pv_done[(g + n - 1) % kRing], ((g + n - 1) / kRing) & 1, abort);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
   }
   // both halves of a row must agree on success; combine the row sums
   float ltot = lsum;
-  if (n_done >= 0) {
-    const float other = pair_exchange(bars->xchg, n_done, half, r, quarter, ok ? lsum : __int_as_float(0x7fc00000));
+  if (n_done >= 0 && alive) {
+    const float other = pair_exchange(bars->xchg, xk++, half, r, quarter, ok ? lsum : __int_as_float(0x7fc00000));
     ok = ok && other == other;
     ltot = lsum + (other == other ? other : 0.0f);
   }
@@ -484,6 +570,10 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
         for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
     }
+    // O has been read: the next job's first PV product may overwrite it
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars->o_free);
   } else if (row_ok) {
     const float fill = ok ? 0.0f : nan;
     const uint32_t w = pack2<T>(fill, fill);
@@ -498,6 +588,17 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem,
     else lse_v = -INFINITY;
     p.lse[(static_cast<size_t>(b) * p.H + h) * p.Nq + q] = lse_v;
   }
+  alive = alive && ok;
+}
+
+template <typename T, int D, bool kCap, bool kAlibi>
+__device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem) {
+  int g = 0, xk = 0;
+  bool alive = true;
+  for_each_job(p, [&](const Job& jb) {
+    softmax_job<T, D, kCap, kAlibi>(p, bars, tmem, jb, g, xk, alive);
+    if (jb.has) g += jb.l - jb.f + 1;
+  });
 }
 
 template <typename T, int D, bool kCap, bool kAlibi>
@@ -507,38 +608,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + C::kTileBytes;
+  uint8_t* sQ = smem;  // two Q buffers
+  uint8_t* sK = smem + C::kQBufs * C::kTileBytes;
   uint8_t* sV = sK + C::kSlotsK * C::kTileBytes;
   Barriers* bars = reinterpret_cast<Barriers*>(sV + C::kSlotsV * C::kTileBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // 1-D grid, the Q tiles of one (b, h) adjacent so they share K/V in L2;
-  // within a head the longest causal work is dispatched first.
-  const int bh = static_cast<int>(blockIdx.x) / p.num_tiles;
-  const int tile = p.num_tiles - 1 - static_cast<int>(blockIdx.x) % p.num_tiles;
-  const int b = bh / p.H, h = bh % p.H;
-  const int q0 = tile * BM;
-
-  // K/V tile range of the Q tile (rows' visible intervals are monotone in q)
-  const int qz = min(q0 + BM - 1, p.Nq - 1);
-  const RowRange ra = row_range(p, q0), rz = row_range(p, qz);
-  const bool has = ra.lo <= rz.hi;
-  const int f = has ? ra.lo / BN : 0;
-  const int l = has ? rz.hi / BN : -1;
-
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    for (int i = 0; i < C::kSlotsK; ++i) mbar_init(&bars->k_full[i], 1);
-    for (int i = 0; i < C::kSlotsV; ++i) mbar_init(&bars->v_full[i], 1);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->q_full[i], 1);
+      mbar_init(&bars->q_empty[i], 1);
       mbar_init(&bars->p_full[i], kSoftmaxWarps);
     }
+    for (int i = 0; i < C::kSlotsK; ++i) mbar_init(&bars->k_full[i], 1);
+    for (int i = 0; i < C::kSlotsV; ++i) mbar_init(&bars->v_full[i], 1);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&bars->s_ready[i], 1);
       mbar_init(&bars->pv_done[i], 1);
     }
+    mbar_init(&bars->o_free, kSoftmaxWarps);
     mbar_init(&bars->qk_idle, 1);
     mbar_init(&bars->pv_idle, 1);
     bars->abort = 0;
@@ -559,13 +648,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp < kSoftmaxWarps) {
-    softmax_group<T, D, kCap, kAlibi>(p, bars, tmem, b, h, q0, has, f, l);
+    softmax_group<T, D, kCap, kAlibi>(p, bars, tmem);
   } else if (warp == kProducerWarp) {
-    if (lane == 0 && has) producer<T, D>(&tmQ, &tmK, &tmV, sQ, sK, sV, bars, b, h, q0, f, l);
+    if (lane == 0) producer<T, D>(p, &tmQ, &tmK, &tmV, sQ, sK, sV, bars);
   } else if (warp == kQkWarp) {
-    if (lane == 0 && has) qk_issuer<T, D>(sQ, sK, bars, tmem, l - f + 1, p.negate_scores != 0);
-  } else {
-    if (lane == 0 && has) pv_issuer<T, D>(sV, bars, tmem, l - f + 1);
+    if (lane == 0) qk_issuer<T, D>(p, sQ, sK, bars, tmem);
+  } else if (warp == kPvWarp) {
+    if (lane == 0) pv_issuer<T, D>(p, sV, bars, tmem);
   }
 
   tc_fence_before();
@@ -587,7 +676,18 @@ cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtenso
   auto kernel = fwd_kernel<T, D, kCap, kAlibi>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.num_tiles * p.B * p.H);
+  // persistent: one CTA per SM at most (one fits per SM: shared memory, TMEM)
+  static int sm_count[64];
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (sm_count[dev] == 0) {
+    e = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+  }
+  const long long items = static_cast<long long>(p.B) * p.H * ((p.num_tiles + 1) / 2);
+  dim3 grid(static_cast<unsigned>(items < sm_count[dev] ? items : sm_count[dev]));
   kernel<<<grid, kThreads, C::kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
