@@ -74,6 +74,14 @@ def fwd_flops(w: W.FwdWorkload) -> float:
     return 4.0 * w.d * w.B * w.H * unmasked_pairs(w)
 
 
+def varlen_flops(w: W.VarlenWorkload, lens) -> float:
+    """4*d*H*(visible query/key pairs) summed over the packed sequences
+    (query and key lengths equal; causal: n(n+1)/2 pairs)."""
+    n = np.asarray(lens, dtype=np.int64)
+    pairs = n * (n + 1) // 2 if w.causal else n * n
+    return 4.0 * w.d * w.H * float(pairs.sum())
+
+
 def decode_kv_bytes(w: W.DecodeWorkload, seqlens: torch.Tensor) -> float:
     L = seqlens.to(torch.int64)
     if w.window_left >= 0:
@@ -524,6 +532,33 @@ def sweep(args):
                           "frac_burst": round(tf / peaks["bf16_tflops"], 4),
                           "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
                           "flops": fwd_flops(w), "peak_source": peak_src, "l2": "flushed"}), flush=True)
+        del x, out, lse
+    vw = W.VARLEN
+    if not args.workloads or vw.name in names:
+        x = W.make_varlen_inputs(vw, device=dev)
+        out = torch.empty_like(x["q"])
+        lse = torch.empty((vw.H, x["q"].shape[0]), dtype=torch.float32, device=dev)
+        run = lambda: fa.fa_fwd_varlen(x["q"], x["k"], x["v"], out, lse, x["cu_q"], x["cu_k"], x["max_q"],
+                                       x["max_k"], vw.scale, vw.causal)
+        for _ in range(args.warmup):
+            run()
+        times = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = ev(), ev()
+            a.record()
+            run()
+            b.record()
+            times.append((a, b))
+        torch.cuda.synchronize()
+        ms = statistics.median([a.elapsed_time(b) for a, b in times])
+        fl = varlen_flops(vw, x["lens"])
+        tf = fl / (ms * 1e-3) / 1e12
+        print(json.dumps({"workload": vw.name, "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                          "frac_burst": round(tf / peaks["bf16_tflops"], 4),
+                          "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+                          "flops": fl, "tokens": int(x["lens"].sum()), "peak_source": peak_src,
+                          "l2": "flushed"}), flush=True)
         del x, out, lse
     for dw in W.DECODE_WORKLOADS:
         if (args.workloads and dw.name not in names) or (not args.workloads and dw is not W.DECODE):

@@ -56,6 +56,8 @@ def _lib_handle():
         vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, f, vp]
         L.fa_fwd.restype = i
+        L.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, i, i, vp, f, vp]
+        L.fa_fwd_varlen.restype = i
         L.fa_fwd_kvcache.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp, f, i, vp, sz,
                                      vp]
         L.fa_fwd_kvcache.restype = i
@@ -124,6 +126,33 @@ def fa_fwd(q, k, v, out, lse, scale: float, causal: bool = False, window_left: i
                                 _dtype_code(q), float(scale), int(bool(causal)), int(window_left),
                                 int(window_right), _ptr(alibi_slopes), float(softcap), _stream(stream))
     _check(code, "fa_fwd")
+
+
+def fa_fwd_varlen(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                  scale: float, causal: bool = False, window_left: int = -1, window_right: int = -1,
+                  alibi_slopes=None, softcap: float = 0.0, stream=None) -> None:
+    """Packed sequences: q [total_q,H,d], k/v [total_k,H,d], out like q, lse fp32 [H,total_q];
+    cu_seqlens_q / cu_seqlens_k int32 [B+1] row offsets on the device."""
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    B = cu_seqlens_q.numel() - 1
+    for t in (q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k):
+        if not t.is_contiguous():
+            raise ValueError("fa_fwd_varlen needs contiguous tensors")
+    if tuple(k.shape) != (total_k, H, d) or tuple(v.shape) != (total_k, H, d) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("fa_fwd_varlen: shape mismatch")
+    if tuple(lse.shape) != (H, total_q) or lse.dtype != torch.float32:
+        raise ValueError("fa_fwd_varlen: lse must be fp32 [H, total_q]")
+    if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32 or cu_seqlens_k.numel() != B + 1:
+        raise ValueError("fa_fwd_varlen: cu_seqlens must be int32 [B + 1]")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype):
+        raise ValueError("fa_fwd_varlen: q, k, v, out must share one dtype")
+    code = _lib_handle().fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
+                                       _ptr(cu_seqlens_k), B, H, int(max_seqlen_q), int(max_seqlen_k), total_q,
+                                       total_k, d, _dtype_code(q), float(scale), int(bool(causal)),
+                                       int(window_left), int(window_right), _ptr(alibi_slopes), float(softcap),
+                                       _stream(stream))
+    _check(code, "fa_fwd_varlen")
 
 
 def fa_kvcache_num_splits(B: int, H: int, d: int, max_blocks: int, page_size: int, num_splits: int = 0) -> int:

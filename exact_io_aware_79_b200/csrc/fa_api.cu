@@ -123,6 +123,74 @@ bool kvcache_sizes_ok(int B, int H, int d, int max_blocks, int page_size) {
 
 }  // namespace
 
+namespace {
+
+// Shared body of fa_fwd and fa_fwd_varlen. Fixed length: cu_q == nullptr, the
+// maps cover [B, N, H, d]. Variable length: the maps cover one batch of
+// total rows and Nq, Nk are the maximum lengths.
+fa_status fwd_common(const void* q, const void* k, const void* v, void* out, float* lse, const int* cu_q,
+                     const int* cu_k, int B, int H, int Nq, int Nk, int total_q, int total_k, int d, fa_dtype dtype,
+                     float scale, int causal, int window_left, int window_right, const float* alibi_slopes,
+                     float softcap, cudaStream_t stream) {
+  const bool varlen = cu_q != nullptr;
+  if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || total_q < 0 || total_k < 0) return FA_ERR_SHAPE;
+  if (Nq > kMaxSeq || Nk > kMaxSeq || total_q > kMaxSeq || total_k > kMaxSeq ||
+      static_cast<long long>(B) * H >= (1LL << 31))
+    return FA_ERR_SHAPE;
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  if (!finite(scale) || !finite(softcap) || softcap < 0.0f) return FA_ERR_ARG;
+  if (window_left < -1 || window_right < -1 || (causal != 0 && causal != 1)) return FA_ERR_ARG;
+  if (static_cast<long long>(B) * H * Nq == 0 || (varlen && total_q == 0)) return FA_OK;
+  if (!q || !out || !lse) return FA_ERR_NULL;
+  const bool any_k = varlen ? total_k > 0 : Nk > 0;
+  if (any_k && (!k || !v)) return FA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k) || !aligned16(v) || !aligned16(lse)) return FA_ERR_ARG;
+  const int tiles = (Nq + 127) / 128;
+  if (static_cast<long long>(tiles) * B * H >= (1LL << 31)) return FA_ERR_SHAPE;
+  fa_status st = check_device();
+  if (st != FA_OK) return st;
+
+  const bool bf16 = dtype == FA_BF16;
+  CUtensorMap tq, tk, tv;
+  // With no keys no K/V tile is ever loaded; q stands in as a valid base.
+  const void* kb = any_k ? k : q;
+  const void* vb = any_k ? v : q;
+  const int mb = varlen ? 1 : B;
+  const int nq = varlen ? total_q : Nq, nk = varlen ? total_k : Nk;
+  if (!make_map(&tq, q, bf16, mb, nq, H, d) || !make_map(&tk, kb, bf16, mb, nk, H, d) ||
+      !make_map(&tv, vb, bf16, mb, nk, H, d))
+    return FA_ERR_CUDA;
+
+  fa::FwdParams p{};
+  p.out = out;
+  p.lse = lse;
+  p.slopes = alibi_slopes;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  p.B = B;
+  p.H = H;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.num_tiles = tiles;
+  p.causal = causal;
+  p.window_left = window_left;
+  p.window_right = window_right;
+  p.use_softcap = softcap > 0.0f;
+  // softmax(scale * q.k) with scale < 0 equals softmax(|scale| * (-q).k): the
+  // kernel negates the QK^T product on the tensor core and works with |scale|.
+  p.negate_scores = scale < 0.0f;
+  const float mag = std::fabs(scale);
+  p.scale_log2 = mag * fa::kLog2e;
+  p.cap_scale = softcap > 0.0f ? mag / softcap : 0.0f;
+  p.cap_log2 = softcap * fa::kLog2e;
+  return fa::launch_fwd(bf16, d, tq, tk, tv, p, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* fa_status_string(fa_status s) {
@@ -143,51 +211,18 @@ const char* fa_status_string(fa_status s) {
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int Nq, int Nk,
                  int d, fa_dtype dtype, float scale, int causal, int window_left, int window_right,
                  const float* alibi_slopes, float softcap, cudaStream_t stream) {
-  if (B < 0 || H < 0 || Nq < 0 || Nk < 0) return FA_ERR_SHAPE;
-  if (Nq > kMaxSeq || Nk > kMaxSeq || static_cast<long long>(B) * H >= (1LL << 31)) return FA_ERR_SHAPE;
-  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
-  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
-  if (!finite(scale) || !finite(softcap) || softcap < 0.0f) return FA_ERR_ARG;
-  if (window_left < -1 || window_right < -1 || (causal != 0 && causal != 1)) return FA_ERR_ARG;
-  if (static_cast<long long>(B) * H * Nq == 0) return FA_OK;
-  if (!q || !out || !lse) return FA_ERR_NULL;
-  if (Nk > 0 && (!k || !v)) return FA_ERR_NULL;
-  if (!aligned16(q) || !aligned16(out) || !aligned16(k) || !aligned16(v) || !aligned16(lse)) return FA_ERR_ARG;
-  const int tiles = (Nq + 127) / 128;
-  if (static_cast<long long>(tiles) * B * H >= (1LL << 31)) return FA_ERR_SHAPE;
-  fa_status st = check_device();
-  if (st != FA_OK) return st;
+  return fwd_common(q, k, v, out, lse, nullptr, nullptr, B, H, Nq, Nk, 0, 0, d, dtype, scale, causal, window_left,
+                    window_right, alibi_slopes, softcap, stream);
+}
 
-  const bool bf16 = dtype == FA_BF16;
-  CUtensorMap tq, tk, tv;
-  // With Nk == 0 no K/V tile is ever loaded; q stands in as a valid base.
-  const void* kb = Nk > 0 ? k : q;
-  const void* vb = Nk > 0 ? v : q;
-  if (!make_map(&tq, q, bf16, B, Nq, H, d) || !make_map(&tk, kb, bf16, B, Nk, H, d) ||
-      !make_map(&tv, vb, bf16, B, Nk, H, d))
-    return FA_ERR_CUDA;
-
-  fa::FwdParams p{};
-  p.out = out;
-  p.lse = lse;
-  p.slopes = alibi_slopes;
-  p.B = B;
-  p.H = H;
-  p.Nq = Nq;
-  p.Nk = Nk;
-  p.num_tiles = tiles;
-  p.causal = causal;
-  p.window_left = window_left;
-  p.window_right = window_right;
-  p.use_softcap = softcap > 0.0f;
-  // softmax(scale * q.k) with scale < 0 equals softmax(|scale| * (-q).k): the
-  // kernel negates the QK^T product on the tensor core and works with |scale|.
-  p.negate_scores = scale < 0.0f;
-  const float mag = std::fabs(scale);
-  p.scale_log2 = mag * fa::kLog2e;
-  p.cap_scale = softcap > 0.0f ? mag / softcap : 0.0f;
-  p.cap_log2 = softcap * fa::kLog2e;
-  return fa::launch_fwd(bf16, d, tq, tk, tv, p, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H, int max_seqlen_q,
+                        int max_seqlen_k, int total_q, int total_k, int d, fa_dtype dtype, float scale, int causal,
+                        int window_left, int window_right, const float* alibi_slopes, float softcap,
+                        cudaStream_t stream) {
+  if (B > 0 && (!cu_seqlens_q || !cu_seqlens_k)) return FA_ERR_NULL;
+  return fwd_common(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q,
+                    total_k, d, dtype, scale, causal, window_left, window_right, alibi_slopes, softcap, stream);
 }
 
 int fa_kvcache_num_splits(int B, int H, int d, int max_blocks, int page_size, int num_splits) {

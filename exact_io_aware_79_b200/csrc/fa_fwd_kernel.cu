@@ -113,14 +113,15 @@ struct RowRange {
   int lo, hi;
 };
 
-__device__ __forceinline__ RowRange row_range(const FwdParams& p, int q) {
-  const long long pos = static_cast<long long>(q) + p.Nk - p.Nq;
-  long long lo = 0, hi = static_cast<long long>(p.Nk) - 1;
+// Nq, Nk: the lengths of the query row's sequence.
+__device__ __forceinline__ RowRange row_range(const FwdParams& p, int Nq, int Nk, int q) {
+  const long long pos = static_cast<long long>(q) + Nk - Nq;
+  long long lo = 0, hi = static_cast<long long>(Nk) - 1;
   if (p.window_left >= 0) lo = max(lo, pos - p.window_left);
   if (p.causal) hi = min(hi, pos);
   if (p.window_right >= 0) hi = min(hi, pos + p.window_right);
   RowRange r;
-  r.lo = static_cast<int>(min(lo, static_cast<long long>(p.Nk)));
+  r.lo = static_cast<int>(min(lo, static_cast<long long>(Nk)));
   r.hi = static_cast<int>(max(hi, -1ll));
   return r;
 }
@@ -141,16 +142,49 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 struct Job {
   int b, h, q0, f, l;  // K/V tiles f..l
   bool has;            // at least one visible key
+  int Nq, Nk;          // lengths of the job's sequence
+  int qrow, krow;      // first row of the sequence in the Q and K/V maps
+  int bcoord;          // batch coordinate in the maps
+  long long obase;     // out row of query 0 of the sequence ((obase + q) * H + h)
+  long long lbase;     // LSE index of query 0 of the sequence, head h
 };
 
-__device__ __forceinline__ Job make_job(const FwdParams& p, int bh, int tile) {
+// Lengths and row offsets of sequence b; false if a variable-length table
+// entry is out of its contract (the sequence is then skipped).
+__device__ __forceinline__ bool seq_of(const FwdParams& p, int b, int& Nq, int& Nk, int& qrow, int& krow) {
+  if (p.cu_q == nullptr) {
+    Nq = p.Nq;
+    Nk = p.Nk;
+    qrow = krow = 0;
+    return true;
+  }
+  const int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
+  if (q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 > p.Nq) return false;
+  if (k0 < 0 || k1 < k0 || k1 > p.total_k || k1 - k0 > p.Nk) return false;
+  Nq = q1 - q0;
+  Nk = k1 - k0;
+  qrow = q0;
+  krow = k0;
+  return true;
+}
+
+__device__ __forceinline__ Job make_job(const FwdParams& p, int b, int h, int Nq, int Nk, int qrow, int krow,
+                                        int tile) {
   Job j;
-  j.b = bh / p.H;
-  j.h = bh % p.H;
+  j.b = b;
+  j.h = h;
   j.q0 = tile * BM;
+  j.Nq = Nq;
+  j.Nk = Nk;
+  j.qrow = qrow;
+  j.krow = krow;
+  const bool varlen = p.cu_q != nullptr;
+  j.bcoord = varlen ? 0 : b;
+  j.obase = varlen ? static_cast<long long>(qrow) : static_cast<long long>(b) * Nq;
+  j.lbase = varlen ? static_cast<long long>(h) * p.total_q + qrow : (static_cast<long long>(b) * p.H + h) * Nq;
   // K/V tile range of the Q tile (rows' visible intervals are monotone in q)
-  const int qz = min(j.q0 + BM - 1, p.Nq - 1);
-  const RowRange ra = row_range(p, j.q0), rz = row_range(p, qz);
+  const int qz = min(j.q0 + BM - 1, Nq - 1);
+  const RowRange ra = row_range(p, Nq, Nk, j.q0), rz = row_range(p, Nq, Nk, qz);
   j.has = ra.lo <= rz.hi;
   j.f = j.has ? ra.lo / BN : 0;
   j.l = j.has ? rz.hi / BN : -1;
@@ -164,9 +198,14 @@ __device__ __forceinline__ void for_each_job(const FwdParams& p, Fn&& fn) {
   const int items = p.B * p.H * per_head;
   for (int w = static_cast<int>(blockIdx.x); w < items; w += static_cast<int>(gridDim.x)) {
     const int bh = w / per_head, pi = w % per_head;
-    const int t_long = p.num_tiles - 1 - pi;
-    fn(make_job(p, bh, t_long));
-    if (pi != t_long) fn(make_job(p, bh, pi));
+    const int b = bh / p.H, h = bh % p.H;
+    int Nq, Nk, qrow, krow;
+    if (!seq_of(p, b, Nq, Nk, qrow, krow)) continue;
+    const int tiles = (Nq + BM - 1) / BM;  // of this sequence (<= num_tiles)
+    if (pi >= (tiles + 1) / 2) continue;
+    const int t_long = tiles - 1 - pi;
+    fn(make_job(p, b, h, Nq, Nk, qrow, krow, t_long));
+    if (pi != t_long) fn(make_job(p, b, h, Nq, Nk, qrow, krow, pi));
   }
 }
 
@@ -190,7 +229,7 @@ __device__ void producer(const FwdParams& p, const CUtensorMap* tmQ, const CUten
 #pragma unroll
     for (int ch = 0; ch < D / 64; ++ch)
       tma_load_4d(map, &full[slot], ring + slot * C::kTileBytes + ch * C::kChunkBytes, ch * 64, jb.h,
-                  key_tile * BN, jb.b, pol_kv);
+                  jb.krow + key_tile * BN, jb.bcoord, pol_kv);
     return true;
   };
   for_each_job(p, [&](const Job& jb) {
@@ -203,7 +242,7 @@ __device__ void producer(const FwdParams& p, const CUtensorMap* tmQ, const CUten
 #pragma unroll
     for (int ch = 0; ch < D / 64; ++ch)
       tma_load_4d(tmQ, &bars->q_full[a % QB], sQ + (a % QB) * C::kTileBytes + ch * C::kChunkBytes, ch * 64, jb.h,
-                  jb.q0, jb.b, pol_q);
+                  jb.qrow + jb.q0, jb.bcoord, pol_q);
     auto load_k = [&](int u) {
       const bool r = load(tmK, sK, bars->k_full, bars->s_ready, C::kSlotsK, g + u, jb, jb.f + u);
       nk += r;
@@ -367,15 +406,15 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
   const int quarter = warp & 3;
   const int half = warp >> 2;
   const int r = quarter * 32 + lane;  // row of the tile == TMEM lane
-  const int b = jb.b, h = jb.h, q0 = jb.q0, f = jb.f, l = jb.l;
+  const int h = jb.h, q0 = jb.q0, f = jb.f, l = jb.l;
   const int q = q0 + r;
-  const bool row_ok = q < p.Nq;
-  const RowRange rr = row_range(p, row_ok ? q : p.Nq - 1);
+  const bool row_ok = q < jb.Nq;
+  const RowRange rr = row_range(p, jb.Nq, jb.Nk, row_ok ? q : jb.Nq - 1);
   // tile-level bounds: a K tile needs no mask when every row of the tile
   // sees all of it (rows' intervals are monotone in q)
-  const int qz = min(q0 + BM - 1, p.Nq - 1);
-  const RowRange first_row = row_range(p, q0), last_row = row_range(p, qz);
-  const int pos = q + p.Nk - p.Nq;
+  const int qz = min(q0 + BM - 1, jb.Nq - 1);
+  const RowRange first_row = row_range(p, jb.Nq, jb.Nk, q0), last_row = row_range(p, jb.Nq, jb.Nk, qz);
+  const int pos = q + jb.Nk - jb.Nq;
   const uint32_t lane_sel = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t tO = tmem + lane_sel + kTmemO + half * kOCols;
   const float slope_l2 = kAlibi ? p.slopes[h] * kLog2e : 0.0f;
@@ -549,7 +588,7 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
   }
 
   // epilogue: O / l -> dtype for this half's columns, LSE = (m + log2 l) ln 2
-  T* orow = reinterpret_cast<T*>(p.out) + ((static_cast<size_t>(b) * p.Nq + (row_ok ? q : 0)) * p.H + h) * D +
+  T* orow = reinterpret_cast<T*>(p.out) + ((jb.obase + (row_ok ? q : 0)) * p.H + h) * D +
             half * kOCols;
   const float inv = ltot > 0.0f ? 1.0f / ltot : 0.0f;
   const float nan = __int_as_float(0x7fc00000);
@@ -586,7 +625,7 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
     if (!ok) lse_v = nan;
     else if (ltot > 0.0f) lse_v = (m + lg2(ltot)) * kLn2;
     else lse_v = -INFINITY;
-    p.lse[(static_cast<size_t>(b) * p.H + h) * p.Nq + q] = lse_v;
+    p.lse[jb.lbase + q] = lse_v;
   }
   alive = alive && ok;
 }

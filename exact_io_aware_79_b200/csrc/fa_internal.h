@@ -12,11 +12,19 @@ namespace fa {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// Forward: one CTA owns one 128-row query tile of one (b, h).
+// Forward: a persistent grid; a job is one 128-row query tile of one (b, h).
+// Fixed length: Q/out [B, Nq, H, d], K/V [B, Nk, H, d], LSE [B, H, Nq].
+// Variable length (cu_q != nullptr): Q/out [total_q, H, d], K/V
+// [total_k, H, d], LSE [H, total_q]; sequence b owns rows
+// cu_q[b] .. cu_q[b+1]-1 and cu_k[b] .. cu_k[b+1]-1, and Nq, Nk are the
+// maximum lengths.
 struct FwdParams {
-  void* out;            // [B, Nq, H, d]
-  float* lse;           // [B, H, Nq]
+  void* out;
+  float* lse;
   const float* slopes;  // [H] or nullptr
+  const int* cu_q;      // [B + 1] or nullptr (fixed length)
+  const int* cu_k;      // [B + 1] or nullptr
+  int total_q, total_k; // variable length: rows of Q and K/V
   int B, H, Nq, Nk;
   int num_tiles;        // ceil(Nq / 128)
   int causal;

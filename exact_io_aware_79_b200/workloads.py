@@ -102,6 +102,30 @@ DECODE = DecodeWorkload("paged_decode_bf16_b64h32d128_page256", 64, 32, 128, tor
 DECODE_SMALL = DecodeWorkload("paged_decode_bf16_b4h32d128_page256", 4, 32, 128, torch.bfloat16,
                               page_size=256, len_lo=1024, len_hi=32768, seed=4)
 
+@dataclasses.dataclass(frozen=True)
+class VarlenWorkload:
+    """Packed sequences: B sequences with query and key lengths drawn
+    uniformly from [len_lo, len_hi] (the same length for q and k)."""
+    name: str
+    B: int
+    H: int
+    d: int
+    dtype: torch.dtype
+    len_lo: int
+    len_hi: int
+    causal: bool = True
+    sigma: float = 1.0
+    seed: int = 5
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+# Variable-length forward: 16 packed causal sequences of 256..4096 tokens
+# (a training batch of documents of mixed length).
+VARLEN = VarlenWorkload("varlen_causal_bf16_b16h16n256-4096d128", 16, 16, 128, torch.bfloat16, 256, 4096)
+
 FWD_WORKLOADS = [TINY, CAUSAL_2K, WINDOW_16K, WINDOW_Q4K_K16K, CAUSAL_Q4K_K16K, ALIBI_SOFTCAP]
 DECODE_WORKLOADS = [DECODE, DECODE_SMALL]
 
@@ -146,6 +170,25 @@ def make_fwd_inputs(w: FwdWorkload, device="cpu", seed: Optional[int] = None):
     out = dict(q=q.to(device), k=k.to(device), v=v.to(device),
                slopes=None if slopes is None else slopes.to(device))
     return out
+
+
+def make_varlen_inputs(w: VarlenWorkload, device="cpu", seed: Optional[int] = None):
+    """Returns dict(q, k, v, cu_q, cu_k, max_q, max_k, lens).
+
+    q, k, v are [total, H, d] (``w.dtype``); cu_q = cu_k are int32 [B + 1]
+    row offsets; lens the B lengths (int64, CPU).
+    """
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(w.seed if seed is None else seed)
+    lens = torch.randint(w.len_lo, w.len_hi + 1, (w.B,), generator=gen, dtype=torch.int64)
+    cu = torch.zeros(w.B + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(lens, 0).to(torch.int32)
+    total = int(cu[-1])
+    q = _normal((total, w.H, w.d), gen, w.sigma, w.dtype, "cpu")
+    k = _normal((total, w.H, w.d), gen, w.sigma, w.dtype, "cpu")
+    v = _normal((total, w.H, w.d), gen, w.sigma, w.dtype, "cpu")
+    return dict(q=q.to(device), k=k.to(device), v=v.to(device), cu_q=cu.to(device), cu_k=cu.clone().to(device),
+                max_q=int(lens.max()), max_k=int(lens.max()), lens=lens)
 
 
 def make_decode_inputs(w: DecodeWorkload, device="cpu", seed: Optional[int] = None,

@@ -90,13 +90,48 @@ typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
  *   alibi_slopes         [H] fp32 device array, or NULL for no ALiBi
  *   softcap              0 = off, else > 0 and finite
  *
- * Limits: B, H, Nq, Nk >= 0; B*H < 2^31; Nq <= 2^24. B*H*Nq == 0 is a no-op;
- * Nk == 0 makes every row empty. d is 64 or 128. out must not alias q, k or v.
+ * Limits: B, H, Nq, Nk >= 0; B*H < 2^31; Nq, Nk <= 2^28. B*H*Nq == 0 is a
+ * no-op; Nk == 0 makes every row empty. d is 64 or 128. out must not alias
+ * q, k or v.
  */
 fa_status fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
                  int B, int H, int Nq, int Nk, int d, fa_dtype dtype, float scale,
                  int causal, int window_left, int window_right,
                  const float *alibi_slopes, float softcap, cudaStream_t stream);
+
+/*
+ * fa_fwd_varlen -- fa_fwd over a batch of sequences of different lengths
+ * packed along the token axis (the pages' "Flash-Attention v2.0 到 v2.7 更新"
+ * names the variable-length interface beside the fixed-shape one). The
+ * pages give no separate formula: each sequence b is attended exactly as
+ * fa_fwd would attend it alone, with its own Nq_b, Nk_b and the same
+ * bottom-right causal alignment, window, ALiBi and softcap rules.
+ *
+ *   q    [total_q, H, d]  fp16/bf16, read; sequence b owns rows
+ *                         cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1
+ *   k, v [total_k, H, d]  fp16/bf16, read; rows cu_seqlens_k[b] ..
+ *   out  [total_q, H, d]  same dtype, written (rows of the sequences only)
+ *   lse  [H, total_q]     fp32, written (natural log)
+ *   cu_seqlens_q, cu_seqlens_k
+ *                         [B + 1] int32 DEVICE arrays of row offsets:
+ *                         nondecreasing, [0] = 0, [B] <= total, and every
+ *                         length at most max_seqlen_q / max_seqlen_k
+ *   max_seqlen_q, max_seqlen_k  bounds of the lengths (the grid is sized
+ *                         from max_seqlen_q)
+ *   the remaining arguments as in fa_fwd
+ *
+ * The offsets are read on the device only (no synchronisation): a sequence
+ * whose entries break the contract is skipped and its rows are left as
+ * they were; no memory outside the buffers is touched. Limits: B, H >= 0,
+ * total_q, total_k >= 0 and <= 2^28, B*H < 2^31. B*H*max_seqlen_q == 0 or
+ * total_q == 0 is a no-op.
+ */
+fa_status fa_fwd_varlen(const void *q, const void *k, const void *v, void *out, float *lse,
+                        const int *cu_seqlens_q, const int *cu_seqlens_k,
+                        int B, int H, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                        int d, fa_dtype dtype, float scale,
+                        int causal, int window_left, int window_right,
+                        const float *alibi_slopes, float softcap, cudaStream_t stream);
 
 /*
  * fa_fwd_kvcache -- split-KV ("flash-decoding") attention of one new query

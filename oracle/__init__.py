@@ -161,6 +161,45 @@ def attn_fwd(q, k, v, scale: float, causal: bool = False, window_left: int = -1,
     return (o, lse, p) if return_probs else (o, lse)
 
 
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, causal: bool = False,
+                    window_left: int = -1, window_right: int = -1, alibi_slopes=None, softcap: float = 0.0,
+                    num_threads: int = 0, dtype_code: Optional[int] = None):
+    """Packed variable-length attention. q [total_q,H,d], k/v [total_k,H,d];
+    sequence b owns query rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 and
+    key rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1, and is attended on its
+    own by the plain definition (attn_fwd with B = 1 and its own Nq, Nk).
+
+    Returns (o [total_q,H,d], lse [H,total_q]); rows outside every sequence
+    are NaN.
+    """
+    qa, code = _as_storage(q, dtype_code)
+    ka, kc = _as_storage(k, dtype_code)
+    va, vc = _as_storage(v, dtype_code)
+    if not (code == kc == vc):
+        raise ValueError("q, k, v must share one storage type")
+    total_q, H, d = qa.shape
+    total_k = ka.shape[0]
+    if ka.shape != (total_k, H, d) or va.shape != ka.shape:
+        raise ValueError("shape mismatch")
+    cq = [int(x) for x in np.asarray(cu_seqlens_q).reshape(-1)]
+    ck = [int(x) for x in np.asarray(cu_seqlens_k).reshape(-1)]
+    if len(cq) != len(ck) or len(cq) < 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k need B + 1 entries each")
+    o = np.full((total_q, H, d), np.nan)
+    lse = np.full((H, total_q), np.nan)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if not (0 <= q0 <= q1 <= total_q and 0 <= k0 <= k1 <= total_k):
+            raise ValueError("cu_seqlens entry %d out of range" % b)
+        if q1 == q0:
+            continue
+        ob, lb = attn_fwd(qa[q0:q1][None], ka[k0:k1][None], va[k0:k1][None], scale, causal, window_left,
+                          window_right, alibi_slopes, softcap, num_threads=num_threads, dtype_code=code)
+        o[q0:q1] = ob[0]
+        lse[:, q0:q1] = lb[0]
+    return o, lse
+
+
 def attn_decode_paged(q, k_cache, v_cache, block_table, cache_seqlens, scale: float,
                       window_left: int = -1, alibi_slopes=None, softcap: float = 0.0,
                       batch: Optional[Sequence[int]] = None, num_splits: int = 1,

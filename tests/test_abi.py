@@ -34,7 +34,7 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    assert {"fa_fwd", "fa_fwd_kvcache", "fa_kvcache_num_splits", "fa_kvcache_workspace_size",
+    assert {"fa_fwd", "fa_fwd_varlen", "fa_fwd_kvcache", "fa_kvcache_num_splits", "fa_kvcache_workspace_size",
             "fa_status_string"} <= set(names)
 
 
@@ -89,6 +89,36 @@ def test_fwd_reaches_the_device_check_without_gpu(lib):
     if torch.cuda.is_available():
         pytest.skip("a device is present")
     assert fwd(lib) == DEVICE
+
+
+def fwd_varlen(lib, q=P, k=P, v=P, out=P, lse=P, cq=P, ck=P, B=3, H=2, mq=300, mk=300, tq=600, tk=600, d=128,
+               dtype=1, scale=0.1, causal=1, wl=-1, wr=-1, slopes=None, cap=0.0):
+    return lib.fa_fwd_varlen(q, k, v, out, lse, cq, ck, B, H, mq, mk, tq, tk, d, dtype, scale, causal, wl, wr,
+                             slopes, cap, None)
+
+
+def test_fwd_varlen_validation(lib):
+    assert fwd_varlen(lib, d=96) == HEADDIM
+    assert fwd_varlen(lib, dtype=5) == DTYPE
+    assert fwd_varlen(lib, B=-1) == SHAPE
+    assert fwd_varlen(lib, tq=-1) == SHAPE
+    assert fwd_varlen(lib, tk=1 << 29) == SHAPE
+    assert fwd_varlen(lib, mq=-2) == SHAPE
+    assert fwd_varlen(lib, wl=-3) == ARG
+    assert fwd_varlen(lib, cap=-2.0) == ARG
+    assert fwd_varlen(lib, causal=3) == ARG
+    assert fwd_varlen(lib, cq=None) == NULL
+    assert fwd_varlen(lib, ck=None) == NULL
+    assert fwd_varlen(lib, q=None) == NULL
+    assert fwd_varlen(lib, k=None) == NULL
+    assert fwd_varlen(lib, lse=P + 4) == ARG
+    # empty problems are no-ops
+    assert fwd_varlen(lib, B=0, cq=None, ck=None, q=None) == OK
+    assert fwd_varlen(lib, tq=0, q=None, out=None, lse=None) == OK
+    assert fwd_varlen(lib, mq=0) == OK
+    # no keys at all needs no K/V pointers
+    assert fwd_varlen(lib, tk=0, mk=0, k=None, v=None) in (OK, DEVICE)
+    assert fwd_varlen(lib) in (OK, DEVICE)
 
 
 def kv(lib, q=P, kc=P, vc=P, bt=P, sl=P, out=P, lse=P, B=4, H=2, d=128, num_pages=64, page=256, mb=16,

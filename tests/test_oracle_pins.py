@@ -431,3 +431,68 @@ def test_decode_rejects_bad_block_table():
     bad[1, 0] = kc.shape[0]            # page index past the pool
     with pytest.raises(ValueError):
         oracle.attn_decode_paged(q, kc, vc, bad, lens, 0.3)
+
+
+# ------------------------------------------------------------ variable length
+
+def varlen_case(lens_q, lens_k, seed, H=2, d=8):
+    cq = np.concatenate([[0], np.cumsum(lens_q)]).astype(np.int32)
+    ck = np.concatenate([[0], np.cumsum(lens_k)]).astype(np.int32)
+    q = rnd((int(cq[-1]), H, d), seed)
+    k = rnd((int(ck[-1]), H, d), seed + 1)
+    v = rnd((int(ck[-1]), H, d), seed + 2)
+    return q, k, v, cq, ck
+
+
+@pytest.mark.parametrize("opts", [
+    dict(causal=True),
+    dict(),
+    dict(causal=True, window_left=2, window_right=0),
+    dict(alibi_slopes=[0.25, 0.7], softcap=3.0, causal=True),
+])
+def test_varlen_matches_brute_force_per_sequence(opts):
+    # ragged lengths, Nq < Nk, Nq > Nk, a sequence without keys and one
+    # without queries: each sequence is its own bottom-right aligned problem
+    lens_q, lens_k = [3, 5, 0, 4, 2], [6, 2, 3, 4, 0]
+    q, k, v, cq, ck = varlen_case(lens_q, lens_k, 11)
+    o, lse = oracle.attn_fwd_varlen(q, k, v, cq, ck, 0.4, **opts)
+    bf = dict(causal=opts.get("causal", False), wl=opts.get("window_left", -1), wr=opts.get("window_right", -1),
+              slopes=opts.get("alibi_slopes"), softcap=opts.get("softcap", 0.0))
+    for b in range(len(lens_q)):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 == q0:
+            continue
+        ob, lb = brute_force(q[q0:q1][None], k[k0:k1][None], v[k0:k1][None], 0.4, **bf)
+        np.testing.assert_allclose(o[q0:q1], ob[0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[:, q0:q1], lb[0], rtol=0, atol=1e-12)
+
+
+def test_varlen_equal_lengths_is_the_batched_problem():
+    B, N, H, d = 3, 7, 2, 8
+    q, k, v = rnd((B, N, H, d), 21), rnd((B, N + 2, H, d), 22), rnd((B, N + 2, H, d), 23)
+    o, lse = oracle.attn_fwd(q, k, v, 0.3, causal=True)
+    cq = np.arange(B + 1, dtype=np.int32) * N
+    ck = np.arange(B + 1, dtype=np.int32) * (N + 2)
+    ov, lv = oracle.attn_fwd_varlen(q.reshape(B * N, H, d), k.reshape(B * (N + 2), H, d),
+                                    v.reshape(B * (N + 2), H, d), cq, ck, 0.3, causal=True)
+    assert np.array_equal(ov, o.reshape(B * N, H, d))
+    assert np.array_equal(lv, lse.transpose(1, 0, 2).reshape(H, B * N))
+
+
+def test_varlen_sequences_do_not_see_each_other():
+    q, k, v, cq, ck = varlen_case([4, 3], [5, 6], 31)
+    o1, l1 = oracle.attn_fwd_varlen(q, k, v, cq, ck, 0.5)
+    k2, v2 = k.copy(), v.copy()
+    k2[ck[1]:] += 1.0
+    v2[ck[1]:] -= 2.0
+    o2, l2 = oracle.attn_fwd_varlen(q, k2, v2, cq, ck, 0.5)
+    assert np.array_equal(o1[:cq[1]], o2[:cq[1]]) and np.array_equal(l1[:, :cq[1]], l2[:, :cq[1]])
+    assert not np.allclose(o1[cq[1]:], o2[cq[1]:])
+
+
+def test_varlen_rows_outside_every_sequence_are_nan():
+    q, k, v, cq, ck = varlen_case([2, 3], [2, 3], 41)
+    q = np.concatenate([q, rnd((2,) + q.shape[1:], 42)])  # two trailing rows no sequence owns
+    o, lse = oracle.attn_fwd_varlen(q, k, v, cq, ck, 0.5)
+    assert np.isnan(o[-2:]).all() and np.isnan(lse[:, -2:]).all()
+    assert not np.isnan(o[:-2]).any()
