@@ -86,7 +86,7 @@ def decode_kv_bytes(w: W.DecodeWorkload, seqlens: torch.Tensor) -> float:
     L = seqlens.to(torch.int64)
     if w.window_left >= 0:
         L = torch.clamp(L, max=w.window_left + 1)
-    return 2.0 * 2.0 * w.H * w.d * float(L.sum())
+    return 2.0 * 2.0 * w.kv_heads * w.d * float(L.sum())
 
 
 def load_peaks():
@@ -570,8 +570,9 @@ def sweep(args):
         for s in [int(x) for x in args.splits.split(",")]:
             nb = fa.fa_kvcache_workspace_size(dw.B, dw.H, dw.d, dw.max_blocks, dw.page_size, s)
             ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
-            run = lambda: fa.fa_fwd_kvcache(xd["q"], xd["k_cache"], xd["v_cache"], xd["block_table"],
-                                            xd["cache_seqlens"], d_out, d_lse, dw.scale, -1, None, 0.0, s, ws)
+            dec = fa.fa_fwd_kvcache_gqa if dw.kv_heads != dw.H else fa.fa_fwd_kvcache
+            run = lambda: dec(xd["q"], xd["k_cache"], xd["v_cache"], xd["block_table"], xd["cache_seqlens"], d_out,
+                              d_lse, dw.scale, -1, None, 0.0, s, ws)
             for _ in range(args.warmup):
                 run()
             times = []

@@ -56,6 +56,13 @@ def _lib_handle():
         vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, f, vp]
         L.fa_fwd.restype = i
+        L.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i, vp, f, vp]
+        L.fa_fwd_gqa.restype = i
+        L.fa_fwd_kvcache_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, vp, f, i, vp,
+                                         sz, vp]
+        L.fa_fwd_kvcache_gqa.restype = i
+        L.fa_kvcache_append.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp]
+        L.fa_kvcache_append.restype = i
         L.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, i, i, vp, f, vp]
         L.fa_fwd_varlen.restype = i
         L.fa_fwd_kvcache.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp, f, i, vp, sz,
@@ -128,6 +135,28 @@ def fa_fwd(q, k, v, out, lse, scale: float, causal: bool = False, window_left: i
     _check(code, "fa_fwd")
 
 
+def fa_fwd_gqa(q, k, v, out, lse, scale: float, causal: bool = False, window_left: int = -1,
+               window_right: int = -1, alibi_slopes=None, softcap: float = 0.0, stream=None) -> None:
+    """Grouped-query forward: q [B,Nq,H,d], k/v [B,Nk,H_kv,d] with H % H_kv == 0; out like q;
+    lse fp32 [B,H,Nq]."""
+    B, Nq, H, d = q.shape
+    Nk, H_kv = k.shape[1], k.shape[2]
+    for t in (q, k, v, out, lse):
+        if not t.is_contiguous():
+            raise ValueError("fa_fwd_gqa needs contiguous tensors")
+    if tuple(k.shape) != (B, Nk, H_kv, d) or tuple(v.shape) != (B, Nk, H_kv, d) or \
+            tuple(out.shape) != tuple(q.shape):
+        raise ValueError("fa_fwd_gqa: shape mismatch")
+    if tuple(lse.shape) != (B, H, Nq) or lse.dtype != torch.float32:
+        raise ValueError("fa_fwd_gqa: lse must be fp32 [B, H, Nq]")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype):
+        raise ValueError("fa_fwd_gqa: q, k, v, out must share one dtype")
+    code = _lib_handle().fa_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, H_kv, Nq, Nk, d,
+                                    _dtype_code(q), float(scale), int(bool(causal)), int(window_left),
+                                    int(window_right), _ptr(alibi_slopes), float(softcap), _stream(stream))
+    _check(code, "fa_fwd_gqa")
+
+
 def fa_fwd_varlen(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
                   scale: float, causal: bool = False, window_left: int = -1, window_right: int = -1,
                   alibi_slopes=None, softcap: float = 0.0, stream=None) -> None:
@@ -188,6 +217,54 @@ def fa_fwd_kvcache(q, k_cache, v_cache, block_table, cache_seqlens, out, lse, sc
         B, H, d, num_pages, page_size, max_blocks, _dtype_code(q), float(scale), int(window_left),
         _ptr(alibi_slopes), float(softcap), int(num_splits), _ptr(workspace), ws_bytes, _stream(stream))
     _check(code, "fa_fwd_kvcache")
+
+
+def fa_fwd_kvcache_gqa(q, k_cache, v_cache, block_table, cache_seqlens, out, lse, scale: float,
+                       window_left: int = -1, alibi_slopes=None, softcap: float = 0.0, num_splits: int = 0,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Grouped-query decode: q [B,1,H,d]; caches [num_pages,page_size,H_kv,d] with H % H_kv == 0;
+    the rest as fa_fwd_kvcache (the workspace size is that of H query heads)."""
+    B, one, H, d = q.shape
+    num_pages, page_size, H_kv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    max_blocks = block_table.shape[1]
+    for t in (q, k_cache, v_cache, block_table, cache_seqlens, out, lse):
+        if not t.is_contiguous():
+            raise ValueError("fa_fwd_kvcache_gqa needs contiguous tensors")
+    if one != 1 or tuple(k_cache.shape) != (num_pages, page_size, H_kv, d) or \
+            tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("fa_fwd_kvcache_gqa: shape mismatch")
+    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32 or block_table.shape[0] != B:
+        raise ValueError("fa_fwd_kvcache_gqa: block_table / cache_seqlens must be int32 [B, ...]")
+    if tuple(lse.shape) != (B, H, 1) or lse.dtype != torch.float32:
+        raise ValueError("fa_fwd_kvcache_gqa: lse must be fp32 [B, H, 1]")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = _lib_handle().fa_fwd_kvcache_gqa(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(cache_seqlens), _ptr(out), _ptr(lse),
+        B, H, H_kv, d, num_pages, page_size, max_blocks, _dtype_code(q), float(scale), int(window_left),
+        _ptr(alibi_slopes), float(softcap), int(num_splits), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(code, "fa_fwd_kvcache_gqa")
+
+
+def fa_kvcache_append(k_new, v_new, k_cache, v_cache, block_table, cache_seqlens, stream=None) -> None:
+    """Writes k_new/v_new [B,n_new,H_kv,d] into the paged caches [num_pages,page_size,H_kv,d] at
+    positions cache_seqlens[b] .. + n_new - 1 (cache_seqlens is not advanced)."""
+    B, n_new, H_kv, d = k_new.shape
+    num_pages, page_size = k_cache.shape[0], k_cache.shape[1]
+    max_blocks = block_table.shape[1]
+    for t in (k_new, v_new, k_cache, v_cache, block_table, cache_seqlens):
+        if not t.is_contiguous():
+            raise ValueError("fa_kvcache_append needs contiguous tensors")
+    if tuple(v_new.shape) != tuple(k_new.shape) or tuple(k_cache.shape) != (num_pages, page_size, H_kv, d) or \
+            tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("fa_kvcache_append: shape mismatch")
+    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32 or block_table.shape[0] != B:
+        raise ValueError("fa_kvcache_append: block_table / cache_seqlens must be int32 [B, ...]")
+    if not (k_new.dtype == v_new.dtype == k_cache.dtype == v_cache.dtype):
+        raise ValueError("fa_kvcache_append: k/v and caches must share one dtype")
+    code = _lib_handle().fa_kvcache_append(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                           _ptr(block_table), _ptr(cache_seqlens), B, n_new, H_kv, d, num_pages,
+                                           page_size, max_blocks, _dtype_code(k_new), _stream(stream))
+    _check(code, "fa_kvcache_append")
 
 
 def fa_fwd_kvcache_noalloc(q, k_cache, v_cache, block_table, cache_seqlens, out, lse, scale: float,

@@ -129,11 +129,12 @@ namespace {
 // maps cover [B, N, H, d]. Variable length: the maps cover one batch of
 // total rows and Nq, Nk are the maximum lengths.
 fa_status fwd_common(const void* q, const void* k, const void* v, void* out, float* lse, const int* cu_q,
-                     const int* cu_k, int B, int H, int Nq, int Nk, int total_q, int total_k, int d, fa_dtype dtype,
-                     float scale, int causal, int window_left, int window_right, const float* alibi_slopes,
-                     float softcap, cudaStream_t stream) {
+                     const int* cu_k, int B, int H, int H_kv, int Nq, int Nk, int total_q, int total_k, int d,
+                     fa_dtype dtype, float scale, int causal, int window_left, int window_right,
+                     const float* alibi_slopes, float softcap, cudaStream_t stream) {
   const bool varlen = cu_q != nullptr;
   if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || total_q < 0 || total_k < 0) return FA_ERR_SHAPE;
+  if (H > 0 && (H_kv < 1 || H_kv > H || H % H_kv != 0)) return FA_ERR_SHAPE;
   if (Nq > kMaxSeq || Nk > kMaxSeq || total_q > kMaxSeq || total_k > kMaxSeq ||
       static_cast<long long>(B) * H >= (1LL << 31))
     return FA_ERR_SHAPE;
@@ -158,8 +159,8 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* out, flo
   const void* vb = any_k ? v : q;
   const int mb = varlen ? 1 : B;
   const int nq = varlen ? total_q : Nq, nk = varlen ? total_k : Nk;
-  if (!make_map(&tq, q, bf16, mb, nq, H, d) || !make_map(&tk, kb, bf16, mb, nk, H, d) ||
-      !make_map(&tv, vb, bf16, mb, nk, H, d))
+  if (!make_map(&tq, q, bf16, mb, nq, H, d) || !make_map(&tk, kb, bf16, mb, nk, H_kv, d) ||
+      !make_map(&tv, vb, bf16, mb, nk, H_kv, d))
     return FA_ERR_CUDA;
 
   fa::FwdParams p{};
@@ -172,6 +173,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* out, flo
   p.total_k = total_k;
   p.B = B;
   p.H = H;
+  p.H_kv = H_kv;
   p.Nq = Nq;
   p.Nk = Nk;
   p.num_tiles = tiles;
@@ -191,63 +193,15 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* out, flo
 
 }  // namespace
 
-extern "C" {
+namespace {
 
-const char* fa_status_string(fa_status s) {
-  switch (s) {
-    case FA_OK: return "FA_OK";
-    case FA_ERR_NULL: return "FA_ERR_NULL: a required pointer is NULL";
-    case FA_ERR_SHAPE: return "FA_ERR_SHAPE: a size is out of range";
-    case FA_ERR_DTYPE: return "FA_ERR_DTYPE: dtype must be FA_FP16 or FA_BF16";
-    case FA_ERR_HEADDIM: return "FA_ERR_HEADDIM: head dimension must be 64 or 128";
-    case FA_ERR_ARG: return "FA_ERR_ARG: invalid scalar argument or unaligned pointer";
-    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: split-KV workspace missing, misaligned or too small";
-    case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call or kernel launch failed";
-    case FA_ERR_DEVICE: return "FA_ERR_DEVICE: no CUDA device or the device is not sm_100";
-  }
-  return "unknown fa_status";
-}
-
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int Nq, int Nk,
-                 int d, fa_dtype dtype, float scale, int causal, int window_left, int window_right,
-                 const float* alibi_slopes, float softcap, cudaStream_t stream) {
-  return fwd_common(q, k, v, out, lse, nullptr, nullptr, B, H, Nq, Nk, 0, 0, d, dtype, scale, causal, window_left,
-                    window_right, alibi_slopes, softcap, stream);
-}
-
-fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
-                        const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H, int max_seqlen_q,
-                        int max_seqlen_k, int total_q, int total_k, int d, fa_dtype dtype, float scale, int causal,
-                        int window_left, int window_right, const float* alibi_slopes, float softcap,
-                        cudaStream_t stream) {
-  if (B > 0 && (!cu_seqlens_q || !cu_seqlens_k)) return FA_ERR_NULL;
-  return fwd_common(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, B, H, max_seqlen_q, max_seqlen_k, total_q,
-                    total_k, d, dtype, scale, causal, window_left, window_right, alibi_slopes, softcap, stream);
-}
-
-int fa_kvcache_num_splits(int B, int H, int d, int max_blocks, int page_size, int num_splits) {
-  if (!kvcache_sizes_ok(B, H, d, max_blocks, page_size)) return -1;
-  if (num_splits < 0 || num_splits > FA_MAX_SPLITS) return -1;
-  if (num_splits > 0) return num_splits;
-  if (B == 0) return 1;
-  return auto_splits(B, H, static_cast<long long>(max_blocks) * page_size);
-}
-
-size_t fa_kvcache_workspace_size(int B, int H, int d, int max_blocks, int page_size, int num_splits) {
-  const int s = fa_kvcache_num_splits(B, H, d, max_blocks, page_size, num_splits);
-  if (s <= 1) return 0;
-  const size_t rows = static_cast<size_t>(s) * B * H;
-  size_t o_bytes = rows * d * sizeof(float);
-  o_bytes = (o_bytes + 255) & ~size_t(255);
-  return o_bytes + rows * sizeof(float);
-}
-
-fa_status fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
-                         const int* cache_seqlens, void* out, float* lse, int B, int H, int d, int num_pages,
-                         int page_size, int max_blocks, fa_dtype dtype, float scale, int window_left,
-                         const float* alibi_slopes, float softcap, int num_splits, void* workspace,
-                         size_t workspace_bytes, cudaStream_t stream) {
+fa_status kvcache_common(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                         const int* cache_seqlens, void* out, float* lse, int B, int H, int H_kv, int d,
+                         int num_pages, int page_size, int max_blocks, fa_dtype dtype, float scale,
+                         int window_left, const float* alibi_slopes, float softcap, int num_splits,
+                         void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (B < 0 || H < 1 || num_pages < 1 || max_blocks < 1) return FA_ERR_SHAPE;
+  if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_SHAPE;
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
   if (d != 64 && d != 128) return FA_ERR_HEADDIM;
   if (page_size < 1 || num_splits < 0 || num_splits > FA_MAX_SPLITS) return FA_ERR_ARG;
@@ -282,6 +236,7 @@ fa_status fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache
   p.slopes = alibi_slopes;
   p.B = B;
   p.H = H;
+  p.H_kv = H_kv;
   p.num_pages = num_pages;
   p.page_size = page_size;
   p.max_blocks = max_blocks;
@@ -294,12 +249,126 @@ fa_status fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache
   const bool bf16 = dtype == FA_BF16;
   if (page_size % 64 == 0) {
     CUtensorMap tk, tv;
-    if (!make_cache_map(&tk, k_cache, bf16, num_pages, page_size, H, d) ||
-        !make_cache_map(&tv, v_cache, bf16, num_pages, page_size, H, d))
+    if (!make_cache_map(&tk, k_cache, bf16, num_pages, page_size, H_kv, d) ||
+        !make_cache_map(&tv, v_cache, bf16, num_pages, page_size, H_kv, d))
       return FA_ERR_CUDA;
     return fa::launch_decode(bf16, d, p, &tk, &tv, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
   }
   return fa::launch_decode(bf16, d, p, nullptr, nullptr, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_NULL: return "FA_ERR_NULL: a required pointer is NULL";
+    case FA_ERR_SHAPE: return "FA_ERR_SHAPE: a size is out of range";
+    case FA_ERR_DTYPE: return "FA_ERR_DTYPE: dtype must be FA_FP16 or FA_BF16";
+    case FA_ERR_HEADDIM: return "FA_ERR_HEADDIM: head dimension must be 64 or 128";
+    case FA_ERR_ARG: return "FA_ERR_ARG: invalid scalar argument or unaligned pointer";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: split-KV workspace missing, misaligned or too small";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: a CUDA call or kernel launch failed";
+    case FA_ERR_DEVICE: return "FA_ERR_DEVICE: no CUDA device or the device is not sm_100";
+  }
+  return "unknown fa_status";
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int Nq, int Nk,
+                 int d, fa_dtype dtype, float scale, int causal, int window_left, int window_right,
+                 const float* alibi_slopes, float softcap, cudaStream_t stream) {
+  return fwd_common(q, k, v, out, lse, nullptr, nullptr, B, H, H, Nq, Nk, 0, 0, d, dtype, scale, causal,
+                    window_left, window_right, alibi_slopes, softcap, stream);
+}
+
+fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int H_kv,
+                     int Nq, int Nk, int d, fa_dtype dtype, float scale, int causal, int window_left,
+                     int window_right, const float* alibi_slopes, float softcap, cudaStream_t stream) {
+  return fwd_common(q, k, v, out, lse, nullptr, nullptr, B, H, H_kv, Nq, Nk, 0, 0, d, dtype, scale, causal,
+                    window_left, window_right, alibi_slopes, softcap, stream);
+}
+
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                        const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H, int max_seqlen_q,
+                        int max_seqlen_k, int total_q, int total_k, int d, fa_dtype dtype, float scale, int causal,
+                        int window_left, int window_right, const float* alibi_slopes, float softcap,
+                        cudaStream_t stream) {
+  if (B > 0 && (!cu_seqlens_q || !cu_seqlens_k)) return FA_ERR_NULL;
+  return fwd_common(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, B, H, H, max_seqlen_q, max_seqlen_k, total_q,
+                    total_k, d, dtype, scale, causal, window_left, window_right, alibi_slopes, softcap, stream);
+}
+
+int fa_kvcache_num_splits(int B, int H, int d, int max_blocks, int page_size, int num_splits) {
+  if (!kvcache_sizes_ok(B, H, d, max_blocks, page_size)) return -1;
+  if (num_splits < 0 || num_splits > FA_MAX_SPLITS) return -1;
+  if (num_splits > 0) return num_splits;
+  if (B == 0) return 1;
+  return auto_splits(B, H, static_cast<long long>(max_blocks) * page_size);
+}
+
+size_t fa_kvcache_workspace_size(int B, int H, int d, int max_blocks, int page_size, int num_splits) {
+  const int s = fa_kvcache_num_splits(B, H, d, max_blocks, page_size, num_splits);
+  if (s <= 1) return 0;
+  const size_t rows = static_cast<size_t>(s) * B * H;
+  size_t o_bytes = rows * d * sizeof(float);
+  o_bytes = (o_bytes + 255) & ~size_t(255);
+  return o_bytes + rows * sizeof(float);
+}
+
+fa_status fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                         const int* cache_seqlens, void* out, float* lse, int B, int H, int d, int num_pages,
+                         int page_size, int max_blocks, fa_dtype dtype, float scale, int window_left,
+                         const float* alibi_slopes, float softcap, int num_splits, void* workspace,
+                         size_t workspace_bytes, cudaStream_t stream) {
+  return kvcache_common(q, k_cache, v_cache, block_table, cache_seqlens, out, lse, B, H, H, d, num_pages, page_size,
+                        max_blocks, dtype, scale, window_left, alibi_slopes, softcap, num_splits, workspace,
+                        workspace_bytes, stream);
+}
+
+fa_status fa_fwd_kvcache_gqa(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                             const int* cache_seqlens, void* out, float* lse, int B, int H, int H_kv, int d,
+                             int num_pages, int page_size, int max_blocks, fa_dtype dtype, float scale,
+                             int window_left, const float* alibi_slopes, float softcap, int num_splits,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return kvcache_common(q, k_cache, v_cache, block_table, cache_seqlens, out, lse, B, H, H_kv, d, num_pages,
+                        page_size, max_blocks, dtype, scale, window_left, alibi_slopes, softcap, num_splits,
+                        workspace, workspace_bytes, stream);
+}
+
+fa_status fa_kvcache_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                            const int* block_table, const int* cache_seqlens, int B, int n_new, int H_kv, int d,
+                            int num_pages, int page_size, int max_blocks, fa_dtype dtype, cudaStream_t stream) {
+  if (B < 0 || n_new < 0 || H_kv < 1 || num_pages < 1 || max_blocks < 1) return FA_ERR_SHAPE;
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  if (page_size < 1) return FA_ERR_ARG;
+  if (static_cast<long long>(max_blocks) * page_size >= (1LL << 31) ||
+      static_cast<long long>(B) * n_new * H_kv >= (1LL << 31) || B > 65535)
+    return FA_ERR_SHAPE;
+  if (static_cast<long long>(B) * n_new == 0) return FA_OK;
+  if (!k_new || !v_new || !k_cache || !v_cache || !block_table || !cache_seqlens) return FA_ERR_NULL;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache)) return FA_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u))
+    return FA_ERR_ARG;
+  fa_status st = check_device();
+  if (st != FA_OK) return st;
+  fa::AppendParams p{};
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.block_table = block_table;
+  p.cache_seqlens = cache_seqlens;
+  p.B = B;
+  p.n_new = n_new;
+  p.H_kv = H_kv;
+  p.d = d;
+  p.num_pages = num_pages;
+  p.page_size = page_size;
+  p.max_blocks = max_blocks;
+  return fa::launch_append(p, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // extern "C"

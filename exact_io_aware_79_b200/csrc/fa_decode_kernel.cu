@@ -94,10 +94,11 @@ __global__ void __launch_bounds__(kWarps * 32) decode_split_kernel(const DecodeP
   const bool alibi = p.slopes != nullptr;
   const float slope_l2 = alibi ? p.slopes[h] * kLog2e : 0.0f;
 
-  const size_t tok_stride = static_cast<size_t>(p.H) * D;  // elements
+  const size_t tok_stride = static_cast<size_t>(p.H_kv) * D;  // elements
   const size_t page_stride = static_cast<size_t>(p.page_size) * tok_stride;
-  const T* kbase = reinterpret_cast<const T*>(p.k_cache) + static_cast<size_t>(h) * D + cl * 8;
-  const T* vbase = reinterpret_cast<const T*>(p.v_cache) + static_cast<size_t>(h) * D + cl * 8;
+  const int hk = h / (p.H / p.H_kv);  // cache head of query head h
+  const T* kbase = reinterpret_cast<const T*>(p.k_cache) + static_cast<size_t>(hk) * D + cl * 8;
+  const T* vbase = reinterpret_cast<const T*>(p.v_cache) + static_cast<size_t>(hk) * D + cl * 8;
   const int* bt = p.block_table + static_cast<size_t>(b) * p.max_blocks;
 
   float m = -INFINITY, lsum = 0.0f;
@@ -275,20 +276,25 @@ template <int D>
 struct TmaCfg {
   static constexpr int kStages = (D == 128) ? 3 : 6;
   static constexpr int kTile = kRows * D * 2;  // bytes of one K (or V) stage
-  static constexpr int kSmem = 2 * kStages * kTile + 4096;
+  static constexpr int kShared = 4096 + 3 * kWarps * 4 * D * 4 / 4;  // barrier block, up to 4 heads
+  static constexpr int kSmem = 2 * kStages * kTile + kShared;
 };
 
-template <int D>
+template <int D, int G>
 struct TmaShared {
   uint64_t full[TmaCfg<D>::kStages];
   uint64_t empty[TmaCfg<D>::kStages];
   int bad[TmaCfg<D>::kStages];
   int abort;
-  float m[kWarps], l[kWarps];
-  float acc[kWarps][D];
+  float m[kWarps][G], l[kWarps][G];
+  float acc[kWarps][G][D];
 };
 
-template <typename T, int D>
+// G query heads per CTA (grouped-query attention: heads that share one cache
+// head read its K/V stream once). CTA slot hs of a (sequence, split) serves
+// query heads hs*G .. hs*G + G - 1, which all map to cache head
+// hs*G / (H / H_kv). G = 1 is the plain per-head kernel.
+template <typename T, int D, int G>
 __global__ void __launch_bounds__((kWarps + 1) * 32)
     decode_split_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                             const DecodeParams p) {
@@ -300,12 +306,14 @@ __global__ void __launch_bounds__((kWarps + 1) * 32)
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* sK = smem;
   uint8_t* sV = smem + NST * C::kTile;
-  TmaShared<D>* sh = reinterpret_cast<TmaShared<D>*>(smem + 2 * NST * C::kTile);
+  TmaShared<D, G>* sh = reinterpret_cast<TmaShared<D, G>*>(smem + 2 * NST * C::kTile);
   volatile int* abort = &sh->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.x % p.H;
-  const int s = blockIdx.x / p.H;
+  const int slots = p.H / G;
+  const int h0 = (blockIdx.x % slots) * G;  // first query head of this CTA
+  const int hk = h0 / (p.H / p.H_kv);        // their cache head
+  const int s = blockIdx.x / slots;
   const int b = blockIdx.y;
   const int L_raw = p.cache_seqlens[b];
   const long long max_len = static_cast<long long>(p.max_blocks) * p.page_size;
@@ -346,8 +354,8 @@ __global__ void __launch_bounds__((kWarps + 1) * 32)
         } else {
           sh->bad[slot] = 0;
           mbar_arrive_expect_tx(&sh->full[slot], 2 * C::kTile);
-          tma_load_4d(&tmK, &sh->full[slot], sK + slot * C::kTile, 0, h, a % p.page_size, pg, pol);
-          tma_load_4d(&tmV, &sh->full[slot], sV + slot * C::kTile, 0, h, a % p.page_size, pg, pol);
+          tma_load_4d(&tmK, &sh->full[slot], sK + slot * C::kTile, 0, hk, a % p.page_size, pg, pol);
+          tma_load_4d(&tmV, &sh->full[slot], sV + slot * C::kTile, 0, hk, a % p.page_size, pg, pol);
         }
         issued = i + 1;
       }
@@ -360,19 +368,23 @@ __global__ void __launch_bounds__((kWarps + 1) * 32)
     // ---------------- consumers
     const int g = lane / LPT;
     const int cl = lane % LPT;
-    float qf[8];
-    widen8<T>(*reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.q) +
-                                              (static_cast<size_t>(b) * p.H + h) * D + cl * 8),
-              qf);
     const float qscale = p.use_softcap ? p.cap_scale : p.scale_log2;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) qf[e] *= qscale;
     const bool alibi = p.slopes != nullptr;
-    const float slope_l2 = alibi ? p.slopes[h] * kLog2e : 0.0f;
-    float m = -INFINITY, lsum = 0.0f;
-    float acc[8];
+    float qf[G][8], slope_l2[G];
+    float m[G], lsum[G], acc[G][8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+    for (int gi = 0; gi < G; ++gi) {
+      widen8<T>(*reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.q) +
+                                                (static_cast<size_t>(b) * p.H + h0 + gi) * D + cl * 8),
+                qf[gi]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qf[gi][e] *= qscale;
+      slope_l2[gi] = alibi ? p.slopes[h0 + gi] * kLog2e : 0.0f;
+      m[gi] = -INFINITY;
+      lsum[gi] = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[gi][e] = 0.0f;
+    }
 
     for (int i = 0; i < n_st; ++i) {
       const int slot = i % NST;
@@ -388,41 +400,62 @@ __global__ void __launch_bounds__((kWarps + 1) * 32)
         const T* kt = reinterpret_cast<const T*>(sK + slot * C::kTile);
         const T* vt = reinterpret_cast<const T*>(sV + slot * C::kTile);
         const int a = a0 + i * kRows;
-        float sc[kSteps];
-        float mt = -INFINITY;
+        // scores of every head for this warp's tokens; each K row is
+        // widened once and serves all G heads
+        float sc[G][kSteps];
+        float mt[G];
+#pragma unroll
+        for (int gi = 0; gi < G; ++gi) mt[gi] = -INFINITY;
 #pragma unroll
         for (int st = 0; st < kSteps; ++st) {
           const int r = warp * (kRows / kWarps) + st * TPW + g;
           float kf[8];
           widen8<T>(*reinterpret_cast<const uint4*>(kt + r * D + cl * 8), kf);
-          float dot = 0.0f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) dot = fmaf(qf[e], kf[e], dot);
-#pragma unroll
-          for (int o = LPT / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
           const int tok = a + r;
-          float t = p.use_softcap ? p.cap_log2 * tanh_via_exp2(dot) : dot;
-          if (alibi) t -= slope_l2 * static_cast<float>(pos - tok);
-          sc[st] = (tok >= t0 && tok < t1) ? t : -INFINITY;
-          mt = fmaxf(mt, sc[st]);
-        }
-        const float m_new = fmaxf(m, mt);
-        if (m_new != -INFINITY) {
-          const float alpha = ex2(m - m_new);
-          lsum *= alpha;
+          const bool vis = tok >= t0 && tok < t1;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[e] *= alpha;
+          for (int gi = 0; gi < G; ++gi) {
+            float dot = 0.0f;
 #pragma unroll
-          for (int st = 0; st < kSteps; ++st) {
-            const int r = warp * (kRows / kWarps) + st * TPW + g;
-            const float pu = ex2(sc[st] - m_new);
-            lsum += pu;
-            float vf[8];
-            widen8<T>(*reinterpret_cast<const uint4*>(vt + r * D + cl * 8), vf);
+            for (int e = 0; e < 8; ++e) dot = fmaf(qf[gi][e], kf[e], dot);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = fmaf(pu, vf[e], acc[e]);
+            for (int o = LPT / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+            float t = p.use_softcap ? p.cap_log2 * tanh_via_exp2(dot) : dot;
+            if (alibi) t -= slope_l2[gi] * static_cast<float>(pos - tok);
+            sc[gi][st] = vis ? t : -INFINITY;
+            mt[gi] = fmaxf(mt[gi], sc[gi][st]);
           }
-          m = m_new;
+        }
+        float mn[G], pw[G][kSteps];
+#pragma unroll
+        for (int gi = 0; gi < G; ++gi) {
+          mn[gi] = fmaxf(m[gi], mt[gi]);
+          if (mn[gi] != -INFINITY) {
+            const float alpha = ex2(m[gi] - mn[gi]);
+            lsum[gi] *= alpha;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[gi][e] *= alpha;
+#pragma unroll
+            for (int st = 0; st < kSteps; ++st) {
+              pw[gi][st] = ex2(sc[gi][st] - mn[gi]);
+              lsum[gi] += pw[gi][st];
+            }
+            m[gi] = mn[gi];
+          } else {
+#pragma unroll
+            for (int st = 0; st < kSteps; ++st) pw[gi][st] = 0.0f;
+          }
+        }
+#pragma unroll
+        for (int st = 0; st < kSteps; ++st) {
+          const int r = warp * (kRows / kWarps) + st * TPW + g;
+          float vf[8];
+          widen8<T>(*reinterpret_cast<const uint4*>(vt + r * D + cl * 8), vf);
+#pragma unroll
+          for (int gi = 0; gi < G; ++gi) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[gi][e] = fmaf(pw[gi][st], vf[e], acc[gi][e]);
+          }
         }
       }
       __syncwarp();
@@ -430,67 +463,73 @@ __global__ void __launch_bounds__((kWarps + 1) * 32)
     }
     // merge the lane groups of this warp, then publish the warp's state
 #pragma unroll
-    for (int o = LPT; o < 32; o <<= 1) {
-      const float m_o = __shfl_xor_sync(0xffffffffu, m, o);
-      const float l_o = __shfl_xor_sync(0xffffffffu, lsum, o);
-      const float mm = fmaxf(m, m_o);
-      const float x = (m == -INFINITY) ? 0.0f : ex2(m - mm);
-      const float x_o = (m_o == -INFINITY) ? 0.0f : ex2(m_o - mm);
-      lsum = lsum * x + l_o * x_o;
+    for (int gi = 0; gi < G; ++gi) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float a_o = __shfl_xor_sync(0xffffffffu, acc[e], o);
-        acc[e] = acc[e] * x + a_o * x_o;
+      for (int o = LPT; o < 32; o <<= 1) {
+        const float m_o = __shfl_xor_sync(0xffffffffu, m[gi], o);
+        const float l_o = __shfl_xor_sync(0xffffffffu, lsum[gi], o);
+        const float mm = fmaxf(m[gi], m_o);
+        const float x = (m[gi] == -INFINITY) ? 0.0f : ex2(m[gi] - mm);
+        const float x_o = (m_o == -INFINITY) ? 0.0f : ex2(m_o - mm);
+        lsum[gi] = lsum[gi] * x + l_o * x_o;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float a_o = __shfl_xor_sync(0xffffffffu, acc[gi][e], o);
+          acc[gi][e] = acc[gi][e] * x + a_o * x_o;
+        }
+        m[gi] = mm;
       }
-      m = mm;
-    }
-    if (lane < LPT) {
+      if (lane < LPT) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) sh->acc[warp][cl * 8 + e] = acc[e];
-    }
-    if (lane == 0) {
-      sh->m[warp] = m;
-      sh->l[warp] = lsum;
+        for (int e = 0; e < 8; ++e) sh->acc[warp][gi][cl * 8 + e] = acc[gi][e];
+      }
+      if (lane == 0) {
+        sh->m[warp][gi] = m[gi];
+        sh->l[warp][gi] = lsum[gi];
+      }
     }
   }
   const bool any_bad = __syncthreads_or(bad) != 0;
 
   const int c = threadIdx.x;
   if (c >= D) return;
-  float M = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sh->m[w]);
-  float ltot = 0.0f, oc = 0.0f;
-  if (M != -INFINITY) {
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float x = (sh->m[w] == -INFINITY) ? 0.0f : ex2(sh->m[w] - M);
-      ltot += sh->l[w] * x;
-      oc += sh->acc[w][c] * x;
-    }
-  }
   const float nan = __int_as_float(0x7fc00000);
-  float o_val, lse_val;
-  if (any_bad) {
-    o_val = nan;
-    lse_val = nan;
-  } else if (ltot > 0.0f) {
-    o_val = oc / ltot;
-    lse_val = (M + lg2(ltot)) * kLn2;
-  } else {
-    o_val = 0.0f;
-    lse_val = -INFINITY;
-  }
-  const size_t row = static_cast<size_t>(b) * p.H + h;
-  if (p.num_splits == 1) {
-    T* out = reinterpret_cast<T*>(p.out) + row * D;
-    if constexpr (std::is_same<T, __nv_bfloat16>::value) out[c] = __float2bfloat16_rn(o_val);
-    else out[c] = __float2half_rn(o_val);
-    if (c == 0) p.lse[row] = lse_val;
-  } else {
-    const size_t prow = static_cast<size_t>(s) * p.B * p.H + row;
-    p.o_part[prow * D + c] = o_val;
-    if (c == 0) p.lse_part[prow] = lse_val;
+#pragma unroll
+  for (int gi = 0; gi < G; ++gi) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sh->m[w][gi]);
+    float ltot = 0.0f, oc = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float x = (sh->m[w][gi] == -INFINITY) ? 0.0f : ex2(sh->m[w][gi] - M);
+        ltot += sh->l[w][gi] * x;
+        oc += sh->acc[w][gi][c] * x;
+      }
+    }
+    float o_val, lse_val;
+    if (any_bad) {
+      o_val = nan;
+      lse_val = nan;
+    } else if (ltot > 0.0f) {
+      o_val = oc / ltot;
+      lse_val = (M + lg2(ltot)) * kLn2;
+    } else {
+      o_val = 0.0f;
+      lse_val = -INFINITY;
+    }
+    const size_t row = static_cast<size_t>(b) * p.H + h0 + gi;
+    if (p.num_splits == 1) {
+      T* out = reinterpret_cast<T*>(p.out) + row * D;
+      if constexpr (std::is_same<T, __nv_bfloat16>::value) out[c] = __float2bfloat16_rn(o_val);
+      else out[c] = __float2half_rn(o_val);
+      if (c == 0) p.lse[row] = lse_val;
+    } else {
+      const size_t prow = static_cast<size_t>(s) * p.B * p.H + row;
+      p.o_part[prow * D + c] = o_val;
+      if (c == 0) p.lse_part[prow] = lse_val;
+    }
   }
 }
 
@@ -498,12 +537,23 @@ template <typename T, int D>
 cudaError_t launch(const DecodeParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV, cudaStream_t stream) {
   dim3 grid(p.H * p.num_splits, p.B);
   if (tmK != nullptr) {
-    using C = TmaCfg<D>;
-    static_assert(sizeof(TmaShared<D>) <= 4096, "decode shared block exceeds its reserve");
-    auto kernel = decode_split_tma_kernel<T, D>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    // query heads per CTA: the largest of 4, 2, 1 that divides the group
+    const int group = p.H / p.H_kv;
+    const int G = group % 4 == 0 ? 4 : (group % 2 == 0 ? 2 : 1);
+    auto go = [&](auto g_tag) -> cudaError_t {
+      constexpr int kG = decltype(g_tag)::value;
+      using C = TmaCfg<D>;
+      static_assert(sizeof(TmaShared<D, kG>) <= C::kShared, "decode shared block exceeds its reserve");
+      auto kernel = decode_split_tma_kernel<T, D, kG>;
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+      if (e != cudaSuccess) return e;
+      dim3 g2(p.H / kG * p.num_splits, p.B);
+      kernel<<<g2, (kWarps + 1) * 32, C::kSmem, stream>>>(*tmK, *tmV, p);
+      return cudaSuccess;
+    };
+    cudaError_t e = G == 4 ? go(std::integral_constant<int, 4>{})
+                           : (G == 2 ? go(std::integral_constant<int, 2>{}) : go(std::integral_constant<int, 1>{}));
     if (e != cudaSuccess) return e;
-    kernel<<<grid, (kWarps + 1) * 32, C::kSmem, stream>>>(*tmK, *tmV, p);
   } else {
     decode_split_kernel<T, D><<<grid, kWarps * 32, 0, stream>>>(p);
   }

@@ -216,6 +216,7 @@ __device__ void producer(const FwdParams& p, const CUtensorMap* tmQ, const CUten
   volatile int* abort = &bars->abort;
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
+  const int group = p.H / p.H_kv;  // query heads per K/V head
   // Tile g goes to slot g % depth of its ring; the slot's previous tile
   // (g - depth) is free once the product that read it is done.
   int g = 0, a = 0;    // tiles and active jobs so far
@@ -228,7 +229,7 @@ __device__ void producer(const FwdParams& p, const CUtensorMap* tmQ, const CUten
     mbar_arrive_expect_tx(&full[slot], C::kTileBytes);
 #pragma unroll
     for (int ch = 0; ch < D / 64; ++ch)
-      tma_load_4d(map, &full[slot], ring + slot * C::kTileBytes + ch * C::kChunkBytes, ch * 64, jb.h,
+      tma_load_4d(map, &full[slot], ring + slot * C::kTileBytes + ch * C::kChunkBytes, ch * 64, jb.h / group,
                   jb.krow + key_tile * BN, jb.bcoord, pol_kv);
     return true;
   };

@@ -26,6 +26,7 @@ struct FwdParams {
   const int* cu_k;      // [B + 1] or nullptr
   int total_q, total_k; // variable length: rows of Q and K/V
   int B, H, Nq, Nk;
+  int H_kv;             // K/V heads (H % H_kv == 0); query head h reads K/V head h / (H / H_kv)
   int num_tiles;        // ceil(Nq / 128)
   int causal;
   int window_left, window_right;  // -1 = unbounded
@@ -49,6 +50,7 @@ struct DecodeParams {
   float* lse_part;           // [S, B, H]      (num_splits > 1)
   const float* slopes;       // [H] or nullptr
   int B, H, num_pages, page_size, max_blocks, num_splits;
+  int H_kv;                  // cache heads; query head h reads cache head h / (H / H_kv)
   int window_left;
   int use_softcap;
   float scale_log2, cap_scale, cap_log2;
@@ -64,5 +66,19 @@ cudaError_t launch_fwd(bool bf16, int d, const CUtensorMap& tmQ, const CUtensorM
 // nullptr for the direct-load split kernel.
 cudaError_t launch_decode(bool bf16, int d, const DecodeParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
                           cudaStream_t stream);
+
+// Writes n_new new tokens per sequence into the paged caches at positions
+// cache_seqlens[b] .. cache_seqlens[b] + n_new - 1.
+struct AppendParams {
+  const void* k_new;  // [B, n_new, H_kv, d]
+  const void* v_new;
+  void* k_cache;      // [num_pages, page_size, H_kv, d]
+  void* v_cache;
+  const int* block_table;    // [B, max_blocks]
+  const int* cache_seqlens;  // [B]
+  int B, n_new, H_kv, d, num_pages, page_size, max_blocks;
+};
+
+cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 
 }  // namespace fa

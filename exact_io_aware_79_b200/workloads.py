@@ -66,10 +66,15 @@ class DecodeWorkload:
     softcap: float = 0.0
     sigma: float = 1.0
     seed: int = 4
+    H_kv: int = 0  # cache heads (grouped-query attention); 0 means H
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.d)
+
+    @property
+    def kv_heads(self) -> int:
+        return self.H_kv or self.H
 
     @property
     def max_blocks(self) -> int:
@@ -127,7 +132,12 @@ class VarlenWorkload:
 VARLEN = VarlenWorkload("varlen_causal_bf16_b16h16n256-4096d128", 16, 16, 128, torch.bfloat16, 256, 4096)
 
 FWD_WORKLOADS = [TINY, CAUSAL_2K, WINDOW_16K, WINDOW_Q4K_K16K, CAUSAL_Q4K_K16K, ALIBI_SOFTCAP]
-DECODE_WORKLOADS = [DECODE, DECODE_SMALL]
+# Grouped-query decode: the same batch and lengths with 32 query heads over 8
+# cache heads (groups of 4).
+DECODE_GQA = DecodeWorkload("paged_decode_gqa_bf16_b64h32kv8d128_page256", 64, 32, 128, torch.bfloat16,
+                            page_size=256, len_lo=1024, len_hi=32768, seed=4, H_kv=8)
+
+DECODE_WORKLOADS = [DECODE, DECODE_SMALL, DECODE_GQA]
 
 
 def alibi_slopes(H: int) -> torch.Tensor:
@@ -213,7 +223,7 @@ def make_decode_inputs(w: DecodeWorkload, device="cpu", seed: Optional[int] = No
     dev = torch.device(device)
     kv_gen = torch.Generator(device=dev)
     kv_gen.manual_seed(s + 1000)
-    shape = (w.num_pages, w.page_size, w.H, w.d)
+    shape = (w.num_pages, w.page_size, w.kv_heads, w.d)
     k_cache = _normal_pages(shape, kv_gen, w.sigma, w.dtype, dev)
     v_cache = _normal_pages(shape, kv_gen, w.sigma, w.dtype, dev)
     slopes = alibi_slopes(w.H) if w.alibi else None

@@ -100,6 +100,21 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *out, float *
                  const float *alibi_slopes, float softcap, cudaStream_t stream);
 
 /*
+ * fa_fwd_gqa -- fa_fwd with grouped-query attention: H query heads share
+ * H_kv key/value heads ("Flash-Attention v2.0 到 v2.7 更新" lists multi-query
+ * and grouped-query attention among the supported forms). Query head h
+ * attends with K/V head h / (H / H_kv); otherwise exactly fa_fwd.
+ *
+ *   k, v [B, Nk, H_kv, d]  (q, out, lse as in fa_fwd)
+ *   H_kv                   1 <= H_kv <= H and H % H_kv == 0, else FA_ERR_SHAPE
+ *                          (H_kv == H is fa_fwd; H_kv == 1 is multi-query)
+ */
+fa_status fa_fwd_gqa(const void *q, const void *k, const void *v, void *out, float *lse,
+                     int B, int H, int H_kv, int Nq, int Nk, int d, fa_dtype dtype, float scale,
+                     int causal, int window_left, int window_right,
+                     const float *alibi_slopes, float softcap, cudaStream_t stream);
+
+/*
  * fa_fwd_varlen -- fa_fwd over a batch of sequences of different lengths
  * packed along the token axis (the pages' "Flash-Attention v2.0 到 v2.7 更新"
  * names the variable-length interface beside the fixed-shape one). The
@@ -176,6 +191,46 @@ fa_status fa_fwd_kvcache(const void *q, const void *k_cache, const void *v_cache
                          fa_dtype dtype, float scale, int window_left,
                          const float *alibi_slopes, float softcap, int num_splits,
                          void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * fa_fwd_kvcache_gqa -- fa_fwd_kvcache with grouped-query attention: the
+ * caches hold H_kv heads ([num_pages, page_size, H_kv, d]); query head h
+ * attends with cache head h / (H / H_kv). 1 <= H_kv <= H and H % H_kv == 0,
+ * else FA_ERR_SHAPE. Split count, workspace size and every other argument
+ * as for fa_fwd_kvcache with the same B, H, d (fa_kvcache_num_splits and
+ * fa_kvcache_workspace_size take H, the query heads).
+ */
+fa_status fa_fwd_kvcache_gqa(const void *q, const void *k_cache, const void *v_cache,
+                             const int *block_table, const int *cache_seqlens,
+                             void *out, float *lse,
+                             int B, int H, int H_kv, int d, int num_pages, int page_size,
+                             int max_blocks, fa_dtype dtype, float scale, int window_left,
+                             const float *alibi_slopes, float softcap, int num_splits,
+                             void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * fa_kvcache_append -- writes n_new new tokens per sequence into the paged
+ * caches: token i of sequence b (k_new[b, i], v_new[b, i]) goes to position
+ * t = cache_seqlens[b] + i, i.e. row t % page_size of page
+ * block_table[b][t / page_size] ("Flash-Attention v2.0 到 v2.7 更新", v2.5).
+ * cache_seqlens is read, not updated: the caller advances it by n_new
+ * before the next decode call.
+ *
+ *   k_new, v_new  [B, n_new, H_kv, d] fp16/bf16 device, read
+ *   k_cache, v_cache  [num_pages, page_size, H_kv, d] same dtype, written
+ *                 at the new positions only
+ *   block_table [B, max_blocks], cache_seqlens [B]  int32 device, read
+ *
+ * Positions at or past max_blocks * page_size, negative lengths and table
+ * entries outside [0, num_pages) are skipped on the device (nothing is
+ * written for them). Limits: B <= 65535; B * n_new * H_kv < 2^31;
+ * max_blocks * page_size < 2^31. B * n_new == 0 is a no-op. Pointers
+ * 16-byte aligned (the int32 arrays 4-byte aligned).
+ */
+fa_status fa_kvcache_append(const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                            const int *block_table, const int *cache_seqlens,
+                            int B, int n_new, int H_kv, int d, int num_pages, int page_size,
+                            int max_blocks, fa_dtype dtype, cudaStream_t stream);
 
 /*
  * Number of splits fa_fwd_kvcache uses for these sizes: num_splits itself

@@ -161,6 +161,29 @@ def attn_fwd(q, k, v, scale: float, causal: bool = False, window_left: int = -1,
     return (o, lse, p) if return_probs else (o, lse)
 
 
+def _expand_heads(a: np.ndarray, H: int, axis: int) -> np.ndarray:
+    """Repeats each of the a.shape[axis] = H_kv heads H / H_kv times, so that
+    query head h meets K/V head h // (H / H_kv)."""
+    H_kv = a.shape[axis]
+    if H_kv < 1 or H % H_kv:
+        raise ValueError("H must be a multiple of the K/V head count")
+    return np.ascontiguousarray(np.repeat(a, H // H_kv, axis=axis))
+
+
+def attn_fwd_gqa(q, k, v, scale: float, causal: bool = False, window_left: int = -1,
+                 window_right: int = -1, alibi_slopes=None, softcap: float = 0.0,
+                 rows: Optional[Sequence[int]] = None, num_threads: int = 0,
+                 dtype_code: Optional[int] = None):
+    """Grouped-query attention: q [B,Nq,H,d], k/v [B,Nk,H_kv,d]; query head h
+    attends with K/V head h // (H / H_kv). Returns (o [B,R,H,d], lse [B,H,R])."""
+    qa, code = _as_storage(q, dtype_code)
+    ka, kc = _as_storage(k, dtype_code)
+    va, vc = _as_storage(v, dtype_code)
+    H = qa.shape[2]
+    return attn_fwd(qa, _expand_heads(ka, H, 2), _expand_heads(va, H, 2), scale, causal, window_left, window_right,
+                    alibi_slopes, softcap, rows=rows, num_threads=num_threads, dtype_code=code)
+
+
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, causal: bool = False,
                     window_left: int = -1, window_right: int = -1, alibi_slopes=None, softcap: float = 0.0,
                     num_threads: int = 0, dtype_code: Optional[int] = None):
@@ -240,6 +263,47 @@ def attn_decode_paged(q, k_cache, v_cache, block_table, cache_seqlens, scale: fl
     if rc:
         raise ValueError("oracle_attn_decode_paged failed: %d" % rc)
     return o, lse
+
+
+def attn_decode_paged_gqa(q, k_cache, v_cache, block_table, cache_seqlens, scale: float,
+                          window_left: int = -1, alibi_slopes=None, softcap: float = 0.0,
+                          batch: Optional[Sequence[int]] = None, num_splits: int = 1,
+                          num_threads: int = 0, dtype_code: Optional[int] = None):
+    """Grouped-query paged decode: q [B,1,H,d]; caches [num_pages,page_size,H_kv,d];
+    query head h reads cache head h // (H / H_kv). Returns as attn_decode_paged."""
+    qa, code = _as_storage(q, dtype_code)
+    ka, _ = _as_storage(k_cache, dtype_code)
+    va, _ = _as_storage(v_cache, dtype_code)
+    H = qa.shape[2]
+    return attn_decode_paged(qa, _expand_heads(ka, H, 2), _expand_heads(va, H, 2), block_table, cache_seqlens,
+                             scale, window_left, alibi_slopes, softcap, batch=batch, num_splits=num_splits,
+                             num_threads=num_threads, dtype_code=code)
+
+
+def kvcache_append(k_new, v_new, k_cache, v_cache, block_table, cache_seqlens):
+    """Returns copies of the caches with the new tokens written in: token i of
+    sequence b goes to position t = cache_seqlens[b] + i, i.e. row
+    t % page_size of page block_table[b][t // page_size]; positions past
+    the table and entries outside [0, num_pages) are skipped. Works on the
+    raw storage (any element type), so the result is bit-exact."""
+    kn, vn = np.asarray(k_new), np.asarray(v_new)
+    kc, vc = np.array(k_cache, copy=True), np.array(v_cache, copy=True)
+    bt = np.asarray(block_table, dtype=np.int64)
+    sl = np.asarray(cache_seqlens, dtype=np.int64).reshape(-1)
+    B, n_new = kn.shape[0], kn.shape[1]
+    num_pages, page = kc.shape[0], kc.shape[1]
+    cap = bt.shape[1] * page
+    for b in range(B):
+        for i in range(n_new):
+            t = int(sl[b]) + i
+            if sl[b] < 0 or t >= cap:
+                continue
+            pg = int(bt[b, t // page])
+            if not 0 <= pg < num_pages:
+                continue
+            kc[pg, t % page] = kn[b, i]
+            vc[pg, t % page] = vn[b, i]
+    return kc, vc
 
 
 def combine_splits(o_part: np.ndarray, lse_part: np.ndarray):

@@ -174,3 +174,56 @@ def test_workspace_size(lib):
     assert ws(64, 32, 128, 128, 256, 16) == o_bytes + rows * 4
     assert ws(64, 32, 128, 128, 256, 0) == ws(64, 32, 128, 128, 256, 16)
     assert ws(4, 2, 96, 16, 256, 4) == 0          # invalid head dim
+
+
+def test_gqa_validation(lib):
+    def g(H=8, H_kv=2, **kw):
+        a = dict(q=P, k=P, v=P, out=P, lse=P, B=1, Nq=128, Nk=128, d=128, dtype=1, scale=0.1, causal=0, wl=-1,
+                 wr=-1, slopes=None, cap=0.0)
+        a.update(kw)
+        return lib.fa_fwd_gqa(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], H, H_kv, a["Nq"], a["Nk"],
+                              a["d"], a["dtype"], a["scale"], a["causal"], a["wl"], a["wr"], a["slopes"], a["cap"],
+                              None)
+    assert g(H_kv=3) == SHAPE        # 8 % 3 != 0
+    assert g(H_kv=0) == SHAPE
+    assert g(H_kv=16) == SHAPE       # more K/V heads than query heads
+    assert g(d=80) == HEADDIM
+    assert g(k=None) == NULL
+    assert g(H_kv=1) in (OK, DEVICE)
+    assert g(H_kv=8) in (OK, DEVICE)
+
+    def gk(H=8, H_kv=2, **kw):
+        a = dict(q=P, kc=P, vc=P, bt=P, sl=P, out=P, lse=P, B=4, d=128, num_pages=64, page=256, mb=16, dtype=1,
+                 scale=0.1, wl=-1, slopes=None, cap=0.0, splits=1, ws=None, ws_bytes=0)
+        a.update(kw)
+        return lib.fa_fwd_kvcache_gqa(a["q"], a["kc"], a["vc"], a["bt"], a["sl"], a["out"], a["lse"], a["B"], H,
+                                      H_kv, a["d"], a["num_pages"], a["page"], a["mb"], a["dtype"], a["scale"],
+                                      a["wl"], a["slopes"], a["cap"], a["splits"], a["ws"], a["ws_bytes"], None)
+    assert gk(H_kv=5) == SHAPE
+    assert gk(H_kv=0) == SHAPE
+    assert gk(bt=None) == NULL
+    assert gk(splits=4, ws=None) == WORKSPACE
+    assert gk(H_kv=4) in (OK, DEVICE)
+
+
+def test_append_validation(lib):
+    def ap(**kw):
+        a = dict(kn=P, vn=P, kc=P, vc=P, bt=P, sl=P, B=4, n=1, Hkv=2, d=128, num_pages=64, page=256, mb=16,
+                 dtype=1)
+        a.update(kw)
+        return lib.fa_kvcache_append(a["kn"], a["vn"], a["kc"], a["vc"], a["bt"], a["sl"], a["B"], a["n"],
+                                     a["Hkv"], a["d"], a["num_pages"], a["page"], a["mb"], a["dtype"], None)
+    assert ap(d=96) == HEADDIM
+    assert ap(dtype=3) == DTYPE
+    assert ap(B=-1) == SHAPE
+    assert ap(n=-1) == SHAPE
+    assert ap(Hkv=0) == SHAPE
+    assert ap(num_pages=0) == SHAPE
+    assert ap(page=0) == ARG
+    assert ap(B=70000) == SHAPE
+    assert ap(kn=None) == NULL
+    assert ap(sl=None) == NULL
+    assert ap(kc=P + 8) == ARG
+    assert ap(bt=P + 2) == ARG
+    assert ap(n=0, kn=None) == OK       # nothing to append
+    assert ap() in (OK, DEVICE)

@@ -496,3 +496,53 @@ def test_varlen_rows_outside_every_sequence_are_nan():
     o, lse = oracle.attn_fwd_varlen(q, k, v, cq, ck, 0.5)
     assert np.isnan(o[-2:]).all() and np.isnan(lse[:, -2:]).all()
     assert not np.isnan(o[:-2]).any()
+
+
+# ------------------------------------------------------------ grouped-query heads and cache append
+
+@pytest.mark.parametrize("H,H_kv", [(4, 2), (6, 3), (4, 1), (3, 3)])
+def test_gqa_query_head_reads_kv_head_h_over_group(H, H_kv):
+    # V of K/V head j is the constant j: every output of query head h is
+    # exactly its K/V head index, whatever the attention weights
+    B, Nq, Nk, d = 2, 5, 7, 4
+    q, k = rnd((B, Nq, H, d), 51), rnd((B, Nk, H_kv, d), 52)
+    v = np.broadcast_to(np.arange(H_kv, dtype=np.float64)[None, None, :, None], (B, Nk, H_kv, d)).copy()
+    o, lse = oracle.attn_fwd_gqa(q, k, v, 0.7, causal=True)
+    for h in range(H):
+        np.testing.assert_allclose(o[:, :, h], h // (H // H_kv), rtol=0, atol=1e-12)
+    # and the scores of head h are those of K head h // group: same LSE as
+    # plain attention against that head
+    for h in range(H):
+        _, l1 = oracle.attn_fwd(q[:, :, h:h + 1], k[:, :, h // (H // H_kv):h // (H // H_kv) + 1], v[:, :, :1], 0.7,
+                                causal=True)
+        np.testing.assert_allclose(lse[:, h], l1[:, 0], rtol=0, atol=1e-12)
+
+
+def test_gqa_decode_reads_cache_head_h_over_group():
+    H, H_kv, d, page, mb = 6, 2, 4, 4, 3
+    q, w_k, w_v, table, lens = decode_case(61, B=2, H=H, d=d, page=page, max_blocks=mb, lens=(9, 5))
+    kc = rnd((2 * mb, page, H_kv, d), 62)
+    vc = np.broadcast_to(np.arange(H_kv, dtype=np.float64)[None, None, :, None], kc.shape).copy()
+    o, lse = oracle.attn_decode_paged_gqa(q, kc, vc, table, lens, 0.5)
+    for h in range(H):
+        np.testing.assert_allclose(o[:, 0, h], h // (H // H_kv), rtol=0, atol=1e-12)
+
+
+def test_append_writes_tokens_where_the_table_says():
+    B, n_new, H, d, page, mb = 3, 5, 2, 4, 4, 4
+    rng = np.random.default_rng(71)
+    table = rng.permutation(B * mb).reshape(B, mb).astype(np.int32)
+    lens = np.array([0, 6, 13], dtype=np.int32)     # the last one runs past the table (16 slots)
+    kc = rng.standard_normal((B * mb, page, H, d))
+    vc = rng.standard_normal((B * mb, page, H, d))
+    kn = rng.standard_normal((B, n_new, H, d))
+    vn = rng.standard_normal((B, n_new, H, d))
+    k2, v2 = oracle.kvcache_append(kn, vn, kc, vc, table, lens)
+    for b in range(B):
+        for t in range(mb * page):
+            pg, row = table[b, t // page], t % page
+            i = t - lens[b]
+            if 0 <= i < n_new:
+                assert np.array_equal(k2[pg, row], kn[b, i]) and np.array_equal(v2[pg, row], vn[b, i])
+            else:
+                assert np.array_equal(k2[pg, row], kc[pg, row]) and np.array_equal(v2[pg, row], vc[pg, row])
