@@ -141,6 +141,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 // running at one time share K/V in L2.
 struct Job {
   int b, h, q0, f, l;  // K/V tiles f..l
+  int hk;              // K/V head of query head h
   bool has;            // at least one visible key
   int Nq, Nk;          // lengths of the job's sequence
   int qrow, krow;      // first row of the sequence in the Q and K/V maps
@@ -173,6 +174,7 @@ __device__ __forceinline__ Job make_job(const FwdParams& p, int b, int h, int Nq
   Job j;
   j.b = b;
   j.h = h;
+  j.hk = p.H_kv == p.H ? h : h / (p.H / p.H_kv);
   j.q0 = tile * BM;
   j.Nq = Nq;
   j.Nk = Nk;
@@ -216,7 +218,6 @@ __device__ void producer(const FwdParams& p, const CUtensorMap* tmQ, const CUten
   volatile int* abort = &bars->abort;
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
-  const int group = p.H / p.H_kv;  // query heads per K/V head
   // Tile g goes to slot g % depth of its ring; the slot's previous tile
   // (g - depth) is free once the product that read it is done.
   int g = 0, a = 0;    // tiles and active jobs so far
@@ -229,7 +230,7 @@ __device__ void producer(const FwdParams& p, const CUtensorMap* tmQ, const CUten
     mbar_arrive_expect_tx(&full[slot], C::kTileBytes);
 #pragma unroll
     for (int ch = 0; ch < D / 64; ++ch)
-      tma_load_4d(map, &full[slot], ring + slot * C::kTileBytes + ch * C::kChunkBytes, ch * 64, jb.h / group,
+      tma_load_4d(map, &full[slot], ring + slot * C::kTileBytes + ch * C::kChunkBytes, ch * 64, jb.hk,
                   jb.krow + key_tile * BN, jb.bcoord, pol_kv);
     return true;
   };
