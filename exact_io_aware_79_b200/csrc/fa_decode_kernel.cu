@@ -364,8 +364,159 @@ __global__ void __launch_bounds__((kWarps + 1) * 32)
       int dummy = 0;
       for (int i = first; i < issued; ++i) mbar_wait(&sh->full[i % NST], (i / NST) & 1, &dummy);
     }
+  } else if constexpr (G > 1) {
+    // ---------------- consumers, G heads: the per-head partial dot products
+    // of a token are reduce-scattered over its LPT lanes, so each lane ends
+    // with the full score of one head (lanes of a token group split into G
+    // subgroups of LPT / G lanes, subgroup j holding head j); the lane keeps
+    // that head's running max and sum, and broadcasts its probabilities to
+    // the other lanes of the token group for the V update.
+    const int g = lane / LPT;
+    const int cl = lane % LPT;
+    const int gbase = lane & ~(LPT - 1);  // first lane of this token group
+    constexpr int SUB = LPT / G;           // lanes per head subgroup
+    const int my = cl / SUB;               // the head this lane scores
+    const float qscale = p.use_softcap ? p.cap_scale : p.scale_log2;
+    const bool alibi = p.slopes != nullptr;
+    float qf[G][8];
+    float acc[G][8];
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) {
+      widen8<T>(*reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.q) +
+                                                (static_cast<size_t>(b) * p.H + h0 + gi) * D + cl * 8),
+                qf[gi]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qf[gi][e] *= qscale;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[gi][e] = 0.0f;
+    }
+    const float slope_l2 = alibi ? p.slopes[h0 + my] * kLog2e : 0.0f;
+    float m = -INFINITY, lsum = 0.0f;  // of head `my`, this token group
+
+    for (int i = 0; i < n_st; ++i) {
+      const int slot = i % NST;
+      bool ok = mbar_wait(&sh->full[slot], (i / NST) & 1, abort);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        bad = true;
+        break;
+      }
+      if (sh->bad[slot]) {
+        bad = true;
+      } else {
+        const T* kt = reinterpret_cast<const T*>(sK + slot * C::kTile);
+        const T* vt = reinterpret_cast<const T*>(sV + slot * C::kTile);
+        const int a = a0 + i * kRows;
+        float sc[kSteps];
+        float mt = -INFINITY;
+#pragma unroll
+        for (int st = 0; st < kSteps; ++st) {
+          const int r = warp * (kRows / kWarps) + st * TPW + g;
+          float kf[8];
+          widen8<T>(*reinterpret_cast<const uint4*>(kt + r * D + cl * 8), kf);
+          float v[G];
+#pragma unroll
+          for (int gi = 0; gi < G; ++gi) {
+            float d0 = 0.0f, d1 = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              d0 = fmaf(qf[gi][e], kf[e], d0);
+              d1 = fmaf(qf[gi][e + 1], kf[e + 1], d1);
+            }
+            v[gi] = d0 + d1;
+          }
+          // reduce-scatter over the token's lanes
+          float s1;
+          if constexpr (G == 4) {
+            const bool up = (cl & (LPT / 2)) != 0;
+            const float a0s = up ? v[0] : v[2], a1s = up ? v[1] : v[3];
+            const float k0 = up ? v[2] : v[0], k1 = up ? v[3] : v[1];
+            const float r0 = k0 + __shfl_xor_sync(0xffffffffu, a0s, LPT / 2);
+            const float r1 = k1 + __shfl_xor_sync(0xffffffffu, a1s, LPT / 2);
+            const bool up2 = (cl & (LPT / 4)) != 0;
+            s1 = (up2 ? r1 : r0) + __shfl_xor_sync(0xffffffffu, up2 ? r0 : r1, LPT / 4);
+          } else {
+            const bool up = (cl & (LPT / 2)) != 0;
+            s1 = (up ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, up ? v[0] : v[1], LPT / 2);
+          }
+#pragma unroll
+          for (int o = SUB / 2; o >= 1; o >>= 1) s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+          const int tok = a + r;
+          float t = p.use_softcap ? p.cap_log2 * tanh_via_exp2(s1) : s1;
+          if (alibi) t -= slope_l2 * static_cast<float>(pos - tok);
+          sc[st] = (tok >= t0 && tok < t1) ? t : -INFINITY;
+          mt = fmaxf(mt, sc[st]);
+        }
+        const float mn = fmaxf(m, mt);
+        float pw[kSteps];
+        float alpha = 1.0f;
+        if (mn != -INFINITY) {
+          alpha = ex2(m - mn);
+          lsum *= alpha;
+#pragma unroll
+          for (int st = 0; st < kSteps; ++st) {
+            pw[st] = ex2(sc[st] - mn);
+            lsum += pw[st];
+          }
+          m = mn;
+        } else {
+#pragma unroll
+          for (int st = 0; st < kSteps; ++st) pw[st] = 0.0f;
+        }
+        // every lane updates all G heads for its 8 columns of V
+#pragma unroll
+        for (int gi = 0; gi < G; ++gi) {
+          const float al = __shfl_sync(0xffffffffu, alpha, gbase + gi * SUB);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[gi][e] *= al;
+        }
+#pragma unroll
+        for (int st = 0; st < kSteps; ++st) {
+          const int r = warp * (kRows / kWarps) + st * TPW + g;
+          float vf[8];
+          widen8<T>(*reinterpret_cast<const uint4*>(vt + r * D + cl * 8), vf);
+#pragma unroll
+          for (int gi = 0; gi < G; ++gi) {
+            const float pg = __shfl_sync(0xffffffffu, pw[st], gbase + gi * SUB);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[gi][e] = fmaf(pg, vf[e], acc[gi][e]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->empty[slot]);
+    }
+    // merge the token groups of this warp per head, then publish
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) {
+      float mg = __shfl_sync(0xffffffffu, m, gbase + gi * SUB);
+      float lg = __shfl_sync(0xffffffffu, lsum, gbase + gi * SUB);
+#pragma unroll
+      for (int o = LPT; o < 32; o <<= 1) {
+        const float m_o = __shfl_xor_sync(0xffffffffu, mg, o);
+        const float l_o = __shfl_xor_sync(0xffffffffu, lg, o);
+        const float mm = fmaxf(mg, m_o);
+        const float x = (mg == -INFINITY) ? 0.0f : ex2(mg - mm);
+        const float x_o = (m_o == -INFINITY) ? 0.0f : ex2(m_o - mm);
+        lg = lg * x + l_o * x_o;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float a_o = __shfl_xor_sync(0xffffffffu, acc[gi][e], o);
+          acc[gi][e] = acc[gi][e] * x + a_o * x_o;
+        }
+        mg = mm;
+      }
+      if (lane < LPT) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sh->acc[warp][gi][cl * 8 + e] = acc[gi][e];
+      }
+      if (lane == 0) {
+        sh->m[warp][gi] = mg;
+        sh->l[warp][gi] = lg;
+      }
+    }
   } else {
-    // ---------------- consumers
+    // ---------------- consumers, one head per lane group
     const int g = lane / LPT;
     const int cl = lane % LPT;
     const float qscale = p.use_softcap ? p.cap_scale : p.scale_log2;
