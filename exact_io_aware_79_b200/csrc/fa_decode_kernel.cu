@@ -378,17 +378,20 @@ __global__ void __launch_bounds__((kWarps + 1) * 32)
     const int my = cl / SUB;               // the head this lane scores
     const float qscale = p.use_softcap ? p.cap_scale : p.scale_log2;
     const bool alibi = p.slopes != nullptr;
-    float qf[G][8];
-    float acc[G][8];
+    // q and the accumulators as packed fp32 pairs (fp32x2 FMA)
+    uint64_t q2[G][4];
+    uint64_t acc2[G][4];
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
+      float qf[8];
       widen8<T>(*reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.q) +
                                                 (static_cast<size_t>(b) * p.H + h0 + gi) * D + cl * 8),
-                qf[gi]);
+                qf);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) qf[gi][e] *= qscale;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[gi][e] = 0.0f;
+      for (int e = 0; e < 4; ++e) {
+        q2[gi][e] = f2_pack(qf[2 * e] * qscale, qf[2 * e + 1] * qscale);
+        acc2[gi][e] = 0;  // 0 bits = +0.0f pair
+      }
     }
     const float slope_l2 = alibi ? p.slopes[h0 + my] * kLog2e : 0.0f;
     float m = -INFINITY, lsum = 0.0f;  // of head `my`, this token group
@@ -414,15 +417,17 @@ __global__ void __launch_bounds__((kWarps + 1) * 32)
           const int r = warp * (kRows / kWarps) + st * TPW + g;
           float kf[8];
           widen8<T>(*reinterpret_cast<const uint4*>(kt + r * D + cl * 8), kf);
+          uint64_t k2[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) k2[e] = f2_pack(kf[2 * e], kf[2 * e + 1]);
           float v[G];
 #pragma unroll
           for (int gi = 0; gi < G; ++gi) {
-            float d0 = 0.0f, d1 = 0.0f;
+            uint64_t d2 = f2_mul(q2[gi][0], k2[0]);
 #pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              d0 = fmaf(qf[gi][e], kf[e], d0);
-              d1 = fmaf(qf[gi][e + 1], kf[e + 1], d1);
-            }
+            for (int e = 1; e < 4; ++e) d2 = f2_fma(q2[gi][e], k2[e], d2);
+            float d0, d1;
+            f2_unpack(d2, d0, d1);
             v[gi] = d0 + d1;
           }
           // reduce-scatter over the token's lanes
@@ -467,19 +472,24 @@ __global__ void __launch_bounds__((kWarps + 1) * 32)
 #pragma unroll
         for (int gi = 0; gi < G; ++gi) {
           const float al = __shfl_sync(0xffffffffu, alpha, gbase + gi * SUB);
+          const uint64_t al2 = f2_pack(al, al);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[gi][e] *= al;
+          for (int e = 0; e < 4; ++e) acc2[gi][e] = f2_mul(acc2[gi][e], al2);
         }
 #pragma unroll
         for (int st = 0; st < kSteps; ++st) {
           const int r = warp * (kRows / kWarps) + st * TPW + g;
           float vf[8];
           widen8<T>(*reinterpret_cast<const uint4*>(vt + r * D + cl * 8), vf);
+          uint64_t v2[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) v2[e] = f2_pack(vf[2 * e], vf[2 * e + 1]);
 #pragma unroll
           for (int gi = 0; gi < G; ++gi) {
             const float pg = __shfl_sync(0xffffffffu, pw[st], gbase + gi * SUB);
+            const uint64_t pg2 = f2_pack(pg, pg);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[gi][e] = fmaf(pg, vf[e], acc[gi][e]);
+            for (int e = 0; e < 4; ++e) acc2[gi][e] = f2_fma(v2[e], pg2, acc2[gi][e]);
           }
         }
       }
@@ -489,6 +499,9 @@ __global__ void __launch_bounds__((kWarps + 1) * 32)
     // merge the token groups of this warp per head, then publish
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) f2_unpack(acc2[gi][e], acc[2 * e], acc[2 * e + 1]);
       float mg = __shfl_sync(0xffffffffu, m, gbase + gi * SUB);
       float lg = __shfl_sync(0xffffffffu, lsum, gbase + gi * SUB);
 #pragma unroll
@@ -501,14 +514,14 @@ __global__ void __launch_bounds__((kWarps + 1) * 32)
         lg = lg * x + l_o * x_o;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float a_o = __shfl_xor_sync(0xffffffffu, acc[gi][e], o);
-          acc[gi][e] = acc[gi][e] * x + a_o * x_o;
+          const float a_o = __shfl_xor_sync(0xffffffffu, acc[e], o);
+          acc[e] = acc[e] * x + a_o * x_o;
         }
         mg = mm;
       }
       if (lane < LPT) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) sh->acc[warp][gi][cl * 8 + e] = acc[gi][e];
+        for (int e = 0; e < 8; ++e) sh->acc[warp][gi][cl * 8 + e] = acc[e];
       }
       if (lane == 0) {
         sh->m[warp][gi] = mg;
