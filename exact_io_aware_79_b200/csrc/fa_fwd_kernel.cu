@@ -10,16 +10,18 @@
 //
 // B200 mapping. The grid is persistent (at most one CTA per SM); a CTA runs
 // jobs, each one 128-row Q tile of one (batch, head), back to back with
-// eleven warps:
-//   warps 0-7  softmax: warps w and w + 4 share TMEM lanes 32 (w % 4) ..
-//              + 31 (one query row per lane) and split each row's 128 keys
-//              into halves, combining the half-row maxima and sums through
-//              shared memory
-//   warp  8    TMA producer: each job's Q tile (two buffers, so the next
-//              job's Q lands early), then K and V tiles into two rings of
+// these warps:
+//   softmax    4 * parts warps: the parts warps w, w + 4, ... share TMEM
+//              lanes 32 (w % 4) .. + 31 (one query row per lane) and split
+//              each row's 128 keys into parts slices, combining the partial
+//              maxima and sums through shared memory (parts = 2 for plain
+//              scores; 4 with softcap or ALiBi, whose per-element work four
+//              warps per sub-partition hide better)
+//   producer   TMA: each job's Q tile (two buffers, so the next job's Q
+//              lands early), then K and V tiles into two rings of
 //              shared-memory slots (128-byte swizzle), expect-tx
-//   warp  9    QK issuer (one elected thread) and TMEM owner
-//   warp 10    PV issuer (one elected thread)
+//   QK issuer  one elected thread; owns TMEM
+//   PV issuer  one elected thread
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   cols   0..127  S buffer 0 (fp32 scores)
 //   cols 128..255  S buffer 1
@@ -57,12 +59,14 @@ namespace {
 
 constexpr int BM = 128;  // query rows per Q tile
 constexpr int BN = 128;  // keys per K/V tile
-constexpr int kThreads = 352;
-constexpr int kSoftmaxWarps = 8;
-constexpr int kProducerWarp = 8;
-constexpr int kQkWarp = 9;   // issues S = Q K^T; owns TMEM
-constexpr int kPvWarp = 10;  // issues O += P V
-static_assert(kThreads == 32 * (kPvWarp + 1), "one warp per role after the softmax warps");
+// Softmax warps per row (per TMEM lane quarter): the score modifiers
+// (softcap, ALiBi) add per-element work that four warps per sub-partition
+// hide better; plain scores run fastest with two. Warp roles: softmax warps
+// 0 .. 4 * parts - 1, then the TMA producer, the QK issuer (owns TMEM) and
+// the PV issuer.
+constexpr int kMaxParts = 4;
+constexpr int parts_of(bool cap, bool alibi) { return (cap || alibi) ? 4 : 2; }
+constexpr int threads_of(bool cap, bool alibi) { return 32 * (4 * parts_of(cap, alibi) + 3); }
 constexpr int kMaxSlots = 6;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kTmemCols = 512;
@@ -74,6 +78,8 @@ constexpr int kRing = 8;
 constexpr uint32_t kTmemO = 256;
 constexpr uint32_t kTmemP = 384;  // two 64-column P buffers
 
+constexpr int kBarrierBytes = 8192;  // barrier block and exchange slots
+
 template <int D>
 struct Cfg {
   static constexpr int kChunkBytes = BM * 128;       // 128 rows x 64 elements x 2 bytes
@@ -83,7 +89,7 @@ struct Cfg {
   static constexpr int kSlotsK = (D == 128) ? 2 : 5;  // K ring depth
   static constexpr int kSlotsV = (D == 128) ? 2 : 5;  // V ring depth
   static constexpr int kSlots = kSlotsK + kSlotsV;
-  static constexpr int kSmemBytes = 1024 + (kQBufs + kSlots) * kTileBytes + 4096;
+  static constexpr int kSmemBytes = 1024 + (kQBufs + kSlots) * kTileBytes + kBarrierBytes;
 };
 
 struct Barriers {
@@ -103,9 +109,9 @@ struct Barriers {
   uint64_t pv_idle;    // all MMAs of the PV thread complete
   uint32_t tmem_base;
   int abort;
-  // per row and exchange parity: the two half-row partial maxima / sums
-  // (NaN marks a half that gave up on a timed-out wait)
-  float xchg[2][2][BM];
+  // per exchange parity, part and row: the partial maxima / sums of the
+  // parts of a row (NaN marks a part that gave up on a timed-out wait)
+  float xchg[2][kMaxParts][BM];
 };
 
 // Visible key interval [lo, hi] of query row q (empty when lo > hi).
@@ -368,45 +374,51 @@ __device__ __forceinline__ float mod_score(const FwdParams& p, float x, float sl
   return t;
 }
 
-// Softmax: eight warps, two per sub-partition. Warp w (w < 4) and warp
-// w + 4 own the same 32 query rows (TMEM lanes 32(w % 4) ..), one row per
-// thread; warp w takes keys 0-63 of each 128-key tile and warp w + 4 keys
-// 64-127. The two halves of a row exchange partial maxima through shared
-// memory under a 64-thread named barrier, so both take the same lazy
-// rescaling decision; each half writes its part of P (16-bit, into columns
-// [32 * half, 32 * half + 32) of the tile's P buffer), rescales and stores
-// its 64 columns of O, and the row sums are combined once at the end.
-// kCap / kAlibi select the score modifiers at compile time; whether a K tile
-// needs the element mask is decided per tile for the whole group, so the
-// common interior tiles run without per-element compares.
-__device__ __forceinline__ void pair_sync(int quarter) {
-  // named barrier 1 + quarter, shared by the two warps of one lane quarter
-  asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+// Softmax: kSoftmaxWarps warps, kParts per sub-partition. The kParts warps
+// w, w + 4, w + 8, ... own the same 32 query rows (TMEM lanes 32(w % 4) ..),
+// one row per thread, and split each 128-key tile into kParts slices of
+// kKeys keys. They exchange partial maxima through shared memory under a
+// named barrier, so all take the same lazy rescaling decision; each writes
+// its slice of P (16-bit, into its columns of the tile's P buffer), rescales
+// and stores its D / kParts columns of O, and the row sums are combined once
+// at the end. kCap / kAlibi select the score modifiers at compile time;
+// whether a K tile needs the element mask is decided per tile for the whole
+// group, so the common interior tiles run without per-element compares.
+template <int kParts>
+__device__ __forceinline__ void part_sync(int quarter) {
+  // named barrier 1 + quarter, shared by the kParts warps of one lane quarter
+  asm volatile("bar.sync %0, %1;" ::"r"(1 + quarter), "r"(32 * kParts) : "memory");
 }
 
-// Exchange of one value between the two halves of a row. Both halves call
-// it the same number of times (the k-th exchange uses slot k & 1, so a slot
-// is rewritten only after the partner has passed the next barrier and hence
-// read it). A half that failed passes NaN; the caller sees the partner's
-// value, NaN if the partner failed.
-__device__ __forceinline__ float pair_exchange(float (&xchg)[2][2][BM], int k, int half, int r, int quarter,
-                                               float v) {
-  xchg[k & 1][half][r] = v;
-  pair_sync(quarter);
-  return xchg[k & 1][half ^ 1][r];
+// Exchange of one value among the kParts warps of a row. All call it the
+// same number of times (the k-th exchange uses slot k & 1, so a slot is
+// rewritten only after every partner has passed the next barrier and hence
+// read it). A part that failed passes NaN. Fills all[] with every part's
+// value (own included).
+template <int kParts>
+__device__ __forceinline__ void part_exchange(float (&xchg)[2][kMaxParts][BM], int k, int part, int r, int quarter,
+                                              float v, float (&all)[kParts]) {
+  xchg[k & 1][part][r] = v;
+  part_sync<kParts>(quarter);
+#pragma unroll
+  for (int i = 0; i < kParts; ++i) all[i] = xchg[k & 1][i][r];
 }
 
 template <typename T, int D, bool kCap, bool kAlibi>
 __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, const Job& jb, int g, int& xk,
                             bool& alive) {
   constexpr bool kPlain = !kCap && !kAlibi;
-  constexpr int kHalf = BN / 2;       // keys per thread per tile
-  constexpr int kOCols = D / 2;       // O columns per thread
+  constexpr int kParts = parts_of(kCap, kAlibi);
+  constexpr int kKeys = BN / kParts;     // keys per thread per tile
+  constexpr int kChunks = kKeys / 32;    // 32-column TMEM loads of S per tile
+  constexpr int kOCols = D / kParts;     // O columns per thread
+  constexpr int kOC = kOCols < 32 ? kOCols : 32;  // O columns per TMEM access
+  static_assert(kKeys % 32 == 0 && kOCols % 16 == 0, "part sizes");
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int quarter = warp & 3;
-  const int half = warp >> 2;
+  const int part = warp >> 2;
   const int r = quarter * 32 + lane;  // row of the tile == TMEM lane
   const int h = jb.h, q0 = jb.q0, f = jb.f, l = jb.l;
   const int q = q0 + r;
@@ -418,19 +430,20 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
   const RowRange first_row = row_range(p, jb.Nq, jb.Nk, q0), last_row = row_range(p, jb.Nq, jb.Nk, qz);
   const int pos = q + jb.Nk - jb.Nq;
   const uint32_t lane_sel = static_cast<uint32_t>(quarter * 32) << 16;
-  const uint32_t tO = tmem + lane_sel + kTmemO + half * kOCols;
+  const uint32_t tO = tmem + lane_sel + kTmemO + part * kOCols;
   const float slope_l2 = kAlibi ? p.slopes[h] * kLog2e : 0.0f;
   const float sl2 = p.scale_log2;  // >= 0 (a negative scale is folded into the MMA)
   const uint64_t mul2 = kPlain ? f2_pack(sl2, sl2) : f2_pack(1.0f, 1.0f);
+  const float nan = __int_as_float(0x7fc00000);
 
   float m = -INFINITY;  // running max of the whole row (log2 units)
-  float lsum = 0.0f;    // this half's running sum of exp2(t - m)
+  float lsum = 0.0f;    // this part's running sum of exp2(t - m)
   bool ok = alive;      // after a failure in an earlier job, only fill
-  bool broke = false;   // left the loop at a shared exchange (both halves do)
+  bool broke = false;   // left the loop at a shared exchange (all parts do)
   const int n = jb.has ? l - f + 1 : 0;
   const int n_run = ok ? n : 0;
-  // Each iteration performs exactly one pair exchange, and every early exit
-  // happens right after one, on a decision both halves share, so the named
+  // Each iteration performs exactly one exchange, and every early exit
+  // happens right after one, on a decision all parts share, so the named
   // barriers can never be left waiting for a partner that has gone.
   for (int it = 0; it < n_run; ++it) {
     const int j = f + it;
@@ -438,24 +451,26 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
     const uint32_t tS = tmem + lane_sel + (gi & 1) * 128;
     ok = ok && mbar_wait(&bars->s_ready[gi % kRing], (gi / kRing) & 1, abort);
     ok = __all_sync(0xffffffffu, ok);
-    uint32_t s[2][32];
-    const int key0 = j * BN + half * kHalf;
+    uint32_t s[kChunks][32];
+    const int key0 = j * BN + part * kKeys;
     const bool masked = j * BN < last_row.lo || j * BN + BN - 1 > first_row.hi;  // uniform over the tile
     if (ok) {
       tc_fence_after();
-      tmem_ld32(tS + half * kHalf, s[0]);
-      tmem_ld32(tS + half * kHalf + 32, s[1]);
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) tmem_ld32(tS + part * kKeys + 32 * c, s[c]);
       tmem_wait_ld();
     } else {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) s[0][e] = s[1][e] = 0u;
+      for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[c][e] = 0u;
     }
-    reg_fence(s[0]);
-    reg_fence(s[1]);
-    // pass 1: transform (modifier paths), mask and this half's max
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) reg_fence(s[c]);
+    // pass 1: transform (modifier paths), mask and this part's max
     float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < kChunks; ++c) {
       if (!kPlain || masked) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
@@ -476,18 +491,24 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
       }
     }
     float mt = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
-    // combine with the other half of the row
-    const float mo = pair_exchange(bars->xchg, xk++, half, r, quarter, ok ? mt : __int_as_float(0x7fc00000));
-    ok = __all_sync(0xffffffffu, ok && mo == mo);
-    if (!ok) {  // both halves of every row of this warp pair see the same NaN
+    // combine with the other parts of the row
+    float all[kParts];
+    part_exchange(bars->xchg, xk++, part, r, quarter, ok ? mt : nan, all);
+    bool none_nan = true;
+#pragma unroll
+    for (int i = 0; i < kParts; ++i) {
+      none_nan = none_nan && all[i] == all[i];
+      mt = fmaxf(mt, all[i]);
+    }
+    ok = __all_sync(0xffffffffu, ok && none_nan);
+    if (!ok) {  // every part of every row of this warp group sees the same NaN
       broke = true;
       break;
     }
-    mt = fmaxf(mt, mo);
     // plain path: the max was taken over raw scores; scale after (sl2 >= 0)
     if (kPlain) mt = (mt == -INFINITY) ? -INFINITY : mt * sl2;
 
-    // lazy max update (identical in both halves of the row)
+    // lazy max update (identical in all parts of the row)
     const float m_new = fmaxf(m, mt);
     float alpha = 1.0f;
     bool rescale = false;
@@ -500,16 +521,16 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
     }
     lsum *= alpha;
     const float m_eff = (m == -INFINITY) ? 0.0f : m;
-    // pass 2: P = exp2(t - m) into columns [32 * half, 32 * half + 32) of the
-    // P buffer; pairs of elements go through packed fp32x2 FMA (scale,
+    // pass 2: P = exp2(t - m) into this part's kKeys / 2 columns of the P
+    // buffer; pairs of elements go through packed fp32x2 FMA (scale,
     // subtract max) and add
     const uint64_t m2 = f2_pack(-m_eff, -m_eff);
     uint64_t rsum2[4] = {0, 0, 0, 0};  // independent packed partial sums (0 bits = +0.0f)
-    uint32_t pk[32];
     auto pass2 = [&](auto emu_tag) {
       constexpr bool kMaskedTile = decltype(emu_tag)::value;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < kChunks; ++c) {
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float x0 = __uint_as_float(s[c][2 * e]);
@@ -533,15 +554,15 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
             p1 = (x1 == -INFINITY) ? 0.0f : p1;
           }
           rsum2[e & 3] = f2_add(rsum2[e & 3], f2_pack(p0, p1));
-          pk[16 * c + e] = pack2<T>(p0, p1);
+          pk[e] = pack2<T>(p0, p1);
         }
+        tmem_st16(tmem + lane_sel + kTmemP + (gi & 1) * 64 + part * (kKeys / 2) + 16 * c, pk);
       }
     };
     if (masked)
       pass2(std::true_type{});
     else
       pass2(std::false_type{});
-    tmem_st32(tmem + lane_sel + kTmemP + (gi & 1) * 64 + half * 32, pk);
     float r0, r1, r2, r3;
     f2_unpack(f2_add(rsum2[0], rsum2[1]), r0, r1);
     f2_unpack(f2_add(rsum2[2], rsum2[3]), r2, r3);
@@ -550,20 +571,22 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
       // O must be idle: wait for the product of the previous tile (the only
       // one that can still be running).
       if (it > 0) {
-        // on a timeout, carry on to the next exchange, which ends both halves
+        // on a timeout, carry on to the next exchange, which ends all parts
         ok = mbar_wait(&bars->pv_done[(gi - 1) % kRing], ((gi - 1) / kRing) & 1, abort);
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
       }
 #pragma unroll
-      for (int cc = 0; cc < kOCols / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tO + 32 * cc, o);
+      for (int cc = 0; cc < kOCols / kOC; ++cc) {
+        uint32_t o[kOC];
+        if constexpr (kOC == 32) tmem_ld32(tO + kOC * cc, o);
+        else tmem_ld16(tO + kOC * cc, o);
         tmem_wait_ld();
         reg_fence(o);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-        tmem_st32(tO + 32 * cc, o);
+        for (int e = 0; e < kOC; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+        if constexpr (kOC == 32) tmem_st32(tO + kOC * cc, o);
+        else tmem_st16(tO + kOC * cc, o);
       }
     }
     lsum += rs;
@@ -572,43 +595,46 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars->p_full[gi & 1]);
   }
-  // the loop ran the same number of exchanges in both halves: it ended at a
+  // the loop ran the same number of exchanges in all parts: it ended at a
   // shared break, or after all n iterations (possibly with a failed wait in
-  // one half, which the final exchange reports to the other)
+  // one part, which the final exchange reports to the others)
   const int n_done = broke ? -1 : n_run;
   if (ok && n > 0) {
     ok = mbar_wait(&bars->pv_done[(g + n - 1) % kRing], ((g + n - 1) / kRing) & 1, abort);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
   }
-  // both halves of a row must agree on success; combine the row sums
+  // all parts of a row must agree on success; combine the row sums
   float ltot = lsum;
   if (n_done >= 0 && alive) {
-    const float other = pair_exchange(bars->xchg, xk++, half, r, quarter, ok ? lsum : __int_as_float(0x7fc00000));
-    ok = ok && other == other;
-    ltot = lsum + (other == other ? other : 0.0f);
+    float all[kParts];
+    part_exchange(bars->xchg, xk++, part, r, quarter, ok ? lsum : nan, all);
+    ltot = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kParts; ++i) ltot += all[i];  // NaN if any part failed
+    ok = ok && ltot == ltot;
+    if (!ok) ltot = 0.0f;
   }
 
-  // epilogue: O / l -> dtype for this half's columns, LSE = (m + log2 l) ln 2
-  T* orow = reinterpret_cast<T*>(p.out) + ((jb.obase + (row_ok ? q : 0)) * p.H + h) * D +
-            half * kOCols;
+  // epilogue: O / l -> dtype for this part's columns, LSE = (m + log2 l) ln 2
+  T* orow = reinterpret_cast<T*>(p.out) + ((jb.obase + (row_ok ? q : 0)) * p.H + h) * D + part * kOCols;
   const float inv = ltot > 0.0f ? 1.0f / ltot : 0.0f;
-  const float nan = __int_as_float(0x7fc00000);
   if (ok && n > 0) {
 #pragma unroll
-    for (int cc = 0; cc < kOCols / 32; ++cc) {
-      uint32_t o[32];
-      tmem_ld32(tO + 32 * cc, o);
+    for (int cc = 0; cc < kOCols / kOC; ++cc) {
+      uint32_t o[kOC];
+      if constexpr (kOC == 32) tmem_ld32(tO + kOC * cc, o);
+      else tmem_ld16(tO + kOC * cc, o);
       tmem_wait_ld();
       reg_fence(o);
       if (row_ok) {
-        uint32_t pk[16];
+        uint32_t pk[kOC / 2];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
+        for (int e = 0; e < kOC / 2; ++e)
           pk[e] = pack2<T>(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cc);
+        uint4* dst = reinterpret_cast<uint4*>(orow + kOC * cc);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        for (int v = 0; v < kOC / 8; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
     }
     // O has been read: the next job's first PV product may overwrite it
@@ -622,7 +648,7 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
 #pragma unroll
     for (int v = 0; v < kOCols / 8; ++v) dst[v] = make_uint4(w, w, w, w);
   }
-  if (row_ok && half == 0) {
+  if (row_ok && part == 0) {
     float lse_v;
     if (!ok) lse_v = nan;
     else if (ltot > 0.0f) lse_v = (m + lg2(ltot)) * kLn2;
@@ -643,10 +669,14 @@ __device__ void softmax_group(const FwdParams& p, Barriers* bars, uint32_t tmem)
 }
 
 template <typename T, int D, bool kCap, bool kAlibi>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_of(kCap, kAlibi), 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = Cfg<D>;
+  constexpr int kSoftmaxWarps = 4 * parts_of(kCap, kAlibi);
+  constexpr int kProducerWarp = kSoftmaxWarps;
+  constexpr int kQkWarp = kSoftmaxWarps + 1;
+  constexpr int kPvWarp = kSoftmaxWarps + 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;  // two Q buffers
@@ -711,7 +741,7 @@ template <typename T, int D, bool kCap, bool kAlibi>
 cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const FwdParams& p,
                    cudaStream_t stream) {
   using C = Cfg<D>;
-  static_assert(sizeof(Barriers) <= 4096, "barrier block exceeds its reserve");
+  static_assert(sizeof(Barriers) <= kBarrierBytes, "barrier block exceeds its reserve");
   static_assert(C::kSmemBytes <= 232448, "shared memory budget exceeded");
   static_assert(C::kSlotsK <= kMaxSlots && C::kSlotsV <= kMaxSlots, "too many K/V slots");
   auto kernel = fwd_kernel<T, D, kCap, kAlibi>;
@@ -729,7 +759,7 @@ cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtenso
   }
   const long long items = static_cast<long long>(p.B) * p.H * ((p.num_tiles + 1) / 2);
   dim3 grid(static_cast<unsigned>(items < sm_count[dev] ? items : sm_count[dev]));
-  kernel<<<grid, kThreads, C::kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
+  kernel<<<grid, threads_of(kCap, kAlibi), C::kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
 
