@@ -189,6 +189,12 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def weak_scaling_value(units_per_rank: float, max_seconds: float, world: int) -> float:
+    """Whole-job throughput of N independent replicas: every rank processes
+    units_per_rank, and the job takes the slowest rank's time."""
+    return world * units_per_rank / max_seconds
+
+
 def physical_gpu(local: int) -> str:
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -326,8 +332,8 @@ def gpu_arm(args):
     region_ms = max_over_ranks(r0.elapsed_time(r1), world, dev)
     fwd_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in fe) / K, world, dev)
     dec_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in de) / K, world, dev)
-    fwd_tflops = world * F / (fwd_ms * 1e-3) / 1e12
-    dec_gbs = world * KVB / (dec_ms * 1e-3) / 1e9
+    fwd_tflops = weak_scaling_value(F, fwd_ms * 1e-3, world) / 1e12
+    dec_gbs = weak_scaling_value(KVB, dec_ms * 1e-3, world) / 1e9
 
     # ---- end to end through the public API with pinned host buffers
     hq, hk, hv = (x[n].cpu().pin_memory() for n in ("q", "k", "v"))
