@@ -199,18 +199,30 @@ __device__ __forceinline__ Job make_job(const FwdParams& p, int b, int h, int Nq
   return j;
 }
 
-// Calls fn(job) for every job of this CTA, in order.
+// Calls fn(job) for every job of this CTA, in order. The work items are
+// numbered consecutively over the sequences (b, then head h, then pair pi;
+// sequence b has H * ceil(T_b / 2) items, T_b its Q tiles), so sequences of
+// different lengths leave no empty slots in the round robin; the walk over
+// the sequences only moves forward.
 template <typename Fn>
 __device__ __forceinline__ void for_each_job(const FwdParams& p, Fn&& fn) {
-  const int per_head = (p.num_tiles + 1) / 2;
-  const int items = p.B * p.H * per_head;
-  for (int w = static_cast<int>(blockIdx.x); w < items; w += static_cast<int>(gridDim.x)) {
-    const int bh = w / per_head, pi = w % per_head;
-    const int b = bh / p.H, h = bh % p.H;
-    int Nq, Nk, qrow, krow;
-    if (!seq_of(p, b, Nq, Nk, qrow, krow)) continue;
-    const int tiles = (Nq + BM - 1) / BM;  // of this sequence (<= num_tiles)
-    if (pi >= (tiles + 1) / 2) continue;
+  // (item counts stay below 2^31: the host checks B * H * ceil(Nq / 128))
+  int b = -1;
+  int base = 0, n_b = 0;  // first item of sequence b, its item count
+  int Nq = 0, Nk = 0, qrow = 0, krow = 0, per_b = 1;
+  for (int w = static_cast<int>(blockIdx.x);; w += static_cast<int>(gridDim.x)) {
+    while (w >= base + n_b) {
+      base += n_b;
+      if (++b >= p.B) return;
+      n_b = 0;
+      if (seq_of(p, b, Nq, Nk, qrow, krow)) {
+        per_b = ((Nq + BM - 1) / BM + 1) / 2;  // pairs of Q tiles per head
+        n_b = p.H * per_b;
+      }
+    }
+    const int li = w - base;
+    const int h = li / per_b, pi = li % per_b;
+    const int tiles = (Nq + BM - 1) / BM;
     const int t_long = tiles - 1 - pi;
     fn(make_job(p, b, h, Nq, Nk, qrow, krow, t_long));
     if (pi != t_long) fn(make_job(p, b, h, Nq, Nk, qrow, krow, pi));
