@@ -272,9 +272,10 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeParams p)
 // per CTA, two CTAs per SM.
 constexpr int kRows = 64;  // tokens per stage
 
-template <int D>
+template <int D, int G = 1>
 struct TmaCfg {
-  static constexpr int kStages = (D == 128) ? 3 : 6;
+  // grouped-query CTAs (G > 1) keep fewer stages so three fit on an SM
+  static constexpr int kStages = (D == 128) ? (G > 1 ? 2 : 3) : (G > 1 ? 4 : 6);
   static constexpr int kTile = kRows * D * 2;  // bytes of one K (or V) stage
   static constexpr int kShared = 4096 + 3 * kWarps * 4 * D * 4 / 4;  // barrier block, up to 4 heads
   static constexpr int kSmem = 2 * kStages * kTile + kShared;
@@ -282,9 +283,9 @@ struct TmaCfg {
 
 template <int D, int G>
 struct TmaShared {
-  uint64_t full[TmaCfg<D>::kStages];
-  uint64_t empty[TmaCfg<D>::kStages];
-  int bad[TmaCfg<D>::kStages];
+  uint64_t full[TmaCfg<D, G>::kStages];
+  uint64_t empty[TmaCfg<D, G>::kStages];
+  int bad[TmaCfg<D, G>::kStages];
   int abort;
   float m[kWarps][G], l[kWarps][G];
   float acc[kWarps][G][D];
@@ -295,10 +296,10 @@ struct TmaShared {
 // query heads hs*G .. hs*G + G - 1, which all map to cache head
 // hs*G / (H / H_kv). G = 1 is the plain per-head kernel.
 template <typename T, int D, int G>
-__global__ void __launch_bounds__((kWarps + 1) * 32)
+__global__ void __launch_bounds__((kWarps + 1) * 32, G > 1 ? 3 : 2)
     decode_split_tma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                             const DecodeParams p) {
-  using C = TmaCfg<D>;
+  using C = TmaCfg<D, G>;
   constexpr int NST = C::kStages;
   constexpr int LPT = D / 8;                  // lanes per token
   constexpr int TPW = 32 / LPT;               // tokens per warp per step
@@ -706,7 +707,7 @@ cudaError_t launch(const DecodeParams& p, const CUtensorMap* tmK, const CUtensor
     const int G = group % 4 == 0 ? 4 : (group % 2 == 0 ? 2 : 1);
     auto go = [&](auto g_tag) -> cudaError_t {
       constexpr int kG = decltype(g_tag)::value;
-      using C = TmaCfg<D>;
+      using C = TmaCfg<D, kG>;
       static_assert(sizeof(TmaShared<D, kG>) <= C::kShared, "decode shared block exceeds its reserve");
       auto kernel = decode_split_tma_kernel<T, D, kG>;
       cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
