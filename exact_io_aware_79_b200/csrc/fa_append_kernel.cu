@@ -1,7 +1,9 @@
 // fa_append_kernel.cu -- writes new K/V tokens into the paged caches
 // ("Flash-Attention v2.0 到 v2.7 更新", v2.5: the cache lives in pages reached
-// through block_table; incremental decoding adds each step's keys and values
-// to it). Token t of sequence b lives in row t % page_size of page
+// through block_table; "解密FlashAttention：如何让大语言模型推理速度翻倍",
+// section 智能緩存機制: the key-value cache keeps the context already
+// processed, so each decoding step adds its keys and values to it). Token t
+// of sequence b lives in row t % page_size of page
 // block_table[b][t / page_size]; the n_new new tokens of sequence b take the
 // positions cache_seqlens[b] .. cache_seqlens[b] + n_new - 1.
 #include "fa_internal.h"

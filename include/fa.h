@@ -101,9 +101,9 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *out, float *
 
 /*
  * fa_fwd_gqa -- fa_fwd with grouped-query attention: H query heads share
- * H_kv key/value heads ("Flash-Attention v2.0 到 v2.7 更新" lists multi-query
- * and grouped-query attention among the supported forms). Query head h
- * attends with K/V head h / (H / H_kv); otherwise exactly fa_fwd.
+ * H_kv key/value heads. The pages do not define this form; the reading
+ * taken is the plain one: query head h attends with K/V head h / (H / H_kv),
+ * and everything else is exactly fa_fwd.
  *
  *   k, v [B, Nk, H_kv, d]  (q, out, lse as in fa_fwd)
  *   H_kv                   1 <= H_kv <= H and H % H_kv == 0, else FA_ERR_SHAPE
@@ -116,11 +116,12 @@ fa_status fa_fwd_gqa(const void *q, const void *k, const void *v, void *out, flo
 
 /*
  * fa_fwd_varlen -- fa_fwd over a batch of sequences of different lengths
- * packed along the token axis (the pages' "Flash-Attention v2.0 到 v2.7 更新"
- * names the variable-length interface beside the fixed-shape one). The
- * pages give no separate formula: each sequence b is attended exactly as
- * fa_fwd would attend it alone, with its own Nq_b, Nk_b and the same
- * bottom-right causal alignment, window, ALiBi and softcap rules.
+ * packed along the token axis ("FlashAttention深度解析：从算法创新到产业变革的
+ * 全面影响", section 未来展望, names variable sequence lengths among the
+ * features being added). The pages give no formula for it: each sequence b
+ * is attended exactly as fa_fwd would attend it alone, with its own Nq_b,
+ * Nk_b and the same bottom-right causal alignment, window, ALiBi and
+ * softcap rules.
  *
  *   q    [total_q, H, d]  fp16/bf16, read; sequence b owns rows
  *                         cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1
@@ -212,7 +213,9 @@ fa_status fa_fwd_kvcache_gqa(const void *q, const void *k_cache, const void *v_c
  * fa_kvcache_append -- writes n_new new tokens per sequence into the paged
  * caches: token i of sequence b (k_new[b, i], v_new[b, i]) goes to position
  * t = cache_seqlens[b] + i, i.e. row t % page_size of page
- * block_table[b][t / page_size] ("Flash-Attention v2.0 到 v2.7 更新", v2.5).
+ * block_table[b][t / page_size] ("Flash-Attention v2.0 到 v2.7 更新", v2.5: the
+ * paged cache; "解密FlashAttention：如何让大语言模型推理速度翻倍", section
+ * 智能緩存機制: the key-value cache keeps the context already processed).
  * cache_seqlens is read, not updated: the caller advances it by n_new
  * before the next decode call.
  *
