@@ -175,7 +175,8 @@ def attn_fwd_gqa(q, k, v, scale: float, causal: bool = False, window_left: int =
                  rows: Optional[Sequence[int]] = None, num_threads: int = 0,
                  dtype_code: Optional[int] = None):
     """Grouped-query attention: q [B,Nq,H,d], k/v [B,Nk,H_kv,d]; query head h
-    attends with K/V head h // (H / H_kv). Returns (o [B,R,H,d], lse [B,H,R])."""
+    attends with K/V head h // (H / H_kv) (the pages do not define the form;
+    this is the plain reading). Returns (o [B,R,H,d], lse [B,H,R])."""
     qa, code = _as_storage(q, dtype_code)
     ka, kc = _as_storage(k, dtype_code)
     va, vc = _as_storage(v, dtype_code)
@@ -191,6 +192,9 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, causal: b
     sequence b owns query rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 and
     key rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1, and is attended on its
     own by the plain definition (attn_fwd with B = 1 and its own Nq, Nk).
+    "FlashAttention深度解析：从算法创新到产业变革的全面影响" (section 未来展望)
+    names variable sequence lengths without a formula; this is the reading
+    that each sequence is its own problem.
 
     Returns (o [total_q,H,d], lse [H,total_q]); rows outside every sequence
     are NaN.
@@ -283,7 +287,9 @@ def attn_decode_paged_gqa(q, k_cache, v_cache, block_table, cache_seqlens, scale
 def kvcache_append(k_new, v_new, k_cache, v_cache, block_table, cache_seqlens):
     """Returns copies of the caches with the new tokens written in: token i of
     sequence b goes to position t = cache_seqlens[b] + i, i.e. row
-    t % page_size of page block_table[b][t // page_size]; positions past
+    t % page_size of page block_table[b][t // page_size] ("Flash-Attention
+    v2.0 到 v2.7 更新", v2.5; "解密FlashAttention：如何让大语言模型推理速度翻倍",
+    section 智能緩存機制); positions past
     the table and entries outside [0, num_pages) are skipped. Works on the
     raw storage (any element type), so the result is bit-exact."""
     kn, vn = np.asarray(k_new), np.asarray(v_new)
