@@ -63,6 +63,10 @@ def _lib_handle():
         L.fa_fwd_kvcache_gqa.restype = i
         L.fa_kvcache_append.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp]
         L.fa_kvcache_append.restype = i
+        L.fa_fwd_qkvpacked.argtypes = [vp, vp, vp, i, i, i, i, i, f, i, i, i, vp, f, vp]
+        L.fa_fwd_qkvpacked.restype = i
+        L.fa_fwd_varlen_qkvpacked.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, f, vp]
+        L.fa_fwd_varlen_qkvpacked.restype = i
         L.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, i, i, vp, f, vp]
         L.fa_fwd_varlen.restype = i
         L.fa_fwd_kvcache.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp, f, i, vp, sz,
@@ -155,6 +159,43 @@ def fa_fwd_gqa(q, k, v, out, lse, scale: float, causal: bool = False, window_lef
                                     _dtype_code(q), float(scale), int(bool(causal)), int(window_left),
                                     int(window_right), _ptr(alibi_slopes), float(softcap), _stream(stream))
     _check(code, "fa_fwd_gqa")
+
+
+def fa_fwd_qkvpacked(qkv, out, lse, scale: float, causal: bool = False, window_left: int = -1,
+                     window_right: int = -1, alibi_slopes=None, softcap: float = 0.0, stream=None) -> None:
+    """qkv [B,N,3,H,d] (slot 0 q, 1 k, 2 v); out [B,N,H,d]; lse fp32 [B,H,N]; all on the device."""
+    B, N, three, H, d = qkv.shape
+    for t in (qkv, out, lse):
+        if not t.is_contiguous():
+            raise ValueError("fa_fwd_qkvpacked needs contiguous tensors")
+    if three != 3 or tuple(out.shape) != (B, N, H, d) or out.dtype != qkv.dtype:
+        raise ValueError("fa_fwd_qkvpacked: shape mismatch")
+    if tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32:
+        raise ValueError("fa_fwd_qkvpacked: lse must be fp32 [B, H, N]")
+    code = _lib_handle().fa_fwd_qkvpacked(_ptr(qkv), _ptr(out), _ptr(lse), B, H, N, d, _dtype_code(qkv),
+                                          float(scale), int(bool(causal)), int(window_left), int(window_right),
+                                          _ptr(alibi_slopes), float(softcap), _stream(stream))
+    _check(code, "fa_fwd_qkvpacked")
+
+
+def fa_fwd_varlen_qkvpacked(qkv, out, lse, cu_seqlens, max_seqlen: int, scale: float, causal: bool = False,
+                            window_left: int = -1, window_right: int = -1, alibi_slopes=None, softcap: float = 0.0,
+                            stream=None) -> None:
+    """qkv [total,3,H,d]; out [total,H,d]; lse fp32 [H,total]; cu_seqlens int32 [B+1] on the device."""
+    total, three, H, d = qkv.shape
+    B = cu_seqlens.numel() - 1
+    for t in (qkv, out, lse, cu_seqlens):
+        if not t.is_contiguous():
+            raise ValueError("fa_fwd_varlen_qkvpacked needs contiguous tensors")
+    if three != 3 or tuple(out.shape) != (total, H, d) or out.dtype != qkv.dtype:
+        raise ValueError("fa_fwd_varlen_qkvpacked: shape mismatch")
+    if tuple(lse.shape) != (H, total) or lse.dtype != torch.float32 or cu_seqlens.dtype != torch.int32:
+        raise ValueError("fa_fwd_varlen_qkvpacked: lse must be fp32 [H, total], cu_seqlens int32")
+    code = _lib_handle().fa_fwd_varlen_qkvpacked(_ptr(qkv), _ptr(out), _ptr(lse), _ptr(cu_seqlens), B, H,
+                                                 int(max_seqlen), total, d, _dtype_code(qkv), float(scale),
+                                                 int(bool(causal)), int(window_left), int(window_right),
+                                                 _ptr(alibi_slopes), float(softcap), _stream(stream))
+    _check(code, "fa_fwd_varlen_qkvpacked")
 
 
 def fa_fwd_varlen(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,

@@ -61,14 +61,15 @@ EncodeTiledFn encode_fn() {
 }
 
 // [B, N, H, d] 16-bit tensor as a 4-D map (d, H, N, B), box (64, 1, 128, 1),
-// 128-byte swizzle; rows past N read as zero.
-bool make_map(CUtensorMap* map, const void* base, bool bf16, int B, int N, int H, int d) {
+// 128-byte swizzle; rows past N read as zero. tok: elements from one token
+// to the next (H * d when contiguous; 3 * H * d inside a packed QKV tensor).
+bool make_map(CUtensorMap* map, const void* base, bool bf16, int B, int N, int H, int d, long long tok = 0) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t n = static_cast<cuuint64_t>(N > 0 ? N : 1);
+  const cuuint64_t t = static_cast<cuuint64_t>(tok > 0 ? tok : static_cast<long long>(H) * d);
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), n, static_cast<cuuint64_t>(B)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
-                           n * static_cast<cuuint64_t>(H) * d * 2};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, t * 2, n * t * 2};
   cuuint32_t box[4] = {64, 1, 128, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
@@ -128,10 +129,13 @@ namespace {
 // Shared body of fa_fwd and fa_fwd_varlen. Fixed length: cu_q == nullptr, the
 // maps cover [B, N, H, d]. Variable length: the maps cover one batch of
 // total rows and Nq, Nk are the maximum lengths.
+// tok_q, tok_kv: elements between consecutive tokens of q and of k/v (0 =
+// contiguous: H * d and H_kv * d).
 fa_status fwd_common(const void* q, const void* k, const void* v, void* out, float* lse, const int* cu_q,
                      const int* cu_k, int B, int H, int H_kv, int Nq, int Nk, int total_q, int total_k, int d,
                      fa_dtype dtype, float scale, int causal, int window_left, int window_right,
-                     const float* alibi_slopes, float softcap, cudaStream_t stream) {
+                     const float* alibi_slopes, float softcap, cudaStream_t stream, long long tok_q = 0,
+                     long long tok_kv = 0) {
   const bool varlen = cu_q != nullptr;
   if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || total_q < 0 || total_k < 0) return FA_ERR_SHAPE;
   if (H > 0 && (H_kv < 1 || H_kv > H || H % H_kv != 0)) return FA_ERR_SHAPE;
@@ -159,8 +163,8 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* out, flo
   const void* vb = any_k ? v : q;
   const int mb = varlen ? 1 : B;
   const int nq = varlen ? total_q : Nq, nk = varlen ? total_k : Nk;
-  if (!make_map(&tq, q, bf16, mb, nq, H, d) || !make_map(&tk, kb, bf16, mb, nk, H_kv, d) ||
-      !make_map(&tv, vb, bf16, mb, nk, H_kv, d))
+  if (!make_map(&tq, q, bf16, mb, nq, H, d, tok_q) || !make_map(&tk, kb, bf16, mb, nk, H_kv, d, tok_kv) ||
+      !make_map(&tv, vb, bf16, mb, nk, H_kv, d, tok_kv))
     return FA_ERR_CUDA;
 
   fa::FwdParams p{};
@@ -288,6 +292,30 @@ fa_status fa_fwd_gqa(const void* q, const void* k, const void* v, void* out, flo
                      int window_right, const float* alibi_slopes, float softcap, cudaStream_t stream) {
   return fwd_common(q, k, v, out, lse, nullptr, nullptr, B, H, H_kv, Nq, Nk, 0, 0, d, dtype, scale, causal,
                     window_left, window_right, alibi_slopes, softcap, stream);
+}
+
+fa_status fa_fwd_qkvpacked(const void* qkv, void* out, float* lse, int B, int H, int N, int d, fa_dtype dtype,
+                           float scale, int causal, int window_left, int window_right, const float* alibi_slopes,
+                           float softcap, cudaStream_t stream) {
+  const long long hd = static_cast<long long>(H) * d;
+  const char* base = static_cast<const char*>(qkv);
+  const void* k = base ? base + hd * 2 : nullptr;
+  const void* v = base ? base + 2 * hd * 2 : nullptr;
+  return fwd_common(qkv, k, v, out, lse, nullptr, nullptr, B, H, H, N, N, 0, 0, d, dtype, scale, causal,
+                    window_left, window_right, alibi_slopes, softcap, stream, 3 * hd, 3 * hd);
+}
+
+fa_status fa_fwd_varlen_qkvpacked(const void* qkv, void* out, float* lse, const int* cu_seqlens, int B, int H,
+                                  int max_seqlen, int total, int d, fa_dtype dtype, float scale, int causal,
+                                  int window_left, int window_right, const float* alibi_slopes, float softcap,
+                                  cudaStream_t stream) {
+  if (B > 0 && !cu_seqlens) return FA_ERR_NULL;
+  const long long hd = static_cast<long long>(H) * d;
+  const char* base = static_cast<const char*>(qkv);
+  const void* k = base ? base + hd * 2 : nullptr;
+  const void* v = base ? base + 2 * hd * 2 : nullptr;
+  return fwd_common(qkv, k, v, out, lse, cu_seqlens, cu_seqlens, B, H, H, max_seqlen, max_seqlen, total, total, d,
+                    dtype, scale, causal, window_left, window_right, alibi_slopes, softcap, stream, 3 * hd, 3 * hd);
 }
 
 fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse,

@@ -115,6 +115,33 @@ fa_status fa_fwd_gqa(const void *q, const void *k, const void *v, void *out, flo
                      const float *alibi_slopes, float softcap, cudaStream_t stream);
 
 /*
+ * fa_fwd_qkvpacked -- fa_fwd with Q, K and V packed in one tensor, the
+ * layout of the interface "FlashAttention深度解析：从算法创新到产业变革的全面
+ * 影响" names beside the separate one (flash_attn_qkvpacked_func):
+ *
+ *   qkv  [B, N, 3, H, d]  fp16/bf16, read; qkv[b, n, 0] is q[b, n],
+ *                         qkv[b, n, 1] is k[b, n], qkv[b, n, 2] is v[b, n]
+ *   out  [B, N, H, d]     written;  lse [B, H, N] fp32, written
+ *
+ * Nq = Nk = N; every other argument, limit and error as in fa_fwd. Nothing
+ * is copied: the kernel reads q, k and v in place through strided maps.
+ */
+fa_status fa_fwd_qkvpacked(const void *qkv, void *out, float *lse, int B, int H, int N, int d,
+                           fa_dtype dtype, float scale, int causal, int window_left, int window_right,
+                           const float *alibi_slopes, float softcap, cudaStream_t stream);
+
+/*
+ * fa_fwd_varlen_qkvpacked -- fa_fwd_varlen with Q, K and V packed:
+ * qkv [total, 3, H, d], out [total, H, d], lse [H, total]; one offset array
+ * cu_seqlens [B + 1] (device int32) for queries and keys alike, and one
+ * bound max_seqlen. Every other argument as in fa_fwd_varlen.
+ */
+fa_status fa_fwd_varlen_qkvpacked(const void *qkv, void *out, float *lse, const int *cu_seqlens,
+                                  int B, int H, int max_seqlen, int total, int d, fa_dtype dtype,
+                                  float scale, int causal, int window_left, int window_right,
+                                  const float *alibi_slopes, float softcap, cudaStream_t stream);
+
+/*
  * fa_fwd_varlen -- fa_fwd over a batch of sequences of different lengths
  * packed along the token axis ("FlashAttention深度解析：从算法创新到产业变革的
  * 全面影响", section 未来展望, names variable sequence lengths among the

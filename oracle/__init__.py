@@ -185,6 +185,20 @@ def attn_fwd_gqa(q, k, v, scale: float, causal: bool = False, window_left: int =
                     alibi_slopes, softcap, rows=rows, num_threads=num_threads, dtype_code=code)
 
 
+def attn_fwd_qkvpacked(qkv, scale: float, causal: bool = False, window_left: int = -1, window_right: int = -1,
+                       alibi_slopes=None, softcap: float = 0.0, rows: Optional[Sequence[int]] = None,
+                       num_threads: int = 0, dtype_code: Optional[int] = None):
+    """Packed layout of "FlashAttention深度解析：从算法创新到产业变革的全面影响"
+    (flash_attn_qkvpacked_func): qkv [B,N,3,H,d] with slot 0 = q, 1 = k,
+    2 = v; attention as attn_fwd on the three slots."""
+    a, code = _as_storage(qkv, dtype_code)
+    if a.ndim != 5 or a.shape[2] != 3:
+        raise ValueError("qkv must be [B, N, 3, H, d]")
+    q, k, v = (np.ascontiguousarray(a[:, :, i]) for i in range(3))
+    return attn_fwd(q, k, v, scale, causal, window_left, window_right, alibi_slopes, softcap, rows=rows,
+                    num_threads=num_threads, dtype_code=code)
+
+
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, causal: bool = False,
                     window_left: int = -1, window_right: int = -1, alibi_slopes=None, softcap: float = 0.0,
                     num_threads: int = 0, dtype_code: Optional[int] = None):

@@ -34,7 +34,7 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    assert {"fa_fwd", "fa_fwd_varlen", "fa_fwd_kvcache", "fa_kvcache_num_splits", "fa_kvcache_workspace_size",
+    assert {"fa_fwd", "fa_fwd_varlen", "fa_fwd_qkvpacked", "fa_fwd_kvcache", "fa_kvcache_num_splits", "fa_kvcache_workspace_size",
             "fa_status_string"} <= set(names)
 
 
@@ -227,3 +227,23 @@ def test_append_validation(lib):
     assert ap(bt=P + 2) == ARG
     assert ap(n=0, kn=None) == OK       # nothing to append
     assert ap() in (OK, DEVICE)
+
+
+def test_qkvpacked_validation(lib):
+    def pk(qkv=P, out=P, lse=P, B=1, H=2, N=128, d=128, dtype=1, cap=0.0, wl=-1):
+        return lib.fa_fwd_qkvpacked(qkv, out, lse, B, H, N, d, dtype, 0.1, 1, wl, -1, None, cap, None)
+    assert pk(d=96) == HEADDIM
+    assert pk(dtype=4) == DTYPE
+    assert pk(N=-1) == SHAPE
+    assert pk(qkv=None) == NULL
+    assert pk(lse=None) == NULL
+    assert pk(cap=-1.0) == ARG
+    assert pk(B=0, qkv=None) == OK
+    assert pk() in (OK, DEVICE)
+
+    def vpk(qkv=P, cu=P, B=2, total=300, mx=200):
+        return lib.fa_fwd_varlen_qkvpacked(qkv, P, P, cu, B, 2, mx, total, 128, 1, 0.1, 1, -1, -1, None, 0.0, None)
+    assert vpk(cu=None) == NULL
+    assert vpk(total=-5) == SHAPE
+    assert vpk(total=0) == OK
+    assert vpk() in (OK, DEVICE)

@@ -546,3 +546,15 @@ def test_append_writes_tokens_where_the_table_says():
                 assert np.array_equal(k2[pg, row], kn[b, i]) and np.array_equal(v2[pg, row], vn[b, i])
             else:
                 assert np.array_equal(k2[pg, row], kc[pg, row]) and np.array_equal(v2[pg, row], vc[pg, row])
+
+
+def test_qkvpacked_slots_are_q_k_v():
+    # distinct q, k, v packed along axis 2 must give exactly the separate
+    # call; swapping any two slots changes the result
+    B, N, H, d = 2, 6, 2, 4
+    q, k, v = rnd((B, N, H, d), 81), rnd((B, N, H, d), 82), rnd((B, N, H, d), 83)
+    o, lse = oracle.attn_fwd(q, k, v, 0.5, causal=True)
+    op, lp = oracle.attn_fwd_qkvpacked(np.stack([q, k, v], axis=2), 0.5, causal=True)
+    assert np.array_equal(o, op) and np.array_equal(lse, lp)
+    ow, _ = oracle.attn_fwd_qkvpacked(np.stack([k, q, v], axis=2), 0.5, causal=True)
+    assert not np.allclose(ow, o)
