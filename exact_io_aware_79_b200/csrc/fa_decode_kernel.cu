@@ -530,26 +530,35 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, G > 1 ? 3 : 2)
       }
     }
   } else {
-    // ---------------- consumers, one head per lane group
+    // ---------------- consumers, one head: the kSteps partial dot products a
+    // lane holds for its token group are reduce-scattered over the group's
+    // LPT lanes, so lane cl ends with the full score of step cl / R (R = LPT /
+    // kSteps lanes share a step); scores, the running max and the sum are
+    // then worked once per token instead of on every lane, and the step's
+    // probability is broadcast back to the group for the V update.
+    static_assert(G == 1, "grouped-query CTAs take the branch above");
+    static_assert(LPT % kSteps == 0, "a token group needs a lane per step");
+    constexpr int R = LPT / kSteps;
     const int g = lane / LPT;
     const int cl = lane % LPT;
+    const int gbase = lane & ~(LPT - 1);
+    const int my_st = cl / R;  // the step whose score this lane ends up with
     const float qscale = p.use_softcap ? p.cap_scale : p.scale_log2;
     const bool alibi = p.slopes != nullptr;
-    float qf[G][8], slope_l2[G];
-    float m[G], lsum[G], acc[G][8];
-#pragma unroll
-    for (int gi = 0; gi < G; ++gi) {
+    uint64_t q2[4], acc2[4];
+    {
+      float qf[8];
       widen8<T>(*reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.q) +
-                                                (static_cast<size_t>(b) * p.H + h0 + gi) * D + cl * 8),
-                qf[gi]);
+                                                (static_cast<size_t>(b) * p.H + h0) * D + cl * 8),
+                qf);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) qf[gi][e] *= qscale;
-      slope_l2[gi] = alibi ? p.slopes[h0 + gi] * kLog2e : 0.0f;
-      m[gi] = -INFINITY;
-      lsum[gi] = 0.0f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[gi][e] = 0.0f;
+      for (int e = 0; e < 4; ++e) {
+        q2[e] = f2_pack(qf[2 * e] * qscale, qf[2 * e + 1] * qscale);
+        acc2[e] = 0;  // +0.0f pair
+      }
     }
+    const float slope_l2 = alibi ? p.slopes[h0] * kLog2e : 0.0f;
+    float m = -INFINITY, lsum = 0.0f;  // lsum: this lane's steps only
 
     for (int i = 0; i < n_st; ++i) {
       const int slot = i % NST;
@@ -565,93 +574,92 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, G > 1 ? 3 : 2)
         const T* kt = reinterpret_cast<const T*>(sK + slot * C::kTile);
         const T* vt = reinterpret_cast<const T*>(sV + slot * C::kTile);
         const int a = a0 + i * kRows;
-        // scores of every head for this warp's tokens; each K row is
-        // widened once and serves all G heads
-        float sc[G][kSteps];
-        float mt[G];
-#pragma unroll
-        for (int gi = 0; gi < G; ++gi) mt[gi] = -INFINITY;
+        float dv[kSteps];
 #pragma unroll
         for (int st = 0; st < kSteps; ++st) {
           const int r = warp * (kRows / kWarps) + st * TPW + g;
           float kf[8];
           widen8<T>(*reinterpret_cast<const uint4*>(kt + r * D + cl * 8), kf);
-          const int tok = a + r;
-          const bool vis = tok >= t0 && tok < t1;
+          uint64_t d2 = f2_mul(q2[0], f2_pack(kf[0], kf[1]));
 #pragma unroll
-          for (int gi = 0; gi < G; ++gi) {
-            float dot = 0.0f;
+          for (int e = 1; e < 4; ++e) d2 = f2_fma(q2[e], f2_pack(kf[2 * e], kf[2 * e + 1]), d2);
+          float d0, d1;
+          f2_unpack(d2, d0, d1);
+          dv[st] = d0 + d1;
+        }
+        // reduce-scatter: at each level the lane keeps the half of its steps
+        // named by its lane bit and adds the partner's copy of that half
 #pragma unroll
-            for (int e = 0; e < 8; ++e) dot = fmaf(qf[gi][e], kf[e], dot);
+        for (int n = kSteps, off = LPT / 2; n > 1; n >>= 1, off >>= 1) {
+          const bool up = (cl & off) != 0;
 #pragma unroll
-            for (int o = LPT / 2; o >= 1; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-            float t = p.use_softcap ? p.cap_log2 * tanh_via_exp2(dot) : dot;
-            if (alibi) t -= slope_l2[gi] * static_cast<float>(pos - tok);
-            sc[gi][st] = vis ? t : -INFINITY;
-            mt[gi] = fmaxf(mt[gi], sc[gi][st]);
+          for (int j = 0; j < n / 2; ++j) {
+            const float keep = up ? dv[j + n / 2] : dv[j];
+            const float send = up ? dv[j] : dv[j + n / 2];
+            dv[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
           }
         }
-        float mn[G], pw[G][kSteps];
 #pragma unroll
-        for (int gi = 0; gi < G; ++gi) {
-          mn[gi] = fmaxf(m[gi], mt[gi]);
-          if (mn[gi] != -INFINITY) {
-            const float alpha = ex2(m[gi] - mn[gi]);
-            lsum[gi] *= alpha;
+        for (int off = R / 2; off >= 1; off >>= 1) dv[0] += __shfl_xor_sync(0xffffffffu, dv[0], off);
+        const int tok = a + warp * (kRows / kWarps) + my_st * TPW + g;
+        float t = p.use_softcap ? p.cap_log2 * tanh_via_exp2(dv[0]) : dv[0];
+        if (alibi) t -= slope_l2 * static_cast<float>(pos - tok);
+        const float sc = (tok >= t0 && tok < t1) ? t : -INFINITY;
+        float mt = sc;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[gi][e] *= alpha;
+        for (int off = R; off < LPT; off <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+        const float mn = fmaxf(m, mt);
+        const bool live = mn != -INFINITY;  // uniform over the token group
+        const float alpha = live ? ex2(m - mn) : 1.0f;
+        const float pw = live ? ex2(sc - mn) : 0.0f;
+        lsum = lsum * alpha + pw;
+        m = live ? mn : m;
+        const uint64_t al2 = f2_pack(alpha, alpha);
 #pragma unroll
-            for (int st = 0; st < kSteps; ++st) {
-              pw[gi][st] = ex2(sc[gi][st] - mn[gi]);
-              lsum[gi] += pw[gi][st];
-            }
-            m[gi] = mn[gi];
-          } else {
-#pragma unroll
-            for (int st = 0; st < kSteps; ++st) pw[gi][st] = 0.0f;
-          }
-        }
+        for (int e = 0; e < 4; ++e) acc2[e] = f2_mul(acc2[e], al2);
 #pragma unroll
         for (int st = 0; st < kSteps; ++st) {
           const int r = warp * (kRows / kWarps) + st * TPW + g;
           float vf[8];
           widen8<T>(*reinterpret_cast<const uint4*>(vt + r * D + cl * 8), vf);
+          const float ps = __shfl_sync(0xffffffffu, pw, gbase + st * R);
+          const uint64_t p2 = f2_pack(ps, ps);
 #pragma unroll
-          for (int gi = 0; gi < G; ++gi) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[gi][e] = fmaf(pw[gi][st], vf[e], acc[gi][e]);
-          }
+          for (int e = 0; e < 4; ++e) acc2[e] = f2_fma(f2_pack(vf[2 * e], vf[2 * e + 1]), p2, acc2[e]);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->empty[slot]);
     }
-    // merge the lane groups of this warp, then publish the warp's state
+    // the group's sum over its distinct steps, then merge the token groups of
+    // this warp and publish the warp's state
 #pragma unroll
-    for (int gi = 0; gi < G; ++gi) {
+    for (int off = R; off < LPT; off <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+    float acc[8];
 #pragma unroll
-      for (int o = LPT; o < 32; o <<= 1) {
-        const float m_o = __shfl_xor_sync(0xffffffffu, m[gi], o);
-        const float l_o = __shfl_xor_sync(0xffffffffu, lsum[gi], o);
-        const float mm = fmaxf(m[gi], m_o);
-        const float x = (m[gi] == -INFINITY) ? 0.0f : ex2(m[gi] - mm);
-        const float x_o = (m_o == -INFINITY) ? 0.0f : ex2(m_o - mm);
-        lsum[gi] = lsum[gi] * x + l_o * x_o;
+    for (int e = 0; e < 4; ++e) f2_unpack(acc2[e], acc[2 * e], acc[2 * e + 1]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float a_o = __shfl_xor_sync(0xffffffffu, acc[gi][e], o);
-          acc[gi][e] = acc[gi][e] * x + a_o * x_o;
-        }
-        m[gi] = mm;
+    for (int o = LPT; o < 32; o <<= 1) {
+      const float m_o = __shfl_xor_sync(0xffffffffu, m, o);
+      const float l_o = __shfl_xor_sync(0xffffffffu, lsum, o);
+      const float mm = fmaxf(m, m_o);
+      const float x = (m == -INFINITY) ? 0.0f : ex2(m - mm);
+      const float x_o = (m_o == -INFINITY) ? 0.0f : ex2(m_o - mm);
+      lsum = lsum * x + l_o * x_o;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float a_o = __shfl_xor_sync(0xffffffffu, acc[e], o);
+        acc[e] = acc[e] * x + a_o * x_o;
       }
-      if (lane < LPT) {
+      m = mm;
+    }
+    if (lane < LPT) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) sh->acc[warp][gi][cl * 8 + e] = acc[gi][e];
-      }
-      if (lane == 0) {
-        sh->m[warp][gi] = m[gi];
-        sh->l[warp][gi] = lsum[gi];
-      }
+      for (int e = 0; e < 8; ++e) sh->acc[warp][0][cl * 8 + e] = acc[e];
+    }
+    if (lane == 0) {
+      sh->m[warp][0] = m;
+      sh->l[warp][0] = lsum;
     }
   }
   const bool any_bad = __syncthreads_or(bad) != 0;

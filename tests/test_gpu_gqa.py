@@ -69,35 +69,39 @@ def decode_inputs(B, H, H_kv, d, page, mb, lens, dtype, seed):
     return q, kc, vc, table, torch.tensor(lens, dtype=torch.int32)
 
 
-def run_decode_gqa(q, kc, vc, table, lens, scale, splits=0, wl=-1):
+def run_decode_gqa(q, kc, vc, table, lens, scale, splits=0, wl=-1, slopes=None, cap=0.0):
     B, _, H, d = q.shape
     mb, page = table.shape[1], kc.shape[1]
     nbytes = fa.fa_kvcache_workspace_size(B, H, d, mb, page, splits)
     ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device="cuda")
     out = torch.empty(q.shape, dtype=q.dtype, device="cuda")
     lse = torch.empty(B, H, 1, dtype=torch.float32, device="cuda")
-    fa.fa_fwd_kvcache_gqa(q.cuda(), kc.cuda(), vc.cuda(), table.cuda(), lens.cuda(), out, lse, scale, wl, None, 0.0,
-                          splits, ws)
+    fa.fa_fwd_kvcache_gqa(q.cuda(), kc.cuda(), vc.cuda(), table.cuda(), lens.cuda(), out, lse, scale, wl,
+                          None if slopes is None else slopes.cuda(), cap, splits, ws)
     torch.cuda.synchronize()
     return out.float().cpu().numpy(), lse.cpu().numpy()
 
 
 DEC = [
-    # (B, H, H_kv, d, page, mb, lens, dtype, wl)
-    (3, 8, 2, 128, 256, 8, (2048, 300, 1), torch.bfloat16, -1),
-    (2, 4, 1, 64, 16, 20, (320, 77), torch.float16, -1),
-    (4, 6, 3, 128, 64, 12, (700, 0, 65, 768), torch.bfloat16, 100),
+    # (B, H, H_kv, d, page, mb, lens, dtype, wl, alibi, cap)
+    (3, 8, 2, 128, 256, 8, (2048, 300, 1), torch.bfloat16, -1, False, 0.0),
+    (2, 4, 1, 64, 16, 20, (320, 77), torch.float16, -1, False, 0.0),
+    (4, 6, 3, 128, 64, 12, (700, 0, 65, 768), torch.bfloat16, 100, False, 0.0),
+    (2, 8, 2, 128, 256, 6, (1500, 257), torch.bfloat16, -1, True, 30.0),     # four heads a CTA, ALiBi + softcap
+    (2, 4, 2, 64, 64, 10, (600, 90), torch.float16, 200, True, 0.0),         # two heads a CTA, ALiBi, window
+    (2, 8, 1, 128, 128, 4, (500, 33), torch.bfloat16, -1, False, 5.0),       # MQA (four heads a CTA), softcap
 ]
 
 
 @pytest.mark.parametrize("splits", [0, 1, 3, 8])
-@pytest.mark.parametrize("case", DEC, ids=lambda c: "B%dH%dkv%dd%dp%d" % c[:5])
+@pytest.mark.parametrize("case", DEC, ids=lambda c: "B%dH%dkv%dd%dp%d_a%d_s%g" % (c[:5] + (c[9], c[10])))
 def test_decode_gqa_matches_oracle(case, splits):
-    B, H, H_kv, d, page, mb, lens, dtype, wl = case
+    B, H, H_kv, d, page, mb, lens, dtype, wl, alibi, cap = case
     q, kc, vc, table, lens_t = decode_inputs(B, H, H_kv, d, page, mb, lens, dtype, seed=sum(lens) + H)
+    slopes = W.alibi_slopes(H) if alibi else None
     scale = 1.0 / math.sqrt(d)
-    out, lse = run_decode_gqa(q, kc, vc, table, lens_t, scale, splits, wl)
-    o_ref, l_ref = oracle.attn_decode_paged_gqa(q, kc, vc, table, lens_t, scale, wl)
+    out, lse = run_decode_gqa(q, kc, vc, table, lens_t, scale, splits, wl, slopes, cap)
+    o_ref, l_ref = oracle.attn_decode_paged_gqa(q, kc, vc, table, lens_t, scale, wl, slopes, cap)
     compare(out, lse, o_ref, l_ref, dtype, "%s splits=%d" % (case, splits))
 
 
