@@ -48,7 +48,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Decode: a capture of the 4-sequence case read 1.003 x its K/V bytes and
 # wrote 2.8 MB of partials (profiles/decode_split_tma_paged_decode_b4h32d128_page256.md);
 # reads scale with the K/V bytes, each byte being read once.
-DECODE_READ_PER_KV_BYTE = 967926912.0 / 965165056.0  # (967,919,616 + 967,934,208) / 2 / K/V bytes
+DECODE_READ_PER_KV_BYTE = 967959936.0 / 965165056.0  # (968,019,712 + 967,900,160) / 2 / K/V bytes
 # Forward, causal B8 H16 N2048 d128: mean of two captured launches
 # (profiles/fwd_kernel_causal_b8h16n2048d128.md, last table).
 FWD_CAUSAL_2K_TRAFFIC = (201453056.0 + 38760448.0 + 201453312.0 + 35730432.0) / 2.0

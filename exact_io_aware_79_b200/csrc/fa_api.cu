@@ -80,20 +80,22 @@ bool make_map(CUtensorMap* map, const void* base, bool bf16, int B, int N, int H
 }
 
 // Paged cache [num_pages, page_size, H, d] as a 4-D map (d, H, page_size,
-// num_pages) with a (d, 1, 64, 1) box and no swizzle: one box is a 64-token
-// slice of one page for one head.
-bool make_cache_map(CUtensorMap* map, const void* base, bool bf16, int num_pages, int page_size, int H, int d) {
+// num_pages). One box is a 64-token slice of one page for one head: all d
+// columns without swizzle, or (swizzled) 64 columns with 128-byte swizzle.
+bool make_cache_map(CUtensorMap* map, const void* base, bool bf16, int num_pages, int page_size, int H, int d,
+                    bool swizzled) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(page_size), static_cast<cuuint64_t>(num_pages)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
                            static_cast<cuuint64_t>(page_size) * H * d * 2};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(d), 1, 64, 1};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(swizzled ? 64 : d), 1, 64, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         swizzled ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -253,8 +255,9 @@ fa_status kvcache_common(const void* q, const void* k_cache, const void* v_cache
   const bool bf16 = dtype == FA_BF16;
   if (page_size % 64 == 0) {
     CUtensorMap tk, tv;
-    if (!make_cache_map(&tk, k_cache, bf16, num_pages, page_size, H_kv, d) ||
-        !make_cache_map(&tv, v_cache, bf16, num_pages, page_size, H_kv, d))
+    const bool sw = fa::decode_on_tensor_cores(H, H_kv);
+    if (!make_cache_map(&tk, k_cache, bf16, num_pages, page_size, H_kv, d, sw) ||
+        !make_cache_map(&tv, v_cache, bf16, num_pages, page_size, H_kv, d, sw))
       return FA_ERR_CUDA;
     return fa::launch_decode(bf16, d, p, &tk, &tv, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
   }

@@ -61,9 +61,14 @@ struct DecodeParams {
 cudaError_t launch_fwd(bool bf16, int d, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                        const FwdParams& p, cudaStream_t stream);
 
-// tmK/tmV: 4-D maps (d, H, page_size, num_pages) of the caches with a
-// (d, 1, 64, 1) box for the TMA-staged split kernel (page_size % 64 == 0), or
-// nullptr for the direct-load split kernel.
+// Grouped-query caches (two or more query heads per cache head) take the
+// tensor-core split kernel; it wants 128-byte-swizzled (64, 1, 64, 1) boxes.
+inline bool decode_on_tensor_cores(int H, int H_kv) { return H_kv > 0 && H / H_kv >= 2; }
+
+// tmK/tmV: 4-D maps (d, H, page_size, num_pages) of the caches for the
+// TMA-staged split kernels (page_size % 64 == 0): a (d, 1, 64, 1) box without
+// swizzle, or (64, 1, 64, 1) boxes with 128-byte swizzle when
+// decode_on_tensor_cores(H, H_kv); nullptr for the direct-load split kernel.
 cudaError_t launch_decode(bool bf16, int d, const DecodeParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
                           cudaStream_t stream);
 

@@ -377,4 +377,43 @@ __device__ __forceinline__ float2 unpack2<__half>(uint32_t u) {
   return __half22float2(v);
 }
 
+// ------------------------------------------------------------------ warp-level MMA
+
+// D = A * B + D for one m16n8k16 tile: A 16x16 row-major in four registers
+// (a[0]: row g, k 2t..2t+1; a[1]: row g+8; a[2]: row g, k 2t+8..2t+9;
+// a[3]: row g+8, k 2t+8..; g = lane / 4, t = lane % 4), B 16x8 column-major
+// in two (b0: k 2t..2t+1, n g; b1: k 2t+8..2t+9), D 16x8 fp32 (d[0..1]: row
+// g, n 2t..2t+1; d[2..3]: row g+8).
+template <typename T>
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1);
+
+template <>
+__device__ __forceinline__ void mma_16816<__nv_bfloat16>(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                                         uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <>
+__device__ __forceinline__ void mma_16816<__half>(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Four transposed 8x8 16-bit matrices from shared memory: lane l gives the
+// address of row l % 8 of matrix l / 8 (16 contiguous bytes); r[i] of lane
+// (g, t) holds elements (2t, g) and (2t+1, g) of matrix i.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+
 }  // namespace fa

@@ -137,7 +137,12 @@ FWD_WORKLOADS = [TINY, CAUSAL_2K, WINDOW_16K, WINDOW_Q4K_K16K, CAUSAL_Q4K_K16K, 
 DECODE_GQA = DecodeWorkload("paged_decode_gqa_bf16_b64h32kv8d128_page256", 64, 32, 128, torch.bfloat16,
                             page_size=256, len_lo=1024, len_hi=32768, seed=4, H_kv=8)
 
-DECODE_WORKLOADS = [DECODE, DECODE_SMALL, DECODE_GQA]
+# The grouped-query decode with 4 sequences (241 MB of unique K/V, above the
+# 126 MB L2): the profiler-capture size of DECODE_GQA.
+DECODE_GQA_SMALL = DecodeWorkload("paged_decode_gqa_bf16_b4h32kv8d128_page256", 4, 32, 128, torch.bfloat16,
+                                  page_size=256, len_lo=1024, len_hi=32768, seed=4, H_kv=8)
+
+DECODE_WORKLOADS = [DECODE, DECODE_SMALL, DECODE_GQA, DECODE_GQA_SMALL]
 
 
 def alibi_slopes(H: int) -> torch.Tensor:

@@ -89,7 +89,10 @@ DEC = [
     (4, 6, 3, 128, 64, 12, (700, 0, 65, 768), torch.bfloat16, 100, False, 0.0),
     (2, 8, 2, 128, 256, 6, (1500, 257), torch.bfloat16, -1, True, 30.0),     # four heads a CTA, ALiBi + softcap
     (2, 4, 2, 64, 64, 10, (600, 90), torch.float16, 200, True, 0.0),         # two heads a CTA, ALiBi, window
-    (2, 8, 1, 128, 128, 4, (500, 33), torch.bfloat16, -1, False, 5.0),       # MQA (four heads a CTA), softcap
+    (2, 8, 1, 128, 128, 4, (500, 33), torch.bfloat16, -1, False, 5.0),       # MQA, eight heads a CTA, softcap
+    (2, 32, 1, 128, 64, 6, (350, 129), torch.bfloat16, -1, True, 20.0),      # MQA, 16 heads a CTA (both row halves)
+    (2, 12, 1, 64, 64, 5, (300, 64), torch.float16, -1, False, 0.0),         # 12 heads a CTA
+    (2, 6, 2, 128, 128, 3, (380, 1), torch.bfloat16, 50, False, 0.0),        # an odd group of 3, window
 ]
 
 
@@ -166,3 +169,24 @@ def test_full_size_gqa_decode_sampled_sequences():
         o_ref, l_ref = oracle.attn_decode_paged_gqa(xd["q"][b:b + 1].cpu(), kc, vc, ident, lens[b:b + 1], w.scale)
         compare(out[b:b + 1].float().cpu().numpy(), lse[b:b + 1].cpu().numpy(), o_ref, l_ref, w.dtype,
                 "sequence %d (splits %d)" % (b, S))
+
+
+@pytest.mark.parametrize("H_kv", [8, 2, 1])
+def test_decode_staged_invalid_table_entry_and_length_give_nan_rows(H_kv):
+    """Page size 64 (the TMA-staged kernels, one head or a group a CTA): a
+    table entry past the pool and a length past the table are never
+    dereferenced; those sequences' rows become NaN and the others match the
+    oracle."""
+    B, H, d, page, mb = 4, 8, 128, 64, 4
+    q, kc, vc, table, lens = decode_inputs(B, H, H_kv, d, page, mb, (100, 200, 60, 7), torch.bfloat16, seed=9)
+    bad_table = table.clone()
+    bad_table[1, 2] = 10**6          # inside sequence 1's 200 tokens
+    bad_lens = lens.clone()
+    bad_lens[2] = mb * page + 1
+    for splits in (1, 4):
+        out, lse = run_decode_gqa(q, kc, vc, bad_table, bad_lens, 0.1, splits)
+        assert np.isnan(out[1]).all() and np.isnan(lse[1]).all()
+        assert np.isnan(out[2]).all() and np.isnan(lse[2]).all()
+        good = [0, 3]
+        o_ref, l_ref = oracle.attn_decode_paged_gqa(q[good], kc, vc, table[good], lens[good], 0.1)
+        compare(out[good], lse[good], o_ref, l_ref, torch.bfloat16, "good rows, splits=%d" % splits)
