@@ -326,6 +326,62 @@ def kvcache_append(k_new, v_new, k_cache, v_cache, block_table, cache_seqlens):
     return kc, vc
 
 
+def attn_bwd(q, k, v, dout, scale: float, causal: bool = False, window_left: int = -1,
+             window_right: int = -1, alibi_slopes=None, softcap: float = 0.0,
+             num_threads: int = 0, dtype_code: Optional[int] = None):
+    """Gradients of L = sum(dout * O) with respect to q, k and v, where O is
+    attn_fwd's output (grouped-query when k, v have fewer heads than q).
+
+    The pages name the backward pass ("FlashAttention深度解析：从算法创新到产业
+    变革的全面影响", section 技术演进, version 2.4; "Flash-Attention v2.0 到 v2.7
+    更新", section v2.4: a deterministic backward) but give no formulas, so
+    this is the chain rule through attn_fwd's definition, per (b, h):
+      dV = P^T dO;  dP = dO V^T
+      dZ_ij = P_ij (dP_ij - sum_k P_ik dP_ik)         (softmax Jacobian)
+      dS_ij = dZ_ij * (1 - tanh(s_ij / c)^2)          if softcap c > 0, else dZ_ij
+      dQ = scale * dS K;  dK = scale * dS^T Q
+    with s_ij = scale * q_i . k_j and P the probabilities of attn_fwd (masked
+    entries 0; the ALiBi term does not depend on q or k). Grouped-query K/V
+    heads receive the sum over the query heads that read them.
+
+    q, dout [B,Nq,H,d]; k, v [B,Nk,H_kv,d]. Returns (dq, dk, dv) as fp64
+    arrays of the input shapes.
+    """
+    qa, code = _as_storage(q, dtype_code)
+    ka, kc = _as_storage(k, dtype_code)
+    va, vc = _as_storage(v, dtype_code)
+    da, dc = _as_storage(dout, dtype_code)
+    if not (code == kc == vc == dc):
+        raise ValueError("q, k, v, dout must share one storage type")
+    B, Nq, H, d = qa.shape
+    Nk, H_kv = ka.shape[1], ka.shape[2]
+    if da.shape != qa.shape or va.shape != ka.shape or ka.shape[0] != B or ka.shape[3] != d:
+        raise ValueError("shape mismatch")
+    ke, ve = _expand_heads(ka, H, 2), _expand_heads(va, H, 2)
+    _, _, P = attn_fwd(qa, ke, ve, scale, causal, window_left, window_right, alibi_slopes, softcap,
+                       return_probs=True, num_threads=num_threads, dtype_code=code)
+    Q, K, V, DO = widen(qa, code), widen(ke, code), widen(ve, code), widen(da, code)
+    dq = np.zeros((B, Nq, H, d))
+    dk = np.zeros((B, Nk, H, d))
+    dv = np.zeros((B, Nk, H, d))
+    for b in range(B):
+        for h in range(H):
+            p = np.nan_to_num(P[b, h], nan=0.0)   # rows with no visible key carry no gradient
+            qh, kh, vh, doh = Q[b, :, h], K[b, :, h], V[b, :, h], DO[b, :, h]
+            dv[b, :, h] = p.T @ doh
+            dp = doh @ vh.T
+            dz = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+            if softcap > 0.0:
+                t = np.tanh(scale * (qh @ kh.T) / softcap)
+                dz = dz * (1.0 - t * t)
+            dq[b, :, h] = scale * (dz @ kh)
+            dk[b, :, h] = scale * (dz.T @ qh)
+    G = H // H_kv
+    dk = dk.reshape(B, Nk, H_kv, G, d).sum(axis=3)
+    dv = dv.reshape(B, Nk, H_kv, G, d).sum(axis=3)
+    return dq, dk, dv
+
+
 def combine_splits(o_part: np.ndarray, lse_part: np.ndarray):
     """Merge of split partials: o_part [S, ..., d], lse_part [S, ...]."""
     S = o_part.shape[0]

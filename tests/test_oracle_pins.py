@@ -558,3 +558,87 @@ def test_qkvpacked_slots_are_q_k_v():
     assert np.array_equal(o, op) and np.array_equal(lse, lp)
     ow, _ = oracle.attn_fwd_qkvpacked(np.stack([k, q, v], axis=2), 0.5, causal=True)
     assert not np.allclose(ow, o)
+
+
+# ---------------------------------------------------------------- backward
+
+def _loss(q, k, v, dout, scale, **opts):
+    o, _ = oracle.attn_fwd_gqa(q, k, v, scale, **opts)
+    return float(np.sum(dout * o))
+
+
+def _finite_difference(x, f, eps=1e-6):
+    g = np.zeros_like(x)
+    for idx in np.ndindex(x.shape):
+        old = x[idx]
+        x[idx] = old + eps
+        fp = f()
+        x[idx] = old - eps
+        fm = f()
+        x[idx] = old
+        g[idx] = (fp - fm) / (2 * eps)
+    return g
+
+
+@pytest.mark.parametrize("H_kv", [2, 1])
+@pytest.mark.parametrize("opts", [
+    {},
+    {"causal": True},
+    {"causal": True, "window_left": 2, "window_right": 0},
+    {"window_left": 1, "window_right": 2},
+    {"causal": True, "alibi_slopes": [0.5, 0.125], "softcap": 1.5},
+    {"alibi_slopes": [0.25, 1.0], "softcap": 0.7},
+], ids=lambda o: "-".join(sorted(o)) or "plain")
+def test_bwd_matches_finite_differences_of_the_forward(opts, H_kv):
+    """Each gradient entry against a central difference of L = sum(dout * O)
+    taken through the forward oracle alone (fp64 inputs): a wrong sign, a
+    transposed product, a dropped softmax-Jacobian term, a missing softcap
+    factor or a group sum over the wrong heads all fail here."""
+    B, H, Nq, Nk, d, scale = 1, 2, 5, 7, 4, 0.7
+    q, k, v = rnd((B, Nq, H, d), 61), rnd((B, Nk, H_kv, d), 62), rnd((B, Nk, H_kv, d), 63)
+    dout = rnd((B, Nq, H, d), 64)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, dout, scale, **opts)
+    f = lambda: _loss(q, k, v, dout, scale, **opts)
+    for got, x, name in ((dq, q, "dq"), (dk, k, "dk"), (dv, v, "dv")):
+        want = _finite_difference(x, f)
+        assert np.abs(got - want).max() < 1e-7, name
+
+
+def test_bwd_single_key_closed_form():
+    """One key: every row's softmax is the constant 1, so O_i = v_0 whatever
+    q and k are: dq = dk = 0 and dv = sum_i dout_i."""
+    B, H, Nq, d = 2, 3, 6, 5
+    q, k, v = rnd((B, Nq, H, d), 71), rnd((B, 1, H, d), 72), rnd((B, 1, H, d), 73)
+    dout = rnd((B, Nq, H, d), 74)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, dout, 0.9)
+    assert np.abs(dq).max() < TOL and np.abs(dk).max() < TOL
+    assert np.abs(dv[:, 0] - dout.sum(axis=1)).max() < 1e-12
+
+
+def test_bwd_zero_query_closed_form():
+    """q = 0 and no mask: P is uniform 1/Nk. Then dv_j = mean-free sum of
+    dout over rows / Nk, dk = 0 (it is scale * dS^T q), and dq_i = (scale/Nk)
+    sum_j (dout_i . v_j - mean_k dout_i . v_k) k_j."""
+    B, H, Nq, Nk, d, scale = 1, 2, 4, 6, 3, 0.8
+    q = np.zeros((B, Nq, H, d))
+    k, v, dout = rnd((B, Nk, H, d), 81), rnd((B, Nk, H, d), 82), rnd((B, Nq, H, d), 83)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, dout, scale)
+    assert np.abs(dk).max() < TOL
+    for h in range(H):
+        assert np.abs(dv[0, :, h] - dout[0, :, h].sum(axis=0) / Nk).max() < 1e-12
+        a = dout[0, :, h] @ v[0, :, h].T                       # [Nq, Nk]
+        want = scale / Nk * ((a - a.mean(axis=1, keepdims=True)) @ k[0, :, h])
+        assert np.abs(dq[0, :, h] - want).max() < 1e-12
+
+
+def test_bwd_rows_without_keys_carry_no_gradient():
+    """Causal with Nq > Nk: the first Nq - Nk rows see no key; their dq is 0
+    and they add nothing to dk, dv."""
+    B, H, Nq, Nk, d = 1, 1, 6, 3, 4
+    q, k, v, dout = rnd((B, Nq, H, d), 91), rnd((B, Nk, H, d), 92), rnd((B, Nk, H, d), 93), rnd((B, Nq, H, d), 94)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, dout, 0.5, causal=True)
+    assert np.all(dq[:, :Nq - Nk] == 0.0)
+    dout2 = dout.copy()
+    dout2[:, :Nq - Nk] = 123.0
+    _, dk2, dv2 = oracle.attn_bwd(q, k, v, dout2, 0.5, causal=True)
+    assert np.abs(dk2 - dk).max() < TOL and np.abs(dv2 - dv).max() < TOL
