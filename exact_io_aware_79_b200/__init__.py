@@ -79,6 +79,10 @@ def _lib_handle():
         L.fa_kvcache_num_splits.restype = i
         L.fa_kvcache_workspace_size.argtypes = [i, i, i, i, i, i]
         L.fa_kvcache_workspace_size.restype = sz
+        L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+        L.fa_bwd_workspace_size.restype = sz
+        L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i, vp, f, vp, sz, vp]
+        L.fa_bwd.restype = i
         L.fa_status_string.argtypes = [i]
         L.fa_status_string.restype = ctypes.c_char_p
         _LIB = L
@@ -159,6 +163,41 @@ def fa_fwd_gqa(q, k, v, out, lse, scale: float, causal: bool = False, window_lef
                                     _dtype_code(q), float(scale), int(bool(causal)), int(window_left),
                                     int(window_right), _ptr(alibi_slopes), float(softcap), _stream(stream))
     _check(code, "fa_fwd_gqa")
+
+
+def fa_bwd_workspace_size(B: int, H: int, Nq: int, d: int) -> int:
+    return int(_lib_handle().fa_bwd_workspace_size(B, H, Nq, d))
+
+
+def fa_bwd(q, k, v, out, lse, dout, dq, dk, dv, scale: float, causal: bool = False, window_left: int = -1,
+           window_right: int = -1, alibi_slopes=None, softcap: float = 0.0,
+           workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Backward of fa_fwd / fa_fwd_gqa: q, out, dout, dq [B,Nq,H,d]; k, v, dk, dv [B,Nk,H_kv,d];
+    lse fp32 [B,H,Nq] from the forward; workspace a byte tensor of fa_bwd_workspace_size bytes
+    (allocated here when None)."""
+    B, Nq, H, d = q.shape
+    Nk, H_kv = k.shape[1], k.shape[2]
+    for t in (q, k, v, out, lse, dout, dq, dk, dv):
+        if not t.is_contiguous():
+            raise ValueError("fa_bwd needs contiguous tensors")
+    if tuple(k.shape) != (B, Nk, H_kv, d) or tuple(v.shape) != tuple(k.shape) or \
+            tuple(dk.shape) != tuple(k.shape) or tuple(dv.shape) != tuple(k.shape) or \
+            tuple(out.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape) or \
+            tuple(dq.shape) != tuple(q.shape):
+        raise ValueError("fa_bwd: shape mismatch")
+    if tuple(lse.shape) != (B, H, Nq) or lse.dtype != torch.float32:
+        raise ValueError("fa_bwd: lse must be fp32 [B, H, Nq]")
+    if len({t.dtype for t in (q, k, v, out, dout, dq, dk, dv)}) != 1:
+        raise ValueError("fa_bwd: q, k, v, out, dout, dq, dk, dv must share one dtype")
+    need = fa_bwd_workspace_size(B, H, Nq, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    code = _lib_handle().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                                _ptr(dv), B, H, H_kv, Nq, Nk, d, _dtype_code(q), float(scale),
+                                int(bool(causal)), int(window_left), int(window_right), _ptr(alibi_slopes),
+                                float(softcap), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(stream))
+    _check(code, "fa_bwd")
 
 
 def fa_fwd_qkvpacked(qkv, out, lse, scale: float, causal: bool = False, window_left: int = -1,

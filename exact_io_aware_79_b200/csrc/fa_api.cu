@@ -60,17 +60,18 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [B, N, H, d] 16-bit tensor as a 4-D map (d, H, N, B), box (64, 1, 128, 1),
+// [B, N, H, d] 16-bit tensor as a 4-D map (d, H, N, B), box (64, 1, rows, 1),
 // 128-byte swizzle; rows past N read as zero. tok: elements from one token
 // to the next (H * d when contiguous; 3 * H * d inside a packed QKV tensor).
-bool make_map(CUtensorMap* map, const void* base, bool bf16, int B, int N, int H, int d, long long tok = 0) {
+bool make_map(CUtensorMap* map, const void* base, bool bf16, int B, int N, int H, int d, long long tok = 0,
+              int rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t n = static_cast<cuuint64_t>(N > 0 ? N : 1);
   const cuuint64_t t = static_cast<cuuint64_t>(tok > 0 ? tok : static_cast<long long>(H) * d);
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), n, static_cast<cuuint64_t>(B)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, t * 2, n * t * 2};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(rows), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -400,6 +401,76 @@ fa_status fa_kvcache_append(const void* k_new, const void* v_new, void* k_cache,
   p.page_size = page_size;
   p.max_blocks = max_blocks;
   return fa::launch_append(p, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int Nq, int d) {
+  if (B < 0 || H < 0 || Nq < 0 || d < 0) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * Nq;
+  return ((rows * d * sizeof(float) + 255) & ~size_t(255)) + ((rows * sizeof(float) + 255) & ~size_t(255));
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+                 void* dq, void* dk, void* dv, int B, int H, int H_kv, int Nq, int Nk, int d, fa_dtype dtype,
+                 float scale, int causal, int window_left, int window_right, const float* alibi_slopes,
+                 float softcap, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || H < 1 || Nq < 0 || Nk < 0) return FA_ERR_SHAPE;
+  if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_SHAPE;
+  if (Nq > kMaxSeq || Nk > kMaxSeq || static_cast<long long>(B) * H_kv > 65535) return FA_ERR_SHAPE;
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  if (!finite(scale) || !finite(softcap) || softcap < 0.0f) return FA_ERR_ARG;
+  if (window_left < -1 || window_right < -1 || (causal != 0 && causal != 1)) return FA_ERR_ARG;
+  if (B == 0 || (Nq == 0 && Nk == 0)) return FA_OK;
+  const size_t kv_bytes = static_cast<size_t>(B) * Nk * H_kv * d * 2;
+  const size_t q_bytes = static_cast<size_t>(B) * Nq * H * d * 2;
+  if (Nk > 0 && (!k || !v || !dk || !dv)) return FA_ERR_NULL;
+  if (Nq > 0 && (!q || !out || !lse || !dout || !dq)) return FA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_ARG;
+  if (Nq > 0 && Nk > 0) {
+    const size_t need = fa_bwd_workspace_size(B, H, Nq, d);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  }
+  fa_status st = check_device();
+  if (st != FA_OK) return st;
+  // with no queries there is no gradient for K and V; with no keys none for Q
+  if (Nq == 0)
+    return (cudaMemsetAsync(dk, 0, kv_bytes, stream) == cudaSuccess &&
+            cudaMemsetAsync(dv, 0, kv_bytes, stream) == cudaSuccess) ? FA_OK : FA_ERR_CUDA;
+  if (Nk == 0) return cudaMemsetAsync(dq, 0, q_bytes, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+
+  const bool bf16 = dtype == FA_BF16;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_map(&tq, q, bf16, B, Nq, H, d, 0, 64) || !make_map(&to, dout, bf16, B, Nq, H, d, 0, 64) ||
+      !make_map(&tk, k, bf16, B, Nk, H_kv, d, 0, 64) || !make_map(&tv, v, bf16, B, Nk, H_kv, d, 0, 64))
+    return FA_ERR_CUDA;
+  fa::BwdParams p{};
+  const size_t rows = static_cast<size_t>(B) * H * Nq;
+  p.out = out;
+  p.dout = dout;
+  p.lse = lse;
+  p.dq_acc = static_cast<float*>(workspace);
+  p.dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                    ((rows * d * sizeof(float) + 255) & ~size_t(255)));
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.slopes = alibi_slopes;
+  p.B = B;
+  p.H = H;
+  p.H_kv = H_kv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.causal = causal;
+  p.window_left = window_left;
+  p.window_right = window_right;
+  p.use_softcap = softcap > 0.0f;
+  p.scale = scale;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.cap_scale = softcap > 0.0f ? scale / softcap : 0.0f;
+  p.cap_log2 = softcap * fa::kLog2e;
+  return fa::launch_bwd(bf16, d, p, tq, tk, tv, to, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -1,0 +1,423 @@
+// fa_bwd_kernel.cu -- attention backward: dQ, dK, dV from Q, K, V, O, LSE, dO.
+//
+// The pages name the backward pass ("FlashAttention深度解析：从算法创新到产业
+// 变革的全面影响", section 技术演进, version 2.4; "Flash-Attention v2.0 到 v2.7
+// 更新", section v2.4) without stating it; it is the gradient of the forward
+// definition, computed the IO-aware way: the forward's per-row LSE lets each
+// tile of P be rebuilt from Q and K without the full matrix, so nothing of
+// size N x N touches HBM. Per (b, h) with s = scale * Q K^T (softcapped,
+// ALiBi-biased and masked as in the forward):
+//   P = exp(s - LSE);  D_i = sum_c dO_ic O_ic  (= sum_j P_ij dP_ij)
+//   dV = P^T dO;  dP = dO V^T;  dS = P o (dP - D) [o tanh' for softcap]
+//   dQ = scale * dS K;  dK = scale * dS^T Q.
+//
+// Kernels: bwd_rowdot (D, one warp per 32 / (d/8) rows), bwd_kernel (one CTA
+// per 64-key block of one (b, cache head): dK and dV stay in registers while
+// the CTA walks the query blocks of every query head that reads the cache
+// head; dQ partials are added into an fp32 accumulator), bwd_dq_cast (dQ =
+// scale * accumulator, to the input type).
+//
+// bwd_kernel's products are warp-level m16n8k16 tensor-core MMAs; each of the
+// four warps owns 16 keys (the rows of its products). K, V and the double-
+// buffered Q and dO tiles arrive by TMA as 64-column boxes with 128-byte
+// swizzle, so each 16-byte chunk c of row r sits at chunk c ^ (r % 8) of its
+// 128-byte line. Fragment bookkeeping (g = lane / 4, t = lane % 4, perm(n) =
+// n / 2 + 4 (n % 2)):
+//  * S^T = K Q^T and dP^T = V dO^T: product row g (g + 8) is key 16 w +
+//    perm(g) (+ 8); column n of query n-tile j is query 8 j + perm(n). The
+//    head-dimension order is permuted so each lane's operands are whole
+//    16-byte chunks (chunk 4 i + t of a row feeds k-steps 2 i and 2 i + 1,
+//    words 0-1 and 2-3), which the sum over k does not notice; perm keeps the
+//    two rows a quarter-warp reads in opposite halves of a swizzle line.
+//  * dV += P^T dO and dK += dS^T Q: the accumulators of query n-tiles 2 k and
+//    2 k + 1 are the A operand of k-step k (queries 16 k + perm(0..7), then
+//    16 k + 8 + perm(0..7)); ldmatrix.trans reads the matching dO / Q rows.
+//  * dQ = dS K: dS^T is stored to shared memory (row = key, column = query in
+//    the n-tile order above); ldmatrix.trans turns it into the A operand with
+//    queries as rows, K (rows = keys in natural order) is the B operand.
+#include "fa_internal.h"
+#include "sm100_ptx.cuh"
+
+#include <type_traits>
+
+namespace fa {
+namespace {
+
+constexpr int kBwdWarps = 4;
+constexpr int kBlk = 64;  // keys per CTA, queries per step
+
+__device__ __forceinline__ int perm8(int n) { return (n >> 1) | ((n & 1) << 2); }
+
+// Byte offset of 16-byte chunk c of row r in a 64-row tile of 64-column
+// boxes with 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw_off(int r, int c) {
+  return static_cast<uint32_t>((c >> 3) * (kBlk * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kTile = kBlk * D * 2;  // one 64-row tile of K, V, Q or dO
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kTile;
+  static constexpr int kOffQ = 2 * kTile;   // two buffers
+  static constexpr int kOffO = 4 * kTile;   // two buffers (dO)
+  static constexpr int kOffS = 6 * kTile;   // dS^T, 64 x 64 16-bit
+  static constexpr int kOffL = kOffS + kBlk * kBlk * 2;  // lse2[2][64], dvec[2][64]
+  static constexpr int kOffBar = kOffL + 4 * kBlk * 4;
+  static constexpr int kSmem = 1024 + kOffBar + 64;  // + slack to align to 1 KB
+};
+
+// D_i = sum_c dO_ic O_ic in fp32, [B, H, Nq].
+template <typename T, int D>
+__global__ void __launch_bounds__(256) bwd_rowdot_kernel(const BwdParams p) {
+  constexpr int LPR = D / 8;  // lanes per row
+  const long long rows = static_cast<long long>(p.B) * p.Nq * p.H;
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / LPR;
+  const int cl = threadIdx.x % LPR;
+  float acc = 0.0f;
+  if (row < rows) {
+    const size_t off = static_cast<size_t>(row) * D + cl * 8;
+    const uint4 a = *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.dout) + off);
+    const uint4 o = *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.out) + off);
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, ow[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = unpack2<T>(aw[e]), y = unpack2<T>(ow[e]);
+      acc = fmaf(x.x, y.x, acc);
+      acc = fmaf(x.y, y.y, acc);
+    }
+  }
+#pragma unroll
+  for (int o = LPR / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (row < rows && cl == 0) {
+    // row = (b * Nq + i) * H + h  ->  dvec[(b * H + h) * Nq + i]
+    const long long h = row % p.H, bi = row / p.H;
+    const long long b = bi / p.Nq, i = bi % p.Nq;
+    p.dvec[(b * p.H + h) * p.Nq + i] = acc;
+  }
+}
+
+// dQ = scale * accumulator, cast to the input type; 4 elements per thread.
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_dq_cast_kernel(const BwdParams p, long long n4) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4 a = reinterpret_cast<const float4*>(p.dq_acc)[i];
+  uint2 w;
+  w.x = pack2<T>(a.x * p.scale, a.y * p.scale);
+  w.y = pack2<T>(a.z * p.scale, a.w * p.scale);
+  reinterpret_cast<uint2*>(p.dq)[i] = w;
+}
+
+// Is key j visible to the query at key position pos (the forward's rule)?
+__device__ __forceinline__ bool key_visible(int pos, int j, int Nk, const BwdParams& p) {
+  if (j >= Nk) return false;
+  if (p.causal && j > pos) return false;
+  if (p.window_left >= 0 && j < pos - p.window_left) return false;
+  if (p.window_right >= 0 && j > pos + p.window_right) return false;
+  return true;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kBwdWarps * 32, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+               const BwdParams p) {
+  using C = BwdCfg<D>;
+  constexpr int KS = D / 16;  // k-steps over the head dimension
+  constexpr int NT = D / 8;   // n-tiles over the head dimension
+  constexpr int NH = NT / 2;  // n-tiles per half of the dQ product
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+  uint8_t* sS = smem + C::kOffS;
+  float* sL = reinterpret_cast<float*>(smem + C::kOffL);        // [2][64] lse * log2(e)
+  float* sDv = sL + 2 * kBlk;                                     // [2][64] D
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);  // full[2], kv
+  int* abort_flag = reinterpret_cast<int*>(bars + 3);
+  volatile int* abort = abort_flag;
+  const uint32_t sK_a = smem_addr(sK), sS_a = smem_addr(sS);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int kb = blockIdx.x;
+  const int b = blockIdx.y / p.H_kv, hk = blockIdx.y % p.H_kv;
+  const int G = p.H / p.H_kv;
+  const int k0 = kb * kBlk;
+  const int off = p.Nk - p.Nq;  // query i sits at key position i + off
+
+  // query rows that can see a key of [k0, k1)
+  const int k1 = min(k0 + kBlk, p.Nk);
+  long long q_lo = 0, q_hi = p.Nq - 1;
+  {
+    int right = -1;  // keys j <= pos + right are the only visible ones (when >= 0)
+    if (p.causal) right = 0;
+    if (p.window_right >= 0) right = p.causal ? min(0, p.window_right) : p.window_right;
+    if (p.causal || p.window_right >= 0) q_lo = max(q_lo, static_cast<long long>(k0) - off - right);
+    if (p.window_left >= 0) q_hi = min(q_hi, static_cast<long long>(k1 - 1) + p.window_left - off);
+  }
+  const int qb_lo = q_lo <= q_hi ? static_cast<int>(q_lo / kBlk) : 0;
+  const int n_qb = q_lo <= q_hi ? static_cast<int>(q_hi / kBlk) - qb_lo + 1 : 0;
+  const int n_it = G * n_qb;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    mbar_init(&bars[2], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const uint64_t pol = l2_policy_evict_last();
+  auto issue = [&](int it) {
+    const int buf = it & 1;
+    const int h = hk * G + it / n_qb;
+    const int q0 = (qb_lo + it % n_qb) * kBlk;
+    mbar_arrive_expect_tx(&bars[buf], 2 * C::kTile);
+#pragma unroll
+    for (int hh = 0; hh < D / 64; ++hh) {
+      tma_load_4d(&tmQ, &bars[buf], smem + C::kOffQ + buf * C::kTile + hh * kBlk * 128, hh * 64, h, q0, b, pol);
+      tma_load_4d(&tmO, &bars[buf], smem + C::kOffO + buf * C::kTile + hh * kBlk * 128, hh * 64, h, q0, b, pol);
+    }
+  };
+  if (threadIdx.x == 0 && n_it > 0) {
+    mbar_arrive_expect_tx(&bars[2], 2 * C::kTile);
+#pragma unroll
+    for (int hh = 0; hh < D / 64; ++hh) {
+      tma_load_4d(&tmK, &bars[2], sK + hh * kBlk * 128, hh * 64, hk, k0, b, pol);
+      tma_load_4d(&tmV, &bars[2], sV + hh * kBlk * 128, hh * 64, hk, k0, b, pol);
+    }
+    issue(0);
+    if (n_it > 1) issue(1);
+  }
+
+  float dv[NT][4], dk[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dv[n][e] = dk[n][e] = 0.0f;
+
+  const int krow0 = warp * 16 + perm8(gq);  // this lane's product rows: krow0, krow0 + 8
+  const bool alibi = p.slopes != nullptr;
+  bool failed = false;
+  int issued = n_it > 1 ? 2 : n_it;
+
+  for (int it = 0; it < n_it; ++it) {
+    const int buf = it & 1;
+    const int h = hk * G + it / n_qb;
+    const int q0 = (qb_lo + it % n_qb) * kBlk;
+    const float slope2 = alibi ? p.slopes[h] * kLog2e : 0.0f;
+    // row vectors of this query block
+    if (threadIdx.x < kBlk) {
+      const int q = q0 + threadIdx.x;
+      const size_t ri = (static_cast<size_t>(b) * p.H + h) * p.Nq + q;
+      sL[buf * kBlk + threadIdx.x] = q < p.Nq ? p.lse[ri] * kLog2e : -INFINITY;
+      sDv[buf * kBlk + threadIdx.x] = q < p.Nq ? p.dvec[ri] : 0.0f;
+    }
+    __syncthreads();  // also: every warp is done with the previous block's dS tile
+    bool ok = true;
+    if (it == 0) ok = mbar_wait(&bars[2], 0, abort);
+    ok = ok && mbar_wait(&bars[buf], (it >> 1) & 1, abort);
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+    const uint8_t* sQ = smem + C::kOffQ + buf * C::kTile;
+    const uint8_t* sO = smem + C::kOffO + buf * C::kTile;
+    const uint32_t sQ_a = smem_addr(sQ), sO_a = smem_addr(sO);
+    const float* lse2 = sL + buf * kBlk;
+    const float* dvec = sDv + buf * kBlk;
+
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      // ---- S^T and dP^T for query n-tiles 4 hf .. 4 hf + 3
+      float sc[4][4], dp[4][4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[jj][e] = dp[jj][e] = 0.0f;
+#pragma unroll
+      for (int i = 0; i < KS / 2; ++i) {
+        const int c = 4 * i + tq;
+        const uint4 k0v = *reinterpret_cast<const uint4*>(sK + sw_off(krow0, c));
+        const uint4 k1v = *reinterpret_cast<const uint4*>(sK + sw_off(krow0 + 8, c));
+        const uint4 v0v = *reinterpret_cast<const uint4*>(sV + sw_off(krow0, c));
+        const uint4 v1v = *reinterpret_cast<const uint4*>(sV + sw_off(krow0 + 8, c));
+        const uint32_t ka0[4] = {k0v.x, k1v.x, k0v.y, k1v.y}, ka1[4] = {k0v.z, k1v.z, k0v.w, k1v.w};
+        const uint32_t va0[4] = {v0v.x, v1v.x, v0v.y, v1v.y}, va1[4] = {v0v.z, v1v.z, v0v.w, v1v.w};
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int r = 8 * (4 * hf + jj) + perm8(gq);
+          const uint4 qw = *reinterpret_cast<const uint4*>(sQ + sw_off(r, c));
+          const uint4 ow = *reinterpret_cast<const uint4*>(sO + sw_off(r, c));
+          mma_16816<T>(sc[jj], ka0, qw.x, qw.y);
+          mma_16816<T>(sc[jj], ka1, qw.z, qw.w);
+          mma_16816<T>(dp[jj], va0, ow.x, ow.y);
+          mma_16816<T>(dp[jj], va1, ow.z, ow.w);
+        }
+      }
+      // ---- P and dS, elementwise (sc <- P, dp <- dS)
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = k0 + krow0 + 8 * (e >> 1);
+          const int ql = 8 * (4 * hf + jj) + tq + 4 * (e & 1);
+          const int q = q0 + ql;
+          const int pos = q + off;
+          const bool vis = q < p.Nq && key_visible(pos, key, p.Nk, p);
+          float logit2, dfac = 1.0f;
+          if (p.use_softcap) {
+            const float th = tanh_via_exp2(sc[jj][e] * p.cap_scale);
+            logit2 = th * p.cap_log2;
+            dfac = 1.0f - th * th;
+          } else {
+            logit2 = sc[jj][e] * p.scale_log2;
+          }
+          if (alibi) logit2 -= slope2 * fabsf(static_cast<float>(pos - key));
+          const float pr = vis ? ex2(logit2 - lse2[ql]) : 0.0f;
+          sc[jj][e] = pr;
+          dp[jj][e] = pr * (dp[jj][e] - dvec[ql]) * dfac;
+        }
+      }
+      // ---- dV += P^T dO, dK += dS^T Q over the query k-steps 2 hf, 2 hf + 1
+#pragma unroll
+      for (int kx = 0; kx < 2; ++kx) {
+        const int kk = 2 * hf + kx;
+        const uint32_t pa[4] = {pack2<T>(sc[2 * kx][0], sc[2 * kx][1]), pack2<T>(sc[2 * kx][2], sc[2 * kx][3]),
+                                pack2<T>(sc[2 * kx + 1][0], sc[2 * kx + 1][1]),
+                                pack2<T>(sc[2 * kx + 1][2], sc[2 * kx + 1][3])};
+        const uint32_t da[4] = {pack2<T>(dp[2 * kx][0], dp[2 * kx][1]), pack2<T>(dp[2 * kx][2], dp[2 * kx][3]),
+                                pack2<T>(dp[2 * kx + 1][0], dp[2 * kx + 1][1]),
+                                pack2<T>(dp[2 * kx + 1][2], dp[2 * kx + 1][3])};
+        const int brow = 16 * kk + ((lane >> 3) & 1) * 8 + perm8(lane & 7);
+#pragma unroll
+        for (int u = 0; u < NT / 2; ++u) {
+          const int cc = 2 * u + (lane >> 4);
+          uint32_t bo[4], bq[4];
+          ldsm_x4_trans(bo, sO_a + sw_off(brow, cc));
+          ldsm_x4_trans(bq, sQ_a + sw_off(brow, cc));
+          mma_16816<T>(dv[2 * u], pa, bo[0], bo[1]);
+          mma_16816<T>(dv[2 * u + 1], pa, bo[2], bo[3]);
+          mma_16816<T>(dk[2 * u], da, bq[0], bq[1]);
+          mma_16816<T>(dk[2 * u + 1], da, bq[2], bq[3]);
+        }
+      }
+      // ---- dS^T to shared memory: row = key (local), column = query position
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int jt = 4 * hf + jj;
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int kr = krow0 + 8 * hr;
+          *reinterpret_cast<uint32_t*>(sS + kr * 128 + ((jt ^ (kr & 7)) << 4) + 4 * tq) =
+              pack2<T>(dp[jj][2 * hr], dp[jj][2 * hr + 1]);
+        }
+      }
+    }
+    __syncthreads();  // dS^T complete; this block's Q and dO buffers are free
+    if (threadIdx.x == 0 && issued < n_it) {
+      issue(issued);
+      ++issued;
+    }
+    // ---- dQ (rows = query positions 16 w .. 16 w + 15) += dS K, in two halves of n-tiles
+    const int hq = h;
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+      float acc[NH][4];
+#pragma unroll
+      for (int n = 0; n < NH; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
+#pragma unroll
+      for (int kk = 0; kk < kBlk / 16; ++kk) {
+        const int mi = lane >> 3;
+        const int akey = 16 * kk + (mi >> 1) * 8 + (lane & 7);
+        const int achunk = 2 * warp + (mi & 1);
+        uint32_t a[4];
+        ldsm_x4_trans(a, sS_a + akey * 128 + ((achunk ^ (akey & 7)) << 4));
+        const int brow = 16 * kk + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int u = 0; u < NH / 2; ++u) {
+          const int cc = nh * NH + 2 * u + (lane >> 4);
+          uint32_t bk[4];
+          ldsm_x4_trans(bk, sK_a + sw_off(brow, cc));
+          mma_16816<T>(acc[2 * u], a, bk[0], bk[1]);
+          mma_16816<T>(acc[2 * u + 1], a, bk[2], bk[3]);
+        }
+      }
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int q = q0 + 16 * warp + 8 * hr + perm8(gq);
+        if (q < p.Nq) {
+          float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.Nq + q) * p.H + hq) * D + nh * NH * 8 + 2 * tq;
+#pragma unroll
+          for (int n = 0; n < NH; ++n) atomicAdd(reinterpret_cast<float2*>(dst + 8 * n),
+                                                 make_float2(acc[n][2 * hr], acc[n][2 * hr + 1]));
+        }
+      }
+    }
+  }
+  // loads still in flight must land before the CTA exits
+  if (threadIdx.x == 0 && failed) {
+    int dummy = 0;
+    for (int i = max(0, issued - 2); i < issued; ++i) mbar_wait(&bars[i & 1], (i >> 1) & 1, &dummy);
+    mbar_wait(&bars[2], 0, &dummy);
+  }
+
+  // ---- dK (scaled) and dV rows of this lane: keys k0 + krow0 (+ 8)
+  const float nan = __int_as_float(0x7fc00000);
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    const int key = k0 + krow0 + 8 * hr;
+    if (key >= p.Nk) continue;
+    const size_t base = ((static_cast<size_t>(b) * p.Nk + key) * p.H_kv + hk) * D + 2 * tq;
+    T* dk_out = reinterpret_cast<T*>(p.dk) + base;
+    T* dv_out = reinterpret_cast<T*>(p.dv) + base;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const float k0f = failed ? nan : dk[n][2 * hr] * p.scale, k1f = failed ? nan : dk[n][2 * hr + 1] * p.scale;
+      const float v0f = failed ? nan : dv[n][2 * hr], v1f = failed ? nan : dv[n][2 * hr + 1];
+      *reinterpret_cast<uint32_t*>(dk_out + 8 * n) = pack2<T>(k0f, k1f);
+      *reinterpret_cast<uint32_t*>(dv_out + 8 * n) = pack2<T>(v0f, v1f);
+    }
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                   const CUtensorMap& tmO, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(p.B) * p.Nq * p.H;
+  const long long elems = rows * D;
+  cudaError_t e = cudaMemsetAsync(p.dq_acc, 0, static_cast<size_t>(elems) * sizeof(float), stream);
+  if (e != cudaSuccess) return e;
+  if (rows > 0) {
+    const long long threads = rows * (D / 8);
+    bwd_rowdot_kernel<T, D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  using C = BwdCfg<D>;
+  auto kernel = bwd_kernel<T, D>;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((p.Nk + kBlk - 1) / kBlk, p.B * p.H_kv);
+  kernel<<<grid, kBwdWarps * 32, C::kSmem, stream>>>(tmQ, tmK, tmV, tmO, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long n4 = elems / 4;
+  if (n4 > 0) bwd_dq_cast_kernel<T><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(p, n4);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(bool bf16, int d, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                       const CUtensorMap& tmV, const CUtensorMap& tmO, cudaStream_t stream) {
+  if (bf16) return d == 128 ? launch<__nv_bfloat16, 128>(p, tmQ, tmK, tmV, tmO, stream)
+                            : launch<__nv_bfloat16, 64>(p, tmQ, tmK, tmV, tmO, stream);
+  return d == 128 ? launch<__half, 128>(p, tmQ, tmK, tmV, tmO, stream)
+                  : launch<__half, 64>(p, tmQ, tmK, tmV, tmO, stream);
+}
+
+}  // namespace fa

@@ -72,6 +72,31 @@ inline bool decode_on_tensor_cores(int H, int H_kv) { return H_kv > 0 && H / H_k
 cudaError_t launch_decode(bool bf16, int d, const DecodeParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
                           cudaStream_t stream);
 
+// Backward: dQ, dK, dV of L = sum(dO * O) from Q, K, V, O, LSE, dO.
+struct BwdParams {
+  const void* out;    // [B, Nq, H, d]
+  const void* dout;   // [B, Nq, H, d]
+  const float* lse;   // [B, H, Nq] (natural log, the forward's)
+  float* dvec;        // [B, H, Nq] workspace: D_i = sum_c dO_ic O_ic
+  float* dq_acc;      // [B, Nq, H, d] workspace: unscaled dQ in fp32
+  void* dq;           // [B, Nq, H, d]
+  void* dk;           // [B, Nk, H_kv, d]
+  void* dv;           // [B, Nk, H_kv, d]
+  const float* slopes;  // [H] or nullptr
+  int B, H, H_kv, Nq, Nk;
+  int causal, window_left, window_right;
+  int use_softcap;
+  float scale;       // softmax scale (dQ, dK factor)
+  float scale_log2;  // scale * log2(e)            (no softcap)
+  float cap_scale;   // scale / softcap             (softcap)
+  float cap_log2;    // softcap * log2(e)           (softcap)
+};
+
+// tmQ/tmO: (d, H, Nq, B) maps of Q and dO, tmK/tmV: (d, H_kv, Nk, B) maps of
+// K and V, all with (64, 1, 64, 1) boxes and 128-byte swizzle.
+cudaError_t launch_bwd(bool bf16, int d, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                       const CUtensorMap& tmV, const CUtensorMap& tmO, cudaStream_t stream);
+
 // Writes n_new new tokens per sequence into the paged caches at positions
 // cache_seqlens[b] .. cache_seqlens[b] + n_new - 1.
 struct AppendParams {

@@ -263,6 +263,46 @@ fa_status fa_kvcache_append(const void *k_new, const void *v_new, void *k_cache,
                             int max_blocks, fa_dtype dtype, cudaStream_t stream);
 
 /*
+ * fa_bwd -- backward pass of fa_fwd / fa_fwd_gqa: the gradients dq, dk, dv
+ * of L = sum(dout * O), where O and lse are what the forward returned for the
+ * same q, k, v and options.
+ *
+ * The pages name the backward pass ("FlashAttention深度解析：从算法创新到产业
+ * 变革的全面影响", section 技术演进, version 2.4; "Flash-Attention v2.0 到 v2.7
+ * 更新", section v2.4) without its formulas; this is the gradient of the
+ * forward's definition. With s = scale * q k^T softcapped, ALiBi-biased and
+ * masked as in fa_fwd, P = exp(s - lse):
+ *   dv = P^T dout;  dP = dout v^T;  D_i = sum_c dout_ic O_ic
+ *   dS = P o (dP - D) (o (1 - tanh^2) under softcap);
+ *   dq = scale * dS k;  dk = scale * dS^T q
+ * Grouped-query k, v heads (H_kv < H) receive the sum over the query heads
+ * that read them. P is rebuilt tile by tile from lse; no N x N array is
+ * written. dq is accumulated in fp32 in the workspace across key blocks with
+ * atomic adds, so its last bits may differ from run to run (the order of the
+ * additions is not fixed); dk and dv are summed in a fixed order.
+ *
+ *   q, out, dout, dq   [B, Nq, H, d]       contiguous, dtype
+ *   k, v, dk, dv       [B, Nk, H_kv, d]    contiguous, dtype
+ *   lse                [B, H, Nq]          fp32 (the forward's, natural log)
+ *   workspace          fa_bwd_workspace_size(B, H, Nq, d) bytes of device
+ *                      memory, 16-byte aligned (fp32 dq accumulator + D)
+ *   scale, causal, window_left, window_right, alibi_slopes, softcap: as fa_fwd
+ * Outputs dq, dk, dv are overwritten (not accumulated). The caller owns every
+ * buffer; the call only enqueues work on `stream`.
+ *
+ * Errors: as fa_fwd_gqa, plus FA_ERR_WORKSPACE when the workspace is missing,
+ * misaligned or too small, and FA_ERR_SHAPE when B * H_kv > 65535.
+ * Nq == 0 gives zero dk, dv; Nk == 0 gives zero dq; B == 0 is a no-op.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int Nq, int d);
+
+fa_status fa_bwd(const void *q, const void *k, const void *v, const void *out, const float *lse,
+                 const void *dout, void *dq, void *dk, void *dv, int B, int H, int H_kv, int Nq, int Nk,
+                 int d, fa_dtype dtype, float scale, int causal, int window_left, int window_right,
+                 const float *alibi_slopes, float softcap, void *workspace, size_t workspace_bytes,
+                 cudaStream_t stream);
+
+/*
  * Number of splits fa_fwd_kvcache uses for these sizes: num_splits itself
  * when it is 1..FA_MAX_SPLITS, else the automatic choice, which depends only
  * on B, H and the longest possible sequence max_blocks * page_size (host-side

@@ -247,3 +247,35 @@ def test_qkvpacked_validation(lib):
     assert vpk(total=-5) == SHAPE
     assert vpk(total=0) == OK
     assert vpk() in (OK, DEVICE)
+
+
+def test_bwd_validation(lib):
+    def bw(**kw):
+        a = dict(q=P, k=P, v=P, out=P, lse=P, dout=P, dq=P, dk=P, dv=P, B=2, H=8, H_kv=2, Nq=100, Nk=200, d=128,
+                 dtype=1, scale=0.1, causal=1, wl=-1, wr=-1, slopes=None, cap=0.0, ws=P,
+                 ws_bytes=lib.fa_bwd_workspace_size(2, 8, 100, 128))
+        a.update(kw)
+        return lib.fa_bwd(a["q"], a["k"], a["v"], a["out"], a["lse"], a["dout"], a["dq"], a["dk"], a["dv"], a["B"],
+                          a["H"], a["H_kv"], a["Nq"], a["Nk"], a["d"], a["dtype"], a["scale"], a["causal"], a["wl"],
+                          a["wr"], a["slopes"], a["cap"], a["ws"], a["ws_bytes"], None)
+    assert bw() == DEVICE
+    assert bw(H_kv=3) == SHAPE
+    assert bw(H_kv=16) == SHAPE
+    assert bw(B=40000, H_kv=2) == SHAPE          # B * H_kv > 65535
+    assert bw(d=96) == HEADDIM
+    assert bw(dtype=7) == DTYPE
+    assert bw(scale=float("nan")) == ARG
+    assert bw(cap=-1.0) == ARG
+    assert bw(wl=-2) == ARG
+    assert bw(causal=2) == ARG
+    assert bw(dout=None) == NULL
+    assert bw(dk=None) == NULL
+    assert bw(dq=P + 8) == ARG                   # not 16-byte aligned
+    assert bw(ws=None) == WORKSPACE
+    assert bw(ws_bytes=lib.fa_bwd_workspace_size(2, 8, 100, 128) - 1) == WORKSPACE
+    assert bw(B=0) == OK
+    assert bw(Nq=0, ws=None, ws_bytes=0) == DEVICE   # zero dk, dv: no workspace needed
+    # fp32 dq accumulator rows (256-byte rounded) + D rows
+    assert lib.fa_bwd_workspace_size(2, 8, 100, 128) == (2 * 8 * 100 * 128 * 4 + 255) // 256 * 256 + \
+        (2 * 8 * 100 * 4 + 255) // 256 * 256
+    assert lib.fa_bwd_workspace_size(-1, 8, 100, 128) == 0

@@ -1,0 +1,116 @@
+"""GPU parity of the backward pass (fa_bwd, through the C ABI) against the
+fp64 oracle's gradients.
+
+Tolerance, from the arithmetic: the kernel rounds P and dS to the input type
+before the products that consume them (dV = P^T dO; dK = dS^T Q; dQ = dS K)
+and rounds dq, dk, dv to it at the end; every sum runs in fp32. Each term thus
+carries a relative error of at most one unit in the last place of the input
+type (2^-8 bf16, 2^-11 fp16), so a gradient entry is off by at most that
+fraction of the sum of its terms' magnitudes, which for these inputs stays
+within a few times the largest entry of the gradient. The bar is
+max |got - want| <= tol * max |want| with tol = 2e-2 (bf16) and 5e-3 (fp16).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import exact_io_aware_79_b200 as fa
+from exact_io_aware_79_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.bfloat16: 2e-2, torch.float16: 5e-3}
+
+
+def inputs(B, H, H_kv, Nq, Nk, d, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, Nq, H, d, generator=g).to(dtype)
+    k = torch.randn(B, Nk, H_kv, d, generator=g).to(dtype)
+    v = torch.randn(B, Nk, H_kv, d, generator=g).to(dtype)
+    do = torch.randn(B, Nq, H, d, generator=g).to(dtype)
+    return q, k, v, do
+
+
+def run(q, k, v, do, scale, causal=False, wl=-1, wr=-1, slopes=None, cap=0.0):
+    B, Nq, H, d = q.shape
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    out = torch.empty_like(qd)
+    lse = torch.empty(B, H, Nq, dtype=torch.float32, device="cuda")
+    sl = None if slopes is None else slopes.cuda()
+    fa.fa_fwd_gqa(qd, kd, vd, out, lse, scale, causal, wl, wr, sl, cap)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    fa.fa_bwd(qd, kd, vd, out, lse, dod, dq, dk, dv, scale, causal, wl, wr, sl, cap)
+    torch.cuda.synchronize()
+    return dq, dk, dv
+
+
+def check(got, want, dtype, what):
+    got = got.float().cpu().numpy()
+    err = float(np.abs(got - want).max())
+    ref = float(np.abs(want).max())
+    assert np.isfinite(got).all(), what
+    assert err <= TOL[dtype] * max(ref, 1e-6), "%s: max error %.3g of max |want| %.3g" % (what, err, ref)
+
+
+CASES = [
+    # (B, H, H_kv, Nq, Nk, d, dtype, causal, wl, wr, alibi, cap)
+    (2, 2, 2, 200, 200, 128, torch.bfloat16, True, -1, -1, False, 0.0),    # ragged, several blocks each way
+    (1, 2, 2, 130, 257, 64, torch.float16, False, -1, -1, False, 0.0),     # Nq < Nk, no mask
+    (1, 2, 1, 257, 129, 64, torch.float16, True, -1, -1, False, 0.0),      # Nq > Nk: rows without keys
+    (1, 4, 2, 190, 190, 128, torch.bfloat16, True, 50, 0, True, 30.0),     # grouped, window, ALiBi, softcap
+    (2, 2, 2, 64, 64, 128, torch.bfloat16, False, 10, 20, False, 0.0),     # two-sided window
+    (1, 8, 2, 100, 300, 128, torch.float16, True, -1, -1, True, 0.0),      # groups of 4, ALiBi, Nq < Nk
+    (1, 2, 2, 1, 70, 128, torch.bfloat16, True, -1, -1, False, 5.0),       # one query row, softcap
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B%dH%dkv%dq%dk%dd%d" % c[:6])
+def test_bwd_matches_oracle(case):
+    B, H, H_kv, Nq, Nk, d, dtype, causal, wl, wr, alibi, cap = case
+    q, k, v, do = inputs(B, H, H_kv, Nq, Nk, d, dtype, seed=Nq + Nk + H)
+    slopes = W.alibi_slopes(H) if alibi else None
+    scale = 1.0 / math.sqrt(d)
+    dq, dk, dv = run(q, k, v, do, scale, causal, wl, wr, slopes, cap)
+    rq, rk, rv = oracle.attn_bwd(q, k, v, do, scale, causal, wl, wr, slopes, cap)
+    check(dq, rq, dtype, "dq")
+    check(dk, rk, dtype, "dk")
+    check(dv, rv, dtype, "dv")
+
+
+def test_bwd_dk_dv_are_reproducible_bit_for_bit():
+    q, k, v, do = inputs(1, 4, 2, 300, 300, 128, torch.bfloat16, seed=3)
+    a = run(q, k, v, do, 0.1, True)
+    b = run(q, k, v, do, 0.1, True)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    assert (a[0].float() - b[0].float()).abs().max().item() <= 1e-2 * a[0].float().abs().max().item()
+
+
+def test_bwd_empty_sides():
+    q, k, v, do = inputs(1, 2, 2, 0, 50, 64, torch.float16, seed=4)
+    dq, dk, dv = run(q, k, v, do, 0.2, False)
+    assert torch.count_nonzero(dk) == 0 and torch.count_nonzero(dv) == 0
+
+
+def test_full_size_causal_bwd_on_sampled_heads():
+    """The causal B8 H16 N2048 d128 workload, gradients of two (batch, head)
+    pairs checked against the oracle on those heads alone (in MHA a head's
+    gradients depend only on its own q, k, v, dout)."""
+    w = W.CAUSAL_2K
+    x = W.make_fwd_inputs(w, device="cuda")
+    g = torch.Generator().manual_seed(77)
+    do = torch.randn(x["q"].shape, generator=g).to(w.dtype).cuda()
+    out = torch.empty_like(x["q"])
+    lse = torch.empty(w.B, w.H, w.Nq, dtype=torch.float32, device="cuda")
+    fa.fa_fwd(x["q"], x["k"], x["v"], out, lse, w.scale, True)
+    dq, dk, dv = torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"])
+    fa.fa_bwd(x["q"], x["k"], x["v"], out, lse, do, dq, dk, dv, w.scale, True)
+    torch.cuda.synchronize()
+    for b, h in ((0, 0), (w.B - 1, w.H - 1)):
+        sl = lambda t: t[b:b + 1, :, h:h + 1].cpu()
+        rq, rk, rv = oracle.attn_bwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(do), w.scale, True)
+        check(sl(dq), rq, w.dtype, "dq (%d, %d)" % (b, h))
+        check(sl(dk), rk, w.dtype, "dk (%d, %d)" % (b, h))
+        check(sl(dv), rv, w.dtype, "dv (%d, %d)" % (b, h))
