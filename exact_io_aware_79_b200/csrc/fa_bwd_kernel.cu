@@ -132,8 +132,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
   uint8_t* sS = smem + C::kOffS;
-  float* sL = reinterpret_cast<float*>(smem + C::kOffL);        // [2][64] lse * log2(e)
-  float* sDv = sL + 2 * kBlk;                                     // [2][64] D
+  float* sL = reinterpret_cast<float*>(smem + C::kOffL);        // [2][lse * log2(e) x 64, D x 64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);  // full[2], kv
   int* abort_flag = reinterpret_cast<int*>(bars + 3);
   volatile int* abort = abort_flag;
@@ -204,22 +203,29 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
   bool failed = false;
   int issued = n_it > 1 ? 2 : n_it;
 
+  // the row vectors (lse, D) of iteration `it`: thread x < 64 fetches lse of
+  // query q0 + x, thread 64 + x its D; read one iteration ahead into a register
+  auto fetch_rowvec = [&](int it) -> float {
+    const int h = hk * G + it / n_qb;
+    const int q = (qb_lo + it % n_qb) * kBlk + (threadIdx.x & (kBlk - 1));
+    if (q >= p.Nq) return threadIdx.x < kBlk ? -INFINITY : 0.0f;
+    const size_t ri = (static_cast<size_t>(b) * p.H + h) * p.Nq + q;
+    return threadIdx.x < kBlk ? p.lse[ri] * kLog2e : p.dvec[ri];
+  };
+  float rv_next = n_it > 0 ? fetch_rowvec(0) : 0.0f;
+
   for (int it = 0; it < n_it; ++it) {
     const int buf = it & 1;
     const int h = hk * G + it / n_qb;
     const int q0 = (qb_lo + it % n_qb) * kBlk;
     const float slope2 = alibi ? p.slopes[h] * kLog2e : 0.0f;
-    // row vectors of this query block
-    if (threadIdx.x < kBlk) {
-      const int q = q0 + threadIdx.x;
-      const size_t ri = (static_cast<size_t>(b) * p.H + h) * p.Nq + q;
-      sL[buf * kBlk + threadIdx.x] = q < p.Nq ? p.lse[ri] * kLog2e : -INFINITY;
-      sDv[buf * kBlk + threadIdx.x] = q < p.Nq ? p.dvec[ri] : 0.0f;
-    }
-    __syncthreads();  // also: every warp is done with the previous block's dS tile
+    sL[buf * 2 * kBlk + threadIdx.x] = rv_next;  // [buf][lse 0..63 | D 0..63]
+    if (it + 1 < n_it) rv_next = fetch_rowvec(it + 1);
     bool ok = true;
     if (it == 0) ok = mbar_wait(&bars[2], 0, abort);
     ok = ok && mbar_wait(&bars[buf], (it >> 1) & 1, abort);
+    // one barrier: row vectors visible, tiles landed everywhere, and every
+    // warp done with the previous block's dS tile
     if (__syncthreads_or(!ok)) {
       failed = true;
       break;
@@ -227,8 +233,15 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
     const uint8_t* sQ = smem + C::kOffQ + buf * C::kTile;
     const uint8_t* sO = smem + C::kOffO + buf * C::kTile;
     const uint32_t sQ_a = smem_addr(sQ), sO_a = smem_addr(sO);
-    const float* lse2 = sL + buf * kBlk;
-    const float* dvec = sDv + buf * kBlk;
+    const float* lse2 = sL + buf * 2 * kBlk;
+    const float* dvec = lse2 + kBlk;
+    // every (key, query) pair of this block pair visible?
+    bool full = k0 + kBlk <= p.Nk && q0 + kBlk <= p.Nq;
+    if (p.causal || p.window_right >= 0) {
+      const int right = p.window_right >= 0 ? (p.causal ? min(0, p.window_right) : p.window_right) : 0;
+      full = full && k0 + kBlk - 1 <= q0 + off + right;
+    }
+    if (p.window_left >= 0) full = full && k0 >= q0 + kBlk - 1 + off - p.window_left;
 
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
@@ -247,41 +260,55 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
         const uint4 v1v = *reinterpret_cast<const uint4*>(sV + sw_off(krow0 + 8, c));
         const uint32_t ka0[4] = {k0v.x, k1v.x, k0v.y, k1v.y}, ka1[4] = {k0v.z, k1v.z, k0v.w, k1v.w};
         const uint32_t va0[4] = {v0v.x, v1v.x, v0v.y, v1v.y}, va1[4] = {v0v.z, v1v.z, v0v.w, v1v.w};
+        uint4 qw[4], ow[4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
           const int r = 8 * (4 * hf + jj) + perm8(gq);
-          const uint4 qw = *reinterpret_cast<const uint4*>(sQ + sw_off(r, c));
-          const uint4 ow = *reinterpret_cast<const uint4*>(sO + sw_off(r, c));
-          mma_16816<T>(sc[jj], ka0, qw.x, qw.y);
-          mma_16816<T>(sc[jj], ka1, qw.z, qw.w);
-          mma_16816<T>(dp[jj], va0, ow.x, ow.y);
-          mma_16816<T>(dp[jj], va1, ow.z, ow.w);
+          qw[jj] = *reinterpret_cast<const uint4*>(sQ + sw_off(r, c));
+          ow[jj] = *reinterpret_cast<const uint4*>(sO + sw_off(r, c));
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          mma_16816<T>(sc[jj], ka0, qw[jj].x, qw[jj].y);
+          mma_16816<T>(dp[jj], va0, ow[jj].x, ow[jj].y);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          mma_16816<T>(sc[jj], ka1, qw[jj].z, qw[jj].w);
+          mma_16816<T>(dp[jj], va1, ow[jj].z, ow[jj].w);
         }
       }
-      // ---- P and dS, elementwise (sc <- P, dp <- dS)
+      // ---- P and dS, elementwise (sc <- P, dp <- dS); blocks with every
+      // (key, query) pair visible skip the per-element mask
+      auto elementwise = [&](auto masked_tag) {
+        constexpr bool kMasked = decltype(masked_tag)::value;
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
+        for (int jj = 0; jj < 4; ++jj) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int key = k0 + krow0 + 8 * (e >> 1);
-          const int ql = 8 * (4 * hf + jj) + tq + 4 * (e & 1);
-          const int q = q0 + ql;
-          const int pos = q + off;
-          const bool vis = q < p.Nq && key_visible(pos, key, p.Nk, p);
-          float logit2, dfac = 1.0f;
-          if (p.use_softcap) {
-            const float th = tanh_via_exp2(sc[jj][e] * p.cap_scale);
-            logit2 = th * p.cap_log2;
-            dfac = 1.0f - th * th;
-          } else {
-            logit2 = sc[jj][e] * p.scale_log2;
+          for (int e = 0; e < 4; ++e) {
+            const int key = k0 + krow0 + 8 * (e >> 1);
+            const int ql = 8 * (4 * hf + jj) + tq + 4 * (e & 1);
+            const int pos = q0 + ql + off;
+            float logit2, dfac = 1.0f;
+            if (p.use_softcap) {
+              const float th = tanh_via_exp2(sc[jj][e] * p.cap_scale);
+              logit2 = th * p.cap_log2;
+              dfac = 1.0f - th * th;
+            } else {
+              logit2 = sc[jj][e] * p.scale_log2;
+            }
+            if (alibi) logit2 -= slope2 * fabsf(static_cast<float>(pos - key));
+            float pr = ex2(logit2 - lse2[ql]);
+            if constexpr (kMasked) {
+              if (!(q0 + ql < p.Nq && key_visible(pos, key, p.Nk, p))) pr = 0.0f;
+            }
+            sc[jj][e] = pr;
+            dp[jj][e] = pr * (dp[jj][e] - dvec[ql]) * dfac;
           }
-          if (alibi) logit2 -= slope2 * fabsf(static_cast<float>(pos - key));
-          const float pr = vis ? ex2(logit2 - lse2[ql]) : 0.0f;
-          sc[jj][e] = pr;
-          dp[jj][e] = pr * (dp[jj][e] - dvec[ql]) * dfac;
         }
-      }
+      };
+      if (full) elementwise(std::false_type{});
+      else elementwise(std::true_type{});
       // ---- dV += P^T dO, dK += dS^T Q over the query k-steps 2 hf, 2 hf + 1
 #pragma unroll
       for (int kx = 0; kx < 2; ++kx) {
@@ -346,15 +373,17 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
           mma_16816<T>(acc[2 * u + 1], a, bk[2], bk[3]);
         }
       }
+      // lanes t and t ^ 1 swap halves: the even lane ends with columns
+      // 4 (t/2) .. +3 of row g, the odd lane the same columns of row g + 8
+      const int hr = tq & 1;
+      const int q = q0 + 16 * warp + 8 * hr + perm8(gq);
+      float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.Nq + q) * p.H + hq) * D + nh * NH * 8 + 4 * (tq >> 1);
 #pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        const int q = q0 + 16 * warp + 8 * hr + perm8(gq);
-        if (q < p.Nq) {
-          float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.Nq + q) * p.H + hq) * D + nh * NH * 8 + 2 * tq;
-#pragma unroll
-          for (int n = 0; n < NH; ++n) atomicAdd(reinterpret_cast<float2*>(dst + 8 * n),
-                                                 make_float2(acc[n][2 * hr], acc[n][2 * hr + 1]));
-        }
+      for (int n = 0; n < NH; ++n) {
+        const float s0 = hr ? acc[n][0] : acc[n][2], s1 = hr ? acc[n][1] : acc[n][3];
+        const float r0 = __shfl_xor_sync(0xffffffffu, s0, 1), r1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+        const float4 v4 = hr ? make_float4(r0, r1, acc[n][2], acc[n][3]) : make_float4(acc[n][0], acc[n][1], r0, r1);
+        if (q < p.Nq) atomicAdd(reinterpret_cast<float4*>(dst + 8 * n), v4);
       }
     }
   }
