@@ -539,10 +539,12 @@ def sweep(args):
                           "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
                           "flops": fwd_flops(w), "peak_source": peak_src, "l2": "flushed"}), flush=True)
         del x, out, lse
-    # backward of a forward workload: "bwd_" + its name; credited 2.5x the
-    # forward's flops (five products of the forward's size against two)
-    for w in W.FWD_WORKLOADS:
-        if "bwd_" + w.name not in names:
+    # backward of a forward workload: "bwd_" + its name ("bwd_det_" + its name
+    # for the deterministic mode); credited 2.5x the forward's flops (five
+    # products of the forward's size against two) in either mode
+    for w, det in [(w, det) for w in W.FWD_WORKLOADS for det in (False, True)]:
+        label = ("bwd_det_" if det else "bwd_") + w.name
+        if label not in names:
             continue
         x = W.make_fwd_inputs(w, device=dev)
         gen = torch.Generator().manual_seed(w.seed + 100)
@@ -554,7 +556,8 @@ def sweep(args):
         dq, dk, dv = torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"])
         ws = torch.empty(max(fa.fa_bwd_workspace_size(w.B, w.H, w.Nq, w.d), 16), dtype=torch.uint8, device=dev)
         run = lambda: fa.fa_bwd(x["q"], x["k"], x["v"], out, lse, dout, dq, dk, dv, w.scale, w.causal,
-                                w.window_left, w.window_right, x["slopes"], w.softcap, ws)
+                                w.window_left, w.window_right, x["slopes"], w.softcap, deterministic=det,
+                                workspace=ws)
         for _ in range(args.warmup):
             run()
         times = []
@@ -569,7 +572,7 @@ def sweep(args):
         ms = statistics.median([a.elapsed_time(b) for a, b in times])
         fl = 2.5 * fwd_flops(w)
         tf = fl / (ms * 1e-3) / 1e12
-        print(json.dumps({"workload": "bwd_" + w.name, "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+        print(json.dumps({"workload": label, "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
                           "frac_burst": round(tf / peaks["bf16_tflops"], 4),
                           "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
                           "flops": fl, "peak_source": peak_src, "l2": "flushed"}), flush=True)

@@ -81,7 +81,8 @@ def _lib_handle():
         L.fa_kvcache_workspace_size.restype = sz
         L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
         L.fa_bwd_workspace_size.restype = sz
-        L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i, vp, f, vp, sz, vp]
+        L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i, vp, f, i, vp, sz,
+                             vp]
         L.fa_bwd.restype = i
         L.fa_status_string.argtypes = [i]
         L.fa_status_string.restype = ctypes.c_char_p
@@ -170,11 +171,11 @@ def fa_bwd_workspace_size(B: int, H: int, Nq: int, d: int) -> int:
 
 
 def fa_bwd(q, k, v, out, lse, dout, dq, dk, dv, scale: float, causal: bool = False, window_left: int = -1,
-           window_right: int = -1, alibi_slopes=None, softcap: float = 0.0,
+           window_right: int = -1, alibi_slopes=None, softcap: float = 0.0, deterministic: bool = False,
            workspace: Optional[torch.Tensor] = None, stream=None) -> None:
     """Backward of fa_fwd / fa_fwd_gqa: q, out, dout, dq [B,Nq,H,d]; k, v, dk, dv [B,Nk,H_kv,d];
     lse fp32 [B,H,Nq] from the forward; workspace a byte tensor of fa_bwd_workspace_size bytes
-    (allocated here when None)."""
+    (allocated here when None); deterministic: dq summed in a fixed order (bit-for-bit repeatable)."""
     B, Nq, H, d = q.shape
     Nk, H_kv = k.shape[1], k.shape[2]
     for t in (q, k, v, out, lse, dout, dq, dk, dv):
@@ -195,7 +196,8 @@ def fa_bwd(q, k, v, out, lse, dout, dq, dk, dv, scale: float, causal: bool = Fal
     code = _lib_handle().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
                                 _ptr(dv), B, H, H_kv, Nq, Nk, d, _dtype_code(q), float(scale),
                                 int(bool(causal)), int(window_left), int(window_right), _ptr(alibi_slopes),
-                                float(softcap), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                float(softcap), int(bool(deterministic)), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(),
                                 _stream(stream))
     _check(code, "fa_bwd")
 

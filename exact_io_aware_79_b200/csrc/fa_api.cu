@@ -412,8 +412,10 @@ size_t fa_bwd_workspace_size(int B, int H, int Nq, int d) {
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
                  void* dq, void* dk, void* dv, int B, int H, int H_kv, int Nq, int Nk, int d, fa_dtype dtype,
                  float scale, int causal, int window_left, int window_right, const float* alibi_slopes,
-                 float softcap, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                 float softcap, int deterministic, void* workspace, size_t workspace_bytes,
+                 cudaStream_t stream) {
   if (B < 0 || H < 1 || Nq < 0 || Nk < 0) return FA_ERR_SHAPE;
+  if (deterministic != 0 && deterministic != 1) return FA_ERR_ARG;
   if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_SHAPE;
   if (Nq > kMaxSeq || Nk > kMaxSeq || static_cast<long long>(B) * H_kv > 65535) return FA_ERR_SHAPE;
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
@@ -466,6 +468,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, c
   p.window_left = window_left;
   p.window_right = window_right;
   p.use_softcap = softcap > 0.0f;
+  p.deterministic = deterministic;
   p.scale = scale;
   p.scale_log2 = scale * fa::kLog2e;
   p.cap_scale = softcap > 0.0f ? scale / softcap : 0.0f;

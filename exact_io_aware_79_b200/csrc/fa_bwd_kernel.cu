@@ -15,7 +15,10 @@
 // per 64-key block of one (b, cache head): dK and dV stay in registers while
 // the CTA walks the query blocks of every query head that reads the cache
 // head; dQ partials are added into an fp32 accumulator), bwd_dq_cast (dQ =
-// scale * accumulator, to the input type).
+// scale * accumulator, to the input type). The deterministic mode (the
+// pages' version 2.4 names a deterministic backward) drops the atomic dQ
+// partials and runs bwd_dq_kernel instead, which sums dQ over the key blocks
+// of each query block in a fixed order; every output then repeats bit for bit.
 //
 // bwd_kernel's products are warp-level m16n8k16 tensor-core MMAs; each of the
 // four warps owns 16 keys (the rows of its products). K, V and the double-
@@ -118,6 +121,8 @@ __device__ __forceinline__ bool key_visible(int pos, int j, int Nk, const BwdPar
   return true;
 }
 
+// Outside the deterministic mode the CTA also adds its dQ partials into the
+// fp32 accumulator; in it bwd_dq_kernel forms dQ instead.
 template <typename T, int D>
 __global__ void __launch_bounds__(kBwdWarps * 32, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -200,6 +205,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
 
   const int krow0 = warp * 16 + perm8(gq);  // this lane's product rows: krow0, krow0 + 8
   const bool alibi = p.slopes != nullptr;
+  const bool dq_on = !p.deterministic;
   bool failed = false;
   int issued = n_it > 1 ? 2 : n_it;
 
@@ -214,6 +220,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
   };
   float rv_next = n_it > 0 ? fetch_rowvec(0) : 0.0f;
 
+#pragma unroll 1
   for (int it = 0; it < n_it; ++it) {
     const int buf = it & 1;
     const int h = hk * G + it / n_qb;
@@ -334,7 +341,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
       }
       // ---- dS^T to shared memory: row = key (local), column = query position
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
+      for (int jj = 0; jj < 4 && dq_on; ++jj) {
         const int jt = 4 * hf + jj;
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
@@ -352,7 +359,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
     // ---- dQ (rows = query positions 16 w .. 16 w + 15) += dS K, in two halves of n-tiles
     const int hq = h;
 #pragma unroll
-    for (int nh = 0; nh < 2; ++nh) {
+    for (int nh = 0; nh < 2 && dq_on; ++nh) {
       float acc[NH][4];
 #pragma unroll
       for (int n = 0; n < NH; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
@@ -413,13 +420,245 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
   }
 }
 
+// Deterministic dQ: one CTA per 64-query block of one (b, query head); each
+// warp owns 16 queries and walks the visible key blocks in increasing order,
+// rebuilding S = Q K^T and dP = dO V^T, so dQ = scale * sum_j dS K is summed
+// in a fixed order (no atomics). Fragment bookkeeping mirrors bwd_kernel with
+// the roles of keys and queries swapped: product row g (g + 8) is query
+// 16 w + perm(g) (+ 8), column n of key n-tile j is key 8 j + perm(n).
+template <int D>
+struct DqCfg {
+  static constexpr int kTile = kBlk * D * 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffO = kTile;
+  static constexpr int kOffK = 2 * kTile;  // two buffers
+  static constexpr int kOffV = 4 * kTile;  // two buffers
+  static constexpr int kOffBar = 6 * kTile;
+  static constexpr int kSmem = 1024 + kOffBar + 64;
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kBwdWarps * 32, 2)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const BwdParams p) {
+  using C = DqCfg<D>;
+  constexpr int KS = D / 16;
+  constexpr int NT = D / 8;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint8_t* sQ = smem + C::kOffQ;
+  const uint8_t* sO = smem + C::kOffO;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);  // full[2], q
+  int* abort_flag = reinterpret_cast<int*>(bars + 3);
+  volatile int* abort = abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int qb = blockIdx.x;
+  const int b = blockIdx.y / p.H, h = blockIdx.y % p.H;
+  const int hk = h / (p.H / p.H_kv);
+  const int q0 = qb * kBlk;
+  const int off = p.Nk - p.Nq;
+
+  // key blocks that hold a key visible to a query of [q0, qmax]
+  const int qmax = min(q0 + kBlk - 1, p.Nq - 1);
+  long long k_lo = 0, k_hi = p.Nk - 1;
+  if (p.causal || p.window_right >= 0) {
+    const int right = p.window_right >= 0 ? (p.causal ? min(0, p.window_right) : p.window_right) : 0;
+    k_hi = min(k_hi, static_cast<long long>(qmax) + off + right);
+  }
+  if (p.window_left >= 0) k_lo = max(k_lo, static_cast<long long>(q0) + off - p.window_left);
+  const int kb_lo = k_lo <= k_hi ? static_cast<int>(k_lo / kBlk) : 0;
+  const int n_it = k_lo <= k_hi ? static_cast<int>(k_hi / kBlk) - kb_lo + 1 : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    mbar_init(&bars[2], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const uint64_t pol = l2_policy_evict_last();
+  auto issue = [&](int it) {
+    const int buf = it & 1;
+    const int k0 = (kb_lo + it) * kBlk;
+    mbar_arrive_expect_tx(&bars[buf], 2 * C::kTile);
+#pragma unroll
+    for (int hh = 0; hh < D / 64; ++hh) {
+      tma_load_4d(&tmK, &bars[buf], smem + C::kOffK + buf * C::kTile + hh * kBlk * 128, hh * 64, hk, k0, b, pol);
+      tma_load_4d(&tmV, &bars[buf], smem + C::kOffV + buf * C::kTile + hh * kBlk * 128, hh * 64, hk, k0, b, pol);
+    }
+  };
+  if (threadIdx.x == 0 && n_it > 0) {
+    mbar_arrive_expect_tx(&bars[2], 2 * C::kTile);
+#pragma unroll
+    for (int hh = 0; hh < D / 64; ++hh) {
+      tma_load_4d(&tmQ, &bars[2], smem + C::kOffQ + hh * kBlk * 128, hh * 64, h, q0, b, pol);
+      tma_load_4d(&tmO, &bars[2], smem + C::kOffO + hh * kBlk * 128, hh * 64, h, q0, b, pol);
+    }
+    issue(0);
+    if (n_it > 1) issue(1);
+  }
+
+  const int qrow0 = warp * 16 + perm8(gq);  // this lane's product rows: qrow0, qrow0 + 8
+  float lse2[2], dvr[2];
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    const int q = q0 + qrow0 + 8 * hr;
+    const size_t ri = (static_cast<size_t>(b) * p.H + h) * p.Nq + q;
+    lse2[hr] = q < p.Nq ? p.lse[ri] * kLog2e : -INFINITY;
+    dvr[hr] = q < p.Nq ? p.dvec[ri] : 0.0f;
+  }
+  const bool alibi = p.slopes != nullptr;
+  const float slope2 = alibi ? p.slopes[h] * kLog2e : 0.0f;
+  float dq[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) dq[n][0] = dq[n][1] = dq[n][2] = dq[n][3] = 0.0f;
+  bool failed = false;
+  int issued = n_it > 1 ? 2 : n_it;
+
+#pragma unroll 1
+  for (int it = 0; it < n_it; ++it) {
+    const int buf = it & 1;
+    const int k0 = (kb_lo + it) * kBlk;
+    bool ok = true;
+    if (it == 0) ok = mbar_wait(&bars[2], 0, abort);
+    ok = ok && mbar_wait(&bars[buf], (it >> 1) & 1, abort);
+    if (__syncthreads_or(!ok)) {
+      failed = true;
+      break;
+    }
+    const uint8_t* sK = smem + C::kOffK + buf * C::kTile;
+    const uint8_t* sV = smem + C::kOffV + buf * C::kTile;
+    const uint32_t sK_a = smem_addr(sK);
+    bool full = k0 + kBlk <= p.Nk && q0 + kBlk <= p.Nq;
+    if (p.causal || p.window_right >= 0) {
+      const int right = p.window_right >= 0 ? (p.causal ? min(0, p.window_right) : p.window_right) : 0;
+      full = full && k0 + kBlk - 1 <= q0 + off + right;
+    }
+    if (p.window_left >= 0) full = full && k0 >= q0 + kBlk - 1 + off - p.window_left;
+
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      // ---- S and dP for key n-tiles 4 hf .. 4 hf + 3
+      float sc[4][4], dp[4][4];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[jj][e] = dp[jj][e] = 0.0f;
+#pragma unroll
+      for (int i = 0; i < KS / 2; ++i) {
+        const int c = 4 * i + tq;
+        const uint4 q0v = *reinterpret_cast<const uint4*>(sQ + sw_off(qrow0, c));
+        const uint4 q1v = *reinterpret_cast<const uint4*>(sQ + sw_off(qrow0 + 8, c));
+        const uint4 o0v = *reinterpret_cast<const uint4*>(sO + sw_off(qrow0, c));
+        const uint4 o1v = *reinterpret_cast<const uint4*>(sO + sw_off(qrow0 + 8, c));
+        const uint32_t qa0[4] = {q0v.x, q1v.x, q0v.y, q1v.y}, qa1[4] = {q0v.z, q1v.z, q0v.w, q1v.w};
+        const uint32_t oa0[4] = {o0v.x, o1v.x, o0v.y, o1v.y}, oa1[4] = {o0v.z, o1v.z, o0v.w, o1v.w};
+        uint4 kw[4], vw[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int r = 8 * (4 * hf + jj) + perm8(gq);
+          kw[jj] = *reinterpret_cast<const uint4*>(sK + sw_off(r, c));
+          vw[jj] = *reinterpret_cast<const uint4*>(sV + sw_off(r, c));
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          mma_16816<T>(sc[jj], qa0, kw[jj].x, kw[jj].y);
+          mma_16816<T>(dp[jj], oa0, vw[jj].x, vw[jj].y);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          mma_16816<T>(sc[jj], qa1, kw[jj].z, kw[jj].w);
+          mma_16816<T>(dp[jj], oa1, vw[jj].z, vw[jj].w);
+        }
+      }
+      // ---- dS, elementwise (dp <- dS)
+      auto elementwise = [&](auto masked_tag) {
+        constexpr bool kMasked = decltype(masked_tag)::value;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int hr = e >> 1;
+            const int ql = qrow0 + 8 * hr;
+            const int key = k0 + 8 * (4 * hf + jj) + tq + 4 * (e & 1);
+            const int pos = q0 + ql + off;
+            float logit2, dfac = 1.0f;
+            if (p.use_softcap) {
+              const float th = tanh_via_exp2(sc[jj][e] * p.cap_scale);
+              logit2 = th * p.cap_log2;
+              dfac = 1.0f - th * th;
+            } else {
+              logit2 = sc[jj][e] * p.scale_log2;
+            }
+            if (alibi) logit2 -= slope2 * fabsf(static_cast<float>(pos - key));
+            float pr = ex2(logit2 - lse2[hr]);
+            if constexpr (kMasked) {
+              if (!(q0 + ql < p.Nq && key_visible(pos, key, p.Nk, p))) pr = 0.0f;
+            }
+            dp[jj][e] = pr * (dp[jj][e] - dvr[hr]) * dfac;
+          }
+        }
+      };
+      if (full) elementwise(std::false_type{});
+      else elementwise(std::true_type{});
+      // ---- dQ += dS K over the key k-steps 2 hf, 2 hf + 1
+#pragma unroll
+      for (int kx = 0; kx < 2; ++kx) {
+        const int kk = 2 * hf + kx;
+        const uint32_t da[4] = {pack2<T>(dp[2 * kx][0], dp[2 * kx][1]), pack2<T>(dp[2 * kx][2], dp[2 * kx][3]),
+                                pack2<T>(dp[2 * kx + 1][0], dp[2 * kx + 1][1]),
+                                pack2<T>(dp[2 * kx + 1][2], dp[2 * kx + 1][3])};
+        const int brow = 16 * kk + ((lane >> 3) & 1) * 8 + perm8(lane & 7);
+#pragma unroll
+        for (int u = 0; u < NT / 2; ++u) {
+          const int cc = 2 * u + (lane >> 4);
+          uint32_t bk[4];
+          ldsm_x4_trans(bk, sK_a + sw_off(brow, cc));
+          mma_16816<T>(dq[2 * u], da, bk[0], bk[1]);
+          mma_16816<T>(dq[2 * u + 1], da, bk[2], bk[3]);
+        }
+      }
+    }
+    __syncthreads();  // this block's K and V buffers are free
+    if (threadIdx.x == 0 && issued < n_it) {
+      issue(issued);
+      ++issued;
+    }
+  }
+  if (threadIdx.x == 0 && failed) {
+    int dummy = 0;
+    for (int i = max(0, issued - 2); i < issued; ++i) mbar_wait(&bars[i & 1], (i >> 1) & 1, &dummy);
+    mbar_wait(&bars[2], 0, &dummy);
+  }
+  const float nan = __int_as_float(0x7fc00000);
+#pragma unroll
+  for (int hr = 0; hr < 2; ++hr) {
+    const int q = q0 + qrow0 + 8 * hr;
+    if (q >= p.Nq) continue;
+    T* out = reinterpret_cast<T*>(p.dq) + ((static_cast<size_t>(b) * p.Nq + q) * p.H + h) * D + 2 * tq;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const float x0 = failed ? nan : dq[n][2 * hr] * p.scale, x1 = failed ? nan : dq[n][2 * hr + 1] * p.scale;
+      *reinterpret_cast<uint32_t*>(out + 8 * n) = pack2<T>(x0, x1);
+    }
+  }
+}
+
 template <typename T, int D>
 cudaError_t launch(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                    const CUtensorMap& tmO, cudaStream_t stream) {
   const long long rows = static_cast<long long>(p.B) * p.Nq * p.H;
   const long long elems = rows * D;
-  cudaError_t e = cudaMemsetAsync(p.dq_acc, 0, static_cast<size_t>(elems) * sizeof(float), stream);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (!p.deterministic) {
+    e = cudaMemsetAsync(p.dq_acc, 0, static_cast<size_t>(elems) * sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+  }
   if (rows > 0) {
     const long long threads = rows * (D / 8);
     bwd_rowdot_kernel<T, D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p);
@@ -434,6 +673,15 @@ cudaError_t launch(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap
   kernel<<<grid, kBwdWarps * 32, C::kSmem, stream>>>(tmQ, tmK, tmV, tmO, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (p.deterministic) {
+    using Cq = DqCfg<D>;
+    auto dq_kernel = bwd_dq_kernel<T, D>;
+    e = cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cq::kSmem);
+    if (e != cudaSuccess) return e;
+    dim3 g2((p.Nq + kBlk - 1) / kBlk, p.B * p.H);
+    dq_kernel<<<g2, kBwdWarps * 32, Cq::kSmem, stream>>>(tmQ, tmK, tmV, tmO, p);
+    return cudaGetLastError();
+  }
   const long long n4 = elems / 4;
   if (n4 > 0) bwd_dq_cast_kernel<T><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(p, n4);
   return cudaGetLastError();

@@ -86,6 +86,7 @@ struct BwdParams {
   int B, H, H_kv, Nq, Nk;
   int causal, window_left, window_right;
   int use_softcap;
+  int deterministic;  // 1: dQ summed in a fixed order (no atomics)
   float scale;       // softmax scale (dQ, dK factor)
   float scale_log2;  // scale * log2(e)            (no softcap)
   float cap_scale;   // scale / softcap             (softcap)

@@ -277,9 +277,13 @@ fa_status fa_kvcache_append(const void *k_new, const void *v_new, void *k_cache,
  *   dq = scale * dS k;  dk = scale * dS^T q
  * Grouped-query k, v heads (H_kv < H) receive the sum over the query heads
  * that read them. P is rebuilt tile by tile from lse; no N x N array is
- * written. dq is accumulated in fp32 in the workspace across key blocks with
- * atomic adds, so its last bits may differ from run to run (the order of the
- * additions is not fixed); dk and dv are summed in a fixed order.
+ * written. dk and dv are summed in a fixed order. With deterministic = 0, dq
+ * is accumulated in fp32 in the workspace across key blocks with atomic
+ * adds, so its last bits may differ from run to run; with deterministic = 1
+ * (the deterministic backward named in "Flash-Attention v2.0 到 v2.7 更新",
+ * section v2.4) a separate pass sums dq over the key blocks of each query
+ * block in a fixed order, rebuilding S and dP there (about 1.4x the
+ * products), and every output repeats bit for bit.
  *
  *   q, out, dout, dq   [B, Nq, H, d]       contiguous, dtype
  *   k, v, dk, dv       [B, Nk, H_kv, d]    contiguous, dtype
@@ -287,6 +291,7 @@ fa_status fa_kvcache_append(const void *k_new, const void *v_new, void *k_cache,
  *   workspace          fa_bwd_workspace_size(B, H, Nq, d) bytes of device
  *                      memory, 16-byte aligned (fp32 dq accumulator + D)
  *   scale, causal, window_left, window_right, alibi_slopes, softcap: as fa_fwd
+ *   deterministic      0 or 1 (see above)
  * Outputs dq, dk, dv are overwritten (not accumulated). The caller owns every
  * buffer; the call only enqueues work on `stream`.
  *
@@ -299,8 +304,8 @@ size_t fa_bwd_workspace_size(int B, int H, int Nq, int d);
 fa_status fa_bwd(const void *q, const void *k, const void *v, const void *out, const float *lse,
                  const void *dout, void *dq, void *dk, void *dv, int B, int H, int H_kv, int Nq, int Nk,
                  int d, fa_dtype dtype, float scale, int causal, int window_left, int window_right,
-                 const float *alibi_slopes, float softcap, void *workspace, size_t workspace_bytes,
-                 cudaStream_t stream);
+                 const float *alibi_slopes, float softcap, int deterministic, void *workspace,
+                 size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Number of splits fa_fwd_kvcache uses for these sizes: num_splits itself

@@ -252,13 +252,15 @@ def test_qkvpacked_validation(lib):
 def test_bwd_validation(lib):
     def bw(**kw):
         a = dict(q=P, k=P, v=P, out=P, lse=P, dout=P, dq=P, dk=P, dv=P, B=2, H=8, H_kv=2, Nq=100, Nk=200, d=128,
-                 dtype=1, scale=0.1, causal=1, wl=-1, wr=-1, slopes=None, cap=0.0, ws=P,
+                 dtype=1, scale=0.1, causal=1, wl=-1, wr=-1, slopes=None, cap=0.0, det=0, ws=P,
                  ws_bytes=lib.fa_bwd_workspace_size(2, 8, 100, 128))
         a.update(kw)
         return lib.fa_bwd(a["q"], a["k"], a["v"], a["out"], a["lse"], a["dout"], a["dq"], a["dk"], a["dv"], a["B"],
                           a["H"], a["H_kv"], a["Nq"], a["Nk"], a["d"], a["dtype"], a["scale"], a["causal"], a["wl"],
-                          a["wr"], a["slopes"], a["cap"], a["ws"], a["ws_bytes"], None)
+                          a["wr"], a["slopes"], a["cap"], a["det"], a["ws"], a["ws_bytes"], None)
     assert bw() == DEVICE
+    assert bw(det=1) == DEVICE
+    assert bw(det=2) == ARG
     assert bw(H_kv=3) == SHAPE
     assert bw(H_kv=16) == SHAPE
     assert bw(B=40000, H_kv=2) == SHAPE          # B * H_kv > 65535

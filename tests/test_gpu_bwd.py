@@ -34,7 +34,7 @@ def inputs(B, H, H_kv, Nq, Nk, d, dtype, seed):
     return q, k, v, do
 
 
-def run(q, k, v, do, scale, causal=False, wl=-1, wr=-1, slopes=None, cap=0.0):
+def run(q, k, v, do, scale, causal=False, wl=-1, wr=-1, slopes=None, cap=0.0, det=False):
     B, Nq, H, d = q.shape
     qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
     out = torch.empty_like(qd)
@@ -42,7 +42,7 @@ def run(q, k, v, do, scale, causal=False, wl=-1, wr=-1, slopes=None, cap=0.0):
     sl = None if slopes is None else slopes.cuda()
     fa.fa_fwd_gqa(qd, kd, vd, out, lse, scale, causal, wl, wr, sl, cap)
     dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
-    fa.fa_bwd(qd, kd, vd, out, lse, dod, dq, dk, dv, scale, causal, wl, wr, sl, cap)
+    fa.fa_bwd(qd, kd, vd, out, lse, dod, dq, dk, dv, scale, causal, wl, wr, sl, cap, deterministic=det)
     torch.cuda.synchronize()
     return dq, dk, dv
 
@@ -67,13 +67,14 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("det", [False, True], ids=["atomic_dq", "deterministic"])
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "B%dH%dkv%dq%dk%dd%d" % c[:6])
-def test_bwd_matches_oracle(case):
+def test_bwd_matches_oracle(case, det):
     B, H, H_kv, Nq, Nk, d, dtype, causal, wl, wr, alibi, cap = case
     q, k, v, do = inputs(B, H, H_kv, Nq, Nk, d, dtype, seed=Nq + Nk + H)
     slopes = W.alibi_slopes(H) if alibi else None
     scale = 1.0 / math.sqrt(d)
-    dq, dk, dv = run(q, k, v, do, scale, causal, wl, wr, slopes, cap)
+    dq, dk, dv = run(q, k, v, do, scale, causal, wl, wr, slopes, cap, det)
     rq, rk, rv = oracle.attn_bwd(q, k, v, do, scale, causal, wl, wr, slopes, cap)
     check(dq, rq, dtype, "dq")
     check(dk, rk, dtype, "dk")
@@ -86,6 +87,16 @@ def test_bwd_dk_dv_are_reproducible_bit_for_bit():
     b = run(q, k, v, do, 0.1, True)
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
     assert (a[0].float() - b[0].float()).abs().max().item() <= 1e-2 * a[0].float().abs().max().item()
+
+
+def test_bwd_deterministic_mode_repeats_every_output_bit_for_bit():
+    q, k, v, do = inputs(1, 4, 2, 300, 300, 128, torch.bfloat16, seed=3)
+    a = run(q, k, v, do, 0.1, True, det=True)
+    b = run(q, k, v, do, 0.1, True, det=True)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    c = run(q, k, v, do, 0.1, True, det=False)   # same dK, dV as the atomic mode
+    assert torch.equal(a[1], c[1]) and torch.equal(a[2], c[2])
 
 
 def test_bwd_empty_sides():
