@@ -101,6 +101,23 @@ bool make_cache_map(CUtensorMap* map, const void* base, bool bf16, int num_pages
   return r == CUDA_SUCCESS;
 }
 
+// fp32 [B, N, H, d] tensor as a 4-D map (d, H, N, B) with (32, 1, 64, 1)
+// boxes and 128-byte swizzle (the backward's dQ accumulator).
+bool make_map_f32(CUtensorMap* map, void* base, int B, int N, int H, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t t = static_cast<cuuint64_t>(H) * d;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 4, t * 4, static_cast<cuuint64_t>(N) * t * 4};
+  cuuint32_t box[4] = {32, 1, 64, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool finite(float x) { return std::isfinite(x); }
 
 // Automatic split count: enough splits that a split of the longest possible
@@ -443,9 +460,10 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, c
   if (Nk == 0) return cudaMemsetAsync(dq, 0, q_bytes, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 
   const bool bf16 = dtype == FA_BF16;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv, to, tdq;
   if (!make_map(&tq, q, bf16, B, Nq, H, d, 0, 64) || !make_map(&to, dout, bf16, B, Nq, H, d, 0, 64) ||
-      !make_map(&tk, k, bf16, B, Nk, H_kv, d, 0, 64) || !make_map(&tv, v, bf16, B, Nk, H_kv, d, 0, 64))
+      !make_map(&tk, k, bf16, B, Nk, H_kv, d, 0, 64) || !make_map(&tv, v, bf16, B, Nk, H_kv, d, 0, 64) ||
+      !make_map_f32(&tdq, workspace, B, Nq, H, d))
     return FA_ERR_CUDA;
   fa::BwdParams p{};
   const size_t rows = static_cast<size_t>(B) * H * Nq;
@@ -473,7 +491,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, c
   p.scale_log2 = scale * fa::kLog2e;
   p.cap_scale = softcap > 0.0f ? scale / softcap : 0.0f;
   p.cap_log2 = softcap * fa::kLog2e;
-  return fa::launch_bwd(bf16, d, p, tq, tk, tv, to, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return fa::launch_bwd(bf16, d, p, tq, tk, tv, to, tdq, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // extern "C"

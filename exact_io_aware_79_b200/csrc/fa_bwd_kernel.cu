@@ -14,7 +14,8 @@
 // Kernels: bwd_rowdot (D, one warp per 32 / (d/8) rows), bwd_kernel (one CTA
 // per 64-key block of one (b, cache head): dK and dV stay in registers while
 // the CTA walks the query blocks of every query head that reads the cache
-// head; dQ partials are added into an fp32 accumulator), bwd_dq_cast (dQ =
+// head; dQ partials are added into an fp32 accumulator by TMA reduce-add),
+// bwd_dq_cast (dQ =
 // scale * accumulator, to the input type). The deterministic mode (the
 // pages' version 2.4 names a deterministic backward) drops the atomic dQ
 // partials and runs bwd_dq_kernel instead, which sums dQ over the key blocks
@@ -127,7 +128,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kBwdWarps * 32, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-               const BwdParams p) {
+               const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int KS = D / 16;  // k-steps over the head dimension
   constexpr int NT = D / 8;   // n-tiles over the head dimension
@@ -352,48 +353,64 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
       }
     }
     __syncthreads();  // dS^T complete; this block's Q and dO buffers are free
+    if (dq_on) {
+      // ---- dQ (rows = query positions 16 w .. 16 w + 15) = dS K, in two halves of n-tiles,
+      // staged as fp32 in this block's idle Q and dO buffers (64-row boxes of 32 columns,
+      // 128-byte swizzle) and added into the accumulator by TMA reduce-add
+      uint8_t* stage[2] = {smem + C::kOffQ + buf * C::kTile, smem + C::kOffO + buf * C::kTile};
+      constexpr int kBoxesPerBuf = D / 64;  // 8 KB fp32 boxes per 16-bit tile buffer
+#pragma unroll
+      for (int nh = 0; nh < 2; ++nh) {
+        float acc[NH][4];
+#pragma unroll
+        for (int n = 0; n < NH; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk) {
+          const int mi = lane >> 3;
+          const int akey = 16 * kk + (mi >> 1) * 8 + (lane & 7);
+          const int achunk = 2 * warp + (mi & 1);
+          uint32_t a[4];
+          ldsm_x4_trans(a, sS_a + akey * 128 + ((achunk ^ (akey & 7)) << 4));
+          const int brow = 16 * kk + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+          for (int u = 0; u < NH / 2; ++u) {
+            const int cc = nh * NH + 2 * u + (lane >> 4);
+            uint32_t bk[4];
+            ldsm_x4_trans(bk, sK_a + sw_off(brow, cc));
+            mma_16816<T>(acc[2 * u], a, bk[0], bk[1]);
+            mma_16816<T>(acc[2 * u + 1], a, bk[2], bk[3]);
+          }
+        }
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int row = 16 * warp + 8 * hr + perm8(gq);
+#pragma unroll
+          for (int n = 0; n < NH; ++n) {
+            const int col = nh * NH * 8 + 8 * n + 2 * tq;
+            const int box = col >> 5, bcol = col & 31;
+            uint8_t* dst = stage[box / kBoxesPerBuf] + (box % kBoxesPerBuf) * (kBlk * 128) + row * 128 +
+                           ((((bcol >> 2) ^ (row & 7))) << 4) + (bcol & 3) * 4;
+            *reinterpret_cast<float2*>(dst) = make_float2(acc[n][2 * hr], acc[n][2 * hr + 1]);
+          }
+        }
+      }
+      fence_proxy_async_shared();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+#pragma unroll
+        for (int box = 0; box < D / 32; ++box)
+          tma_reduce_add_4d(&tmDQ, stage[box / kBoxesPerBuf] + (box % kBoxesPerBuf) * (kBlk * 128), box * 32, h, q0,
+                            b);
+        bulk_commit_group();
+        bulk_wait_read_all();  // the staging buffers are reloaded next
+      }
+    }
     if (threadIdx.x == 0 && issued < n_it) {
       issue(issued);
       ++issued;
     }
-    // ---- dQ (rows = query positions 16 w .. 16 w + 15) += dS K, in two halves of n-tiles
-    const int hq = h;
-#pragma unroll
-    for (int nh = 0; nh < 2 && dq_on; ++nh) {
-      float acc[NH][4];
-#pragma unroll
-      for (int n = 0; n < NH; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
-#pragma unroll
-      for (int kk = 0; kk < kBlk / 16; ++kk) {
-        const int mi = lane >> 3;
-        const int akey = 16 * kk + (mi >> 1) * 8 + (lane & 7);
-        const int achunk = 2 * warp + (mi & 1);
-        uint32_t a[4];
-        ldsm_x4_trans(a, sS_a + akey * 128 + ((achunk ^ (akey & 7)) << 4));
-        const int brow = 16 * kk + (mi & 1) * 8 + (lane & 7);
-#pragma unroll
-        for (int u = 0; u < NH / 2; ++u) {
-          const int cc = nh * NH + 2 * u + (lane >> 4);
-          uint32_t bk[4];
-          ldsm_x4_trans(bk, sK_a + sw_off(brow, cc));
-          mma_16816<T>(acc[2 * u], a, bk[0], bk[1]);
-          mma_16816<T>(acc[2 * u + 1], a, bk[2], bk[3]);
-        }
-      }
-      // lanes t and t ^ 1 swap halves: the even lane ends with columns
-      // 4 (t/2) .. +3 of row g, the odd lane the same columns of row g + 8
-      const int hr = tq & 1;
-      const int q = q0 + 16 * warp + 8 * hr + perm8(gq);
-      float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.Nq + q) * p.H + hq) * D + nh * NH * 8 + 4 * (tq >> 1);
-#pragma unroll
-      for (int n = 0; n < NH; ++n) {
-        const float s0 = hr ? acc[n][0] : acc[n][2], s1 = hr ? acc[n][1] : acc[n][3];
-        const float r0 = __shfl_xor_sync(0xffffffffu, s0, 1), r1 = __shfl_xor_sync(0xffffffffu, s1, 1);
-        const float4 v4 = hr ? make_float4(r0, r1, acc[n][2], acc[n][3]) : make_float4(acc[n][0], acc[n][1], r0, r1);
-        if (q < p.Nq) atomicAdd(reinterpret_cast<float4*>(dst + 8 * n), v4);
-      }
-    }
   }
+  if (threadIdx.x == 0) bulk_wait_all();
   // loads still in flight must land before the CTA exits
   if (threadIdx.x == 0 && failed) {
     int dummy = 0;
@@ -651,7 +668,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2)
 
 template <typename T, int D>
 cudaError_t launch(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                   const CUtensorMap& tmO, cudaStream_t stream) {
+                   const CUtensorMap& tmO, const CUtensorMap& tmDQ, cudaStream_t stream) {
   const long long rows = static_cast<long long>(p.B) * p.Nq * p.H;
   const long long elems = rows * D;
   cudaError_t e = cudaSuccess;
@@ -670,7 +687,7 @@ cudaError_t launch(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid((p.Nk + kBlk - 1) / kBlk, p.B * p.H_kv);
-  kernel<<<grid, kBwdWarps * 32, C::kSmem, stream>>>(tmQ, tmK, tmV, tmO, p);
+  kernel<<<grid, kBwdWarps * 32, C::kSmem, stream>>>(tmQ, tmK, tmV, tmO, tmDQ, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (p.deterministic) {
@@ -690,11 +707,12 @@ cudaError_t launch(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap
 }  // namespace
 
 cudaError_t launch_bwd(bool bf16, int d, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                       const CUtensorMap& tmV, const CUtensorMap& tmO, cudaStream_t stream) {
-  if (bf16) return d == 128 ? launch<__nv_bfloat16, 128>(p, tmQ, tmK, tmV, tmO, stream)
-                            : launch<__nv_bfloat16, 64>(p, tmQ, tmK, tmV, tmO, stream);
-  return d == 128 ? launch<__half, 128>(p, tmQ, tmK, tmV, tmO, stream)
-                  : launch<__half, 64>(p, tmQ, tmK, tmV, tmO, stream);
+                       const CUtensorMap& tmV, const CUtensorMap& tmO, const CUtensorMap& tmDQ,
+                       cudaStream_t stream) {
+  if (bf16) return d == 128 ? launch<__nv_bfloat16, 128>(p, tmQ, tmK, tmV, tmO, tmDQ, stream)
+                            : launch<__nv_bfloat16, 64>(p, tmQ, tmK, tmV, tmO, tmDQ, stream);
+  return d == 128 ? launch<__half, 128>(p, tmQ, tmK, tmV, tmO, tmDQ, stream)
+                  : launch<__half, 64>(p, tmQ, tmK, tmV, tmO, tmDQ, stream);
 }
 
 }  // namespace fa

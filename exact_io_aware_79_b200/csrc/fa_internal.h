@@ -94,9 +94,11 @@ struct BwdParams {
 };
 
 // tmQ/tmO: (d, H, Nq, B) maps of Q and dO, tmK/tmV: (d, H_kv, Nk, B) maps of
-// K and V, all with (64, 1, 64, 1) boxes and 128-byte swizzle.
+// K and V, all with (64, 1, 64, 1) boxes and 128-byte swizzle; tmDQ: the fp32
+// dQ accumulator as (d, H, Nq, B) with (32, 1, 64, 1) boxes, 128-byte swizzle.
 cudaError_t launch_bwd(bool bf16, int d, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                       const CUtensorMap& tmV, const CUtensorMap& tmO, cudaStream_t stream);
+                       const CUtensorMap& tmV, const CUtensorMap& tmO, const CUtensorMap& tmDQ,
+                       cudaStream_t stream);
 
 // Writes n_new new tokens per sequence into the paged caches at positions
 // cache_seqlens[b] .. cache_seqlens[b] + n_new - 1.
