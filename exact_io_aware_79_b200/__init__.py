@@ -84,6 +84,9 @@ def _lib_handle():
         L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i, vp, f, i, vp, sz,
                              vp]
         L.fa_bwd.restype = i
+        L.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, i, i, i,
+                                    vp, f, i, vp, sz, vp]
+        L.fa_bwd_varlen.restype = i
         L.fa_status_string.argtypes = [i]
         L.fa_status_string.restype = ctypes.c_char_p
         _LIB = L
@@ -200,6 +203,40 @@ def fa_bwd(q, k, v, out, lse, dout, dq, dk, dv, scale: float, causal: bool = Fal
                                 workspace.numel() * workspace.element_size(),
                                 _stream(stream))
     _check(code, "fa_bwd")
+
+
+def fa_bwd_varlen(q, k, v, out, lse, dout, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                  max_seqlen_k: int, scale: float, causal: bool = False, window_left: int = -1,
+                  window_right: int = -1, alibi_slopes=None, softcap: float = 0.0, deterministic: bool = False,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Backward of fa_fwd_varlen: q, out, dout, dq [total_q,H,d]; k, v, dk, dv [total_k,H_kv,d];
+    lse fp32 [H,total_q]; cu_seqlens_* int32 [B+1] on the device."""
+    total_q, H, d = q.shape
+    total_k, H_kv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.numel() - 1
+    for t in (q, k, v, out, lse, dout, dq, dk, dv, cu_seqlens_q, cu_seqlens_k):
+        if not t.is_contiguous():
+            raise ValueError("fa_bwd_varlen needs contiguous tensors")
+    if tuple(k.shape) != (total_k, H_kv, d) or tuple(v.shape) != tuple(k.shape) or \
+            tuple(dk.shape) != tuple(k.shape) or tuple(dv.shape) != tuple(k.shape) or \
+            tuple(out.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape) or \
+            tuple(dq.shape) != tuple(q.shape) or cu_seqlens_k.numel() != B + 1:
+        raise ValueError("fa_bwd_varlen: shape mismatch")
+    if tuple(lse.shape) != (H, total_q) or lse.dtype != torch.float32:
+        raise ValueError("fa_bwd_varlen: lse must be fp32 [H, total_q]")
+    if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
+        raise ValueError("fa_bwd_varlen: cu_seqlens must be int32")
+    need = fa_bwd_workspace_size(1, H, total_q, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    code = _lib_handle().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                                       _ptr(dk), _ptr(dv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, H, H_kv,
+                                       int(max_seqlen_q), int(max_seqlen_k), total_q, total_k, d, _dtype_code(q),
+                                       float(scale), int(bool(causal)), int(window_left), int(window_right),
+                                       _ptr(alibi_slopes), float(softcap), int(bool(deterministic)),
+                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream(stream))
+    _check(code, "fa_bwd_varlen")
 
 
 def fa_fwd_qkvpacked(qkv, out, lse, scale: float, causal: bool = False, window_left: int = -1,

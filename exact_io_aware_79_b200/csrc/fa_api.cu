@@ -494,4 +494,84 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, c
   return fa::launch_bwd(bf16, d, p, tq, tk, tv, to, tdq, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                        const int* cu_seqlens_k, int B, int H, int H_kv, int max_seqlen_q, int max_seqlen_k,
+                        int total_q, int total_k, int d, fa_dtype dtype, float scale, int causal, int window_left,
+                        int window_right, const float* alibi_slopes, float softcap, int deterministic,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || H < 1 || max_seqlen_q < 0 || max_seqlen_k < 0 || total_q < 0 || total_k < 0) return FA_ERR_SHAPE;
+  if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_SHAPE;
+  if (max_seqlen_q > kMaxSeq || max_seqlen_k > kMaxSeq || total_q > kMaxSeq || total_k > kMaxSeq ||
+      static_cast<long long>(B) * H > 65535)
+    return FA_ERR_SHAPE;
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  if (!finite(scale) || !finite(softcap) || softcap < 0.0f) return FA_ERR_ARG;
+  if (window_left < -1 || window_right < -1 || (causal != 0 && causal != 1)) return FA_ERR_ARG;
+  if (deterministic != 0 && deterministic != 1) return FA_ERR_ARG;
+  if (total_q == 0 && total_k == 0) return FA_OK;
+  if (B > 0 && (!cu_seqlens_q || !cu_seqlens_k)) return FA_ERR_NULL;
+  if (total_k > 0 && (!k || !v || !dk || !dv)) return FA_ERR_NULL;
+  if (total_q > 0 && (!q || !out || !lse || !dout || !dq)) return FA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return FA_ERR_ARG;
+  const bool work = B > 0 && total_q > 0 && total_k > 0 && max_seqlen_q > 0 && max_seqlen_k > 0;
+  if (work) {
+    const size_t need = fa_bwd_workspace_size(1, H, total_q, d);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  }
+  fa_status st = check_device();
+  if (st != FA_OK) return st;
+  const size_t kv_bytes = static_cast<size_t>(total_k) * H_kv * d * 2;
+  const size_t q_bytes = static_cast<size_t>(total_q) * H * d * 2;
+  if (!work) {
+    // no query or no key anywhere: the gradients that exist are zero
+    if (total_k > 0 && (cudaMemsetAsync(dk, 0, kv_bytes, stream) != cudaSuccess ||
+                        cudaMemsetAsync(dv, 0, kv_bytes, stream) != cudaSuccess))
+      return FA_ERR_CUDA;
+    if (total_q > 0 && cudaMemsetAsync(dq, 0, q_bytes, stream) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_OK;
+  }
+  const bool bf16 = dtype == FA_BF16;
+  CUtensorMap tq, tk, tv, to, tdq;
+  if (!make_map(&tq, q, bf16, 1, total_q, H, d, 0, 64) || !make_map(&to, dout, bf16, 1, total_q, H, d, 0, 64) ||
+      !make_map(&tk, k, bf16, 1, total_k, H_kv, d, 0, 64) || !make_map(&tv, v, bf16, 1, total_k, H_kv, d, 0, 64) ||
+      !make_map_f32(&tdq, workspace, 1, total_q, H, d))
+    return FA_ERR_CUDA;
+  fa::BwdParams p{};
+  const size_t rows = static_cast<size_t>(total_q) * H;
+  p.out = out;
+  p.dout = dout;
+  p.lse = lse;
+  p.dq_acc = static_cast<float*>(workspace);
+  p.dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                    ((rows * d * sizeof(float) + 255) & ~size_t(255)));
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.slopes = alibi_slopes;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  p.B = B;
+  p.H = H;
+  p.H_kv = H_kv;
+  p.Nq = max_seqlen_q;
+  p.Nk = max_seqlen_k;
+  p.causal = causal;
+  p.window_left = window_left;
+  p.window_right = window_right;
+  p.use_softcap = softcap > 0.0f;
+  p.deterministic = deterministic;
+  p.scale = scale;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.cap_scale = softcap > 0.0f ? scale / softcap : 0.0f;
+  p.cap_log2 = softcap * fa::kLog2e;
+  return fa::launch_bwd(bf16, d, p, tq, tk, tv, to, tdq, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // extern "C"

@@ -124,6 +124,35 @@ __device__ __forceinline__ bool key_visible(int pos, int j, int Nk, const BwdPar
 
 // Outside the deterministic mode the CTA also adds its dQ partials into the
 // fp32 accumulator; in it bwd_dq_kernel forms dQ instead.
+// Sequence b's lengths and first rows (packed layout), or the fixed-length
+// problem's; false when its offsets break the contract (the sequence is
+// skipped).
+__device__ __forceinline__ bool bwd_seq(const BwdParams& p, int b, int& Nq, int& Nk, long long& qrow,
+                                        long long& krow) {
+  if (p.cu_q == nullptr) {
+    Nq = p.Nq;
+    Nk = p.Nk;
+    qrow = static_cast<long long>(b) * p.Nq;
+    krow = static_cast<long long>(b) * p.Nk;
+    return true;
+  }
+  const int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
+  if (q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 > p.Nq) return false;
+  if (k0 < 0 || k1 < k0 || k1 > p.total_k || k1 - k0 > p.Nk) return false;
+  Nq = q1 - q0;
+  Nk = k1 - k0;
+  qrow = q0;
+  krow = k0;
+  return true;
+}
+
+// Index of (query head h, query q of this sequence) in lse and dvec:
+// [B, H, Nq] for fixed lengths, [H, total_q] packed.
+__device__ __forceinline__ size_t rowvec_index(const BwdParams& p, int b, int h, long long qrow, int q) {
+  return p.cu_q == nullptr ? (static_cast<size_t>(b) * p.H + h) * p.Nq + q
+                           : static_cast<size_t>(h) * p.total_q + static_cast<size_t>(qrow + q);
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kBwdWarps * 32, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -150,11 +179,18 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
   const int b = blockIdx.y / p.H_kv, hk = blockIdx.y % p.H_kv;
   const int G = p.H / p.H_kv;
   const int k0 = kb * kBlk;
-  const int off = p.Nk - p.Nq;  // query i sits at key position i + off
+  int Nq, Nk;
+  long long qrow, krow;
+  if (!bwd_seq(p, b, Nq, Nk, qrow, krow) || k0 >= Nk) return;  // uniform over the CTA
+  // tensor-map coordinates: (row, batch) = (q, b) for fixed lengths, (qrow + q, 0) packed
+  const int tb = p.cu_q == nullptr ? b : 0;
+  const int tq0 = p.cu_q == nullptr ? 0 : static_cast<int>(qrow);
+  const int tk0 = p.cu_q == nullptr ? 0 : static_cast<int>(krow);
+  const int off = Nk - Nq;  // query i sits at key position i + off
 
   // query rows that can see a key of [k0, k1)
-  const int k1 = min(k0 + kBlk, p.Nk);
-  long long q_lo = 0, q_hi = p.Nq - 1;
+  const int k1 = min(k0 + kBlk, Nk);
+  long long q_lo = 0, q_hi = Nq - 1;
   {
     int right = -1;  // keys j <= pos + right are the only visible ones (when >= 0)
     if (p.causal) right = 0;
@@ -183,16 +219,18 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
     mbar_arrive_expect_tx(&bars[buf], 2 * C::kTile);
 #pragma unroll
     for (int hh = 0; hh < D / 64; ++hh) {
-      tma_load_4d(&tmQ, &bars[buf], smem + C::kOffQ + buf * C::kTile + hh * kBlk * 128, hh * 64, h, q0, b, pol);
-      tma_load_4d(&tmO, &bars[buf], smem + C::kOffO + buf * C::kTile + hh * kBlk * 128, hh * 64, h, q0, b, pol);
+      tma_load_4d(&tmQ, &bars[buf], smem + C::kOffQ + buf * C::kTile + hh * kBlk * 128, hh * 64, h, tq0 + q0, tb,
+                  pol);
+      tma_load_4d(&tmO, &bars[buf], smem + C::kOffO + buf * C::kTile + hh * kBlk * 128, hh * 64, h, tq0 + q0, tb,
+                  pol);
     }
   };
   if (threadIdx.x == 0 && n_it > 0) {
     mbar_arrive_expect_tx(&bars[2], 2 * C::kTile);
 #pragma unroll
     for (int hh = 0; hh < D / 64; ++hh) {
-      tma_load_4d(&tmK, &bars[2], sK + hh * kBlk * 128, hh * 64, hk, k0, b, pol);
-      tma_load_4d(&tmV, &bars[2], sV + hh * kBlk * 128, hh * 64, hk, k0, b, pol);
+      tma_load_4d(&tmK, &bars[2], sK + hh * kBlk * 128, hh * 64, hk, tk0 + k0, tb, pol);
+      tma_load_4d(&tmV, &bars[2], sV + hh * kBlk * 128, hh * 64, hk, tk0 + k0, tb, pol);
     }
     issue(0);
     if (n_it > 1) issue(1);
@@ -215,8 +253,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
   auto fetch_rowvec = [&](int it) -> float {
     const int h = hk * G + it / n_qb;
     const int q = (qb_lo + it % n_qb) * kBlk + (threadIdx.x & (kBlk - 1));
-    if (q >= p.Nq) return threadIdx.x < kBlk ? -INFINITY : 0.0f;
-    const size_t ri = (static_cast<size_t>(b) * p.H + h) * p.Nq + q;
+    if (q >= Nq) return threadIdx.x < kBlk ? -INFINITY : 0.0f;
+    const size_t ri = rowvec_index(p, b, h, qrow, q);
     return threadIdx.x < kBlk ? p.lse[ri] * kLog2e : p.dvec[ri];
   };
   float rv_next = n_it > 0 ? fetch_rowvec(0) : 0.0f;
@@ -244,7 +282,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
     const float* lse2 = sL + buf * 2 * kBlk;
     const float* dvec = lse2 + kBlk;
     // every (key, query) pair of this block pair visible?
-    bool full = k0 + kBlk <= p.Nk && q0 + kBlk <= p.Nq;
+    bool full = k0 + kBlk <= Nk && q0 + kBlk <= Nq;
     if (p.causal || p.window_right >= 0) {
       const int right = p.window_right >= 0 ? (p.causal ? min(0, p.window_right) : p.window_right) : 0;
       full = full && k0 + kBlk - 1 <= q0 + off + right;
@@ -308,7 +346,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
             if (alibi) logit2 -= slope2 * fabsf(static_cast<float>(pos - key));
             float pr = ex2(logit2 - lse2[ql]);
             if constexpr (kMasked) {
-              if (!(q0 + ql < p.Nq && key_visible(pos, key, p.Nk, p))) pr = 0.0f;
+              if (!(q0 + ql < Nq && key_visible(pos, key, Nk, p))) pr = 0.0f;
             }
             sc[jj][e] = pr;
             dp[jj][e] = pr * (dp[jj][e] - dvec[ql]) * dfac;
@@ -399,8 +437,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
       if (threadIdx.x == 0) {
 #pragma unroll
         for (int box = 0; box < D / 32; ++box)
-          tma_reduce_add_4d(&tmDQ, stage[box / kBoxesPerBuf] + (box % kBoxesPerBuf) * (kBlk * 128), box * 32, h, q0,
-                            b);
+          tma_reduce_add_4d(&tmDQ, stage[box / kBoxesPerBuf] + (box % kBoxesPerBuf) * (kBlk * 128), box * 32, h,
+                            tq0 + q0, tb);
         bulk_commit_group();
         bulk_wait_read_all();  // the staging buffers are reloaded next
       }
@@ -423,8 +461,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
 #pragma unroll
   for (int hr = 0; hr < 2; ++hr) {
     const int key = k0 + krow0 + 8 * hr;
-    if (key >= p.Nk) continue;
-    const size_t base = ((static_cast<size_t>(b) * p.Nk + key) * p.H_kv + hk) * D + 2 * tq;
+    if (key >= Nk) continue;
+    const size_t base = (static_cast<size_t>(krow + key) * p.H_kv + hk) * D + 2 * tq;
     T* dk_out = reinterpret_cast<T*>(p.dk) + base;
     T* dv_out = reinterpret_cast<T*>(p.dv) + base;
 #pragma unroll
@@ -476,11 +514,17 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2)
   const int b = blockIdx.y / p.H, h = blockIdx.y % p.H;
   const int hk = h / (p.H / p.H_kv);
   const int q0 = qb * kBlk;
-  const int off = p.Nk - p.Nq;
+  int Nq, Nk;
+  long long qrow, krow;
+  if (!bwd_seq(p, b, Nq, Nk, qrow, krow) || q0 >= Nq) return;  // uniform over the CTA
+  const int tb = p.cu_q == nullptr ? b : 0;
+  const int tq0 = p.cu_q == nullptr ? 0 : static_cast<int>(qrow);
+  const int tk0 = p.cu_q == nullptr ? 0 : static_cast<int>(krow);
+  const int off = Nk - Nq;
 
   // key blocks that hold a key visible to a query of [q0, qmax]
-  const int qmax = min(q0 + kBlk - 1, p.Nq - 1);
-  long long k_lo = 0, k_hi = p.Nk - 1;
+  const int qmax = min(q0 + kBlk - 1, Nq - 1);
+  long long k_lo = 0, k_hi = Nk - 1;
   if (p.causal || p.window_right >= 0) {
     const int right = p.window_right >= 0 ? (p.causal ? min(0, p.window_right) : p.window_right) : 0;
     k_hi = min(k_hi, static_cast<long long>(qmax) + off + right);
@@ -505,16 +549,18 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2)
     mbar_arrive_expect_tx(&bars[buf], 2 * C::kTile);
 #pragma unroll
     for (int hh = 0; hh < D / 64; ++hh) {
-      tma_load_4d(&tmK, &bars[buf], smem + C::kOffK + buf * C::kTile + hh * kBlk * 128, hh * 64, hk, k0, b, pol);
-      tma_load_4d(&tmV, &bars[buf], smem + C::kOffV + buf * C::kTile + hh * kBlk * 128, hh * 64, hk, k0, b, pol);
+      tma_load_4d(&tmK, &bars[buf], smem + C::kOffK + buf * C::kTile + hh * kBlk * 128, hh * 64, hk, tk0 + k0, tb,
+                  pol);
+      tma_load_4d(&tmV, &bars[buf], smem + C::kOffV + buf * C::kTile + hh * kBlk * 128, hh * 64, hk, tk0 + k0, tb,
+                  pol);
     }
   };
   if (threadIdx.x == 0 && n_it > 0) {
     mbar_arrive_expect_tx(&bars[2], 2 * C::kTile);
 #pragma unroll
     for (int hh = 0; hh < D / 64; ++hh) {
-      tma_load_4d(&tmQ, &bars[2], smem + C::kOffQ + hh * kBlk * 128, hh * 64, h, q0, b, pol);
-      tma_load_4d(&tmO, &bars[2], smem + C::kOffO + hh * kBlk * 128, hh * 64, h, q0, b, pol);
+      tma_load_4d(&tmQ, &bars[2], smem + C::kOffQ + hh * kBlk * 128, hh * 64, h, tq0 + q0, tb, pol);
+      tma_load_4d(&tmO, &bars[2], smem + C::kOffO + hh * kBlk * 128, hh * 64, h, tq0 + q0, tb, pol);
     }
     issue(0);
     if (n_it > 1) issue(1);
@@ -525,9 +571,9 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2)
 #pragma unroll
   for (int hr = 0; hr < 2; ++hr) {
     const int q = q0 + qrow0 + 8 * hr;
-    const size_t ri = (static_cast<size_t>(b) * p.H + h) * p.Nq + q;
-    lse2[hr] = q < p.Nq ? p.lse[ri] * kLog2e : -INFINITY;
-    dvr[hr] = q < p.Nq ? p.dvec[ri] : 0.0f;
+    const size_t ri = rowvec_index(p, b, h, qrow, q);
+    lse2[hr] = q < Nq ? p.lse[ri] * kLog2e : -INFINITY;
+    dvr[hr] = q < Nq ? p.dvec[ri] : 0.0f;
   }
   const bool alibi = p.slopes != nullptr;
   const float slope2 = alibi ? p.slopes[h] * kLog2e : 0.0f;
@@ -551,7 +597,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2)
     const uint8_t* sK = smem + C::kOffK + buf * C::kTile;
     const uint8_t* sV = smem + C::kOffV + buf * C::kTile;
     const uint32_t sK_a = smem_addr(sK);
-    bool full = k0 + kBlk <= p.Nk && q0 + kBlk <= p.Nq;
+    bool full = k0 + kBlk <= Nk && q0 + kBlk <= Nq;
     if (p.causal || p.window_right >= 0) {
       const int right = p.window_right >= 0 ? (p.causal ? min(0, p.window_right) : p.window_right) : 0;
       full = full && k0 + kBlk - 1 <= q0 + off + right;
@@ -615,7 +661,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2)
             if (alibi) logit2 -= slope2 * fabsf(static_cast<float>(pos - key));
             float pr = ex2(logit2 - lse2[hr]);
             if constexpr (kMasked) {
-              if (!(q0 + ql < p.Nq && key_visible(pos, key, p.Nk, p))) pr = 0.0f;
+              if (!(q0 + ql < Nq && key_visible(pos, key, Nk, p))) pr = 0.0f;
             }
             dp[jj][e] = pr * (dp[jj][e] - dvr[hr]) * dfac;
           }
@@ -656,8 +702,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2)
 #pragma unroll
   for (int hr = 0; hr < 2; ++hr) {
     const int q = q0 + qrow0 + 8 * hr;
-    if (q >= p.Nq) continue;
-    T* out = reinterpret_cast<T*>(p.dq) + ((static_cast<size_t>(b) * p.Nq + q) * p.H + h) * D + 2 * tq;
+    if (q >= Nq) continue;
+    T* out = reinterpret_cast<T*>(p.dq) + (static_cast<size_t>(qrow + q) * p.H + h) * D + 2 * tq;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       const float x0 = failed ? nan : dq[n][2 * hr] * p.scale, x1 = failed ? nan : dq[n][2 * hr + 1] * p.scale;
@@ -669,7 +715,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2)
 template <typename T, int D>
 cudaError_t launch(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                    const CUtensorMap& tmO, const CUtensorMap& tmDQ, cudaStream_t stream) {
-  const long long rows = static_cast<long long>(p.B) * p.Nq * p.H;
+  // query rows x heads of q, dO, dQ: B * Nq fixed, total_q packed
+  const long long rows = (p.cu_q == nullptr ? static_cast<long long>(p.B) * p.Nq : p.total_q) * p.H;
   const long long elems = rows * D;
   cudaError_t e = cudaSuccess;
   if (!p.deterministic) {
@@ -678,7 +725,12 @@ cudaError_t launch(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap
   }
   if (rows > 0) {
     const long long threads = rows * (D / 8);
-    bwd_rowdot_kernel<T, D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p);
+    BwdParams pr = p;  // the row-dot kernel sees the packed layout as one sequence of total_q rows
+    if (p.cu_q != nullptr) {
+      pr.B = 1;
+      pr.Nq = p.total_q;
+    }
+    bwd_rowdot_kernel<T, D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(pr);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -83,7 +83,10 @@ struct BwdParams {
   void* dk;           // [B, Nk, H_kv, d]
   void* dv;           // [B, Nk, H_kv, d]
   const float* slopes;  // [H] or nullptr
-  int B, H, H_kv, Nq, Nk;
+  const int* cu_q;      // [B + 1] row offsets (packed sequences) or nullptr (fixed length)
+  const int* cu_k;      // [B + 1] or nullptr
+  int total_q, total_k; // packed: rows of q and of k
+  int B, H, H_kv, Nq, Nk;  // packed: Nq, Nk bound the sequence lengths
   int causal, window_left, window_right;
   int use_softcap;
   int deterministic;  // 1: dQ summed in a fixed order (no atomics)

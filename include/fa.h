@@ -308,6 +308,30 @@ fa_status fa_bwd(const void *q, const void *k, const void *v, const void *out, c
                  size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * fa_bwd_varlen -- fa_bwd for packed sequences of different lengths, the
+ * backward of fa_fwd_varlen (with H_kv key/value heads, H % H_kv == 0):
+ *
+ *   q, out, dout, dq   [total_q, H, d]     sequence b owns rows cu_seqlens_q[b] ..
+ *   k, v, dk, dv       [total_k, H_kv, d]  sequence b owns rows cu_seqlens_k[b] ..
+ *   lse                [H, total_q]        fp32, the forward's (natural log)
+ *   cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k: as fa_fwd_varlen
+ *   workspace          fa_bwd_workspace_size(1, H, total_q, d) bytes
+ *   the remaining arguments as in fa_bwd
+ *
+ * Each sequence's gradients are those fa_bwd gives for it alone. The offsets
+ * are read on the device only: a sequence whose entries break the contract
+ * is skipped, its dk and dv rows left as they were; dq rows that belong to no
+ * valid sequence are written as zero. Limits: B * H <= 65535, total_q,
+ * total_k <= 2^28.
+ */
+fa_status fa_bwd_varlen(const void *q, const void *k, const void *v, const void *out, const float *lse,
+                        const void *dout, void *dq, void *dk, void *dv, const int *cu_seqlens_q,
+                        const int *cu_seqlens_k, int B, int H, int H_kv, int max_seqlen_q, int max_seqlen_k,
+                        int total_q, int total_k, int d, fa_dtype dtype, float scale, int causal,
+                        int window_left, int window_right, const float *alibi_slopes, float softcap,
+                        int deterministic, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Number of splits fa_fwd_kvcache uses for these sizes: num_splits itself
  * when it is 1..FA_MAX_SPLITS, else the automatic choice, which depends only
  * on B, H and the longest possible sequence max_blocks * page_size (host-side

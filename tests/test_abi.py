@@ -281,3 +281,25 @@ def test_bwd_validation(lib):
     assert lib.fa_bwd_workspace_size(2, 8, 100, 128) == (2 * 8 * 100 * 128 * 4 + 255) // 256 * 256 + \
         (2 * 8 * 100 * 4 + 255) // 256 * 256
     assert lib.fa_bwd_workspace_size(-1, 8, 100, 128) == 0
+
+
+def test_bwd_varlen_validation(lib):
+    def bv(**kw):
+        a = dict(q=P, k=P, v=P, out=P, lse=P, dout=P, dq=P, dk=P, dv=P, cq=P, ck=P, B=3, H=4, H_kv=2, mq=300,
+                 mk=300, tq=500, tk=600, d=128, dtype=1, scale=0.1, causal=1, wl=-1, wr=-1, slopes=None, cap=0.0,
+                 det=0, ws=P, ws_bytes=lib.fa_bwd_workspace_size(1, 4, 500, 128))
+        a.update(kw)
+        return lib.fa_bwd_varlen(a["q"], a["k"], a["v"], a["out"], a["lse"], a["dout"], a["dq"], a["dk"], a["dv"],
+                                 a["cq"], a["ck"], a["B"], a["H"], a["H_kv"], a["mq"], a["mk"], a["tq"], a["tk"],
+                                 a["d"], a["dtype"], a["scale"], a["causal"], a["wl"], a["wr"], a["slopes"],
+                                 a["cap"], a["det"], a["ws"], a["ws_bytes"], None)
+    assert bv() == DEVICE
+    assert bv(H_kv=3) == SHAPE
+    assert bv(B=20000) == SHAPE                  # B * H > 65535
+    assert bv(tq=-1) == SHAPE
+    assert bv(d=80) == HEADDIM
+    assert bv(cq=None) == NULL
+    assert bv(cq=P + 2) == ARG                   # int32 array not 4-byte aligned
+    assert bv(det=3) == ARG
+    assert bv(ws=None) == WORKSPACE
+    assert bv(tq=0, tk=0) == OK

@@ -125,3 +125,115 @@ def test_full_size_causal_bwd_on_sampled_heads():
         check(sl(dq), rq, w.dtype, "dq (%d, %d)" % (b, h))
         check(sl(dk), rk, w.dtype, "dk (%d, %d)" % (b, h))
         check(sl(dv), rv, w.dtype, "dv (%d, %d)" % (b, h))
+
+
+# ---------------------------------------------------------------- packed sequences
+
+def _packed(lens, H, d, dtype, g):
+    total = int(sum(lens))
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
+    return torch.randn(total, H, d, generator=g).to(dtype), cu
+
+
+def _varlen_reference(q, k, v, do, cu_q, cu_k, scale, **opts):
+    """Per-sequence oracle gradients, stitched back into the packed layout."""
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    for b in range(cu_q.numel() - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        if q1 == q0 or k1 == k0:
+            continue
+        sl = lambda t, a, z: t[a:z].unsqueeze(0)
+        rq, rk, rv = oracle.attn_bwd(sl(q, q0, q1), sl(k, k0, k1), sl(v, k0, k1), sl(do, q0, q1), scale, **opts)
+        dq[q0:q1], dk[k0:k1], dv[k0:k1] = rq[0], rk[0], rv[0]
+    return dq, dk, dv
+
+
+VARLEN = [
+    # (lens_q, lens_k, H, d, dtype, opts)
+    ((130, 1, 257, 0, 64), (130, 1, 257, 0, 64), 2, 128, torch.bfloat16, {"causal": True}),
+    ((50, 200), (120, 90), 2, 64, torch.float16, {"window_left": 30, "window_right": 10}),
+    ((70, 190), (70, 190), 2, 128, torch.bfloat16, {"causal": True, "softcap": 20.0}),
+]
+
+
+@pytest.mark.parametrize("det", [False, True], ids=["atomic_dq", "deterministic"])
+@pytest.mark.parametrize("case", VARLEN, ids=lambda c: "q%s_k%s" % ("-".join(map(str, c[0])), "-".join(map(str, c[1]))))
+def test_bwd_varlen_matches_per_sequence_oracle(case, det):
+    lens_q, lens_k, H, d, dtype, opts = case
+    g = torch.Generator().manual_seed(sum(lens_q) + 7)
+    q, cu_q = _packed(lens_q, H, d, dtype, g)
+    k, cu_k = _packed(lens_k, H, d, dtype, g)
+    v, _ = _packed(lens_k, H, d, dtype, g)
+    do, _ = _packed(lens_q, H, d, dtype, g)
+    scale = 1.0 / math.sqrt(d)
+    qd, kd, vd, dod, cqd, ckd = (t.cuda() for t in (q, k, v, do, cu_q, cu_k))
+    out = torch.empty_like(qd)
+    lse = torch.empty(H, q.shape[0], dtype=torch.float32, device="cuda")
+    fw = dict(causal=opts.get("causal", False), window_left=opts.get("window_left", -1),
+              window_right=opts.get("window_right", -1), softcap=opts.get("softcap", 0.0))
+    fa.fa_fwd_varlen(qd, kd, vd, out, lse, cqd, ckd, max(lens_q), max(lens_k), scale, **fw)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    fa.fa_bwd_varlen(qd, kd, vd, out, lse, dod, dq, dk, dv, cqd, ckd, max(lens_q), max(lens_k), scale,
+                     deterministic=det, **fw)
+    torch.cuda.synchronize()
+    rq, rk, rv = _varlen_reference(q, k, v, do, cu_q, cu_k, scale, **fw)
+    check(dq, rq, dtype, "dq")
+    check(dk, rk, dtype, "dk")
+    check(dv, rv, dtype, "dv")
+
+
+def test_bwd_varlen_grouped_heads_with_oracle_forward():
+    """Grouped-query packed sequences; O and LSE come from the oracle's
+    forward (rounded as a forward would return them)."""
+    lens, H, H_kv, d, dtype = (100, 190), 4, 2, 128, torch.bfloat16
+    g = torch.Generator().manual_seed(11)
+    q, cu = _packed(lens, H, d, dtype, g)
+    k, _ = _packed(lens, H_kv, d, dtype, g)
+    v, _ = _packed(lens, H_kv, d, dtype, g)
+    do, _ = _packed(lens, H, d, dtype, g)
+    slopes = W.alibi_slopes(H)
+    scale = 0.09
+    out = torch.empty_like(q)
+    lse = torch.empty(H, q.shape[0], dtype=torch.float32)
+    for b in range(len(lens)):
+        a, z = int(cu[b]), int(cu[b + 1])
+        o, l = oracle.attn_fwd_gqa(q[a:z].unsqueeze(0), k[a:z].unsqueeze(0), v[a:z].unsqueeze(0), scale, True,
+                                   alibi_slopes=slopes)
+        out[a:z] = torch.from_numpy(o[0]).to(dtype)
+        lse[:, a:z] = torch.from_numpy(l[0]).float()
+    qd, kd, vd, dod, od, ld, cud = (t.cuda() for t in (q, k, v, do, out, lse, cu))
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    fa.fa_bwd_varlen(qd, kd, vd, od, ld, dod, dq, dk, dv, cud, cud, max(lens), max(lens), scale, True,
+                     alibi_slopes=slopes.cuda())
+    torch.cuda.synchronize()
+    rq, rk, rv = _varlen_reference(q, k, v, do, cu, cu, scale, causal=True, alibi_slopes=slopes)
+    check(dq, rq, dtype, "dq")
+    check(dk, rk, dtype, "dk")
+    check(dv, rv, dtype, "dv")
+
+
+def test_bwd_varlen_skips_a_sequence_with_broken_offsets():
+    lens, H, d = (80, 120, 60), 2, 64
+    g = torch.Generator().manual_seed(12)
+    q, cu = _packed(lens, H, d, torch.float16, g)
+    k, _ = _packed(lens, H, d, torch.float16, g)
+    v, _ = _packed(lens, H, d, torch.float16, g)
+    do, _ = _packed(lens, H, d, torch.float16, g)
+    qd, kd, vd, dod, cud = (t.cuda() for t in (q, k, v, do, cu))
+    out = torch.empty_like(qd)
+    lse = torch.empty(H, q.shape[0], dtype=torch.float32, device="cuda")
+    fa.fa_fwd_varlen(qd, kd, vd, out, lse, cud, cud, max(lens), max(lens), 0.125, causal=True)
+    bad = cu.clone()
+    bad[2] = 500                      # sequence 1 ends past total, sequence 2 starts there
+    dq, dk, dv = torch.empty_like(qd), torch.full_like(kd, 7.0), torch.full_like(vd, 7.0)
+    fa.fa_bwd_varlen(qd, kd, vd, out, lse, dod, dq, dk, dv, bad.cuda(), bad.cuda(), max(lens), max(lens), 0.125,
+                     causal=True)
+    torch.cuda.synchronize()
+    rq, rk, rv = _varlen_reference(q, k, v, do, cu, cu, 0.125, causal=True)
+    a = int(cu[1])
+    check(dq[:a], rq[:a], torch.float16, "dq of the valid sequence")
+    check(dk[:a], rk[:a], torch.float16, "dk of the valid sequence")
+    assert torch.all(dk[a:] == 7.0) and torch.all(dv[a:] == 7.0)    # skipped: left as they were
+    assert torch.count_nonzero(dq[a:]) == 0                          # rows of no valid sequence
