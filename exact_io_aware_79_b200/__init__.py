@@ -435,3 +435,40 @@ def decode(q, k_cache, v_cache, block_table, cache_seqlens, scale: Optional[floa
     fa_fwd_kvcache(q, k_cache, v_cache, block_table, cache_seqlens, out, lse,
                    d ** -0.5 if scale is None else scale, window_left, alibi_slopes, softcap, num_splits, ws)
     return out, lse
+
+
+class _AttentionFn(torch.autograd.Function):
+    """fa_fwd_gqa forward, fa_bwd backward (argument marshalling only)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, scale, causal, window_left, window_right, alibi_slopes, softcap, deterministic):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        B, Nq, H, d = q.shape
+        out = torch.empty_like(q)
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+        fa_fwd_gqa(q, k, v, out, lse, scale, causal, window_left, window_right, alibi_slopes, softcap)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.opts = (scale, causal, window_left, window_right, alibi_slopes, softcap, deterministic)
+        return out, lse
+
+    @staticmethod
+    def backward(ctx, dout, dlse):
+        q, k, v, out, lse = ctx.saved_tensors
+        scale, causal, window_left, window_right, alibi_slopes, softcap, deterministic = ctx.opts
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        fa_bwd(q, k, v, out, lse, dout.contiguous(), dq, dk, dv, scale, causal, window_left, window_right,
+               alibi_slopes, softcap, deterministic)
+        return dq, dk, dv, None, None, None, None, None, None, None
+
+
+def attention_func(q, k, v, scale: Optional[float] = None, causal: bool = False, window_left: int = -1,
+                   window_right: int = -1, alibi_slopes=None, softcap: float = 0.0, deterministic: bool = False,
+                   return_lse: bool = False):
+    """Differentiable attention: q [B,Nq,H,d], k/v [B,Nk,H_kv,d] (H % H_kv == 0) on the device.
+    Forward through fa_fwd_gqa, backward through fa_bwd (gradients for q, k, v; the LSE output
+    carries no gradient). Returns out, or (out, lse) with return_lse."""
+    d = q.shape[-1]
+    out, lse = _AttentionFn.apply(q, k, v, d ** -0.5 if scale is None else float(scale), bool(causal),
+                                  int(window_left), int(window_right), alibi_slopes, float(softcap),
+                                  bool(deterministic))
+    return (out, lse) if return_lse else out

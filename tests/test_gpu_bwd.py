@@ -237,3 +237,17 @@ def test_bwd_varlen_skips_a_sequence_with_broken_offsets():
     check(dk[:a], rk[:a], torch.float16, "dk of the valid sequence")
     assert torch.all(dk[a:] == 7.0) and torch.all(dv[a:] == 7.0)    # skipped: left as they were
     assert torch.count_nonzero(dq[a:]) == 0                          # rows of no valid sequence
+
+
+def test_attention_func_autograd_gradients_match_the_oracle():
+    """loss = sum(out * dout) through attention_func; the gradients that
+    autograd hands back are fa_bwd's and must match the oracle's."""
+    B, H, H_kv, N, d, dtype = 1, 4, 2, 150, 64, torch.bfloat16
+    q, k, v, do = inputs(B, H, H_kv, N, N, d, dtype, seed=21)
+    qd, kd, vd = (t.cuda().requires_grad_(True) for t in (q, k, v))
+    out = fa.attention_func(qd, kd, vd, causal=True, window_left=40, softcap=15.0)
+    (out.float() * do.cuda().float()).sum().backward()
+    rq, rk, rv = oracle.attn_bwd(q, k, v, do, d ** -0.5, True, 40, -1, None, 15.0)
+    check(qd.grad, rq, dtype, "q.grad")
+    check(kd.grad, rk, dtype, "k.grad")
+    check(vd.grad, rv, dtype, "v.grad")
