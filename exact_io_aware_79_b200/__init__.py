@@ -87,6 +87,11 @@ def _lib_handle():
         L.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, i, i, i,
                                     vp, f, i, vp, sz, vp]
         L.fa_bwd_varlen.restype = i
+        L.fa_bwd_qkvpacked.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp, f, i, vp, sz, vp]
+        L.fa_bwd_qkvpacked.restype = i
+        L.fa_bwd_varlen_qkvpacked.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, f, i, vp,
+                                              sz, vp]
+        L.fa_bwd_varlen_qkvpacked.restype = i
         L.fa_status_string.argtypes = [i]
         L.fa_status_string.restype = ctypes.c_char_p
         _LIB = L
@@ -237,6 +242,57 @@ def fa_bwd_varlen(q, k, v, out, lse, dout, dq, dk, dv, cu_seqlens_q, cu_seqlens_
                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
                                        _stream(stream))
     _check(code, "fa_bwd_varlen")
+
+
+def fa_bwd_qkvpacked(qkv, out, lse, dout, dqkv, scale: float, causal: bool = False, window_left: int = -1,
+                     window_right: int = -1, alibi_slopes=None, softcap: float = 0.0, deterministic: bool = False,
+                     workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Backward of fa_fwd_qkvpacked: qkv, dqkv [B,N,3,H,d]; out, dout [B,N,H,d]; lse fp32 [B,H,N]."""
+    B, N, three, H, d = qkv.shape
+    for t in (qkv, out, lse, dout, dqkv):
+        if not t.is_contiguous():
+            raise ValueError("fa_bwd_qkvpacked needs contiguous tensors")
+    if three != 3 or tuple(dqkv.shape) != tuple(qkv.shape) or tuple(out.shape) != (B, N, H, d) or \
+            tuple(dout.shape) != (B, N, H, d) or len({qkv.dtype, out.dtype, dout.dtype, dqkv.dtype}) != 1:
+        raise ValueError("fa_bwd_qkvpacked: shape mismatch")
+    if tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32:
+        raise ValueError("fa_bwd_qkvpacked: lse must be fp32 [B, H, N]")
+    if workspace is None:
+        workspace = torch.empty(max(fa_bwd_workspace_size(B, H, N, d), 16), dtype=torch.uint8, device=qkv.device)
+    code = _lib_handle().fa_bwd_qkvpacked(_ptr(qkv), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dqkv), B, H, N, d,
+                                          _dtype_code(qkv), float(scale), int(bool(causal)), int(window_left),
+                                          int(window_right), _ptr(alibi_slopes), float(softcap),
+                                          int(bool(deterministic)), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(code, "fa_bwd_qkvpacked")
+
+
+def fa_bwd_varlen_qkvpacked(qkv, out, lse, dout, dqkv, cu_seqlens, max_seqlen: int, scale: float,
+                            causal: bool = False, window_left: int = -1, window_right: int = -1, alibi_slopes=None,
+                            softcap: float = 0.0, deterministic: bool = False,
+                            workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Backward of fa_fwd_varlen_qkvpacked: qkv, dqkv [total,3,H,d]; out, dout [total,H,d];
+    lse fp32 [H,total]; cu_seqlens int32 [B+1] on the device."""
+    total, three, H, d = qkv.shape
+    B = cu_seqlens.numel() - 1
+    for t in (qkv, out, lse, dout, dqkv, cu_seqlens):
+        if not t.is_contiguous():
+            raise ValueError("fa_bwd_varlen_qkvpacked needs contiguous tensors")
+    if three != 3 or tuple(dqkv.shape) != tuple(qkv.shape) or tuple(out.shape) != (total, H, d) or \
+            tuple(dout.shape) != (total, H, d) or len({qkv.dtype, out.dtype, dout.dtype, dqkv.dtype}) != 1:
+        raise ValueError("fa_bwd_varlen_qkvpacked: shape mismatch")
+    if tuple(lse.shape) != (H, total) or lse.dtype != torch.float32 or cu_seqlens.dtype != torch.int32:
+        raise ValueError("fa_bwd_varlen_qkvpacked: lse must be fp32 [H, total], cu_seqlens int32")
+    if workspace is None:
+        workspace = torch.empty(max(fa_bwd_workspace_size(1, H, total, d), 16), dtype=torch.uint8,
+                                device=qkv.device)
+    code = _lib_handle().fa_bwd_varlen_qkvpacked(_ptr(qkv), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dqkv),
+                                                 _ptr(cu_seqlens), B, H, int(max_seqlen), total, d,
+                                                 _dtype_code(qkv), float(scale), int(bool(causal)),
+                                                 int(window_left), int(window_right), _ptr(alibi_slopes),
+                                                 float(softcap), int(bool(deterministic)), _ptr(workspace),
+                                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(code, "fa_bwd_varlen_qkvpacked")
 
 
 def fa_fwd_qkvpacked(qkv, out, lse, scale: float, causal: bool = False, window_left: int = -1,

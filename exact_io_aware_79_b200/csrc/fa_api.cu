@@ -219,6 +219,99 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* out, flo
 
 namespace {
 
+// Backward for fixed-length (cu_q == nullptr) and packed sequences. tok: the
+// token stride, in elements, of q, k, v and of dq, dk, dv when they live in
+// one packed [.., 3, H, d] tensor (0 = contiguous); dout and out are always
+// contiguous.
+fa_status bwd_common(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, const int* cu_q, const int* cu_k, int B, int H,
+                     int H_kv, int Nq, int Nk, int total_q, int total_k, int d, fa_dtype dtype, float scale,
+                     int causal, int window_left, int window_right, const float* alibi_slopes, float softcap,
+                     int deterministic, void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                     bool packed_rows = false, long long tok = 0) {
+  // packed_rows: the rows are [total, H, d] (cu_q given, or B == 0 with the packed call)
+  if (B < 0 || H < 1 || Nq < 0 || Nk < 0 || total_q < 0 || total_k < 0) return FA_ERR_SHAPE;
+  if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_SHAPE;
+  if (Nq > kMaxSeq || Nk > kMaxSeq || total_q > kMaxSeq || total_k > kMaxSeq) return FA_ERR_SHAPE;
+  if (static_cast<long long>(B) * (packed_rows ? H : H_kv) > 65535) return FA_ERR_SHAPE;
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  if (!finite(scale) || !finite(softcap) || softcap < 0.0f) return FA_ERR_ARG;
+  if (window_left < -1 || window_right < -1 || (causal != 0 && causal != 1)) return FA_ERR_ARG;
+  if (deterministic != 0 && deterministic != 1) return FA_ERR_ARG;
+  // rows of q (and dq) and of k (and dk, dv)
+  const long long rows_q = packed_rows ? total_q : static_cast<long long>(B) * Nq;
+  const long long rows_k = packed_rows ? total_k : static_cast<long long>(B) * Nk;
+  if (rows_q == 0 && rows_k == 0) return FA_OK;
+  if (rows_k > 0 && (!k || !v || !dk || !dv)) return FA_ERR_NULL;
+  if (rows_q > 0 && (!q || !out || !lse || !dout || !dq)) return FA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_k) & 3u))
+    return FA_ERR_ARG;
+  const bool work = rows_q > 0 && rows_k > 0 && Nq > 0 && Nk > 0 && B > 0;
+  if (work) {
+    const size_t need = fa_bwd_workspace_size(1, H, static_cast<int>(rows_q), d);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  }
+  fa_status st = check_device();
+  if (st != FA_OK) return st;
+  const long long q_tok = tok > 0 ? tok : static_cast<long long>(H) * d;
+  const long long kv_tok = tok > 0 ? tok : static_cast<long long>(H_kv) * d;
+  if (!work) {
+    // no query or no key: the gradients that exist are zero
+    if (rows_k > 0 && (cudaMemset2DAsync(dk, kv_tok * 2, 0, static_cast<size_t>(H_kv) * d * 2, rows_k, stream) !=
+                           cudaSuccess ||
+                       cudaMemset2DAsync(dv, kv_tok * 2, 0, static_cast<size_t>(H_kv) * d * 2, rows_k, stream) !=
+                           cudaSuccess))
+      return FA_ERR_CUDA;
+    if (rows_q > 0 &&
+        cudaMemset2DAsync(dq, q_tok * 2, 0, static_cast<size_t>(H) * d * 2, rows_q, stream) != cudaSuccess)
+      return FA_ERR_CUDA;
+    return FA_OK;
+  }
+  const bool bf16 = dtype == FA_BF16;
+  const int mb = packed_rows ? 1 : B, nq = packed_rows ? total_q : Nq, nk = packed_rows ? total_k : Nk;
+  CUtensorMap tq, tk, tv, to, tdq;
+  if (!make_map(&tq, q, bf16, mb, nq, H, d, tok, 64) || !make_map(&to, dout, bf16, mb, nq, H, d, 0, 64) ||
+      !make_map(&tk, k, bf16, mb, nk, H_kv, d, tok, 64) || !make_map(&tv, v, bf16, mb, nk, H_kv, d, tok, 64) ||
+      !make_map_f32(&tdq, workspace, mb, nq, H, d))
+    return FA_ERR_CUDA;
+  fa::BwdParams p{};
+  const size_t rows = static_cast<size_t>(rows_q) * H;
+  p.out = out;
+  p.dout = dout;
+  p.lse = lse;
+  p.dq_acc = static_cast<float*>(workspace);
+  p.dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                    ((rows * d * sizeof(float) + 255) & ~size_t(255)));
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.dq_tok = q_tok;
+  p.dkv_tok = kv_tok;
+  p.slopes = alibi_slopes;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  p.B = B;
+  p.H = H;
+  p.H_kv = H_kv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.causal = causal;
+  p.window_left = window_left;
+  p.window_right = window_right;
+  p.use_softcap = softcap > 0.0f;
+  p.deterministic = deterministic;
+  p.scale = scale;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.cap_scale = softcap > 0.0f ? scale / softcap : 0.0f;
+  p.cap_log2 = softcap * fa::kLog2e;
+  return fa::launch_bwd(bf16, d, p, tq, tk, tv, to, tdq, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 fa_status kvcache_common(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
                          const int* cache_seqlens, void* out, float* lse, int B, int H, int H_kv, int d,
                          int num_pages, int page_size, int max_blocks, fa_dtype dtype, float scale,
@@ -431,67 +524,9 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, c
                  float scale, int causal, int window_left, int window_right, const float* alibi_slopes,
                  float softcap, int deterministic, void* workspace, size_t workspace_bytes,
                  cudaStream_t stream) {
-  if (B < 0 || H < 1 || Nq < 0 || Nk < 0) return FA_ERR_SHAPE;
-  if (deterministic != 0 && deterministic != 1) return FA_ERR_ARG;
-  if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_SHAPE;
-  if (Nq > kMaxSeq || Nk > kMaxSeq || static_cast<long long>(B) * H_kv > 65535) return FA_ERR_SHAPE;
-  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
-  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
-  if (!finite(scale) || !finite(softcap) || softcap < 0.0f) return FA_ERR_ARG;
-  if (window_left < -1 || window_right < -1 || (causal != 0 && causal != 1)) return FA_ERR_ARG;
-  if (B == 0 || (Nq == 0 && Nk == 0)) return FA_OK;
-  const size_t kv_bytes = static_cast<size_t>(B) * Nk * H_kv * d * 2;
-  const size_t q_bytes = static_cast<size_t>(B) * Nq * H * d * 2;
-  if (Nk > 0 && (!k || !v || !dk || !dv)) return FA_ERR_NULL;
-  if (Nq > 0 && (!q || !out || !lse || !dout || !dq)) return FA_ERR_NULL;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
-      !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
-    return FA_ERR_ARG;
-  if (Nq > 0 && Nk > 0) {
-    const size_t need = fa_bwd_workspace_size(B, H, Nq, d);
-    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return FA_ERR_WORKSPACE;
-  }
-  fa_status st = check_device();
-  if (st != FA_OK) return st;
-  // with no queries there is no gradient for K and V; with no keys none for Q
-  if (Nq == 0)
-    return (cudaMemsetAsync(dk, 0, kv_bytes, stream) == cudaSuccess &&
-            cudaMemsetAsync(dv, 0, kv_bytes, stream) == cudaSuccess) ? FA_OK : FA_ERR_CUDA;
-  if (Nk == 0) return cudaMemsetAsync(dq, 0, q_bytes, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-
-  const bool bf16 = dtype == FA_BF16;
-  CUtensorMap tq, tk, tv, to, tdq;
-  if (!make_map(&tq, q, bf16, B, Nq, H, d, 0, 64) || !make_map(&to, dout, bf16, B, Nq, H, d, 0, 64) ||
-      !make_map(&tk, k, bf16, B, Nk, H_kv, d, 0, 64) || !make_map(&tv, v, bf16, B, Nk, H_kv, d, 0, 64) ||
-      !make_map_f32(&tdq, workspace, B, Nq, H, d))
-    return FA_ERR_CUDA;
-  fa::BwdParams p{};
-  const size_t rows = static_cast<size_t>(B) * H * Nq;
-  p.out = out;
-  p.dout = dout;
-  p.lse = lse;
-  p.dq_acc = static_cast<float*>(workspace);
-  p.dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                    ((rows * d * sizeof(float) + 255) & ~size_t(255)));
-  p.dq = dq;
-  p.dk = dk;
-  p.dv = dv;
-  p.slopes = alibi_slopes;
-  p.B = B;
-  p.H = H;
-  p.H_kv = H_kv;
-  p.Nq = Nq;
-  p.Nk = Nk;
-  p.causal = causal;
-  p.window_left = window_left;
-  p.window_right = window_right;
-  p.use_softcap = softcap > 0.0f;
-  p.deterministic = deterministic;
-  p.scale = scale;
-  p.scale_log2 = scale * fa::kLog2e;
-  p.cap_scale = softcap > 0.0f ? scale / softcap : 0.0f;
-  p.cap_log2 = softcap * fa::kLog2e;
-  return fa::launch_bwd(bf16, d, p, tq, tk, tv, to, tdq, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return bwd_common(q, k, v, out, lse, dout, dq, dk, dv, nullptr, nullptr, B, H, H_kv, Nq, Nk, 0, 0, d, dtype, scale,
+                    causal, window_left, window_right, alibi_slopes, softcap, deterministic, workspace,
+                    workspace_bytes, stream);
 }
 
 fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* out, const float* lse,
@@ -500,78 +535,42 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
                         int total_q, int total_k, int d, fa_dtype dtype, float scale, int causal, int window_left,
                         int window_right, const float* alibi_slopes, float softcap, int deterministic,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  if (B < 0 || H < 1 || max_seqlen_q < 0 || max_seqlen_k < 0 || total_q < 0 || total_k < 0) return FA_ERR_SHAPE;
-  if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_SHAPE;
-  if (max_seqlen_q > kMaxSeq || max_seqlen_k > kMaxSeq || total_q > kMaxSeq || total_k > kMaxSeq ||
-      static_cast<long long>(B) * H > 65535)
-    return FA_ERR_SHAPE;
-  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
-  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
-  if (!finite(scale) || !finite(softcap) || softcap < 0.0f) return FA_ERR_ARG;
-  if (window_left < -1 || window_right < -1 || (causal != 0 && causal != 1)) return FA_ERR_ARG;
-  if (deterministic != 0 && deterministic != 1) return FA_ERR_ARG;
-  if (total_q == 0 && total_k == 0) return FA_OK;
   if (B > 0 && (!cu_seqlens_q || !cu_seqlens_k)) return FA_ERR_NULL;
-  if (total_k > 0 && (!k || !v || !dk || !dv)) return FA_ERR_NULL;
-  if (total_q > 0 && (!q || !out || !lse || !dout || !dq)) return FA_ERR_NULL;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
-      !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
-      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
-    return FA_ERR_ARG;
-  const bool work = B > 0 && total_q > 0 && total_k > 0 && max_seqlen_q > 0 && max_seqlen_k > 0;
-  if (work) {
-    const size_t need = fa_bwd_workspace_size(1, H, total_q, d);
-    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return FA_ERR_WORKSPACE;
-  }
-  fa_status st = check_device();
-  if (st != FA_OK) return st;
-  const size_t kv_bytes = static_cast<size_t>(total_k) * H_kv * d * 2;
-  const size_t q_bytes = static_cast<size_t>(total_q) * H * d * 2;
-  if (!work) {
-    // no query or no key anywhere: the gradients that exist are zero
-    if (total_k > 0 && (cudaMemsetAsync(dk, 0, kv_bytes, stream) != cudaSuccess ||
-                        cudaMemsetAsync(dv, 0, kv_bytes, stream) != cudaSuccess))
-      return FA_ERR_CUDA;
-    if (total_q > 0 && cudaMemsetAsync(dq, 0, q_bytes, stream) != cudaSuccess) return FA_ERR_CUDA;
-    return FA_OK;
-  }
-  const bool bf16 = dtype == FA_BF16;
-  CUtensorMap tq, tk, tv, to, tdq;
-  if (!make_map(&tq, q, bf16, 1, total_q, H, d, 0, 64) || !make_map(&to, dout, bf16, 1, total_q, H, d, 0, 64) ||
-      !make_map(&tk, k, bf16, 1, total_k, H_kv, d, 0, 64) || !make_map(&tv, v, bf16, 1, total_k, H_kv, d, 0, 64) ||
-      !make_map_f32(&tdq, workspace, 1, total_q, H, d))
-    return FA_ERR_CUDA;
-  fa::BwdParams p{};
-  const size_t rows = static_cast<size_t>(total_q) * H;
-  p.out = out;
-  p.dout = dout;
-  p.lse = lse;
-  p.dq_acc = static_cast<float*>(workspace);
-  p.dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                    ((rows * d * sizeof(float) + 255) & ~size_t(255)));
-  p.dq = dq;
-  p.dk = dk;
-  p.dv = dv;
-  p.slopes = alibi_slopes;
-  p.cu_q = cu_seqlens_q;
-  p.cu_k = cu_seqlens_k;
-  p.total_q = total_q;
-  p.total_k = total_k;
-  p.B = B;
-  p.H = H;
-  p.H_kv = H_kv;
-  p.Nq = max_seqlen_q;
-  p.Nk = max_seqlen_k;
-  p.causal = causal;
-  p.window_left = window_left;
-  p.window_right = window_right;
-  p.use_softcap = softcap > 0.0f;
-  p.deterministic = deterministic;
-  p.scale = scale;
-  p.scale_log2 = scale * fa::kLog2e;
-  p.cap_scale = softcap > 0.0f ? scale / softcap : 0.0f;
-  p.cap_log2 = softcap * fa::kLog2e;
-  return fa::launch_bwd(bf16, d, p, tq, tk, tv, to, tdq, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  if (B < 0) return FA_ERR_SHAPE;
+  return bwd_common(q, k, v, out, lse, dout, dq, dk, dv, B > 0 ? cu_seqlens_q : nullptr,
+                    B > 0 ? cu_seqlens_k : nullptr, B, H, H_kv, max_seqlen_q, max_seqlen_k, total_q, total_k, d,
+                    dtype, scale, causal, window_left, window_right, alibi_slopes, softcap, deterministic, workspace,
+                    workspace_bytes, stream, true);
+}
+
+fa_status fa_bwd_qkvpacked(const void* qkv, const void* out, const float* lse, const void* dout, void* dqkv, int B,
+                           int H, int N, int d, fa_dtype dtype, float scale, int causal, int window_left,
+                           int window_right, const float* alibi_slopes, float softcap, int deterministic,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const long long hd = static_cast<long long>(H) * d;
+  const char* in = static_cast<const char*>(qkv);
+  char* o = static_cast<char*>(dqkv);
+  return bwd_common(qkv, in ? in + hd * 2 : nullptr, in ? in + 2 * hd * 2 : nullptr, out, lse, dout, dqkv,
+                    o ? o + hd * 2 : nullptr, o ? o + 2 * hd * 2 : nullptr, nullptr, nullptr, B, H, H, N, N, 0, 0, d,
+                    dtype, scale, causal, window_left, window_right, alibi_slopes, softcap, deterministic, workspace,
+                    workspace_bytes, stream, false, 3 * hd);
+}
+
+fa_status fa_bwd_varlen_qkvpacked(const void* qkv, const void* out, const float* lse, const void* dout, void* dqkv,
+                                  const int* cu_seqlens, int B, int H, int max_seqlen, int total, int d,
+                                  fa_dtype dtype, float scale, int causal, int window_left, int window_right,
+                                  const float* alibi_slopes, float softcap, int deterministic, void* workspace,
+                                  size_t workspace_bytes, cudaStream_t stream) {
+  if (B > 0 && !cu_seqlens) return FA_ERR_NULL;
+  if (B < 0) return FA_ERR_SHAPE;
+  const long long hd = static_cast<long long>(H) * d;
+  const char* in = static_cast<const char*>(qkv);
+  char* o = static_cast<char*>(dqkv);
+  return bwd_common(qkv, in ? in + hd * 2 : nullptr, in ? in + 2 * hd * 2 : nullptr, out, lse, dout, dqkv,
+                    o ? o + hd * 2 : nullptr, o ? o + 2 * hd * 2 : nullptr, B > 0 ? cu_seqlens : nullptr,
+                    B > 0 ? cu_seqlens : nullptr, B, H, H, max_seqlen, max_seqlen, total, total, d, dtype, scale,
+                    causal, window_left, window_right, alibi_slopes, softcap, deterministic, workspace,
+                    workspace_bytes, stream, true, 3 * hd);
 }
 
 }  // extern "C"

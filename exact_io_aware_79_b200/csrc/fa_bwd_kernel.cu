@@ -102,15 +102,17 @@ __global__ void __launch_bounds__(256) bwd_rowdot_kernel(const BwdParams p) {
 }
 
 // dQ = scale * accumulator, cast to the input type; 4 elements per thread.
+// The accumulator is [tokens, H, d]; dq rows are dq_tok elements apart.
 template <typename T>
-__global__ void __launch_bounds__(256) bwd_dq_cast_kernel(const BwdParams p, long long n4) {
+__global__ void __launch_bounds__(256) bwd_dq_cast_kernel(const BwdParams p, long long n4, int hd) {
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n4) return;
   const float4 a = reinterpret_cast<const float4*>(p.dq_acc)[i];
   uint2 w;
   w.x = pack2<T>(a.x * p.scale, a.y * p.scale);
   w.y = pack2<T>(a.z * p.scale, a.w * p.scale);
-  reinterpret_cast<uint2*>(p.dq)[i] = w;
+  const long long e = 4 * i, token = e / hd;
+  *reinterpret_cast<uint2*>(reinterpret_cast<T*>(p.dq) + token * p.dq_tok + (e - token * hd)) = w;
 }
 
 // Is key j visible to the query at key position pos (the forward's rule)?
@@ -462,7 +464,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
   for (int hr = 0; hr < 2; ++hr) {
     const int key = k0 + krow0 + 8 * hr;
     if (key >= Nk) continue;
-    const size_t base = (static_cast<size_t>(krow + key) * p.H_kv + hk) * D + 2 * tq;
+    const size_t base = static_cast<size_t>(krow + key) * p.dkv_tok + static_cast<size_t>(hk) * D + 2 * tq;
     T* dk_out = reinterpret_cast<T*>(p.dk) + base;
     T* dv_out = reinterpret_cast<T*>(p.dv) + base;
 #pragma unroll
@@ -703,7 +705,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2)
   for (int hr = 0; hr < 2; ++hr) {
     const int q = q0 + qrow0 + 8 * hr;
     if (q >= Nq) continue;
-    T* out = reinterpret_cast<T*>(p.dq) + (static_cast<size_t>(qrow + q) * p.H + h) * D + 2 * tq;
+    T* out = reinterpret_cast<T*>(p.dq) + static_cast<size_t>(qrow + q) * p.dq_tok + static_cast<size_t>(h) * D +
+             2 * tq;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       const float x0 = failed ? nan : dq[n][2 * hr] * p.scale, x1 = failed ? nan : dq[n][2 * hr + 1] * p.scale;
@@ -752,7 +755,8 @@ cudaError_t launch(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap
     return cudaGetLastError();
   }
   const long long n4 = elems / 4;
-  if (n4 > 0) bwd_dq_cast_kernel<T><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(p, n4);
+  if (n4 > 0)
+    bwd_dq_cast_kernel<T><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(p, n4, p.H * D);
   return cudaGetLastError();
 }
 

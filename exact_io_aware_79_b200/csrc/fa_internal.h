@@ -86,6 +86,8 @@ struct BwdParams {
   const int* cu_q;      // [B + 1] row offsets (packed sequences) or nullptr (fixed length)
   const int* cu_k;      // [B + 1] or nullptr
   int total_q, total_k; // packed: rows of q and of k
+  long long dq_tok;     // elements from one token's dq row to the next (H * d, or 3 * H * d in a packed dqkv)
+  long long dkv_tok;    // the same for dk, dv (H_kv * d, or 3 * H * d)
   int B, H, H_kv, Nq, Nk;  // packed: Nq, Nk bound the sequence lengths
   int causal, window_left, window_right;
   int use_softcap;

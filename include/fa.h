@@ -332,6 +332,30 @@ fa_status fa_bwd_varlen(const void *q, const void *k, const void *v, const void 
                         int deterministic, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * fa_bwd_qkvpacked, fa_bwd_varlen_qkvpacked -- the backward of
+ * fa_fwd_qkvpacked / fa_fwd_varlen_qkvpacked: gradients of q, k and v written
+ * into one packed tensor laid out like qkv.
+ *
+ *   qkv               [B, N, 3, H, d] (fixed) or [total, 3, H, d] (packed)
+ *   out, dout         [B, N, H, d] or [total, H, d], contiguous
+ *   lse               [B, H, N] or [H, total], the forward's
+ *   dqkv              like qkv, written: slot 0 dq, 1 dk, 2 dv
+ *   cu_seqlens        [B + 1] device offsets (varlen form; q and k alike)
+ *   workspace         fa_bwd_workspace_size(B, H, N, d), or (1, H, total, d)
+ * Everything else as fa_bwd / fa_bwd_varlen (H_kv = H).
+ */
+fa_status fa_bwd_qkvpacked(const void *qkv, const void *out, const float *lse, const void *dout, void *dqkv,
+                           int B, int H, int N, int d, fa_dtype dtype, float scale, int causal,
+                           int window_left, int window_right, const float *alibi_slopes, float softcap,
+                           int deterministic, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+fa_status fa_bwd_varlen_qkvpacked(const void *qkv, const void *out, const float *lse, const void *dout,
+                                  void *dqkv, const int *cu_seqlens, int B, int H, int max_seqlen, int total,
+                                  int d, fa_dtype dtype, float scale, int causal, int window_left,
+                                  int window_right, const float *alibi_slopes, float softcap, int deterministic,
+                                  void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Number of splits fa_fwd_kvcache uses for these sizes: num_splits itself
  * when it is 1..FA_MAX_SPLITS, else the automatic choice, which depends only
  * on B, H and the longest possible sequence max_blocks * page_size (host-side

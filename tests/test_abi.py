@@ -303,3 +303,20 @@ def test_bwd_varlen_validation(lib):
     assert bv(det=3) == ARG
     assert bv(ws=None) == WORKSPACE
     assert bv(tq=0, tk=0) == OK
+
+
+def test_bwd_qkvpacked_validation(lib):
+    ws = lib.fa_bwd_workspace_size(2, 4, 100, 128)
+    f = lambda **kw: lib.fa_bwd_qkvpacked(kw.get("qkv", P), P, P, P, kw.get("dqkv", P), 2, 4, 100,
+                                          kw.get("d", 128), 1, 0.1, 1, -1, -1, None, 0.0, kw.get("det", 0),
+                                          kw.get("ws", P), ws, None)
+    assert f() == DEVICE
+    assert f(d=48) == HEADDIM
+    assert f(dqkv=None) == NULL
+    assert f(det=5) == ARG
+    assert f(ws=None) == WORKSPACE
+    g = lambda **kw: lib.fa_bwd_varlen_qkvpacked(P, P, P, P, P, kw.get("cu", P), 3, 4, 100, 250, 128, 1, 0.1, 1,
+                                                 -1, -1, None, 0.0, 0, P, lib.fa_bwd_workspace_size(1, 4, 250, 128),
+                                                 None)
+    assert g() == DEVICE
+    assert g(cu=None) == NULL

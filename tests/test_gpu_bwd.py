@@ -251,3 +251,43 @@ def test_attention_func_autograd_gradients_match_the_oracle():
     check(qd.grad, rq, dtype, "q.grad")
     check(kd.grad, rk, dtype, "k.grad")
     check(vd.grad, rv, dtype, "v.grad")
+
+
+# ---------------------------------------------------------------- packed QKV
+
+@pytest.mark.parametrize("det", [False, True], ids=["atomic_dq", "deterministic"])
+def test_bwd_qkvpacked_matches_oracle(det):
+    B, N, H, d, dtype = 2, 190, 2, 128, torch.bfloat16
+    g = torch.Generator().manual_seed(31)
+    qkv = torch.randn(B, N, 3, H, d, generator=g).to(dtype)
+    do = torch.randn(B, N, H, d, generator=g).to(dtype)
+    qkvd, dod = qkv.cuda(), do.cuda()
+    out = torch.empty(B, N, H, d, dtype=dtype, device="cuda")
+    lse = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+    fa.fa_fwd_qkvpacked(qkvd, out, lse, 0.1, True, 60, -1)
+    dqkv = torch.full_like(qkvd, 3.0)
+    fa.fa_bwd_qkvpacked(qkvd, out, lse, dod, dqkv, 0.1, True, 60, -1, deterministic=det)
+    torch.cuda.synchronize()
+    refs = oracle.attn_bwd(qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2], do, 0.1, True, 60, -1)
+    for slot, (ref, name) in enumerate(zip(refs, ("dq", "dk", "dv"))):
+        check(dqkv[:, :, slot], ref, dtype, name)
+
+
+def test_bwd_varlen_qkvpacked_matches_per_sequence_oracle():
+    lens, H, d, dtype = (120, 1, 200), 2, 64, torch.float16
+    total = sum(lens)
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
+    g = torch.Generator().manual_seed(32)
+    qkv = torch.randn(total, 3, H, d, generator=g).to(dtype)
+    do = torch.randn(total, H, d, generator=g).to(dtype)
+    qkvd, dod, cud = qkv.cuda(), do.cuda(), cu.cuda()
+    out = torch.empty(total, H, d, dtype=dtype, device="cuda")
+    lse = torch.empty(H, total, dtype=torch.float32, device="cuda")
+    fa.fa_fwd_varlen_qkvpacked(qkvd, out, lse, cud, max(lens), 0.125, causal=True)
+    dqkv = torch.empty_like(qkvd)
+    fa.fa_bwd_varlen_qkvpacked(qkvd, out, lse, dod, dqkv, cud, max(lens), 0.125, causal=True)
+    torch.cuda.synchronize()
+    rq, rk, rv = _varlen_reference(qkv[:, 0], qkv[:, 1], qkv[:, 2], do, cu, cu, 0.125, causal=True)
+    check(dqkv[:, 0], rq, dtype, "dq")
+    check(dqkv[:, 1], rk, dtype, "dk")
+    check(dqkv[:, 2], rv, dtype, "dv")
