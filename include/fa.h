@@ -296,7 +296,8 @@ fa_status fa_kvcache_append(const void *k_new, const void *v_new, void *k_cache,
  * buffer; the call only enqueues work on `stream`.
  *
  * Errors: as fa_fwd_gqa, plus FA_ERR_WORKSPACE when the workspace is missing,
- * misaligned or too small, and FA_ERR_SHAPE when B * H_kv > 65535.
+ * misaligned or too small, and FA_ERR_SHAPE when B * H_kv > 65535 (B * H
+ * with deterministic = 1).
  * Nq == 0 gives zero dk, dv; Nk == 0 gives zero dq; B == 0 is a no-op.
  */
 size_t fa_bwd_workspace_size(int B, int H, int Nq, int d);

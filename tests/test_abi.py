@@ -264,6 +264,9 @@ def test_bwd_validation(lib):
     assert bw(H_kv=3) == SHAPE
     assert bw(H_kv=16) == SHAPE
     assert bw(B=40000, H_kv=2) == SHAPE          # B * H_kv > 65535
+    big = lib.fa_bwd_workspace_size(8192, 8, 100, 128)
+    assert bw(B=8192, H_kv=2, ws_bytes=big) == DEVICE          # B * H_kv = 16384
+    assert bw(B=8192, H_kv=2, det=1, ws_bytes=big) == SHAPE    # the deterministic dQ grid has B * H = 65536 rows
     assert bw(d=96) == HEADDIM
     assert bw(dtype=7) == DTYPE
     assert bw(scale=float("nan")) == ARG
