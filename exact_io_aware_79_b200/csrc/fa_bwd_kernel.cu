@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
   const bool dq_on = !p.deterministic;
   bool failed = false;
   int issued = n_it > 1 ? 2 : n_it;
+  bool reload_pending = false;  // thread 0: a dQ reduce still reads this block's Q/dO buffers
 
   // the row vectors (lse, D) of iteration `it`: thread x < 64 fetches lse of
   // query q0 + x, thread 64 + x its D; read one iteration ahead into a register
@@ -277,6 +278,16 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
     if (__syncthreads_or(!ok)) {
       failed = true;
       break;
+    }
+    if (threadIdx.x == 0 && reload_pending) {
+      // the previous block's dQ boxes have been read out of its Q/dO buffers
+      // by now (a block of compute ago at most): reload them
+      bulk_wait_read_all();
+      if (issued < n_it) {
+        issue(issued);
+        ++issued;
+      }
+      reload_pending = false;
     }
     const uint8_t* sQ = smem + C::kOffQ + buf * C::kTile;
     const uint8_t* sO = smem + C::kOffO + buf * C::kTile;
@@ -442,10 +453,9 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
           tma_reduce_add_4d(&tmDQ, stage[box / kBoxesPerBuf] + (box % kBoxesPerBuf) * (kBlk * 128), box * 32, h,
                             tq0 + q0, tb);
         bulk_commit_group();
-        bulk_wait_read_all();  // the staging buffers are reloaded next
+        reload_pending = true;  // the staging buffers are reloaded after the next barrier
       }
-    }
-    if (threadIdx.x == 0 && issued < n_it) {
+    } else if (threadIdx.x == 0 && issued < n_it) {
       issue(issued);
       ++issued;
     }
