@@ -103,3 +103,70 @@ def test_mutant_is_caught(source, name):
             caught = run_battery()
     oracle.load_library()
     assert caught > 0, "mutant %s passed every pin" % name
+
+
+# ---------------------------------------------------------------- backward
+
+BWD_MUTANTS = {
+    "softmax_jacobian_dropped": ("dz = p * (dp - np.sum(p * dp, axis=1, keepdims=True))", "dz = p * dp"),
+    "softcap_factor_dropped": ("dz = dz * (1.0 - t * t)", "dz = dz"),
+    "dk_from_dout": ("dk[b, :, h] = scale * (dz.T @ qh)", "dk[b, :, h] = scale * (dz.T @ doh)"),
+    "dq_missing_scale": ("dq[b, :, h] = scale * (dz @ kh)", "dq[b, :, h] = dz @ kh"),
+    "dp_with_k": ("dp = doh @ vh.T", "dp = doh @ kh.T"),
+    "dv_not_transposed": ("dv[b, :, h] = p.T @ doh", "dv[b, :, h] = (p @ doh.T[:, : p.shape[1]].T)"),
+    "group_sum_wrong_order": ("dk = dk.reshape(B, Nk, H_kv, G, d).sum(axis=3)",
+                              "dk = dk.reshape(B, Nk, G, H_kv, d).sum(axis=2)"),
+}
+
+
+def _grouped_finite_difference_check():
+    """Finite differences with four query heads over two K/V heads (groups
+    of two), so a group sum over the wrong heads shows."""
+    B, H, H_kv, Nq, Nk, d, scale = 1, 4, 2, 4, 5, 3, 0.6
+    q, k, v = pins.rnd((B, Nq, H, d), 101), pins.rnd((B, Nk, H_kv, d), 102), pins.rnd((B, Nk, H_kv, d), 103)
+    dout = pins.rnd((B, Nq, H, d), 104)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, dout, scale, causal=True)
+    f = lambda: pins._loss(q, k, v, dout, scale, causal=True)
+    for got, x in ((dq, q), (dk, k), (dv, v)):
+        assert np.abs(got - pins._finite_difference(x, f)).max() < 1e-7
+
+
+def bwd_battery():
+    for opts in ({}, {"causal": True, "window_left": 2, "window_right": 0},
+                 {"causal": True, "alibi_slopes": [0.5, 0.125], "softcap": 1.5}):
+        for H_kv in (2, 1):
+            yield lambda opts=opts, H_kv=H_kv: pins.test_bwd_matches_finite_differences_of_the_forward(opts, H_kv)
+    yield pins.test_bwd_single_key_closed_form
+    yield pins.test_bwd_zero_query_closed_form
+    yield pins.test_bwd_rows_without_keys_carry_no_gradient
+    yield _grouped_finite_difference_check
+
+
+def _bwd_mutant(snippet, replacement):
+    import inspect
+    src = inspect.getsource(oracle.attn_bwd)
+    assert src.count(snippet) == 1, snippet
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(snippet, replacement), "<mutant>", "exec"), ns)
+    return ns["attn_bwd"]
+
+
+def _bwd_failures(fn, monkeypatch):
+    monkeypatch.setattr(oracle, "attn_bwd", fn)
+    failed = 0
+    for check in bwd_battery():
+        try:
+            check()
+        except Exception:
+            failed += 1
+    return failed
+
+
+def test_unmodified_backward_oracle_passes_the_battery(monkeypatch):
+    assert _bwd_failures(oracle.attn_bwd, monkeypatch) == 0
+
+
+@pytest.mark.parametrize("name", sorted(BWD_MUTANTS))
+def test_each_backward_mutant_fails_a_pin(name, monkeypatch):
+    snippet, replacement = BWD_MUTANTS[name]
+    assert _bwd_failures(_bwd_mutant(snippet, replacement), monkeypatch) > 0, name
