@@ -323,3 +323,24 @@ def test_bwd_qkvpacked_validation(lib):
                                                  None)
     assert g() == DEVICE
     assert g(cu=None) == NULL
+
+
+def test_header_is_plain_c_and_every_entry_links(lib, tmp_path):
+    """The boundary needs no C++ and no torch: a C99 program that takes the
+    address of every function the header declares compiles with -Werror and
+    links against the library."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    names = declared_functions()
+    src = tmp_path / "abi_user.c"
+    src.write_text('#include "fa.h"\n#include <stdio.h>\nint main(void) {\n  void (*fns[])(void) = {\n' +
+                   ",\n".join("    (void (*)(void))%s" % n for n in names) +
+                   '\n  };\n  printf("%d\\n", (int)(sizeof(fns) / sizeof(fns[0])));\n  return 0;\n}\n')
+    libdir = os.path.dirname(lib._name)
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    out = tmp_path / "abi_user"
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc,
+                        str(src), "-L", libdir, "-lfa_b200", "-o", str(out)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
