@@ -187,6 +187,27 @@ def make_fwd_inputs(w: FwdWorkload, device="cpu", seed: Optional[int] = None):
     return out
 
 
+def make_fwd_inputs_fp8(w: FwdWorkload, fmt: torch.dtype = torch.float8_e4m3fn, device="cpu",
+                        seed: Optional[int] = None):
+    """8-bit inputs for a forward workload: the fp32 draws of make_fwd_inputs
+    (same seed, before rounding to w.dtype), each tensor scaled so that its
+    largest magnitude maps to the format's largest finite value, then rounded
+    to `fmt`. Returns dict(q, k, v, descale_q, descale_k, descale_v, slopes):
+    element x8 stands for x8 * descale_x."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(w.seed if seed is None else seed)
+    top = torch.finfo(fmt).max
+    out = {}
+    for name, n in (("q", w.Nq), ("k", w.Nk), ("v", w.Nk)):
+        x = torch.randn((w.B, n, w.H, w.d), generator=gen, dtype=torch.float32) * w.sigma
+        descale = float(x.abs().max()) / top if x.numel() else 1.0
+        out[name] = (x / descale).to(fmt).to(device)
+        out["descale_" + name] = descale
+    slopes = alibi_slopes(w.H) if w.alibi else None
+    out["slopes"] = None if slopes is None else slopes.to(device)
+    return out
+
+
 def make_varlen_inputs(w: VarlenWorkload, device="cpu", seed: Optional[int] = None):
     """Returns dict(q, k, v, cu_q, cu_k, max_q, max_k, lens).
 

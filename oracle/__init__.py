@@ -5,8 +5,9 @@ may import this package. It loads ``liboracle.so`` (built from
 ``attn_oracle.c``; see that file's header for the definition it follows and
 the readings of the pages it takes) and shares no code with the CUDA path.
 
-Inputs may be torch CPU tensors (fp16, bf16 or fp64) or numpy arrays
-(float16 / float64, or uint16 bit patterns with an explicit ``dtype``).
+Inputs may be torch CPU tensors (fp16, bf16, float8_e4m3fn, float8_e5m2 or
+fp64) or numpy arrays (float16 / float64, or uint16 / uint8 bit patterns
+with an explicit ``dtype``).
 Everything is returned as float64 numpy arrays.
 """
 from __future__ import annotations
@@ -19,7 +20,7 @@ import numpy as np
 
 from . import build as _build
 
-F16, BF16, F64 = 0, 1, 2
+F16, BF16, F64, E4M3, E5M2 = 0, 1, 2, 3, 4
 
 _lib = None
 
@@ -67,6 +68,10 @@ def _as_storage(x, dtype_code: Optional[int] = None):
         import torch
         if isinstance(x, torch.Tensor):
             x = x.detach().cpu().contiguous()
+            if x.dtype == torch.float8_e4m3fn:
+                return x.view(torch.uint8).numpy(), E4M3
+            if x.dtype == torch.float8_e5m2:
+                return x.view(torch.uint8).numpy(), E5M2
             if x.dtype == torch.bfloat16:
                 return x.view(torch.int16).numpy().view(np.uint16), BF16
             if x.dtype == torch.float16:
@@ -159,6 +164,27 @@ def attn_fwd(q, k, v, scale: float, causal: bool = False, window_left: int = -1,
     if rc:
         raise ValueError("oracle_attn_fwd failed: %d" % rc)
     return (o, lse, p) if return_probs else (o, lse)
+
+
+def attn_fwd_fp8(q, k, v, scale: float, descale_q: float = 1.0, descale_k: float = 1.0, descale_v: float = 1.0,
+                 causal: bool = False, window_left: int = -1, window_right: int = -1, alibi_slopes=None,
+                 softcap: float = 0.0, rows: Optional[Sequence[int]] = None, num_threads: int = 0,
+                 dtype_code: Optional[int] = None):
+    """Attention on 8-bit inputs (the FP8 forward named in "FlashAttention深度解析：
+    从算法创新到产业变革的全面影响", section 未来展望, and "IO感知技术革命", section
+    H100架构的性能跃升; neither states the form): q, k, v hold E4M3 or E5M2
+    values x8 standing for x8 * descale_x, so the result is attn_fwd of the
+    dequantised inputs: the score scale becomes scale * descale_q * descale_k
+    and O is multiplied by descale_v (O is linear in V; LSE is unchanged).
+    Returns (o, lse) as attn_fwd."""
+    qa, code = _as_storage(q, dtype_code)
+    ka, kc = _as_storage(k, dtype_code)
+    va, vc = _as_storage(v, dtype_code)
+    if code not in (E4M3, E5M2) or not (code == kc == vc):
+        raise ValueError("q, k, v must share one 8-bit storage type")
+    o, lse = attn_fwd(qa, ka, va, float(scale) * float(descale_q) * float(descale_k), causal, window_left,
+                      window_right, alibi_slopes, softcap, rows=rows, num_threads=num_threads, dtype_code=code)
+    return o * float(descale_v), lse
 
 
 def _expand_heads(a: np.ndarray, H: int, axis: int) -> np.ndarray:

@@ -45,8 +45,9 @@
  *     to one contiguous key range of the sequence, and the merge of the
  *     partials is lse = ln sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s.
  *
- * Inputs may be given as fp16 or bf16 storage (the already-rounded values the
- * GPU sees; they are widened to fp64 exactly) or as fp64.
+ * Inputs may be given as fp16, bf16, fp8 E4M3 or fp8 E5M2 storage (the
+ * already-rounded values the GPU sees; they are widened to fp64 exactly) or
+ * as fp64.
  */
 #include <math.h>
 #include <stdint.h>
@@ -57,6 +58,8 @@
 #define ORACLE_F16 0
 #define ORACLE_BF16 1
 #define ORACLE_F64 2
+#define ORACLE_E4M3 3
+#define ORACLE_E5M2 4
 
 /* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
 static double widen_f16(uint16_t bits)
@@ -83,10 +86,50 @@ static double widen_bf16(uint16_t bits)
     return (double)f;
 }
 
+/* 8-bit floats (the FP8 forward that "FlashAttention深度解析" names, section
+ * 未来展望). E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 fraction bits; no
+ * infinities, exponent and fraction all ones is NaN, so the largest value is
+ * 1.75 * 2^8 = 448. */
+static double widen_e4m3(uint8_t bits)
+{
+    int sign = bits >> 7;
+    int expo = (bits >> 3) & 0xf;
+    int frac = bits & 0x7;
+    double mag;
+    if (expo == 15 && frac == 7)
+        return NAN;
+    if (expo == 0)
+        mag = ldexp((double)frac, -9);               /* subnormal: (frac / 8) * 2^(1-7) */
+    else
+        mag = ldexp((double)(8 + frac), expo - 10);  /* (1.frac) * 2^(e-7) */
+    return sign ? -mag : mag;
+}
+
+/* E5M2: 1 sign bit, 5 exponent bits (bias 15), 2 fraction bits, IEEE-style
+ * infinities and NaNs at exponent 31. */
+static double widen_e5m2(uint8_t bits)
+{
+    int sign = bits >> 7;
+    int expo = (bits >> 2) & 0x1f;
+    int frac = bits & 0x3;
+    double mag;
+    if (expo == 31)
+        mag = frac ? NAN : INFINITY;
+    else if (expo == 0)
+        mag = ldexp((double)frac, -16);              /* subnormal: (frac / 4) * 2^(1-15) */
+    else
+        mag = ldexp((double)(4 + frac), expo - 17);  /* (1.frac) * 2^(e-15) */
+    return sign ? -mag : mag;
+}
+
 static double load_elem(const void *base, long idx, int dtype)
 {
     if (dtype == ORACLE_F64)
         return ((const double *)base)[idx];
+    if (dtype == ORACLE_E4M3)
+        return widen_e4m3(((const uint8_t *)base)[idx]);
+    if (dtype == ORACLE_E5M2)
+        return widen_e5m2(((const uint8_t *)base)[idx]);
     uint16_t bits = ((const uint16_t *)base)[idx];
     return dtype == ORACLE_BF16 ? widen_bf16(bits) : widen_f16(bits);
 }
@@ -94,7 +137,7 @@ static double load_elem(const void *base, long idx, int dtype)
 /* Widens n stored elements to fp64 (exposed so tests can pin the decoders). */
 int oracle_widen(const void *src, int dtype, double *dst, long n)
 {
-    if (dtype < 0 || dtype > 2)
+    if (dtype < 0 || dtype > 4)
         return 1;
     for (long i = 0; i < n; ++i)
         dst[i] = load_elem(src, i, dtype);
@@ -207,7 +250,7 @@ int oracle_attn_fwd(const void *q, const void *k, const void *v, int dtype,
 {
     if (!q || !k || !v || !o || !lse || B < 0 || H < 0 || Nq < 0 || Nk < 0 || d <= 0)
         return 1;
-    if (dtype < 0 || dtype > 2)
+    if (dtype < 0 || dtype > 4)
         return 1;
     if (!rows)
         n_rows = Nq;
@@ -302,7 +345,7 @@ int oracle_attn_decode_paged(const void *q, const void *k_cache, const void *v_c
 {
     if (!q || !k_cache || !v_cache || !block_table || !cache_seqlens || !o || !lse)
         return 1;
-    if (B < 0 || H <= 0 || d <= 0 || page_size <= 0 || max_blocks < 0 || dtype < 0 || dtype > 2)
+    if (B < 0 || H <= 0 || d <= 0 || page_size <= 0 || max_blocks < 0 || dtype < 0 || dtype > 4)
         return 1;
     if (!batch)
         n_batch = B;

@@ -35,6 +35,9 @@ MUTANTS = {
     "split_drops_a_key": ("long b = a + chunk;", "long b = a + chunk - 1;"),
     "fp16_exponent_bias": ("mag = ldexp((double)(1024 + frac), expo - 25);",
                            "mag = ldexp((double)(1024 + frac), expo - 24);"),
+    "e4m3_exponent_bias": ("mag = ldexp((double)(8 + frac), expo - 10);",
+                           "mag = ldexp((double)(8 + frac), expo - 9);"),
+    "e5m2_subnormal_scale": ("mag = ldexp((double)frac, -16);", "mag = ldexp((double)frac, -15);"),
 }
 
 
@@ -57,6 +60,8 @@ def battery():
     yield lambda: pins.test_permuted_block_table_is_a_reindexing({})
     yield lambda: pins.test_any_split_count_matches_one_split(3, {})
     yield lambda: pins.test_half_precision_storage_is_widened_exactly()
+    yield lambda: pins.test_widen_fp8_every_bit_pattern(oracle.E4M3, pins.torch.float8_e4m3fn)
+    yield lambda: pins.test_widen_fp8_every_bit_pattern(oracle.E5M2, pins.torch.float8_e5m2)
 
 
 def run_battery():

@@ -642,3 +642,36 @@ def test_bwd_rows_without_keys_carry_no_gradient():
     dout2[:, :Nq - Nk] = 123.0
     _, dk2, dv2 = oracle.attn_bwd(q, k, v, dout2, 0.5, causal=True)
     assert np.abs(dk2 - dk).max() < TOL and np.abs(dv2 - dv).max() < TOL
+
+
+# ---------------------------------------------------------------- 8-bit inputs
+
+@pytest.mark.parametrize("code,tdtype", [(oracle.E4M3, torch.float8_e4m3fn), (oracle.E5M2, torch.float8_e5m2)],
+                         ids=["e4m3", "e5m2"])
+def test_widen_fp8_every_bit_pattern(code, tdtype):
+    """Every 8-bit pattern against torch's own float8 conversion (an
+    independent implementation of the same formats)."""
+    bits = np.arange(256, dtype=np.uint8)
+    got = oracle.widen(bits, code)
+    want = torch.from_numpy(bits).view(tdtype).to(torch.float64).numpy()
+    assert np.array_equal(got, want, equal_nan=True)
+
+
+@pytest.mark.parametrize("tdtype", [torch.float8_e4m3fn, torch.float8_e5m2], ids=["e4m3", "e5m2"])
+@pytest.mark.parametrize("opts", [dict(causal=True), dict(causal=False, window_left=3, window_right=1),
+                                  dict(causal=True, alibi_slopes=[0.25, 0.5], softcap=2.0)])
+def test_fp8_attention_is_attention_of_the_dequantised_inputs(tdtype, opts):
+    B, H, Nq, Nk, d = 1, 2, 6, 9, 16
+    g = torch.Generator().manual_seed(41)
+    q8, k8, v8 = (torch.randn(B, n, H, d, generator=g).mul(8.0).to(tdtype) for n in (Nq, Nk, Nk))
+    dq, dk, dv, scale = 0.02, 0.05, 0.3, 0.25
+    o, lse = oracle.attn_fwd_fp8(q8, k8, v8, scale, dq, dk, dv, **opts)
+    deq = lambda t, s: t.to(torch.float64).numpy() * s
+    o_ref, l_ref = oracle.attn_fwd(deq(q8, dq), deq(k8, dk), deq(v8, dv), scale, **opts)
+    assert np.abs(o - o_ref).max() < 1e-12 and np.abs(lse - l_ref).max() < 1e-12
+
+
+def test_fp8_oracle_rejects_mixed_storage():
+    x = torch.zeros(1, 2, 1, 16).to(torch.float8_e4m3fn)
+    with pytest.raises(ValueError):
+        oracle.attn_fwd_fp8(x, x.to(torch.float32).to(torch.float8_e5m2), x, 0.1)
