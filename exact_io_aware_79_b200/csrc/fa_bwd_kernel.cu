@@ -49,6 +49,8 @@ namespace {
 
 constexpr int kBwdWarps = 4;
 constexpr int kBlk = 64;  // keys per CTA, queries per step
+// each CTA thread fetches one of the block's 64 lse and 64 D values
+static_assert(kBwdWarps * 32 == 2 * kBlk, "row-vector fetch assumes two values per query row per thread pair");
 
 __device__ __forceinline__ int perm8(int n) { return (n >> 1) | ((n & 1) << 2); }
 
@@ -66,7 +68,7 @@ struct BwdCfg {
   static constexpr int kOffQ = 2 * kTile;   // two buffers
   static constexpr int kOffO = 4 * kTile;   // two buffers (dO)
   static constexpr int kOffS = 6 * kTile;   // dS^T, 64 x 64 16-bit
-  static constexpr int kOffL = kOffS + kBlk * kBlk * 2;  // lse2[2][64], dvec[2][64]
+  static constexpr int kOffL = kOffS + kBlk * kBlk * 2;  // [2 buffers][lse * log2(e) x 64, D x 64] fp32
   static constexpr int kOffBar = kOffL + 4 * kBlk * 4;
   static constexpr int kSmem = 1024 + kOffBar + 64;  // + slack to align to 1 KB
 };
