@@ -331,9 +331,21 @@ fa_status kvcache_common(const void* q, const void* k_cache, const void* v_cache
   if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return FA_ERR_ARG;
-  const int S = fa_kvcache_num_splits(B, H, d, max_blocks, page_size, num_splits);
+  int S = fa_kvcache_num_splits(B, H, d, max_blocks, page_size, num_splits);
   const size_t need = fa_kvcache_workspace_size(B, H, d, max_blocks, page_size, num_splits);
   if (S > 1 && (!workspace || !aligned16(workspace) || workspace_bytes < need)) return FA_ERR_WORKSPACE;
+  if (num_splits == 0 && S > 1 && page_size % 64 == 0 && fa::decode_on_tensor_cores(H, H_kv)) {
+    // a grouped-query CTA serves G query heads and streams their cache head
+    // once: aim the automatic count at the CTAs launched (about 2048 * G keys
+    // a split, enough CTAs to fill the GPU), never above S, so the workspace
+    // sized for S still holds the partials
+    const long long G = fa::decode_group_heads(H, H_kv);
+    const long long max_len = static_cast<long long>(max_blocks) * page_size;
+    const long long units = static_cast<long long>(B) * (H / G);
+    long long s = ((max_len + 2047) / 2048 + G - 1) / G;
+    s = std::max(s, std::min((4LL * kNumSms + units - 1) / units, (max_len + 255) / 256));
+    S = static_cast<int>(std::max(1LL, std::min(s, static_cast<long long>(S))));
+  }
   fa_status st = check_device();
   if (st != FA_OK) return st;
 

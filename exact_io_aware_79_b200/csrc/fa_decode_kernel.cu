@@ -877,15 +877,8 @@ template <typename T, int D>
 cudaError_t launch(const DecodeParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV, cudaStream_t stream) {
   dim3 grid(p.H * p.num_splits, p.B);
   if (tmK != nullptr && decode_on_tensor_cores(p.H, p.H_kv)) {
-    // query heads per CTA: the largest divisor of the group that fits the 16 product rows
-    const int group = p.H / p.H_kv;
-    int G = 1;
-    for (int g = kMmaRows; g >= 1; --g) {
-      if (group % g == 0) {
-        G = g;
-        break;
-      }
-    }
+    static_assert(kMmaRows == 16, "decode_group_heads assumes 16 product rows");
+    const int G = decode_group_heads(p.H, p.H_kv);  // query heads per CTA
     using C = MmaCfg<D>;
     auto kernel = decode_split_mma_kernel<T, D>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);

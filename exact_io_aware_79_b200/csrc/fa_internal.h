@@ -65,6 +65,15 @@ cudaError_t launch_fwd(bool bf16, int d, const CUtensorMap& tmQ, const CUtensorM
 // tensor-core split kernel; it wants 128-byte-swizzled (64, 1, 64, 1) boxes.
 inline bool decode_on_tensor_cores(int H, int H_kv) { return H_kv > 0 && H / H_kv >= 2; }
 
+// Query heads one grouped-query decode CTA serves: the largest divisor of the
+// group H / H_kv that fits the 16 rows of its products.
+inline int decode_group_heads(int H, int H_kv) {
+  const int group = H / H_kv;
+  for (int g = 16; g > 1; --g)
+    if (group % g == 0) return g;
+  return 1;
+}
+
 // tmK/tmV: 4-D maps (d, H, page_size, num_pages) of the caches for the
 // TMA-staged split kernels (page_size % 64 == 0): a (d, 1, 64, 1) box without
 // swizzle, or (64, 1, 64, 1) boxes with 128-byte swizzle when

@@ -1,11 +1,13 @@
 /*
  * fa.h -- C ABI of the B200 (sm_100a) exact-attention library.
  *
- * Two operations, both exact scaled-dot-product attention
+ * Exact scaled-dot-product attention
  *     O = softmax(S) V,   S = scale * Q K^T  (+ score modifiers, + mask),
  * computed tile by tile with an online softmax so that neither the score
  * matrix S nor the probability matrix P ever reaches device memory, plus the
- * per-row natural log-sum-exp LSE_i = ln sum_j exp(S_ij).
+ * per-row natural log-sum-exp LSE_i = ln sum_j exp(S_ij): the forward (fixed
+ * length, packed sequences, packed QKV, grouped-query heads), the paged
+ * split-KV decode (with the cache append), and the backward (dQ, dK, dV).
  *
  * Sources (web pages about FlashAttention; their formulas were lost in
  * extraction, so the readings below state the plain form that the rest of the
@@ -22,7 +24,7 @@
  *     softcapping: "Flash-Attention v2.0 到 v2.7 更新", opening paragraph and
  *     sections v2.1, v2.2, v2.3, v2.4, v2.5, v2.6.
  *
- * Conventions shared by both calls
+ * Conventions shared by the calls
  *   - Every tensor pointer is a DEVICE pointer to contiguous memory, 16-byte
  *     aligned, owned by the caller. The library allocates nothing, keeps no
  *     pointer after a call returns and holds no global state besides a
@@ -224,9 +226,12 @@ fa_status fa_fwd_kvcache(const void *q, const void *k_cache, const void *v_cache
  * fa_fwd_kvcache_gqa -- fa_fwd_kvcache with grouped-query attention: the
  * caches hold H_kv heads ([num_pages, page_size, H_kv, d]); query head h
  * attends with cache head h / (H / H_kv). 1 <= H_kv <= H and H % H_kv == 0,
- * else FA_ERR_SHAPE. Split count, workspace size and every other argument
- * as for fa_fwd_kvcache with the same B, H, d (fa_kvcache_num_splits and
- * fa_kvcache_workspace_size take H, the query heads).
+ * else FA_ERR_SHAPE. Workspace size and every other argument as for
+ * fa_fwd_kvcache with the same B, H, d (fa_kvcache_num_splits and
+ * fa_kvcache_workspace_size take H, the query heads). With num_splits = 0
+ * and several query heads per cache head, the automatic count may be lower
+ * than fa_kvcache_num_splits reports (one CTA serves a group of query heads
+ * and reads its cache head once), never higher, so that workspace suffices.
  */
 fa_status fa_fwd_kvcache_gqa(const void *q, const void *k_cache, const void *v_cache,
                              const int *block_table, const int *cache_seqlens,
