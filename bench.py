@@ -2,7 +2,9 @@
 """Benchmark of the exact-attention hot path on B200.
 
 One step = one pass of the whole path over one batch of synthetic input:
-  1. fa_fwd on the causal training shape (B=8, H=16, Nq=Nk=2048, d=128, bf16);
+  1. fa_fwd on the long sliding-window shape (B=1, H=16, Nq=Nk=16384,
+     d=128, bf16, causal, window_left=4096): the N >= 8K, d = 128 forward
+     the throughput target is stated for;
   2. fa_fwd_kvcache on the paged decode batch (B=64, H=32, d=128, bf16,
      pages of 256 tokens, lengths U[1024, 32768], automatic split count):
      split kernel + merge kernel.
@@ -10,7 +12,10 @@ The headline value is the forward's TFLOP/s (4*d*H*B*(unmasked query/key
 pairs) per launch over its CUDA-event time); the decode's KV GB/s
 (2*2*H*d bytes per cached token over the call's time) is reported beside it.
 Both inputs exceed the 126 MB L2 (forward Q+K+V 201 MB, decode K/V 34 GB),
-so no explicit flush is needed between iterations.
+so no explicit flush is needed between iterations. After the timed steps
+every forward workload of the suite (causal 2K, window 16K, window and causal
+Nq 4K / Nk 16K, ALiBi + softcap) is timed on its own with L2 flushed between
+launches and reported under "forward_configs".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
   python bench.py --sweep          # every forward workload and decode split
@@ -44,14 +49,21 @@ METRIC = "attn fwd TFLOP/s (% of BF16 peak); paged-decode KV GB/s (% of HBM BW)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# ncu captures of the kernels as they stand; each entry names its capture.
-# Decode: a capture of the 4-sequence case read 1.003 x its K/V bytes and
-# wrote 2.8 MB of partials (profiles/decode_split_tma_paged_decode_b4h32d128_page256.md);
-# reads scale with the K/V bytes, each byte being read once.
+# ncu captures of the kernels as they stand.
+# Decode: a capture of the split kernel on the 4-sequence case (B=4, H=32,
+# d=128, pages of 256) read 1.003 x its K/V bytes and wrote 2.8 MB of
+# partials; reads scale with the K/V bytes, each byte being read once.
 DECODE_READ_PER_KV_BYTE = 967959936.0 / 965165056.0  # (968,019,712 + 967,900,160) / 2 / K/V bytes
-# Forward, causal B8 H16 N2048 d128: mean of two captured launches
-# (profiles/fwd_kernel_causal_b8h16n2048d128.md, last table).
-FWD_CAUSAL_2K_TRAFFIC = (201453056.0 + 38760448.0 + 201453312.0 + 35730432.0) / 2.0
+# Forward: per-launch DRAM bytes of captures of the forward kernel on the
+# named workload, for the kernel version they were taken on; None where no
+# capture of the present kernel exists.
+FWD_TRAFFIC = {
+    W.WINDOW_16K.name: 201647104.0 + 45596672.0,
+    W.CAUSAL_2K.name: (201453056.0 + 38760448.0 + 201453312.0 + 35730432.0) / 2.0,
+}
+# Forward workloads timed one by one after the step (L2 flushed between launches).
+FWD_CONFIGS = [W.CAUSAL_2K, W.WINDOW_16K, W.WINDOW_Q4K_K16K, W.CAUSAL_Q4K_K16K, W.ALIBI_SOFTCAP]
+HEADLINE_FWD = W.WINDOW_16K
 
 
 # ---------------------------------------------------------------- algorithmic work
@@ -59,6 +71,11 @@ FWD_CAUSAL_2K_TRAFFIC = (201453056.0 + 38760448.0 + 201453312.0 + 35730432.0) / 
 def unmasked_pairs(w: W.FwdWorkload) -> int:
     """Query/key pairs that survive the mask, per (batch, head): sum over
     rows of the visible interval length (interval arithmetic, no oracle)."""
+    return int(visible_keys_per_row(w).sum())
+
+
+def visible_keys_per_row(w: W.FwdWorkload) -> np.ndarray:
+    """Number of keys each query row sees (interval arithmetic)."""
     i = np.arange(w.Nq, dtype=np.int64)
     pos = i + w.Nk - w.Nq
     lo = np.zeros_like(i) if w.window_left < 0 else np.maximum(0, pos - w.window_left)
@@ -67,7 +84,7 @@ def unmasked_pairs(w: W.FwdWorkload) -> int:
         hi = np.minimum(hi, pos)
     if w.window_right >= 0:
         hi = np.minimum(hi, pos + w.window_right)
-    return int(np.maximum(0, hi - lo + 1).sum())
+    return np.maximum(0, hi - lo + 1)
 
 
 def fwd_flops(w: W.FwdWorkload) -> float:
@@ -210,16 +227,7 @@ def oracle_fwd_sample(w: W.FwdWorkload, x, budget_s: float):
     """Times the oracle on a growing sample of query rows (all batches and
     heads) until about budget_s of CPU work; returns (TFLOP/s, rows, seconds)."""
     import oracle
-    rows_all = np.arange(w.Nq)
-    i = rows_all
-    pos = i + w.Nk - w.Nq
-    lo = np.zeros_like(i) if w.window_left < 0 else np.maximum(0, pos - w.window_left)
-    hi = np.full_like(i, w.Nk - 1)
-    if w.causal:
-        hi = np.minimum(hi, pos)
-    if w.window_right >= 0:
-        hi = np.minimum(hi, pos + w.window_right)
-    vis = np.maximum(0, hi - lo + 1)
+    vis = visible_keys_per_row(w)
     n = 2
     rng = np.random.default_rng(0)
     while True:
@@ -275,7 +283,7 @@ def gpu_arm(args):
     dev = torch.device("cuda", local)
     peaks, peak_src = load_peaks()
 
-    fw = W.CAUSAL_2K
+    fw = HEADLINE_FWD
     dw = W.DECODE
     x = W.make_fwd_inputs(fw, device=dev)
     xd = W.make_decode_inputs(dw, device=dev)
@@ -334,6 +342,9 @@ def gpu_arm(args):
     dec_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in de) / K, world, dev)
     fwd_tflops = weak_scaling_value(F, fwd_ms * 1e-3, world) / 1e12
     dec_gbs = weak_scaling_value(KVB, dec_ms * 1e-3, world) / 1e9
+
+    # ---- every forward workload on its own (L2 flushed between launches)
+    fwd_configs = time_fwd_configs(fa, dev, world, peaks, args, physical_gpu(local))
 
     # ---- end to end through the public API with pinned host buffers
     hq, hk, hv = (x[n].cpu().pin_memory() for n in ("q", "k", "v"))
@@ -399,7 +410,9 @@ def gpu_arm(args):
                           "sample": "%s (repeats x sequences) of %d sequences, all heads, %.1f s; credited "
                                     "bytes = K+V of the sampled sequences" % (seqs, dw.B, t_d)}}
 
-    peak_t = peaks["bf16_tflops_sustained"]
+    # the forward is one sub-millisecond launch inside the step, so its
+    # roofline is the burst tensor peak
+    peak_t = peaks["bf16_tflops"]
     peak_h = peaks["hbm_gbs"]
     result = {
         "metric": METRIC,
@@ -420,7 +433,8 @@ def gpu_arm(args):
                         "flops_per_launch": F},
             "decode": {"B": dw.B, "H": dw.H, "d": dw.d, "page_size": dw.page_size,
                        "seqlens": [dw.len_lo, dw.len_hi], "num_splits": splits, "kv_bytes_per_launch": KVB},
-            "l2": "inputs larger than L2 (forward Q+K+V 201 MB, decode K/V 34 GB); no flush",
+            "l2": "step: inputs larger than L2 (forward Q+K+V 201 MB, decode K/V 34 GB), no flush; "
+                  "forward_configs: L2 flushed (256 MB write) before every launch",
             "parallelism": "replicas" if world > 1 else "single GPU",
         },
         "roofline": {"kernel": "decode (split + merge)", "bound": "hbm", "achieved": round(dec_gbs / world, 1),
@@ -428,12 +442,14 @@ def gpu_arm(args):
                      "traffic": round(DECODE_READ_PER_KV_BYTE * KVB),
                      "traffic_source": "ncu capture of the 4-sequence case, scaled by K/V bytes",
                      "peak_source": peak_src},
-        "roofline_fwd": {"kernel": "fwd_kernel", "bound": "tensor", "achieved": round(fwd_tflops / world, 2),
-                         "peak": peak_t, "unit": "TFLOP/s", "frac": round(fwd_tflops / world / peak_t, 4),
-                         "frac_of_burst": round(fwd_tflops / world / peaks["bf16_tflops"], 4),
-                         "traffic": round(FWD_CAUSAL_2K_TRAFFIC) if fw is W.CAUSAL_2K else None,
+        "roofline_fwd": {"kernel": "fwd_kernel", "workload": fw.name, "bound": "tensor",
+                         "achieved": round(fwd_tflops / world, 2), "peak": peak_t, "unit": "TFLOP/s",
+                         "frac": round(fwd_tflops / world / peak_t, 4),
+                         "frac_of_sustained": round(fwd_tflops / world / peaks["bf16_tflops_sustained"], 4),
+                         "traffic": round(FWD_TRAFFIC[fw.name]) if FWD_TRAFFIC.get(fw.name) else None,
                          "traffic_source": "ncu capture of this workload",
-                         "peak_source": peak_src + " sustained"},
+                         "peak_source": peak_src + " burst"},
+        "forward_configs": fwd_configs,
         "decode": {"value": round(dec_gbs, 1), "unit": "GB/s", "ms_per_launch": round(dec_ms, 4)},
         "fwd_ms_per_launch": round(fwd_ms, 4),
         "e2e": {"value": round(world * F / (e_fwd_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
@@ -452,6 +468,50 @@ def gpu_arm(args):
         torch.distributed.destroy_process_group()
 
 
+def time_fwd_configs(fa, dev, world, peaks, args, gpu_index):
+    """Times fa_fwd on every workload of FWD_CONFIGS: W warm-up launches, then
+    the median of K CUDA-event-timed launches, each after a 256 MB write that
+    flushes L2; returns {workload: {ms, TFLOP/s, frac of the burst peak}}
+    with the SM clocks seen while they ran."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    res = {}
+    sampler = ClockSampler(gpu_index)
+    sampler.start()
+    t0 = time.time()
+    for w in FWD_CONFIGS:
+        x = W.make_fwd_inputs(w, device=dev)
+        out = torch.empty_like(x["q"])
+        lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+        run = lambda: fa.fa_fwd(x["q"], x["k"], x["v"], out, lse, w.scale, w.causal, w.window_left,
+                                w.window_right, x["slopes"], w.softcap)
+        for _ in range(max(3, args.warmup)):
+            run()
+        times = []
+        n = max(5, min(args.steps, args.config_steps))
+        barrier(world)
+        for _ in range(n):
+            flush.zero_()
+            a, b = ev(), ev()
+            a.record()
+            run()
+            b.record()
+            times.append((a, b))
+        torch.cuda.synchronize()
+        ms = max_over_ranks(statistics.median([a.elapsed_time(b) for a, b in times]), world, dev)
+        tf = weak_scaling_value(fwd_flops(w), ms * 1e-3, world) / 1e12
+        res[w.name] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                       "frac": round(tf / world / peaks["bf16_tflops"], 4), "flops_per_launch": fwd_flops(w),
+                       "launches": n}
+        del x, out, lse
+    t1 = time.time()
+    sampler.stop()
+    res["peak"] = "measured burst bf16 %.1f TFLOP/s" % peaks["bf16_tflops"]
+    res["clocks"] = sampler.summary(t0, t1)
+    del flush
+    return res
+
+
 # ---------------------------------------------------------------- reference arm (the oracle)
 
 def reference_arm(args):
@@ -459,14 +519,13 @@ def reference_arm(args):
     if rank != 0:
         return
     import oracle
-    fw = W.CAUSAL_2K
+    fw = HEADLINE_FWD
     x = W.make_fwd_inputs(fw)
     budget = max(0.3, min(3.0, 150.0 / max(1, args.steps + args.warmup)))
     # size one step's row sample once, then time K steps of it
     _, rows, _ = oracle_fwd_sample(fw, x, budget)
     rng = np.random.default_rng(1)
-    i = np.arange(fw.Nq)
-    vis = np.minimum(i, fw.Nq - 1) + 1  # causal, Nq == Nk
+    vis = visible_keys_per_row(fw)
     times, flops = [], 0.0
     for s in range(args.warmup + args.steps):
         sel = np.sort(rng.choice(fw.Nq, size=rows, replace=False))
@@ -629,8 +688,9 @@ def sweep(args):
             torch.cuda.synchronize()
             ms = statistics.median([a.elapsed_time(b) for a, b in times])
             gbs = KVB / (ms * 1e-3) / 1e9
-            print(json.dumps({"workload": dw.name, "num_splits": s or "auto(%d)" % fa.fa_kvcache_num_splits(
-                dw.B, dw.H, dw.d, dw.max_blocks, dw.page_size, 0), "ms": round(ms, 4), "GB/s": round(gbs, 1),
+            print(json.dumps({"workload": dw.name, "num_splits": s or "auto(%d)" % fa.fa_kvcache_num_splits_gqa(
+                dw.B, dw.H, dw.kv_heads, dw.d, dw.max_blocks, dw.page_size, 0), "ms": round(ms, 4),
+                "GB/s": round(gbs, 1),
                 "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "kv_bytes": KVB, "peak_source": peak_src}),
                 flush=True)
         del xd
@@ -643,6 +703,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--config-steps", type=int, default=20, help="timed launches per forward_configs entry")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work per baseline leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true")

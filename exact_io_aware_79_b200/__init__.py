@@ -77,6 +77,8 @@ def _lib_handle():
         L.fa_fwd_kvcache_noalloc.restype = i
         L.fa_kvcache_num_splits.argtypes = [i, i, i, i, i, i]
         L.fa_kvcache_num_splits.restype = i
+        L.fa_kvcache_num_splits_gqa.argtypes = [i, i, i, i, i, i, i]
+        L.fa_kvcache_num_splits_gqa.restype = i
         L.fa_kvcache_workspace_size.argtypes = [i, i, i, i, i, i]
         L.fa_kvcache_workspace_size.restype = sz
         L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
@@ -128,6 +130,23 @@ def _check(code: int, where: str):
         raise FaError(code, where)
 
 
+def _on_device(where: str, tensors, alibi_slopes=None, H: int = 0, workspace=None) -> None:
+    """Checks, before anything is launched, that every tensor lives on the
+    device of the first one (a CUDA device), and that alibi_slopes, when
+    given, is a contiguous fp32 [H] tensor there: a host pointer or another
+    GPU's pointer handed to a kernel would be an illegal device access, not
+    an error the library could report."""
+    ref = tensors[0]
+    extra = [t for t in (alibi_slopes, workspace) if t is not None]
+    for t in list(tensors) + extra:
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.device != ref.device:
+            raise ValueError("%s: every tensor must be a CUDA tensor on %s" % (
+                where, ref.device if ref.is_cuda else "one CUDA device"))
+    if alibi_slopes is not None and (alibi_slopes.dtype != torch.float32 or tuple(alibi_slopes.shape) != (H,)
+                                     or not alibi_slopes.is_contiguous()):
+        raise ValueError("%s: alibi_slopes must be a contiguous fp32 tensor of shape [%d]" % (where, H))
+
+
 def fa_status_string(code: int) -> str:
     return _lib_handle().fa_status_string(code).decode()
 
@@ -146,6 +165,7 @@ def fa_fwd(q, k, v, out, lse, scale: float, causal: bool = False, window_left: i
         raise ValueError("fa_fwd: lse must be fp32 [B, H, Nq]")
     if not (q.dtype == k.dtype == v.dtype == out.dtype):
         raise ValueError("fa_fwd: q, k, v, out must share one dtype")
+    _on_device("fa_fwd", (q, k, v, out, lse), alibi_slopes, H)
     code = _lib_handle().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Nq, Nk, d,
                                 _dtype_code(q), float(scale), int(bool(causal)), int(window_left),
                                 int(window_right), _ptr(alibi_slopes), float(softcap), _stream(stream))
@@ -168,6 +188,7 @@ def fa_fwd_gqa(q, k, v, out, lse, scale: float, causal: bool = False, window_lef
         raise ValueError("fa_fwd_gqa: lse must be fp32 [B, H, Nq]")
     if not (q.dtype == k.dtype == v.dtype == out.dtype):
         raise ValueError("fa_fwd_gqa: q, k, v, out must share one dtype")
+    _on_device("fa_fwd_gqa", (q, k, v, out, lse), alibi_slopes, H)
     code = _lib_handle().fa_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, H_kv, Nq, Nk, d,
                                     _dtype_code(q), float(scale), int(bool(causal)), int(window_left),
                                     int(window_right), _ptr(alibi_slopes), float(softcap), _stream(stream))
@@ -198,6 +219,7 @@ def fa_bwd(q, k, v, out, lse, dout, dq, dk, dv, scale: float, causal: bool = Fal
         raise ValueError("fa_bwd: lse must be fp32 [B, H, Nq]")
     if len({t.dtype for t in (q, k, v, out, dout, dq, dk, dv)}) != 1:
         raise ValueError("fa_bwd: q, k, v, out, dout, dq, dk, dv must share one dtype")
+    _on_device("fa_bwd", (q, k, v, out, lse, dout, dq, dk, dv), alibi_slopes, H, workspace=workspace)
     need = fa_bwd_workspace_size(B, H, Nq, d)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
@@ -231,6 +253,8 @@ def fa_bwd_varlen(q, k, v, out, lse, dout, dq, dk, dv, cu_seqlens_q, cu_seqlens_
         raise ValueError("fa_bwd_varlen: lse must be fp32 [H, total_q]")
     if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
         raise ValueError("fa_bwd_varlen: cu_seqlens must be int32")
+    _on_device("fa_bwd_varlen", (q, k, v, out, lse, dout, dq, dk, dv, cu_seqlens_q, cu_seqlens_k),
+               alibi_slopes, H, workspace=workspace)
     need = fa_bwd_workspace_size(1, H, total_q, d)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
@@ -257,6 +281,7 @@ def fa_bwd_qkvpacked(qkv, out, lse, dout, dqkv, scale: float, causal: bool = Fal
         raise ValueError("fa_bwd_qkvpacked: shape mismatch")
     if tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32:
         raise ValueError("fa_bwd_qkvpacked: lse must be fp32 [B, H, N]")
+    _on_device("fa_bwd_qkvpacked", (qkv, out, lse, dout, dqkv), alibi_slopes, H, workspace=workspace)
     if workspace is None:
         workspace = torch.empty(max(fa_bwd_workspace_size(B, H, N, d), 16), dtype=torch.uint8, device=qkv.device)
     code = _lib_handle().fa_bwd_qkvpacked(_ptr(qkv), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dqkv), B, H, N, d,
@@ -283,6 +308,8 @@ def fa_bwd_varlen_qkvpacked(qkv, out, lse, dout, dqkv, cu_seqlens, max_seqlen: i
         raise ValueError("fa_bwd_varlen_qkvpacked: shape mismatch")
     if tuple(lse.shape) != (H, total) or lse.dtype != torch.float32 or cu_seqlens.dtype != torch.int32:
         raise ValueError("fa_bwd_varlen_qkvpacked: lse must be fp32 [H, total], cu_seqlens int32")
+    _on_device("fa_bwd_varlen_qkvpacked", (qkv, out, lse, dout, dqkv, cu_seqlens),
+               alibi_slopes, H, workspace=workspace)
     if workspace is None:
         workspace = torch.empty(max(fa_bwd_workspace_size(1, H, total, d), 16), dtype=torch.uint8,
                                 device=qkv.device)
@@ -306,6 +333,7 @@ def fa_fwd_qkvpacked(qkv, out, lse, scale: float, causal: bool = False, window_l
         raise ValueError("fa_fwd_qkvpacked: shape mismatch")
     if tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32:
         raise ValueError("fa_fwd_qkvpacked: lse must be fp32 [B, H, N]")
+    _on_device("fa_fwd_qkvpacked", (qkv, out, lse), alibi_slopes, H)
     code = _lib_handle().fa_fwd_qkvpacked(_ptr(qkv), _ptr(out), _ptr(lse), B, H, N, d, _dtype_code(qkv),
                                           float(scale), int(bool(causal)), int(window_left), int(window_right),
                                           _ptr(alibi_slopes), float(softcap), _stream(stream))
@@ -325,6 +353,7 @@ def fa_fwd_varlen_qkvpacked(qkv, out, lse, cu_seqlens, max_seqlen: int, scale: f
         raise ValueError("fa_fwd_varlen_qkvpacked: shape mismatch")
     if tuple(lse.shape) != (H, total) or lse.dtype != torch.float32 or cu_seqlens.dtype != torch.int32:
         raise ValueError("fa_fwd_varlen_qkvpacked: lse must be fp32 [H, total], cu_seqlens int32")
+    _on_device("fa_fwd_varlen_qkvpacked", (qkv, out, lse, cu_seqlens), alibi_slopes, H)
     code = _lib_handle().fa_fwd_varlen_qkvpacked(_ptr(qkv), _ptr(out), _ptr(lse), _ptr(cu_seqlens), B, H,
                                                  int(max_seqlen), total, d, _dtype_code(qkv), float(scale),
                                                  int(bool(causal)), int(window_left), int(window_right),
@@ -351,6 +380,7 @@ def fa_fwd_varlen(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: i
         raise ValueError("fa_fwd_varlen: cu_seqlens must be int32 [B + 1]")
     if not (q.dtype == k.dtype == v.dtype == out.dtype):
         raise ValueError("fa_fwd_varlen: q, k, v, out must share one dtype")
+    _on_device("fa_fwd_varlen", (q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k), alibi_slopes, H)
     code = _lib_handle().fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
                                        _ptr(cu_seqlens_k), B, H, int(max_seqlen_q), int(max_seqlen_k), total_q,
                                        total_k, d, _dtype_code(q), float(scale), int(bool(causal)),
@@ -361,6 +391,12 @@ def fa_fwd_varlen(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: i
 
 def fa_kvcache_num_splits(B: int, H: int, d: int, max_blocks: int, page_size: int, num_splits: int = 0) -> int:
     return int(_lib_handle().fa_kvcache_num_splits(B, H, d, max_blocks, page_size, num_splits))
+
+
+def fa_kvcache_num_splits_gqa(B: int, H: int, H_kv: int, d: int, max_blocks: int, page_size: int,
+                              num_splits: int = 0) -> int:
+    """Split count fa_fwd_kvcache_gqa launches with H_kv cache heads."""
+    return int(_lib_handle().fa_kvcache_num_splits_gqa(B, H, H_kv, d, max_blocks, page_size, num_splits))
 
 
 def fa_kvcache_workspace_size(B: int, H: int, d: int, max_blocks: int, page_size: int,
@@ -382,10 +418,13 @@ def fa_fwd_kvcache(q, k_cache, v_cache, block_table, cache_seqlens, out, lse, sc
     if one != 1 or tuple(k_cache.shape) != (num_pages, page_size, H, d) or \
             tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
         raise ValueError("fa_fwd_kvcache: shape mismatch")
-    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32 or block_table.shape[0] != B:
-        raise ValueError("fa_fwd_kvcache: block_table / cache_seqlens must be int32 [B, ...]")
+    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32 or block_table.shape[0] != B or \
+            tuple(cache_seqlens.shape) != (B,) or block_table.dim() != 2:
+        raise ValueError("fa_fwd_kvcache: block_table must be int32 [B, max_blocks], cache_seqlens int32 [B]")
     if tuple(lse.shape) != (B, H, 1) or lse.dtype != torch.float32:
         raise ValueError("fa_fwd_kvcache: lse must be fp32 [B, H, 1]")
+    _on_device("fa_fwd_kvcache", (q, k_cache, v_cache, block_table, cache_seqlens, out, lse),
+               alibi_slopes, H, workspace=workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     code = _lib_handle().fa_fwd_kvcache(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(cache_seqlens), _ptr(out), _ptr(lse),
@@ -408,10 +447,13 @@ def fa_fwd_kvcache_gqa(q, k_cache, v_cache, block_table, cache_seqlens, out, lse
     if one != 1 or tuple(k_cache.shape) != (num_pages, page_size, H_kv, d) or \
             tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
         raise ValueError("fa_fwd_kvcache_gqa: shape mismatch")
-    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32 or block_table.shape[0] != B:
-        raise ValueError("fa_fwd_kvcache_gqa: block_table / cache_seqlens must be int32 [B, ...]")
+    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32 or block_table.shape[0] != B or \
+            tuple(cache_seqlens.shape) != (B,) or block_table.dim() != 2:
+        raise ValueError("fa_fwd_kvcache_gqa: block_table must be int32 [B, max_blocks], cache_seqlens int32 [B]")
     if tuple(lse.shape) != (B, H, 1) or lse.dtype != torch.float32:
         raise ValueError("fa_fwd_kvcache_gqa: lse must be fp32 [B, H, 1]")
+    _on_device("fa_fwd_kvcache_gqa", (q, k_cache, v_cache, block_table, cache_seqlens, out, lse),
+               alibi_slopes, H, workspace=workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     code = _lib_handle().fa_fwd_kvcache_gqa(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(cache_seqlens), _ptr(out), _ptr(lse),
@@ -432,10 +474,12 @@ def fa_kvcache_append(k_new, v_new, k_cache, v_cache, block_table, cache_seqlens
     if tuple(v_new.shape) != tuple(k_new.shape) or tuple(k_cache.shape) != (num_pages, page_size, H_kv, d) or \
             tuple(v_cache.shape) != tuple(k_cache.shape):
         raise ValueError("fa_kvcache_append: shape mismatch")
-    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32 or block_table.shape[0] != B:
-        raise ValueError("fa_kvcache_append: block_table / cache_seqlens must be int32 [B, ...]")
+    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32 or block_table.shape[0] != B or \
+            tuple(cache_seqlens.shape) != (B,) or block_table.dim() != 2:
+        raise ValueError("fa_kvcache_append: block_table must be int32 [B, max_blocks], cache_seqlens int32 [B]")
     if not (k_new.dtype == v_new.dtype == k_cache.dtype == v_cache.dtype):
         raise ValueError("fa_kvcache_append: k/v and caches must share one dtype")
+    _on_device("fa_kvcache_append", (k_new, v_new, k_cache, v_cache, block_table, cache_seqlens))
     code = _lib_handle().fa_kvcache_append(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
                                            _ptr(block_table), _ptr(cache_seqlens), B, n_new, H_kv, d, num_pages,
                                            page_size, max_blocks, _dtype_code(k_new), _stream(stream))
@@ -458,10 +502,13 @@ def fa_fwd_kvcache_noalloc(q, k_cache, v_cache, block_table, cache_seqlens, out,
     if one != 1 or tuple(k_cache.shape) != (num_pages, page_size, H, d) or \
             tuple(v_cache.shape) != tuple(k_cache.shape) or tuple(out.shape) != tuple(q.shape):
         raise ValueError("fa_fwd_kvcache_noalloc: shape mismatch")
-    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32 or block_table.shape[0] != B:
-        raise ValueError("fa_fwd_kvcache_noalloc: block_table / cache_seqlens must be int32 [B, ...]")
+    if block_table.dtype != torch.int32 or cache_seqlens.dtype != torch.int32 or block_table.shape[0] != B or \
+            tuple(cache_seqlens.shape) != (B,) or block_table.dim() != 2:
+        raise ValueError("fa_fwd_kvcache_noalloc: block_table must be int32 [B, max_blocks], cache_seqlens int32 [B]")
     if tuple(lse.shape) != (B, H, 1) or lse.dtype != torch.float32:
         raise ValueError("fa_fwd_kvcache_noalloc: lse must be fp32 [B, H, 1]")
+    _on_device("fa_fwd_kvcache_noalloc", (q, k_cache, v_cache, block_table, cache_seqlens, out, lse),
+               alibi_slopes, H)
     code = _lib_handle().fa_fwd_kvcache_noalloc(
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(cache_seqlens), _ptr(out), _ptr(lse),
         B, H, d, num_pages, page_size, max_blocks, _dtype_code(q), float(scale), int(window_left),

@@ -133,6 +133,34 @@ int auto_splits(int B, int H, long long max_len) {
   return static_cast<int>(s);
 }
 
+// Split count a decode launch uses. An explicit num_splits is used as
+// given. The automatic count is auto_splits; a grouped-query cache on the
+// tensor-core kernel (one CTA serves G query heads and streams their cache
+// head once) aims instead at the CTAs launched: about 2048 * G keys a split
+// and enough CTAs to fill the GPU, never above the one-head count, so a
+// workspace sized by fa_kvcache_workspace_size always holds the partials.
+// Returns -1 for invalid sizes.
+int launch_splits(int B, int H, int H_kv, int d, int max_blocks, int page_size, int num_splits) {
+  const int S = fa_kvcache_num_splits(B, H, d, max_blocks, page_size, num_splits);
+  if (S < 0 || H_kv < 1 || H_kv > H || H % H_kv != 0) return -1;
+  if (num_splits != 0 || S <= 1 || page_size % 64 != 0 || !fa::decode_on_tensor_cores(H, H_kv)) return S;
+  const long long G = fa::decode_group_heads(H, H_kv);
+  const long long max_len = static_cast<long long>(max_blocks) * page_size;
+  const long long units = static_cast<long long>(B) * (H / G);
+  long long s = ((max_len + 2047) / 2048 + G - 1) / G;
+  s = std::max(s, std::min((4LL * kNumSms + units - 1) / units, (max_len + 255) / 256));
+  return static_cast<int>(std::max(1LL, std::min(s, static_cast<long long>(S))));
+}
+
+// Workspace bytes of S split partials: O_part [S, B, H, d] fp32, padded to
+// 256 bytes, then LSE_part [S, B, H] fp32.
+size_t partial_bytes(int S, int B, int H, int d) {
+  if (S <= 1) return 0;
+  const size_t rows = static_cast<size_t>(S) * B * H;
+  const size_t o_bytes = (rows * d * sizeof(float) + 255) & ~size_t(255);
+  return o_bytes + rows * sizeof(float);
+}
+
 bool kvcache_sizes_ok(int B, int H, int d, int max_blocks, int page_size) {
   if (B < 0 || H < 1 || max_blocks < 1 || page_size < 1) return false;
   if (d != 64 && d != 128) return false;
@@ -331,21 +359,10 @@ fa_status kvcache_common(const void* q, const void* k_cache, const void* v_cache
   if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return FA_ERR_ARG;
-  int S = fa_kvcache_num_splits(B, H, d, max_blocks, page_size, num_splits);
-  const size_t need = fa_kvcache_workspace_size(B, H, d, max_blocks, page_size, num_splits);
-  if (S > 1 && (!workspace || !aligned16(workspace) || workspace_bytes < need)) return FA_ERR_WORKSPACE;
-  if (num_splits == 0 && S > 1 && page_size % 64 == 0 && fa::decode_on_tensor_cores(H, H_kv)) {
-    // a grouped-query CTA serves G query heads and streams their cache head
-    // once: aim the automatic count at the CTAs launched (about 2048 * G keys
-    // a split, enough CTAs to fill the GPU), never above S, so the workspace
-    // sized for S still holds the partials
-    const long long G = fa::decode_group_heads(H, H_kv);
-    const long long max_len = static_cast<long long>(max_blocks) * page_size;
-    const long long units = static_cast<long long>(B) * (H / G);
-    long long s = ((max_len + 2047) / 2048 + G - 1) / G;
-    s = std::max(s, std::min((4LL * kNumSms + units - 1) / units, (max_len + 255) / 256));
-    S = static_cast<int>(std::max(1LL, std::min(s, static_cast<long long>(S))));
-  }
+  const int S = launch_splits(B, H, H_kv, d, max_blocks, page_size, num_splits);
+  if (S < 1) return FA_ERR_SHAPE;
+  if (S > 1 && (!workspace || !aligned16(workspace) || workspace_bytes < partial_bytes(S, B, H, d)))
+    return FA_ERR_WORKSPACE;
   fa_status st = check_device();
   if (st != FA_OK) return st;
 
@@ -359,9 +376,9 @@ fa_status kvcache_common(const void* q, const void* k_cache, const void* v_cache
   p.lse = lse;
   if (S > 1) {
     const size_t rows = static_cast<size_t>(S) * B * H;
-    size_t o_bytes = (rows * d * sizeof(float) + 255) & ~size_t(255);
     p.o_part = static_cast<float*>(workspace);
-    p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + o_bytes);
+    p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + partial_bytes(S, B, H, d) -
+                                          rows * sizeof(float));
   }
   p.slopes = alibi_slopes;
   p.B = B;
@@ -463,13 +480,13 @@ int fa_kvcache_num_splits(int B, int H, int d, int max_blocks, int page_size, in
   return auto_splits(B, H, static_cast<long long>(max_blocks) * page_size);
 }
 
+int fa_kvcache_num_splits_gqa(int B, int H, int H_kv, int d, int max_blocks, int page_size, int num_splits) {
+  return launch_splits(B, H, H_kv, d, max_blocks, page_size, num_splits);
+}
+
 size_t fa_kvcache_workspace_size(int B, int H, int d, int max_blocks, int page_size, int num_splits) {
   const int s = fa_kvcache_num_splits(B, H, d, max_blocks, page_size, num_splits);
-  if (s <= 1) return 0;
-  const size_t rows = static_cast<size_t>(s) * B * H;
-  size_t o_bytes = rows * d * sizeof(float);
-  o_bytes = (o_bytes + 255) & ~size_t(255);
-  return o_bytes + rows * sizeof(float);
+  return s > 1 ? partial_bytes(s, B, H, d) : 0;
 }
 
 fa_status fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, const int* block_table,

@@ -449,7 +449,8 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
   const float nan = __int_as_float(0x7fc00000);
 
   float m = -INFINITY;  // running max of the whole row (log2 units)
-  float lsum = 0.0f;    // this part's running sum of exp2(t - m)
+  float lsum = 0.0f;    // this part's running sum of exp2(t - m) (for LSE)
+  float qsum = 0.0f;    // the same sum of P as rounded for the PV product (for O)
   bool ok = alive;      // after a failure in an earlier job, only fill
   bool broke = false;   // left the loop at a shared exchange (all parts do)
   const int n = jb.has ? l - f + 1 : 0;
@@ -532,12 +533,17 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
       rescale = true;
     }
     lsum *= alpha;
+    qsum *= alpha;
     const float m_eff = (m == -INFINITY) ? 0.0f : m;
     // pass 2: P = exp2(t - m) into this part's kKeys / 2 columns of the P
     // buffer; pairs of elements go through packed fp32x2 FMA (scale,
-    // subtract max) and add
+    // subtract max) and add. O is normalised by the sum of P exactly as the
+    // PV product sees it (the 16-bit values), so rounding P to 16 bits
+    // perturbs the weights of a convex combination of V rows rather than its
+    // total; LSE takes the sum of the unrounded values.
     const uint64_t m2 = f2_pack(-m_eff, -m_eff);
     uint64_t rsum2[4] = {0, 0, 0, 0};  // independent packed partial sums (0 bits = +0.0f)
+    uint64_t qsum2[2] = {0, 0};        // the same, of the 16-bit P
     auto pass2 = [&](auto emu_tag) {
       constexpr bool kMaskedTile = decltype(emu_tag)::value;
 #pragma unroll
@@ -567,6 +573,7 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
           }
           rsum2[e & 3] = f2_add(rsum2[e & 3], f2_pack(p0, p1));
           pk[e] = pack2<T>(p0, p1);
+          qsum2[e & 1] = f2_add(qsum2[e & 1], widen2<T>(pk[e]));
         }
         tmem_st16(tmem + lane_sel + kTmemP + (gi & 1) * 64 + part * (kKeys / 2) + 16 * c, pk);
       }
@@ -575,10 +582,12 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
       pass2(std::true_type{});
     else
       pass2(std::false_type{});
-    float r0, r1, r2, r3;
+    float r0, r1, r2, r3, u0, u1;
     f2_unpack(f2_add(rsum2[0], rsum2[1]), r0, r1);
     f2_unpack(f2_add(rsum2[2], rsum2[3]), r2, r3);
+    f2_unpack(f2_add(qsum2[0], qsum2[1]), u0, u1);
     const float rs = (r0 + r1) + (r2 + r3);
+    qsum += u0 + u1;
     if (__any_sync(0xffffffffu, rescale)) {
       // O must be idle: wait for the product of the previous tile (the only
       // one that can still be running).
@@ -616,21 +625,26 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
   }
-  // all parts of a row must agree on success; combine the row sums
-  float ltot = lsum;
+  // all parts of a row must agree on success; combine the row sums (two
+  // exchanges, made by all parts alike)
+  float ltot = lsum, qtot = qsum;
   if (n_done >= 0 && alive) {
     float all[kParts];
     part_exchange(bars->xchg, xk++, part, r, quarter, ok ? lsum : nan, all);
     ltot = 0.0f;
 #pragma unroll
     for (int i = 0; i < kParts; ++i) ltot += all[i];  // NaN if any part failed
-    ok = ok && ltot == ltot;
-    if (!ok) ltot = 0.0f;
+    part_exchange(bars->xchg, xk++, part, r, quarter, ok ? qsum : nan, all);
+    qtot = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kParts; ++i) qtot += all[i];
+    ok = ok && ltot == ltot && qtot == qtot;
+    if (!ok) ltot = qtot = 0.0f;
   }
 
   // epilogue: O / l -> dtype for this part's columns, LSE = (m + log2 l) ln 2
   T* orow = reinterpret_cast<T*>(p.out) + ((jb.obase + (row_ok ? q : 0)) * p.H + h) * D + part * kOCols;
-  const float inv = ltot > 0.0f ? 1.0f / ltot : 0.0f;
+  const float inv = qtot > 0.0f ? 1.0f / qtot : 0.0f;
   if (ok && n > 0) {
 #pragma unroll
     for (int cc = 0; cc < kOCols / kOC; ++cc) {

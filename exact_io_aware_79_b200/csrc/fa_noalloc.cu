@@ -14,6 +14,8 @@
 // In host code its name is only a host-side stand-in, so the device address
 // is looked up with cudaGetSymbolAddress once per device (on the first call
 // made with that device current) and that address is what the kernels get.
+// Only a successful lookup is kept: after a failed one (say, made during a
+// stream capture) the next call on that device looks the address up again.
 #include "fa.h"
 #include "fa_internal.h"
 
@@ -27,9 +29,8 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_split_scratch[kScratchBytes];
 
-std::once_flag g_setup_once[kMaxDevices];
-void* g_scratch_addr[kMaxDevices];
-cudaError_t g_setup_status[kMaxDevices];
+std::mutex g_setup_mutex;
+void* g_scratch_addr[kMaxDevices];  // set once a lookup on the device succeeded
 
 // Device address of g_split_scratch on the current device.
 fa_status scratch_for_current_device(void** addr) {
@@ -39,12 +40,16 @@ fa_status scratch_for_current_device(void** addr) {
     return FA_ERR_DEVICE;
   }
   if (dev >= kMaxDevices) return FA_ERR_DEVICE;
-  std::call_once(g_setup_once[dev], [dev]() {
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
     void* p = nullptr;
-    g_setup_status[dev] = cudaGetSymbolAddress(&p, g_split_scratch);
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_split_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      cudaGetLastError();  // clear the (non-sticky) error so a later call starts clean
+      return FA_ERR_CUDA;
+    }
     g_scratch_addr[dev] = p;
-  });
-  if (g_setup_status[dev] != cudaSuccess || g_scratch_addr[dev] == nullptr) return FA_ERR_CUDA;
+  }
   *addr = g_scratch_addr[dev];
   return FA_OK;
 }

@@ -253,6 +253,20 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Warpgroup-collective register reallocation: the four warps of a warpgroup
+// raise (inc) or lower (dec) their per-thread register count to N. A block
+// keeps the registers it was launched with; inc waits until other
+// warpgroups' dec have returned enough of them.
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------ descriptors
 
 // Shared-memory matrix descriptor for tcgen05.mma (sm_100 format): start
@@ -386,6 +400,24 @@ template <>
 __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// The two 16-bit values of a pack2 result, widened exactly to an fp32 pair
+// (f2_pack order: low half first). For bf16 the widening is a shift and a
+// mask of the bit pattern.
+template <typename T>
+__device__ __forceinline__ uint64_t widen2(uint32_t u);
+
+template <>
+__device__ __forceinline__ uint64_t widen2<__nv_bfloat16>(uint32_t u) {
+  return f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
+template <>
+__device__ __forceinline__ uint64_t widen2<__half>(uint32_t u) {
+  __half2 v = *reinterpret_cast<__half2*>(&u);
+  const float2 f = __half22float2(v);
+  return f2_pack(f.x, f.y);
 }
 
 template <typename T>

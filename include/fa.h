@@ -370,6 +370,17 @@ fa_status fa_bwd_varlen_qkvpacked(const void *qkv, const void *out, const float 
 int fa_kvcache_num_splits(int B, int H, int d, int max_blocks, int page_size, int num_splits);
 
 /*
+ * Number of splits fa_fwd_kvcache_gqa launches with H_kv cache heads: the
+ * same as fa_kvcache_num_splits for an explicit num_splits or H_kv == H;
+ * with grouped heads on 64-multiple pages and num_splits = 0 the automatic
+ * count is aimed at the CTAs the grouped kernel launches (one per group of
+ * query heads), never above fa_kvcache_num_splits(B, H, ...), so the
+ * workspace fa_kvcache_workspace_size reports always suffices. Returns -1
+ * for invalid sizes.
+ */
+int fa_kvcache_num_splits_gqa(int B, int H, int H_kv, int d, int max_blocks, int page_size, int num_splits);
+
+/*
  * Bytes of workspace fa_fwd_kvcache needs for these sizes (0 when a single
  * split is used). Returns 0 for invalid sizes as well; fa_fwd_kvcache then
  * reports the invalid argument.
@@ -399,7 +410,9 @@ size_t fa_kvcache_workspace_size(int B, int H, int d, int max_blocks, int page_s
  *     smaller explicit num_splits or use fa_fwd_kvcache.
  *   - The first call on a device that needs the array (more than one split)
  *     looks up the array's device address for that device, with that device
- *     current; make that first call before any stream capture.
+ *     current; make that first call before any stream capture. A failed
+ *     lookup returns FA_ERR_CUDA and is not remembered: the next call on that
+ *     device tries again.
  *   - All calls on a device share the one array and it keeps the last call's
  *     partials. Each call overwrites every partial it reads, so nothing needs
  *     clearing, but calls whose kernels overlap on the GPU (different streams

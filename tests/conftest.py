@@ -24,3 +24,17 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Prints the achieved maximum errors of every parity check that ran."""
+    from tests import parity
+    if not parity.RECORD:
+        return
+    tr = terminalreporter
+    tr.section("parity: achieved max errors (O max-abs, worst error / bound, LSE max-abs)")
+    worst = max(r[2] for r in parity.RECORD)
+    for what, o_err, ratio, l_err in parity.RECORD:
+        tr.write_line("%-90.90s  O %.3e  %.3f  LSE %.3e" % (what, o_err, ratio, l_err))
+    tr.write_line("%d checks; largest O error / bound %.3f; largest LSE error %.3e" % (
+        len(parity.RECORD), worst, max(r[3] for r in parity.RECORD)))

@@ -166,6 +166,23 @@ def test_split_count_resolution(lib):
         assert 1 <= ns(*args, 0) <= 64
 
 
+def test_grouped_query_split_count(lib):
+    """The grouped-query query reports the count the grouped kernel launches:
+    aimed at its CTAs (one per group of query heads), never above the
+    one-head count; explicit counts, one-head caches and pages that are not
+    multiples of 64 (no grouped kernel) keep the one-head answer."""
+    ng, ns = lib.fa_kvcache_num_splits_gqa, lib.fa_kvcache_num_splits
+    assert ns(64, 32, 128, 128, 256, 0) == 16
+    assert ng(64, 32, 8, 128, 128, 256, 0) == 4     # groups of 4: 4 * 2048 keys a split
+    assert ng(64, 32, 32, 128, 128, 256, 0) == 16   # H_kv == H: the one-head count
+    assert ng(64, 32, 8, 128, 128, 256, 7) == 7     # explicit
+    assert ng(64, 32, 8, 128, 2048, 16, 0) == ns(64, 32, 128, 2048, 16, 0)  # 16-token pages
+    assert ng(64, 32, 5, 128, 128, 256, 0) == -1    # H not a multiple of H_kv
+    for B, H, Hk, mb, page in [(1, 32, 8, 128, 256), (3, 16, 1, 40, 64), (64, 32, 4, 128, 256)]:
+        s = ng(B, H, Hk, 128, mb, page, 0)
+        assert 1 <= s <= ns(B, H, 128, mb, page, 0)
+
+
 def test_workspace_size(lib):
     ws = lib.fa_kvcache_workspace_size
     assert ws(64, 32, 128, 128, 256, 1) == 0

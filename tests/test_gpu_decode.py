@@ -1,6 +1,6 @@
 """GPU parity of fa_fwd_kvcache (through the C ABI) against the fp64 oracle.
 
-Same tolerances as the forward (O bound times the input scale sigma). Block-table indexing is checked bit-exactly
+Same tolerances as the forward (tests/parity.py). Block-table indexing is checked bit-exactly
 with one-hot probes whose expected output is an integer code of the probed
 token's logical index.
 """
@@ -13,11 +13,9 @@ import torch
 import oracle
 import exact_io_aware_79_b200 as fa
 from exact_io_aware_79_b200 import workloads as W
+from tests import parity
 
 pytestmark = pytest.mark.gpu
-
-O_TOL = {torch.bfloat16: 1.6e-2, torch.float16: 4e-3}
-LSE_TOL = 1e-3
 
 
 def case_inputs(B, H, d, page, max_blocks, lens, dtype, seed, sigma=1.0):
@@ -37,14 +35,8 @@ def run_gpu(q, kc, vc, table, lens, scale, wl=-1, slopes=None, cap=0.0, splits=0
     return out.float().cpu().numpy(), lse.cpu().numpy()
 
 
-def compare(out, lse, o_ref, l_ref, dtype, what, sigma=1.0):
-    fin = np.isfinite(l_ref)
-    assert np.array_equal(np.isfinite(lse), fin), what
-    assert np.all(lse[~fin] == -np.inf), what
-    o_err = float(np.abs(out - o_ref).max())
-    l_err = float(np.abs(lse[fin] - l_ref[fin]).max()) if fin.any() else 0.0
-    assert o_err <= O_TOL[dtype] * sigma, "%s: O error %.3g" % (what, o_err)
-    assert l_err <= LSE_TOL, "%s: LSE error %.3g" % (what, l_err)
+def compare(out, lse, o_ref, l_ref, dtype, what):
+    return parity.check(out, lse, o_ref, l_ref, dtype, "decode " + what)
 
 
 CASES = [
@@ -70,7 +62,7 @@ def test_decode_matches_oracle(case, splits):
     scale = 1.0 / math.sqrt(d)
     out, lse = run_gpu(q, kc, vc, table, lens_t, scale, wl, slopes, cap, splits)
     o_ref, l_ref = oracle.attn_decode_paged(q, kc, vc, table, lens_t, scale, wl, slopes, cap)
-    compare(out, lse, o_ref, l_ref, dtype, "%s splits=%d" % (case, splits), sigma)
+    compare(out, lse, o_ref, l_ref, dtype, "%s splits=%d" % (case, splits))
 
 
 def test_identity_table_equals_contiguous_forward():
@@ -87,8 +79,8 @@ def test_identity_table_equals_contiguous_forward():
     for b in range(B):
         L = int(lens[b])
         o2, l2 = fa.attention(q[b:b + 1].cuda(), k[b:b + 1, :L].cuda(), v[b:b + 1, :L].cuda(), 0.1, causal=True)
-        assert np.abs(out[b] - o2[0].float().cpu().numpy()).max() <= 1.6e-2
-        assert np.abs(lse[b] - l2[0].cpu().numpy()).max() <= 1e-3
+        assert np.abs(out[b] - o2[0].float().cpu().numpy()).max() <= parity.O_SPEC[torch.bfloat16]
+        assert np.abs(lse[b] - l2[0].cpu().numpy()).max() <= parity.LSE_SPEC
 
 
 @pytest.mark.parametrize("splits", [1, 16])

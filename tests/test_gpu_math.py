@@ -1,0 +1,71 @@
+"""The hand-written math inside the attention kernels, on its own.
+
+ex2_poly_x2 (2^x on the FMA pipe: a cubic for 2^f on |f| <= 1/2, the
+integer part added to the exponent field) and tanh_via_exp2 (the softcap's
+tanh) are evaluated by test-only kernels (tests/kernels/math_check.cu,
+compiled here with nvcc) on dense input sweeps, against fp64 exp2 / tanh
+evaluated on the device, and the worst errors are asserted against the
+bounds their comments state:
+  * 2^f relative error <= 7.5e-5 for every fp32 f with |f| <= 1/2;
+  * the same over the whole range -126 < x <= 127 (steps of 2^-10), and for
+    x <= -126 (and x = -inf) a result in [0, 2^-125], never NaN or inf;
+  * tanh absolute error <= 2.5e-7 on +-10^[-8, 3] (log-spaced) and at 0.
+"""
+import ctypes
+import os
+import subprocess
+
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(ROOT, "exact_io_aware_79_b200", "csrc")
+
+
+@pytest.fixture(scope="module")
+def lib(tmp_path_factory):
+    out = str(tmp_path_factory.mktemp("mathcheck") / "libmathcheck.so")
+    subprocess.run([os.environ.get("NVCC", "nvcc"), "-gencode", "arch=compute_100a,code=sm_100a", "-O3",
+                    "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "-I", CSRC, "-o", out,
+                    os.path.join(HERE, "kernels", "math_check.cu")], check=True)
+    L = ctypes.CDLL(out)
+    vp, d, i = ctypes.c_void_p, ctypes.c_double, ctypes.c_int
+    L.check_ex2_poly_reduced.argtypes = [vp, vp]
+    L.check_ex2_poly_range.argtypes = [vp, d, d, i, vp]
+    L.check_tanh.argtypes = [vp, d, d, i, vp]
+    return L
+
+
+def _run(fn, *args):
+    worst = torch.zeros(4, dtype=torch.float32, device="cuda")
+    s = torch.cuda.current_stream()
+    assert fn(ctypes.c_void_p(worst.data_ptr()), *args, ctypes.c_void_p(s.cuda_stream)) == 0
+    torch.cuda.synchronize()
+    return worst.cpu().tolist()
+
+
+def test_ex2_poly_every_reduced_argument(lib):
+    w = _run(lib.check_ex2_poly_reduced)
+    print("ex2_poly_x2: max relative error on |f| <= 1/2: %.3e" % w[0])
+    assert 0.0 < w[0] <= 7.5e-5
+
+
+def test_ex2_poly_whole_range_and_underflow(lib):
+    lo, step = -140.0, 2.0 ** -10
+    n = int((127.0 - lo) / step) + 1
+    w = _run(lib.check_ex2_poly_range, ctypes.c_double(lo), ctypes.c_double(step), n)
+    print("ex2_poly_x2: max relative error on (-126, 127]: %.3e; largest result below -126: %.3e" % (w[0], w[1]))
+    assert w[2] == 0.0, "NaN, negative or infinite result"
+    assert w[0] <= 7.5e-5 * (1 + 1e-3)
+    assert w[1] <= 2.0 ** -125
+
+
+def test_tanh_via_exp2_absolute_error(lib):
+    n = 200000
+    w = _run(lib.check_tanh, ctypes.c_double(-8.0), ctypes.c_double(11.0 / n), n)
+    print("tanh_via_exp2: max absolute error: %.3e" % w[0])
+    assert w[1] == 0.0, "NaN result"
+    assert w[0] <= 2.5e-7

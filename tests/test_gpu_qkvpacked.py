@@ -1,6 +1,5 @@
 """GPU parity of the packed-QKV entry points (through the C ABI) against the
-fp64 oracle, with the fa_fwd tolerances (O: 1.6e-2 bf16 / 4e-3 fp16 times
-the input scale; LSE: 1e-3; empty rows exactly O = 0, LSE = -inf)."""
+fp64 oracle, with the fa_fwd tolerances (tests/parity.py)."""
 import math
 
 import numpy as np
@@ -10,21 +9,13 @@ import torch
 import oracle
 import exact_io_aware_79_b200 as fa
 from exact_io_aware_79_b200 import workloads as W
+from tests import parity
 
 pytestmark = pytest.mark.gpu
 
-O_TOL = {torch.bfloat16: 1.6e-2, torch.float16: 4e-3}
-LSE_TOL = 1e-3
 
-
-def compare(out, lse, o_ref, l_ref, dtype, what, sigma=1.0):
-    fin = np.isfinite(l_ref)
-    assert np.array_equal(np.isfinite(lse), fin), what
-    assert np.all(lse[~fin] == -np.inf), what
-    o_err = float(np.abs(out - o_ref).max())
-    l_err = float(np.abs(lse[fin] - l_ref[fin]).max()) if fin.any() else 0.0
-    assert o_err <= O_TOL[dtype] * sigma, "%s: O error %.3g" % (what, o_err)
-    assert l_err <= LSE_TOL, "%s: LSE error %.3g" % (what, l_err)
+def compare(out, lse, o_ref, l_ref, dtype, what):
+    return parity.check(out, lse, o_ref, l_ref, dtype, "qkvpacked " + what)
 
 
 CASES = [
@@ -47,7 +38,7 @@ def test_qkvpacked_matches_oracle(case):
     fa.fa_fwd_qkvpacked(qkv.cuda(), out, lse, scale, causal, wl, wr, None if slopes is None else slopes.cuda(), cap)
     torch.cuda.synchronize()
     o_ref, l_ref = oracle.attn_fwd_qkvpacked(qkv, scale, causal, wl, wr, slopes, cap)
-    compare(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, dtype, str(case), sigma)
+    compare(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, dtype, str(case))
 
 
 def test_varlen_qkvpacked_matches_oracle():
