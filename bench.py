@@ -54,16 +54,18 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # d=128, pages of 256) read 1.003 x its K/V bytes and wrote 2.8 MB of
 # partials; reads scale with the K/V bytes, each byte being read once.
 DECODE_READ_PER_KV_BYTE = 967959936.0 / 965165056.0  # (968,019,712 + 967,900,160) / 2 / K/V bytes
-# Forward: per-launch DRAM bytes of captures of the forward kernel on the
-# named workload, for the kernel version they were taken on; None where no
-# capture of the present kernel exists.
-FWD_TRAFFIC = {
-    W.WINDOW_16K.name: 201647104.0 + 45596672.0,
-    W.CAUSAL_2K.name: (201453056.0 + 38760448.0 + 201453312.0 + 35730432.0) / 2.0,
-}
+# Forward: per-launch DRAM bytes of ncu captures of the forward kernel as it
+# stands, on the named workload; a workload without such a capture reports
+# None.
+FWD_TRAFFIC = {}
 # Forward workloads timed one by one after the step (L2 flushed between launches).
 FWD_CONFIGS = [W.CAUSAL_2K, W.WINDOW_16K, W.WINDOW_Q4K_K16K, W.CAUSAL_Q4K_K16K, W.ALIBI_SOFTCAP]
 HEADLINE_FWD = W.WINDOW_16K
+# The 8-bit forward, timed the same way on these workloads' shapes (E4M3
+# inputs with per-tensor descales); its roofline is the fp8 tensor peak,
+# taken as twice the measured bf16 burst (the nominal dense fp8 / bf16 ratio).
+FP8_CONFIGS = [W.WINDOW_16K]
+FP8_OVER_BF16 = 2.0
 
 
 # ---------------------------------------------------------------- algorithmic work
@@ -504,9 +506,38 @@ def time_fwd_configs(fa, dev, world, peaks, args, gpu_index):
                        "frac": round(tf / world / peaks["bf16_tflops"], 4), "flops_per_launch": fwd_flops(w),
                        "launches": n}
         del x, out, lse
+    for w in FP8_CONFIGS:
+        x = W.make_fwd_inputs_fp8(w, device=dev)
+        out = torch.empty(x["q"].shape, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(fa.fa_fwd_fp8_workspace_size(w.B, w.H, w.Nk, w.d), 16), dtype=torch.uint8, device=dev)
+        run = lambda: fa.fa_fwd_fp8(x["q"], x["k"], x["v"], out, lse, w.scale, x["descale_q"], x["descale_k"],
+                                    x["descale_v"], w.causal, w.window_left, w.window_right, x["slopes"], w.softcap,
+                                    ws)
+        for _ in range(max(3, args.warmup)):
+            run()
+        times = []
+        n = max(5, min(args.steps, args.config_steps))
+        barrier(world)
+        for _ in range(n):
+            flush.zero_()
+            a, b = ev(), ev()
+            a.record()
+            run()
+            b.record()
+            times.append((a, b))
+        torch.cuda.synchronize()
+        ms = max_over_ranks(statistics.median([a.elapsed_time(b) for a, b in times]), world, dev)
+        tf = weak_scaling_value(fwd_flops(w), ms * 1e-3, world) / 1e12
+        res["fp8_e4m3_" + w.name] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                                     "frac": round(tf / world / (FP8_OVER_BF16 * peaks["bf16_tflops"]), 4),
+                                     "frac_of_bf16_burst": round(tf / world / peaks["bf16_tflops"], 4),
+                                     "flops_per_launch": fwd_flops(w), "launches": n,
+                                     "note": "includes the V transpose pre-pass"}
+        del x, out, lse, ws
     t1 = time.time()
     sampler.stop()
-    res["peak"] = "measured burst bf16 %.1f TFLOP/s" % peaks["bf16_tflops"]
+    res["peak"] = "measured burst bf16 %.1f TFLOP/s (fp8: %.0f x that)" % (peaks["bf16_tflops"], FP8_OVER_BF16)
     res["clocks"] = sampler.summary(t0, t1)
     del flush
     return res
@@ -598,6 +629,35 @@ def sweep(args):
                           "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
                           "flops": fwd_flops(w), "peak_source": peak_src, "l2": "flushed"}), flush=True)
         del x, out, lse
+    # 8-bit forward of a forward workload: "fp8_" + its name (E4M3)
+    for w in W.FWD_WORKLOADS:
+        if "fp8_" + w.name not in names or w.d != 128:
+            continue
+        x = W.make_fwd_inputs_fp8(w, device=dev)
+        out = torch.empty(x["q"].shape, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(fa.fa_fwd_fp8_workspace_size(w.B, w.H, w.Nk, w.d), 16), dtype=torch.uint8, device=dev)
+        run = lambda: fa.fa_fwd_fp8(x["q"], x["k"], x["v"], out, lse, w.scale, x["descale_q"], x["descale_k"],
+                                    x["descale_v"], w.causal, w.window_left, w.window_right, x["slopes"], w.softcap,
+                                    ws)
+        for _ in range(args.warmup):
+            run()
+        times = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = ev(), ev()
+            a.record()
+            run()
+            b.record()
+            times.append((a, b))
+        torch.cuda.synchronize()
+        ms = statistics.median([a.elapsed_time(b) for a, b in times])
+        tf = fwd_flops(w) / (ms * 1e-3) / 1e12
+        print(json.dumps({"workload": "fp8_" + w.name, "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                          "frac_fp8_peak": round(tf / (FP8_OVER_BF16 * peaks["bf16_tflops"]), 4),
+                          "frac_bf16_burst": round(tf / peaks["bf16_tflops"], 4),
+                          "flops": fwd_flops(w), "peak_source": peak_src, "l2": "flushed"}), flush=True)
+        del x, out, lse, ws
     # backward of a forward workload: "bwd_" + its name ("bwd_det_" + its name
     # for the deterministic mode); credited 2.5x the forward's flops (five
     # products of the forward's size against two) in either mode

@@ -10,6 +10,9 @@ every call raises if the library cannot be loaded.
 Entry points with the C names:
     fa_fwd(q, k, v, out, lse, scale, causal, window_left, window_right,
            alibi_slopes, softcap)
+    fa_fwd_fp8(q8, k8, v8, out, lse, scale, descale_q, descale_k, descale_v,
+               causal, window_left, window_right, alibi_slopes, softcap,
+               workspace)
     fa_fwd_kvcache(q, k_cache, v_cache, block_table, cache_seqlens, out, lse,
                    scale, window_left, alibi_slopes, softcap, num_splits,
                    workspace)
@@ -29,6 +32,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libfa_b200.so")
 
 FA_FP16, FA_BF16 = 0, 1
+FA_E4M3, FA_E5M2 = 0, 1
 FA_MAX_SPLITS = 64
 FA_NOALLOC_SCRATCH_BYTES = 32 << 20
 STATUS = {
@@ -58,6 +62,10 @@ def _lib_handle():
         L.fa_fwd.restype = i
         L.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i, vp, f, vp]
         L.fa_fwd_gqa.restype = i
+        L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, f, f, f, i, i, i, vp, f, vp, sz, vp]
+        L.fa_fwd_fp8.restype = i
+        L.fa_fwd_fp8_workspace_size.argtypes = [i, i, i, i]
+        L.fa_fwd_fp8_workspace_size.restype = sz
         L.fa_fwd_kvcache_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, vp, f, i, vp,
                                          sz, vp]
         L.fa_fwd_kvcache_gqa.restype = i
@@ -193,6 +201,60 @@ def fa_fwd_gqa(q, k, v, out, lse, scale: float, causal: bool = False, window_lef
                                     _dtype_code(q), float(scale), int(bool(causal)), int(window_left),
                                     int(window_right), _ptr(alibi_slopes), float(softcap), _stream(stream))
     _check(code, "fa_fwd_gqa")
+
+
+def _fp8_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float8_e4m3fn:
+        return FA_E4M3
+    if t.dtype == torch.float8_e5m2:
+        return FA_E5M2
+    return -1
+
+
+def fa_fwd_fp8_workspace_size(B: int, H_kv: int, Nk: int, d: int) -> int:
+    return int(_lib_handle().fa_fwd_fp8_workspace_size(B, H_kv, Nk, d))
+
+
+def fa_fwd_fp8(q, k, v, out, lse, scale: float, descale_q: float = 1.0, descale_k: float = 1.0,
+               descale_v: float = 1.0, causal: bool = False, window_left: int = -1, window_right: int = -1,
+               alibi_slopes=None, softcap: float = 0.0, workspace: Optional[torch.Tensor] = None,
+               stream=None) -> None:
+    """8-bit forward: q [B,Nq,H,d], k/v [B,Nk,H_kv,d] float8_e4m3fn or float8_e5m2 (one format);
+    out bf16 [B,Nq,H,d]; lse fp32 [B,H,Nq]; element x8 stands for x8 * descale_x; workspace a
+    byte tensor of fa_fwd_fp8_workspace_size bytes (allocated here when None)."""
+    B, Nq, H, d = q.shape
+    Nk, H_kv = k.shape[1], k.shape[2]
+    for t in (q, k, v, out, lse):
+        if not t.is_contiguous():
+            raise ValueError("fa_fwd_fp8 needs contiguous tensors")
+    if tuple(k.shape) != (B, Nk, H_kv, d) or tuple(v.shape) != tuple(k.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("fa_fwd_fp8: shape mismatch")
+    if out.dtype != torch.bfloat16 or tuple(lse.shape) != (B, H, Nq) or lse.dtype != torch.float32:
+        raise ValueError("fa_fwd_fp8: out must be bf16 [B, Nq, H, d], lse fp32 [B, H, Nq]")
+    if not (q.dtype == k.dtype == v.dtype) or _fp8_code(q) < 0:
+        raise ValueError("fa_fwd_fp8: q, k, v must share one 8-bit float type")
+    _on_device("fa_fwd_fp8", (q, k, v, out, lse), alibi_slopes, H, workspace=workspace)
+    if workspace is None:
+        workspace = torch.empty(max(fa_fwd_fp8_workspace_size(B, H_kv, Nk, d), 16), dtype=torch.uint8,
+                                device=q.device)
+    code = _lib_handle().fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, H_kv, Nq, Nk, d,
+                                    _fp8_code(q), float(scale), float(descale_q), float(descale_k),
+                                    float(descale_v), int(bool(causal)), int(window_left), int(window_right),
+                                    _ptr(alibi_slopes), float(softcap), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(code, "fa_fwd_fp8")
+
+
+def attention_fp8(q, k, v, scale: Optional[float] = None, descale_q: float = 1.0, descale_k: float = 1.0,
+                  descale_v: float = 1.0, causal: bool = False, window_left: int = -1, window_right: int = -1,
+                  alibi_slopes=None, softcap: float = 0.0):
+    """Allocating form of fa_fwd_fp8; returns (out bf16, lse)."""
+    B, Nq, H, d = q.shape
+    out = torch.empty((B, Nq, H, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    fa_fwd_fp8(q, k, v, out, lse, d ** -0.5 if scale is None else scale, descale_q, descale_k, descale_v, causal,
+               window_left, window_right, alibi_slopes, softcap)
+    return out, lse
 
 
 def fa_bwd_workspace_size(B: int, H: int, Nq: int, d: int) -> int:

@@ -103,6 +103,42 @@ bool make_cache_map(CUtensorMap* map, const void* base, bool bf16, int num_pages
 
 // fp32 [B, N, H, d] tensor as a 4-D map (d, H, N, B) with (32, 1, 64, 1)
 // boxes and 128-byte swizzle (the backward's dQ accumulator).
+// 8-bit [B, N, H, d] tensor (d = 128): a (128, 1, 128, 1) box of bytes, one
+// 128-byte swizzle row per token.
+bool make_map_u8(CUtensorMap* map, const void* base, int B, int N, int H, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t n = static_cast<cuuint64_t>(N > 0 ? N : 1);
+  const cuuint64_t t = static_cast<cuuint64_t>(H) * d;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), n, static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d), t, n * t};
+  cuuint32_t box[4] = {128, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Transposed 8-bit V [B, H_kv, d, Nk_pad]: a (128, 128, 1, 1) box (128 keys of
+// 128 rows of d), 128-byte swizzle.
+bool make_map_vt(CUtensorMap* map, void* base, int B, int H_kv, int d, int Nk_pad) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t np = static_cast<cuuint64_t>(Nk_pad);
+  cuuint64_t dims[4] = {np, static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H_kv), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {np, np * d, np * d * H_kv};
+  cuuint32_t box[4] = {128, 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Keys of the transposed 8-bit V rounded up to 16 (16-byte rows for TMA).
+long long fp8_keys_padded(int Nk) { return (static_cast<long long>(Nk) + 15) / 16 * 16; }
+
 bool make_map_f32(CUtensorMap* map, void* base, int B, int N, int H, int d) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
@@ -240,6 +276,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* out, flo
   p.scale_log2 = mag * fa::kLog2e;
   p.cap_scale = softcap > 0.0f ? mag / softcap : 0.0f;
   p.cap_log2 = softcap * fa::kLog2e;
+  p.out_scale = 1.0f;
   return fa::launch_fwd(bf16, d, tq, tk, tv, p, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -478,6 +515,74 @@ int fa_kvcache_num_splits(int B, int H, int d, int max_blocks, int page_size, in
   if (num_splits > 0) return num_splits;
   if (B == 0) return 1;
   return auto_splits(B, H, static_cast<long long>(max_blocks) * page_size);
+}
+
+size_t fa_fwd_fp8_workspace_size(int B, int H_kv, int Nk, int d) {
+  if (B < 0 || H_kv < 1 || Nk < 0 || d != 128 || Nk > kMaxSeq) return 0;
+  return static_cast<size_t>(B) * H_kv * d * static_cast<size_t>(fp8_keys_padded(Nk));
+}
+
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int H_kv,
+                     int Nq, int Nk, int d, fa_fp8_format fmt, float scale, float descale_q, float descale_k,
+                     float descale_v, int causal, int window_left, int window_right, const float* alibi_slopes,
+                     float softcap, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || H < 0 || Nq < 0 || Nk < 0) return FA_ERR_SHAPE;
+  if (H > 0 && (H_kv < 1 || H_kv > H || H % H_kv != 0)) return FA_ERR_SHAPE;
+  if (Nq > kMaxSeq || Nk > kMaxSeq || static_cast<long long>(B) * H >= (1LL << 31)) return FA_ERR_SHAPE;
+  if (B > 65535 || H_kv > 65535) return FA_ERR_SHAPE;  // grid of the V transpose
+  if (fmt != FA_E4M3 && fmt != FA_E5M2) return FA_ERR_DTYPE;
+  if (d != 128) return FA_ERR_HEADDIM;
+  if (!finite(scale) || !finite(softcap) || softcap < 0.0f) return FA_ERR_ARG;
+  if (!finite(descale_q) || !finite(descale_k) || !finite(descale_v) || descale_q <= 0.0f || descale_k <= 0.0f ||
+      descale_v <= 0.0f)
+    return FA_ERR_ARG;
+  if (window_left < -1 || window_right < -1 || (causal != 0 && causal != 1)) return FA_ERR_ARG;
+  if (static_cast<long long>(B) * H * Nq == 0) return FA_OK;
+  if (!q || !out || !lse) return FA_ERR_NULL;
+  if (Nk > 0 && (!k || !v)) return FA_ERR_NULL;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k) || !aligned16(v) || !aligned16(lse)) return FA_ERR_ARG;
+  const int tiles = (Nq + 127) / 128;
+  if (static_cast<long long>(tiles) * B * H >= (1LL << 31)) return FA_ERR_SHAPE;
+  const size_t need = fa_fwd_fp8_workspace_size(B, H_kv, Nk, d);
+  if (need > 0 && (!workspace || !aligned16(workspace) || workspace_bytes < need)) return FA_ERR_WORKSPACE;
+  fa_status st = check_device();
+  if (st != FA_OK) return st;
+
+  const int Nk_pad = static_cast<int>(fp8_keys_padded(Nk));
+  CUtensorMap tq, tk, tvt;
+  // with no keys no K or V tile is ever loaded; q stands in as a valid base
+  const void* kb = Nk > 0 ? k : q;
+  void* vtb = Nk > 0 ? workspace : const_cast<void*>(q);
+  if (!make_map_u8(&tq, q, B, Nq, H, d) || !make_map_u8(&tk, kb, B, Nk, H_kv, d) ||
+      !make_map_vt(&tvt, vtb, B, H_kv, d, Nk > 0 ? Nk_pad : 16))
+    return FA_ERR_CUDA;
+  if (Nk > 0 && fa::launch_v_transpose(v, workspace, B, Nk, H_kv, Nk_pad, stream) != cudaSuccess) return FA_ERR_CUDA;
+
+  fa::FwdParams p{};
+  p.out = out;
+  p.lse = lse;
+  p.slopes = alibi_slopes;
+  p.B = B;
+  p.H = H;
+  p.H_kv = H_kv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.num_tiles = tiles;
+  p.causal = causal;
+  p.window_left = window_left;
+  p.window_right = window_right;
+  p.use_softcap = softcap > 0.0f;
+  // the scores of the 8-bit values are scaled by scale * descale_q *
+  // descale_k; O by descale_v
+  const float eff = scale * descale_q * descale_k;
+  if (!finite(eff)) return FA_ERR_ARG;
+  p.negate_scores = eff < 0.0f;
+  const float mag = std::fabs(eff);
+  p.scale_log2 = mag * fa::kLog2e;
+  p.cap_scale = softcap > 0.0f ? mag / softcap : 0.0f;
+  p.cap_log2 = softcap * fa::kLog2e;
+  p.out_scale = descale_v;
+  return fa::launch_fwd_fp8(fmt == FA_E5M2 ? 1 : 0, tq, tk, tvt, p, stream) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 int fa_kvcache_num_splits_gqa(int B, int H, int H_kv, int d, int max_blocks, int page_size, int num_splits) {

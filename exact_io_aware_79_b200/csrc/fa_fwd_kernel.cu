@@ -80,14 +80,50 @@ constexpr uint32_t kTmemP = 384;  // two 64-column P buffers
 
 constexpr int kBarrierBytes = 8192;  // barrier block and exchange slots
 
-template <int D>
+// Input element types: fp16 / bf16 (products of kind::f16, P rounded to the
+// input type, O written in it), or 8-bit floats (tags below: products of
+// kind::f8f6f4, P rounded to the same 8-bit format, O written as bf16).
+struct Fp8E4M3 {};
+struct Fp8E5M2 {};
+
+template <typename T>
+struct Elem {
+  using Out = T;
+  static constexpr int kBytes = 2;
+  static constexpr bool kFp8 = false;
+  static constexpr uint32_t kFmt = 0;
+};
+template <>
+struct Elem<Fp8E4M3> {
+  using Out = __nv_bfloat16;
+  static constexpr int kBytes = 1;
+  static constexpr bool kFp8 = true;
+  static constexpr uint32_t kFmt = 0;
+};
+template <>
+struct Elem<Fp8E5M2> {
+  using Out = __nv_bfloat16;
+  static constexpr int kBytes = 1;
+  static constexpr bool kFp8 = true;
+  static constexpr uint32_t kFmt = 1;
+};
+
+// Shared-memory tiles: 128 rows of d elements in 128-byte swizzle chunks
+// (64 elements of 16 bits or 128 of 8 bits each); a chunk of 128 rows is
+// 16 KB. 8-bit V arrives transposed (d rows of 128 keys), so that both
+// operands of the PV product are K-major as well.
+template <typename T, int D>
 struct Cfg {
-  static constexpr int kChunkBytes = BM * 128;       // 128 rows x 64 elements x 2 bytes
-  static constexpr int kTileBytes = BM * D * 2;      // one Q, K or V tile
+  static constexpr int kRowBytes = D * Elem<T>::kBytes;
+  static constexpr int kChunks = kRowBytes / 128;           // swizzle chunks per row
+  static constexpr int kChunkElems = 128 / Elem<T>::kBytes;  // elements per chunk row
+  static constexpr int kChunkBytes = BM * 128;               // one chunk of 128 rows
+  static constexpr int kTileBytes = BM * kRowBytes;          // one Q, K or V tile
+  static constexpr int kSteps = kRowBytes / 32;              // MMAs of an S product (32 bytes of d each)
   // two Q buffers, so the next job's Q lands while this one's runs
-  static constexpr int kQBufs = 2;                    // active job a uses buffer a % kQBufs
-  static constexpr int kSlotsK = (D == 128) ? 2 : 5;  // K ring depth
-  static constexpr int kSlotsV = (D == 128) ? 2 : 5;  // V ring depth
+  static constexpr int kQBufs = 2;                           // active job a uses buffer a % kQBufs
+  static constexpr int kSlotsK = (kTileBytes <= 16384) ? 5 : 2;  // K ring depth
+  static constexpr int kSlotsV = kSlotsK;                        // V ring depth
   static constexpr int kSlots = kSlotsK + kSlotsV;
   static constexpr int kSmemBytes = 1024 + (kQBufs + kSlots) * kTileBytes + kBarrierBytes;
 };
@@ -232,7 +268,7 @@ __device__ __forceinline__ void for_each_job(const FwdParams& p, Fn&& fn) {
 template <typename T, int D>
 __device__ void producer(const FwdParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                          uint8_t* sQ, uint8_t* sK, uint8_t* sV, Barriers* bars) {
-  using C = Cfg<D>;
+  using C = Cfg<T, D>;
   volatile int* abort = &bars->abort;
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
@@ -246,9 +282,14 @@ __device__ void producer(const FwdParams& p, const CUtensorMap* tmQ, const CUten
     const int slot = gi % depth;
     if (gi >= depth && !mbar_wait(&freed[(gi - depth) % kRing], ((gi - depth) / kRing) & 1, abort)) return false;
     mbar_arrive_expect_tx(&full[slot], C::kTileBytes);
+    if (Elem<T>::kFp8 && map == tmV) {
+      // transposed V: box of 128 keys (the inner coordinate) x d rows
+      tma_load_4d(map, &full[slot], ring + slot * C::kTileBytes, key_tile * BN, 0, jb.hk, jb.bcoord, pol_kv);
+      return true;
+    }
 #pragma unroll
-    for (int ch = 0; ch < D / 64; ++ch)
-      tma_load_4d(map, &full[slot], ring + slot * C::kTileBytes + ch * C::kChunkBytes, ch * 64, jb.hk,
+    for (int ch = 0; ch < C::kChunks; ++ch)
+      tma_load_4d(map, &full[slot], ring + slot * C::kTileBytes + ch * C::kChunkBytes, ch * C::kChunkElems, jb.hk,
                   jb.krow + key_tile * BN, jb.bcoord, pol_kv);
     return true;
   };
@@ -260,9 +301,9 @@ __device__ void producer(const FwdParams& p, const CUtensorMap* tmQ, const CUten
     if (a >= QB && !(ok = mbar_wait(&bars->q_empty[a % QB], ((a - QB) / QB) & 1, abort))) return;
     mbar_arrive_expect_tx(&bars->q_full[a % QB], C::kTileBytes);
 #pragma unroll
-    for (int ch = 0; ch < D / 64; ++ch)
-      tma_load_4d(tmQ, &bars->q_full[a % QB], sQ + (a % QB) * C::kTileBytes + ch * C::kChunkBytes, ch * 64, jb.h,
-                  jb.qrow + jb.q0, jb.bcoord, pol_q);
+    for (int ch = 0; ch < C::kChunks; ++ch)
+      tma_load_4d(tmQ, &bars->q_full[a % QB], sQ + (a % QB) * C::kTileBytes + ch * C::kChunkBytes,
+                  ch * C::kChunkElems, jb.h, jb.qrow + jb.q0, jb.bcoord, pol_q);
     auto load_k = [&](int u) {
       const bool r = load(tmK, sK, bars->k_full, bars->s_ready, C::kSlotsK, g + u, jb, jb.f + u);
       nk += r;
@@ -300,10 +341,12 @@ __device__ void producer(const FwdParams& p, const CUtensorMap* tmQ, const CUten
 // softmax that it may write P(g).
 template <typename T, int D>
 __device__ void qk_issuer(const FwdParams& p, uint8_t* sQ, uint8_t* sK, Barriers* bars, uint32_t tmem) {
-  using C = Cfg<D>;
+  using C = Cfg<T, D>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  constexpr bool kFp8 = Elem<T>::kFp8;
   // a negative softmax scale is applied as -Q K^T (A-negate bit) times |scale|
-  const uint32_t idesc = instr_desc_f16(kBf16, BM, BN, false) | (p.negate_scores ? (1u << 13) : 0u);
+  const uint32_t idesc = (kFp8 ? instr_desc_f8(Elem<T>::kFmt, BM, BN) : instr_desc_f16(kBf16, BM, BN, false)) |
+                         (p.negate_scores ? (1u << 13) : 0u);
   volatile int* abort = &bars->abort;
   const uint32_t sQaddr = smem_addr(sQ), sKaddr = smem_addr(sK);
   int g = 0, a = 0;
@@ -325,9 +368,12 @@ __device__ void qk_issuer(const FwdParams& p, uint8_t* sQ, uint8_t* sK, Barriers
       const uint32_t d_t = tmem + (gi & 1) * 128;
       const uint64_t kdesc = smem_desc_sw128(sKaddr + slot * C::kTileBytes, 16, 1024);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
+      for (int kk = 0; kk < C::kSteps; ++kk) {
         const uint32_t off = ((kk / 4) * C::kChunkBytes + (kk % 4) * 32) >> 4;
-        mma_ss(d_t, qdesc + off, kdesc + off, idesc, kk > 0 ? 1u : 0u);
+        if constexpr (kFp8)
+          mma_ss_f8(d_t, qdesc + off, kdesc + off, idesc, kk > 0 ? 1u : 0u);
+        else
+          mma_ss(d_t, qdesc + off, kdesc + off, idesc, kk > 0 ? 1u : 0u);
       }
       tc_commit(&bars->s_ready[gi % kRing]);
     }
@@ -347,9 +393,10 @@ __device__ void qk_issuer(const FwdParams& p, uint8_t* sQ, uint8_t* sK, Barriers
 // softmax warps have read O of the previous active job.
 template <typename T, int D>
 __device__ void pv_issuer(const FwdParams& p, uint8_t* sV, Barriers* bars, uint32_t tmem) {
-  using C = Cfg<D>;
+  using C = Cfg<T, D>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-  constexpr uint32_t idesc = instr_desc_f16(kBf16, BM, D, true);
+  constexpr bool kFp8 = Elem<T>::kFp8;
+  constexpr uint32_t idesc = kFp8 ? instr_desc_f8(Elem<T>::kFmt, BM, D) : instr_desc_f16(kBf16, BM, D, true);
   volatile int* abort = &bars->abort;
   const uint32_t sVaddr = smem_addr(sV);
   int g = 0, a = 0;
@@ -365,10 +412,19 @@ __device__ void pv_issuer(const FwdParams& p, uint8_t* sV, Barriers* bars, uint3
       if (!(ok = mbar_wait(&bars->v_full[slot], (gi / C::kSlotsV) & 1, abort))) return;
       tc_fence_after();
       const uint32_t a_t = tmem + kTmemP + (gi & 1) * 64;
-      const uint64_t vdesc = smem_desc_sw128(sVaddr + slot * C::kTileBytes, C::kChunkBytes, 1024);
+      if constexpr (kFp8) {
+        // B = V^T tile (d rows of 128 key bytes, K-major); 32 keys per MMA =
+        // 8 TMEM columns of P (four 8-bit values per column)
+        const uint64_t vdesc = smem_desc_sw128(sVaddr + slot * C::kTileBytes, 16, 1024);
 #pragma unroll
-      for (int kk = 0; kk < BN / 16; ++kk)
-        mma_ts(tmem + kTmemO, a_t + kk * 8, vdesc + ((kk * 2048) >> 4), idesc, (u > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BN / 32; ++kk)
+          mma_ts_f8(tmem + kTmemO, a_t + kk * 8, vdesc + ((kk * 32) >> 4), idesc, (u > 0 || kk > 0) ? 1u : 0u);
+      } else {
+        const uint64_t vdesc = smem_desc_sw128(sVaddr + slot * C::kTileBytes, C::kChunkBytes, 1024);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(tmem + kTmemO, a_t + kk * 8, vdesc + ((kk * 2048) >> 4), idesc, (u > 0 || kk > 0) ? 1u : 0u);
+      }
       tc_commit(&bars->pv_done[gi % kRing]);
     }
     g += n;
@@ -572,10 +628,24 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
             p1 = (x1 == -INFINITY) ? 0.0f : p1;
           }
           rsum2[e & 3] = f2_add(rsum2[e & 3], f2_pack(p0, p1));
-          pk[e] = pack2<T>(p0, p1);
-          qsum2[e & 1] = f2_add(qsum2[e & 1], widen2<T>(pk[e]));
+          if constexpr (Elem<T>::kFp8) {
+            // P <= 2^8 fits the 8-bit format's range; the pair's 16 bits
+            // are merged four keys to a column below
+            pk[e] = pack2_f8<Elem<T>::kFmt>(p0, p1);
+            qsum2[e & 1] = f2_add(qsum2[e & 1], widen2_f8<Elem<T>::kFmt>(pk[e]));
+          } else {
+            pk[e] = pack2<T>(p0, p1);
+            qsum2[e & 1] = f2_add(qsum2[e & 1], widen2<T>(pk[e]));
+          }
         }
-        tmem_st16(tmem + lane_sel + kTmemP + (gi & 1) * 64 + part * (kKeys / 2) + 16 * c, pk);
+        if constexpr (Elem<T>::kFp8) {
+          uint32_t pk4[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pk4[i] = pk[2 * i] | (pk[2 * i + 1] << 16);
+          tmem_st8(tmem + lane_sel + kTmemP + (gi & 1) * 64 + part * (kKeys / 4) + 8 * c, pk4);
+        } else {
+          tmem_st16(tmem + lane_sel + kTmemP + (gi & 1) * 64 + part * (kKeys / 2) + 16 * c, pk);
+        }
       }
     };
     if (masked)
@@ -643,8 +713,10 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
   }
 
   // epilogue: O / l -> dtype for this part's columns, LSE = (m + log2 l) ln 2
-  T* orow = reinterpret_cast<T*>(p.out) + ((jb.obase + (row_ok ? q : 0)) * p.H + h) * D + part * kOCols;
-  const float inv = qtot > 0.0f ? 1.0f / qtot : 0.0f;
+  using Out = typename Elem<T>::Out;
+  Out* orow = reinterpret_cast<Out*>(p.out) + ((jb.obase + (row_ok ? q : 0)) * p.H + h) * D + part * kOCols;
+  // (out_scale: the dequantisation factor of 8-bit V, else 1)
+  const float inv = qtot > 0.0f ? p.out_scale / qtot : 0.0f;
   if (ok && n > 0) {
 #pragma unroll
     for (int cc = 0; cc < kOCols / kOC; ++cc) {
@@ -657,7 +729,7 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
         uint32_t pk[kOC / 2];
 #pragma unroll
         for (int e = 0; e < kOC / 2; ++e)
-          pk[e] = pack2<T>(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+          pk[e] = pack2<Out>(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
         uint4* dst = reinterpret_cast<uint4*>(orow + kOC * cc);
 #pragma unroll
         for (int v = 0; v < kOC / 8; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
@@ -669,7 +741,7 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
     if (lane == 0) mbar_arrive(&bars->o_free);
   } else if (row_ok) {
     const float fill = ok ? 0.0f : nan;
-    const uint32_t w = pack2<T>(fill, fill);
+    const uint32_t w = pack2<Out>(fill, fill);
     uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
     for (int v = 0; v < kOCols / 8; ++v) dst[v] = make_uint4(w, w, w, w);
@@ -698,7 +770,7 @@ template <typename T, int D, bool kCap, bool kAlibi>
 __global__ void __launch_bounds__(threads_of(kCap, kAlibi), 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = Cfg<D>;
+  using C = Cfg<T, D>;
   constexpr int kSoftmaxWarps = 4 * parts_of(kCap, kAlibi);
   constexpr int kProducerWarp = kSoftmaxWarps;
   constexpr int kQkWarp = kSoftmaxWarps + 1;
@@ -766,7 +838,7 @@ __global__ void __launch_bounds__(threads_of(kCap, kAlibi), 1)
 template <typename T, int D, bool kCap, bool kAlibi>
 cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const FwdParams& p,
                    cudaStream_t stream) {
-  using C = Cfg<D>;
+  using C = Cfg<T, D>;
   static_assert(sizeof(Barriers) <= kBarrierBytes, "barrier block exceeds its reserve");
   static_assert(C::kSmemBytes <= 232448, "shared memory budget exceeded");
   static_assert(C::kSlotsK <= kMaxSlots && C::kSlotsV <= kMaxSlots, "too many K/V slots");
@@ -807,6 +879,59 @@ cudaError_t launch_fwd(bool bf16, int d, const CUtensorMap& tmQ, const CUtensorM
                             : launch_mods<__nv_bfloat16, 64>(tmQ, tmK, tmV, p, stream);
   return d == 128 ? launch_mods<__half, 128>(tmQ, tmK, tmV, p, stream)
                   : launch_mods<__half, 64>(tmQ, tmK, tmV, p, stream);
+}
+
+cudaError_t launch_fwd_fp8(int fmt, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmVt,
+                           const FwdParams& p, cudaStream_t stream) {
+  return fmt == 0 ? launch_mods<Fp8E4M3, 128>(tmQ, tmK, tmVt, p, stream)
+                  : launch_mods<Fp8E5M2, 128>(tmQ, tmK, tmVt, p, stream);
+}
+
+namespace {
+
+// V [B, Nk, H_kv, 128] (8-bit) -> V^T [B, H_kv, 128, Nk_pad], keys Nk ..
+// Nk_pad - 1 zero-filled: one CTA per (64-key block, head, batch) stages the
+// block in shared memory, 16-byte loads and stores.
+__global__ void __launch_bounds__(256) v_transpose_kernel(const uint8_t* __restrict__ v, uint8_t* __restrict__ vt,
+                                                          int Nk, int H_kv, int Nk_pad) {
+  constexpr int D = 128;
+  constexpr int kPitch = D + 16;  // bytes per staged key row
+  __shared__ __align__(16) uint8_t tile[64 * kPitch];
+  const int k0 = static_cast<int>(blockIdx.x) * 64;
+  const int hk = static_cast<int>(blockIdx.y);
+  const long long b = blockIdx.z;
+  for (int idx = threadIdx.x; idx < 64 * (D / 16); idx += blockDim.x) {
+    const int key = idx / (D / 16), c16 = idx % (D / 16);
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (k0 + key < Nk)
+      val = *reinterpret_cast<const uint4*>(v + ((b * Nk + k0 + key) * H_kv + hk) * D + 16 * c16);
+    *reinterpret_cast<uint4*>(tile + key * kPitch + 16 * c16) = val;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < D * 4; idx += blockDim.x) {
+    const int c = idx / 4, part = idx % 4;
+    if (k0 + 16 * part >= Nk_pad) continue;
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int kk = 16 * part + 4 * i;
+      w[i] = static_cast<uint32_t>(tile[kk * kPitch + c]) | (static_cast<uint32_t>(tile[(kk + 1) * kPitch + c]) << 8) |
+             (static_cast<uint32_t>(tile[(kk + 2) * kPitch + c]) << 16) |
+             (static_cast<uint32_t>(tile[(kk + 3) * kPitch + c]) << 24);
+    }
+    *reinterpret_cast<uint4*>(vt + ((b * H_kv + hk) * D + c) * static_cast<long long>(Nk_pad) + k0 + 16 * part) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_v_transpose(const void* v, void* vt, int B, int Nk, int H_kv, int Nk_pad, cudaStream_t stream) {
+  if (B == 0 || H_kv == 0 || Nk_pad == 0) return cudaSuccess;
+  dim3 grid(static_cast<unsigned>((Nk_pad + 63) / 64), static_cast<unsigned>(H_kv), static_cast<unsigned>(B));
+  v_transpose_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(v), static_cast<uint8_t*>(vt), Nk, H_kv,
+                                               Nk_pad);
+  return cudaGetLastError();
 }
 
 }  // namespace fa

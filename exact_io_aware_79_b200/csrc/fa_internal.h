@@ -35,6 +35,7 @@ struct FwdParams {
   float scale_log2;  // |scale| * log2(e)                (no softcap)
   float cap_scale;   // scale / softcap                   (softcap)
   float cap_log2;    // softcap * log2(e)                 (softcap)
+  float out_scale;   // O factor: the dequantisation factor of 8-bit V, else 1
 };
 
 // Paged decode, split kernel + merge kernel.
@@ -60,6 +61,17 @@ struct DecodeParams {
 // as 4-D tensors (d, H, N, B) with a (64, 1, 128, 1) box and 128-byte swizzle.
 cudaError_t launch_fwd(bool bf16, int d, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                        const FwdParams& p, cudaStream_t stream);
+
+// The forward on 8-bit inputs (fmt 0 = E4M3, 1 = E5M2; d = 128; output bf16):
+// Q and K maps (d, H, N, B) with a (128, 1, 128, 1) box of bytes, 128-byte
+// swizzle; tmVt: the transposed V written by launch_v_transpose, a map
+// (Nk_pad, d, H_kv, B) with a (128, 128, 1, 1) box.
+cudaError_t launch_fwd_fp8(int fmt, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmVt,
+                           const FwdParams& p, cudaStream_t stream);
+
+// V [B, Nk, H_kv, 128] (8-bit) -> V^T [B, H_kv, 128, Nk_pad] with keys
+// Nk .. Nk_pad - 1 set to zero (Nk_pad a multiple of 16).
+cudaError_t launch_v_transpose(const void* v, void* vt, int B, int Nk, int H_kv, int Nk_pad, cudaStream_t stream);
 
 // Grouped-query caches (two or more query heads per cache head) take the
 // tensor-core split kernel; it wants 128-byte-swizzled (64, 1, 64, 1) boxes.

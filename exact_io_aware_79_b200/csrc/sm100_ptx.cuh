@@ -187,6 +187,29 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// The same products with 8-bit operands (kind::f8f6f4: E4M3 or E5M2 as the
+// instruction descriptor says, fp32 accumulator); each consumes 32 bytes of
+// the K dimension.
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives once on `bar` when every tcgen05 operation this thread issued so
 // far has completed.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
@@ -226,6 +249,14 @@ template <int N>
 __device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
 #pragma unroll
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+// r[0..7] -> 8 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(r[0]),
+      "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
 }
 
 // r[0..15] -> 16 consecutive 32-bit TMEM columns of this thread's lane.
@@ -290,6 +321,16 @@ __host__ __device__ constexpr uint32_t instr_desc_f16(bool bf16, int M, int N, b
          | ((bf16 ? 1u : 0u) << 7)                    // A format
          | ((bf16 ? 1u : 0u) << 10)                   // B format
          | ((b_mn_major ? 1u : 0u) << 16)             // B major
+         | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
+}
+
+// Instruction descriptor for kind::f8f6f4 with an fp32 accumulator: fmt 0 =
+// E4M3, 1 = E5M2 for both operands; both K-major.
+__host__ __device__ constexpr uint32_t instr_desc_f8(uint32_t fmt, int M, int N) {
+  return (1u << 4)                                    // D format: f32
+         | (fmt << 7)                                 // A format
+         | (fmt << 10)                                // B format
          | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
 }
@@ -416,6 +457,33 @@ __device__ __forceinline__ uint64_t widen2<__nv_bfloat16>(uint32_t u) {
 template <>
 __device__ __forceinline__ uint64_t widen2<__half>(uint32_t u) {
   __half2 v = *reinterpret_cast<__half2*>(&u);
+  const float2 f = __half22float2(v);
+  return f2_pack(f.x, f.y);
+}
+
+// Two fp32 values rounded to 8-bit floats (fmt 0 = E4M3, 1 = E5M2; round to
+// nearest, saturating to the largest finite value) in the 16 bits of one
+// pair, lo in the low byte.
+template <uint32_t kFmt>
+__device__ __forceinline__ uint32_t pack2_f8(float lo, float hi) {
+  uint16_t h;
+  if constexpr (kFmt == 0)
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(hi), "f"(lo));
+  else
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(h) : "f"(hi), "f"(lo));
+  return h;
+}
+
+// The pair of pack2_f8, widened exactly to an fp32 pair (lo first).
+template <uint32_t kFmt>
+__device__ __forceinline__ uint64_t widen2_f8(uint32_t u) {
+  uint32_t h2;
+  const uint16_t h = static_cast<uint16_t>(u);
+  if constexpr (kFmt == 0)
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(h));
+  else
+    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h2) : "h"(h));
+  __half2 v = *reinterpret_cast<__half2*>(&h2);
   const float2 f = __half22float2(v);
   return f2_pack(f.x, f.y);
 }

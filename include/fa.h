@@ -30,7 +30,8 @@
  *     pointer after a call returns and holds no global state besides a
  *     per-device cache of device properties and the fixed device array of
  *     fa_fwd_kvcache_noalloc.
- *   - Element types: Q, K, V and O are fp16 or bf16 (fa_dtype); LSE is fp32;
+ *   - Element types: Q, K, V and O are fp16 or bf16 (fa_dtype), or for
+ *     fa_fwd_fp8 8-bit Q, K, V (fa_fp8_format) and bf16 O; LSE is fp32;
  *     block tables and lengths are int32; ALiBi slopes are fp32. Arithmetic
  *     is fp32 (the two products run on tensor cores with fp32 accumulation).
  *   - Score modifiers, applied in this order to s = scale * (q . k):
@@ -76,6 +77,7 @@ typedef enum {
 } fa_status;
 
 typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
+typedef enum { FA_E4M3 = 0, FA_E5M2 = 1 } fa_fp8_format;
 
 #define FA_MAX_SPLITS 64
 
@@ -100,6 +102,44 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *out, float *
                  int B, int H, int Nq, int Nk, int d, fa_dtype dtype, float scale,
                  int causal, int window_left, int window_right,
                  const float *alibi_slopes, float softcap, cudaStream_t stream);
+
+/*
+ * fa_fwd_fp8 -- the forward on 8-bit inputs. "FlashAttention深度解析：从算法
+ * 创新到产业变革的全面影响" (section 未来展望) and "IO感知技术革命" (section
+ * H100架构的性能跃升) name an FP8 forward without stating its form; the
+ * reading taken: q, k, v hold 8-bit floats x8 that stand for x8 * descale_x
+ * (one fp32 factor per tensor), and the result is fa_fwd's attention of
+ * those dequantised values, written as bf16.
+ *
+ *   q    [B, Nq, H, d]      8-bit (fmt), read
+ *   k, v [B, Nk, H_kv, d]   8-bit (fmt), read (H % H_kv == 0, as fa_fwd_gqa)
+ *   out  [B, Nq, H, d]      bf16, written
+ *   lse  [B, H, Nq]         fp32, written (natural log)
+ *   fmt                     FA_E4M3 or FA_E5M2 (all three tensors), else
+ *                           FA_ERR_DTYPE
+ *   scale, descale_q/k/v    the scores are (scale * descale_q * descale_k) *
+ *                           (q8 . k8), O is scaled by descale_v; the
+ *                           descales finite and > 0, else FA_ERR_ARG
+ *   causal, windows, alibi_slopes, softcap   as in fa_fwd
+ *   workspace               device buffer of fa_fwd_fp8_workspace_size()
+ *                           bytes, 16-byte aligned, caller-owned (V is
+ *                           transposed into it first, so both products read
+ *                           K-major 8-bit operands), else FA_ERR_WORKSPACE
+ *
+ * Both products run on the tensor cores with 8-bit operands (kind::f8f6f4,
+ * fp32 accumulation); P is rounded to fmt before the PV product (relative
+ * error 2^-4 for E4M3, 2^-3 for E5M2, larger for values below the format's
+ * normal range), and O is divided by the sum of P as rounded, so those
+ * roundings perturb the weights of a convex combination of V rows. d must be
+ * 128 (FA_ERR_HEADDIM otherwise). Other limits as in fa_fwd.
+ */
+size_t fa_fwd_fp8_workspace_size(int B, int H_kv, int Nk, int d);
+fa_status fa_fwd_fp8(const void *q, const void *k, const void *v, void *out, float *lse,
+                     int B, int H, int H_kv, int Nq, int Nk, int d, fa_fp8_format fmt,
+                     float scale, float descale_q, float descale_k, float descale_v,
+                     int causal, int window_left, int window_right,
+                     const float *alibi_slopes, float softcap,
+                     void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * fa_fwd_gqa -- fa_fwd with grouped-query attention: H query heads share

@@ -89,6 +89,8 @@ def test_host_tensors_are_rejected_before_any_launch(no_library):
         lambda: fa.fa_fwd_kvcache_gqa(one, kc, kc, table, lens, one, lse1, 0.1),
         lambda: fa.fa_fwd_kvcache_noalloc(one, kc, kc, table, lens, one, lse1, 0.1),
         lambda: fa.fa_kvcache_append(one, one, kc, kc, table, lens),
+        lambda: fa.fa_fwd_fp8(q.to(torch.float8_e4m3fn), q.to(torch.float8_e4m3fn), q.to(torch.float8_e4m3fn),
+                              t(B, N, H, d), lse, 0.1),
     ]
     for i, call in enumerate(calls):
         with pytest.raises(ValueError, match="CUDA"):
