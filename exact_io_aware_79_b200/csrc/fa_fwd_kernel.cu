@@ -11,28 +11,30 @@
 // B200 mapping. The grid is persistent (at most one CTA per SM); a CTA runs
 // jobs, each one 128-row Q tile of one (batch, head), back to back with
 // these warps:
-//   softmax    4 * parts warps: the parts warps w, w + 4, ... share TMEM
-//              lanes 32 (w % 4) .. + 31 (one query row per lane) and split
-//              each row's 128 keys into parts slices, combining the partial
-//              maxima and sums through shared memory (parts = 2 for plain
-//              scores; 4 with softcap or ALiBi, whose per-element work four
-//              warps per sub-partition hide better)
+//   softmax    8 warps in two parts: warps w and w + 4 share TMEM lanes
+//              32 (w % 4) .. + 31 (one query row per lane); part 0 takes
+//              keys 0..63 of every tile, part 1 keys 64..127. Each part runs
+//              its own online softmax (its own running max, sums and O
+//              accumulator), so the two never wait for each other within a
+//              job; they merge their results once, at the end of the job
 //   producer   TMA: each job's Q tile (two buffers, so the next job's Q
 //              lands early), then K and V tiles into two rings of
 //              shared-memory slots (128-byte swizzle), expect-tx
 //   QK issuer  one elected thread; owns TMEM
 //   PV issuer  one elected thread
 // Tensor memory (512 columns x 128 lanes x 32 bit):
-//   cols   0..127  S buffer 0 (fp32 scores)
+//   cols   0..127  S buffer 0 (fp32 scores): part p's 64 keys in columns
+//                  64 p .. 64 p + 63, overwritten by its P (16-bit, two per
+//                  column, or 8-bit, four per column) once it has read them;
+//                  the PV products read P straight from TMEM
 //   cols 128..255  S buffer 1
-//   cols 256..383  O (fp32, d columns)
-//   cols 384..447  P buffer 0 (16-bit probabilities, two per column; the PV
-//                  product reads them straight from TMEM)
-//   cols 448..511  P buffer 1
-// K/V tiles are numbered across the CTA's jobs; tile g uses S and P buffer
-// g & 1. The QK thread computes S(g) as soon as K(g) has landed and the PV
-// product of tile g - 2 (the last reader of both buffers) is done; the PV
-// thread computes O += P(g) V(g) as soon as the softmax has published P(g).
+//   cols 256..383  O_0: part 0's accumulator (fp32, d columns)
+//   cols 384..511  O_1: part 1's
+// K/V tiles are numbered across the CTA's jobs; tile g uses S buffer g & 1.
+// The QK thread computes S(g) as soon as K(g) has landed and the PV product
+// of tile g - 2 (the last reader of the buffer, P(g - 2) included) is done;
+// the PV thread computes O_p += P_p(g) V_p(g) for both parts as soon as the
+// softmax has published P(g).
 // Across a job boundary the next job's first scores are computed while the
 // softmax warps write out the previous job's O. The two
 // products are independent, so they sit in different threads: each thread
@@ -42,10 +44,12 @@
 // current one, so the step time is max(softmax, tensor core) rather than
 // their sum.
 //
-// Rescaling is lazy: a row keeps its old max unless a new tile raises it by
-// more than 8 (log2 units), so P stays <= 2^8 and O is rescaled only when it
-// must be (after waiting for the previous PV product). The result is the
-// same softmax (m cancels in O / l).
+// Rescaling is lazy: a part keeps its old max unless a new tile raises it
+// by more than 8 (log2 units), so P stays <= 2^8 and O_p is rescaled only
+// when it must be (after waiting for the previous PV product). The result is
+// the same softmax (the maxima cancel in O / l): at the end of a job
+// O = (a_0 O_0 + a_1 O_1) / (a_0 q_0 + a_1 q_1) with a_p = 2^(m_p - max m),
+// q_p the part's sum of P as rounded.
 #include "fa_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -59,13 +63,12 @@ namespace {
 
 constexpr int BM = 128;  // query rows per Q tile
 constexpr int BN = 128;  // keys per K/V tile
-// Softmax warps per row (per TMEM lane quarter): the score modifiers
-// (softcap, ALiBi) add per-element work that four warps per sub-partition
-// hide better; plain scores run fastest with two. Warp roles: softmax warps
-// 0 .. 4 * parts - 1, then the TMA producer, the QK issuer (owns TMEM) and
-// the PV issuer.
-constexpr int kMaxParts = 4;
-constexpr int parts_of(bool cap, bool alibi) { return (cap || alibi) ? 4 : 2; }
+// Softmax warps per row (per TMEM lane quarter): two, each with its own O
+// accumulator (two fill the 512 TMEM columns with the two S buffers). Warp
+// roles: softmax warps 0 .. 7, then the TMA producer, the QK issuer (owns
+// TMEM) and the PV issuer.
+constexpr int kMaxParts = 2;
+constexpr int parts_of(bool, bool) { return 2; }
 constexpr int threads_of(bool cap, bool alibi) { return 32 * (4 * parts_of(cap, alibi) + 3); }
 constexpr int kMaxSlots = 6;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -75,8 +78,8 @@ constexpr uint32_t kTmemCols = 512;
 // advances only through steps that need the waiter to have passed first
 // (P of a later tile, or a K/V load issued after the wait).
 constexpr int kRing = 8;
-constexpr uint32_t kTmemO = 256;
-constexpr uint32_t kTmemP = 384;  // two 64-column P buffers
+constexpr uint32_t kTmemO = 256;        // O accumulator of part 0; part 1's follows
+constexpr uint32_t kTmemOStride = 128;
 
 constexpr int kBarrierBytes = 8192;  // barrier block and exchange slots
 
@@ -386,11 +389,13 @@ __device__ void qk_issuer(const FwdParams& p, uint8_t* sQ, uint8_t* sK, Barriers
   drain_wait(&bars->qk_idle, 0);
 }
 
-// O (+)= P(g) V_g: A = P from TMEM (16-bit, two keys per column, P buffer
-// g & 1), B = V tile stored keys x d with d contiguous (MN-major): 16 keys =
-// 2048 bytes, the second 64-wide d chunk lies 16 KB further (leading byte
-// offset). The first product of a job overwrites O, so it waits until the
-// softmax warps have read O of the previous active job.
+// O_p (+)= P_p(g) V_g[keys of part p] for p = 0, 1: A = P from TMEM (the
+// first columns of part p's S columns in buffer g & 1), B = V tile stored
+// keys x d with d contiguous (MN-major): 16 keys = 2048 bytes, the second
+// 64-wide d chunk lies 16 KB further (leading byte offset); 8-bit V arrives
+// transposed (K-major). The first products of a job overwrite O_0 and O_1,
+// so they wait until the softmax warps have read both of the previous
+// active job.
 template <typename T, int D>
 __device__ void pv_issuer(const FwdParams& p, uint8_t* sV, Barriers* bars, uint32_t tmem) {
   using C = Cfg<T, D>;
@@ -411,19 +416,25 @@ __device__ void pv_issuer(const FwdParams& p, uint8_t* sV, Barriers* bars, uint3
       const int slot = gi % C::kSlotsV;
       if (!(ok = mbar_wait(&bars->v_full[slot], (gi / C::kSlotsV) & 1, abort))) return;
       tc_fence_after();
-      const uint32_t a_t = tmem + kTmemP + (gi & 1) * 64;
-      if constexpr (kFp8) {
-        // B = V^T tile (d rows of 128 key bytes, K-major); 32 keys per MMA =
-        // 8 TMEM columns of P (four 8-bit values per column)
-        const uint64_t vdesc = smem_desc_sw128(sVaddr + slot * C::kTileBytes, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < BN / 32; ++kk)
-          mma_ts_f8(tmem + kTmemO, a_t + kk * 8, vdesc + ((kk * 32) >> 4), idesc, (u > 0 || kk > 0) ? 1u : 0u);
-      } else {
-        const uint64_t vdesc = smem_desc_sw128(sVaddr + slot * C::kTileBytes, C::kChunkBytes, 1024);
+      for (int part = 0; part < 2; ++part) {
+        // part p's P lies in the first columns of its own 64 S columns;
+        // O_p += P_p V[keys 64 p .. 64 p + 63]
+        const uint32_t a_t = tmem + (gi & 1) * 128 + part * 64;
+        const uint32_t d_t = tmem + kTmemO + part * kTmemOStride;
+        if constexpr (kFp8) {
+          // B = V^T tile (d rows of 128 key bytes, K-major); 32 keys per MMA
+          // = 8 TMEM columns of P (four 8-bit values per column)
+          const uint64_t vdesc = smem_desc_sw128(sVaddr + slot * C::kTileBytes, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(tmem + kTmemO, a_t + kk * 8, vdesc + ((kk * 2048) >> 4), idesc, (u > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BN / 64; ++kk)
+            mma_ts_f8(d_t, a_t + kk * 8, vdesc + ((part * 64 + kk * 32) >> 4), idesc, (u > 0 || kk > 0) ? 1u : 0u);
+        } else {
+          const uint64_t vdesc = smem_desc_sw128(sVaddr + slot * C::kTileBytes, C::kChunkBytes, 1024);
+#pragma unroll
+          for (int kk = 0; kk < BN / 32; ++kk)
+            mma_ts(d_t, a_t + kk * 8, vdesc + (((part * 4 + kk) * 2048) >> 4), idesc, (u > 0 || kk > 0) ? 1u : 0u);
+        }
       }
       tc_commit(&bars->pv_done[gi % kRing]);
     }
@@ -442,16 +453,14 @@ __device__ __forceinline__ float mod_score(const FwdParams& p, float x, float sl
   return t;
 }
 
-// Softmax: kSoftmaxWarps warps, kParts per sub-partition. The kParts warps
-// w, w + 4, w + 8, ... own the same 32 query rows (TMEM lanes 32(w % 4) ..),
-// one row per thread, and split each 128-key tile into kParts slices of
-// kKeys keys. They exchange partial maxima through shared memory under a
-// named barrier, so all take the same lazy rescaling decision; each writes
-// its slice of P (16-bit, into its columns of the tile's P buffer), rescales
-// and stores its D / kParts columns of O, and the row sums are combined once
-// at the end. kCap / kAlibi select the score modifiers at compile time;
-// whether a K tile needs the element mask is decided per tile for the whole
-// group, so the common interior tiles run without per-element compares.
+// Softmax: 8 warps, two per sub-partition. The parts warps w and w + 4 own
+// the same 32 query rows (TMEM lanes 32(w % 4) ..), one row per thread, and
+// each handles its own half of every 128-key tile with its own running
+// state; the halves meet only in the job's epilogue, through shared memory
+// under a named barrier. kCap / kAlibi select the score modifiers at compile
+// time; whether a K tile needs the element mask is decided per tile for the
+// whole group, so the common interior tiles run without per-element
+// compares.
 template <int kParts>
 __device__ __forceinline__ void part_sync(int quarter) {
   // named barrier 1 + quarter, shared by the kParts warps of one lane quarter
@@ -479,9 +488,10 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
   constexpr int kParts = parts_of(kCap, kAlibi);
   constexpr int kKeys = BN / kParts;     // keys per thread per tile
   constexpr int kChunks = kKeys / 32;    // 32-column TMEM loads of S per tile
-  constexpr int kOCols = D / kParts;     // O columns per thread
-  constexpr int kOC = kOCols < 32 ? kOCols : 32;  // O columns per TMEM access
-  static_assert(kKeys % 32 == 0 && kOCols % 16 == 0, "part sizes");
+  constexpr int kOCols = D / kParts;     // output columns per thread in the epilogue
+  constexpr int kPCols = kKeys * Elem<T>::kBytes / 4;  // TMEM columns of this part's P
+  static_assert(kKeys % 32 == 0 && kOCols % 32 == 0 && kParts == 2, "part sizes");
+  using Out = typename Elem<T>::Out;
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -498,42 +508,35 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
   const RowRange first_row = row_range(p, jb.Nq, jb.Nk, q0), last_row = row_range(p, jb.Nq, jb.Nk, qz);
   const int pos = q + jb.Nk - jb.Nq;
   const uint32_t lane_sel = static_cast<uint32_t>(quarter * 32) << 16;
-  const uint32_t tO = tmem + lane_sel + kTmemO + part * kOCols;
+  const uint32_t tO = tmem + lane_sel + kTmemO + part * kTmemOStride;  // this part's O accumulator
   const float slope_l2 = kAlibi ? p.slopes[h] * kLog2e : 0.0f;
   const float sl2 = p.scale_log2;  // >= 0 (a negative scale is folded into the MMA)
   const uint64_t mul2 = kPlain ? f2_pack(sl2, sl2) : f2_pack(1.0f, 1.0f);
   const float nan = __int_as_float(0x7fc00000);
 
-  float m = -INFINITY;  // running max of the whole row (log2 units)
-  float lsum = 0.0f;    // this part's running sum of exp2(t - m) (for LSE)
+  // This part's own online softmax over its kKeys keys of every tile: its
+  // own running max, sums and O accumulator, merged with the other part's
+  // once, at the end of the job.
+  float m = -INFINITY;  // running max of this part's keys (log2 units)
+  float lsum = 0.0f;    // running sum of exp2(t - m) (for LSE)
   float qsum = 0.0f;    // the same sum of P as rounded for the PV product (for O)
   bool ok = alive;      // after a failure in an earlier job, only fill
-  bool broke = false;   // left the loop at a shared exchange (all parts do)
   const int n = jb.has ? l - f + 1 : 0;
   const int n_run = ok ? n : 0;
-  // Each iteration performs exactly one exchange, and every early exit
-  // happens right after one, on a decision all parts share, so the named
-  // barriers can never be left waiting for a partner that has gone.
   for (int it = 0; it < n_run; ++it) {
     const int j = f + it;
     const int gi = g + it;  // tile number across the CTA's jobs
-    const uint32_t tS = tmem + lane_sel + (gi & 1) * 128;
-    ok = ok && mbar_wait(&bars->s_ready[gi % kRing], (gi / kRing) & 1, abort);
+    const uint32_t tS = tmem + lane_sel + (gi & 1) * 128 + part * 64;  // this part's S, then P, columns
+    ok = mbar_wait(&bars->s_ready[gi % kRing], (gi / kRing) & 1, abort);
     ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
     uint32_t s[kChunks][32];
     const int key0 = j * BN + part * kKeys;
     const bool masked = j * BN < last_row.lo || j * BN + BN - 1 > first_row.hi;  // uniform over the tile
-    if (ok) {
-      tc_fence_after();
+    tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) tmem_ld32(tS + part * kKeys + 32 * c, s[c]);
-      tmem_wait_ld();
-    } else {
-#pragma unroll
-      for (int c = 0; c < kChunks; ++c)
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c][e] = 0u;
-    }
+    for (int c = 0; c < kChunks; ++c) tmem_ld32(tS + 32 * c, s[c]);
+    tmem_wait_ld();
 #pragma unroll
     for (int c = 0; c < kChunks; ++c) reg_fence(s[c]);
     // pass 1: transform (modifier paths), mask and this part's max
@@ -560,29 +563,15 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
       }
     }
     float mt = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]);
-    // combine with the other parts of the row
-    float all[kParts];
-    part_exchange(bars->xchg, xk++, part, r, quarter, ok ? mt : nan, all);
-    bool none_nan = true;
-#pragma unroll
-    for (int i = 0; i < kParts; ++i) {
-      none_nan = none_nan && all[i] == all[i];
-      mt = fmaxf(mt, all[i]);
-    }
-    ok = __all_sync(0xffffffffu, ok && none_nan);
-    if (!ok) {  // every part of every row of this warp group sees the same NaN
-      broke = true;
-      break;
-    }
     // plain path: the max was taken over raw scores; scale after (sl2 >= 0)
     if (kPlain) mt = (mt == -INFINITY) ? -INFINITY : mt * sl2;
 
-    // lazy max update (identical in all parts of the row)
+    // lazy max update
     const float m_new = fmaxf(m, mt);
     float alpha = 1.0f;
     bool rescale = false;
     if (m == -INFINITY) {
-      m = m_new;  // nothing accumulated yet for this row (O row is 0, l is 0)
+      m = m_new;  // nothing accumulated yet for this part (its O is 0, l is 0)
     } else if (m_new > m + kRescaleThreshold) {
       alpha = ex2(m - m_new);
       m = m_new;
@@ -591,17 +580,17 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
     lsum *= alpha;
     qsum *= alpha;
     const float m_eff = (m == -INFINITY) ? 0.0f : m;
-    // pass 2: P = exp2(t - m) into this part's kKeys / 2 columns of the P
-    // buffer; pairs of elements go through packed fp32x2 FMA (scale,
-    // subtract max) and add. O is normalised by the sum of P exactly as the
-    // PV product sees it (the 16-bit values), so rounding P to 16 bits
-    // perturbs the weights of a convex combination of V rows rather than its
-    // total; LSE takes the sum of the unrounded values.
+    // pass 2: P = exp2(t - m) over this part's own S columns (read above);
+    // pairs of elements go through packed fp32x2 FMA (scale, subtract max)
+    // and add. O is normalised by the sum of P exactly as the PV product
+    // sees it (the rounded values), so rounding P perturbs the weights of a
+    // convex combination of V rows rather than its total; LSE takes the sum
+    // of the unrounded values.
     const uint64_t m2 = f2_pack(-m_eff, -m_eff);
     uint64_t rsum2[4] = {0, 0, 0, 0};  // independent packed partial sums (0 bits = +0.0f)
-    uint64_t qsum2[2] = {0, 0};        // the same, of the 16-bit P
-    auto pass2 = [&](auto emu_tag) {
-      constexpr bool kMaskedTile = decltype(emu_tag)::value;
+    uint64_t qsum2[2] = {0, 0};        // the same, of the rounded P
+    auto pass2 = [&](auto masked_tag) {
+      constexpr bool kMaskedTile = decltype(masked_tag)::value;
 #pragma unroll
       for (int c = 0; c < kChunks; ++c) {
         uint32_t pk[16];
@@ -642,9 +631,9 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
           uint32_t pk4[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) pk4[i] = pk[2 * i] | (pk[2 * i + 1] << 16);
-          tmem_st8(tmem + lane_sel + kTmemP + (gi & 1) * 64 + part * (kKeys / 4) + 8 * c, pk4);
+          tmem_st8(tS + 8 * c, pk4);
         } else {
-          tmem_st16(tmem + lane_sel + kTmemP + (gi & 1) * 64 + part * (kKeys / 2) + 16 * c, pk);
+          tmem_st16(tS + 16 * c, pk);
         }
       }
     };
@@ -656,86 +645,102 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
     f2_unpack(f2_add(rsum2[0], rsum2[1]), r0, r1);
     f2_unpack(f2_add(rsum2[2], rsum2[3]), r2, r3);
     f2_unpack(f2_add(qsum2[0], qsum2[1]), u0, u1);
-    const float rs = (r0 + r1) + (r2 + r3);
+    lsum += (r0 + r1) + (r2 + r3);
     qsum += u0 + u1;
     if (__any_sync(0xffffffffu, rescale)) {
-      // O must be idle: wait for the product of the previous tile (the only
-      // one that can still be running).
+      // this part's O must be idle: wait for the product of the previous
+      // tile (the only one that can still be running)
       if (it > 0) {
-        // on a timeout, carry on to the next exchange, which ends all parts
         ok = mbar_wait(&bars->pv_done[(gi - 1) % kRing], ((gi - 1) / kRing) & 1, abort);
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
       }
+      if (ok) {
 #pragma unroll
-      for (int cc = 0; cc < kOCols / kOC; ++cc) {
-        uint32_t o[kOC];
-        if constexpr (kOC == 32) tmem_ld32(tO + kOC * cc, o);
-        else tmem_ld16(tO + kOC * cc, o);
-        tmem_wait_ld();
-        reg_fence(o);
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * cc, o);
+          tmem_wait_ld();
+          reg_fence(o);
 #pragma unroll
-        for (int e = 0; e < kOC; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-        if constexpr (kOC == 32) tmem_st32(tO + kOC * cc, o);
-        else tmem_st16(tO + kOC * cc, o);
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + 32 * cc, o);
+        }
       }
     }
-    lsum += rs;
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars->p_full[gi & 1]);
+    if (!ok) break;
   }
-  // the loop ran the same number of exchanges in all parts: it ended at a
-  // shared break, or after all n iterations (possibly with a failed wait in
-  // one part, which the final exchange reports to the others)
-  const int n_done = broke ? -1 : n_run;
-  if (ok && n > 0) {
+  if (ok && n_run > 0) {
     ok = mbar_wait(&bars->pv_done[(g + n - 1) % kRing], ((g + n - 1) / kRing) & 1, abort);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
   }
-  // all parts of a row must agree on success; combine the row sums (two
-  // exchanges, made by all parts alike)
-  float ltot = lsum, qtot = qsum;
-  if (n_done >= 0 && alive) {
-    float all[kParts];
-    part_exchange(bars->xchg, xk++, part, r, quarter, ok ? lsum : nan, all);
-    ltot = 0.0f;
+  // Merge the parts of the row (three exchanges, made by both parts of
+  // every job that had keys, while no earlier job failed): M = max m_p,
+  // a_p = 2^(m_p - M); O = sum a_p O_p / sum a_p q_p, LSE from sum a_p l_p.
+  float a_self = 0.0f, a_other = 0.0f, ltot = 0.0f, qtot = 0.0f;
+  if (alive && n > 0) {
+    float mm[kParts], ll[kParts], qq[kParts];
+    part_exchange(bars->xchg, xk++, part, r, quarter, ok ? m : nan, mm);
+    part_exchange(bars->xchg, xk++, part, r, quarter, ok ? lsum : nan, ll);
+    part_exchange(bars->xchg, xk++, part, r, quarter, ok ? qsum : nan, qq);
+    float M = -INFINITY;
+    bool none_nan = true;
 #pragma unroll
-    for (int i = 0; i < kParts; ++i) ltot += all[i];  // NaN if any part failed
-    part_exchange(bars->xchg, xk++, part, r, quarter, ok ? qsum : nan, all);
-    qtot = 0.0f;
+    for (int i = 0; i < kParts; ++i) {
+      none_nan = none_nan && ll[i] == ll[i] && qq[i] == qq[i] && !(mm[i] != mm[i]);
+      M = fmaxf(M, mm[i]);
+    }
+    ok = ok && none_nan;
+    if (ok) {
 #pragma unroll
-    for (int i = 0; i < kParts; ++i) qtot += all[i];
-    ok = ok && ltot == ltot && qtot == qtot;
-    if (!ok) ltot = qtot = 0.0f;
+      for (int i = 0; i < kParts; ++i) {
+        const float ai = (mm[i] == -INFINITY) ? 0.0f : ex2(mm[i] - M);
+        ltot += ai * ll[i];
+        qtot += ai * qq[i];
+        if (i == part) a_self = ai;
+        else a_other = ai;
+      }
+      m = M;
+    }
   }
 
-  // epilogue: O / l -> dtype for this part's columns, LSE = (m + log2 l) ln 2
-  using Out = typename Elem<T>::Out;
+  // epilogue: this part's kOCols output columns of the row, from both O
+  // accumulators: (a_0 O_0 + a_1 O_1) / (a_0 q_0 + a_1 q_1), as Out;
+  // LSE = (M + log2 l) ln 2
   Out* orow = reinterpret_cast<Out*>(p.out) + ((jb.obase + (row_ok ? q : 0)) * p.H + h) * D + part * kOCols;
   // (out_scale: the dequantisation factor of 8-bit V, else 1)
   const float inv = qtot > 0.0f ? p.out_scale / qtot : 0.0f;
+  const uint32_t tO_self = tO + part * kOCols;                                  // own O, own columns
+  const uint32_t tO_other = tmem + lane_sel + kTmemO + (1 - part) * kTmemOStride + part * kOCols;
   if (ok && n > 0) {
 #pragma unroll
-    for (int cc = 0; cc < kOCols / kOC; ++cc) {
-      uint32_t o[kOC];
-      if constexpr (kOC == 32) tmem_ld32(tO + kOC * cc, o);
-      else tmem_ld16(tO + kOC * cc, o);
+    for (int cc = 0; cc < kOCols / 32; ++cc) {
+      uint32_t o[32], o2[32];
+      tmem_ld32(tO_self + 32 * cc, o);
+      tmem_ld32(tO_other + 32 * cc, o2);
       tmem_wait_ld();
       reg_fence(o);
+      reg_fence(o2);
       if (row_ok) {
-        uint32_t pk[kOC / 2];
+        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < kOC / 2; ++e)
-          pk[e] = pack2<Out>(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        uint4* dst = reinterpret_cast<uint4*>(orow + kOC * cc);
+        for (int e = 0; e < 16; ++e) {
+          const float v0 = (a_self * __uint_as_float(o[2 * e]) + a_other * __uint_as_float(o2[2 * e])) * inv;
+          const float v1 = (a_self * __uint_as_float(o[2 * e + 1]) + a_other * __uint_as_float(o2[2 * e + 1])) * inv;
+          pk[e] = pack2<Out>(v0, v1);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cc);
 #pragma unroll
-        for (int v = 0; v < kOC / 8; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
       }
     }
-    // O has been read: the next job's first PV product may overwrite it
+    // both O accumulators have been read (by both parts, which each arrive
+    // here): the next job's first PV product may overwrite them
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars->o_free);
