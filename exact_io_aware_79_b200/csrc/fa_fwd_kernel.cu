@@ -447,10 +447,11 @@ __device__ void pv_issuer(const FwdParams& p, uint8_t* sV, Barriers* bars, uint3
 
 // Score transform of one element in log2 units (softcap and ALiBi paths).
 template <bool kCap, bool kAlibi>
-__device__ __forceinline__ float mod_score(const FwdParams& p, float x, float slope_l2, int dist) {
-  float t = kCap ? p.cap_log2 * tanh_via_exp2(x * p.cap_scale) : x * p.scale_log2;
-  if (kAlibi) t -= slope_l2 * fabsf(static_cast<float>(dist));
-  return t;
+__device__ __forceinline__ float mod_score(const FwdParams& p, float x, float cap_k, float slope_l2, float dist) {
+  // dist = pos - key as a float (integers below 2^24 exactly)
+  const float bias = kAlibi ? -slope_l2 * fabsf(dist) : 0.0f;
+  if (kCap) return softcap_fma(x, cap_k, p.cap_log2, bias);
+  return fmaf(x, p.scale_log2, bias);
 }
 
 // Softmax: 8 warps, two per sub-partition. The parts warps w and w + 4 own
@@ -510,6 +511,7 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
   const uint32_t lane_sel = static_cast<uint32_t>(quarter * 32) << 16;
   const uint32_t tO = tmem + lane_sel + kTmemO + part * kTmemOStride;  // this part's O accumulator
   const float slope_l2 = kAlibi ? p.slopes[h] * kLog2e : 0.0f;
+  const float cap_k = p.cap_scale * 2.8853900817779268f;  // 2 log2(e) / softcap * |scale|
   const float sl2 = p.scale_log2;  // >= 0 (a negative scale is folded into the MMA)
   const uint64_t mul2 = kPlain ? f2_pack(sl2, sl2) : f2_pack(1.0f, 1.0f);
   const float nan = __int_as_float(0x7fc00000);
@@ -532,6 +534,9 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
     if (!ok) break;
     uint32_t s[kChunks][32];
     const int key0 = j * BN + part * kKeys;
+    // distance of the tile's first key from the row's position; element e of
+    // the tile is dpos - e away (ALiBi)
+    const float dpos = kAlibi ? static_cast<float>(pos - key0) : 0.0f;
     const bool masked = j * BN < last_row.lo || j * BN + BN - 1 > first_row.hi;  // uniform over the tile
     tc_fence_after();
 #pragma unroll
@@ -548,7 +553,7 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
         for (int e = 0; e < 32; ++e) {
           float x = __uint_as_float(s[c][e]);
           const int key = key0 + 32 * c + e;
-          if (!kPlain) x = mod_score<kCap, kAlibi>(p, x, slope_l2, pos - key);
+          if (!kPlain) x = mod_score<kCap, kAlibi>(p, x, cap_k, slope_l2, dpos - static_cast<float>(32 * c + e));
           if (masked) x = (key >= rr.lo && key <= rr.hi) ? x : -INFINITY;
           s[c][e] = __float_as_uint(x);
         }

@@ -72,7 +72,29 @@ __global__ void tanh_abs_error(float* worst, double lo, double step, int n) {
   }
 }
 
+// |softcap_fma(x, 2 log2(e) / s, c, b) - (c tanh(x / s) + b)| for x =
+// +-10^(lo + i * step) * s, and x = 0 (s, c, b as given).
+__global__ void softcap_abs_error(float* worst, double lo, double step, int n, float s, float c, float b) {
+  const float k = static_cast<float>(2.0 * 1.4426950408889634 / s);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= n; i += gridDim.x * blockDim.x) {
+    const double a = (i == n) ? 0.0 : pow(10.0, lo + step * i) * s;
+    for (int sg = 0; sg < 2; ++sg) {
+      const float x = static_cast<float>(sg ? -a : a);
+      const float t = fa::softcap_fma(x, k, c, b);
+      const double e = fabs(static_cast<double>(t) - (c * tanh(static_cast<double>(x) / s) + b));
+      if (t != t) worst[1] = 1.0f;
+      atomic_max_pos(&worst[0], static_cast<float>(e));
+    }
+  }
+}
+
 }  // namespace
+
+extern "C" int check_softcap(float* worst, double lo, double step, int n, float s, float c, float b,
+                             cudaStream_t st) {
+  softcap_abs_error<<<148 * 4, 256, 0, st>>>(worst, lo, step, n, s, c, b);
+  return static_cast<int>(cudaGetLastError());
+}
 
 extern "C" int check_ex2_poly_reduced(float* worst, cudaStream_t s) {
   // |f| <= 1/2: bit patterns 0 .. 0x3f000000, each with both signs

@@ -9,11 +9,17 @@ bounds their comments state:
   * 2^f relative error <= 7.5e-5 for every fp32 f with |f| <= 1/2;
   * the same over the whole range -126 < x <= 127 (steps of 2^-10), and for
     x <= -126 (and x = -inf) a result in [0, 2^-125], never NaN or inf;
-  * tanh absolute error <= 2.5e-7 on +-10^[-8, 3] (log-spaced) and at 0.
+  * tanh absolute error <= 2.5e-7 on +-10^[-8, 3] (log-spaced) and at 0;
+  * the forward's folded softcap c tanh(x / s) + b (softcap_fma, the scale
+    2 log2(e) / s folded into one multiply) within c (2.5e-7 + 2^-22) plus
+    an ulp of c + |b| (the final rounding), for c, s = 50 (and the log2(e)
+    scaled c the kernel uses) over the same range of x / s.
 """
 import ctypes
 import os
 import subprocess
+
+import numpy as np
 
 import pytest
 import torch
@@ -36,6 +42,7 @@ def lib(tmp_path_factory):
     L.check_ex2_poly_reduced.argtypes = [vp, vp]
     L.check_ex2_poly_range.argtypes = [vp, d, d, i, vp]
     L.check_tanh.argtypes = [vp, d, d, i, vp]
+    L.check_softcap.argtypes = [vp, d, d, i, ctypes.c_float, ctypes.c_float, ctypes.c_float, vp]
     return L
 
 
@@ -69,3 +76,15 @@ def test_tanh_via_exp2_absolute_error(lib):
     print("tanh_via_exp2: max absolute error: %.3e" % w[0])
     assert w[1] == 0.0, "NaN result"
     assert w[0] <= 2.5e-7
+
+
+@pytest.mark.parametrize("c,b", [(50.0, 0.0), (50.0 * 1.4426950408889634, 0.0), (50.0 * 1.4426950408889634, -37.5)])
+def test_softcap_fma_absolute_error(lib, c, b):
+    n = 200000
+    w = _run(lib.check_softcap, ctypes.c_double(-8.0), ctypes.c_double(11.0 / n), n, ctypes.c_float(50.0),
+             ctypes.c_float(c), ctypes.c_float(b))
+    ulp = np.spacing(np.float32(c + abs(b)))
+    bound = c * (2.5e-7 + 2.0 ** -22) + float(ulp)
+    print("softcap_fma(c=%g, b=%g): max absolute error %.3e (bound %.3e)" % (c, b, w[0], bound))
+    assert w[1] == 0.0, "NaN result"
+    assert w[0] <= bound
