@@ -57,7 +57,7 @@ DECODE_READ_PER_KV_BYTE = 967959936.0 / 965165056.0  # (968,019,712 + 967,900,16
 # Forward: per-launch DRAM bytes of ncu captures of the forward kernel as it
 # stands, on the named workload; a workload without such a capture reports
 # None.
-FWD_TRAFFIC = {}
+FWD_TRAFFIC = {W.WINDOW_16K.name: 201630208.0 + 44653568.0}
 # Forward workloads timed one by one after the step (L2 flushed between launches).
 FWD_CONFIGS = [W.CAUSAL_2K, W.WINDOW_16K, W.WINDOW_Q4K_K16K, W.CAUSAL_Q4K_K16K, W.ALIBI_SOFTCAP]
 HEADLINE_FWD = W.WINDOW_16K
