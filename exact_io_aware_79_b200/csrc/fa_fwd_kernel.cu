@@ -604,20 +604,15 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
           const float x0 = __uint_as_float(s[c][2 * e]);
           const float x1 = __uint_as_float(s[c][2 * e + 1]);
           const uint64_t a2 = f2_fma(f2_pack(x0, x1), mul2, m2);
-          float p0, p1;
-          if ((e & 7) >= 5) {
-            // three pairs in eight take exp2 on the FMA pipe, so the MUFU is
-            // not the only unit doing exponentials
-            f2_unpack(ex2_poly_x2(a2), p0, p1);
-          } else {
-            float a0, a1;
-            f2_unpack(a2, a0, a1);
-            p0 = ex2(a0);
-            p1 = ex2(a1);
-          }
+          // every exponential on the MUFU (ex2.approx): the issue slots, not
+          // the MUFU, bound this loop, and a polynomial on the FMA pipe would
+          // cost about five times the issue slots
+          float a0, a1;
+          f2_unpack(a2, a0, a1);
+          float p0 = ex2(a0), p1 = ex2(a1);
           if (kMaskedTile) {
-            // masked entries hold -inf: the polynomial path would give a
-            // tiny nonzero value and -inf * 0 a NaN, so select them out
+            // masked entries hold -inf, and a zero scale makes -inf * 0 a
+            // NaN: select them out
             p0 = (x0 == -INFINITY) ? 0.0f : p0;
             p1 = (x1 == -INFINITY) ? 0.0f : p1;
           }

@@ -391,33 +391,6 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   return r;
 }
 
-// 2^x for a pair of floats on the FMA pipe, leaving the MUFU free. x is
-// clamped below at -126 and split as x = n + f with n = round(x) (adding and
-// subtracting 1.5 * 2^23 rounds to the nearest integer) and |f| <= 1/2; 2^f
-// comes from a cubic fitted here for least maximum relative error on
-// [-1/2, 1/2] (iteratively reweighted least squares; max relative error
-// 7.5e-5 in fp32 Horner form), and n is added to its exponent field (the low
-// bits of the rounded sum hold n, so shifting them left by 23 places n on the
-// exponent). Valid for x <= 127; x <= -126, -inf included, gives at most
-// 2^-125 (a subnormal or zero), never a wrapped sign.
-__device__ __forceinline__ uint64_t ex2_poly_x2(uint64_t x2) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  float a, b;
-  f2_unpack(x2, a, b);
-  const uint64_t xc = f2_pack(fmaxf(a, -126.0f), fmaxf(b, -126.0f));
-  const uint64_t t = f2_add(xc, f2_pack(kRound, kRound));
-  const uint64_t n = f2_add(t, f2_pack(-kRound, -kRound));
-  const uint64_t fr = f2_fma(n, f2_pack(-1.0f, -1.0f), xc);
-  uint64_t p = f2_fma(f2_pack(0x1.c3f76p-5f, 0x1.c3f76p-5f), fr, f2_pack(0x1.f0de1cp-3f, 0x1.f0de1cp-3f));
-  p = f2_fma(p, fr, f2_pack(0x1.62f31ap-1f, 0x1.62f31ap-1f));
-  p = f2_fma(p, fr, f2_pack(0x1.fff692p-1f, 0x1.fff692p-1f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
-                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
-}
-
 // tanh(y) = 1 - 2 / (exp(2y) + 1), with exp(2y) = 2^(2 y log2(e)).
 // Absolute error stays near 1e-7 over the whole range (exp2 and the
 // reciprocal are each accurate to a few ulp; the subtraction from 1 loses

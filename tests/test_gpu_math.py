@@ -1,14 +1,10 @@
 """The hand-written math inside the attention kernels, on its own.
 
-ex2_poly_x2 (2^x on the FMA pipe: a cubic for 2^f on |f| <= 1/2, the
-integer part added to the exponent field) and tanh_via_exp2 (the softcap's
-tanh) are evaluated by test-only kernels (tests/kernels/math_check.cu,
-compiled here with nvcc) on dense input sweeps, against fp64 exp2 / tanh
-evaluated on the device, and the worst errors are asserted against the
-bounds their comments state:
-  * 2^f relative error <= 7.5e-5 for every fp32 f with |f| <= 1/2;
-  * the same over the whole range -126 < x <= 127 (steps of 2^-10), and for
-    x <= -126 (and x = -inf) a result in [0, 2^-125], never NaN or inf;
+tanh_via_exp2 (the softcap's tanh in the decode and backward kernels) and
+softcap_fma (the forward's softcap) are evaluated by test-only kernels
+(tests/kernels/math_check.cu, compiled here with nvcc) on dense input
+sweeps, against fp64 tanh evaluated on the device, and the worst errors are
+asserted against the bounds their comments state:
   * tanh absolute error <= 2.5e-7 on +-10^[-8, 3] (log-spaced) and at 0;
   * the forward's folded softcap c tanh(x / s) + b (softcap_fma, the scale
     2 log2(e) / s folded into one multiply) within c (2.5e-7 + 2^-22) plus
@@ -39,8 +35,6 @@ def lib(tmp_path_factory):
                     os.path.join(HERE, "kernels", "math_check.cu")], check=True)
     L = ctypes.CDLL(out)
     vp, d, i = ctypes.c_void_p, ctypes.c_double, ctypes.c_int
-    L.check_ex2_poly_reduced.argtypes = [vp, vp]
-    L.check_ex2_poly_range.argtypes = [vp, d, d, i, vp]
     L.check_tanh.argtypes = [vp, d, d, i, vp]
     L.check_softcap.argtypes = [vp, d, d, i, ctypes.c_float, ctypes.c_float, ctypes.c_float, vp]
     return L
@@ -52,22 +46,6 @@ def _run(fn, *args):
     assert fn(ctypes.c_void_p(worst.data_ptr()), *args, ctypes.c_void_p(s.cuda_stream)) == 0
     torch.cuda.synchronize()
     return worst.cpu().tolist()
-
-
-def test_ex2_poly_every_reduced_argument(lib):
-    w = _run(lib.check_ex2_poly_reduced)
-    print("ex2_poly_x2: max relative error on |f| <= 1/2: %.3e" % w[0])
-    assert 0.0 < w[0] <= 7.5e-5
-
-
-def test_ex2_poly_whole_range_and_underflow(lib):
-    lo, step = -140.0, 2.0 ** -10
-    n = int((127.0 - lo) / step) + 1
-    w = _run(lib.check_ex2_poly_range, ctypes.c_double(lo), ctypes.c_double(step), n)
-    print("ex2_poly_x2: max relative error on (-126, 127]: %.3e; largest result below -126: %.3e" % (w[0], w[1]))
-    assert w[2] == 0.0, "NaN, negative or infinite result"
-    assert w[0] <= 7.5e-5 * (1 + 1e-3)
-    assert w[1] <= 2.0 ** -125
 
 
 def test_tanh_via_exp2_absolute_error(lib):
