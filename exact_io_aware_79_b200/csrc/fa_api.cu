@@ -351,6 +351,7 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* ou
   p.dq_acc = static_cast<float*>(workspace);
   p.dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                     ((rows * d * sizeof(float) + 255) & ~size_t(255)));
+  p.job_counter = reinterpret_cast<int*>(reinterpret_cast<char*>(p.dvec) + ((rows * sizeof(float) + 255) & ~size_t(255)));
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
@@ -651,7 +652,8 @@ fa_status fa_kvcache_append(const void* k_new, const void* v_new, void* k_cache,
 size_t fa_bwd_workspace_size(int B, int H, int Nq, int d) {
   if (B < 0 || H < 0 || Nq < 0 || d < 0) return 0;
   const size_t rows = static_cast<size_t>(B) * H * Nq;
-  return ((rows * d * sizeof(float) + 255) & ~size_t(255)) + ((rows * sizeof(float) + 255) & ~size_t(255));
+  // fp32 dQ accumulator, D, and the job counter of the tensor-core kernel
+  return ((rows * d * sizeof(float) + 255) & ~size_t(255)) + ((rows * sizeof(float) + 255) & ~size_t(255)) + 256;
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,

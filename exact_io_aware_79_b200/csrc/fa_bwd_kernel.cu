@@ -39,6 +39,7 @@
 //  * dQ = dS K: dS^T is stored to shared memory (row = key, column = query in
 //    the n-tile order above); ldmatrix.trans turns it into the A operand with
 //    queries as rows, K (rows = keys in natural order) is the B operand.
+#include "fa_bwd_common.cuh"
 #include "fa_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -95,6 +96,7 @@ __global__ void __launch_bounds__(256) bwd_rowdot_kernel(const BwdParams p) {
   }
 #pragma unroll
   for (int o = LPR / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && p.job_counter != nullptr) *p.job_counter = 0;
   if (row < rows && cl == 0) {
     // row = (b * Nq + i) * H + h  ->  dvec[(b * H + h) * Nq + i]
     const long long h = row % p.H, bi = row / p.H;
@@ -128,35 +130,6 @@ __device__ __forceinline__ bool key_visible(int pos, int j, int Nk, const BwdPar
 
 // Outside the deterministic mode the CTA also adds its dQ partials into the
 // fp32 accumulator; in it bwd_dq_kernel forms dQ instead.
-// Sequence b's lengths and first rows (packed layout), or the fixed-length
-// problem's; false when its offsets break the contract (the sequence is
-// skipped).
-__device__ __forceinline__ bool bwd_seq(const BwdParams& p, int b, int& Nq, int& Nk, long long& qrow,
-                                        long long& krow) {
-  if (p.cu_q == nullptr) {
-    Nq = p.Nq;
-    Nk = p.Nk;
-    qrow = static_cast<long long>(b) * p.Nq;
-    krow = static_cast<long long>(b) * p.Nk;
-    return true;
-  }
-  const int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
-  if (q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 > p.Nq) return false;
-  if (k0 < 0 || k1 < k0 || k1 > p.total_k || k1 - k0 > p.Nk) return false;
-  Nq = q1 - q0;
-  Nk = k1 - k0;
-  qrow = q0;
-  krow = k0;
-  return true;
-}
-
-// Index of (query head h, query q of this sequence) in lse and dvec:
-// [B, H, Nq] for fixed lengths, [H, total_q] packed.
-__device__ __forceinline__ size_t rowvec_index(const BwdParams& p, int b, int h, long long qrow, int q) {
-  return p.cu_q == nullptr ? (static_cast<size_t>(b) * p.H + h) * p.Nq + q
-                           : static_cast<size_t>(h) * p.total_q + static_cast<size_t>(qrow + q);
-}
-
 template <typename T, int D>
 __global__ void __launch_bounds__(kBwdWarps * 32, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -749,13 +722,18 @@ cudaError_t launch(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  using C = BwdCfg<D>;
-  auto kernel = bwd_kernel<T, D>;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-  if (e != cudaSuccess) return e;
-  dim3 grid((p.Nk + kBlk - 1) / kBlk, p.B * p.H_kv);
-  kernel<<<grid, kBwdWarps * 32, C::kSmem, stream>>>(tmQ, tmK, tmV, tmO, tmDQ, p);
-  e = cudaGetLastError();
+  if constexpr (D == 128) {
+    // the tensor-core kernel (its job counter was zeroed by the row-dot kernel)
+    e = launch_bwd_tc(std::is_same<T, __nv_bfloat16>::value, p, tmQ, tmK, tmV, tmO, tmDQ, stream);
+  } else {
+    using C = BwdCfg<D>;
+    auto kernel = bwd_kernel<T, D>;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((p.Nk + kBlk - 1) / kBlk, p.B * p.H_kv);
+    kernel<<<grid, kBwdWarps * 32, C::kSmem, stream>>>(tmQ, tmK, tmV, tmO, tmDQ, p);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
   if (p.deterministic) {
     using Cq = DqCfg<D>;

@@ -100,6 +100,7 @@ struct BwdParams {
   const float* lse;   // [B, H, Nq] (natural log, the forward's)
   float* dvec;        // [B, H, Nq] workspace: D_i = sum_c dO_ic O_ic
   float* dq_acc;      // [B, Nq, H, d] workspace: unscaled dQ in fp32
+  int* job_counter;   // workspace: next job of the tensor-core kernel (zeroed by the row-dot kernel)
   void* dq;           // [B, Nq, H, d]
   void* dk;           // [B, Nk, H_kv, d]
   void* dv;           // [B, Nk, H_kv, d]
@@ -125,6 +126,13 @@ struct BwdParams {
 cudaError_t launch_bwd(bool bf16, int d, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                        const CUtensorMap& tmV, const CUtensorMap& tmO, const CUtensorMap& tmDQ,
                        cudaStream_t stream);
+
+// The d = 128 key-block kernel on the tensor cores (dK, dV, and the dQ
+// partials unless p.deterministic): persistent CTAs claim jobs from
+// *p.job_counter, which must be zero at launch. The maps as for launch_bwd.
+cudaError_t launch_bwd_tc(bool bf16, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                          const CUtensorMap& tmV, const CUtensorMap& tmO, const CUtensorMap& tmDQ,
+                          cudaStream_t stream);
 
 // Writes n_new new tokens per sequence into the paged caches at positions
 // cache_seqlens[b] .. cache_seqlens[b] + n_new - 1.

@@ -315,7 +315,7 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
 
 // Instruction descriptor for kind::f16 with an fp32 accumulator.
 // bf16: both operands bf16 (else both fp16). b_mn_major: B is stored with its
-// N dimension contiguous (else K contiguous). A is always K-major.
+// N dimension contiguous (else K contiguous); A is K-major.
 __host__ __device__ constexpr uint32_t instr_desc_f16(bool bf16, int M, int N, bool b_mn_major) {
   return (1u << 4)                                    // D format: f32
          | ((bf16 ? 1u : 0u) << 7)                    // A format
@@ -323,6 +323,12 @@ __host__ __device__ constexpr uint32_t instr_desc_f16(bool bf16, int M, int N, b
          | ((b_mn_major ? 1u : 0u) << 16)             // B major
          | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
+}
+
+// The same with A stored M-major (its M dimension contiguous) when
+// a_mn_major (bit 15, the transpose-A flag).
+__host__ __device__ constexpr uint32_t instr_desc_f16_ab(bool bf16, int M, int N, bool a_mn_major, bool b_mn_major) {
+  return instr_desc_f16(bf16, M, N, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
 }
 
 // Instruction descriptor for kind::f8f6f4 with an fp32 accumulator: fmt 0 =

@@ -334,7 +334,8 @@ fa_status fa_kvcache_append(const void *k_new, const void *v_new, void *k_cache,
  *   k, v, dk, dv       [B, Nk, H_kv, d]    contiguous, dtype
  *   lse                [B, H, Nq]          fp32 (the forward's, natural log)
  *   workspace          fa_bwd_workspace_size(B, H, Nq, d) bytes of device
- *                      memory, 16-byte aligned (fp32 dq accumulator + D)
+ *                      memory, 16-byte aligned (fp32 dq accumulator, D, and
+ *                      the d = 128 kernel's job counter)
  *   scale, causal, window_left, window_right, alibi_slopes, softcap: as fa_fwd
  *   deterministic      0 or 1 (see above)
  * Outputs dq, dk, dv are overwritten (not accumulated). The caller owns every

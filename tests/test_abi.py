@@ -297,9 +297,9 @@ def test_bwd_validation(lib):
     assert bw(ws_bytes=lib.fa_bwd_workspace_size(2, 8, 100, 128) - 1) == WORKSPACE
     assert bw(B=0) == OK
     assert bw(Nq=0, ws=None, ws_bytes=0) == DEVICE   # zero dk, dv: no workspace needed
-    # fp32 dq accumulator rows (256-byte rounded) + D rows
+    # fp32 dq accumulator rows (256-byte rounded) + D rows + 256 bytes (the job counter)
     assert lib.fa_bwd_workspace_size(2, 8, 100, 128) == (2 * 8 * 100 * 128 * 4 + 255) // 256 * 256 + \
-        (2 * 8 * 100 * 4 + 255) // 256 * 256
+        (2 * 8 * 100 * 4 + 255) // 256 * 256 + 256
     assert lib.fa_bwd_workspace_size(-1, 8, 100, 128) == 0
 
 
