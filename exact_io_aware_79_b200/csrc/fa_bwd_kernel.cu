@@ -74,7 +74,8 @@ struct BwdCfg {
   static constexpr int kSmem = 1024 + kOffBar + 64;  // + slack to align to 1 KB
 };
 
-// D_i = sum_c dO_ic O_ic in fp32, [B, H, Nq].
+// D_i = sum_c dO_ic O_ic in fp32, [B, H, Nq]; outside the deterministic mode
+// the same threads zero the fp32 dQ accumulator's rows (their 8 columns).
 template <typename T, int D>
 __global__ void __launch_bounds__(256) bwd_rowdot_kernel(const BwdParams p) {
   constexpr int LPR = D / 8;  // lanes per row
@@ -87,6 +88,11 @@ __global__ void __launch_bounds__(256) bwd_rowdot_kernel(const BwdParams p) {
     const uint4 a = *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.dout) + off);
     const uint4 o = *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.out) + off);
     const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, ow[4] = {o.x, o.y, o.z, o.w};
+    if (!p.deterministic) {
+      float4* z = reinterpret_cast<float4*>(p.dq_acc + off);
+      z[0] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      z[1] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 x = unpack2<T>(aw[e]), y = unpack2<T>(ow[e]);
@@ -707,10 +713,6 @@ cudaError_t launch(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap
   const long long rows = (p.cu_q == nullptr ? static_cast<long long>(p.B) * p.Nq : p.total_q) * p.H;
   const long long elems = rows * D;
   cudaError_t e = cudaSuccess;
-  if (!p.deterministic) {
-    e = cudaMemsetAsync(p.dq_acc, 0, static_cast<size_t>(elems) * sizeof(float), stream);
-    if (e != cudaSuccess) return e;
-  }
   if (rows > 0) {
     const long long threads = rows * (D / 8);
     BwdParams pr = p;  // the row-dot kernel sees the packed layout as one sequence of total_q rows

@@ -14,9 +14,8 @@
 // fixed-order dQ, adds the dQ partials into an fp32 accumulator.
 //
 // A job is one block of 128 keys of one (sequence, cache head). CTAs are
-// persistent and claim jobs from a counter in the workspace, key block 0 of
-// every head first (under a causal mask the first key blocks see the most
-// queries, so the longest jobs start first). K and V of the job stay in
+// persistent and claim jobs from a counter in the workspace, in groups of a
+// few heads, key block first within a group (see tc_job). K and V of the job stay in
 // shared memory and dK, dV accumulate in tensor memory while the CTA walks,
 // 64 queries at a time, the query blocks of every query head that reads the
 // cache head and sees a key of the block. Per query block g:
@@ -32,7 +31,8 @@
 // One shared-memory dS^T tile serves as the K-major A of dK and as the
 // N-major B of dQ^T, and the K tile as the K-major A of S^T and the M-major
 // A of dQ^T, so neither is transposed. dQ^T (one TMEM lane per dimension,
-// one column per query) leaves through shared memory by TMA reduce-add.
+// one column per query) leaves through shared memory by TMA reduce-add into
+// the fp32 accumulator.
 //
 // Warps: 0-7 elementwise (warp w reads TMEM lanes 32 (w % 4) .. + 31, the
 // queries 32 (w / 4) .. + 31 of the block); 8-11 drain dQ^T and write dK,
@@ -45,7 +45,7 @@
 // dS^T tiles (16 KB), four fp32 dQ boxes of 32 dimensions x 64 queries
 // (8 KB each), the row vectors of two blocks, barriers.
 // Every wait is bounded; after a timeout the CTA stops, and the dK / dV rows
-// and the dQ boxes of the jobs it had claimed are written as NaN.
+// and the dQ partials of the jobs it had claimed are written as NaN.
 #include "fa_bwd_common.cuh"
 #include "fa_internal.h"
 #include "sm100_ptx.cuh"
@@ -77,8 +77,13 @@ constexpr int kOffK = 0;
 constexpr int kOffV = kTileKV;
 constexpr int kOffQ = 2 * kTileKV;
 constexpr int kOffO = kOffQ + kStages * kTileQ;
+constexpr int kDsBufs = 2;  // dS^T tiles
+// a block's Q / dO stage and dS^T tile are freed by the same blk_done phase,
+// which the producer has already seen for block g - kStages when block g
+// is loaded
+static_assert(kDsBufs <= kStages && kStages < kRing, "stage and dS^T reuse outrun the barrier ring");
 constexpr int kOffS = kOffO + kStages * kTileQ;
-constexpr int kOffDQ = kOffS + 2 * kTileS;
+constexpr int kOffDQ = kOffS + kDsBufs * kTileS;  // four fp32 dQ boxes of 32 dimensions x 64 queries
 constexpr int kOffRow = kOffDQ + 4 * 8192;
 constexpr int kOffBar = kOffRow + 2 * 2 * kQb * 4;
 constexpr int kBarBytes = 512;
@@ -89,8 +94,7 @@ struct TcBars {
   uint64_t q_full[kStages];
   uint64_t s_ready[kRing];   // S^T, dP^T of block g complete
   uint64_t p_ready[kRing];   // P^T in TMEM, dS^T in shared memory (elementwise warps)
-  uint64_t p_free[kRing];    // dV of block g complete: its S^T columns are free
-  uint64_t dq_ready[kRing];  // dQ^T of block g complete
+  uint64_t p_free[kRing];    // dV (and dQ^T) of block g complete: its S^T columns are free, dQ^T is ready
   uint64_t dq_free[kRing];   // dQ^T of block g read out of TMEM (drain warps)
   uint64_t blk_done[kRing];  // every product of block g complete: its Q / dO stage and dS^T tile are free
   uint64_t acc_ready;        // dK, dV of the job complete (one phase per job with blocks)
@@ -120,9 +124,19 @@ struct TcJob {
   long long qrow, krow;
 };
 
-// Jobs are numbered key block first: j = kb * (B * H_kv) + b * H_kv + hk.
-__device__ __forceinline__ void tc_job(const BwdParams& p, int j, TcJob& J) {
-  const int bh = j % (p.B * p.H_kv), kb = j / (p.B * p.H_kv);
+// Jobs are numbered in groups of up to kHeadGroup (sequence, cache head)
+// pairs, key block first within a group: the CTAs running at one time work
+// on the key blocks of a few heads, so the Q / dO tiles and dQ rows those
+// heads share stay in L2, and the longest jobs of a group (under a causal
+// mask, its first key blocks) come first.
+constexpr int kHeadGroup = 8;
+
+__device__ __forceinline__ void tc_job(const BwdParams& p, int n_kb, int j, TcJob& J) {
+  const int BH = p.B * p.H_kv;
+  const int grp = j / (n_kb * kHeadGroup);
+  const int rem = j - grp * n_kb * kHeadGroup;
+  const int gs = min(kHeadGroup, BH - grp * kHeadGroup);
+  const int kb = rem / gs, bh = grp * kHeadGroup + rem % gs;
   J.b = bh / p.H_kv;
   J.hk = bh % p.H_kv;
   J.k0 = kb * kKeys;
@@ -179,7 +193,7 @@ __device__ __forceinline__ int take_job_warp(TcBars* bars, int t, int lane, bool
 
 __device__ void tc_producer(const BwdParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                             const CUtensorMap* tmV, const CUtensorMap* tmO, uint8_t* smem, TcBars* bars,
-                            int total_jobs) {
+                            int n_kb, int total_jobs) {
   volatile int* abort = &bars->abort;
   const uint64_t pol = l2_policy_evict_last();
   auto load_q = [&](int gi, int h, int q0, int tq0, int tb) -> bool {
@@ -206,7 +220,7 @@ __device__ void tc_producer(const BwdParams& p, const CUtensorMap* tmQ, const CU
     mbar_arrive(&bars->job_full[slot]);
     if (j < 0) break;
     TcJob J;
-    tc_job(p, j, J);
+    tc_job(p, n_kb, j, J);
     if (J.n <= 0) continue;
     const int n = J.n, g0 = nq;
     // the first two query blocks, then K and V (they wait for the previous
@@ -247,7 +261,7 @@ __device__ void tc_producer(const BwdParams& p, const CUtensorMap* tmQ, const CU
 // ---------------------------------------------------------------- MMA issuer
 
 template <typename T, bool kDq>
-__device__ void tc_mma(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t tmem) {
+__device__ void tc_mma(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t tmem, int n_kb) {
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t idesc_s = instr_desc_f16(kBf16, kKeys, kQb, false);     // S^T, dP^T
   constexpr uint32_t idesc_kv = instr_desc_f16(kBf16, kKeys, kD, true);      // dV, dK
@@ -264,12 +278,11 @@ __device__ void tc_mma(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t
   int g = 0, a = 0;
   auto sdp = [&](int x) -> bool {
     const int st = x % kStages, b = x & 1;
+    // S^T(x) goes over P^T(x - 2) (read by dV(x - 2)), dP^T(x) over
+    // dQ^T(x - 2) (read out by the drain warps); S^T is issued as soon as it
+    // may be, so the tensor pipe has it while the drain finishes
     if (!mbar_wait(&bars->q_full[st], (x / kStages) & 1, abort)) return false;
-    if (x >= 2) {
-      // S^T(x) goes over P^T(x - 2), dP^T(x) over dQ^T(x - 2)
-      if (!mbar_wait(&bars->p_free[(x - 2) % kRing], ((x - 2) / kRing) & 1, abort)) return false;
-      if (kDq && !mbar_wait(&bars->dq_free[(x - 2) % kRing], ((x - 2) / kRing) & 1, abort)) return false;
-    }
+    if (x >= 2 && !mbar_wait(&bars->p_free[(x - 2) % kRing], ((x - 2) / kRing) & 1, abort)) return false;
     tc_fence_after();
     const uint64_t qd = smem_desc_sw128(sb + kOffQ + st * kTileQ, 16, 1024);
     const uint64_t od = smem_desc_sw128(sb + kOffO + st * kTileQ, 16, 1024);
@@ -279,6 +292,8 @@ __device__ void tc_mma(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t
       const uint32_t oa = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4, ob = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
       mma_ss(ts, kdesc + oa, qd + ob, idesc_s, kk > 0 ? 1u : 0u);
     }
+    if (kDq && x >= 2 && !mbar_wait(&bars->dq_free[(x - 2) % kRing], ((x - 2) / kRing) & 1, abort)) return false;
+    tc_fence_after();
 #pragma unroll
     for (int kk = 0; kk < kD / 16; ++kk) {
       const uint32_t oa = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4, ob = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
@@ -291,7 +306,7 @@ __device__ void tc_mma(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t
     const int j = take_job(bars, t, &failed);
     if (j < 0) break;
     TcJob J;
-    tc_job(p, j, J);
+    tc_job(p, n_kb, j, J);
     if (J.n <= 0) continue;
     const int n = J.n;
     if (!mbar_wait(&bars->kv_full, a & 1, abort) || !sdp(g) || (n > 1 && !sdp(g + 1))) {
@@ -309,21 +324,22 @@ __device__ void tc_mma(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t
       const uint32_t ts = tmem + kColR + 128 * b;
       const uint64_t od_mn = smem_desc_sw128(sb + kOffO + st * kTileQ, 8192, 1024);
       const uint64_t qd_mn = smem_desc_sw128(sb + kOffQ + st * kTileQ, 8192, 1024);
-      const uint64_t ds = smem_desc_sw128(sb + kOffS + b * kTileS, 16, 1024);
-      const uint64_t ds_mn = smem_desc_sw128(sb + kOffS + b * kTileS, 8192, 1024);
+      const uint64_t ds = smem_desc_sw128(sb + kOffS + (gi % kDsBufs) * kTileS, 16, 1024);
+      const uint64_t ds_mn = smem_desc_sw128(sb + kOffS + (gi % kDsBufs) * kTileS, 8192, 1024);
       // dV += P^T dO: the 16 queries of step kk are TMEM columns 32 (kk / 2) + 8 (kk % 2) ..
 #pragma unroll
       for (int kk = 0; kk < kQb / 16; ++kk)
         mma_ts(tmem + kColDV, ts + 32 * (kk >> 1) + 8 * (kk & 1), od_mn + ((kk * 2048) >> 4), idesc_kv,
                (u > 0 || kk > 0) ? 1u : 0u);
-      tc_commit(&bars->p_free[gi % kRing]);
       if constexpr (kDq) {
         // dQ^T = K^T dS^T over the 128 keys, into the dP^T columns
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
           mma_ss(ts + 64, ktdesc + ((kk * 2048) >> 4), ds_mn + ((kk * 2048) >> 4), idesc_q, kk > 0 ? 1u : 0u);
-        tc_commit(&bars->dq_ready[gi % kRing]);
       }
+      // one commit point for both: the S^T columns are free (dV read P^T)
+      // and dQ^T is complete (every commit point costs the tensor pipe time)
+      tc_commit(&bars->p_free[gi % kRing]);
       // dK += dS^T Q
 #pragma unroll
       for (int kk = 0; kk < kQb / 16; ++kk)
@@ -348,25 +364,26 @@ __device__ void tc_mma(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t
 
 // ---------------------------------------------------------------- elementwise
 
-// P^T and dS^T of 32 queries (columns c = 0..31 of this warp's half) for
+// P^T and dS^T of 8 queries (columns c0 .. c0 + 7 of this warp's 32) for
 // this thread's key: s, dp the fp32 bits of S^T and dP^T; lsen = -LSE log2 e
 // and dneg = -D of the 32 queries; visible columns lo..hi (masked blocks);
-// dist0 = (position of query 0) - key (ALiBi).
+// dist0 = (position of query 0) - key (ALiBi). Packed pairs -> pw, dsw.
 template <typename T, bool kCap, bool kAlibi, bool kMasked>
-__device__ __forceinline__ void ew_math(const BwdParams& p, const uint32_t (&s)[32], const uint32_t (&dp)[32],
-                                        const float* lsen, const float* dneg, float slope2, float dist0, int lo,
-                                        int hi, uint32_t (&pw)[16], uint32_t (&dsw)[16]) {
+__device__ __forceinline__ void ew_math8(const BwdParams& p, int c0, const uint32_t (&s)[32],
+                                         const uint32_t (&dp)[32], const float* lsen, const float* dneg,
+                                         float slope2, float dist0, int lo, int hi, uint32_t (&pw)[4],
+                                         uint32_t (&dsw)[4]) {
 #pragma unroll
-  for (int c = 0; c < 32; c += 4) {
-    const float4 ln4 = *reinterpret_cast<const float4*>(lsen + c);
-    const float4 dn4 = *reinterpret_cast<const float4*>(dneg + c);
+  for (int c = 0; c < 8; c += 4) {
+    const float4 ln4 = *reinterpret_cast<const float4*>(lsen + c0 + c);
+    const float4 dn4 = *reinterpret_cast<const float4*>(dneg + c0 + c);
     const float ln[4] = {ln4.x, ln4.y, ln4.z, ln4.w}, dn[4] = {dn4.x, dn4.y, dn4.z, dn4.w};
 #pragma unroll
     for (int e = 0; e < 4; e += 2) {
       float pr[2], dv[2];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const int cc = c + e + i;
+        const int cc = c0 + c + e + i;
         const float x = __uint_as_float(s[cc]);
         float l2, f = 1.0f;
         if constexpr (kCap) {
@@ -390,19 +407,34 @@ __device__ __forceinline__ void ew_math(const BwdParams& p, const uint32_t (&s)[
   }
 }
 
+// All 32 queries of this thread: P^T to TMEM (tp: this half's first S^T
+// column), dS^T to its shared-memory row (drow), 8 queries at a time.
+template <typename T, bool kCap, bool kAlibi, bool kMasked>
+__device__ __forceinline__ void ew_block(const BwdParams& p, const uint32_t (&s)[32], const uint32_t (&dp)[32],
+                                         const float* lsen, const float* dneg, float slope2, float dist0, int lo,
+                                         int hi, uint32_t tp, uint8_t* drow, int half, int row) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t pw[4], dsw[4];
+    ew_math8<T, kCap, kAlibi, kMasked>(p, 8 * i, s, dp, lsen, dneg, slope2, dist0, lo, hi, pw, dsw);
+    tmem_st4(tp + 4 * i, pw[0], pw[1], pw[2], pw[3]);
+    *reinterpret_cast<uint4*>(drow + ((((4 * half + i) ^ (row & 7))) << 4)) = make_uint4(dsw[0], dsw[1], dsw[2], dsw[3]);
+  }
+}
+
 template <typename T, bool kCap, bool kAlibi>
-__device__ __forceinline__ void ew_math_any(bool masked, const BwdParams& p, const uint32_t (&s)[32],
-                                            const uint32_t (&dp)[32], const float* lsen, const float* dneg,
-                                            float slope2, float dist0, int lo, int hi, uint32_t (&pw)[16],
-                                            uint32_t (&dsw)[16]) {
+__device__ __forceinline__ void ew_block_any(bool masked, const BwdParams& p, const uint32_t (&s)[32],
+                                             const uint32_t (&dp)[32], const float* lsen, const float* dneg,
+                                             float slope2, float dist0, int lo, int hi, uint32_t tp, uint8_t* drow,
+                                             int half, int row) {
   if (masked)
-    ew_math<T, kCap, kAlibi, true>(p, s, dp, lsen, dneg, slope2, dist0, lo, hi, pw, dsw);
+    ew_block<T, kCap, kAlibi, true>(p, s, dp, lsen, dneg, slope2, dist0, lo, hi, tp, drow, half, row);
   else
-    ew_math<T, kCap, kAlibi, false>(p, s, dp, lsen, dneg, slope2, dist0, lo, hi, pw, dsw);
+    ew_block<T, kCap, kAlibi, false>(p, s, dp, lsen, dneg, slope2, dist0, lo, hi, tp, drow, half, row);
 }
 
 template <typename T>
-__device__ void tc_elementwise(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t tmem, int warp,
+__device__ void tc_elementwise(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t tmem, int n_kb, int warp,
                                int lane) {
   volatile int* abort = &bars->abort;
   const int quarter = warp & 3, half = warp >> 2;
@@ -419,19 +451,22 @@ __device__ void tc_elementwise(const BwdParams& p, uint8_t* smem, TcBars* bars, 
     const int j = take_job_warp(bars, t, lane, &failed);
     if (j < 0) break;
     TcJob J;
-    tc_job(p, j, J);
+    tc_job(p, n_kb, j, J);
     if (J.n <= 0) continue;
     const int n = J.n;
     const int key = J.k0 + row;
-    // row vector entry of block u for this thread (et < 128)
+    // row vector entry of block u for this thread (et < 128): LSE of query
+    // et (et < 64) or D of query et - 64, as loaded; the value is only
+    // transformed when it is stored a block later, so the load stays in
+    // flight meanwhile
     auto fetch = [&](int u) -> float {
       int h, q0;
       tc_block(p, J, u, h, q0);
       const int q = q0 + (et & (kQb - 1));
       if (et >= 2 * kQb) return 0.0f;
-      if (q >= J.Nq) return et < kQb ? -INFINITY : 0.0f;
+      if (q >= J.Nq) return et < kQb ? INFINITY : 0.0f;
       const size_t ri = rowvec_index(p, J.b, h, J.qrow, q);
-      return et < kQb ? -p.lse[ri] * kLog2e : -p.dvec[ri];
+      return et < kQb ? p.lse[ri] : p.dvec[ri];
     };
     float rv = fetch(0);
     for (int u = 0; u < n; ++u) {
@@ -447,7 +482,7 @@ __device__ void tc_elementwise(const BwdParams& p, uint8_t* smem, TcBars* bars, 
       // the slot's previous block (gi - 2) before S^T(gi) could be computed
       // (that product waited for dV(gi - 2), which waited for all of them).
       if (warp < 4) {
-        srow[b * 2 * kQb + et] = rv;
+        srow[b * 2 * kQb + et] = et < kQb ? -rv * kLog2e : -rv;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->rv_ready[b]);
       }
@@ -457,6 +492,13 @@ __device__ void tc_elementwise(const BwdParams& p, uint8_t* smem, TcBars* bars, 
         break;
       }
       if (u + 1 < n) rv = fetch(u + 1);
+      // dS^T tile gi % kDsBufs was last read by the products of block gi - kDsBufs
+      ok = gi < kDsBufs ||
+           mbar_wait(&bars->blk_done[(gi - kDsBufs) % kRing], ((gi - kDsBufs) / kRing) & 1, abort);
+      if (__any_sync(0xffffffffu, !ok)) {
+        failed = true;
+        break;
+      }
       tc_fence_after();
       uint32_t s[32], dp[32];
       tmem_ld32(tl + kColR + 128 * b + 32 * half, s);
@@ -478,26 +520,15 @@ __device__ void tc_elementwise(const BwdParams& p, uint8_t* smem, TcBars* bars, 
       tmem_wait_ld();
       reg_fence(s);
       reg_fence(dp);
-      uint32_t pw[16], dsw[16];
+      const uint32_t tp = tl + kColR + 128 * b + 32 * half;  // P^T over this half's first S^T columns
+      uint8_t* drow = sds + (gi % kDsBufs) * kTileS + row * 128;
       if (p.use_softcap) {
-        if (alibi) ew_math_any<T, true, true>(!full, p, s, dp, lsen, dneg, slope2, dist0, lo, hi, pw, dsw);
-        else ew_math_any<T, true, false>(!full, p, s, dp, lsen, dneg, slope2, dist0, lo, hi, pw, dsw);
+        if (alibi) ew_block_any<T, true, true>(!full, p, s, dp, lsen, dneg, slope2, dist0, lo, hi, tp, drow, half, row);
+        else ew_block_any<T, true, false>(!full, p, s, dp, lsen, dneg, slope2, dist0, lo, hi, tp, drow, half, row);
       } else {
-        if (alibi) ew_math_any<T, false, true>(!full, p, s, dp, lsen, dneg, slope2, dist0, lo, hi, pw, dsw);
-        else ew_math_any<T, false, false>(!full, p, s, dp, lsen, dneg, slope2, dist0, lo, hi, pw, dsw);
+        if (alibi) ew_block_any<T, false, true>(!full, p, s, dp, lsen, dneg, slope2, dist0, lo, hi, tp, drow, half, row);
+        else ew_block_any<T, false, false>(!full, p, s, dp, lsen, dneg, slope2, dist0, lo, hi, tp, drow, half, row);
       }
-      tmem_st16(tl + kColR + 128 * b + 32 * half, pw);
-      // dS^T tile b was last read by the products of block gi - 2
-      ok = gi < 2 || mbar_wait(&bars->blk_done[(gi - 2) % kRing], ((gi - 2) / kRing) & 1, abort);
-      if (__any_sync(0xffffffffu, !ok)) {
-        failed = true;
-        break;
-      }
-      uint8_t* drow = sds + b * kTileS + row * 128;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<uint4*>(drow + ((((4 * half + i) ^ (row & 7))) << 4)) =
-            make_uint4(dsw[4 * i], dsw[4 * i + 1], dsw[4 * i + 2], dsw[4 * i + 3]);
       tmem_wait_st();
       fence_proxy_async_shared();
       tc_fence_before();
@@ -526,7 +557,7 @@ __device__ __forceinline__ void store_row16(T* dst, const uint32_t (&r)[32], flo
 
 template <typename T, bool kDq>
 __device__ void tc_drain(const BwdParams& p, const CUtensorMap* tmDQ, uint8_t* smem, TcBars* bars, uint32_t tmem,
-                         int wq, int lane) {
+                         int n_kb, int wq, int lane) {
   volatile int* abort = &bars->abort;
   const uint32_t tl = tmem + (static_cast<uint32_t>(32 * wq) << 16);
   float* stage = reinterpret_cast<float*>(smem + kOffDQ + wq * 8192);
@@ -537,7 +568,7 @@ __device__ void tc_drain(const BwdParams& p, const CUtensorMap* tmDQ, uint8_t* s
     const int j = take_job_warp(bars, t, lane, &tfail);
     if (j < 0) break;  // no job left, or none published after a failure
     TcJob J;
-    tc_job(p, j, J);
+    tc_job(p, n_kb, j, J);
     if (J.n < 0) continue;
     const int key = J.k0 + 32 * wq + lane;
     T* dk_row = reinterpret_cast<T*>(p.dk) + static_cast<size_t>(J.krow + key) * p.dkv_tok +
@@ -565,15 +596,18 @@ __device__ void tc_drain(const BwdParams& p, const CUtensorMap* tmDQ, uint8_t* s
         int h, q0;
         tc_block(p, J, u, h, q0);
         if (!failed) {
-          const bool ok = mbar_wait(&bars->dq_ready[gi % kRing], (gi / kRing) & 1, abort);
+          const bool ok = mbar_wait(&bars->p_free[gi % kRing], (gi / kRing) & 1, abort);
           failed = __any_sync(0xffffffffu, !ok);
         }
-        if (lane == 0) bulk_wait_read_all();  // this warp's previous reduce has read the box
+        if (lane == 0) bulk_wait_read_all();  // this warp's previous reduce has read its box
         __syncwarp();
         if (!failed) tc_fence_after();
         // box row q (query), dimension 32 wq + lane: 16-byte chunk lane / 4 of
         // the 128-byte row, swizzled by q % 8; 32 queries at a time
         const uint32_t col = kColR + 128 * (gi & 1) + 64;
+        uint32_t pa[8];  // shared address of this lane's word in rows q = 0..7 (mod 8)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) pa[k] = smem_addr(stage) + k * 128 + ((((lane >> 2) ^ k)) << 4) + 4 * (lane & 3);
 #pragma unroll 1
         for (int hq = 0; hq < 2; ++hq) {
           uint32_t r[32];
@@ -591,8 +625,7 @@ __device__ void tc_drain(const BwdParams& p, const CUtensorMap* tmDQ, uint8_t* s
           const float nan = __int_as_float(0x7fc00000);
 #pragma unroll
           for (int q = 0; q < 32; ++q)
-            stage[(32 * hq + q) * 32 + ((((lane >> 2) ^ (q & 7))) << 2) + (lane & 3)] =
-                failed ? nan : __uint_as_float(r[q]);
+            st_shared_f32(pa[q & 7] + (32 * hq + (q & ~7)) * 128, failed ? nan : __uint_as_float(r[q]));
         }
         fence_proxy_async_shared();
         __syncwarp();
@@ -608,20 +641,18 @@ __device__ void tc_drain(const BwdParams& p, const CUtensorMap* tmDQ, uint8_t* s
       failed = __any_sync(0xffffffffu, !ok);
     }
     if (!failed) tc_fence_after();
+    // 32 columns at a time: dV's four pieces, then dK's (scaled)
 #pragma unroll 1
-    for (int c = 0; c < kD / 32; ++c) {
-      uint32_t rv[32], rk[32];
+    for (int c = 0; c < 2 * kD / 32; ++c) {
+      const bool is_k = c >= kD / 32;
+      const int cc = is_k ? c - kD / 32 : c;
+      uint32_t r[32];
       if (!failed) {
-        tmem_ld32(tl + kColDV + 32 * c, rv);
-        tmem_ld32(tl + kColDK + 32 * c, rk);
+        tmem_ld32(tl + (is_k ? kColDK : kColDV) + 32 * cc, r);
         tmem_wait_ld();
-        reg_fence(rv);
-        reg_fence(rk);
+        reg_fence(r);
       }
-      if (key < J.Nk) {
-        store_row16<T>(dv_row + 32 * c, rv, 1.0f, failed);
-        store_row16<T>(dk_row + 32 * c, rk, p.scale, failed);
-      }
+      if (key < J.Nk) store_row16<T>((is_k ? dk_row : dv_row) + 32 * cc, r, is_k ? p.scale : 1.0f, failed);
     }
     tc_fence_before();
     __syncwarp();
@@ -638,7 +669,7 @@ template <typename T, bool kDq>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                  const __grid_constant__ CUtensorMap tmDQ, const BwdParams p, int total_jobs) {
+                  const __grid_constant__ CUtensorMap tmDQ, const BwdParams p, int n_kb, int total_jobs) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   TcBars* bars = reinterpret_cast<TcBars*>(smem + kOffBar);
@@ -650,7 +681,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->s_ready[i], 1);
       mbar_init(&bars->p_ready[i], kEwWarps);
       mbar_init(&bars->p_free[i], 1);
-      mbar_init(&bars->dq_ready[i], 1);
       mbar_init(&bars->dq_free[i], 4);
       mbar_init(&bars->blk_done[i], 1);
     }
@@ -683,13 +713,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp < kEwWarps) {
-    tc_elementwise<T>(p, smem, bars, tmem, warp, lane);
+    tc_elementwise<T>(p, smem, bars, tmem, n_kb, warp, lane);
   } else if (warp < kDrainWarp0 + 4) {
-    tc_drain<T, kDq>(p, &tmDQ, smem, bars, tmem, warp & 3, lane);
+    tc_drain<T, kDq>(p, &tmDQ, smem, bars, tmem, n_kb, warp & 3, lane);
   } else if (warp == kProdWarp) {
-    if (lane == 0) tc_producer(p, &tmQ, &tmK, &tmV, &tmO, smem, bars, total_jobs);
+    if (lane == 0) tc_producer(p, &tmQ, &tmK, &tmV, &tmO, smem, bars, n_kb, total_jobs);
   } else if (warp == kMmaWarp) {
-    if (lane == 0) tc_mma<T, kDq>(p, smem, bars, tmem);
+    if (lane == 0) tc_mma<T, kDq>(p, smem, bars, tmem, n_kb);
   }
 
   tc_fence_before();
@@ -721,7 +751,8 @@ cudaError_t launch_tc(const BwdParams& p, const CUtensorMap& tmQ, const CUtensor
   if (jobs == 0) return cudaSuccess;
   if (jobs > 0x7fffffffLL) return cudaErrorInvalidValue;
   const int grid = static_cast<int>(jobs < sm_count[dev] ? jobs : sm_count[dev]);
-  kernel<<<grid, kThreads, kSmem, stream>>>(tmQ, tmK, tmV, tmO, tmDQ, p, static_cast<int>(jobs));
+  kernel<<<grid, kThreads, kSmem, stream>>>(tmQ, tmK, tmV, tmO, tmDQ, p, static_cast<int>(n_kb),
+                                            static_cast<int>(jobs));
   return cudaGetLastError();
 }
 

@@ -128,8 +128,10 @@ cudaError_t launch_bwd(bool bf16, int d, const BwdParams& p, const CUtensorMap& 
                        cudaStream_t stream);
 
 // The d = 128 key-block kernel on the tensor cores (dK, dV, and the dQ
-// partials unless p.deterministic): persistent CTAs claim jobs from
-// *p.job_counter, which must be zero at launch. The maps as for launch_bwd.
+// partials added into p.dq_acc by TMA reduce-add through tmDQ unless
+// p.deterministic): persistent CTAs claim jobs
+// from *p.job_counter, which must be zero at launch. The maps as for
+// launch_bwd.
 cudaError_t launch_bwd_tc(bool bf16, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                           const CUtensorMap& tmV, const CUtensorMap& tmO, const CUtensorMap& tmDQ,
                           cudaStream_t stream);
