@@ -15,7 +15,8 @@ Both inputs exceed the 126 MB L2 (forward Q+K+V 201 MB, decode K/V 34 GB),
 so no explicit flush is needed between iterations. After the timed steps
 every forward workload of the suite (causal 2K, window 16K, window and causal
 Nq 4K / Nk 16K, ALiBi + softcap) is timed on its own with L2 flushed between
-launches and reported under "forward_configs".
+launches and reported under "forward_configs", and the backward pass (causal
+2K in both dQ modes, window 16K, ALiBi + softcap) under "backward_configs".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
   python bench.py --sweep          # every forward workload and decode split
@@ -57,7 +58,11 @@ DECODE_READ_PER_KV_BYTE = 967959936.0 / 965165056.0  # (968,019,712 + 967,900,16
 # Forward: per-launch DRAM bytes of ncu captures of the forward kernel as it
 # stands, on the named workload; a workload without such a capture reports
 # None.
-FWD_TRAFFIC = {W.WINDOW_16K.name: 201630208.0 + 44653568.0}
+FWD_TRAFFIC = {W.WINDOW_16K.name: 201685248.0 + 45675776.0}
+# Backward workloads timed after the step (atomic dQ, and the deterministic
+# mode on the first); credited 2.5 x the forward's flops (five products of
+# the forward's size against two).
+BWD_CONFIGS = [W.CAUSAL_2K, W.WINDOW_16K, W.ALIBI_SOFTCAP]
 # Forward workloads timed one by one after the step (L2 flushed between launches).
 FWD_CONFIGS = [W.CAUSAL_2K, W.WINDOW_16K, W.WINDOW_Q4K_K16K, W.CAUSAL_Q4K_K16K, W.ALIBI_SOFTCAP]
 HEADLINE_FWD = W.WINDOW_16K
@@ -347,6 +352,8 @@ def gpu_arm(args):
 
     # ---- every forward workload on its own (L2 flushed between launches)
     fwd_configs = time_fwd_configs(fa, dev, world, peaks, args, physical_gpu(local))
+    # ---- the backward pass on its workloads (L2 flushed between calls)
+    bwd_configs = time_bwd_configs(fa, dev, world, peaks, args, physical_gpu(local))
 
     # ---- end to end through the public API with pinned host buffers
     hq, hk, hv = (x[n].cpu().pin_memory() for n in ("q", "k", "v"))
@@ -436,7 +443,7 @@ def gpu_arm(args):
             "decode": {"B": dw.B, "H": dw.H, "d": dw.d, "page_size": dw.page_size,
                        "seqlens": [dw.len_lo, dw.len_hi], "num_splits": splits, "kv_bytes_per_launch": KVB},
             "l2": "step: inputs larger than L2 (forward Q+K+V 201 MB, decode K/V 34 GB), no flush; "
-                  "forward_configs: L2 flushed (256 MB write) before every launch",
+                  "forward_configs, backward_configs: L2 flushed (256 MB write) before every call",
             "parallelism": "replicas" if world > 1 else "single GPU",
         },
         "roofline": {"kernel": "decode (split + merge)", "bound": "hbm", "achieved": round(dec_gbs / world, 1),
@@ -452,6 +459,7 @@ def gpu_arm(args):
                          "traffic_source": "ncu capture of this workload",
                          "peak_source": peak_src + " burst"},
         "forward_configs": fwd_configs,
+        "backward_configs": bwd_configs,
         "decode": {"value": round(dec_gbs, 1), "unit": "GB/s", "ms_per_launch": round(dec_ms, 4)},
         "fwd_ms_per_launch": round(fwd_ms, 4),
         "e2e": {"value": round(world * F / (e_fwd_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
@@ -538,6 +546,58 @@ def time_fwd_configs(fa, dev, world, peaks, args, gpu_index):
     t1 = time.time()
     sampler.stop()
     res["peak"] = "measured burst bf16 %.1f TFLOP/s (fp8: %.0f x that)" % (peaks["bf16_tflops"], FP8_OVER_BF16)
+    res["clocks"] = sampler.summary(t0, t1)
+    del flush
+    return res
+
+
+def time_bwd_configs(fa, dev, world, peaks, args, gpu_index):
+    """Times fa_bwd (row-dot kernel, the key-block kernel, and the dQ cast or
+    the deterministic dQ pass) on BWD_CONFIGS like time_fwd_configs: L2
+    flushed before each timed call, median of the CUDA-event times."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    res = {}
+    sampler = ClockSampler(gpu_index)
+    sampler.start()
+    t0 = time.time()
+    for i, w in enumerate(BWD_CONFIGS):
+        x = W.make_fwd_inputs(w, device=dev)
+        gen = torch.Generator().manual_seed(w.seed + 100)
+        dout = torch.randn(x["q"].shape, generator=gen).to(w.dtype).to(dev)
+        out = torch.empty_like(x["q"])
+        lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+        fa.fa_fwd(x["q"], x["k"], x["v"], out, lse, w.scale, w.causal, w.window_left, w.window_right,
+                  x["slopes"], w.softcap)
+        dq, dk, dv = torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"])
+        ws = torch.empty(max(fa.fa_bwd_workspace_size(w.B, w.H, w.Nq, w.d), 16), dtype=torch.uint8, device=dev)
+        for det in ((False, True) if i == 0 else (False,)):
+            run = lambda: fa.fa_bwd(x["q"], x["k"], x["v"], out, lse, dout, dq, dk, dv, w.scale, w.causal,
+                                    w.window_left, w.window_right, x["slopes"], w.softcap, deterministic=det,
+                                    workspace=ws)
+            for _ in range(max(3, args.warmup)):
+                run()
+            times = []
+            n = max(5, min(args.steps, args.config_steps))
+            barrier(world)
+            for _ in range(n):
+                flush.zero_()
+                a, b = ev(), ev()
+                a.record()
+                run()
+                b.record()
+                times.append((a, b))
+            torch.cuda.synchronize()
+            ms = max_over_ranks(statistics.median([a.elapsed_time(b) for a, b in times]), world, dev)
+            fl = 2.5 * fwd_flops(w)
+            tf = weak_scaling_value(fl, ms * 1e-3, world) / 1e12
+            res[("deterministic_" if det else "") + w.name] = {
+                "ms": round(ms, 4), "TFLOP/s": round(tf, 1), "frac": round(tf / world / peaks["bf16_tflops"], 4),
+                "flops_per_call": fl, "launches": n}
+        del x, dout, out, lse, dq, dk, dv, ws
+    t1 = time.time()
+    sampler.stop()
+    res["peak"] = "measured burst bf16 %.1f TFLOP/s" % peaks["bf16_tflops"]
     res["clocks"] = sampler.summary(t0, t1)
     del flush
     return res
