@@ -1,9 +1,11 @@
-// fa_bwd_common.cuh -- indexing shared by the backward kernels: a sequence's
-// lengths and first rows (fixed-length or packed layout) and the position of
-// a (query head, query) in the LSE and D row vectors.
+// fa_bwd_common.cuh -- shared by the backward kernels: a sequence's lengths
+// and first rows (fixed-length or packed layout), the position of a (query
+// head, query) in the LSE and D row vectors, and the job-claim ring of the
+// persistent tensor-core kernels.
 #pragma once
 
 #include "fa_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace fa {
 
@@ -42,6 +44,59 @@ __device__ __forceinline__ size_t rowvec_index(const BwdParams& p, int b, int h,
 __device__ __forceinline__ int bwd_right_bound(const BwdParams& p) {
   if (p.window_right >= 0) return p.causal ? min(0, p.window_right) : p.window_right;
   return p.causal ? 0 : -1;
+}
+
+// ---- persistent kernels: jobs claimed from a counter, broadcast through
+// a ring of job ids (Bars: job_full[kJobRing], job_empty[kJobRing] mbarriers,
+// int job_id[kJobRing], int abort)
+
+constexpr int kJobRing = 4;
+
+// Job t of this CTA from the claim ring (every user reads every slot once
+// and then frees it); -1 when the grid has no job left or the wait failed
+// (then *failed is set and the slot is not freed). One thread.
+template <typename Bars>
+__device__ __forceinline__ int take_job(Bars* bars, int t, bool* failed) {
+  const int slot = t % kJobRing;
+  if (!mbar_wait(&bars->job_full[slot], (t / kJobRing) & 1, &bars->abort)) {
+    *failed = true;
+    return -1;
+  }
+  const int j = *reinterpret_cast<volatile int*>(&bars->job_id[slot]);
+  mbar_arrive(&bars->job_empty[slot]);
+  return j;
+}
+
+// The same for a whole warp: lane 0 takes the job, every lane gets it.
+template <typename Bars>
+__device__ __forceinline__ int take_job_warp(Bars* bars, int t, int lane, bool* failed) {
+  bool f = false;
+  int j = -1;
+  if (lane == 0) j = take_job(bars, t, &f);
+  j = __shfl_sync(0xffffffffu, j, 0);
+  if (__shfl_sync(0xffffffffu, f ? 1 : 0, 0)) *failed = true;
+  return j;
+}
+
+// Claims the next job for slot t of the ring (after its previous users
+// freed it) and publishes it; -1 once the counter passes total_jobs (that
+// is published too, so every user stops). False if the wait failed.
+template <typename Bars>
+__device__ __forceinline__ bool publish_job(Bars* bars, int* counter, int total_jobs, int t, int* job) {
+  const int slot = t % kJobRing;
+  if (t >= kJobRing && !mbar_wait(&bars->job_empty[slot], ((t / kJobRing) - 1) & 1, &bars->abort)) return false;
+  int j = atomicAdd(counter, 1);
+  if (j >= total_jobs) j = -1;
+  bars->job_id[slot] = j;
+  mbar_arrive(&bars->job_full[slot]);
+  *job = j;
+  return true;
+}
+
+// A bounded wait that ignores the abort flag (draining work in flight).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  int dummy = 0;
+  mbar_wait(bar, parity, &dummy);
 }
 
 }  // namespace fa

@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(256) bwd_rowdot_kernel(const BwdParams p) {
   }
 #pragma unroll
   for (int o = LPR / 2; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && p.job_counter != nullptr) *p.job_counter = 0;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && p.job_counter != nullptr) p.job_counter[0] = p.job_counter[1] = 0;
   if (row < rows && cl == 0) {
     // row = (b * Nq + i) * H + h  ->  dvec[(b * H + h) * Nq + i]
     const long long h = row % p.H, bi = row / p.H;
@@ -738,6 +738,9 @@ cudaError_t launch(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap
   }
   if (e != cudaSuccess) return e;
   if (p.deterministic) {
+    // the fixed-order dQ pass: on the tensor cores for d = 128 (its job
+    // counter was zeroed by the row-dot kernel), warp-level otherwise
+    if constexpr (D == 128) return launch_bwd_dq_tc(std::is_same<T, __nv_bfloat16>::value, p, tmQ, tmK, tmV, tmO, stream);
     using Cq = DqCfg<D>;
     auto dq_kernel = bwd_dq_kernel<T, D>;
     e = cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cq::kSmem);

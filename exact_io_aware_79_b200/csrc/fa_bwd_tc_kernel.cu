@@ -60,7 +60,6 @@ constexpr int kKeys = 128;  // keys per job
 constexpr int kQb = 64;     // queries per block
 constexpr int kStages = 3;  // Q / dO stages
 constexpr int kRing = 4;    // per-block barrier rings
-constexpr int kJobRing = 4;
 constexpr int kEwWarps = 8;
 constexpr int kDrainWarp0 = 8;
 constexpr int kProdWarp = 12;
@@ -109,11 +108,6 @@ struct TcBars {
 };
 static_assert(sizeof(TcBars) <= kBarBytes, "barrier block exceeds its reserve");
 static_assert(kSmem <= 232448, "shared memory budget exceeded");
-
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-  int dummy = 0;
-  mbar_wait(bar, parity, &dummy);
-}
 
 // One job: key block kb of (sequence b, cache head hk), with the query
 // blocks (of kQb queries) that can see one of its keys.
@@ -165,29 +159,6 @@ __device__ __forceinline__ void tc_block(const BwdParams& p, const TcJob& J, int
   q0 = (J.qb_lo + u % J.n_qb) * kQb;
 }
 
-// Job t of this CTA from the claim ring (every user reads every slot once
-// and then frees it); -1 when the grid has no job left or the wait failed
-// (then *failed is set and the slot is not freed). One thread.
-__device__ __forceinline__ int take_job(TcBars* bars, int t, bool* failed) {
-  const int slot = t % kJobRing;
-  if (!mbar_wait(&bars->job_full[slot], (t / kJobRing) & 1, &bars->abort)) {
-    *failed = true;
-    return -1;
-  }
-  const int j = *reinterpret_cast<volatile int*>(&bars->job_id[slot]);
-  mbar_arrive(&bars->job_empty[slot]);
-  return j;
-}
-
-// The same for a whole warp: lane 0 takes the job, every lane gets it.
-__device__ __forceinline__ int take_job_warp(TcBars* bars, int t, int lane, bool* failed) {
-  bool f = false;
-  int j = -1;
-  if (lane == 0) j = take_job(bars, t, &f);
-  j = __shfl_sync(0xffffffffu, j, 0);
-  if (__shfl_sync(0xffffffffu, f ? 1 : 0, 0)) *failed = true;
-  return j;
-}
 
 // ---------------------------------------------------------------- producer
 
@@ -212,13 +183,8 @@ __device__ void tc_producer(const BwdParams& p, const CUtensorMap* tmQ, const CU
   bool ok = true;
   int nq = 0, a = 0;  // Q / dO stages and K / V tiles loaded so far (blocks are numbered by nq)
   for (int t = 0; ok; ++t) {
-    const int slot = t % kJobRing;
-    if (t >= kJobRing && !mbar_wait(&bars->job_empty[slot], ((t / kJobRing) - 1) & 1, abort)) break;
-    int j = atomicAdd(p.job_counter, 1);
-    if (j >= total_jobs) j = -1;
-    bars->job_id[slot] = j;
-    mbar_arrive(&bars->job_full[slot]);
-    if (j < 0) break;
+    int j;
+    if (!publish_job(bars, p.job_counter, total_jobs, t, &j) || j < 0) break;
     TcJob J;
     tc_job(p, n_kb, j, J);
     if (J.n <= 0) continue;

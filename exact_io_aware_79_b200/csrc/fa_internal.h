@@ -100,7 +100,8 @@ struct BwdParams {
   const float* lse;   // [B, H, Nq] (natural log, the forward's)
   float* dvec;        // [B, H, Nq] workspace: D_i = sum_c dO_ic O_ic
   float* dq_acc;      // [B, Nq, H, d] workspace: unscaled dQ in fp32
-  int* job_counter;   // workspace: next job of the tensor-core kernel (zeroed by the row-dot kernel)
+  int* job_counter;   // workspace: next job of the tensor-core kernels, [0] key blocks, [1] dQ tiles
+                      // (zeroed by the row-dot kernel)
   void* dq;           // [B, Nq, H, d]
   void* dk;           // [B, Nk, H_kv, d]
   void* dv;           // [B, Nk, H_kv, d]
@@ -135,6 +136,13 @@ cudaError_t launch_bwd(bool bf16, int d, const BwdParams& p, const CUtensorMap& 
 cudaError_t launch_bwd_tc(bool bf16, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                           const CUtensorMap& tmV, const CUtensorMap& tmO, const CUtensorMap& tmDQ,
                           cudaStream_t stream);
+
+// The deterministic mode's dQ pass for d = 128 on the tensor cores: dq =
+// scale * sum over key blocks (fixed order) of dS K, written to p.dq;
+// persistent CTAs claim 128-query tiles from p.job_counter[1], which must be
+// zero at launch. The maps as for launch_bwd.
+cudaError_t launch_bwd_dq_tc(bool bf16, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                             const CUtensorMap& tmV, const CUtensorMap& tmO, cudaStream_t stream);
 
 // Writes n_new new tokens per sequence into the paged caches at positions
 // cache_seqlens[b] .. cache_seqlens[b] + n_new - 1.
