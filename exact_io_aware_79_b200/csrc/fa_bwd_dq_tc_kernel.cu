@@ -1,5 +1,5 @@
 // fa_bwd_dq_tc_kernel.cu -- the deterministic backward's dQ pass on the
-// Blackwell tensor cores, head dimension 128.
+// Blackwell tensor cores, head dimensions 64 and 128.
 //
 // The pages name a deterministic backward ("Flash-Attention v2.0 到 v2.7
 // 更新", section v2.4; "FlashAttention深度解析：从算法创新到产业变革的全面影响",
@@ -22,7 +22,7 @@
 //   dQ += dS K     M = 128 queries, N = d, K = 64 keys        A from TMEM, B = K d-major
 // S and dP take one of three 128-column TMEM buffers (the buffer of block g
 // is its K/V stage, so the barrier that frees a K/V stage frees the buffer);
-// dQ accumulates in columns 0..127 and is scaled, rounded and stored by the
+// dQ accumulates in columns 0..d-1 and is scaled, rounded and stored by the
 // elementwise warps at the end of the job.
 //
 // Warps: 0-7 elementwise (warp w: TMEM lanes 32 (w % 4) .., keys 32 (w / 4)
@@ -42,7 +42,6 @@
 namespace fa {
 namespace {
 
-constexpr int kD = 128;
 constexpr int kBM = 128;  // queries per job
 constexpr int kBN = 64;   // keys per block
 constexpr int kStages = 3;
@@ -56,8 +55,9 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDQ = 0, kColBuf = 128;  // buffer s: S at 128 + 128 s, dP at + 64
 constexpr int kHeadGroup = 8;
 
-constexpr int kTileQ = kBM * kD * 2;  // 32 KB: 64-column chunks of 16 KB
-constexpr int kTileK = kBN * kD * 2;  // 16 KB: 64-column chunks of 8 KB
+// Shared-memory regions are sized for d = 128 (d = 64 fills half of each)
+constexpr int kTileQ = kBM * 128 * 2;  // 32 KB: 64-column chunks of 16 KB
+constexpr int kTileK = kBN * 128 * 2;  // 16 KB: 64-column chunks of 8 KB
 constexpr int kOffQ = 0;
 constexpr int kOffO = 2 * kTileQ;
 constexpr int kOffK = 4 * kTileQ;
@@ -125,6 +125,7 @@ __device__ __forceinline__ void dq_job(const BwdParams& p, int n_qt, int j, DqJo
 
 // ---------------------------------------------------------------- producer
 
+template <int D>
 __device__ void dq_producer(const BwdParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                             const CUtensorMap* tmV, const CUtensorMap* tmO, uint8_t* smem, DqBars* bars,
                             int n_qt, int total_jobs) {
@@ -140,9 +141,9 @@ __device__ void dq_producer(const BwdParams& p, const CUtensorMap* tmQ, const CU
     if (J.n <= 0) continue;
     const int qb = a % 2;
     if (a >= 2 && !mbar_wait(&bars->q_free[qb], ((a - 2) / 2) & 1, abort)) break;
-    mbar_arrive_expect_tx(&bars->q_full[qb], 2 * kTileQ);
+    mbar_arrive_expect_tx(&bars->q_full[qb], 2 * kBM * D * 2);
 #pragma unroll
-    for (int c = 0; c < kD / 64; ++c) {
+    for (int c = 0; c < D / 64; ++c) {
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         tma_load_4d(tmQ, &bars->q_full[qb], smem + kOffQ + qb * kTileQ + c * 16384 + r * 8192, 64 * c, J.h,
@@ -158,10 +159,10 @@ __device__ void dq_producer(const BwdParams& p, const CUtensorMap* tmQ, const CU
         ok = false;
         break;
       }
-      mbar_arrive_expect_tx(&bars->kv_full[st], 2 * kTileK);
+      mbar_arrive_expect_tx(&bars->kv_full[st], 2 * kBN * D * 2);
       const int k0 = (J.kb_lo + u) * kBN;
 #pragma unroll
-      for (int c = 0; c < kD / 64; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         tma_load_4d(tmK, &bars->kv_full[st], smem + kOffK + st * kTileK + c * 8192, 64 * c, J.hk, J.tk0 + k0, J.tb,
                     pol);
         tma_load_4d(tmV, &bars->kv_full[st], smem + kOffV + st * kTileK + c * 8192, 64 * c, J.hk, J.tk0 + k0, J.tb,
@@ -177,11 +178,11 @@ __device__ void dq_producer(const BwdParams& p, const CUtensorMap* tmQ, const CU
 
 // ---------------------------------------------------------------- MMA issuer
 
-template <typename T>
+template <typename T, int D>
 __device__ void dq_mma(const BwdParams& p, uint8_t* smem, DqBars* bars, uint32_t tmem, int n_qt) {
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t idesc_s = instr_desc_f16(kBf16, kBM, kBN, false);  // S, dP
-  constexpr uint32_t idesc_q = instr_desc_f16(kBf16, kBM, kD, true);    // dQ: B = K d-major
+  constexpr uint32_t idesc_q = instr_desc_f16(kBf16, kBM, D, true);     // dQ: B = K d-major
   volatile int* abort = &bars->abort;
   const uint32_t sb = smem_addr(smem);
   bool failed = false;
@@ -197,12 +198,12 @@ __device__ void dq_mma(const BwdParams& p, uint8_t* smem, DqBars* bars, uint32_t
     const uint64_t vd = smem_desc_sw128(sb + kOffV + st * kTileK, 16, 1024);
     const uint32_t ts = tmem + kColBuf + 128 * st;
 #pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk) {
+    for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t oa = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4, ob = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
       mma_ss(ts, qd + oa, kd + ob, idesc_s, kk > 0 ? 1u : 0u);
     }
 #pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk) {
+    for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t oa = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4, ob = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
       mma_ss(ts + 64, od + oa, vd + ob, idesc_s, kk > 0 ? 1u : 0u);
     }
@@ -322,7 +323,7 @@ __device__ __forceinline__ void store_dq32(T* dst, const uint32_t (&r)[32], floa
     reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
 }
 
-template <typename T>
+template <typename T, int D>
 __device__ void dq_elementwise(const BwdParams& p, DqBars* bars, uint32_t tmem, int n_qt, int warp, int lane) {
   volatile int* abort = &bars->abort;
   const int quarter = warp & 3, half = warp >> 2;
@@ -341,14 +342,14 @@ __device__ void dq_elementwise(const BwdParams& p, DqBars* bars, uint32_t tmem, 
     if (J.n < 0) continue;
     const int q = J.q0 + row;
     T* dq_row = reinterpret_cast<T*>(p.dq) + static_cast<size_t>(J.qrow + q) * p.dq_tok +
-                static_cast<size_t>(J.h) * kD + 64 * half;
+                static_cast<size_t>(J.h) * D + (D / 2) * half;
     if (J.n == 0) {
       // no key visible to the tile: dQ = 0 (NaN after a failure)
       uint32_t z[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) z[i] = 0u;
       if (q < J.Nq)
-        for (int c = 0; c < 2; ++c) store_dq32<T>(dq_row + 32 * c, z, 1.0f, failed ? 2 : 1);
+        for (int c = 0; c < D / 64; ++c) store_dq32<T>(dq_row + 32 * c, z, 1.0f, failed ? 2 : 1);
       continue;
     }
     const int n = J.n;
@@ -396,17 +397,17 @@ __device__ void dq_elementwise(const BwdParams& p, DqBars* bars, uint32_t tmem, 
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->ds_ready[gi % kRing]);
     }
-    // the job's dQ: this warp's 32 rows, columns 64 half .. + 63
+    // the job's dQ: this warp's 32 rows, columns (d / 2) half .. + d / 2 - 1
     if (!failed) {
       const bool ok = mbar_wait(&bars->acc_ready, a & 1, abort);
       failed = __any_sync(0xffffffffu, !ok);
     }
     if (!failed) tc_fence_after();
 #pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < D / 64; ++c) {
       uint32_t r[32];
       if (!failed) {
-        tmem_ld32(tl + kColDQ + 64 * half + 32 * c, r);
+        tmem_ld32(tl + kColDQ + (D / 2) * half + 32 * c, r);
         tmem_wait_ld();
         reg_fence(r);
       }
@@ -422,7 +423,7 @@ __device__ void dq_elementwise(const BwdParams& p, DqBars* bars, uint32_t tmem, 
 
 // ---------------------------------------------------------------- kernel
 
-template <typename T>
+template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -470,11 +471,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp < kEwWarps) {
-    dq_elementwise<T>(p, bars, tmem, n_qt, warp, lane);
+    dq_elementwise<T, D>(p, bars, tmem, n_qt, warp, lane);
   } else if (warp == kProdWarp) {
-    if (lane == 0) dq_producer(p, &tmQ, &tmK, &tmV, &tmO, smem, bars, n_qt, total_jobs);
+    if (lane == 0) dq_producer<D>(p, &tmQ, &tmK, &tmV, &tmO, smem, bars, n_qt, total_jobs);
   } else if (warp == kMmaWarp) {
-    if (lane == 0) dq_mma<T>(p, smem, bars, tmem, n_qt);
+    if (lane == 0) dq_mma<T, D>(p, smem, bars, tmem, n_qt);
   }
 
   tc_fence_before();
@@ -486,10 +487,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <typename T>
+template <typename T, int D>
 cudaError_t launch_dq(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                       const CUtensorMap& tmO, cudaStream_t stream) {
-  auto kernel = bwd_dq_tc_kernel<T>;
+  auto kernel = bwd_dq_tc_kernel<T, D>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   static int sm_count[64];
@@ -512,10 +513,13 @@ cudaError_t launch_dq(const BwdParams& p, const CUtensorMap& tmQ, const CUtensor
 
 }  // namespace
 
-cudaError_t launch_bwd_dq_tc(bool bf16, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+cudaError_t launch_bwd_dq_tc(bool bf16, int d, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, const CUtensorMap& tmO, cudaStream_t stream) {
-  return bf16 ? launch_dq<__nv_bfloat16>(p, tmQ, tmK, tmV, tmO, stream)
-              : launch_dq<__half>(p, tmQ, tmK, tmV, tmO, stream);
+  if (d == 128)
+    return bf16 ? launch_dq<__nv_bfloat16, 128>(p, tmQ, tmK, tmV, tmO, stream)
+                : launch_dq<__half, 128>(p, tmQ, tmK, tmV, tmO, stream);
+  return bf16 ? launch_dq<__nv_bfloat16, 64>(p, tmQ, tmK, tmV, tmO, stream)
+              : launch_dq<__half, 64>(p, tmQ, tmK, tmV, tmO, stream);
 }
 
 }  // namespace fa

@@ -1,6 +1,6 @@
 // fa_bwd_tc_kernel.cu -- the backward pass's main kernel on the Blackwell
 // tensor cores (tcgen05 products with TMEM accumulators, TMA tiles), head
-// dimension 128.
+// dimensions 64 and 128.
 //
 // It computes the gradient of the forward's definition (the pages name the
 // backward pass: "FlashAttention深度解析：从算法创新到产业变革的全面影响",
@@ -27,6 +27,8 @@
 //     16-bit rows of 64 queries (128-byte swizzle)
 //   dV  += P^T dO    M = 128 keys, N = d, K = 64 queries      A in TMEM, B = dO d-major
 //   dQ^T = K^T dS^T  M = d, N = 64 queries, K = 128 keys      A = K d-major, B = dS^T query-major
+//                    (d = 64: an M = 128 product whose rows 64..127 read the
+//                    V tile after K and are never used)
 //   dK  += dS^T Q    M = 128 keys, N = d, K = 64 queries      A = dS^T, B = Q d-major
 // One shared-memory dS^T tile serves as the K-major A of dK and as the
 // N-major B of dQ^T, and the K tile as the K-major A of S^T and the M-major
@@ -38,12 +40,13 @@
 // queries 32 (w / 4) .. + 31 of the block); 8-11 drain dQ^T and write dK,
 // dV at the end of a job; 12 the TMA producer (and job claims); 13 the MMA
 // issuer (one thread, owns TMEM).
-// TMEM: dV [0, 128), dK [128, 256); for block parity b, S^T in
-// [256 + 128 b, + 64) with P^T over it, dP^T in [320 + 128 b, + 64) with dQ^T
+// TMEM: dV [0, d), dK [d, 2 d); for block parity b, S^T in
+// [2 d + 128 b, + 64) with P^T over it, dP^T 64 columns further with dQ^T
 // over it once the elementwise warps have read dP^T.
-// Shared memory: K, V (32 KB each), three Q / dO stages (16 KB each), two
-// dS^T tiles (16 KB), four fp32 dQ boxes of 32 dimensions x 64 queries
-// (8 KB each), the row vectors of two blocks, barriers.
+// Shared memory (d = 128): K, V (32 KB each), three Q / dO stages (16 KB
+// each), two dS^T tiles (16 KB), four fp32 dQ boxes of 32 dimensions x 64
+// queries (8 KB each), the row vectors of two blocks, barriers; d = 64
+// halves the K, V, Q, dO and dQ parts.
 // Every wait is bounded; after a timeout the CTA stops, and the dK / dV rows
 // and the dQ partials of the jobs it had claimed are written as NaN.
 #include "fa_bwd_common.cuh"
@@ -55,7 +58,6 @@
 namespace fa {
 namespace {
 
-constexpr int kD = 128;
 constexpr int kKeys = 128;  // keys per job
 constexpr int kQb = 64;     // queries per block
 constexpr int kStages = 3;  // Q / dO stages
@@ -67,26 +69,36 @@ constexpr int kMmaWarp = 13;
 constexpr int kThreads = 14 * 32;
 constexpr int kJobUsers = 1 + kEwWarps + 4;  // MMA thread, elementwise warps, drain warps
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColDV = 0, kColDK = 128, kColR = 256;
-
-constexpr int kTileKV = kKeys * kD * 2;  // 32 KB: 64-column chunks of 16 KB
-constexpr int kTileQ = kQb * kD * 2;     // 16 KB: 64-column chunks of 8 KB
 constexpr int kTileS = kKeys * kQb * 2;  // 16 KB: 128 rows of 128 bytes
-constexpr int kOffK = 0;
-constexpr int kOffV = kTileKV;
-constexpr int kOffQ = 2 * kTileKV;
-constexpr int kOffO = kOffQ + kStages * kTileQ;
 constexpr int kDsBufs = 2;  // dS^T tiles
 // a block's Q / dO stage and dS^T tile are freed by the same blk_done phase,
 // which the producer has already seen for block g - kStages when block g
 // is loaded
 static_assert(kDsBufs <= kStages && kStages < kRing, "stage and dS^T reuse outrun the barrier ring");
-constexpr int kOffS = kOffO + kStages * kTileQ;
-constexpr int kOffDQ = kOffS + kDsBufs * kTileS;  // four fp32 dQ boxes of 32 dimensions x 64 queries
-constexpr int kOffRow = kOffDQ + 4 * 8192;
-constexpr int kOffBar = kOffRow + 2 * 2 * kQb * 4;
 constexpr int kBarBytes = 512;
-constexpr int kSmem = kOffBar + kBarBytes + 1024;  // + slack to align to 1 KB
+
+// Layout for head dimension D (64 or 128).
+template <int D>
+struct TcCfg {
+  static constexpr int kTileKV = kKeys * D * 2;  // K or V: D / 64 chunks of 16 KB (128 rows of 128 bytes)
+  static constexpr int kTileQ = kQb * D * 2;     // a Q or dO stage: D / 64 chunks of 8 KB
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kTileKV;
+  static constexpr int kOffQ = 2 * kTileKV;
+  static constexpr int kOffO = kOffQ + kStages * kTileQ;
+  static constexpr int kOffS = kOffO + kStages * kTileQ;
+  static constexpr int kOffDQ = kOffS + kDsBufs * kTileS;  // D / 32 fp32 dQ boxes of 32 dimensions x 64 queries
+  static constexpr int kOffRow = kOffDQ + (D / 32) * 8192;
+  static constexpr int kOffBar = kOffRow + 2 * 2 * kQb * 4;
+  static constexpr int kSmem = kOffBar + kBarBytes + 1024;  // + slack to align to 1 KB
+  // TMEM: dV [0, D), dK [D, 2 D), then per block parity b S^T at 2 D + 128 b
+  // and dP^T (later dQ^T) 64 columns further
+  static constexpr uint32_t kColDV = 0, kColDK = D, kColR = 2 * D;
+  // dQ^T has D rows (TMEM lanes); the drain warps holding them
+  static constexpr int kDqWarps = D / 32;
+  static_assert(kSmem <= 232448, "shared memory budget exceeded");
+  static_assert(kColR + 256 <= 512, "TMEM budget exceeded");
+};
 
 struct TcBars {
   uint64_t kv_full;
@@ -107,7 +119,6 @@ struct TcBars {
   int abort;
 };
 static_assert(sizeof(TcBars) <= kBarBytes, "barrier block exceeds its reserve");
-static_assert(kSmem <= 232448, "shared memory budget exceeded");
 
 // One job: key block kb of (sequence b, cache head hk), with the query
 // blocks (of kQb queries) that can see one of its keys.
@@ -162,9 +173,11 @@ __device__ __forceinline__ void tc_block(const BwdParams& p, const TcJob& J, int
 
 // ---------------------------------------------------------------- producer
 
+template <int D>
 __device__ void tc_producer(const BwdParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK,
                             const CUtensorMap* tmV, const CUtensorMap* tmO, uint8_t* smem, TcBars* bars,
                             int n_kb, int total_jobs) {
+  using C = TcCfg<D>;
   volatile int* abort = &bars->abort;
   const uint64_t pol = l2_policy_evict_last();
   auto load_q = [&](int gi, int h, int q0, int tq0, int tb) -> bool {
@@ -172,11 +185,11 @@ __device__ void tc_producer(const BwdParams& p, const CUtensorMap* tmQ, const CU
     // the stage's previous block (gi - kStages) must be done with it
     if (gi >= kStages && !mbar_wait(&bars->blk_done[(gi - kStages) % kRing], ((gi - kStages) / kRing) & 1, abort))
       return false;
-    mbar_arrive_expect_tx(&bars->q_full[st], 2 * kTileQ);
+    mbar_arrive_expect_tx(&bars->q_full[st], 2 * C::kTileQ);
 #pragma unroll
-    for (int c = 0; c < kD / 64; ++c) {
-      tma_load_4d(tmQ, &bars->q_full[st], smem + kOffQ + st * kTileQ + c * 8192, 64 * c, h, tq0 + q0, tb, pol);
-      tma_load_4d(tmO, &bars->q_full[st], smem + kOffO + st * kTileQ + c * 8192, 64 * c, h, tq0 + q0, tb, pol);
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_4d(tmQ, &bars->q_full[st], smem + C::kOffQ + st * C::kTileQ + c * 8192, 64 * c, h, tq0 + q0, tb, pol);
+      tma_load_4d(tmO, &bars->q_full[st], smem + C::kOffO + st * C::kTileQ + c * 8192, 64 * c, h, tq0 + q0, tb, pol);
     }
     return true;
   };
@@ -198,14 +211,14 @@ __device__ void tc_producer(const BwdParams& p, const CUtensorMap* tmQ, const CU
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&bars->kv_full, 2 * kTileKV);
+        mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTileKV);
 #pragma unroll
-        for (int c = 0; c < kD / 64; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
-            tma_load_4d(tmK, &bars->kv_full, smem + kOffK + c * 16384 + r * 8192, 64 * c, J.hk,
+            tma_load_4d(tmK, &bars->kv_full, smem + C::kOffK + c * 16384 + r * 8192, 64 * c, J.hk,
                         J.tk0 + J.k0 + 64 * r, J.tb, pol);
-            tma_load_4d(tmV, &bars->kv_full, smem + kOffV + c * 16384 + r * 8192, 64 * c, J.hk,
+            tma_load_4d(tmV, &bars->kv_full, smem + C::kOffV + c * 16384 + r * 8192, 64 * c, J.hk,
                         J.tk0 + J.k0 + 64 * r, J.tb, pol);
           }
         }
@@ -226,20 +239,23 @@ __device__ void tc_producer(const BwdParams& p, const CUtensorMap* tmQ, const CU
 
 // ---------------------------------------------------------------- MMA issuer
 
-template <typename T, bool kDq>
+template <typename T, int D, bool kDq>
 __device__ void tc_mma(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t tmem, int n_kb) {
+  using C = TcCfg<D>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr uint32_t idesc_s = instr_desc_f16(kBf16, kKeys, kQb, false);     // S^T, dP^T
-  constexpr uint32_t idesc_kv = instr_desc_f16(kBf16, kKeys, kD, true);      // dV, dK
-  constexpr uint32_t idesc_q = instr_desc_f16_ab(kBf16, kD, kQb, true, true);  // dQ^T
+  constexpr uint32_t idesc_kv = instr_desc_f16(kBf16, kKeys, D, true);       // dV, dK
+  // dQ^T always as an M = 128 product: for D = 64 its rows 64..127 come from
+  // the V tile that follows K (16 KB on) and are never read
+  constexpr uint32_t idesc_q = instr_desc_f16_ab(kBf16, 128, kQb, true, true);
   volatile int* abort = &bars->abort;
   const uint32_t sb = smem_addr(smem);
   // K-major descriptors step K by 32 bytes within a 128-byte row (and by a
   // whole chunk every 4 steps); the d-major / query-major ones step K by 16
   // rows of 128 bytes (2048 bytes)
-  const uint64_t kdesc = smem_desc_sw128(sb + kOffK, 16, 1024);
-  const uint64_t vdesc = smem_desc_sw128(sb + kOffV, 16, 1024);
-  const uint64_t ktdesc = smem_desc_sw128(sb + kOffK, 16384, 1024);
+  const uint64_t kdesc = smem_desc_sw128(sb + C::kOffK, 16, 1024);
+  const uint64_t vdesc = smem_desc_sw128(sb + C::kOffV, 16, 1024);
+  const uint64_t ktdesc = smem_desc_sw128(sb + C::kOffK, 16384, 1024);
   bool failed = false;
   int g = 0, a = 0;
   auto sdp = [&](int x) -> bool {
@@ -250,18 +266,18 @@ __device__ void tc_mma(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t
     if (!mbar_wait(&bars->q_full[st], (x / kStages) & 1, abort)) return false;
     if (x >= 2 && !mbar_wait(&bars->p_free[(x - 2) % kRing], ((x - 2) / kRing) & 1, abort)) return false;
     tc_fence_after();
-    const uint64_t qd = smem_desc_sw128(sb + kOffQ + st * kTileQ, 16, 1024);
-    const uint64_t od = smem_desc_sw128(sb + kOffO + st * kTileQ, 16, 1024);
-    const uint32_t ts = tmem + kColR + 128 * b;
+    const uint64_t qd = smem_desc_sw128(sb + C::kOffQ + st * C::kTileQ, 16, 1024);
+    const uint64_t od = smem_desc_sw128(sb + C::kOffO + st * C::kTileQ, 16, 1024);
+    const uint32_t ts = tmem + C::kColR + 128 * b;
 #pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk) {
+    for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t oa = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4, ob = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
       mma_ss(ts, kdesc + oa, qd + ob, idesc_s, kk > 0 ? 1u : 0u);
     }
     if (kDq && x >= 2 && !mbar_wait(&bars->dq_free[(x - 2) % kRing], ((x - 2) / kRing) & 1, abort)) return false;
     tc_fence_after();
 #pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk) {
+    for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t oa = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4, ob = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
       mma_ss(ts + 64, vdesc + oa, od + ob, idesc_s, kk > 0 ? 1u : 0u);
     }
@@ -287,15 +303,15 @@ __device__ void tc_mma(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t
         break;
       }
       tc_fence_after();
-      const uint32_t ts = tmem + kColR + 128 * b;
-      const uint64_t od_mn = smem_desc_sw128(sb + kOffO + st * kTileQ, 8192, 1024);
-      const uint64_t qd_mn = smem_desc_sw128(sb + kOffQ + st * kTileQ, 8192, 1024);
-      const uint64_t ds = smem_desc_sw128(sb + kOffS + (gi % kDsBufs) * kTileS, 16, 1024);
-      const uint64_t ds_mn = smem_desc_sw128(sb + kOffS + (gi % kDsBufs) * kTileS, 8192, 1024);
+      const uint32_t ts = tmem + C::kColR + 128 * b;
+      const uint64_t od_mn = smem_desc_sw128(sb + C::kOffO + st * C::kTileQ, 8192, 1024);
+      const uint64_t qd_mn = smem_desc_sw128(sb + C::kOffQ + st * C::kTileQ, 8192, 1024);
+      const uint64_t ds = smem_desc_sw128(sb + C::kOffS + (gi % kDsBufs) * kTileS, 16, 1024);
+      const uint64_t ds_mn = smem_desc_sw128(sb + C::kOffS + (gi % kDsBufs) * kTileS, 8192, 1024);
       // dV += P^T dO: the 16 queries of step kk are TMEM columns 32 (kk / 2) + 8 (kk % 2) ..
 #pragma unroll
       for (int kk = 0; kk < kQb / 16; ++kk)
-        mma_ts(tmem + kColDV, ts + 32 * (kk >> 1) + 8 * (kk & 1), od_mn + ((kk * 2048) >> 4), idesc_kv,
+        mma_ts(tmem + C::kColDV, ts + 32 * (kk >> 1) + 8 * (kk & 1), od_mn + ((kk * 2048) >> 4), idesc_kv,
                (u > 0 || kk > 0) ? 1u : 0u);
       if constexpr (kDq) {
         // dQ^T = K^T dS^T over the 128 keys, into the dP^T columns
@@ -309,7 +325,7 @@ __device__ void tc_mma(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t
       // dK += dS^T Q
 #pragma unroll
       for (int kk = 0; kk < kQb / 16; ++kk)
-        mma_ss(tmem + kColDK, ds + ((kk * 32) >> 4), qd_mn + ((kk * 2048) >> 4), idesc_kv,
+        mma_ss(tmem + C::kColDK, ds + ((kk * 32) >> 4), qd_mn + ((kk * 2048) >> 4), idesc_kv,
                (u > 0 || kk > 0) ? 1u : 0u);
       tc_commit(&bars->blk_done[gi % kRing]);
       // one phase per job: the drain warps wait on it instead of on the last
@@ -399,16 +415,17 @@ __device__ __forceinline__ void ew_block_any(bool masked, const BwdParams& p, co
     ew_block<T, kCap, kAlibi, false>(p, s, dp, lsen, dneg, slope2, dist0, lo, hi, tp, drow, half, row);
 }
 
-template <typename T>
+template <typename T, int D>
 __device__ void tc_elementwise(const BwdParams& p, uint8_t* smem, TcBars* bars, uint32_t tmem, int n_kb, int warp,
                                int lane) {
+  using C = TcCfg<D>;
   volatile int* abort = &bars->abort;
   const int quarter = warp & 3, half = warp >> 2;
   const int row = 32 * quarter + lane;
   const int et = warp * 32 + lane;  // 0..255: threads 0..127 fetch the row vectors
   const uint32_t tl = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
-  float* srow = reinterpret_cast<float*>(smem + kOffRow);  // [2][-lse log2 e x 64 | -D x 64]
-  uint8_t* sds = smem + kOffS;
+  float* srow = reinterpret_cast<float*>(smem + C::kOffRow);  // [2][-lse log2 e x 64 | -D x 64]
+  uint8_t* sds = smem + C::kOffS;
   const bool alibi = p.slopes != nullptr;
   const int right = bwd_right_bound(p);
   bool failed = false;
@@ -467,8 +484,8 @@ __device__ void tc_elementwise(const BwdParams& p, uint8_t* smem, TcBars* bars, 
       }
       tc_fence_after();
       uint32_t s[32], dp[32];
-      tmem_ld32(tl + kColR + 128 * b + 32 * half, s);
-      tmem_ld32(tl + kColR + 128 * b + 64 + 32 * half, dp);
+      tmem_ld32(tl + C::kColR + 128 * b + 32 * half, s);
+      tmem_ld32(tl + C::kColR + 128 * b + 64 + 32 * half, dp);
       // block-level mask decision (uniform over the CTA)
       bool full = J.k0 + kKeys <= J.Nk && q0 + kQb <= J.Nq;
       if (right >= 0) full = full && J.k0 + kKeys - 1 <= q0 + J.off + right;
@@ -486,7 +503,7 @@ __device__ void tc_elementwise(const BwdParams& p, uint8_t* smem, TcBars* bars, 
       tmem_wait_ld();
       reg_fence(s);
       reg_fence(dp);
-      const uint32_t tp = tl + kColR + 128 * b + 32 * half;  // P^T over this half's first S^T columns
+      const uint32_t tp = tl + C::kColR + 128 * b + 32 * half;  // P^T over this half's first S^T columns
       uint8_t* drow = sds + (gi % kDsBufs) * kTileS + row * 128;
       if (p.use_softcap) {
         if (alibi) ew_block_any<T, true, true>(!full, p, s, dp, lsen, dneg, slope2, dist0, lo, hi, tp, drow, half, row);
@@ -521,12 +538,14 @@ __device__ __forceinline__ void store_row16(T* dst, const uint32_t (&r)[32], flo
     reinterpret_cast<uint4*>(dst)[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
 }
 
-template <typename T, bool kDq>
+template <typename T, int D, bool kDq>
 __device__ void tc_drain(const BwdParams& p, const CUtensorMap* tmDQ, uint8_t* smem, TcBars* bars, uint32_t tmem,
                          int n_kb, int wq, int lane) {
   volatile int* abort = &bars->abort;
+  using C = TcCfg<D>;
   const uint32_t tl = tmem + (static_cast<uint32_t>(32 * wq) << 16);
-  float* stage = reinterpret_cast<float*>(smem + kOffDQ + wq * 8192);
+  float* stage = reinterpret_cast<float*>(smem + C::kOffDQ + wq * 8192);
+  const bool dq_rows = wq < C::kDqWarps;  // this warp's lanes hold dQ^T rows (dimensions)
   bool failed = false;  // warp-uniform
   int g = 0, a = 0;
   for (int t = 0;; ++t) {
@@ -538,9 +557,9 @@ __device__ void tc_drain(const BwdParams& p, const CUtensorMap* tmDQ, uint8_t* s
     if (J.n < 0) continue;
     const int key = J.k0 + 32 * wq + lane;
     T* dk_row = reinterpret_cast<T*>(p.dk) + static_cast<size_t>(J.krow + key) * p.dkv_tok +
-                static_cast<size_t>(J.hk) * kD;
+                static_cast<size_t>(J.hk) * D;
     T* dv_row = reinterpret_cast<T*>(p.dv) + static_cast<size_t>(J.krow + key) * p.dkv_tok +
-                static_cast<size_t>(J.hk) * kD;
+                static_cast<size_t>(J.hk) * D;
     if (J.n == 0) {
       // no query sees these keys: zero gradients (NaN after a failure)
       if (key < J.Nk) {
@@ -548,7 +567,7 @@ __device__ void tc_drain(const BwdParams& p, const CUtensorMap* tmDQ, uint8_t* s
 #pragma unroll
         for (int i = 0; i < 32; ++i) z[i] = 0u;
 #pragma unroll
-        for (int c = 0; c < kD / 32; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           store_row16<T>(dk_row + 32 * c, z, 1.0f, failed);
           store_row16<T>(dv_row + 32 * c, z, 1.0f, failed);
         }
@@ -556,7 +575,7 @@ __device__ void tc_drain(const BwdParams& p, const CUtensorMap* tmDQ, uint8_t* s
       continue;
     }
     const int n = J.n;
-    if constexpr (kDq) {
+    if (kDq && dq_rows) {
       for (int u = 0; u < n; ++u) {
         const int gi = g + u;
         int h, q0;
@@ -570,7 +589,7 @@ __device__ void tc_drain(const BwdParams& p, const CUtensorMap* tmDQ, uint8_t* s
         if (!failed) tc_fence_after();
         // box row q (query), dimension 32 wq + lane: 16-byte chunk lane / 4 of
         // the 128-byte row, swizzled by q % 8; 32 queries at a time
-        const uint32_t col = kColR + 128 * (gi & 1) + 64;
+        const uint32_t col = C::kColR + 128 * (gi & 1) + 64;
         uint32_t pa[8];  // shared address of this lane's word in rows q = 0..7 (mod 8)
 #pragma unroll
         for (int k = 0; k < 8; ++k) pa[k] = smem_addr(stage) + k * 128 + ((((lane >> 2) ^ k)) << 4) + 4 * (lane & 3);
@@ -609,12 +628,12 @@ __device__ void tc_drain(const BwdParams& p, const CUtensorMap* tmDQ, uint8_t* s
     if (!failed) tc_fence_after();
     // 32 columns at a time: dV's four pieces, then dK's (scaled)
 #pragma unroll 1
-    for (int c = 0; c < 2 * kD / 32; ++c) {
-      const bool is_k = c >= kD / 32;
-      const int cc = is_k ? c - kD / 32 : c;
+    for (int c = 0; c < 2 * D / 32; ++c) {
+      const bool is_k = c >= D / 32;
+      const int cc = is_k ? c - D / 32 : c;
       uint32_t r[32];
       if (!failed) {
-        tmem_ld32(tl + (is_k ? kColDK : kColDV) + 32 * cc, r);
+        tmem_ld32(tl + (is_k ? C::kColDK : C::kColDV) + 32 * cc, r);
         tmem_wait_ld();
         reg_fence(r);
       }
@@ -631,14 +650,15 @@ __device__ void tc_drain(const BwdParams& p, const CUtensorMap* tmDQ, uint8_t* s
 
 // ---------------------------------------------------------------- kernel
 
-template <typename T, bool kDq>
+template <typename T, int D, bool kDq>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const __grid_constant__ CUtensorMap tmDQ, const BwdParams p, int n_kb, int total_jobs) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  TcBars* bars = reinterpret_cast<TcBars*>(smem + kOffBar);
+  using C = TcCfg<D>;
+  TcBars* bars = reinterpret_cast<TcBars*>(smem + C::kOffBar);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -647,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->s_ready[i], 1);
       mbar_init(&bars->p_ready[i], kEwWarps);
       mbar_init(&bars->p_free[i], 1);
-      mbar_init(&bars->dq_free[i], 4);
+      mbar_init(&bars->dq_free[i], C::kDqWarps);
       mbar_init(&bars->blk_done[i], 1);
     }
     mbar_init(&bars->acc_ready, 1);
@@ -679,13 +699,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp < kEwWarps) {
-    tc_elementwise<T>(p, smem, bars, tmem, n_kb, warp, lane);
+    tc_elementwise<T, D>(p, smem, bars, tmem, n_kb, warp, lane);
   } else if (warp < kDrainWarp0 + 4) {
-    tc_drain<T, kDq>(p, &tmDQ, smem, bars, tmem, n_kb, warp & 3, lane);
+    tc_drain<T, D, kDq>(p, &tmDQ, smem, bars, tmem, n_kb, warp & 3, lane);
   } else if (warp == kProdWarp) {
-    if (lane == 0) tc_producer(p, &tmQ, &tmK, &tmV, &tmO, smem, bars, n_kb, total_jobs);
+    if (lane == 0) tc_producer<D>(p, &tmQ, &tmK, &tmV, &tmO, smem, bars, n_kb, total_jobs);
   } else if (warp == kMmaWarp) {
-    if (lane == 0) tc_mma<T, kDq>(p, smem, bars, tmem, n_kb);
+    if (lane == 0) tc_mma<T, D, kDq>(p, smem, bars, tmem, n_kb);
   }
 
   tc_fence_before();
@@ -697,10 +717,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <typename T, bool kDq>
+template <typename T, int D, bool kDq>
 cudaError_t launch_tc(const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                       const CUtensorMap& tmO, const CUtensorMap& tmDQ, cudaStream_t stream) {
-  auto kernel = bwd_tc_kernel<T, kDq>;
+  constexpr int kSmem = TcCfg<D>::kSmem;
+  auto kernel = bwd_tc_kernel<T, D, kDq>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   static int sm_count[64];
@@ -724,14 +745,21 @@ cudaError_t launch_tc(const BwdParams& p, const CUtensorMap& tmQ, const CUtensor
 
 }  // namespace
 
-cudaError_t launch_bwd_tc(bool bf16, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+template <int D>
+cudaError_t launch_tc_d(bool bf16, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                        const CUtensorMap& tmV, const CUtensorMap& tmO, const CUtensorMap& tmDQ, cudaStream_t stream) {
+  const bool dq = !p.deterministic;
+  if (bf16) return dq ? launch_tc<__nv_bfloat16, D, true>(p, tmQ, tmK, tmV, tmO, tmDQ, stream)
+                      : launch_tc<__nv_bfloat16, D, false>(p, tmQ, tmK, tmV, tmO, tmDQ, stream);
+  return dq ? launch_tc<__half, D, true>(p, tmQ, tmK, tmV, tmO, tmDQ, stream)
+            : launch_tc<__half, D, false>(p, tmQ, tmK, tmV, tmO, tmDQ, stream);
+}
+
+cudaError_t launch_bwd_tc(bool bf16, int d, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                           const CUtensorMap& tmV, const CUtensorMap& tmO, const CUtensorMap& tmDQ,
                           cudaStream_t stream) {
-  const bool dq = !p.deterministic;
-  if (bf16) return dq ? launch_tc<__nv_bfloat16, true>(p, tmQ, tmK, tmV, tmO, tmDQ, stream)
-                      : launch_tc<__nv_bfloat16, false>(p, tmQ, tmK, tmV, tmO, tmDQ, stream);
-  return dq ? launch_tc<__half, true>(p, tmQ, tmK, tmV, tmO, tmDQ, stream)
-            : launch_tc<__half, false>(p, tmQ, tmK, tmV, tmO, tmDQ, stream);
+  return d == 128 ? launch_tc_d<128>(bf16, p, tmQ, tmK, tmV, tmO, tmDQ, stream)
+                  : launch_tc_d<64>(bf16, p, tmQ, tmK, tmV, tmO, tmDQ, stream);
 }
 
 }  // namespace fa

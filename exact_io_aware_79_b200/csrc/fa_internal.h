@@ -128,20 +128,20 @@ cudaError_t launch_bwd(bool bf16, int d, const BwdParams& p, const CUtensorMap& 
                        const CUtensorMap& tmV, const CUtensorMap& tmO, const CUtensorMap& tmDQ,
                        cudaStream_t stream);
 
-// The d = 128 key-block kernel on the tensor cores (dK, dV, and the dQ
+// The key-block kernel on the tensor cores (d = 64 or 128; dK, dV, and the dQ
 // partials added into p.dq_acc by TMA reduce-add through tmDQ unless
 // p.deterministic): persistent CTAs claim jobs
 // from *p.job_counter, which must be zero at launch. The maps as for
 // launch_bwd.
-cudaError_t launch_bwd_tc(bool bf16, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+cudaError_t launch_bwd_tc(bool bf16, int d, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                           const CUtensorMap& tmV, const CUtensorMap& tmO, const CUtensorMap& tmDQ,
                           cudaStream_t stream);
 
-// The deterministic mode's dQ pass for d = 128 on the tensor cores: dq =
+// The deterministic mode's dQ pass (d = 64 or 128) on the tensor cores: dq =
 // scale * sum over key blocks (fixed order) of dS K, written to p.dq;
 // persistent CTAs claim 128-query tiles from p.job_counter[1], which must be
 // zero at launch. The maps as for launch_bwd.
-cudaError_t launch_bwd_dq_tc(bool bf16, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+cudaError_t launch_bwd_dq_tc(bool bf16, int d, const BwdParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                              const CUtensorMap& tmV, const CUtensorMap& tmO, cudaStream_t stream);
 
 // Writes n_new new tokens per sequence into the paged caches at positions
