@@ -4,6 +4,7 @@
 #include "fa_internal.h"
 
 #include <atomic>
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cuda.h>
@@ -298,8 +299,12 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* ou
   if (B < 0 || H < 1 || Nq < 0 || Nk < 0 || total_q < 0 || total_k < 0) return FA_ERR_SHAPE;
   if (H_kv < 1 || H_kv > H || H % H_kv != 0) return FA_ERR_SHAPE;
   if (Nq > kMaxSeq || Nk > kMaxSeq || total_q > kMaxSeq || total_k > kMaxSeq) return FA_ERR_SHAPE;
-  // grid y: B * H_kv key-block CTAs, B * H query-block CTAs (deterministic or packed)
-  if (static_cast<long long>(B) * (packed_rows || deterministic ? H : H_kv) > 65535) return FA_ERR_SHAPE;
+  // jobs of the persistent kernels (128-key blocks of every (sequence, cache
+  // head); in the deterministic mode also 128-query tiles of every (sequence,
+  // query head)) are numbered in an int
+  if ((static_cast<long long>(Nk) + 127) / 128 * B * H_kv > INT_MAX ||
+      (deterministic && (static_cast<long long>(Nq) + 127) / 128 * B * H > INT_MAX))
+    return FA_ERR_SHAPE;
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
   if (d != 64 && d != 128) return FA_ERR_HEADDIM;
   if (!finite(scale) || !finite(softcap) || softcap < 0.0f) return FA_ERR_ARG;

@@ -28,8 +28,9 @@
 namespace fa {
 namespace {
 
-// D_i = sum_c dO_ic O_ic in fp32, [B, H, Nq]; outside the deterministic mode
-// the same threads zero the fp32 dQ accumulator's rows (their 8 columns).
+// D_i = sum_c dO_ic O_ic in fp32, [B, H, Nq]; the same threads zero their 8
+// columns of the fp32 dQ accumulator or, in the deterministic mode, of dq
+// itself (the fixed-order pass writes only the rows of valid sequences).
 template <typename T, int D>
 __global__ void __launch_bounds__(256) bwd_rowdot_kernel(const BwdParams p) {
   constexpr int LPR = D / 8;  // lanes per row
@@ -46,6 +47,10 @@ __global__ void __launch_bounds__(256) bwd_rowdot_kernel(const BwdParams p) {
       float4* z = reinterpret_cast<float4*>(p.dq_acc + off);
       z[0] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       z[1] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    } else {
+      const long long token = row / p.H, h = row % p.H;
+      *reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dq) + token * p.dq_tok + h * D + cl * 8) =
+          make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {

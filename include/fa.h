@@ -335,15 +335,16 @@ fa_status fa_kvcache_append(const void *k_new, const void *v_new, void *k_cache,
  *   lse                [B, H, Nq]          fp32 (the forward's, natural log)
  *   workspace          fa_bwd_workspace_size(B, H, Nq, d) bytes of device
  *                      memory, 16-byte aligned (fp32 dq accumulator, D, and
- *                      the d = 128 kernel's job counter)
+ *                      the job counters of the persistent kernels)
  *   scale, causal, window_left, window_right, alibi_slopes, softcap: as fa_fwd
  *   deterministic      0 or 1 (see above)
  * Outputs dq, dk, dv are overwritten (not accumulated). The caller owns every
  * buffer; the call only enqueues work on `stream`.
  *
  * Errors: as fa_fwd_gqa, plus FA_ERR_WORKSPACE when the workspace is missing,
- * misaligned or too small, and FA_ERR_SHAPE when B * H_kv > 65535 (B * H
- * with deterministic = 1).
+ * misaligned or too small, and FA_ERR_SHAPE when ceil(Nk / 128) * B * H_kv
+ * (the key-block jobs) or, with deterministic = 1, ceil(Nq / 128) * B * H
+ * (the query-tile jobs) exceeds 2^31 - 1.
  * Nq == 0 gives zero dk, dv; Nk == 0 gives zero dq; B == 0 is a no-op.
  */
 size_t fa_bwd_workspace_size(int B, int H, int Nq, int d);
@@ -368,8 +369,8 @@ fa_status fa_bwd(const void *q, const void *k, const void *v, const void *out, c
  * Each sequence's gradients are those fa_bwd gives for it alone. The offsets
  * are read on the device only: a sequence whose entries break the contract
  * is skipped, its dk and dv rows left as they were; dq rows that belong to no
- * valid sequence are written as zero. Limits: B * H <= 65535, total_q,
- * total_k <= 2^28.
+ * valid sequence are written as zero. Limits: total_q, total_k <= 2^28, and
+ * the job counts of fa_bwd.
  */
 fa_status fa_bwd_varlen(const void *q, const void *k, const void *v, const void *out, const float *lse,
                         const void *dout, void *dq, void *dk, void *dv, const int *cu_seqlens_q,

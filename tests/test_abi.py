@@ -280,10 +280,13 @@ def test_bwd_validation(lib):
     assert bw(det=2) == ARG
     assert bw(H_kv=3) == SHAPE
     assert bw(H_kv=16) == SHAPE
-    assert bw(B=40000, H_kv=2) == SHAPE          # B * H_kv > 65535
-    big = lib.fa_bwd_workspace_size(8192, 8, 100, 128)
-    assert bw(B=8192, H_kv=2, ws_bytes=big) == DEVICE          # B * H_kv = 16384
-    assert bw(B=8192, H_kv=2, det=1, ws_bytes=big) == SHAPE    # the deterministic dQ grid has B * H = 65536 rows
+    # jobs of the persistent kernels must number below 2^31: ceil(Nk / 128) B H_kv
+    # (and ceil(Nq / 128) B H in the deterministic mode)
+    assert bw(B=1024, Nk=1 << 28) == SHAPE        # 2^21 * 1024 * 2 = 2^32 key-block jobs
+    big = lib.fa_bwd_workspace_size(40000, 8, 100, 128)
+    assert bw(B=40000, H_kv=2, ws_bytes=big) == DEVICE              # B * H_kv = 80000: fine
+    assert bw(B=40000, H_kv=2, det=1, ws_bytes=big) == DEVICE       # B * H = 320000: fine
+    assert bw(B=1024, Nq=1 << 28, det=1) == SHAPE    # 2^21 * 1024 * 8 = 2^34 query-tile jobs
     assert bw(d=96) == HEADDIM
     assert bw(dtype=7) == DTYPE
     assert bw(scale=float("nan")) == ARG
@@ -315,7 +318,7 @@ def test_bwd_varlen_validation(lib):
                                  a["cap"], a["det"], a["ws"], a["ws_bytes"], None)
     assert bv() == DEVICE
     assert bv(H_kv=3) == SHAPE
-    assert bv(B=20000) == SHAPE                  # B * H > 65535
+    assert bv(B=20000) in (OK, DEVICE)          # no grid limit on B * H (persistent kernels)
     assert bv(tq=-1) == SHAPE
     assert bv(d=80) == HEADDIM
     assert bv(cq=None) == NULL

@@ -214,7 +214,8 @@ def test_bwd_varlen_grouped_heads_with_oracle_forward():
     check(dv, rv, dtype, "dv")
 
 
-def test_bwd_varlen_skips_a_sequence_with_broken_offsets():
+@pytest.mark.parametrize("det", [False, True], ids=["atomic_dq", "deterministic"])
+def test_bwd_varlen_skips_a_sequence_with_broken_offsets(det):
     lens, H, d = (80, 120, 60), 2, 64
     g = torch.Generator().manual_seed(12)
     q, cu = _packed(lens, H, d, torch.float16, g)
@@ -228,8 +229,9 @@ def test_bwd_varlen_skips_a_sequence_with_broken_offsets():
     bad = cu.clone()
     bad[2] = 500                      # sequence 1 ends past total, sequence 2 starts there
     dq, dk, dv = torch.empty_like(qd), torch.full_like(kd, 7.0), torch.full_like(vd, 7.0)
+    dq.fill_(float("nan"))            # every row of dq is written, valid sequence or not
     fa.fa_bwd_varlen(qd, kd, vd, out, lse, dod, dq, dk, dv, bad.cuda(), bad.cuda(), max(lens), max(lens), 0.125,
-                     causal=True)
+                     causal=True, deterministic=det)
     torch.cuda.synchronize()
     rq, rk, rv = _varlen_reference(q, k, v, do, cu, cu, 0.125, causal=True)
     a = int(cu[1])
