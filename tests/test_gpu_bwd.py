@@ -64,6 +64,7 @@ CASES = [
     (2, 2, 2, 64, 64, 128, torch.bfloat16, False, 10, 20, False, 0.0),     # two-sided window
     (1, 8, 2, 100, 300, 128, torch.float16, True, -1, -1, True, 0.0),      # groups of 4, ALiBi, Nq < Nk
     (1, 2, 2, 1, 70, 128, torch.bfloat16, True, -1, -1, False, 5.0),       # one query row, softcap
+    (2, 4, 2, 300, 333, 64, torch.bfloat16, True, 100, 0, True, 30.0),     # d = 64 bf16: grouped, window, ALiBi, softcap
 ]
 
 
