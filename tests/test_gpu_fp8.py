@@ -107,6 +107,8 @@ CASES = [
     (1, 2, 2, 384, 384, torch.float8_e5m2, True, -1, -1, False, 0.0, 1.0, 8),
     (1, 2, 1, 1, 333, torch.float8_e5m2, True, -1, -1, True, 5.0, 1.0, 9),
     (1, 2, 2, 2048, 2048, torch.float8_e4m3fn, True, -1, -1, False, 0.0, 1.0, 10),
+    (1, 3, 3, 600, 450, torch.float8_e4m3fn, False, 200, 150, True, 30.0, 1.5, 12),
+    (1, 2, 2, 257, 700, torch.float8_e4m3fn, False, -1, -1, True, 0.0, 1.0, 13),
 ]
 
 

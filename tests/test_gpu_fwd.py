@@ -52,6 +52,7 @@ SMALL = [
     (1, 2, 513, 513, 128, torch.bfloat16, False, 50, 70, False, 0.0, 1.0),
     (1, 4, 640, 640, 128, torch.bfloat16, True, -1, -1, True, 50.0, 2.0),
     (1, 3, 257, 385, 64, torch.float16, False, -1, -1, True, 0.0, 1.0),
+    (1, 3, 600, 450, 128, torch.bfloat16, False, 200, 150, True, 30.0, 1.5),
     (1, 2, 384, 384, 128, torch.float16, True, 130, -1, False, 5.0, 1.5),
     (2, 2, 1, 1, 128, torch.bfloat16, True, -1, -1, False, 0.0, 1.0),
     (1, 1, 1, 333, 128, torch.bfloat16, True, -1, -1, True, 0.0, 1.0),
