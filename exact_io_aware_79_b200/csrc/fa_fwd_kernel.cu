@@ -238,6 +238,16 @@ __device__ __forceinline__ Job make_job(const FwdParams& p, int b, int h, int Nq
   return j;
 }
 
+// The K/V tile a job visits u-th: f, .., l, or l, .., f with ALiBi (kRev).
+// With ALiBi a row's scores grow toward its own position, so visiting the
+// nearest keys first sets the running max at the first tile and the lazy
+// rescale (which waits for the previous PV product) rarely fires; in key
+// order it fired on nearly every tile for the steeper heads.
+template <bool kRev>
+__device__ __forceinline__ int tile_at(const Job& jb, int u) {
+  return kRev ? jb.l - u : jb.f + u;
+}
+
 // Calls fn(job) for every job of this CTA, in order. The work items are
 // numbered consecutively over the sequences (b, then head h, then pair pi;
 // sequence b has H * ceil(T_b / 2) items, T_b its Q tiles), so sequences of
@@ -268,7 +278,7 @@ __device__ __forceinline__ void for_each_job(const FwdParams& p, Fn&& fn) {
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kRev>
 __device__ void producer(const FwdParams& p, const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
                          uint8_t* sQ, uint8_t* sK, uint8_t* sV, Barriers* bars) {
   using C = Cfg<T, D>;
@@ -308,12 +318,12 @@ __device__ void producer(const FwdParams& p, const CUtensorMap* tmQ, const CUten
       tma_load_4d(tmQ, &bars->q_full[a % QB], sQ + (a % QB) * C::kTileBytes + ch * C::kChunkBytes,
                   ch * C::kChunkElems, jb.h, jb.qrow + jb.q0, jb.bcoord, pol_q);
     auto load_k = [&](int u) {
-      const bool r = load(tmK, sK, bars->k_full, bars->s_ready, C::kSlotsK, g + u, jb, jb.f + u);
+      const bool r = load(tmK, sK, bars->k_full, bars->s_ready, C::kSlotsK, g + u, jb, tile_at<kRev>(jb, u));
       nk += r;
       return r;
     };
     auto load_v = [&](int u) {
-      const bool r = load(tmV, sV, bars->v_full, bars->pv_done, C::kSlotsV, g + u, jb, jb.f + u);
+      const bool r = load(tmV, sV, bars->v_full, bars->pv_done, C::kSlotsV, g + u, jb, tile_at<kRev>(jb, u));
       nv += r;
       return r;
     };
@@ -526,7 +536,7 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
   const int n = jb.has ? l - f + 1 : 0;
   const int n_run = ok ? n : 0;
   for (int it = 0; it < n_run; ++it) {
-    const int j = f + it;
+    const int j = tile_at<kAlibi>(jb, it);
     const int gi = g + it;  // tile number across the CTA's jobs
     const uint32_t tS = tmem + lane_sel + (gi & 1) * 128 + part * 64;  // this part's S, then P, columns
     ok = mbar_wait(&bars->s_ready[gi % kRing], (gi / kRing) & 1, abort);
@@ -854,7 +864,7 @@ __global__ void __launch_bounds__(threads_of(kCap, kAlibi), 1)
   if (warp < kSoftmaxWarps) {
     softmax_group<T, D, kCap, kAlibi>(p, bars, tmem);
   } else if (warp == kProducerWarp) {
-    if (lane == 0) producer<T, D>(p, &tmQ, &tmK, &tmV, sQ, sK, sV, bars);
+    if (lane == 0) producer<T, D, kAlibi>(p, &tmQ, &tmK, &tmV, sQ, sK, sV, bars);
   } else if (warp == kQkWarp) {
     if (lane == 0) qk_issuer<T, D>(p, sQ, sK, bars, tmem);
   } else if (warp == kPvWarp) {
