@@ -554,49 +554,25 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
     tmem_wait_ld();
 #pragma unroll
     for (int c = 0; c < kChunks; ++c) reg_fence(s[c]);
-    // ALiBi: when every key of this part's tile that the row sees lies on
-    // one side of its position (always, for a causal row), the bias
-    // -slope |pos - key| is linear in the key's offset o within the tile,
-    // and c + bias = lin_base + lin_slope * o is one FMA per score (keys the
-    // row does not see get a wrong bias here and are masked below). Taken by
-    // the 8-bit instantiations only: there it measured faster (383 against
-    // 365 TFLOP/s, ALiBi + softcap 50, B4 H32 N4096 causal); with 16-bit
-    // operands it measured slower (360 against 397 for this loop without it).
-    constexpr bool kLinAlibi = kAlibi && Elem<T>::kFp8;
-    bool lin = false;
-    float lin_slope = 0.0f, lin_base = 0.0f;
-    if constexpr (kLinAlibi) {
-      const bool left = rr.hi <= pos || key0 + kKeys - 1 <= pos;  // keys <= pos
-      const bool right = rr.lo >= pos || key0 >= pos;              // keys >= pos
-      lin = __all_sync(0xffffffffu, left || right);
-      lin_slope = left ? slope_l2 : -slope_l2;
-      lin_base = fmaf(-lin_slope, dpos, kCap ? p.cap_log2 : 0.0f);
-    }
     // pass 1: transform (modifier paths), mask and this part's max
     float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
     for (int c = 0; c < kChunks; ++c) {
       if (!kPlain || masked) {
-        auto transform = [&](auto lin_tag) {
-          constexpr bool kLin = decltype(lin_tag)::value;
+        // (written as a lambda: this form of the loop measured 397 against
+        // 375 TFLOP/s for ALiBi + softcap, the same arithmetic inline)
+        auto transform = [&]() {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             float x = __uint_as_float(s[c][e]);
             const int key = key0 + 32 * c + e;
-            if constexpr (kLin) {
-              const float cb = fmaf(lin_slope, static_cast<float>(32 * c + e), lin_base);
-              x = kCap ? softcap_fma_sum(x, cap_k, p.cap_log2, cb) : fmaf(x, p.scale_log2, cb);
-            } else if constexpr (!kPlain) {
+            if constexpr (!kPlain)
               x = mod_score<kCap, kAlibi>(p, x, cap_k, slope_l2, dpos - static_cast<float>(32 * c + e));
-            }
             if (masked) x = (key >= rr.lo && key <= rr.hi) ? x : -INFINITY;
             s[c][e] = __float_as_uint(x);
           }
         };
-        if (kLinAlibi && lin)
-          transform(std::integral_constant<bool, kLinAlibi>{});
-        else
-          transform(std::false_type{});
+        transform();
       }
 #pragma unroll
       for (int e = 0; e < 32; e += 8) {

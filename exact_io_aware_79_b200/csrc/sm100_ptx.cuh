@@ -419,17 +419,12 @@ __device__ __forceinline__ float tanh_via_exp2(float y) {
 }
 
 // c * tanh(y) + b from the same identity, with the scale k = 2 log2(e) / s
-// of y = x / s folded into one multiply and cb = c + b into the last FMA:
-// cb - 2 c / (2^(k x) + 1). For k x above 128 the power is +inf and the
+// of y = x / s folded into one multiply and c, b into the last FMA:
+// c - 2 c / (2^(k x) + 1) + b. For k x above 128 the power is +inf and the
 // result c + b; far below, 0 and -c + b (the limits of tanh).
-__device__ __forceinline__ float softcap_fma_sum(float x, float k, float c, float cb) {
-  const float e = ex2(x * k);
-  return fmaf(-2.0f * c, rcp(e + 1.0f), cb);
-}
-
-// The same with cb = c + b given (softcap_fma_sum), or b (softcap_fma).
 __device__ __forceinline__ float softcap_fma(float x, float k, float c, float b) {
-  return softcap_fma_sum(x, k, c, c + b);
+  const float e = ex2(x * k);
+  return fmaf(-2.0f * c, rcp(e + 1.0f), c + b);
 }
 
 template <typename T>
