@@ -82,6 +82,10 @@ constexpr uint32_t kTmemO = 256;        // O accumulator of part 0; part 1's fol
 constexpr uint32_t kTmemOStride = 128;
 
 constexpr int kBarrierBytes = 8192;  // barrier block and exchange slots
+// O staging of the epilogue, after the barrier block: per softmax warp its
+// 32 rows x 32 output columns (64 bytes a row)
+constexpr int kStageWarpBytes = 32 * 64;
+constexpr int kStageBytes = 8 * kStageWarpBytes;
 
 // Input element types: fp16 / bf16 (products of kind::f16, P rounded to the
 // input type, O written in it), or 8-bit floats (tags below: products of
@@ -128,7 +132,7 @@ struct Cfg {
   static constexpr int kSlotsK = (kTileBytes <= 16384) ? 5 : 2;  // K ring depth
   static constexpr int kSlotsV = kSlotsK;                        // V ring depth
   static constexpr int kSlots = kSlotsK + kSlotsV;
-  static constexpr int kSmemBytes = 1024 + (kQBufs + kSlots) * kTileBytes + kBarrierBytes;
+  static constexpr int kSmemBytes = 1024 + (kQBufs + kSlots) * kTileBytes + kBarrierBytes + kStageBytes;
 };
 
 struct Barriers {
@@ -734,6 +738,13 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
   const uint32_t tO_self = tO + part * kOCols;                                  // own O, own columns
   const uint32_t tO_other = tmem + lane_sel + kTmemO + (1 - part) * kTmemOStride + part * kOCols;
   if (ok && n > 0) {
+    // Each row's 32 columns of a round go through this warp's staging tile
+    // (16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3), so that both
+    // the row-wise writes and the chunk-wise reads hit every bank once),
+    // and leave as stores of 8 rows x 64 bytes; a thread storing its own
+    // row would touch 32 separate lines per instruction.
+    uint8_t* stage = reinterpret_cast<uint8_t*>(bars) + kBarrierBytes + warp * kStageWarpBytes;
+    Out* ocol = reinterpret_cast<Out*>(p.out) + static_cast<long long>(h) * D + part * kOCols;
 #pragma unroll
     for (int cc = 0; cc < kOCols / 32; ++cc) {
       uint32_t o[32], o2[32];
@@ -742,18 +753,27 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
       tmem_wait_ld();
       reg_fence(o);
       reg_fence(o2);
-      if (row_ok) {
-        uint32_t pk[16];
+      uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float v0 = (a_self * __uint_as_float(o[2 * e]) + a_other * __uint_as_float(o2[2 * e])) * inv;
-          const float v1 = (a_self * __uint_as_float(o[2 * e + 1]) + a_other * __uint_as_float(o2[2 * e + 1])) * inv;
-          pk[e] = pack2<Out>(v0, v1);
-        }
-        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cc);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+      for (int e = 0; e < 16; ++e) {
+        const float v0 = (a_self * __uint_as_float(o[2 * e]) + a_other * __uint_as_float(o2[2 * e])) * inv;
+        const float v1 = (a_self * __uint_as_float(o[2 * e + 1]) + a_other * __uint_as_float(o2[2 * e + 1])) * inv;
+        pk[e] = pack2<Out>(v0, v1);
       }
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        *reinterpret_cast<uint4*>(stage + lane * 64 + ((v ^ ((lane >> 1) & 3)) * 16)) =
+            make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int rl = 8 * i + (lane >> 2), ch = lane & 3;  // row of the warp's 32, 16-byte chunk
+        const uint4 val = *reinterpret_cast<const uint4*>(stage + rl * 64 + ((ch ^ ((rl >> 1) & 3)) * 16));
+        const int qr = q0 + quarter * 32 + rl;
+        if (qr < jb.Nq)
+          *reinterpret_cast<uint4*>(ocol + (jb.obase + qr) * p.H * D + 32 * cc + 8 * ch) = val;
+      }
+      __syncwarp();
     }
     // both O accumulators have been read (by both parts, which each arrive
     // here): the next job's first PV product may overwrite them
