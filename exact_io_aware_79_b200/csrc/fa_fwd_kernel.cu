@@ -657,7 +657,9 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
         }
       }
     };
-    if (masked)
+    // masked entries hold -inf, whose exponential is 0 unless a zero scale
+    // turns -inf * 0 into a NaN (plain path): only then select them out
+    if (kPlain && masked && sl2 == 0.0f)
       pass2(std::true_type{});
     else
       pass2(std::false_type{});
