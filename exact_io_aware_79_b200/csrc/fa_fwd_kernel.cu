@@ -552,6 +552,11 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
     // the tile is dpos - e away (ALiBi)
     const float dpos = kAlibi ? static_cast<float>(pos - key0) : 0.0f;
     const bool masked = j * BN < last_row.lo || j * BN + BN - 1 > first_row.hi;  // uniform over the tile
+    // key visible iff (unsigned)(key - mlo) <= mspan (an empty interval:
+    // mlo = -1, mspan = 0, and no key >= 0 passes)
+    const bool row_has = rr.lo <= rr.hi;
+    const int mlo = row_has ? rr.lo : -1;
+    const unsigned mspan = row_has ? static_cast<unsigned>(rr.hi - rr.lo) : 0u;
     tc_fence_after();
 #pragma unroll
     for (int c = 0; c < kChunks; ++c) tmem_ld32(tS + 32 * c, s[c]);
@@ -572,7 +577,7 @@ __device__ void softmax_job(const FwdParams& p, Barriers* bars, uint32_t tmem, c
             const int key = key0 + 32 * c + e;
             if constexpr (!kPlain)
               x = mod_score<kCap, kAlibi>(p, x, cap_k, slope_l2, dpos - static_cast<float>(32 * c + e));
-            if (masked) x = (key >= rr.lo && key <= rr.hi) ? x : -INFINITY;
+            if (masked) x = (static_cast<unsigned>(key - mlo) <= mspan) ? x : -INFINITY;
             s[c][e] = __float_as_uint(x);
           }
         };
