@@ -58,7 +58,7 @@ DECODE_READ_PER_KV_BYTE = 967959936.0 / 965165056.0  # (968,019,712 + 967,900,16
 # Forward: per-launch DRAM bytes of ncu captures of the forward kernel as it
 # stands, on the named workload; a workload without such a capture reports
 # None.
-FWD_TRAFFIC = {W.WINDOW_16K.name: 201912576.0 + 48537856.0}
+FWD_TRAFFIC = {W.WINDOW_16K.name: 201669888.0 + 48675840.0}
 # Backward workloads timed after the step (atomic dQ, and the deterministic
 # mode on the first); credited 2.5 x the forward's flops (five products of
 # the forward's size against two).
